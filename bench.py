@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Benchmark of the chunkwise gated delta rule on B200: one JSON line on rank 0.
+
+A step is one pass of the whole path over one batch of synthetic input: the
+forward (o, u, S_T) and the backward (dq, dk, dv, d log alpha, dbeta, dS0) of
+Gated DeltaNet at B=8, T=4096, H=8, dk=dv=128, bf16 I/O, fp32 state, chunk 64
+(the headline workload "delta-rule fwd+bwd tokens/s at B=8,T=4096,H=8,d=128
+bf16").  Inputs are drawn once by the seeded generator and are resident in HBM
+before the timed region.  Each step is timed with CUDA events on the launching
+stream; L2 is flushed (256 MiB write) between steps, outside the events.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs an independent replica
+(the path has no cross-(b, h) exchange, so there is no data-path collective);
+value = all ranks' tokens / the slowest rank's time ("scaling": "weak").
+
+--impl reference times the fp64 CPU oracle (the checker, test infrastructure) on
+a bounded sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "delta-rule fwd+bwd tokens/s at B=8,T=4096,H=8,d=128 bf16; % of roofline"
+WORKLOAD_ID = 2
+FLUSH_BYTES = 256 << 20
+
+
+# ---------------------------------------------------------------------------------------------
+# algorithmic counts (per token-head unless stated)
+def alg_counts(B, T, H, dk, dv, C, variant, elem, s0=False, du=True):
+    gw = {0: 0, 1: 1, 2: dk}[variant]
+    th = B * T * H
+    heads = B * H
+    fwd_flops = th * (6 * dk * dv + 3 * C * dk + 2 * C * dv + C * C / 3)
+    fwd_bytes = th * elem * (2 * dk + 3 * dv + gw + 1) + heads * 4 * dk * dv * (1 + int(s0))
+    bwd_in_out = (4 * dk + 4 * dv + 2 * gw + 2) - (0 if du else dv)
+    bwd_bytes = th * elem * bwd_in_out + heads * 4 * dk * dv * (2 + int(s0))
+    return {"fwd_flops": fwd_flops, "fwd_bytes": fwd_bytes, "bwd_flops": 2 * fwd_flops, "bwd_bytes": bwd_bytes}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_uuid: str | None):
+        self.proc = None
+        self.lines = []
+        self.uuid = device_uuid
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+def cpu_oracle_sample(w, steps=1, seed=0):
+    """Time the fp64 oracle (fwd + bwd) on a bounded sample of the workload.
+
+    The sample is `units` (b, h) sequences of the full length T (one per host
+    core, the oracle's own threading unit), drawn by the same generator.  The
+    rate is extrapolated to the whole workload by the (b, h) count.
+    """
+    import numpy as np
+    import torch
+
+    import oracle
+    from gated_delta_rule_107_b200.inputs import make_inputs
+
+    cores = os.cpu_count() or 1
+    units = max(1, min(cores, w.B * w.H))
+    x = make_inputs(w.variant, w.dtype, 1, w.T, units, w.dk, w.dv, seed=w.seed + 77, grads=True, du=True)
+    a = {k: (None if v is None else v.double().numpy()) for k, v in x.items()}
+    oracle.load_library()
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        oracle.fwd(a["q"], a["k"], a["v"], a["loga"], a["beta"], None, variant=w.variant, nthreads=units)
+        oracle.bwd(a["q"], a["k"], a["v"], a["loga"], a["beta"], None, a["dO"], a["du"], a["dS_T"],
+                   variant=w.variant, nthreads=units)
+        times.append(time.perf_counter() - t0)
+    t = statistics.median(times)
+    full_time = t * (w.B * w.H) / units
+    value = w.B * w.T / full_time
+    sample = (f"fp64 oracle fwd+bwd on {units} (b,h) sequences of T={w.T} (of {w.B * w.H}); "
+              f"{t:.2f} s per sample, extrapolated by the (b,h) count")
+    return {"value": value, "unit": "tokens/s", "cores": units, "kind": "oracle", "sample": sample,
+            "sample_seconds": t}, times, np
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from gated_delta_rule_107_b200.inputs import WORKLOADS
+    w = WORKLOADS[WORKLOAD_ID]
+    cpu_oracle_sample(w, steps=max(args.warmup, 0) or 1)  # warm-up
+    base, times, _ = cpu_oracle_sample(w, steps=args.steps)
+    ms = statistics.mean(times) * (w.B * w.H) / base["cores"] * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": base["value"], "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name + " fwd+bwd", "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
+                   "chunk": 64, "variant": "gdn", "parallelism": "oracle threads over (b,h)"},
+        "cpu_baseline": base,
+        "e2e": {"value": base["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from gated_delta_rule_107_b200 import binding
+    from gated_delta_rule_107_b200.inputs import WORKLOADS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (B200); the CPU oracle arm is --impl reference")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    w = WORKLOADS[WORKLOAD_ID]
+    B, T, H, dk, dv, C, var = w.B, w.T, w.H, w.dk, w.dv, 64, w.variant
+    dt = binding.DR_BF16
+    x = make_inputs(var, w.dtype, B, T, H, dk, dv, seed=w.seed + 1000 * rank, grads=True, du=True, device=dev)
+    elem = 2
+
+    fwd_names = binding.launches(B, T, H, dk, dv, var, C, dt, 0)
+    bwd_names = binding.launches(B, T, H, dk, dv, var, C, dt, 1)
+    ws_bytes = max(binding.workspace_size(B, T, H, dk, dv, var, C, dt, 0),
+                   binding.workspace_size(B, T, H, dk, dv, var, C, dt, 1))
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(x["v"])
+    u = torch.empty_like(x["v"])
+    S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    grads = {"dq": torch.empty_like(x["q"]), "dk": torch.empty_like(x["k"]), "dv": torch.empty_like(x["v"]),
+             "dalpha": torch.empty_like(x["loga"]), "dbeta": torch.empty_like(x["beta"]),
+             "dS0": torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)}
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+
+    fev = [torch.cuda.Event(enable_timing=True) for _ in range(len(fwd_names) + 1)]
+    bev = [torch.cuda.Event(enable_timing=True) for _ in range(len(bwd_names) + 1)]
+    farr, barr = binding.event_array(fev), binding.event_array(bev)
+
+    def step(timed: bool):
+        fa = (p(x["q"]), p(x["k"]), p(x["v"]), p(x["loga"]), p(x["beta"]), None, p(o), p(u), p(S_T),
+              B, T, H, dk, dv, var, C, dt, p(ws), ws_bytes, sp)
+        ba = (p(x["q"]), p(x["k"]), p(x["v"]), p(x["loga"]), p(x["beta"]), None, p(x["dO"]), p(x["du"]),
+              p(x["dS_T"]), p(grads["dq"]), p(grads["dk"]), p(grads["dv"]), p(grads["dalpha"]), p(grads["dbeta"]),
+              p(grads["dS0"]), B, T, H, dk, dv, var, C, dt, p(ws), ws_bytes, sp)
+        if timed:
+            rc1 = binding.fwd_timed_raw(*fa, farr, len(fev))
+            rc2 = binding.bwd_timed_raw(*ba, barr, len(bev))
+        else:
+            rc1 = binding.fwd_raw(*fa)
+            rc2 = binding.bwd_raw(*ba)
+        if rc1 or rc2:
+            raise RuntimeError(f"delta_rule call failed: {binding.strerror(rc1 or rc2)}")
+
+    for _ in range(max(args.warmup, 3)):
+        step(False)
+    torch.cuda.synchronize()
+    if binding.sync_status() != binding.DR_OK:
+        raise RuntimeError("device error word set during warm-up")
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    t_pre = time.perf_counter()
+    while time.perf_counter() - t_pre < 0.4:  # load the GPU before the first sample
+        step(False)
+        torch.cuda.synchronize()
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms, kern = [], {n: [] for n in set(fwd_names) | set(bwd_names)}
+    fwd_ms, bwd_ms = [], []
+    for _ in range(args.steps):
+        flush.fill_(1)
+        step(True)
+        torch.cuda.synchronize()
+        fms = [fev[i].elapsed_time(fev[i + 1]) for i in range(len(fwd_names))]
+        bms = [bev[i].elapsed_time(bev[i + 1]) for i in range(len(bwd_names))]
+        for n, t in zip(fwd_names, fms):
+            kern[n].append(t)
+        for n, t in zip(["bwd:" + n for n in bwd_names], bms):
+            kern.setdefault(n, []).append(t)
+        fwd_ms.append(fev[0].elapsed_time(fev[-1]))
+        bwd_ms.append(bev[0].elapsed_time(bev[-1]))
+        step_ms.append(fev[0].elapsed_time(bev[-1]))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    if binding.sync_status() != binding.DR_OK:
+        raise RuntimeError("device error word set during the timed region")
+
+    ms = statistics.mean(step_ms)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    tokens = B * T * world
+    value = tokens / (ms / 1e3)
+
+    # ---- end to end through the public API with host buffers ----
+    host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in x.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    outs = [o, u, S_T] + [g for g in grads.values() if g is not None]
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    dev_in = {k: (torch.empty_like(v) if v is not None else None) for k, v in x.items()}
+
+    def e2e_step():
+        for k_, v_ in host.items():
+            if v_ is not None:
+                dev_in[k_].copy_(v_, non_blocking=True)
+        binding.delta_rule_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["loga"], dev_in["beta"], None,
+                               variant=var, chunk=C, workspace=ws, out=o, u=u, S_T=S_T)
+        binding.delta_rule_bwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["loga"], dev_in["beta"], None,
+                               dev_in["dO"], dev_in["du"], dev_in["dS_T"], variant=var, chunk=C, workspace=ws,
+                               grads=grads)
+        for src, dst in zip(outs, host_out):
+            dst.copy_(src, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, min(args.steps, 10))
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    peaks = load_peaks()
+    cnt = alg_counts(B, T, H, dk, dv, C, var, elem)
+    kern_ms = {n: statistics.mean(v) for n, v in kern.items() if v}
+    total = sum(kern_ms.values())
+    dominant = max(kern_ms, key=kern_ms.get)
+    f_ms = statistics.mean(fwd_ms)
+    b_ms = statistics.mean(bwd_ms)
+    # roofline of the forward (one fused kernel on the tensor-core path): algorithmic bytes / time
+    f_bytes = cnt["fwd_bytes"]
+    achieved = f_bytes / (f_ms / 1e3) / 1e9
+    fwd_label = fwd_names[0] if len(fwd_names) == 1 else "forward call (" + "+".join(fwd_names) + ")"
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tfile):
+        try:
+            from gated_delta_rule_107_b200.build import source_digest
+            with open(tfile) as f:
+                tr = json.load(f)
+            ent = tr.get(fwd_label)
+            if ent and ent.get("source_digest") == source_digest():
+                traffic = ent["bytes_per_launch"]
+        except Exception:
+            traffic = None
+    step_time_roof = max((cnt["fwd_bytes"] + cnt["bwd_bytes"]) / (peaks["hbm_gbs"] * 1e9),
+                         (cnt["fwd_flops"] + cnt["bwd_flops"]) / (peaks["bf16_tflops_sustained"] * 1e12))
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name + " fwd+bwd", "B": B, "T": T, "H": H, "dk": dk, "dv": dv, "chunk": C,
+                   "variant": "gdn", "io": "bf16, fp32 state", "l2": "flushed between steps (256 MiB write)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "kernel": fwd_label,
+                     "alg_bytes_per_launch": f_bytes, "ms_per_launch": f_ms,
+                     "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"},
+        "step_roofline": {"alg_bytes": cnt["fwd_bytes"] + cnt["bwd_bytes"],
+                          "alg_flops": cnt["fwd_flops"] + cnt["bwd_flops"], "roofline_ms": step_time_roof * 1e3,
+                          "frac": step_time_roof * 1e3 / ms, "fwd_ms": f_ms, "bwd_ms": b_ms},
+        "kernels": {n: {"ms": round(t, 4), "share": round(t / total, 4)} for n, t in kern_ms.items()},
+        "dominant_kernel": dominant,
+        "gpu_launches": args.steps * (len(fwd_names) + len(bwd_names)),
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "clocks": clocks,
+        "gpu": torch.cuda.get_device_name(dev),
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(w, steps=1)[0]
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,200 @@
+"""ctypes binding of libdeltarule.so (the C ABI in include/delta_rule.h).
+
+Argument marshalling only: every step of the computation runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the current stream.  There is
+no fallback: if the shared library is missing or a call fails, an exception is
+raised.
+
+Low level: ``workspace_size``, ``fwd_raw``, ``bwd_raw``, ``strerror``,
+``sync_status`` mirror the C entry points one to one (integer pointers).
+High level: ``delta_rule_fwd`` / ``delta_rule_bwd`` take torch CUDA tensors,
+allocate outputs and the workspace with torch, and call the C ABI on the
+current stream.  ``delta_rule_fwd_host`` is the same call for host tensors
+(copies in, computes, copies out).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+DR_DELTANET, DR_GATED, DR_KDA = 0, 1, 2
+DR_F32, DR_BF16 = 0, 1
+DR_OK, DR_ERR_ARG, DR_ERR_UNSUPPORTED, DR_ERR_ALIGN, DR_ERR_WORKSPACE, DR_ERR_CUDA, DR_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5, -6
+VARIANTS = {"deltanet": DR_DELTANET, "gdn": DR_GATED, "gated": DR_GATED, "kda": DR_KDA}
+DTYPES = {torch.float32: DR_F32, torch.bfloat16: DR_BF16}
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdeltarule.so")
+EXPORTS = ("delta_rule_workspace_size", "delta_rule_fwd", "delta_rule_bwd", "delta_rule_strerror",
+           "delta_rule_sync_status", "delta_rule_launches", "delta_rule_fwd_timed", "delta_rule_bwd_timed")
+
+_lib = None
+
+
+class DeltaRuleError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {strerror(code)} ({code})")
+        self.code = code
+
+
+def load(path: str | None = None):
+    """Load libdeltarule.so (built by gated_delta_rule_107_b200.build); raises if it is absent."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError(f"{p} not found: build it with `python -m gated_delta_rule_107_b200.build` "
+                          "(the CUDA library is required; there is no fallback)")
+    lib = ctypes.CDLL(p)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.delta_rule_workspace_size.argtypes = [i] * 9
+    lib.delta_rule_workspace_size.restype = sz
+    lib.delta_rule_fwd.argtypes = [vp] * 9 + [i] * 8 + [vp, sz, vp]
+    lib.delta_rule_fwd.restype = i
+    lib.delta_rule_bwd.argtypes = [vp] * 15 + [i] * 8 + [vp, sz, vp]
+    lib.delta_rule_bwd.restype = i
+    lib.delta_rule_strerror.argtypes = [i]
+    lib.delta_rule_strerror.restype = ctypes.c_char_p
+    lib.delta_rule_sync_status.argtypes = [vp]
+    lib.delta_rule_sync_status.restype = i
+    lib.delta_rule_launches.argtypes = [i] * 9 + [ctypes.POINTER(ctypes.c_char_p), i]
+    lib.delta_rule_launches.restype = i
+    lib.delta_rule_fwd_timed.argtypes = [vp] * 9 + [i] * 8 + [vp, sz, vp, ctypes.POINTER(vp), i]
+    lib.delta_rule_fwd_timed.restype = i
+    lib.delta_rule_bwd_timed.argtypes = [vp] * 15 + [i] * 8 + [vp, sz, vp, ctypes.POINTER(vp), i]
+    lib.delta_rule_bwd_timed.restype = i
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def strerror(code: int) -> str:
+    return load().delta_rule_strerror(int(code)).decode()
+
+
+def workspace_size(B, T, H, dk, dv, variant, chunk, dtype, for_bwd) -> int:
+    n = load().delta_rule_workspace_size(B, T, H, dk, dv, variant, chunk, dtype, int(bool(for_bwd)))
+    if n == ctypes.c_size_t(-1).value:
+        raise DeltaRuleError(DR_ERR_ARG, "delta_rule_workspace_size")
+    return n
+
+
+def launches(B, T, H, dk, dv, variant, chunk, dtype, for_bwd) -> list[str]:
+    """Names of the kernels one call launches, in launch order."""
+    names = (ctypes.c_char_p * 16)()
+    n = load().delta_rule_launches(B, T, H, dk, dv, variant, chunk, dtype, int(bool(for_bwd)), names, 16)
+    if n < 0:
+        raise DeltaRuleError(n, "delta_rule_launches")
+    return [names[i].decode() for i in range(n)]
+
+
+def event_array(events):
+    """ctypes array of the raw cudaEvent_t handles of torch.cuda.Event objects."""
+    arr = (ctypes.c_void_p * len(events))()
+    for i, e in enumerate(events):
+        arr[i] = e.cuda_event
+    return arr
+
+
+def fwd_raw(*args) -> int:
+    return load().delta_rule_fwd(*args)
+
+
+def bwd_raw(*args) -> int:
+    return load().delta_rule_bwd(*args)
+
+
+def fwd_timed_raw(*args) -> int:
+    return load().delta_rule_fwd_timed(*args)
+
+
+def bwd_timed_raw(*args) -> int:
+    return load().delta_rule_bwd_timed(*args)
+
+
+def sync_status(stream=None) -> int:
+    s = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    return load().delta_rule_sync_status(s)
+
+
+# ------------------------------------------------------------------------------------------------
+def _p(t):
+    return None if t is None else t.data_ptr()
+
+
+def _variant(v) -> int:
+    return VARIANTS[v] if isinstance(v, str) else int(v)
+
+
+def _check(code, what):
+    if code != DR_OK:
+        raise DeltaRuleError(code, what)
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def delta_rule_fwd(q, k, v, alpha, beta, S0=None, variant="gdn", chunk=64, want_u=True, want_state=True,
+                   workspace: torch.Tensor | None = None, out=None, u=None, S_T=None):
+    """Forward on CUDA tensors.  Returns (o, u or None, S_T or None).
+
+    q, k: [B,T,H,dk]; v: [B,T,H,dv]; alpha: log gate [B,T,H] (gdn) / [B,T,H,dk] (kda) / None (deltanet);
+    beta: [B,T,H]; S0: fp32 [B,H,dk,dv] or None.  All per-token tensors share one dtype (fp32 or bf16).
+    """
+    var = _variant(variant)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = DTYPES[q.dtype]
+    dev = q.device
+    out = torch.empty((B, T, H, dv), dtype=q.dtype, device=dev) if out is None else out
+    if want_u and u is None:
+        u = torch.empty((B, T, H, dv), dtype=q.dtype, device=dev)
+    if want_state and S_T is None:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    need = workspace_size(B, T, H, dk, dv, var, chunk, dt, 0)
+    if workspace is None or workspace.numel() < need:
+        workspace = _workspace(need, dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = fwd_raw(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(out), _p(u), _p(S_T),
+                 B, T, H, dk, dv, var, chunk, dt, _p(workspace), need, stream)
+    _check(rc, "delta_rule_fwd")
+    return out, u, S_T
+
+
+def delta_rule_bwd(q, k, v, alpha, beta, S0, dout, du=None, dS_T=None, variant="gdn", chunk=64,
+                   want_dS0=True, workspace: torch.Tensor | None = None, grads: dict | None = None):
+    """Backward on CUDA tensors.  Returns dict(dq, dk, dv, dalpha (None for deltanet), dbeta, dS0)."""
+    var = _variant(variant)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = DTYPES[q.dtype]
+    dev = q.device
+    g = dict(grads or {})
+    g.setdefault("dq", torch.empty_like(q))
+    g.setdefault("dk", torch.empty_like(k))
+    g.setdefault("dv", torch.empty_like(v))
+    g.setdefault("dalpha", torch.empty_like(alpha) if (var != DR_DELTANET and alpha is not None) else None)
+    g.setdefault("dbeta", torch.empty_like(beta))
+    g.setdefault("dS0", torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if want_dS0 else None)
+    need = workspace_size(B, T, H, dk, dv, var, chunk, dt, 1)
+    if workspace is None or workspace.numel() < need:
+        workspace = _workspace(need, dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = bwd_raw(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(dout), _p(du), _p(dS_T),
+                 _p(g["dq"]), _p(g["dk"]), _p(g["dv"]), _p(g["dalpha"]), _p(g["dbeta"]), _p(g["dS0"]),
+                 B, T, H, dk, dv, var, chunk, dt, _p(workspace), need, stream)
+    _check(rc, "delta_rule_bwd")
+    return g
+
+
+def delta_rule_fwd_host(q, k, v, alpha, beta, S0=None, variant="gdn", chunk=64, device="cuda"):
+    """The forward for host (CPU, ideally pinned) tensors: copy in, compute, copy out."""
+    dev = torch.device(device)
+    cp = [None if x is None else x.to(dev, non_blocking=True) for x in (q, k, v, alpha, beta, S0)]
+    o, u, S = delta_rule_fwd(*cp, variant=variant, chunk=chunk)
+    return o.to("cpu"), u.to("cpu"), S.to("cpu")

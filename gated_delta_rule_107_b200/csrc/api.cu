@@ -1,0 +1,219 @@
+// api.cu -- the C ABI declared in include/delta_rule.h.
+//
+// Argument validation, workspace planning and dispatch.  No compute happens on
+// the host: every step of the path runs in the kernels of simt_path.cu and
+// tc_fwd.cu.  Validation failures return before anything is enqueued.
+#include <limits.h>
+
+#include "../../include/delta_rule.h"
+#include "dr_common.cuh"
+#include "simt_path.cuh"
+#include "tc_path.cuh"
+
+using namespace dr;
+
+namespace {
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Checks shape / enum arguments; fills geo.  Returns DR_OK or an error code.
+int check_shape(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype, Geo *geo) {
+    if (B < 0 || T < 0 || H < 0) return DR_ERR_ARG;
+    if (variant < DR_DELTANET || variant > DR_KDA) return DR_ERR_ARG;
+    if (dtype != DR_F32 && dtype != DR_BF16) return DR_ERR_ARG;
+    if (chunk != 16 && chunk != 32 && chunk != 64) return chunk > 0 ? DR_ERR_UNSUPPORTED : DR_ERR_ARG;
+    if (dk <= 0 || dv <= 0) return DR_ERR_ARG;
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return DR_ERR_UNSUPPORTED;
+    // every element index must fit comfortably in 63 bits; grids in 2^31 - 1 / 65535
+    const double elems = (double)B * T * H * (dk > dv ? dk : dv);
+    if (elems > 9.0e18 / 16) return DR_ERR_ARG;
+    const long long N = T == 0 ? 0 : ((long long)T + chunk - 1) / chunk;
+    if (N > INT_MAX || H > 65535 || B > 65535) return DR_ERR_UNSUPPORTED;
+    geo->B = B; geo->T = T; geo->H = H; geo->dk = dk; geo->dv = dv; geo->C = chunk; geo->N = (int)N;
+    geo->variant = variant;
+    return DR_OK;
+}
+
+// Which kernels serve a call: the tensor-core forward for bf16, d = 128, C = 64.
+bool use_tc_fwd(const Geo &g, int dtype) { return tc_fwd_supported(g, dtype == DR_BF16); }
+
+size_t ws_bytes(const Geo &g, int dtype, bool bwd) {
+    if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
+    if (!bwd && use_tc_fwd(g, dtype)) return tc_fwd_ws_bytes(g);
+    return simt_ws_bytes(g, bwd);
+}
+
+int launch_status(cudaError_t e) { return e == cudaSuccess ? DR_OK : DR_ERR_CUDA; }
+
+// T == 0: S_T := S0 (or 0), dS0 := dS_T (or 0).
+int copy_state(float *dst, const float *src, const Geo &g, cudaStream_t s) {
+    if (!dst) return DR_OK;
+    const size_t bytes = (size_t)g.B * g.H * g.dk * g.dv * sizeof(float);
+    if (bytes == 0) return DR_OK;
+    cudaError_t e = src ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s) : cudaMemsetAsync(dst, 0, bytes, s);
+    return launch_status(e);
+}
+
+}  // namespace
+
+extern "C" size_t delta_rule_workspace_size(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype,
+                                            int for_bwd) {
+    Geo g;
+    if (check_shape(B, T, H, dk, dv, variant, chunk, dtype, &g) != DR_OK) return (size_t)-1;
+    return ws_bytes(g, dtype, for_bwd != 0);
+}
+
+static int fwd_impl(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                    const float *S0, void *out, void *u, float *S_T, int B, int T, int H, int dk, int dv, int variant,
+                    int chunk, int dtype, void *workspace, size_t ws_bytes_given, void *stream, Rec &rec) {
+    Geo g;
+    int rc = check_shape(B, T, H, dk, dv, variant, chunk, dtype, &g);
+    if (rc != DR_OK) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    const bool empty = (size_t)B * H == 0;
+    if (T == 0 || empty) return empty ? DR_OK : copy_state(S_T, S0, g, s);
+    if (!q || !k || !v || !beta || !out) return DR_ERR_ARG;
+    if (variant != DR_DELTANET && !alpha) return DR_ERR_ARG;
+    const void *ptrs[] = {q, k, v, variant != DR_DELTANET ? alpha : nullptr, beta, S0, out, u, S_T};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return DR_ERR_ALIGN;
+    const size_t need = ws_bytes(g, dtype, false);
+    if (need > 0) {
+        if (!workspace || ws_bytes_given < need) return DR_ERR_WORKSPACE;
+        if (((uintptr_t)workspace & 255u) != 0) return DR_ERR_ALIGN;
+    }
+    Tensors t = {};
+    t.q = q; t.k = k; t.v = v; t.alpha = alpha; t.beta = beta; t.S0 = S0; t.out = out; t.u = u; t.S_T = S_T;
+    if (use_tc_fwd(g, dtype)) return launch_status(tc_fwd(g, t, workspace, s, rec));
+    const SimtWs w = simt_ws_carve(g, false, workspace);
+    return launch_status(simt_fwd(g, t, dtype == DR_BF16, w, s, rec));
+}
+
+static int bwd_impl(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                    const float *S0, const void *dout, const void *du, const float *dS_T, void *dq, void *dk_,
+                    void *dv_, void *dalpha, void *dbeta, float *dS0, int B, int T, int H, int dk, int dv, int variant,
+                    int chunk, int dtype, void *workspace, size_t ws_bytes_given, void *stream, Rec &rec) {
+    Geo g;
+    int rc = check_shape(B, T, H, dk, dv, variant, chunk, dtype, &g);
+    if (rc != DR_OK) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    const bool empty = (size_t)B * H == 0;
+    if (T == 0 || empty) return empty ? DR_OK : copy_state(dS0, dS_T, g, s);
+    if (!q || !k || !v || !beta || !dout || !dq || !dk_ || !dv_ || !dbeta) return DR_ERR_ARG;
+    if (variant != DR_DELTANET && (!alpha || !dalpha)) return DR_ERR_ARG;
+    const void *ptrs[] = {q, k, v, variant != DR_DELTANET ? alpha : nullptr, beta, S0, dout, du, dS_T, dq, dk_, dv_,
+                          variant != DR_DELTANET ? dalpha : nullptr, dbeta, dS0};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return DR_ERR_ALIGN;
+    const size_t need = ws_bytes(g, dtype, true);
+    if (!workspace || ws_bytes_given < need) return DR_ERR_WORKSPACE;
+    if (((uintptr_t)workspace & 255u) != 0) return DR_ERR_ALIGN;
+    Tensors t = {};
+    t.q = q; t.k = k; t.v = v; t.alpha = alpha; t.beta = beta; t.S0 = S0;
+    t.dout = dout; t.du = du; t.dS_T = dS_T;
+    t.dq = dq; t.dk = dk_; t.dv = dv_; t.dalpha = dalpha; t.dbeta = dbeta; t.dS0 = dS0;
+    const SimtWs w = simt_ws_carve(g, true, workspace);
+    return launch_status(simt_bwd(g, t, dtype == DR_BF16, w, s, rec));
+}
+
+// Number of kernel launches of one call and their names (launch order).
+static int launch_plan(const Geo &g, int dtype, bool bwd, const char **names, int max_names) {
+    int n = 0;
+    const char *const *src = nullptr;
+    if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
+    if (!bwd && use_tc_fwd(g, dtype)) {
+        n = tc_fwd_launches(names, max_names);
+        return n;
+    }
+    src = bwd ? SIMT_BWD_KERNELS : SIMT_FWD_KERNELS;
+    n = bwd ? 5 : 3;
+    for (int i = 0; names && i < n && i < max_names; ++i) names[i] = src[i];
+    return n;
+}
+
+static int make_rec(const Geo &g, int dtype, bool bwd, void *const *events, int n_events, Rec *rec) {
+    if (n_events == 0 || events == nullptr) return DR_OK;
+    const int n = launch_plan(g, dtype, bwd, nullptr, 0);
+    if (n_events < n + 1) return DR_ERR_ARG;
+    rec->ev = (cudaEvent_t *)events;
+    rec->n = n + 1;
+    return DR_OK;
+}
+
+extern "C" int delta_rule_fwd(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                              const float *S0, void *out, void *u, float *S_T, int B, int T, int H, int dk, int dv,
+                              int variant, int chunk, int dtype, void *workspace, size_t ws_bytes_given,
+                              void *stream) {
+    Rec rec;
+    return fwd_impl(q, k, v, alpha, beta, S0, out, u, S_T, B, T, H, dk, dv, variant, chunk, dtype, workspace,
+                    ws_bytes_given, stream, rec);
+}
+
+extern "C" int delta_rule_fwd_timed(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                                    const float *S0, void *out, void *u, float *S_T, int B, int T, int H, int dk,
+                                    int dv, int variant, int chunk, int dtype, void *workspace, size_t ws_bytes_given,
+                                    void *stream, void *const *events, int n_events) {
+    Geo g;
+    int rc = check_shape(B, T, H, dk, dv, variant, chunk, dtype, &g);
+    if (rc != DR_OK) return rc;
+    Rec rec;
+    rc = make_rec(g, dtype, false, events, n_events, &rec);
+    if (rc != DR_OK) return rc;
+    return fwd_impl(q, k, v, alpha, beta, S0, out, u, S_T, B, T, H, dk, dv, variant, chunk, dtype, workspace,
+                    ws_bytes_given, stream, rec);
+}
+
+extern "C" int delta_rule_bwd(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                              const float *S0, const void *dout, const void *du, const float *dS_T, void *dq,
+                              void *dk_, void *dv_, void *dalpha, void *dbeta, float *dS0, int B, int T, int H, int dk,
+                              int dv, int variant, int chunk, int dtype, void *workspace, size_t ws_bytes_given,
+                              void *stream) {
+    Rec rec;
+    return bwd_impl(q, k, v, alpha, beta, S0, dout, du, dS_T, dq, dk_, dv_, dalpha, dbeta, dS0, B, T, H, dk, dv,
+                    variant, chunk, dtype, workspace, ws_bytes_given, stream, rec);
+}
+
+extern "C" int delta_rule_bwd_timed(const void *q, const void *k, const void *v, const void *alpha,
+                                    const void *beta, const float *S0, const void *dout, const void *du,
+                                    const float *dS_T, void *dq, void *dk_, void *dv_, void *dalpha, void *dbeta,
+                                    float *dS0, int B, int T, int H, int dk, int dv, int variant, int chunk,
+                                    int dtype, void *workspace, size_t ws_bytes_given, void *stream,
+                                    void *const *events, int n_events) {
+    Geo g;
+    int rc = check_shape(B, T, H, dk, dv, variant, chunk, dtype, &g);
+    if (rc != DR_OK) return rc;
+    Rec rec;
+    rc = make_rec(g, dtype, true, events, n_events, &rec);
+    if (rc != DR_OK) return rc;
+    return bwd_impl(q, k, v, alpha, beta, S0, dout, du, dS_T, dq, dk_, dv_, dalpha, dbeta, dS0, B, T, H, dk, dv,
+                    variant, chunk, dtype, workspace, ws_bytes_given, stream, rec);
+}
+
+extern "C" int delta_rule_launches(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype,
+                                   int for_bwd, const char **names, int max_names) {
+    Geo g;
+    const int rc = check_shape(B, T, H, dk, dv, variant, chunk, dtype, &g);
+    if (rc != DR_OK) return rc;
+    return launch_plan(g, dtype, for_bwd != 0, names, max_names);
+}
+
+extern "C" const char *delta_rule_strerror(int code) {
+    switch (code) {
+        case DR_OK: return "ok";
+        case DR_ERR_ARG: return "invalid argument";
+        case DR_ERR_UNSUPPORTED: return "unsupported shape or option";
+        case DR_ERR_ALIGN: return "misaligned pointer (16 B; workspace 256 B)";
+        case DR_ERR_WORKSPACE: return "workspace missing or too small";
+        case DR_ERR_CUDA: return "CUDA error";
+        case DR_ERR_TIMEOUT: return "device wait timed out";
+        default: return "unknown error code";
+    }
+}
+
+extern "C" int delta_rule_sync_status(void *stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return DR_ERR_CUDA;
+    int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, g_dev_error, sizeof(int)) != cudaSuccess) return DR_ERR_CUDA;
+    if (word && cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(int)) != cudaSuccess) return DR_ERR_CUDA;
+    return (word & DEVERR_TIMEOUT) ? DR_ERR_TIMEOUT : DR_OK;
+}

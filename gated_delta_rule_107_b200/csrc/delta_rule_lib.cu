@@ -1,0 +1,5 @@
+// delta_rule_lib.cu -- single translation unit of libdeltarule.so (the device error
+// word and all kernels live in one module, so no relocatable device code is needed).
+#include "simt_path.cu"
+#include "tc_fwd.cu"
+#include "api.cu"

@@ -1,0 +1,668 @@
+// simt_path.cu -- chunkwise gated delta rule on CUDA cores, fp32 arithmetic.
+//
+// This path serves fp32 I/O (where the result must agree with fp64 to ~1e-4,
+// beyond what bf16 tensor-core operands allow) and every shape the tensor-core
+// path does not specialise.  It follows the chunked form of the recurrence of
+// "线性注意力架构演进与Kimi Delta Attention创新实践" section 2.1, solved per chunk
+// with the UT transform of section 6.2 and log-space cumulative gates of
+// section 7.1.  For one (b, h) and chunk of C tokens with incoming state S:
+//
+//   g_r   = sum_{i<=r} log alpha_i          (per channel; broadcast for Gated)
+//   A_ri  = beta_r sum_c k_rc k_ic e^{g_rc - g_ic}          (i < r)
+//   P_ri  =        sum_c q_rc k_ic e^{g_rc - g_ic}          (i <= r)
+//   W     = (I+A)^-1 diag(beta) (e^{g} .* K),  U~ = (I+A)^-1 diag(beta) V
+//   U     = U~ - W S                  (rows are the write values u_t)
+//   O     = (e^{g} .* Q) S + P U
+//   S+    = Diag(e^{g_C}) S + (K .* e^{g_C - g})^T U
+//
+// Every exponent above is of a non-positive number when log alpha <= 0, so no
+// intermediate can overflow (no e^{-g} factorisation is used on this path).
+//
+// Kernels (one CTA of 256 threads each):
+//   k_prep        grid (N, H, B)     g, A, P, then W and U~ by forward substitution
+//   k_scan        grid (dv/32, H, B) serial state chain over chunks, U, S_n
+//   k_out         grid (N, H, B)     O = Qtil S_n + P U
+//   k_scan_bwd    grid (dv/32, H, B) reverse chain: dU_n and dS_{n+1}
+//   k_bwd_state   grid (N, H, B)     dO S^T, -dU S^T, U dS+^T, rowsum(S .* dS+)
+//   k_bwd_intra   grid (N, H, B)     everything inside the chunk -> dq dk dv dbeta dlog-alpha
+#include "simt_path.cuh"
+
+namespace dr {
+
+static constexpr int NT = 256;  // threads per CTA
+static constexpr int JB = 32;   // dv columns per CTA in the scans
+
+template <typename TI> struct IO {
+    const TI *q, *k, *v, *alpha, *beta, *dout, *du;
+    TI *out, *u, *dq, *dk, *dv, *dalpha, *dbeta;
+};
+
+template <typename TI> static IO<TI> io_of(const Tensors &t) {
+    IO<TI> x;
+    x.q = (const TI *)t.q; x.k = (const TI *)t.k; x.v = (const TI *)t.v;
+    x.alpha = (const TI *)t.alpha; x.beta = (const TI *)t.beta;
+    x.dout = (const TI *)t.dout; x.du = (const TI *)t.du;
+    x.out = (TI *)t.out; x.u = (TI *)t.u; x.dq = (TI *)t.dq; x.dk = (TI *)t.dk; x.dv = (TI *)t.dv;
+    x.dalpha = (TI *)t.dalpha; x.dbeta = (TI *)t.dbeta;
+    return x;
+}
+
+// raw log gate of token row `row`, channel c (0 for DeltaNet)
+template <typename TI>
+__device__ __forceinline__ float raw_gate(const Geo &g, const TI *alpha, size_t row, int c) {
+    if (g.variant == VAR_KDA) return to_f(alpha[row * g.dk + c]);
+    if (g.variant == VAR_GATED) return to_f(alpha[row]);
+    return 0.f;
+}
+
+// ---------------------------------------------------------------------------------------------
+// k_prep: per chunk, cumulative gates, A and P, then W and U~ by forward substitution.
+// smem: ks, qs, gs [C][dk]; vs [C][dv]; Am, Pm [C][C]; bs [C]
+template <typename TI>
+__global__ void __launch_bounds__(NT) k_prep(Geo g, IO<TI> io, SimtWs w) {
+    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int C = g.C, DK = g.dk, DV = g.dv;
+    const int t0 = n * C, L = min(C, g.T - t0);
+    extern __shared__ float sm[];
+    float *ks = sm, *qs = ks + C * DK, *gs = qs + C * DK, *vs = gs + C * DK;
+    float *Am = vs + C * DV, *Pm = Am + C * C, *bs = Pm + C * C;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    for (int x = tid; x < C * DK; x += NT) {
+        const int r = x / DK, c = x % DK;
+        float kv = 0.f, qv = 0.f, gv = 0.f;
+        if (r < L) {
+            const size_t row = g.row(b, t0 + r, h);
+            kv = to_f(io.k[row * DK + c]);
+            qv = to_f(io.q[row * DK + c]);
+            gv = raw_gate(g, io.alpha, row, c);
+        }
+        ks[x] = kv; qs[x] = qv; gs[x] = gv;
+    }
+    for (int x = tid; x < C * DV; x += NT) {
+        const int r = x / DV, j = x % DV;
+        vs[x] = r < L ? to_f(io.v[g.row(b, t0 + r, h) * DV + j]) : 0.f;
+    }
+    for (int r = tid; r < C; r += NT) bs[r] = r < L ? to_f(io.beta[g.row(b, t0 + r, h)]) : 0.f;
+    __syncthreads();
+    for (int c = tid; c < DK; c += NT)
+        for (int r = 1; r < C; ++r) gs[r * DK + c] += gs[(r - 1) * DK + c];
+    __syncthreads();
+
+    // A (strictly lower) and P (lower incl. diagonal), one warp per row
+    for (int r = warp; r < C; r += NT / 32) {
+        for (int i = 0; i < C; ++i) {
+            float a = 0.f, p = 0.f;
+            if (i <= r) {
+                if (g.variant == VAR_KDA) {
+                    for (int c = lane; c < DK; c += 32) {
+                        const float e = __expf(gs[r * DK + c] - gs[i * DK + c]);
+                        const float kic = ks[i * DK + c] * e;
+                        a += ks[r * DK + c] * kic;
+                        p += qs[r * DK + c] * kic;
+                    }
+                } else {
+                    for (int c = lane; c < DK; c += 32) {
+                        a += ks[r * DK + c] * ks[i * DK + c];
+                        p += qs[r * DK + c] * ks[i * DK + c];
+                    }
+                }
+                a = warp_sum(a);
+                p = warp_sum(p);
+                if (g.variant == VAR_GATED) {
+                    const float e = __expf(gs[r * DK] - gs[i * DK]);
+                    a *= e;
+                    p *= e;
+                }
+            }
+            if (lane == 0) {
+                Am[r * C + i] = (i < r) ? bs[r] * a : 0.f;
+                Pm[r * C + i] = p;
+            }
+        }
+    }
+    __syncthreads();
+    {
+        const size_t ci = g.chunk(b, h, n);
+        float *Pg = w.P + ci * C * C;
+        for (int x = tid; x < C * C; x += NT) Pg[x] = Pm[x];
+        float *Gg = w.G + ci * C * DK;
+        for (int x = tid; x < C * DK; x += NT) Gg[x] = gs[x];
+    }
+    // right-hand sides: beta e^{g} k and beta v
+    for (int x = tid; x < C * DK; x += NT) ks[x] *= bs[x / DK] * __expf(gs[x]);
+    for (int x = tid; x < C * DV; x += NT) vs[x] *= bs[x / DV];
+    __syncthreads();
+    // forward substitution (I + A) X = R, one thread per column of [W | U~]
+    for (int x = tid; x < DK + DV; x += NT) {
+        float *col = x < DK ? ks + x : vs + (x - DK);
+        const int ld = x < DK ? DK : DV;
+        for (int r = 1; r < C; ++r) {
+            float acc = col[r * ld];
+            for (int i = 0; i < r; ++i) acc -= Am[r * C + i] * col[i * ld];
+            col[r * ld] = acc;
+        }
+    }
+    __syncthreads();
+    {
+        const size_t ci = g.chunk(b, h, n);
+        float *Wg = w.W + ci * C * DK;
+        for (int x = tid; x < C * DK; x += NT) Wg[x] = ks[x];
+        float *Ug = w.Ut + ci * C * DV;
+        for (int x = tid; x < C * DV; x += NT) Ug[x] = vs[x];
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// k_scan: serial over chunks for one (b, h) and 32 state columns.
+// smem: S [dk][JB]; Ws, Kb [C][dk]; Us [C][JB]; gam [dk]
+template <typename TI>
+__global__ void __launch_bounds__(NT) k_scan(Geo g, IO<TI> io, SimtWs w, const float *S0, float *ST, int write_u) {
+    const int j0 = blockIdx.x * JB, h = blockIdx.y, b = blockIdx.z;
+    const int C = g.C, DK = g.dk, DV = g.dv;
+    extern __shared__ float sm[];
+    float *S = sm, *Ws = S + DK * JB, *Kb = Ws + C * DK, *Us = Kb + C * DK, *gam = Us + C * JB;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const size_t soff = ((size_t)b * g.H + h) * DK * DV;
+
+    for (int x = tid; x < DK * JB; x += NT) {
+        const int c = x / JB, j = x % JB;
+        S[x] = S0 ? S0[soff + (size_t)c * DV + j0 + j] : 0.f;
+    }
+    for (int n = 0; n < g.N; ++n) {
+        const int t0 = n * C, L = min(C, g.T - t0);
+        const size_t ci = g.chunk(b, h, n);
+        const float *Wg = w.W + ci * C * DK, *Gg = w.G + ci * C * DK, *Ug = w.Ut + ci * C * DV;
+        __syncthreads();
+        for (int x = tid; x < C * DK; x += NT) {
+            const int r = x / DK, c = x % DK;
+            Ws[x] = Wg[x];
+            const float kv = r < L ? to_f(io.k[g.row(b, t0 + r, h) * DK + c]) : 0.f;
+            Kb[x] = kv * __expf(Gg[(C - 1) * DK + c] - Gg[x]);
+        }
+        for (int c = tid; c < DK; c += NT) gam[c] = __expf(Gg[(C - 1) * DK + c]);
+        for (int x = tid; x < C * JB; x += NT) Us[x] = Ug[(x / JB) * DV + j0 + (x % JB)];
+        {
+            float *Sg = w.Sn + ci * DK * DV;
+            for (int x = tid; x < DK * JB; x += NT) Sg[(x / JB) * DV + j0 + (x % JB)] = S[x];
+        }
+        __syncthreads();
+        // U = U~ - W S
+        for (int r = warp; r < C; r += NT / 32) {
+            float acc = Us[r * JB + lane];
+            for (int c = 0; c < DK; ++c) acc -= Ws[r * DK + c] * S[c * JB + lane];
+            Us[r * JB + lane] = acc;
+            w.Un[(ci * C + r) * DV + j0 + lane] = acc;
+            if (write_u && r < L) io.u[g.row(b, t0 + r, h) * DV + j0 + lane] = from_f<TI>(acc);
+        }
+        __syncthreads();
+        // S <- Diag(gamma_C) S + Kbar^T U
+        for (int c = warp; c < DK; c += NT / 32) {
+            float acc = gam[c] * S[c * JB + lane];
+            for (int r = 0; r < C; ++r) acc += Kb[r * DK + c] * Us[r * JB + lane];
+            S[c * JB + lane] = acc;
+        }
+    }
+    __syncthreads();
+    if (ST)
+        for (int x = tid; x < DK * JB; x += NT) ST[soff + (size_t)(x / JB) * DV + j0 + (x % JB)] = S[x];
+}
+
+// ---------------------------------------------------------------------------------------------
+// k_out: O = Qtil S_n + P U for one chunk.
+// smem: Qs [C][dk]; Pm [C][C]; Sb [dk][JB]; Ub [C][JB]
+template <typename TI>
+__global__ void __launch_bounds__(NT) k_out(Geo g, IO<TI> io, SimtWs w) {
+    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int C = g.C, DK = g.dk, DV = g.dv;
+    const int t0 = n * C, L = min(C, g.T - t0);
+    extern __shared__ float sm[];
+    float *Qs = sm, *Pm = Qs + C * DK, *Sb = Pm + C * C, *Ub = Sb + DK * JB;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const size_t ci = g.chunk(b, h, n);
+    const float *Gg = w.G + ci * C * DK;
+    for (int x = tid; x < C * DK; x += NT) {
+        const int r = x / DK, c = x % DK;
+        Qs[x] = r < L ? to_f(io.q[g.row(b, t0 + r, h) * DK + c]) * __expf(Gg[x]) : 0.f;
+    }
+    for (int x = tid; x < C * C; x += NT) Pm[x] = w.P[ci * C * C + x];
+    for (int jb = 0; jb < DV; jb += JB) {
+        __syncthreads();
+        for (int x = tid; x < DK * JB; x += NT) Sb[x] = w.Sn[ci * DK * DV + (size_t)(x / JB) * DV + jb + (x % JB)];
+        for (int x = tid; x < C * JB; x += NT) Ub[x] = w.Un[(ci * C + x / JB) * DV + jb + (x % JB)];
+        __syncthreads();
+        for (int r = warp; r < L; r += NT / 32) {
+            float acc = 0.f;
+            for (int c = 0; c < DK; ++c) acc += Qs[r * DK + c] * Sb[c * JB + lane];
+            for (int i = 0; i <= r; ++i) acc += Pm[r * C + i] * Ub[i * JB + lane];
+            io.out[g.row(b, t0 + r, h) * DV + jb + lane] = from_f<TI>(acc);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// k_scan_bwd: reverse chain over chunks for one (b, h) and 32 columns:
+//   dU_n = du_n + P^T dO_n + Kbar dS_{n+1};  dS_n = Diag(gamma_C) dS_{n+1} + Qtil^T dO_n - W^T dU_n
+// smem: dS [dk][JB]; Qs, Ws, Kb [C][dk]; Pm [C][C]; dOs, dUs [C][JB]; gam [dk]
+template <typename TI>
+__global__ void __launch_bounds__(NT) k_scan_bwd(Geo g, IO<TI> io, SimtWs w, const float *dST, float *dS0) {
+    const int j0 = blockIdx.x * JB, h = blockIdx.y, b = blockIdx.z;
+    const int C = g.C, DK = g.dk, DV = g.dv;
+    extern __shared__ float sm[];
+    float *dS = sm, *Qs = dS + DK * JB, *Ws = Qs + C * DK, *Kb = Ws + C * DK, *Pm = Kb + C * DK;
+    float *dOs = Pm + C * C, *dUs = dOs + C * JB, *gam = dUs + C * JB;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const size_t soff = ((size_t)b * g.H + h) * DK * DV;
+    for (int x = tid; x < DK * JB; x += NT) dS[x] = dST ? dST[soff + (size_t)(x / JB) * DV + j0 + (x % JB)] : 0.f;
+    for (int n = g.N - 1; n >= 0; --n) {
+        const int t0 = n * C, L = min(C, g.T - t0);
+        const size_t ci = g.chunk(b, h, n);
+        const float *Wg = w.W + ci * C * DK, *Gg = w.G + ci * C * DK;
+        __syncthreads();
+        for (int x = tid; x < C * DK; x += NT) {
+            const int r = x / DK, c = x % DK;
+            float qv = 0.f, kv = 0.f;
+            if (r < L) {
+                const size_t row = g.row(b, t0 + r, h);
+                qv = to_f(io.q[row * DK + c]);
+                kv = to_f(io.k[row * DK + c]);
+            }
+            Qs[x] = qv * __expf(Gg[x]);
+            Kb[x] = kv * __expf(Gg[(C - 1) * DK + c] - Gg[x]);
+            Ws[x] = Wg[x];
+        }
+        for (int c = tid; c < DK; c += NT) gam[c] = __expf(Gg[(C - 1) * DK + c]);
+        for (int x = tid; x < C * C; x += NT) Pm[x] = w.P[ci * C * C + x];
+        for (int x = tid; x < C * JB; x += NT) {
+            const int r = x / JB, j = x % JB;
+            float o = 0.f, uu = 0.f;
+            if (r < L) {
+                const size_t row = g.row(b, t0 + r, h);
+                o = io.dout ? to_f(io.dout[row * DV + j0 + j]) : 0.f;
+                uu = io.du ? to_f(io.du[row * DV + j0 + j]) : 0.f;
+            }
+            dOs[x] = o;
+            dUs[x] = uu;
+        }
+        {
+            float *dSg = w.dSn + ci * DK * DV;
+            for (int x = tid; x < DK * JB; x += NT) dSg[(x / JB) * DV + j0 + (x % JB)] = dS[x];
+        }
+        __syncthreads();
+        for (int r = warp; r < C; r += NT / 32) {
+            float acc = dUs[r * JB + lane];
+            for (int rr = r; rr < C; ++rr) acc += Pm[rr * C + r] * dOs[rr * JB + lane];
+            for (int c = 0; c < DK; ++c) acc += Kb[r * DK + c] * dS[c * JB + lane];
+            dUs[r * JB + lane] = acc;
+            w.dUn[(ci * C + r) * DV + j0 + lane] = acc;
+        }
+        __syncthreads();
+        for (int c = warp; c < DK; c += NT / 32) {
+            float acc = gam[c] * dS[c * JB + lane];
+            for (int r = 0; r < C; ++r) acc += Qs[r * DK + c] * dOs[r * JB + lane] - Ws[r * DK + c] * dUs[r * JB + lane];
+            dS[c * JB + lane] = acc;
+        }
+    }
+    __syncthreads();
+    if (dS0)
+        for (int x = tid; x < DK * JB; x += NT) dS0[soff + (size_t)(x / JB) * DV + j0 + (x % JB)] = dS[x];
+}
+
+// ---------------------------------------------------------------------------------------------
+// k_bwd_state: the chunk's products with S_n and dS_{n+1}:
+//   Qd = dO S^T,  dWm = -dU S^T,  Tm = U dS+^T  ([C][dk] each),  RS = rowsum(S .* dS+)  ([dk])
+// smem: Qd, dWm, Tm [C][dk]; Sb, dSb [dk][JB+1]; dOb, dUb, Ub [C][JB]; rs [dk]
+template <typename TI>
+__global__ void __launch_bounds__(NT) k_bwd_state(Geo g, IO<TI> io, SimtWs w) {
+    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int C = g.C, DK = g.dk, DV = g.dv;
+    const int t0 = n * C, L = min(C, g.T - t0);
+    constexpr int LD = JB + 1;
+    extern __shared__ float sm[];
+    float *Qd = sm, *dWm = Qd + C * DK, *Tm = dWm + C * DK, *Sb = Tm + C * DK, *dSb = Sb + DK * LD;
+    float *dOb = dSb + DK * LD, *dUb = dOb + C * JB, *Ub = dUb + C * JB, *rs = Ub + C * JB;
+    const int tid = threadIdx.x;
+    const size_t ci = g.chunk(b, h, n);
+    for (int x = tid; x < C * DK; x += NT) Qd[x] = dWm[x] = Tm[x] = 0.f;
+    for (int c = tid; c < DK; c += NT) rs[c] = 0.f;
+    for (int jb = 0; jb < DV; jb += JB) {
+        __syncthreads();
+        for (int x = tid; x < DK * JB; x += NT) {
+            const int c = x / JB, j = x % JB;
+            Sb[c * LD + j] = w.Sn[ci * DK * DV + (size_t)c * DV + jb + j];
+            dSb[c * LD + j] = w.dSn[ci * DK * DV + (size_t)c * DV + jb + j];
+        }
+        for (int x = tid; x < C * JB; x += NT) {
+            const int r = x / JB, j = x % JB;
+            dOb[x] = (r < L && io.dout) ? to_f(io.dout[g.row(b, t0 + r, h) * DV + jb + j]) : 0.f;
+            dUb[x] = w.dUn[(ci * C + r) * DV + jb + j];
+            Ub[x] = w.Un[(ci * C + r) * DV + jb + j];
+        }
+        __syncthreads();
+        for (int x = tid; x < C * DK; x += NT) {
+            const int r = x / DK, c = x % DK;
+            float a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            for (int j = 0; j < JB; ++j) {
+                const float s = Sb[c * LD + j];
+                a1 += dOb[r * JB + j] * s;
+                a2 += dUb[r * JB + j] * s;
+                a3 += Ub[r * JB + j] * dSb[c * LD + j];
+            }
+            Qd[x] += a1;
+            dWm[x] -= a2;
+            Tm[x] += a3;
+        }
+        for (int c = tid; c < DK; c += NT) {
+            float a = 0.f;
+            for (int j = 0; j < JB; ++j) a += Sb[c * LD + j] * dSb[c * LD + j];
+            rs[c] += a;
+        }
+    }
+    __syncthreads();
+    for (int x = tid; x < C * DK; x += NT) {
+        w.Qd[ci * C * DK + x] = Qd[x];
+        w.dWm[ci * C * DK + x] = dWm[x];
+        w.Tm[ci * C * DK + x] = Tm[x];
+    }
+    for (int c = tid; c < DK; c += NT) w.RS[ci * DK + c] = rs[c];
+}
+
+// ---------------------------------------------------------------------------------------------
+// k_bwd_intra: all remaining gradients of one chunk.
+//   [dB_k | dB_v] = (I+A)^-T [dW | dU]                         (back substitution)
+//   dA_ri = -(dB_k,r . W_i + dB_v,r . U~_i)  (i<r);  dM = diag(beta) dA
+//   dP_ri = dO_r . U_i  (i<=r)
+//   then the gradients through e^{g} q, e^{g} k, k e^{-g} pairs, k e^{g_C - g}, e^{g_C},
+//   beta, and the reverse in-chunk cumsum of dg into d log alpha.
+// smem: ks, qs, gs [C][dk]; Y [C][dk+dv]; M, dM, dP [C][C]; bs, dbs, red [C]
+template <typename TI>
+__global__ void __launch_bounds__(NT) k_bwd_intra(Geo g, IO<TI> io, SimtWs w) {
+    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int C = g.C, DK = g.dk, DV = g.dv, DY = g.dk + g.dv;
+    const int t0 = n * C, L = min(C, g.T - t0);
+    extern __shared__ float sm[];
+    float *ks = sm, *qs = ks + C * DK, *gs = qs + C * DK, *Y = gs + C * DK;
+    float *M = Y + C * DY, *dM = M + C * C, *dP = dM + C * C, *bs = dP + C * C, *dbs = bs + C, *red = dbs + C;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool kda = g.variant == VAR_KDA;
+    const size_t ci = g.chunk(b, h, n);
+    const float *Gg = w.G + ci * C * DK;
+
+    for (int x = tid; x < C * DK; x += NT) {
+        const int r = x / DK, c = x % DK;
+        float kv = 0.f, qv = 0.f;
+        if (r < L) {
+            const size_t row = g.row(b, t0 + r, h);
+            kv = to_f(io.k[row * DK + c]);
+            qv = to_f(io.q[row * DK + c]);
+        }
+        ks[x] = kv; qs[x] = qv; gs[x] = Gg[x];
+        Y[r * DY + c] = w.dWm[ci * C * DK + x];
+    }
+    for (int x = tid; x < C * DV; x += NT) Y[(x / DV) * DY + DK + (x % DV)] = w.dUn[ci * C * DV + x];
+    for (int r = tid; r < C; r += NT) {
+        bs[r] = r < L ? to_f(io.beta[g.row(b, t0 + r, h)]) : 0.f;
+        dbs[r] = 0.f;
+    }
+    __syncthreads();
+    // M_ri = sum_c k_rc k_ic e^{g_rc - g_ic}  (i < r)
+    for (int r = warp; r < C; r += NT / 32) {
+        for (int i = 0; i < C; ++i) {
+            float m = 0.f;
+            if (i < r) {
+                if (kda) {
+                    for (int c = lane; c < DK; c += 32) m += ks[r * DK + c] * ks[i * DK + c] * __expf(gs[r * DK + c] - gs[i * DK + c]);
+                } else {
+                    for (int c = lane; c < DK; c += 32) m += ks[r * DK + c] * ks[i * DK + c];
+                }
+                m = warp_sum(m);
+                if (g.variant == VAR_GATED) m *= __expf(gs[r * DK] - gs[i * DK]);
+            }
+            if (lane == 0) M[r * C + i] = m;
+        }
+    }
+    __syncthreads();
+    // back substitution: Y_i -= sum_{r>i} beta_r M_ri Y_r, i descending
+    for (int x = tid; x < DY; x += NT) {
+        for (int i = C - 2; i >= 0; --i) {
+            float acc = Y[i * DY + x];
+            for (int r = i + 1; r < C; ++r) acc -= bs[r] * M[r * C + i] * Y[r * DY + x];
+            Y[i * DY + x] = acc;
+        }
+    }
+    __syncthreads();
+    // dA, dM = beta dA, dbeta (A part), dP
+    {
+        const float *Wg = w.W + ci * C * DK, *Ug = w.Ut + ci * C * DV, *Un = w.Un + ci * C * DV;
+        for (int r = warp; r < C; r += NT / 32) {
+            float db = 0.f;
+            for (int i = 0; i < C; ++i) {
+                float da = 0.f, dp = 0.f;
+                if (i < r) {
+                    for (int c = lane; c < DK; c += 32) da += Y[r * DY + c] * Wg[i * DK + c];
+                    for (int j = lane; j < DV; j += 32) da += Y[r * DY + DK + j] * Ug[i * DV + j];
+                    da = -warp_sum(da);
+                    db += da * M[r * C + i];
+                }
+                if (i <= r && r < L && io.dout) {
+                    const size_t row = g.row(b, t0 + r, h);
+                    for (int j = lane; j < DV; j += 32) dp += to_f(io.dout[row * DV + j]) * Un[i * DV + j];
+                    dp = warp_sum(dp);
+                }
+                if (lane == 0) {
+                    dM[r * C + i] = bs[r] * da;
+                    dP[r * C + i] = dp;
+                }
+            }
+            if (lane == 0) dbs[r] += db;
+        }
+    }
+    __syncthreads();
+    // per (r, c) gradients; dg_rc overwrites Y[r][c] (dB_k) -- each entry touched by one thread
+    {
+        const float *Qd = w.Qd + ci * C * DK, *Tm = w.Tm + ci * C * DK;
+        for (int r = warp; r < C; r += NT / 32) {
+            float dbk = 0.f;
+            const size_t row = g.row(b, t0 + min(r, L - 1), h);
+            for (int c = lane; c < DK; c += 32) {
+                const float grc = gs[r * DK + c], gam = __expf(grc), kv = ks[r * DK + c], qv = qs[r * DK + c];
+                const float gL = gs[(C - 1) * DK + c];
+                float X = 0.f, Yv = 0.f, Z = 0.f;
+                for (int i = 0; i <= r; ++i) {
+                    const float e = __expf(grc - gs[i * DK + c]) * ks[i * DK + c];
+                    X += dP[r * C + i] * e;
+                    Yv += dM[r * C + i] * e;  // dM[r][r] == 0
+                }
+                for (int rr = r; rr < C; ++rr) {
+                    const float e = __expf(gs[rr * DK + c] - grc);
+                    Z += (dM[rr * C + r] * ks[rr * DK + c] + dP[rr * C + r] * qs[rr * DK + c]) * e;
+                }
+                const float qd = Qd[r * DK + c], tm = Tm[r * DK + c], dBk = Y[r * DY + c];
+                const float eb = __expf(gL - grc);
+                const float dq = gam * qd + X;
+                const float dk = Yv + Z + bs[r] * gam * dBk + eb * tm;
+                const float dg = qv * (gam * qd + X) + kv * (Yv - Z) + bs[r] * gam * kv * dBk - kv * eb * tm;
+                dbk += gam * kv * dBk;
+                Y[r * DY + c] = dg;
+                if (r < L) {
+                    io.dq[row * DK + c] = from_f<TI>(dq);
+                    io.dk[row * DK + c] = from_f<TI>(dk);
+                }
+            }
+            float dbv = 0.f;
+            for (int j = lane; j < DV; j += 32) {
+                const float dBv = Y[r * DY + DK + j];
+                if (r < L) {
+                    dbv += dBv * to_f(io.v[row * DV + j]);
+                    io.dv[row * DV + j] = from_f<TI>(bs[r] * dBv);
+                }
+            }
+            const float s = warp_sum(dbk + dbv);
+            if (lane == 0) dbs[r] += s;
+        }
+    }
+    __syncthreads();
+    if (g.variant == VAR_DELTANET) {
+        for (int r = tid; r < L; r += NT) io.dbeta[g.row(b, t0 + r, h)] = from_f<TI>(dbs[r]);
+        return;
+    }
+    // dg_C: Kbar . Tm summed over rows, and gamma_C rowsum(S .* dS+); added to the last row
+    {
+        const float *Tm = w.Tm + ci * C * DK;
+        for (int c = tid; c < DK; c += NT) {
+            const float gL = gs[(C - 1) * DK + c];
+            float acc = __expf(gL) * w.RS[ci * DK + c];
+            for (int r = 0; r < C; ++r) acc += ks[r * DK + c] * __expf(gL - gs[r * DK + c]) * Tm[r * DK + c];
+            Y[(C - 1) * DY + c] += acc;
+        }
+    }
+    __syncthreads();
+    if (kda) {
+        for (int c = tid; c < DK; c += NT) {
+            float run = 0.f;
+            for (int r = C - 1; r >= 0; --r) {
+                run += Y[r * DY + c];
+                if (r < L) io.dalpha[g.row(b, t0 + r, h) * DK + c] = from_f<TI>(run);
+            }
+        }
+    } else {
+        for (int r = warp; r < C; r += NT / 32) {
+            float s = 0.f;
+            for (int c = lane; c < DK; c += 32) s += Y[r * DY + c];
+            s = warp_sum(s);
+            if (lane == 0) red[r] = s;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            float run = 0.f;
+            for (int r = C - 1; r >= 0; --r) {
+                run += red[r];
+                if (r < L) io.dalpha[g.row(b, t0 + r, h)] = from_f<TI>(run);
+            }
+        }
+    }
+    for (int r = tid; r < L; r += NT) io.dbeta[g.row(b, t0 + r, h)] = from_f<TI>(dbs[r]);
+}
+
+// ---------------------------------------------------------------------------------------------
+// host side
+static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t simt_ws_bytes(const Geo &g, bool bwd) {
+    const size_t nc = (size_t)g.B * g.H * g.N, C = g.C, DK = g.dk, DV = g.dv;
+    size_t s = 0;
+    s += al256(nc * C * DK * 4);   // W
+    s += al256(nc * C * DV * 4);   // Ut
+    s += al256(nc * C * DK * 4);   // G
+    s += al256(nc * C * C * 4);    // P
+    s += al256(nc * DK * DV * 4);  // Sn
+    s += al256(nc * C * DV * 4);   // Un
+    if (bwd) {
+        s += al256(nc * DK * DV * 4);     // dSn
+        s += al256(nc * C * DV * 4);      // dUn
+        s += 3 * al256(nc * C * DK * 4);  // Qd dWm Tm
+        s += al256(nc * DK * 4);          // RS
+    }
+    return s;
+}
+
+SimtWs simt_ws_carve(const Geo &g, bool bwd, void *base) {
+    const size_t nc = (size_t)g.B * g.H * g.N, C = g.C, DK = g.dk, DV = g.dv;
+    char *p = (char *)base;
+    auto take = [&](size_t bytes) { float *r = (float *)p; p += al256(bytes); return r; };
+    SimtWs w = {};
+    w.W = take(nc * C * DK * 4);
+    w.Ut = take(nc * C * DV * 4);
+    w.G = take(nc * C * DK * 4);
+    w.P = take(nc * C * C * 4);
+    w.Sn = take(nc * DK * DV * 4);
+    w.Un = take(nc * C * DV * 4);
+    if (bwd) {
+        w.dSn = take(nc * DK * DV * 4);
+        w.dUn = take(nc * C * DV * 4);
+        w.Qd = take(nc * C * DK * 4);
+        w.dWm = take(nc * C * DK * 4);
+        w.Tm = take(nc * C * DK * 4);
+        w.RS = take(nc * DK * 4);
+    }
+    return w;
+}
+
+template <typename K> static cudaError_t prep_attr(K kern, size_t smem) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+}
+
+#define DR_TRY(x)                                \
+    do {                                         \
+        cudaError_t e__ = (x);                   \
+        if (e__ != cudaSuccess) return e__;      \
+    } while (0)
+
+const char *const SIMT_FWD_KERNELS[3] = {"k_prep", "k_scan", "k_out"};
+const char *const SIMT_BWD_KERNELS[5] = {"k_prep", "k_scan", "k_scan_bwd", "k_bwd_state", "k_bwd_intra"};
+
+template <typename TI>
+static cudaError_t forward_chain(const Geo &g, const IO<TI> &io, const SimtWs &w, const float *S0, float *ST,
+                                 int write_u, cudaStream_t s, Rec &rec) {
+    const size_t C = g.C, DK = g.dk, DV = g.dv;
+    const dim3 gc(g.N, g.H, g.B), gs(g.dv / JB, g.H, g.B);
+    const size_t sm_prep = 4 * (3 * C * DK + C * DV + 2 * C * C + C);
+    DR_TRY(prep_attr(k_prep<TI>, sm_prep));
+    const size_t sm_scan = 4 * (DK * JB + 2 * C * DK + C * JB + DK);
+    DR_TRY(prep_attr(k_scan<TI>, sm_scan));
+    rec.mark(s);
+    k_prep<TI><<<gc, NT, sm_prep, s>>>(g, io, w);
+    DR_TRY(cudaGetLastError());
+    rec.mark(s);
+    k_scan<TI><<<gs, NT, sm_scan, s>>>(g, io, w, S0, ST, write_u);
+    return cudaGetLastError();
+}
+
+template <typename TI>
+static cudaError_t fwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec) {
+    const IO<TI> io = io_of<TI>(t);
+    const size_t C = g.C, DK = g.dk;
+    const size_t sm_out = 4 * (C * DK + C * C + DK * JB + C * JB);
+    DR_TRY(prep_attr(k_out<TI>, sm_out));
+    DR_TRY(forward_chain<TI>(g, io, w, t.S0, t.S_T, t.u != nullptr, s, rec));
+    rec.mark(s);
+    k_out<TI><<<dim3(g.N, g.H, g.B), NT, sm_out, s>>>(g, io, w);
+    DR_TRY(cudaGetLastError());
+    rec.mark(s);
+    return cudaSuccess;
+}
+
+template <typename TI>
+static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec) {
+    const IO<TI> io = io_of<TI>(t);
+    const size_t C = g.C, DK = g.dk, DV = g.dv;
+    const dim3 gc(g.N, g.H, g.B), gs(g.dv / JB, g.H, g.B);
+    const size_t sm_sb = 4 * (DK * JB + 3 * C * DK + C * C + 2 * C * JB + DK);
+    const size_t sm_st = 4 * (3 * C * DK + 2 * DK * (JB + 1) + 3 * C * JB + DK);
+    const size_t sm_in = 4 * (3 * C * DK + C * (DK + DV) + 3 * C * C + 3 * C);
+    DR_TRY(prep_attr(k_scan_bwd<TI>, sm_sb));
+    DR_TRY(prep_attr(k_bwd_state<TI>, sm_st));
+    DR_TRY(prep_attr(k_bwd_intra<TI>, sm_in));
+    DR_TRY(forward_chain<TI>(g, io, w, t.S0, nullptr, 0, s, rec));
+    rec.mark(s);
+    k_scan_bwd<TI><<<gs, NT, sm_sb, s>>>(g, io, w, t.dS_T, t.dS0);
+    DR_TRY(cudaGetLastError());
+    rec.mark(s);
+    k_bwd_state<TI><<<gc, NT, sm_st, s>>>(g, io, w);
+    DR_TRY(cudaGetLastError());
+    rec.mark(s);
+    k_bwd_intra<TI><<<gc, NT, sm_in, s>>>(g, io, w);
+    DR_TRY(cudaGetLastError());
+    rec.mark(s);
+    return cudaSuccess;
+}
+
+cudaError_t simt_fwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec) {
+    return bf16 ? fwd_t<__nv_bfloat16>(g, t, w, s, rec) : fwd_t<float>(g, t, w, s, rec);
+}
+
+cudaError_t simt_bwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec) {
+    return bf16 ? bwd_t<__nv_bfloat16>(g, t, w, s, rec) : bwd_t<float>(g, t, w, s, rec);
+}
+
+}  // namespace dr

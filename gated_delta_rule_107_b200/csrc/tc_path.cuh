@@ -1,0 +1,13 @@
+// tc_path.cuh -- the tcgen05 tensor-core path (bf16 I/O, dk = dv = 128, chunk 64).
+#pragma once
+#include "dr_common.cuh"
+
+namespace dr {
+
+bool tc_fwd_supported(const Geo &g, bool bf16);
+size_t tc_fwd_ws_bytes(const Geo &g);
+cudaError_t tc_fwd(const Geo &g, const Tensors &t, void *workspace, cudaStream_t s, Rec &rec);
+// number of launches of tc_fwd and their names
+int tc_fwd_launches(const char **names, int max_names);
+
+}  // namespace dr

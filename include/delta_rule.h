@@ -1,0 +1,155 @@
+/*
+ * delta_rule.h -- C ABI of the B200 (sm_100a) chunkwise gated delta-rule library
+ * (libdeltarule.so, built from gated_delta_rule_107_b200/csrc).
+ *
+ * The operation.  For every batch b and head h, with a state S in R^{dk x dv}
+ * (row c = key channel), the library evaluates the recurrence of
+ * "线性注意力架构演进与Kimi Delta Attention创新实践" (Kimi Delta Attention page),
+ * section 2.1:
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ * for three variants ("线性注意力架构：机制、权衡与跨层路由" explainer, core
+ * method 1; ETH news article, section 二):
+ *     DR_DELTANET  alpha_t == 1                      (no gate input)
+ *     DR_GATED     one scalar alpha_t per token, head (Gated DeltaNet)
+ *     DR_KDA       alpha_t in (0,1)^dk per channel    (Kimi Delta Attention)
+ * and also returns the per-token write value that Cross-Layer Value Routing
+ * forwards to the next layer (explainer section 4; chatpaper abstract):
+ *     u_t = beta_t (v_t - (Diag(alpha_t) S_{t-1})^T k_t),
+ * so that S_t = Diag(alpha_t) S_{t-1} + k_t u_t^T.
+ *
+ * It is computed chunk by chunk (chunks of `chunk` tokens, page section 6.1)
+ * with the UT / WY transform of each chunk's triangular system (section 6.2)
+ * and in-chunk cumulative gates accumulated in log space (section 7.1); the
+ * state is carried in fp32 (section 7.2).  The result does not depend on the
+ * chunk size except through rounding.
+ *
+ * Conventions shared by every entry point
+ *   Layout     token-major, contiguous, row-major:
+ *                q, k, dq, dk             [B, T, H, dk]
+ *                v, out, u, dout, du, dv  [B, T, H, dv]
+ *                alpha, dalpha            [B, T, H] (DR_GATED) or [B, T, H, dk] (DR_KDA);
+ *                                         unused for DR_DELTANET (may be NULL)
+ *                beta, dbeta              [B, T, H]
+ *                S0, S_T, dS_T, dS0       [B, H, dk, dv], always fp32
+ *   alpha      is the LOG gate, log(alpha_t) <= 0 (any real value is accepted;
+ *              positive values grow the state).
+ *   dtype      DR_F32 or DR_BF16: the element type of every per-token tensor
+ *              (q, k, v, alpha, beta, out, u and all their gradients).  States are
+ *              fp32.  Arithmetic is fp32 with fp32 accumulation; bf16 results are
+ *              rounded to nearest-even once, at the store.
+ *   Shapes     B, H >= 0; T >= 0; dk, dv in {64, 128}; chunk in {16, 32, 64}.
+ *              T need not be a multiple of chunk (the tail chunk is masked).
+ *              T == 0 is valid: the forward copies S0 (or zeros) to S_T and the
+ *              backward copies dS_T (or zeros) to dS0.
+ *   Pointers   device pointers (cudaMalloc / torch CUDA memory), 16-byte aligned.
+ *              The caller owns every buffer; the library allocates nothing, keeps
+ *              no pointer after returning and has no global state except the
+ *              device error word below.  Inputs are never written.  Outputs must
+ *              not alias inputs or each other.
+ *   Workspace  caller-provided device scratch of at least
+ *              delta_rule_workspace_size(...) bytes, 256-byte aligned; its
+ *              contents on entry do not matter.  Two calls that run at the same
+ *              time need distinct workspaces.
+ *   Stream     `stream` is a cudaStream_t (NULL = the legacy default stream).  All
+ *              work is enqueued on it; the call returns without synchronising.
+ *   Errors     every entry point validates its arguments first and returns a
+ *              negative DR_ERR_* code without launching anything when they are
+ *              bad.  Launch failures return DR_ERR_CUDA.  Faults detected on the
+ *              device (a bounded wait that ran out) set a device error word that
+ *              delta_rule_sync_status() reports.  Nothing prints, throws or aborts.
+ */
+#ifndef DELTA_RULE_H
+#define DELTA_RULE_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { DR_DELTANET = 0, DR_GATED = 1, DR_KDA = 2 } dr_variant;
+typedef enum { DR_F32 = 0, DR_BF16 = 1 } dr_dtype;
+
+enum {
+    DR_OK = 0,
+    DR_ERR_ARG = -1,         /* bad shape, enum value, or missing required pointer */
+    DR_ERR_UNSUPPORTED = -2, /* well-formed but not implemented (e.g. dk = 96)      */
+    DR_ERR_ALIGN = -3,       /* a pointer is not 16-byte (workspace: 256-byte) aligned */
+    DR_ERR_WORKSPACE = -4,   /* workspace missing or smaller than required          */
+    DR_ERR_CUDA = -5,        /* a CUDA runtime call or kernel launch failed         */
+    DR_ERR_TIMEOUT = -6      /* a device-side bounded wait expired (see sync_status) */
+};
+
+/*
+ * Bytes of workspace that delta_rule_fwd (for_bwd = 0) or delta_rule_bwd
+ * (for_bwd = 1) needs for these arguments.  Returns 0 when no workspace is
+ * needed, and (size_t)-1 when the arguments are invalid.
+ */
+size_t delta_rule_workspace_size(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype,
+                                 int for_bwd);
+
+/*
+ * Forward.  Evaluates the recurrence above from the initial state S0
+ * (NULL = zero) and writes
+ *   out  o_t = S_t^T q_t                                   (required)
+ *   u    the write values u_t                              (NULL = not written)
+ *   S_T  the state after the last token, fp32              (NULL = not written)
+ */
+int delta_rule_fwd(const void *q, const void *k, const void *v, const void *alpha, const void *beta, const float *S0,
+                   void *out, void *u, float *S_T, int B, int T, int H, int dk, int dv, int variant, int chunk,
+                   int dtype, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Backward.  Gradients of L = <dout, o> + <du, u> + <dS_T, S_T> with respect to
+ * every forward input, for the same forward arguments.  du and dS_T may be NULL
+ * (treated as zero).  Outputs: dq, dk_, dv_, dbeta (required); dalpha (the
+ * gradient of the LOG gate, same shape as alpha; required for DR_GATED / DR_KDA,
+ * ignored for DR_DELTANET); dS0 (fp32, NULL = not written).  The forward states
+ * are recomputed inside the call (no saved activations are needed).
+ */
+int delta_rule_bwd(const void *q, const void *k, const void *v, const void *alpha, const void *beta, const float *S0,
+                   const void *dout, const void *du, const float *dS_T, void *dq, void *dk_, void *dv_, void *dalpha,
+                   void *dbeta, float *dS0, int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype,
+                   void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Measurement hooks.  delta_rule_launches() returns how many kernels one
+ * delta_rule_fwd (for_bwd = 0) or delta_rule_bwd (for_bwd = 1) call with these
+ * arguments launches, and stores a static name for launch i in names[i] for
+ * i < max_names (names may be NULL); it returns a negative DR_ERR_* code for
+ * invalid arguments.  The *_timed variants do exactly what delta_rule_fwd /
+ * delta_rule_bwd do and in addition record the caller's cudaEvent_t events[i] on
+ * `stream` immediately before launch i and events[n] after the last launch
+ * (n = delta_rule_launches(...)), so that each kernel's device time is the
+ * elapsed time between consecutive events.  n_events must be 0 (record nothing)
+ * or at least n + 1, else DR_ERR_ARG.
+ */
+int delta_rule_launches(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype, int for_bwd,
+                        const char **names, int max_names);
+int delta_rule_fwd_timed(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                         const float *S0, void *out, void *u, float *S_T, int B, int T, int H, int dk, int dv,
+                         int variant, int chunk, int dtype, void *workspace, size_t ws_bytes, void *stream,
+                         void *const *events, int n_events);
+int delta_rule_bwd_timed(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                         const float *S0, const void *dout, const void *du, const float *dS_T, void *dq, void *dk_,
+                         void *dv_, void *dalpha, void *dbeta, float *dS0, int B, int T, int H, int dk, int dv,
+                         int variant, int chunk, int dtype, void *workspace, size_t ws_bytes, void *stream,
+                         void *const *events, int n_events);
+
+/* Static text for a DR_* code ("ok", "invalid argument", ...). */
+const char *delta_rule_strerror(int code);
+
+/*
+ * Synchronises `stream`, then reads and clears the calling device's error word.
+ * Returns DR_OK, DR_ERR_TIMEOUT if a kernel reported an expired wait since the
+ * last call, or DR_ERR_CUDA if the synchronisation itself failed.
+ */
+int delta_rule_sync_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DELTA_RULE_H */

@@ -1,0 +1,61 @@
+"""The C-ABI library builds, loads and exports every declared symbol (no GPU needed).
+
+Only argument-validation calls are made here; they return before any CUDA call.
+"""
+import ctypes
+import glob
+import os
+import re
+import shutil
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b(delta_rule_\w+)\s*\(", text):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if shutil.which("nvcc") is None and not os.path.exists(os.path.join(ROOT, "gated_delta_rule_107_b200",
+                                                                        "libdeltarule.so")):
+        pytest.skip("no nvcc and no prebuilt library")
+    from gated_delta_rule_107_b200 import binding, build
+    build.build()
+    return binding.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert "delta_rule_fwd" in names and "delta_rule_bwd" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    so = os.path.join(ROOT, "gated_delta_rule_107_b200", "libdeltarule.so")
+    out = subprocess.run(["nm", "-D", "--defined-only", so], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (delta_rule_\w+)", out))
+    assert set(names) <= exported
+
+
+def test_no_compute_validation_paths(lib):
+    from gated_delta_rule_107_b200 import binding
+    assert binding.workspace_size(8, 4096, 8, 128, 128, 1, 64, 1, 0) >= 0
+    assert binding.workspace_size(8, 4096, 8, 128, 128, 1, 64, 1, 1) > 0
+    assert lib.delta_rule_workspace_size(1, 10, 1, 96, 128, 1, 64, 1, 0) == ctypes.c_size_t(-1).value
+    assert lib.delta_rule_workspace_size(1, 10, 1, 128, 128, 9, 64, 1, 0) == ctypes.c_size_t(-1).value
+    assert lib.delta_rule_workspace_size(1, 10, 1, 128, 128, 1, 0, 1, 0) == ctypes.c_size_t(-1).value
+    # invalid enums / shapes are rejected before any CUDA call
+    args = [None] * 9 + [1, 10, 1, 128, 128, 7, 64, 1, None, 0, None]
+    assert binding.fwd_raw(*args) == binding.DR_ERR_ARG
+    args = [None] * 15 + [1, 10, 1, 128, 96, 1, 64, 1, None, 0, None]
+    assert binding.bwd_raw(*args) == binding.DR_ERR_UNSUPPORTED
+    assert binding.strerror(binding.DR_ERR_TIMEOUT) == "device wait timed out"
+    assert binding.strerror(12345) == "unknown error code"
