@@ -219,6 +219,9 @@ def run_ours(args):
 
     fev = [torch.cuda.Event(enable_timing=True) for _ in range(len(fwd_names) + 1)]
     bev = [torch.cuda.Event(enable_timing=True) for _ in range(len(bwd_names) + 1)]
+    for e in fev + bev:  # torch creates the CUDA event handle on first record
+        e.record(stream)
+    torch.cuda.synchronize()
     farr, barr = binding.event_array(fev), binding.event_array(bev)
 
     def step(timed: bool):

@@ -121,7 +121,11 @@ def sync_status(stream=None) -> int:
 
 # ------------------------------------------------------------------------------------------------
 def _p(t):
-    return None if t is None else t.data_ptr()
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("delta_rule tensors must be contiguous (the C ABI takes dense [B,T,H,d] / [B,H,dk,dv])")
+    return t.data_ptr()
 
 
 def _variant(v) -> int:

@@ -15,6 +15,7 @@ using namespace dr;
 namespace {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+bool aligned_elem(const void *p, int dtype) { return ((uintptr_t)p & (dtype == DR_BF16 ? 1u : 3u)) == 0; }
 
 // Checks shape / enum arguments; fills geo.  Returns DR_OK or an error code.
 int check_shape(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype, Geo *geo) {
@@ -74,9 +75,11 @@ static int fwd_impl(const void *q, const void *k, const void *v, const void *alp
     if (T == 0 || empty) return empty ? DR_OK : copy_state(S_T, S0, g, s);
     if (!q || !k || !v || !beta || !out) return DR_ERR_ARG;
     if (variant != DR_DELTANET && !alpha) return DR_ERR_ARG;
-    const void *ptrs[] = {q, k, v, variant != DR_DELTANET ? alpha : nullptr, beta, S0, out, u, S_T};
+    // tiles moved by TMA / vector accesses need 16 B; per-token scalars only their element size
+    const void *ptrs[] = {q, k, v, variant == DR_KDA ? alpha : nullptr, S0, out, u, S_T};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return DR_ERR_ALIGN;
+    if (!aligned_elem(beta, dtype) || (variant == DR_GATED && !aligned_elem(alpha, dtype))) return DR_ERR_ALIGN;
     const size_t need = ws_bytes(g, dtype, false);
     if (need > 0) {
         if (!workspace || ws_bytes_given < need) return DR_ERR_WORKSPACE;
@@ -101,10 +104,12 @@ static int bwd_impl(const void *q, const void *k, const void *v, const void *alp
     if (T == 0 || empty) return empty ? DR_OK : copy_state(dS0, dS_T, g, s);
     if (!q || !k || !v || !beta || !dout || !dq || !dk_ || !dv_ || !dbeta) return DR_ERR_ARG;
     if (variant != DR_DELTANET && (!alpha || !dalpha)) return DR_ERR_ARG;
-    const void *ptrs[] = {q, k, v, variant != DR_DELTANET ? alpha : nullptr, beta, S0, dout, du, dS_T, dq, dk_, dv_,
-                          variant != DR_DELTANET ? dalpha : nullptr, dbeta, dS0};
+    const void *ptrs[] = {q, k, v, variant == DR_KDA ? alpha : nullptr, S0, dout, du, dS_T, dq, dk_, dv_,
+                          variant == DR_KDA ? dalpha : nullptr, dS0};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return DR_ERR_ALIGN;
+    if (!aligned_elem(beta, dtype) || !aligned_elem(dbeta, dtype)) return DR_ERR_ALIGN;
+    if (variant == DR_GATED && (!aligned_elem(alpha, dtype) || !aligned_elem(dalpha, dtype))) return DR_ERR_ALIGN;
     const size_t need = ws_bytes(g, dtype, true);
     if (!workspace || ws_bytes_given < need) return DR_ERR_WORKSPACE;
     if (((uintptr_t)workspace & 255u) != 0) return DR_ERR_ALIGN;
@@ -159,8 +164,9 @@ extern "C" int delta_rule_fwd_timed(const void *q, const void *k, const void *v,
     Rec rec;
     rc = make_rec(g, dtype, false, events, n_events, &rec);
     if (rc != DR_OK) return rc;
-    return fwd_impl(q, k, v, alpha, beta, S0, out, u, S_T, B, T, H, dk, dv, variant, chunk, dtype, workspace,
-                    ws_bytes_given, stream, rec);
+    rc = fwd_impl(q, k, v, alpha, beta, S0, out, u, S_T, B, T, H, dk, dv, variant, chunk, dtype, workspace,
+                  ws_bytes_given, stream, rec);
+    return (rc == DR_OK && rec.bad) ? DR_ERR_ARG : rc;
 }
 
 extern "C" int delta_rule_bwd(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
@@ -185,8 +191,9 @@ extern "C" int delta_rule_bwd_timed(const void *q, const void *k, const void *v,
     Rec rec;
     rc = make_rec(g, dtype, true, events, n_events, &rec);
     if (rc != DR_OK) return rc;
-    return bwd_impl(q, k, v, alpha, beta, S0, dout, du, dS_T, dq, dk_, dv_, dalpha, dbeta, dS0, B, T, H, dk, dv,
-                    variant, chunk, dtype, workspace, ws_bytes_given, stream, rec);
+    rc = bwd_impl(q, k, v, alpha, beta, S0, dout, du, dS_T, dq, dk_, dv_, dalpha, dbeta, dS0, B, T, H, dk, dv,
+                  variant, chunk, dtype, workspace, ws_bytes_given, stream, rec);
+    return (rc == DR_OK && rec.bad) ? DR_ERR_ARG : rc;
 }
 
 extern "C" int delta_rule_launches(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype,

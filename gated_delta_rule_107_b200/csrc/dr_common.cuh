@@ -58,8 +58,12 @@ struct Tensors {
 struct Rec {
     cudaEvent_t *ev = nullptr;
     int n = 0, i = 0;
+    bool bad = false;  // an event could not be recorded (invalid handle)
     void mark(cudaStream_t s) {
-        if (ev && i < n) cudaEventRecord(ev[i++], s);
+        if (ev && i < n && cudaEventRecord(ev[i++], s) != cudaSuccess) {
+            cudaGetLastError();  // consume it: it is not a launch failure
+            bad = true;
+        }
     }
 };
 

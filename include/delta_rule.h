@@ -44,7 +44,10 @@
  *              T need not be a multiple of chunk (the tail chunk is masked).
  *              T == 0 is valid: the forward copies S0 (or zeros) to S_T and the
  *              backward copies dS_T (or zeros) to dS0.
- *   Pointers   device pointers (cudaMalloc / torch CUDA memory), 16-byte aligned.
+ *   Pointers   device pointers (cudaMalloc / torch CUDA memory).  Tensors with a
+ *              channel dimension (q, k, v, out, u, the KDA gate and all their
+ *              gradients) and the fp32 states must be 16-byte aligned; beta, dbeta
+ *              and the Gated-DeltaNet gate need only their element alignment.
  *              The caller owns every buffer; the library allocates nothing, keeps
  *              no pointer after returning and has no global state except the
  *              device error word below.  Inputs are never written.  Outputs must
@@ -121,7 +124,7 @@ int delta_rule_bwd(const void *q, const void *k, const void *v, const void *alph
  * arguments launches, and stores a static name for launch i in names[i] for
  * i < max_names (names may be NULL); it returns a negative DR_ERR_* code for
  * invalid arguments.  The *_timed variants do exactly what delta_rule_fwd /
- * delta_rule_bwd do and in addition record the caller's cudaEvent_t events[i] on
+ * delta_rule_bwd do and in addition record the caller's cudaEvent_t events[i] (created handles) on
  * `stream` immediately before launch i and events[n] after the last launch
  * (n = delta_rule_launches(...)), so that each kernel's device time is the
  * elapsed time between consecutive events.  n_events must be 0 (record nothing)

@@ -68,6 +68,9 @@ def test_invalid_arguments_return_codes():
             a[i] = val
         assert binding.fwd_raw(*a) == code, name
     assert binding.strerror(binding.DR_ERR_ALIGN).startswith("misaligned")
+    with pytest.raises(ValueError):
+        binding.delta_rule_fwd(x["q"][:, ::2], x["k"][:, ::2], x["v"][:, ::2], x["loga"][:, ::2],
+                               x["beta"][:, ::2], None, variant="gdn")
     assert binding.sync_status() == binding.DR_OK
 
 
@@ -77,7 +80,7 @@ def test_outputs_do_not_write_past_their_ends():
     for var in ("deltanet", "gdn", "kda"):
         x = gen(var, "bf16", B, T, H, d, d, seed=3, s0_std=0.1, grads=True)
         pad = 4096
-        sentinel = -12345.0
+        sentinel = -12288.0  # exactly representable in bf16 and fp32
 
         def guarded(shape, dtype):
             n = 1
@@ -114,14 +117,36 @@ def test_split_sequence_state_handoff():
     x = gen("kda", "f32", 1, 300, 2, 64, 64, seed=4, s0_std=0.1)
     full = gpu_fwd(x, "kda")
     t1 = 131
-    a = {k: (v[:, :t1].contiguous() if (v is not None and k != "S0") else v) for k, v in x.items()}
-    b = {k: (v[:, t1:].contiguous() if (v is not None and k != "S0") else v) for k, v in x.items()}
+    a = {k: (v[:, :t1] if (v is not None and k != "S0") else v) for k, v in x.items()}
+    b = {k: (v[:, t1:] if (v is not None and k != "S0") else v) for k, v in x.items()}
     ra = gpu_fwd(a, "kda")
     b["S0"] = ra["S_T"]
     rb = gpu_fwd(b, "kda")
     assert torch.allclose(torch.cat([ra["o"], rb["o"]], 1), full["o"], atol=2e-5, rtol=1e-4)
     assert torch.allclose(rb["S_T"], full["S_T"], atol=2e-5, rtol=1e-4)
     compare_fwd(full, oracle_fwd(x, "kda"), "f32")
+
+
+def test_split_sequence_tensor_core_path():
+    """Same hand-off on the bf16 tensor-core forward (offset views as inputs)."""
+    x = gen("gdn", "bf16", 2, 333, 2, 128, 128, seed=8, s0_std=0.1)
+    full = gpu_fwd(x, "gdn")
+    t1 = 192
+    a = {k: (v[:, :t1].contiguous() if (v is not None and k != "S0") else v) for k, v in x.items()}
+    b = {k: (v[:, t1:].contiguous() if (v is not None and k != "S0") else v) for k, v in x.items()}
+    ra = gpu_fwd(a, "gdn")
+    b["S0"] = ra["S_T"]
+    rb = gpu_fwd(b, "gdn")
+    ref = oracle_fwd(x, "gdn")
+    from parity_util import rel_err, np64
+    assert rel_err(np64(torch.cat([ra["o"], rb["o"]], 1)), ref["o"]) < 2e-2
+    assert rel_err(np64(rb["S_T"]), ref["S_T"]) < 2e-2
+
+
+def test_bf16_d128_uses_the_tensor_core_kernel():
+    assert binding.launches(8, 4096, 8, 128, 128, 1, 64, 1, 0) == ["k_fwd_tc"]
+    assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 0) == ["k_fwd_tc"]
+    assert binding.launches(1, 256, 2, 64, 64, 0, 64, 0, 0) == ["k_prep", "k_scan", "k_out"]
 
 
 def test_host_buffer_entry_point():
