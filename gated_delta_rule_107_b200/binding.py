@@ -27,7 +27,7 @@ DTYPES = {torch.float32: DR_F32, torch.bfloat16: DR_BF16}
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdeltarule.so")
 EXPORTS = ("delta_rule_workspace_size", "delta_rule_fwd", "delta_rule_bwd", "delta_rule_strerror",
-           "delta_rule_sync_status", "delta_rule_launches", "delta_rule_fwd_timed", "delta_rule_bwd_timed")
+           "delta_rule_sync_status", "delta_rule_launches", "delta_rule_fwd_timed", "delta_rule_bwd_timed", "delta_rule_fwd_noalloc")
 
 _lib = None
 
@@ -65,6 +65,8 @@ def load(path: str | None = None):
     lib.delta_rule_fwd_timed.restype = i
     lib.delta_rule_bwd_timed.argtypes = [vp] * 15 + [i] * 8 + [vp, sz, vp, ctypes.POINTER(vp), i]
     lib.delta_rule_bwd_timed.restype = i
+    lib.delta_rule_fwd_noalloc.argtypes = [vp] * 9 + [i] * 8 + [vp]
+    lib.delta_rule_fwd_noalloc.restype = i
     if path is None:
         _lib = lib
     return lib
@@ -104,6 +106,11 @@ def fwd_raw(*args) -> int:
 
 def bwd_raw(*args) -> int:
     return load().delta_rule_bwd(*args)
+
+
+def fwd_noalloc_raw(*args) -> int:
+    """delta_rule_fwd_noalloc: the forward with the library's built-in scratch (no workspace argument)."""
+    return load().delta_rule_fwd_noalloc(*args)
 
 
 def fwd_timed_raw(*args) -> int:

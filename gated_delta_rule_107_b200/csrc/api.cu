@@ -12,7 +12,7 @@
 
 using namespace dr;
 
-namespace {
+namespace dr {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 bool aligned_elem(const void *p, int dtype) { return ((uintptr_t)p & (dtype == DR_BF16 ? 1u : 3u)) == 0; }
@@ -55,7 +55,7 @@ int copy_state(float *dst, const float *src, const Geo &g, cudaStream_t s) {
     return launch_status(e);
 }
 
-}  // namespace
+}  // namespace dr
 
 extern "C" size_t delta_rule_workspace_size(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype,
                                             int for_bwd) {

@@ -3,3 +3,4 @@
 #include "simt_path.cu"
 #include "tc_fwd.cu"
 #include "api.cu"
+#include "noalloc.cu"

@@ -142,6 +142,32 @@ int delta_rule_bwd_timed(const void *q, const void *k, const void *v, const void
                          int variant, int chunk, int dtype, void *workspace, size_t ws_bytes, void *stream,
                          void *const *events, int n_events);
 
+/*
+ * Forward without any device allocation (no counterpart in the method; it is a
+ * deployment convenience).  Some callers cannot call cudaMalloc at all: code
+ * inside a CUDA graph being captured, allocator-less embedded runtimes, and
+ * plugins that a host framework hands only their input and output buffers.
+ * This entry point computes exactly what delta_rule_fwd computes (same
+ * arguments, minus the workspace), always on the CUDA-core forward kernels,
+ * with their scratch taken from a buffer of DELTA_RULE_NOALLOC_SCRATCH_BYTES
+ * that is compiled into the library; every GPU that loads the library holds it
+ * until the process exits.  The caller still passes every input and output.
+ *   - Problems whose scratch (delta_rule_workspace_size of the CUDA-core
+ *     forward) exceeds the buffer return DR_ERR_WORKSPACE without launching;
+ *     about 210 KB per (batch, head, chunk) at dk = dv = 128, chunk 64.
+ *   - The first call on each device looks up the buffer's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one buffer and it keeps the last call's
+ *     contents (nothing in it needs to start at zero): calls whose kernels
+ *     overlap on the GPU (different streams, or different threads without
+ *     ordering) race and corrupt each other's results.
+ */
+#define DELTA_RULE_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int delta_rule_fwd_noalloc(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                           const float *S0, void *out, void *u, float *S_T, int B, int T, int H, int dk, int dv,
+                           int variant, int chunk, int dtype, void *stream);
+
 /* Static text for a DR_* code ("ok", "invalid argument", ...). */
 const char *delta_rule_strerror(int code);
 
