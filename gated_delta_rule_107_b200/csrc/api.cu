@@ -127,7 +127,7 @@ static int launch_plan(const Geo &g, int dtype, bool bwd, const char **names, in
     const char *const *src = nullptr;
     if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
     if (!bwd && use_tc_fwd(g, dtype)) {
-        n = tc_fwd_launches(names, max_names);
+        n = tc_fwd_launches(g, names, max_names);
         return n;
     }
     src = bwd ? SIMT_BWD_KERNELS : SIMT_FWD_KERNELS;

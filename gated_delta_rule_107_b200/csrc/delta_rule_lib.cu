@@ -2,5 +2,6 @@
 // word and all kernels live in one module, so no relocatable device code is needed).
 #include "simt_path.cu"
 #include "tc_fwd.cu"
+#include "tc_fwd2.cu"
 #include "api.cu"
 #include "noalloc.cu"

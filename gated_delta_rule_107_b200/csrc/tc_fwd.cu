@@ -29,6 +29,7 @@
 #include "tc_host.cuh"
 #include "tc_path.cuh"
 #include "tc_ptx.cuh"
+#include "tc_tile.cuh"
 
 namespace dr {
 namespace tcf {
@@ -85,39 +86,6 @@ struct Args {
     float *ST;           // [B,H,dk,dv] or null
     int B, T, H, dv, N;
 };
-
-__device__ __forceinline__ float bf(const void *p, size_t i) {
-    return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
-}
-
-// element (r, c) of a token-major tile of 64-row panels (panel stride 8K)
-__device__ __forceinline__ uint32_t tok_off(int r, int c) {
-    return (uint32_t)((c >> 6) * 8192) + swz(r, (c & 63) >> 3) + (c & 7) * 2;
-}
-
-__device__ __forceinline__ void st_chunk(unsigned char *base, uint32_t off, const float *v) {
-    uint4 w;
-    w.x = pack_bf16(v[0], v[1]);
-    w.y = pack_bf16(v[2], v[3]);
-    w.z = pack_bf16(v[4], v[5]);
-    w.w = pack_bf16(v[6], v[7]);
-    *reinterpret_cast<uint4 *>(base + off) = w;
-}
-
-__device__ __forceinline__ void ld_chunk(const unsigned char *base, uint32_t off, float *v) {
-    const uint4 w = *reinterpret_cast<const uint4 *>(base + off);
-    v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
-    v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
-}
-
-// 64 fp32 columns of this thread's TMEM lane
-__device__ __forceinline__ void tmem_row64(uint32_t taddr, float *v) {
-    tmem_ld16(taddr + 0, v);
-    tmem_ld16(taddr + 16, v + 16);
-    tmem_ld16(taddr + 32, v + 32);
-    tmem_ld16(taddr + 48, v + 48);
-    wait_ld();
-}
 
 template <int VAR>
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -636,13 +604,14 @@ bool tc_fwd_supported(const Geo &g, bool bf16) {
 
 size_t tc_fwd_ws_bytes(const Geo &) { return 0; }
 
-int tc_fwd_launches(const char **names, int max_names) {
-    if (names && max_names > 0) names[0] = "k_fwd_tc";
+int tc_fwd_launches(const Geo &g, const char **names, int max_names) {
+    if (names && max_names > 0) names[0] = (g.variant == VAR_KDA) ? "k_fwd_tc" : "k_fwd_tc2";
     return 1;
 }
 
 cudaError_t tc_fwd(const Geo &g, const Tensors &t, void *, cudaStream_t s, Rec &rec) {
     using namespace tcf;
+    if (g.variant != VAR_KDA) return tc_fwd2(g, t, s, rec);
     CUtensorMap mq, mk, mv, mg;
     const uint64_t Bn = g.B, T = g.T, H = g.H;
     bool ok = tc::make_map_4d_bf16(&mq, t.q, DK, H, T, Bn, 64) && tc::make_map_4d_bf16(&mk, t.k, DK, H, T, Bn, 64) &&

@@ -1,0 +1,556 @@
+// tc_fwd2.cu -- warp-specialised fused forward for Gated DeltaNet and DeltaNet (sm_100a).
+//
+// Same per-chunk algebra as tc_fwd.cu ("线性注意力架构演进与Kimi Delta Attention创新实践",
+// sections 2.1, 6.1, 6.2, 7.1), reorganised so that the preparation of chunk m+1 runs
+// while the state chain processes chunk m:
+//
+//   warp 0       producer: TMA loads of k and q (interleaved per 64-channel panel so
+//                that [k ; q] is one 128-row operand), of v, and plain loads of the
+//                scalar gate and beta
+//   warps 1-4    preparation warpgroup, per chunk:
+//                  P1  [k ; q] . k^T                -> k.k^T, q.k^T   (TMEM)
+//                      A = beta_r e^{g_r-g_i} k_r.k_i (i<r), P = e^{g_r-g_i} q_r.k_i (i<=r)
+//                  T = (I + A)^-1                    (tc_inverse.cuh)
+//                  IPT [I ; P] . T = R = [T ; P T]
+//                  P3  (R diag(beta e^g)) . k       = [W ; P W]
+//                  P4  (R diag(beta))     . v       = [U~ ; P U~]  -> accumulator D[m%2]
+//                  A_chain = [-W ; e^g q - P W]
+//   warps 5-8    chain warpgroup, per chunk:
+//                  C1  D += A_chain . S             -> rows 0-63 U, rows 64-127 O
+//                  C3  E = k^T . (e^{g_C - g} U)    (the decay to the chunk end is
+//                                                     applied to U's rows, not to k)
+//                  S <- e^{g_C} S + E               (fp32 registers)
+//
+// The gate enters only as row / column multipliers in epilogues: e^{g_r - g_i} is
+// split at the chunk midpoint g_m into e^{g_r - g_m} e^{g_m - g_i}; a chunk whose
+// cumulative log gate strays more than 80 from g_m uses exact per-pair exponentials.
+// Hand-offs between the warpgroups are mbarriers; the accumulator D is double-buffered
+// in TMEM; every wait is bounded (~1 s) and aborts are agreed on per warpgroup.
+#include "tc_host.cuh"
+#include "tc_inverse.cuh"
+#include "tc_path.cuh"
+#include "tc_ptx.cuh"
+#include "tc_tile.cuh"
+
+namespace dr {
+namespace tcf2 {
+
+using namespace dr::tc;
+using dr::tcf::ld_chunk;
+using dr::tcf::st_chunk;
+using dr::tcf::tmem_row64;
+
+constexpr int C = 64, DK = 128, DVB = 64;
+constexpr int NTHREADS = 288;
+
+// ---- shared memory (bytes from a 1024-aligned base) ----
+constexpr uint32_t SLOT = 32768;                 // [k_p0 | q_p0 | k_p1 | q_p1], 8K each
+constexpr uint32_t OFF_V = 2 * SLOT;             //  8K  v (64 tokens x 64)
+constexpr uint32_t OFF_KC = OFF_V + 8192;        // 2 x 16K  chain copy of k (2 panels of 8K)
+constexpr uint32_t OFF_RR = OFF_KC + 32768;      // 32K  R diag(beta) | R diag(beta e^g); inverse scratch
+constexpr uint32_t OFF_IP = OFF_RR + 32768;      // 16K  [I ; P]
+constexpr uint32_t OFF_TT = OFF_IP + 16384;      //  8K  T (MN-major B)
+constexpr uint32_t OFF_AC = OFF_TT + 8192;       // 32K  A_chain (128 rows x 2 panels of 16K)
+constexpr uint32_t OFF_U = OFF_AC + 32768;       //  8K  e^{g_C - g} U
+constexpr uint32_t OFF_S = OFF_U + 8192;         // 16K  bf16 S
+constexpr uint32_t OFF_MISC = OFF_S + 16384;     //  8K
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 8192;
+
+// misc
+constexpr uint32_t M_BAR = 0;        // 16 mbarriers
+constexpr uint32_t M_TMEM = 128, M_ABORT = 132, M_BIG = 136;
+constexpr uint32_t M_GB = 256;       // [2][2][64]: raw log gate, beta
+constexpr uint32_t M_PF = 1280;      // prep factors [7][64]
+constexpr uint32_t M_CF = 3072;      // chain factors [2][80]: e^{gC-g} (64), e^{gC}
+constexpr uint32_t M_YS = 4096;      // inverse scratch [3][256]
+static_assert(M_YS + 3 * 256 * 4 <= 8192, "misc overflow");
+enum { PF_GC = 0, PF_ROWA, PF_ROWP, PF_COLA, PF_BV, PF_BK, PF_EG };
+
+// TMEM columns
+constexpr uint32_t TM_G1 = 0, TM_X = 64, TM_D0 = 192, TM_E = 320, TM_COLS = 512;
+
+enum {
+    B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_VFULL, B_VEMPTY, B_PMMA, B_CMMA,
+    B_READY0, B_READY1, B_ACFREE, B_DFREE0, B_DFREE1, B_KCFREE0, B_KCFREE1, B_NUM
+};
+
+struct Args {
+    const void *alpha, *beta;
+    const float *S0;
+    void *out, *u;
+    float *ST;
+    int B, T, H, dv, N;
+};
+
+__device__ __forceinline__ void st_row_global(void *base, size_t elem_off, const float *v) {
+    uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(base) + elem_off);
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+        uint4 w;
+        w.x = pack_bf16(v[ch * 8 + 0], v[ch * 8 + 1]);
+        w.y = pack_bf16(v[ch * 8 + 2], v[ch * 8 + 3]);
+        w.z = pack_bf16(v[ch * 8 + 4], v[ch * 8 + 5]);
+        w.w = pack_bf16(v[ch * 8 + 6], v[ch * 8 + 7]);
+        dst[ch] = w;
+    }
+}
+
+template <int VAR>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    k_fwd_tc2(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, Args a) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_MISC + M_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + M_TMEM);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + M_ABORT);
+    volatile int *bigflag = reinterpret_cast<volatile int *>(sm + OFF_MISC + M_BIG);
+    float *gb = reinterpret_cast<float *>(sm + OFF_MISC + M_GB);
+    float *pf = reinterpret_cast<float *>(sm + OFF_MISC + M_PF);
+    float *cf = reinterpret_cast<float *>(sm + OFF_MISC + M_CF);
+    float *ysc = reinterpret_cast<float *>(sm + OFF_MISC + M_YS);
+
+    const int half = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int j0 = half * DVB;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = a.T, H = a.H, DV = a.dv, N = a.N;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < B_NUM; ++i) mbar_init(&bar[i], (i == B_FULL0 || i == B_FULL1) ? 2 : 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, TM_COLS);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *tmem_slot;
+
+    if (warp == 0) {
+        // ================================ producer ================================
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+        }
+        int issued[2] = {0, 0}, v_issued = 0;
+        for (int m = 0; m < N; ++m) {
+            const int s = m & 1, t0 = m * C;
+            if (m >= 2 && !mbar_wait(&bar[B_EMPTY0 + s], ((m >> 1) - 1) & 1, abort_flag)) break;
+            unsigned char *slot = sm + s * SLOT;
+            if (lane == 0) {
+                mbar_arrive_tx(&bar[B_FULL0 + s], 4 * 8192);
+                tma_load_4d(slot + 0, &tm_k, 0, h, t0, b, &bar[B_FULL0 + s]);
+                tma_load_4d(slot + 8192, &tm_q, 0, h, t0, b, &bar[B_FULL0 + s]);
+                tma_load_4d(slot + 16384, &tm_k, 64, h, t0, b, &bar[B_FULL0 + s]);
+                tma_load_4d(slot + 24576, &tm_q, 64, h, t0, b, &bar[B_FULL0 + s]);
+            }
+            float *gbs = gb + s * 128;
+            for (int r = lane; r < C; r += 32) {
+                const int t = t0 + r;
+                const size_t row = ((size_t)b * T + t) * H + h;
+                float lg = 0.f, bt = 0.f;
+                if (t < T) {
+                    if (VAR == VAR_GATED) lg = tcf::bf(a.alpha, row);
+                    bt = tcf::bf(a.beta, row);
+                }
+                gbs[r] = lg;
+                gbs[64 + r] = bt;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[B_FULL0 + s]);
+            issued[s]++;
+            if (m >= 1 && !mbar_wait(&bar[B_VEMPTY], (m - 1) & 1, abort_flag)) break;
+            if (lane == 0) {
+                mbar_arrive_tx(&bar[B_VFULL], 8192);
+                tma_load_4d(sm + OFF_V, &tm_v, j0, h, t0, b, &bar[B_VFULL]);
+            }
+            v_issued++;
+        }
+        if (*abort_flag) {
+            volatile int dummy = 0;
+            for (int s = 0; s < 2; ++s)
+                if (issued[s] > 0) mbar_wait(&bar[B_FULL0 + s], (issued[s] - 1) & 1, &dummy, 100000000ull);
+            if (v_issued > 0) mbar_wait(&bar[B_VFULL], (v_issued - 1) & 1, &dummy, 100000000ull);
+        }
+    } else if (warp <= 4) {
+        // ============================ preparation warpgroup ============================
+        const int wt = threadIdx.x - 32;
+        const int q4 = warp & 3, trow = q4 * 32 + lane;
+        const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
+        uint32_t ph = 0;
+        bool pending = false;
+        auto wsync = [&]() { named_sync(1, 128); };
+        auto wabort = [&]() -> bool { return named_sync_any(1, 128, *abort_flag != 0); };
+        auto mma_done = [&]() -> bool {
+            mbar_wait(&bar[B_PMMA], ph & 1, abort_flag);
+            ph++;
+            fence_after_sync();
+            const bool ok = !wabort();
+            if (ok) pending = false;
+            return ok;
+        };
+        float *Asc = reinterpret_cast<float *>(sm + OFF_RR);
+        float *Tf = Asc + 4096;
+        for (int m = 0; m < N; ++m) {
+            const int s = m & 1, bb = m & 1;
+            unsigned char *slot = sm + s * SLOT;
+            mbar_wait(&bar[B_FULL0 + s], (m >> 1) & 1, abort_flag);
+            if (m >= 2) mbar_wait(&bar[B_KCFREE0 + bb], ((m >> 1) - 1) & 1, abort_flag);
+            if (wabort()) break;
+            // ---------------- gates and factors; chain copy of k ----------------
+            if (wt < 32) {
+                const float *lg = gb + s * 128, *bt = lg + 64;
+                float x0 = lg[lane], x1 = lg[lane + 32];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y0 = __shfl_up_sync(0xffffffffu, x0, o);
+                    const float y1 = __shfl_up_sync(0xffffffffu, x1, o);
+                    if (lane >= o) { x0 += y0; x1 += y1; }
+                }
+                x1 += __shfl_sync(0xffffffffu, x0, 31);
+                const float gC = __shfl_sync(0xffffffffu, x1, 31);
+                const float gm = __shfl_sync(0xffffffffu, x0, 31);
+                float dev = fmaxf(fabsf(x0 - gm), fabsf(x1 - gm));
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) dev = fmaxf(dev, __shfl_xor_sync(0xffffffffu, dev, o));
+                const float b0 = bt[lane], b1 = bt[lane + 32];
+                pf[PF_GC * 64 + lane] = x0;
+                pf[PF_GC * 64 + lane + 32] = x1;
+                pf[PF_ROWA * 64 + lane] = b0 * __expf(x0 - gm);
+                pf[PF_ROWA * 64 + lane + 32] = b1 * __expf(x1 - gm);
+                pf[PF_ROWP * 64 + lane] = __expf(x0 - gm);
+                pf[PF_ROWP * 64 + lane + 32] = __expf(x1 - gm);
+                pf[PF_COLA * 64 + lane] = __expf(gm - x0);
+                pf[PF_COLA * 64 + lane + 32] = __expf(gm - x1);
+                pf[PF_BV * 64 + lane] = b0;
+                pf[PF_BV * 64 + lane + 32] = b1;
+                pf[PF_BK * 64 + lane] = b0 * __expf(x0);
+                pf[PF_BK * 64 + lane + 32] = b1 * __expf(x1);
+                pf[PF_EG * 64 + lane] = __expf(x0);
+                pf[PF_EG * 64 + lane + 32] = __expf(x1);
+                float *cfb = cf + bb * 80;
+                cfb[lane] = __expf(gC - x0);
+                cfb[lane + 32] = __expf(gC - x1);
+                if (lane == 0) {
+                    cfb[64] = __expf(gC);
+                    *bigflag = dev > 80.f;
+                }
+            }
+            {
+                unsigned char *kc = sm + OFF_KC + bb * 16384;
+                for (int x = wt; x < 1024; x += 128) {
+                    const int p = x >> 9, r = (x >> 3) & 63, ch = x & 7;
+                    const uint32_t o = swz(r, ch);
+                    *reinterpret_cast<uint4 *>(kc + p * 8192 + o) = *reinterpret_cast<const uint4 *>(slot + p * 16384 + o);
+                }
+            }
+            fence_proxy_async();
+            wsync();
+            // ---------------- P1: [k ; q] . k^T ----------------
+            if (wt == 0) {
+                fence_after_sync();
+                const uint32_t id = idesc_bf16(128, 64, 0, 0);
+                const uint32_t sa = smem_u32(slot);
+#pragma unroll
+                for (int st = 0; st < 8; ++st) {
+                    const uint32_t ad = sa + (st >> 2) * 16384 + (st & 3) * 32;
+                    mma_bf16(tbase + TM_G1, sdesc(ad, 16, 1024), sdesc(ad, 16, 1024), id, st > 0);
+                }
+                mma_commit(&bar[B_PMMA]);
+            }
+            pending = true;
+            if (!mma_done()) break;
+            // ---------------- A, P, T ----------------
+            {
+                float g1[64];
+                tmem_row64(tl + TM_G1, g1);
+                const bool big = *bigflag != 0;
+                const float *gc = pf + PF_GC * 64, *cola = pf + PF_COLA * 64;
+                if (trow < 64) {
+                    const int r = trow;
+                    const float rf = pf[PF_ROWA * 64 + r], br = pf[PF_BV * 64 + r];
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) {
+                        float f = big ? br * __expf(gc[r] - gc[i]) : rf * cola[i];
+                        if (VAR == VAR_DELTANET) f = br;
+                        Asc[sw64(r, i)] = (i < r) ? g1[i] * f : 0.f;
+                    }
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        float w[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) w[e] = (ch * 8 + e == r) ? 1.f : 0.f;
+                        st_chunk(sm + OFF_IP, swz(r, ch), w);
+                    }
+                } else {
+                    const int r = trow - 64;
+                    const float rf = pf[PF_ROWP * 64 + r];
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) {
+                        float f = big ? __expf(gc[r] - gc[i]) : rf * cola[i];
+                        if (VAR == VAR_DELTANET) f = 1.f;
+                        g1[i] = (i <= r) ? g1[i] * f : 0.f;
+                    }
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_IP, swz(trow, ch), g1 + ch * 8);
+                }
+                fence_before_sync();
+                wsync();
+                unit_lower_inverse64(Asc, Tf, ysc, wt, wsync);
+                if (wt < 64) {
+                    const int i = wt;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        float w[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int n = ch * 8 + e;
+                            w[e] = (n <= i) ? Tf[sw64(i, n)] : 0.f;
+                        }
+                        st_chunk(sm + OFF_TT, swz(i, ch), w);
+                    }
+                }
+                fence_proxy_async();
+                wsync();
+            }
+            // ---------------- IPT: R = [I ; P] T ----------------
+            if (wt == 0) {
+                fence_after_sync();
+                const uint32_t id = idesc_bf16(128, 64, 0, 1);
+                const uint32_t ip = smem_u32(sm + OFF_IP), tt = smem_u32(sm + OFF_TT);
+#pragma unroll
+                for (int st = 0; st < 4; ++st)
+                    mma_bf16(tbase + TM_G1, sdesc(ip + st * 32, 16, 1024), sdesc(tt + st * 2048, 1024, 1024), id,
+                             st > 0);
+                mma_commit(&bar[B_PMMA]);
+            }
+            pending = true;
+            if (!mma_done()) break;
+            // ---------------- R diag(beta), R diag(beta e^g) ----------------
+            {
+                float rv[64];
+                tmem_row64(tl + TM_G1, rv);
+                const float *bv = pf + PF_BV * 64, *bk = pf + PF_BK * 64;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    float w[8], w2[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        w[e] = rv[ch * 8 + e] * bv[ch * 8 + e];
+                        w2[e] = rv[ch * 8 + e] * bk[ch * 8 + e];
+                    }
+                    st_chunk(sm + OFF_RR, swz(trow, ch), w);
+                    st_chunk(sm + OFF_RR + 16384, swz(trow, ch), w2);
+                }
+            }
+            mbar_wait(&bar[B_VFULL], m & 1, abort_flag);
+            if (m >= 2) mbar_wait(&bar[B_DFREE0 + bb], ((m >> 1) - 1) & 1, abort_flag);
+            fence_proxy_async();
+            fence_before_sync();
+            if (wabort()) break;
+            // ---------------- P3: X = [W ; P W];  P4: D = [U~ ; P U~] ----------------
+            if (wt == 0) {
+                fence_after_sync();
+                const uint32_t rr = smem_u32(sm + OFF_RR), sk = smem_u32(slot), vv = smem_u32(sm + OFF_V);
+                const uint32_t id3 = idesc_bf16(128, 128, 0, 1), id4 = idesc_bf16(128, 64, 0, 1);
+#pragma unroll
+                for (int st = 0; st < 4; ++st)
+                    mma_bf16(tbase + TM_X, sdesc(rr + 16384 + st * 32, 16, 1024), sdesc(sk + st * 2048, 16384, 1024),
+                             id3, st > 0);
+#pragma unroll
+                for (int st = 0; st < 4; ++st)
+                    mma_bf16(tbase + TM_D0 + bb * 64, sdesc(rr + st * 32, 16, 1024),
+                             sdesc(vv + st * 2048, 1024, 1024), id4, st > 0);
+                mma_commit(&bar[B_PMMA]);
+            }
+            pending = true;
+            if (!mma_done()) break;
+            if (wt == 0) mbar_arrive(&bar[B_VEMPTY]);
+            // ---------------- A_chain ----------------
+            if (m >= 1) mbar_wait(&bar[B_ACFREE], (m - 1) & 1, abort_flag);
+            if (wabort()) break;
+            {
+                const int r = trow;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float xv[64];
+                    tmem_row64(tl + TM_X + hh * 64, xv);
+                    if (r < 64) {
+#pragma unroll
+                        for (int i = 0; i < 64; ++i) xv[i] = -xv[i];
+                    } else {
+                        const int rr = r - 64;
+                        const float sc = pf[PF_EG * 64 + rr];
+#pragma unroll
+                        for (int ch = 0; ch < 8; ++ch) {
+                            float qv[8];
+                            ld_chunk(slot, (uint32_t)hh * 16384 + 8192 + swz(rr, ch), qv);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) xv[ch * 8 + e] = qv[e] * sc - xv[ch * 8 + e];
+                        }
+                    }
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_AC, (uint32_t)hh * 16384 + swz(r, ch), xv + ch * 8);
+                }
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            wsync();
+            if (wt == 0) {
+                mbar_arrive(&bar[B_EMPTY0 + s]);
+                mbar_arrive(&bar[B_READY0 + bb]);
+            }
+        }
+        if (*abort_flag && pending) {
+            volatile int dummy = 0;
+            mbar_wait(&bar[B_PMMA], ph & 1, &dummy, 100000000ull);
+        }
+    } else {
+        // ================================ chain warpgroup ================================
+        const int wc = threadIdx.x - 160;
+        const int q4 = warp & 3, trow = q4 * 32 + lane;
+        const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
+        uint32_t ph = 0;
+        bool pending = false;
+        auto wsync = [&]() { named_sync(2, 128); };
+        auto wabort = [&]() -> bool { return named_sync_any(2, 128, *abort_flag != 0); };
+        auto mma_done = [&]() -> bool {
+            mbar_wait(&bar[B_CMMA], ph & 1, abort_flag);
+            ph++;
+            fence_after_sync();
+            const bool ok = !wabort();
+            if (ok) pending = false;
+            return ok;
+        };
+        float S[DVB];
+        {
+            const float *s0 = a.S0 ? a.S0 + (((size_t)b * H + h) * DK + trow) * DV + j0 : nullptr;
+#pragma unroll
+            for (int j = 0; j < DVB; ++j) S[j] = s0 ? s0[j] : 0.f;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_S, swz(trow, ch), S + ch * 8);
+        }
+        fence_proxy_async();
+        wsync();
+        for (int m = 0; m < N; ++m) {
+            const int bb = m & 1, t0 = m * C;
+            const int L = min(C, T - t0);
+            mbar_wait(&bar[B_READY0 + bb], (m >> 1) & 1, abort_flag);
+            if (wabort()) break;
+            // ---------------- C1: D += A_chain . S ----------------
+            if (wc == 0) {
+                fence_after_sync();
+                const uint32_t id = idesc_bf16(128, 64, 0, 1);
+                const uint32_t ac = smem_u32(sm + OFF_AC), ss = smem_u32(sm + OFF_S);
+#pragma unroll
+                for (int st = 0; st < 8; ++st)
+                    mma_bf16(tbase + TM_D0 + bb * 64, sdesc(ac + (st >> 2) * 16384 + (st & 3) * 32, 16, 1024),
+                             sdesc(ss + st * 2048, 1024, 1024), id, 1);
+                mma_commit(&bar[B_CMMA]);
+            }
+            pending = true;
+            if (!mma_done()) break;
+            if (wc == 0) mbar_arrive(&bar[B_ACFREE]);
+            // ---------------- write values and outputs ----------------
+            {
+                float dv[64];
+                tmem_row64(tl + TM_D0 + bb * 64, dv);
+                if (trow < 64) {
+                    const int r = trow;
+                    if (a.u && r < L) st_row_global(a.u, (((size_t)b * T + t0 + r) * H + h) * DV + j0, dv);
+                    const float f = cf[bb * 80 + r];
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) dv[i] *= f;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_U, swz(r, ch), dv + ch * 8);
+                } else {
+                    const int r = trow - 64;
+                    if (r < L) st_row_global(a.out, (((size_t)b * T + t0 + r) * H + h) * DV + j0, dv);
+                }
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            wsync();
+            if (wc == 0) mbar_arrive(&bar[B_DFREE0 + bb]);
+            // ---------------- C3: E = k^T (e^{gC-g} U) ----------------
+            if (wc == 0) {
+                fence_after_sync();
+                const uint32_t id = idesc_bf16(128, 64, 1, 1);
+                const uint32_t kc = smem_u32(sm + OFF_KC + bb * 16384), uu = smem_u32(sm + OFF_U);
+#pragma unroll
+                for (int st = 0; st < 4; ++st)
+                    mma_bf16(tbase + TM_E, sdesc(kc + st * 2048, 8192, 1024), sdesc(uu + st * 2048, 1024, 1024), id,
+                             st > 0);
+                mma_commit(&bar[B_CMMA]);
+            }
+            pending = true;
+            if (!mma_done()) break;
+            // ---------------- S <- e^{gC} S + E ----------------
+            {
+                float ev[64];
+                tmem_row64(tl + TM_E, ev);
+                const float gmc = cf[bb * 80 + 64];
+#pragma unroll
+                for (int j = 0; j < DVB; ++j) S[j] = gmc * S[j] + ev[j];
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_S, swz(trow, ch), S + ch * 8);
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            wsync();
+            if (wc == 0) mbar_arrive(&bar[B_KCFREE0 + bb]);
+        }
+        if (*abort_flag == 0) {
+            if (a.ST) {
+                float *dst = a.ST + (((size_t)b * H + h) * DK + trow) * DV + j0;
+#pragma unroll
+                for (int j = 0; j < DVB; j += 4)
+                    *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+            }
+        } else if (pending) {
+            volatile int dummy = 0;
+            mbar_wait(&bar[B_CMMA], ph & 1, &dummy, 100000000ull);
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == 0) tmem_dealloc(tbase, TM_COLS);
+}
+
+}  // namespace tcf2
+
+// Launch the warp-specialised forward (Gated DeltaNet / DeltaNet).
+cudaError_t tc_fwd2(const Geo &g, const Tensors &t, cudaStream_t s, Rec &rec) {
+    using namespace tcf2;
+    CUtensorMap mq, mk, mv;
+    const uint64_t Bn = g.B, T = g.T, H = g.H;
+    const bool ok = tc::make_map_4d_bf16(&mq, t.q, DK, H, T, Bn, 64) &&
+                    tc::make_map_4d_bf16(&mk, t.k, DK, H, T, Bn, 64) &&
+                    tc::make_map_4d_bf16(&mv, t.v, g.dv, H, T, Bn, 64);
+    if (!ok) return cudaErrorInvalidValue;
+    Args a;
+    a.alpha = t.alpha; a.beta = t.beta; a.S0 = t.S0; a.out = t.out; a.u = t.u; a.ST = t.S_T;
+    a.B = g.B; a.T = g.T; a.H = g.H; a.dv = g.dv; a.N = g.N;
+    const dim3 grid(g.dv / DVB, g.H, g.B);
+    const size_t smem = SMEM_BYTES + 1024;
+    cudaError_t e;
+    if (g.variant == VAR_GATED) {
+        e = cudaFuncSetAttribute(k_fwd_tc2<VAR_GATED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        rec.mark(s);
+        k_fwd_tc2<VAR_GATED><<<grid, NTHREADS, smem, s>>>(mq, mk, mv, a);
+    } else {
+        e = cudaFuncSetAttribute(k_fwd_tc2<VAR_DELTANET>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        rec.mark(s);
+        k_fwd_tc2<VAR_DELTANET><<<grid, NTHREADS, smem, s>>>(mq, mk, mv, a);
+    }
+    e = cudaGetLastError();
+    rec.mark(s);
+    return e;
+}
+
+}  // namespace dr

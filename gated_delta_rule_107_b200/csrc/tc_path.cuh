@@ -7,7 +7,9 @@ namespace dr {
 bool tc_fwd_supported(const Geo &g, bool bf16);
 size_t tc_fwd_ws_bytes(const Geo &g);
 cudaError_t tc_fwd(const Geo &g, const Tensors &t, void *workspace, cudaStream_t s, Rec &rec);
+// warp-specialised forward for Gated DeltaNet / DeltaNet (tc_fwd2.cu)
+cudaError_t tc_fwd2(const Geo &g, const Tensors &t, cudaStream_t s, Rec &rec);
 // number of launches of tc_fwd and their names
-int tc_fwd_launches(const char **names, int max_names);
+int tc_fwd_launches(const Geo &g, const char **names, int max_names);
 
 }  // namespace dr

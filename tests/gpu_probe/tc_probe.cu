@@ -11,6 +11,7 @@
 
 #include "../../gated_delta_rule_107_b200/csrc/dr_common.cuh"
 #include "../../gated_delta_rule_107_b200/csrc/tc_host.cuh"
+#include "../../gated_delta_rule_107_b200/csrc/tc_inverse.cuh"
 #include "../../gated_delta_rule_107_b200/csrc/tc_ptx.cuh"
 
 using namespace dr;
@@ -154,4 +155,28 @@ extern "C" int probe_tma(const void *X, void *out, int Bn, int T, int H, int d, 
         return -100;
     }
     return hs;
+}
+
+// probe_inverse: T = (I + A)^-1 of a strictly lower-triangular 64 x 64 A (row-major fp32)
+// by the warpgroup routine of tc_inverse.cuh.
+__global__ void k_probe_inverse(const float *A, float *T) {
+    __shared__ float sA[4096], sT[4096], ys[768];
+    const int tid = threadIdx.x;
+    for (int x = tid; x < 4096; x += 128) {
+        sA[sw64(x >> 6, x & 63)] = A[x];
+        sT[x] = 0.f;
+    }
+    __syncthreads();
+    unit_lower_inverse64(sA, sT, ys, tid, [] { __syncthreads(); });
+    for (int x = tid; x < 4096; x += 128) T[x] = sT[sw64(x >> 6, x & 63)];
+}
+
+extern "C" int probe_inverse(const float *A, float *T) {
+    k_probe_inverse<<<1, 128>>>(A, T);
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        fprintf(stderr, "probe_inverse: %s\n", cudaGetErrorString(e));
+        return -100;
+    }
+    return 0;
 }

@@ -21,7 +21,7 @@ LIB = os.path.join(HERE, "libtcprobe.so")
 @pytest.fixture(scope="module")
 def probe():
     deps = [SRC] + [os.path.join(HERE, "..", "..", "gated_delta_rule_107_b200", "csrc", f)
-                    for f in ("tc_ptx.cuh", "tc_host.cuh", "dr_common.cuh")]
+                    for f in ("tc_ptx.cuh", "tc_host.cuh", "dr_common.cuh", "tc_inverse.cuh")]
     if not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(p) for p in deps):
         subprocess.check_call(["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O2", "-std=c++17",
                                "-Xcompiler", "-fPIC", "-shared", "-o", LIB, SRC])
@@ -31,6 +31,8 @@ def probe():
     lib.probe_mma.restype = i
     lib.probe_tma.argtypes = [vp, vp] + [i] * 8
     lib.probe_tma.restype = i
+    lib.probe_inverse.argtypes = [vp, vp]
+    lib.probe_inverse.restype = i
     return lib
 
 
@@ -71,3 +73,24 @@ def test_tma_box_matches_swizzle(probe, b, h, t0, c0):
     rows = min(64, T - t0)
     ref[:rows] = X[b, t0:t0 + rows, h, c0:c0 + 64]
     assert torch.equal(out, ref)
+
+
+@pytest.mark.parametrize("seed,harsh", ((0, False), (1, False), (2, True)))
+def test_unit_lower_inverse(probe, seed, harsh):
+    """The warpgroup inverse of I + A (diagonal blocks + tf32 column chains) vs fp64."""
+    g = torch.Generator().manual_seed(seed)
+    k = torch.randn(64, 128, generator=g, dtype=torch.float64)
+    if harsh:  # strongly correlated keys, beta = 1: larger entries of A and of its inverse
+        k = k + 2.0 * torch.randn(1, 128, generator=g, dtype=torch.float64)
+    k = k / k.norm(dim=1, keepdim=True)
+    beta = torch.ones(64, dtype=torch.float64) if harsh else torch.sigmoid(torch.randn(64, generator=g,
+                                                                                       dtype=torch.float64))
+    gcum = torch.cumsum(-torch.nn.functional.softplus(torch.randn(64, generator=g, dtype=torch.float64) - 3), 0)
+    A = torch.tril(beta[:, None] * (k @ k.T) * torch.exp(gcum[:, None] - gcum[None, :]), -1)
+    ref = torch.linalg.inv(torch.eye(64, dtype=torch.float64) + A)
+    Ad = A.float().cuda().contiguous()
+    Td = torch.full((64, 64), float("nan"), device="cuda")
+    assert probe.probe_inverse(Ad.data_ptr(), Td.data_ptr()) == 0
+    Tl = torch.tril(Td.double().cpu())
+    err = (Tl - ref).abs().max().item() / ref.abs().max().item()
+    assert err < 2e-3, f"inverse rel err {err}"

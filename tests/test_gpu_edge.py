@@ -144,7 +144,8 @@ def test_split_sequence_tensor_core_path():
 
 
 def test_bf16_d128_uses_the_tensor_core_kernel():
-    assert binding.launches(8, 4096, 8, 128, 128, 1, 64, 1, 0) == ["k_fwd_tc"]
+    assert binding.launches(8, 4096, 8, 128, 128, 1, 64, 1, 0) == ["k_fwd_tc2"]
+    assert binding.launches(8, 4096, 8, 128, 128, 0, 64, 1, 0) == ["k_fwd_tc2"]
     assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 0) == ["k_fwd_tc"]
     assert binding.launches(1, 256, 2, 64, 64, 0, 64, 0, 0) == ["k_prep", "k_scan", "k_out"]
 
