@@ -58,11 +58,10 @@ constexpr uint32_t SMEM_BYTES = OFF_MISC + 8192;
 
 // misc
 constexpr uint32_t M_BAR = 0;        // 16 mbarriers
-constexpr uint32_t M_TMEM = 128, M_ABORT = 132, M_BIG = 136;
-constexpr uint32_t M_GB = 256;       // [2][2][64]: raw log gate, beta
-constexpr uint32_t M_PF = 1280;      // prep factors [7][64]
-constexpr uint32_t M_CF = 3072;      // chain factors [2][80]: e^{gC-g} (64), e^{gC}
-constexpr uint32_t M_YS = 4096;      // inverse scratch [3][256]
+constexpr uint32_t M_TMEM = 128, M_ABORT = 132, M_BIG = 136;  // M_BIG: int[2], per slot
+constexpr uint32_t M_PF = 256;       // prep factors [2 slots][7][64]
+constexpr uint32_t M_CF = 3840;      // chain factors [2][80]: e^{gC-g} (64), e^{gC}
+constexpr uint32_t M_YS = 4608;      // inverse scratch [3][256]
 static_assert(M_YS + 3 * 256 * 4 <= 8192, "misc overflow");
 enum { PF_GC = 0, PF_ROWA, PF_ROWP, PF_COLA, PF_BV, PF_BK, PF_EG };
 
@@ -106,8 +105,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + M_TMEM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + M_ABORT);
     volatile int *bigflag = reinterpret_cast<volatile int *>(sm + OFF_MISC + M_BIG);
-    float *gb = reinterpret_cast<float *>(sm + OFF_MISC + M_GB);
-    float *pf = reinterpret_cast<float *>(sm + OFF_MISC + M_PF);
+    float *pf_all = reinterpret_cast<float *>(sm + OFF_MISC + M_PF);
     float *cf = reinterpret_cast<float *>(sm + OFF_MISC + M_CF);
     float *ysc = reinterpret_cast<float *>(sm + OFF_MISC + M_YS);
 
@@ -137,26 +135,67 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int issued[2] = {0, 0}, v_issued = 0;
         for (int m = 0; m < N; ++m) {
             const int s = m & 1, t0 = m * C;
+            // slot s and its factors are free once the preparation of chunk m-2 is done;
+            // the chain's copy of k and its factors once the chain finished chunk m-2
             if (m >= 2 && !mbar_wait(&bar[B_EMPTY0 + s], ((m >> 1) - 1) & 1, abort_flag)) break;
+            if (m >= 2 && !mbar_wait(&bar[B_KCFREE0 + s], ((m >> 1) - 1) & 1, abort_flag)) break;
             unsigned char *slot = sm + s * SLOT;
             if (lane == 0) {
-                mbar_arrive_tx(&bar[B_FULL0 + s], 4 * 8192);
+                unsigned char *kc = sm + OFF_KC + s * 16384;
+                mbar_arrive_tx(&bar[B_FULL0 + s], 6 * 8192);
                 tma_load_4d(slot + 0, &tm_k, 0, h, t0, b, &bar[B_FULL0 + s]);
                 tma_load_4d(slot + 8192, &tm_q, 0, h, t0, b, &bar[B_FULL0 + s]);
                 tma_load_4d(slot + 16384, &tm_k, 64, h, t0, b, &bar[B_FULL0 + s]);
                 tma_load_4d(slot + 24576, &tm_q, 64, h, t0, b, &bar[B_FULL0 + s]);
+                tma_load_4d(kc, &tm_k, 0, h, t0, b, &bar[B_FULL0 + s]);
+                tma_load_4d(kc + 8192, &tm_k, 64, h, t0, b, &bar[B_FULL0 + s]);
             }
-            float *gbs = gb + s * 128;
-            for (int r = lane; r < C; r += 32) {
-                const int t = t0 + r;
-                const size_t row = ((size_t)b * T + t) * H + h;
-                float lg = 0.f, bt = 0.f;
-                if (t < T) {
-                    if (VAR == VAR_GATED) lg = tcf::bf(a.alpha, row);
-                    bt = tcf::bf(a.beta, row);
+            // in-chunk cumulative log gate and the row / column factors of this chunk
+            {
+                float lg[2], bt[2];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int t = t0 + lane + 32 * hh;
+                    const size_t row = ((size_t)b * T + t) * H + h;
+                    lg[hh] = 0.f;
+                    bt[hh] = 0.f;
+                    if (t < T) {
+                        if (VAR == VAR_GATED) lg[hh] = tcf::bf(a.alpha, row);
+                        bt[hh] = tcf::bf(a.beta, row);
+                    }
                 }
-                gbs[r] = lg;
-                gbs[64 + r] = bt;
+                float x0 = lg[0], x1 = lg[1];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y0 = __shfl_up_sync(0xffffffffu, x0, o);
+                    const float y1 = __shfl_up_sync(0xffffffffu, x1, o);
+                    if (lane >= o) { x0 += y0; x1 += y1; }
+                }
+                x1 += __shfl_sync(0xffffffffu, x0, 31);
+                const float gC = __shfl_sync(0xffffffffu, x1, 31);
+                const float gm = __shfl_sync(0xffffffffu, x0, 31);
+                float dev = fmaxf(fabsf(x0 - gm), fabsf(x1 - gm));
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) dev = fmaxf(dev, __shfl_xor_sync(0xffffffffu, dev, o));
+                float *pf = pf_all + s * 448;
+                const float xs[2] = {x0, x1};
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int r = lane + 32 * hh;
+                    const float x = xs[hh], e = __expf(x), d = __expf(x - gm);
+                    pf[PF_GC * 64 + r] = x;
+                    pf[PF_ROWA * 64 + r] = bt[hh] * d;
+                    pf[PF_ROWP * 64 + r] = d;
+                    pf[PF_COLA * 64 + r] = __expf(gm - x);
+                    pf[PF_BV * 64 + r] = bt[hh];
+                    pf[PF_BK * 64 + r] = bt[hh] * e;
+                    pf[PF_EG * 64 + r] = e;
+                    cf[s * 80 + r] = __expf(gC - x);
+                }
+                if (lane == 0) {
+                    cf[s * 80 + 64] = __expf(gC);
+                    bigflag[s] = dev > 80.f;
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[B_FULL0 + s]);
@@ -197,57 +236,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int s = m & 1, bb = m & 1;
             unsigned char *slot = sm + s * SLOT;
             mbar_wait(&bar[B_FULL0 + s], (m >> 1) & 1, abort_flag);
-            if (m >= 2) mbar_wait(&bar[B_KCFREE0 + bb], ((m >> 1) - 1) & 1, abort_flag);
             if (wabort()) break;
-            // ---------------- gates and factors; chain copy of k ----------------
-            if (wt < 32) {
-                const float *lg = gb + s * 128, *bt = lg + 64;
-                float x0 = lg[lane], x1 = lg[lane + 32];
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float y0 = __shfl_up_sync(0xffffffffu, x0, o);
-                    const float y1 = __shfl_up_sync(0xffffffffu, x1, o);
-                    if (lane >= o) { x0 += y0; x1 += y1; }
-                }
-                x1 += __shfl_sync(0xffffffffu, x0, 31);
-                const float gC = __shfl_sync(0xffffffffu, x1, 31);
-                const float gm = __shfl_sync(0xffffffffu, x0, 31);
-                float dev = fmaxf(fabsf(x0 - gm), fabsf(x1 - gm));
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) dev = fmaxf(dev, __shfl_xor_sync(0xffffffffu, dev, o));
-                const float b0 = bt[lane], b1 = bt[lane + 32];
-                pf[PF_GC * 64 + lane] = x0;
-                pf[PF_GC * 64 + lane + 32] = x1;
-                pf[PF_ROWA * 64 + lane] = b0 * __expf(x0 - gm);
-                pf[PF_ROWA * 64 + lane + 32] = b1 * __expf(x1 - gm);
-                pf[PF_ROWP * 64 + lane] = __expf(x0 - gm);
-                pf[PF_ROWP * 64 + lane + 32] = __expf(x1 - gm);
-                pf[PF_COLA * 64 + lane] = __expf(gm - x0);
-                pf[PF_COLA * 64 + lane + 32] = __expf(gm - x1);
-                pf[PF_BV * 64 + lane] = b0;
-                pf[PF_BV * 64 + lane + 32] = b1;
-                pf[PF_BK * 64 + lane] = b0 * __expf(x0);
-                pf[PF_BK * 64 + lane + 32] = b1 * __expf(x1);
-                pf[PF_EG * 64 + lane] = __expf(x0);
-                pf[PF_EG * 64 + lane + 32] = __expf(x1);
-                float *cfb = cf + bb * 80;
-                cfb[lane] = __expf(gC - x0);
-                cfb[lane + 32] = __expf(gC - x1);
-                if (lane == 0) {
-                    cfb[64] = __expf(gC);
-                    *bigflag = dev > 80.f;
-                }
-            }
-            {
-                unsigned char *kc = sm + OFF_KC + bb * 16384;
-                for (int x = wt; x < 1024; x += 128) {
-                    const int p = x >> 9, r = (x >> 3) & 63, ch = x & 7;
-                    const uint32_t o = swz(r, ch);
-                    *reinterpret_cast<uint4 *>(kc + p * 8192 + o) = *reinterpret_cast<const uint4 *>(slot + p * 16384 + o);
-                }
-            }
-            fence_proxy_async();
-            wsync();
+            const float *pf = pf_all + s * 448;
             // ---------------- P1: [k ; q] . k^T ----------------
             if (wt == 0) {
                 fence_after_sync();
@@ -266,16 +256,40 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             {
                 float g1[64];
                 tmem_row64(tl + TM_G1, g1);
-                const bool big = *bigflag != 0;
+                const bool big = bigflag[s] != 0;
                 const float *gc = pf + PF_GC * 64, *cola = pf + PF_COLA * 64;
-                if (trow < 64) {
-                    const int r = trow;
-                    const float rf = pf[PF_ROWA * 64 + r], br = pf[PF_BV * 64 + r];
+                const bool arow = trow < 64;
+                const int r = arow ? trow : trow - 64;
+                // gate factor of each (r, i): e^{g_r - g_i}, split at the midpoint unless the range is large
+                float f[64];
+                if (VAR == VAR_DELTANET) {
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) {
-                        float f = big ? br * __expf(gc[r] - gc[i]) : rf * cola[i];
-                        if (VAR == VAR_DELTANET) f = br;
-                        Asc[sw64(r, i)] = (i < r) ? g1[i] * f : 0.f;
+                    for (int i = 0; i < 64; ++i) f[i] = 1.f;
+                } else if (!big) {
+                    const float4 *c4 = reinterpret_cast<const float4 *>(cola);
+#pragma unroll
+                    for (int i4 = 0; i4 < 16; ++i4) {
+                        const float4 c = c4[i4];
+                        f[4 * i4] = c.x; f[4 * i4 + 1] = c.y; f[4 * i4 + 2] = c.z; f[4 * i4 + 3] = c.w;
+                    }
+                    const float rf = pf[PF_ROWP * 64 + r];
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) f[i] *= rf;
+                } else {
+                    const float gr = gc[r];
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) f[i] = __expf(gr - gc[i]);
+                }
+                if (arow) {
+                    const float br = pf[PF_BV * 64 + r];
+#pragma unroll
+                    for (int i4 = 0; i4 < 16; ++i4) {
+                        float4 v;
+                        v.x = (4 * i4 + 0 < r) ? g1[4 * i4 + 0] * f[4 * i4 + 0] * br : 0.f;
+                        v.y = (4 * i4 + 1 < r) ? g1[4 * i4 + 1] * f[4 * i4 + 1] * br : 0.f;
+                        v.z = (4 * i4 + 2 < r) ? g1[4 * i4 + 2] * f[4 * i4 + 2] * br : 0.f;
+                        v.w = (4 * i4 + 3 < r) ? g1[4 * i4 + 3] * f[4 * i4 + 3] * br : 0.f;
+                        *reinterpret_cast<float4 *>(&Asc[sw64(r, 4 * i4)]) = v;
                     }
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) {
@@ -285,14 +299,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         st_chunk(sm + OFF_IP, swz(r, ch), w);
                     }
                 } else {
-                    const int r = trow - 64;
-                    const float rf = pf[PF_ROWP * 64 + r];
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) {
-                        float f = big ? __expf(gc[r] - gc[i]) : rf * cola[i];
-                        if (VAR == VAR_DELTANET) f = 1.f;
-                        g1[i] = (i <= r) ? g1[i] * f : 0.f;
-                    }
+                    for (int i = 0; i < 64; ++i) g1[i] = (i <= r) ? g1[i] * f[i] : 0.f;
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_IP, swz(trow, ch), g1 + ch * 8);
                 }
@@ -303,12 +311,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const int i = wt;
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) {
-                        float w[8];
+                        const float4 lo = *reinterpret_cast<const float4 *>(&Tf[sw64(i, ch * 8)]);
+                        const float4 hi = *reinterpret_cast<const float4 *>(&Tf[sw64(i, ch * 8 + 4)]);
+                        float w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int n = ch * 8 + e;
-                            w[e] = (n <= i) ? Tf[sw64(i, n)] : 0.f;
-                        }
+                        for (int e = 0; e < 8; ++e) w[e] = (ch * 8 + e <= i) ? w[e] : 0.f;
                         st_chunk(sm + OFF_TT, swz(i, ch), w);
                     }
                 }

@@ -14,9 +14,10 @@
 namespace dr {
 namespace tc {
 
-// fp32 64 x 64 tile with an XOR swizzle on the column (conflict-free row writes by
-// 32 threads that each own one row).
-__device__ __forceinline__ int sw64(int r, int c) { return r * 64 + (c ^ (r & 31)); }
+// fp32 64 x 64 tile with an XOR swizzle of 4-float groups by the row (conflict-free
+// float4 row writes by threads that each own one row, and conflict-free A-fragment
+// reads of the warp-level MMAs below).
+__device__ __forceinline__ int sw64(int r, int c) { return r * 64 + (c ^ ((r & 7) << 2)); }
 
 __device__ __forceinline__ uint32_t to_tf32(float x) {
     uint32_t r;
