@@ -118,6 +118,11 @@ static int bwd_impl(const void *q, const void *k, const void *v, const void *alp
     t.dout = dout; t.du = du; t.dS_T = dS_T;
     t.dq = dq; t.dk = dk_; t.dv = dv_; t.dalpha = dalpha; t.dbeta = dbeta; t.dS0 = dS0;
     const SimtWs w = simt_ws_carve(g, true, workspace);
+    if (tc_bwd_recompute_supported(g, dtype == DR_BF16)) {
+        rc = launch_status(tc_bwd_recompute(g, t, w, s, rec));
+        if (rc != DR_OK) return rc;
+        return launch_status(simt_bwd(g, t, true, w, s, rec, true));
+    }
     return launch_status(simt_bwd(g, t, dtype == DR_BF16, w, s, rec));
 }
 
@@ -130,8 +135,13 @@ static int launch_plan(const Geo &g, int dtype, bool bwd, const char **names, in
         n = tc_fwd_launches(g, names, max_names);
         return n;
     }
-    src = bwd ? SIMT_BWD_KERNELS : SIMT_FWD_KERNELS;
-    n = bwd ? 5 : 3;
+    if (bwd && tc_bwd_recompute_supported(g, dtype == DR_BF16)) {
+        src = TC_BWD_KERNELS;
+        n = 4;
+    } else {
+        src = bwd ? SIMT_BWD_KERNELS : SIMT_FWD_KERNELS;
+        n = bwd ? 5 : 3;
+    }
     for (int i = 0; names && i < n && i < max_names; ++i) names[i] = src[i];
     return n;
 }

@@ -458,6 +458,18 @@ __global__ void __launch_bounds__(NT) k_bwd_intra(Geo g, IO<TI> io, SimtWs w) {
         }
     }
     __syncthreads();
+    if (!kda) {
+        // scalar gates: fold the pair factor e^{g_r - g_i} (<= 1) into dM and dP once
+        for (int x = tid; x < C * C; x += NT) {
+            const int r = x / C, i = x % C;
+            if (i <= r) {
+                const float e = (g.variant == VAR_GATED) ? __expf(gs[r * DK] - gs[i * DK]) : 1.f;
+                dM[x] *= e;
+                dP[x] *= e;
+            }
+        }
+        __syncthreads();
+    }
     // per (r, c) gradients; dg_rc overwrites Y[r][c] (dB_k) -- each entry touched by one thread
     {
         const float *Qd = w.Qd + ci * C * DK, *Tm = w.Tm + ci * C * DK;
@@ -468,14 +480,23 @@ __global__ void __launch_bounds__(NT) k_bwd_intra(Geo g, IO<TI> io, SimtWs w) {
                 const float grc = gs[r * DK + c], gam = __expf(grc), kv = ks[r * DK + c], qv = qs[r * DK + c];
                 const float gL = gs[(C - 1) * DK + c];
                 float X = 0.f, Yv = 0.f, Z = 0.f;
-                for (int i = 0; i <= r; ++i) {
-                    const float e = __expf(grc - gs[i * DK + c]) * ks[i * DK + c];
-                    X += dP[r * C + i] * e;
-                    Yv += dM[r * C + i] * e;  // dM[r][r] == 0
-                }
-                for (int rr = r; rr < C; ++rr) {
-                    const float e = __expf(gs[rr * DK + c] - grc);
-                    Z += (dM[rr * C + r] * ks[rr * DK + c] + dP[rr * C + r] * qs[rr * DK + c]) * e;
+                if (kda) {
+                    for (int i = 0; i <= r; ++i) {
+                        const float e = __expf(grc - gs[i * DK + c]) * ks[i * DK + c];
+                        X += dP[r * C + i] * e;
+                        Yv += dM[r * C + i] * e;  // dM[r][r] == 0
+                    }
+                    for (int rr = r; rr < C; ++rr) {
+                        const float e = __expf(gs[rr * DK + c] - grc);
+                        Z += (dM[rr * C + r] * ks[rr * DK + c] + dP[rr * C + r] * qs[rr * DK + c]) * e;
+                    }
+                } else {
+                    for (int i = 0; i <= r; ++i) {
+                        const float kic = ks[i * DK + c];
+                        X += dP[r * C + i] * kic;
+                        Yv += dM[r * C + i] * kic;
+                    }
+                    for (int rr = r; rr < C; ++rr) Z += dM[rr * C + r] * ks[rr * DK + c] + dP[rr * C + r] * qs[rr * DK + c];
                 }
                 const float qd = Qd[r * DK + c], tm = Tm[r * DK + c], dBk = Y[r * DY + c];
                 const float eb = __expf(gL - grc);
@@ -600,6 +621,7 @@ template <typename K> static cudaError_t prep_attr(K kern, size_t smem) {
 
 const char *const SIMT_FWD_KERNELS[3] = {"k_prep", "k_scan", "k_out"};
 const char *const SIMT_BWD_KERNELS[5] = {"k_prep", "k_scan", "k_scan_bwd", "k_bwd_state", "k_bwd_intra"};
+const char *const TC_BWD_KERNELS[4] = {"k_fwd_tc2", "k_scan_bwd", "k_bwd_state", "k_bwd_intra"};
 
 template <typename TI>
 static cudaError_t forward_chain(const Geo &g, const IO<TI> &io, const SimtWs &w, const float *S0, float *ST,
@@ -633,7 +655,8 @@ static cudaError_t fwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaSt
 }
 
 template <typename TI>
-static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec) {
+static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec,
+                         bool recomputed) {
     const IO<TI> io = io_of<TI>(t);
     const size_t C = g.C, DK = g.dk, DV = g.dv;
     const dim3 gc(g.N, g.H, g.B), gs(g.dv / JB, g.H, g.B);
@@ -643,8 +666,10 @@ static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaSt
     DR_TRY(prep_attr(k_scan_bwd<TI>, sm_sb));
     DR_TRY(prep_attr(k_bwd_state<TI>, sm_st));
     DR_TRY(prep_attr(k_bwd_intra<TI>, sm_in));
-    DR_TRY(forward_chain<TI>(g, io, w, t.S0, nullptr, 0, s, rec));
-    rec.mark(s);
+    if (!recomputed) {
+        DR_TRY(forward_chain<TI>(g, io, w, t.S0, nullptr, 0, s, rec));
+        rec.mark(s);  // (after a tensor-core recompute, its end event already marks this point)
+    }
     k_scan_bwd<TI><<<gs, NT, sm_sb, s>>>(g, io, w, t.dS_T, t.dS0);
     DR_TRY(cudaGetLastError());
     rec.mark(s);
@@ -661,8 +686,9 @@ cudaError_t simt_fwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w,
     return bf16 ? fwd_t<__nv_bfloat16>(g, t, w, s, rec) : fwd_t<float>(g, t, w, s, rec);
 }
 
-cudaError_t simt_bwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec) {
-    return bf16 ? bwd_t<__nv_bfloat16>(g, t, w, s, rec) : bwd_t<float>(g, t, w, s, rec);
+cudaError_t simt_bwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec,
+                     bool recomputed) {
+    return bf16 ? bwd_t<__nv_bfloat16>(g, t, w, s, rec, recomputed) : bwd_t<float>(g, t, w, s, rec, recomputed);
 }
 
 }  // namespace dr

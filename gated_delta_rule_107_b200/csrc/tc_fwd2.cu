@@ -31,6 +31,7 @@
 #include "tc_path.cuh"
 #include "tc_ptx.cuh"
 #include "tc_tile.cuh"
+#include "simt_path.cuh"
 
 namespace dr {
 namespace tcf2 {
@@ -79,6 +80,8 @@ struct Args {
     void *out, *u;
     float *ST;
     int B, T, H, dv, N;
+    // recompute mode (backward): fp32 chunk products for the CUDA-core backward kernels
+    float *W, *Ut, *G, *P, *Sn, *Un;
 };
 
 __device__ __forceinline__ void st_row_global(void *base, size_t elem_off, const float *v) {
@@ -94,7 +97,10 @@ __device__ __forceinline__ void st_row_global(void *base, size_t elem_off, const
     }
 }
 
-template <int VAR>
+// SAVE = 0: forward (o, u, S_T).  SAVE = 1: recompute for the backward -- no o / u / S_T;
+// instead the chunk products W, U~, g, P, the entering state S_n and the write values U
+// are stored in the fp32 chunk-major layout the CUDA-core backward kernels read.
+template <int VAR, int SAVE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_fwd_tc2(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, Args a) {
@@ -195,6 +201,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (lane == 0) {
                     cf[s * 80 + 64] = __expf(gC);
                     bigflag[s] = dev > 80.f;
+                }
+                if (SAVE && half == 0) {
+                    float *Gc = a.G + ((((size_t)b * H + h) * N + m) * C) * DK;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const float4 x4 = make_float4(xs[hh], xs[hh], xs[hh], xs[hh]);
+                        float4 *dst = reinterpret_cast<float4 *>(Gc + (size_t)(lane + 32 * hh) * DK);
+#pragma unroll
+                        for (int c4 = 0; c4 < DK / 4; ++c4) dst[c4] = x4;
+                    }
                 }
             }
             __syncwarp();
@@ -303,6 +319,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     for (int i = 0; i < 64; ++i) g1[i] = (i <= r) ? g1[i] * f[i] : 0.f;
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_IP, swz(trow, ch), g1 + ch * 8);
+                    if (SAVE && half == 0) {
+                        float4 *dst = reinterpret_cast<float4 *>(a.P + ((((size_t)b * H + h) * N + m) * C + r) * C);
+#pragma unroll
+                        for (int i4 = 0; i4 < 16; ++i4)
+                            dst[i4] = make_float4(g1[4 * i4], g1[4 * i4 + 1], g1[4 * i4 + 2], g1[4 * i4 + 3]);
+                    }
                 }
                 fence_before_sync();
                 wsync();
@@ -375,6 +397,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             pending = true;
             if (!mma_done()) break;
             if (wt == 0) mbar_arrive(&bar[B_VEMPTY]);
+            if (SAVE && trow < 64) {
+                const size_t ci = ((size_t)b * H + h) * N + m;
+                float rv[64];
+                tmem_row64(tl + TM_D0 + bb * 64, rv);
+                float4 *du = reinterpret_cast<float4 *>(a.Ut + (ci * C + trow) * DV + j0);
+#pragma unroll
+                for (int i4 = 0; i4 < 16; ++i4) du[i4] = make_float4(rv[4 * i4], rv[4 * i4 + 1], rv[4 * i4 + 2], rv[4 * i4 + 3]);
+                if (half == 0) {
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        tmem_row64(tl + TM_X + hh * 64, rv);
+                        float4 *dw = reinterpret_cast<float4 *>(a.W + (ci * C + trow) * DK + hh * 64);
+#pragma unroll
+                        for (int i4 = 0; i4 < 16; ++i4)
+                            dw[i4] = make_float4(rv[4 * i4], rv[4 * i4 + 1], rv[4 * i4 + 2], rv[4 * i4 + 3]);
+                    }
+                }
+            }
             // ---------------- A_chain ----------------
             if (m >= 1) mbar_wait(&bar[B_ACFREE], (m - 1) & 1, abort_flag);
             if (wabort()) break;
@@ -446,6 +486,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int L = min(C, T - t0);
             mbar_wait(&bar[B_READY0 + bb], (m >> 1) & 1, abort_flag);
             if (wabort()) break;
+            if (SAVE) {
+                float4 *dst = reinterpret_cast<float4 *>(a.Sn + ((((size_t)b * H + h) * N + m) * DK + trow) * DV + j0);
+#pragma unroll
+                for (int j4 = 0; j4 < DVB / 4; ++j4) dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
+            }
             // ---------------- C1: D += A_chain . S ----------------
             if (wc == 0) {
                 fence_after_sync();
@@ -466,7 +511,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tmem_row64(tl + TM_D0 + bb * 64, dv);
                 if (trow < 64) {
                     const int r = trow;
-                    if (a.u && r < L) st_row_global(a.u, (((size_t)b * T + t0 + r) * H + h) * DV + j0, dv);
+                    if (SAVE) {
+                        float4 *dst = reinterpret_cast<float4 *>(a.Un + ((((size_t)b * H + h) * N + m) * C + r) * DV + j0);
+#pragma unroll
+                        for (int j4 = 0; j4 < 16; ++j4)
+                            dst[j4] = make_float4(dv[4 * j4], dv[4 * j4 + 1], dv[4 * j4 + 2], dv[4 * j4 + 3]);
+                    } else if (a.u && r < L) {
+                        st_row_global(a.u, (((size_t)b * T + t0 + r) * H + h) * DV + j0, dv);
+                    }
                     const float f = cf[bb * 80 + r];
 #pragma unroll
                     for (int i = 0; i < 64; ++i) dv[i] *= f;
@@ -474,7 +526,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_U, swz(r, ch), dv + ch * 8);
                 } else {
                     const int r = trow - 64;
-                    if (r < L) st_row_global(a.out, (((size_t)b * T + t0 + r) * H + h) * DV + j0, dv);
+                    if (!SAVE && r < L) st_row_global(a.out, (((size_t)b * T + t0 + r) * H + h) * DV + j0, dv);
                 }
             }
             fence_proxy_async();
@@ -510,7 +562,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (wc == 0) mbar_arrive(&bar[B_KCFREE0 + bb]);
         }
         if (*abort_flag == 0) {
-            if (a.ST) {
+            if (!SAVE && a.ST) {
                 float *dst = a.ST + (((size_t)b * H + h) * DK + trow) * DV + j0;
 #pragma unroll
                 for (int j = 0; j < DVB; j += 4)
@@ -529,8 +581,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 }  // namespace tcf2
 
-// Launch the warp-specialised forward (Gated DeltaNet / DeltaNet).
-cudaError_t tc_fwd2(const Geo &g, const Tensors &t, cudaStream_t s, Rec &rec) {
+template <int VAR, int SAVE>
+static cudaError_t launch_tc2(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const tcf2::Args &a,
+                              dim3 grid, size_t smem, cudaStream_t s, Rec &rec) {
+    cudaError_t e = cudaFuncSetAttribute(tcf2::k_fwd_tc2<VAR, SAVE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    rec.mark(s);
+    tcf2::k_fwd_tc2<VAR, SAVE><<<grid, tcf2::NTHREADS, smem, s>>>(mq, mk, mv, a);
+    e = cudaGetLastError();
+    rec.mark(s);
+    return e;
+}
+
+static cudaError_t tc2_common(const Geo &g, const Tensors &t, const SimtWs *w, cudaStream_t s, Rec &rec) {
     using namespace tcf2;
     CUtensorMap mq, mk, mv;
     const uint64_t Bn = g.B, T = g.T, H = g.H;
@@ -538,26 +602,27 @@ cudaError_t tc_fwd2(const Geo &g, const Tensors &t, cudaStream_t s, Rec &rec) {
                     tc::make_map_4d_bf16(&mk, t.k, DK, H, T, Bn, 64) &&
                     tc::make_map_4d_bf16(&mv, t.v, g.dv, H, T, Bn, 64);
     if (!ok) return cudaErrorInvalidValue;
-    Args a;
+    Args a = {};
     a.alpha = t.alpha; a.beta = t.beta; a.S0 = t.S0; a.out = t.out; a.u = t.u; a.ST = t.S_T;
     a.B = g.B; a.T = g.T; a.H = g.H; a.dv = g.dv; a.N = g.N;
+    if (w) {
+        a.W = w->W; a.Ut = w->Ut; a.G = w->G; a.P = w->P; a.Sn = w->Sn; a.Un = w->Un;
+    }
     const dim3 grid(g.dv / DVB, g.H, g.B);
     const size_t smem = SMEM_BYTES + 1024;
-    cudaError_t e;
-    if (g.variant == VAR_GATED) {
-        e = cudaFuncSetAttribute(k_fwd_tc2<VAR_GATED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        rec.mark(s);
-        k_fwd_tc2<VAR_GATED><<<grid, NTHREADS, smem, s>>>(mq, mk, mv, a);
-    } else {
-        e = cudaFuncSetAttribute(k_fwd_tc2<VAR_DELTANET>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        rec.mark(s);
-        k_fwd_tc2<VAR_DELTANET><<<grid, NTHREADS, smem, s>>>(mq, mk, mv, a);
-    }
-    e = cudaGetLastError();
-    rec.mark(s);
-    return e;
+    if (g.variant == VAR_GATED)
+        return w ? launch_tc2<VAR_GATED, 1>(mq, mk, mv, a, grid, smem, s, rec)
+                 : launch_tc2<VAR_GATED, 0>(mq, mk, mv, a, grid, smem, s, rec);
+    return w ? launch_tc2<VAR_DELTANET, 1>(mq, mk, mv, a, grid, smem, s, rec)
+             : launch_tc2<VAR_DELTANET, 0>(mq, mk, mv, a, grid, smem, s, rec);
+}
+
+// Warp-specialised forward (Gated DeltaNet / DeltaNet).
+cudaError_t tc_fwd2(const Geo &g, const Tensors &t, cudaStream_t s, Rec &rec) { return tc2_common(g, t, nullptr, s, rec); }
+
+// The same kernel in recompute mode: fills W, U~, g, P, S_n, U of the CUDA-core backward workspace.
+cudaError_t tc_bwd_recompute(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec) {
+    return tc2_common(g, t, &w, s, rec);
 }
 
 }  // namespace dr
