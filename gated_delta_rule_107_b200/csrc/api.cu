@@ -87,9 +87,14 @@ static int fwd_impl(const void *q, const void *k, const void *v, const void *alp
     }
     Tensors t = {};
     t.q = q; t.k = k; t.v = v; t.alpha = alpha; t.beta = beta; t.S0 = S0; t.out = out; t.u = u; t.S_T = S_T;
-    if (use_tc_fwd(g, dtype)) return launch_status(tc_fwd(g, t, workspace, s, rec));
-    const SimtWs w = simt_ws_carve(g, false, workspace);
-    return launch_status(simt_fwd(g, t, dtype == DR_BF16, w, s, rec));
+    if (use_tc_fwd(g, dtype)) {
+        rc = launch_status(tc_fwd(g, t, workspace, s, rec));
+    } else {
+        const SimtWs w = simt_ws_carve(g, false, workspace);
+        rc = launch_status(simt_fwd(g, t, dtype == DR_BF16, w, s, rec));
+    }
+    rec.mark(s);  // end of the last launch
+    return rc;
 }
 
 static int bwd_impl(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
@@ -120,10 +125,14 @@ static int bwd_impl(const void *q, const void *k, const void *v, const void *alp
     const SimtWs w = simt_ws_carve(g, true, workspace);
     if (tc_bwd_recompute_supported(g, dtype == DR_BF16)) {
         rc = launch_status(tc_bwd_recompute(g, t, w, s, rec));
-        if (rc != DR_OK) return rc;
-        return launch_status(simt_bwd(g, t, true, w, s, rec, true));
+        if (rc == DR_OK) rc = launch_status(tc_bwd_reverse(g, t, w, s, rec));
+        if (rc == DR_OK) rc = launch_status(tc_bwd_state(g, t, w, s, rec));
+        if (rc == DR_OK) rc = launch_status(simt_bwd(g, t, true, w, s, rec, true, true));
+    } else {
+        rc = launch_status(simt_bwd(g, t, dtype == DR_BF16, w, s, rec));
     }
-    return launch_status(simt_bwd(g, t, dtype == DR_BF16, w, s, rec));
+    rec.mark(s);  // end of the last launch
+    return rc;
 }
 
 // Number of kernel launches of one call and their names (launch order).

@@ -3,5 +3,6 @@
 #include "simt_path.cu"
 #include "tc_fwd.cu"
 #include "tc_fwd2.cu"
+#include "tc_bwd.cu"
 #include "api.cu"
 #include "noalloc.cu"

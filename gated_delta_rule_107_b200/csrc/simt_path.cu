@@ -621,7 +621,7 @@ template <typename K> static cudaError_t prep_attr(K kern, size_t smem) {
 
 const char *const SIMT_FWD_KERNELS[3] = {"k_prep", "k_scan", "k_out"};
 const char *const SIMT_BWD_KERNELS[5] = {"k_prep", "k_scan", "k_scan_bwd", "k_bwd_state", "k_bwd_intra"};
-const char *const TC_BWD_KERNELS[4] = {"k_fwd_tc2", "k_scan_bwd", "k_bwd_state", "k_bwd_intra"};
+const char *const TC_BWD_KERNELS[4] = {"k_fwd_tc2(recompute)", "k_fwd_tc2(reverse)", "k_bwd_state_tc", "k_bwd_intra"};
 
 template <typename TI>
 static cudaError_t forward_chain(const Geo &g, const IO<TI> &io, const SimtWs &w, const float *S0, float *ST,
@@ -649,14 +649,12 @@ static cudaError_t fwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaSt
     DR_TRY(forward_chain<TI>(g, io, w, t.S0, t.S_T, t.u != nullptr, s, rec));
     rec.mark(s);
     k_out<TI><<<dim3(g.N, g.H, g.B), NT, sm_out, s>>>(g, io, w);
-    DR_TRY(cudaGetLastError());
-    rec.mark(s);
-    return cudaSuccess;
+    return cudaGetLastError();
 }
 
 template <typename TI>
 static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec,
-                         bool recomputed) {
+                         bool recomputed, bool only_intra) {
     const IO<TI> io = io_of<TI>(t);
     const size_t C = g.C, DK = g.dk, DV = g.dv;
     const dim3 gc(g.N, g.H, g.B), gs(g.dv / JB, g.H, g.B);
@@ -666,20 +664,18 @@ static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaSt
     DR_TRY(prep_attr(k_scan_bwd<TI>, sm_sb));
     DR_TRY(prep_attr(k_bwd_state<TI>, sm_st));
     DR_TRY(prep_attr(k_bwd_intra<TI>, sm_in));
-    if (!recomputed) {
-        DR_TRY(forward_chain<TI>(g, io, w, t.S0, nullptr, 0, s, rec));
-        rec.mark(s);  // (after a tensor-core recompute, its end event already marks this point)
+    if (!only_intra) {
+        if (!recomputed) DR_TRY(forward_chain<TI>(g, io, w, t.S0, nullptr, 0, s, rec));
+        rec.mark(s);
+        k_scan_bwd<TI><<<gs, NT, sm_sb, s>>>(g, io, w, t.dS_T, t.dS0);
+        DR_TRY(cudaGetLastError());
+        rec.mark(s);
+        k_bwd_state<TI><<<gc, NT, sm_st, s>>>(g, io, w);
+        DR_TRY(cudaGetLastError());
     }
-    k_scan_bwd<TI><<<gs, NT, sm_sb, s>>>(g, io, w, t.dS_T, t.dS0);
-    DR_TRY(cudaGetLastError());
-    rec.mark(s);
-    k_bwd_state<TI><<<gc, NT, sm_st, s>>>(g, io, w);
-    DR_TRY(cudaGetLastError());
     rec.mark(s);
     k_bwd_intra<TI><<<gc, NT, sm_in, s>>>(g, io, w);
-    DR_TRY(cudaGetLastError());
-    rec.mark(s);
-    return cudaSuccess;
+    return cudaGetLastError();
 }
 
 cudaError_t simt_fwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec) {
@@ -687,8 +683,9 @@ cudaError_t simt_fwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w,
 }
 
 cudaError_t simt_bwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec,
-                     bool recomputed) {
-    return bf16 ? bwd_t<__nv_bfloat16>(g, t, w, s, rec, recomputed) : bwd_t<float>(g, t, w, s, rec, recomputed);
+                     bool recomputed, bool only_intra) {
+    return bf16 ? bwd_t<__nv_bfloat16>(g, t, w, s, rec, recomputed, only_intra)
+                : bwd_t<float>(g, t, w, s, rec, recomputed, only_intra);
 }
 
 }  // namespace dr

@@ -24,9 +24,11 @@ struct SimtWs {
 size_t simt_ws_bytes(const Geo &g, bool bwd);
 SimtWs simt_ws_carve(const Geo &g, bool bwd, void *base);
 cudaError_t simt_fwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec);
-// recomputed = true: W, U~, G, P, S_n, U are already in the workspace (tensor-core recompute)
+// recomputed = true: W, U~, G, P, S_n, U are already in the workspace (tensor-core recompute);
+// only_intra = true: dS_{n+1}, dU, Qd, dWm, Tm, RS are too (tensor-core reverse chain and
+// state products) and only the intra-chunk gradient kernel runs.
 cudaError_t simt_bwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec,
-                     bool recomputed = false);
+                     bool recomputed = false, bool only_intra = false);
 // kernel names in launch order (for the timed entry points)
 extern const char *const SIMT_FWD_KERNELS[3];
 extern const char *const SIMT_BWD_KERNELS[5];

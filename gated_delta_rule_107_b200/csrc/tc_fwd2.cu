@@ -67,7 +67,7 @@ static_assert(M_YS + 3 * 256 * 4 <= 8192, "misc overflow");
 enum { PF_GC = 0, PF_ROWA, PF_ROWP, PF_COLA, PF_BV, PF_BK, PF_EG };
 
 // TMEM columns
-constexpr uint32_t TM_G1 = 0, TM_X = 64, TM_D0 = 192, TM_E = 320, TM_COLS = 512;
+constexpr uint32_t TM_G1 = 0, TM_X = 64, TM_D0 = 192, TM_E = 320, TM_G = 384, TM_COLS = 512;
 
 enum {
     B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_VFULL, B_VEMPTY, B_PMMA, B_CMMA,
@@ -82,6 +82,9 @@ struct Args {
     int B, T, H, dv, N;
     // recompute mode (backward): fp32 chunk products for the CUDA-core backward kernels
     float *W, *Ut, *G, *P, *Sn, *Un;
+    // reverse mode: dL/dS of the state leaving each chunk; whether du is given
+    float *dSn;
+    int has_du;
 };
 
 __device__ __forceinline__ void st_row_global(void *base, size_t elem_off, const float *v) {
@@ -97,13 +100,23 @@ __device__ __forceinline__ void st_row_global(void *base, size_t elem_off, const
     }
 }
 
-// SAVE = 0: forward (o, u, S_T).  SAVE = 1: recompute for the backward -- no o / u / S_T;
-// instead the chunk products W, U~, g, P, the entering state S_n and the write values U
-// are stored in the fp32 chunk-major layout the CUDA-core backward kernels read.
-template <int VAR, int SAVE>
+// MODE 0: forward (o, u, S_T).
+// MODE 1: recompute for the backward -- no o / u / S_T; instead the chunk products W, U~,
+//         g, P, the entering state S_n and the write values U are stored in the fp32
+//         chunk-major layout the backward kernels read.
+// MODE 2: the backward's reverse state chain.  Chunks are visited last to first; the
+//         preparation is the same (A_chain = [-W ; Q~ - P W]) minus P4, the chain's copy
+//         of k is scaled to Kbar = e^{g_C - g} k, and the chain warpgroup evaluates
+//           dS_n = e^{g_C} dS_{n+1} + A_chain^T [du ; dO] + ((-W)^T Kbar) dS_{n+1}
+//         (= e^{g_C} dS+ + Qtil^T dO - W^T dU with dU = du + P^T dO + Kbar dS+),
+//         storing dS_{n+1} for every chunk and dS_0 at the end.  S0 / S_T carry dS_T / dS0,
+//         the v map carries dO and the x map du.
+template <int VAR, int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_fwd_tc2(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, Args a) {
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_x, Args a) {
+    constexpr int SAVE = (MODE == 1);
+    constexpr bool REV = (MODE == 2);
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -140,7 +153,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         int issued[2] = {0, 0}, v_issued = 0;
         for (int m = 0; m < N; ++m) {
-            const int s = m & 1, t0 = m * C;
+            const int mc = REV ? N - 1 - m : m;  // chunk processed in iteration m
+            const int s = m & 1, t0 = mc * C;
             // slot s and its factors are free once the preparation of chunk m-2 is done;
             // the chain's copy of k and its factors once the chain finished chunk m-2
             if (m >= 2 && !mbar_wait(&bar[B_EMPTY0 + s], ((m >> 1) - 1) & 1, abort_flag)) break;
@@ -203,7 +217,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     bigflag[s] = dev > 80.f;
                 }
                 if (SAVE && half == 0) {
-                    float *Gc = a.G + ((((size_t)b * H + h) * N + m) * C) * DK;
+                    float *Gc = a.G + ((((size_t)b * H + h) * N + mc) * C) * DK;
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         const float4 x4 = make_float4(xs[hh], xs[hh], xs[hh], xs[hh]);
@@ -218,8 +232,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             issued[s]++;
             if (m >= 1 && !mbar_wait(&bar[B_VEMPTY], (m - 1) & 1, abort_flag)) break;
             if (lane == 0) {
-                mbar_arrive_tx(&bar[B_VFULL], 8192);
-                tma_load_4d(sm + OFF_V, &tm_v, j0, h, t0, b, &bar[B_VFULL]);
+                if (REV) {  // dO (and du) of this chunk for the chain
+                    mbar_arrive_tx(&bar[B_VFULL], a.has_du ? 16384 : 8192);
+                    tma_load_4d(sm + OFF_U, &tm_v, j0, h, t0, b, &bar[B_VFULL]);
+                    if (a.has_du) tma_load_4d(sm + OFF_V, &tm_x, j0, h, t0, b, &bar[B_VFULL]);
+                } else {
+                    mbar_arrive_tx(&bar[B_VFULL], 8192);
+                    tma_load_4d(sm + OFF_V, &tm_v, j0, h, t0, b, &bar[B_VFULL]);
+                }
             }
             v_issued++;
         }
@@ -249,11 +269,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float *Asc = reinterpret_cast<float *>(sm + OFF_RR);
         float *Tf = Asc + 4096;
         for (int m = 0; m < N; ++m) {
+            const int mc = REV ? N - 1 - m : m;
             const int s = m & 1, bb = m & 1;
             unsigned char *slot = sm + s * SLOT;
             mbar_wait(&bar[B_FULL0 + s], (m >> 1) & 1, abort_flag);
             if (wabort()) break;
             const float *pf = pf_all + s * 448;
+            if (REV) {  // the chain's copy of k becomes Kbar = e^{g_C - g} k
+                unsigned char *kc = sm + OFF_KC + bb * 16384;
+                const float *rowf = cf + bb * 80;
+                for (int x = wt; x < 1024; x += 128) {
+                    const int p = x >> 9, r = (x >> 3) & 63, ch = x & 7;
+                    const uint32_t o = (uint32_t)p * 8192 + swz(r, ch);
+                    float kv[8];
+                    ld_chunk(kc, o, kv);
+                    const float f = rowf[r];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) kv[e] *= f;
+                    st_chunk(kc, o, kv);
+                }
+            }
             // ---------------- P1: [k ; q] . k^T ----------------
             if (wt == 0) {
                 fence_after_sync();
@@ -320,7 +355,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_IP, swz(trow, ch), g1 + ch * 8);
                     if (SAVE && half == 0) {
-                        float4 *dst = reinterpret_cast<float4 *>(a.P + ((((size_t)b * H + h) * N + m) * C + r) * C);
+                        float4 *dst = reinterpret_cast<float4 *>(a.P + ((((size_t)b * H + h) * N + mc) * C + r) * C);
 #pragma unroll
                         for (int i4 = 0; i4 < 16; ++i4)
                             dst[i4] = make_float4(g1[4 * i4], g1[4 * i4 + 1], g1[4 * i4 + 2], g1[4 * i4 + 3]);
@@ -374,8 +409,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     st_chunk(sm + OFF_RR + 16384, swz(trow, ch), w2);
                 }
             }
-            mbar_wait(&bar[B_VFULL], m & 1, abort_flag);
-            if (m >= 2) mbar_wait(&bar[B_DFREE0 + bb], ((m >> 1) - 1) & 1, abort_flag);
+            if (!REV) {
+                mbar_wait(&bar[B_VFULL], m & 1, abort_flag);
+                if (m >= 2) mbar_wait(&bar[B_DFREE0 + bb], ((m >> 1) - 1) & 1, abort_flag);
+            }
             fence_proxy_async();
             fence_before_sync();
             if (wabort()) break;
@@ -388,17 +425,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 for (int st = 0; st < 4; ++st)
                     mma_bf16(tbase + TM_X, sdesc(rr + 16384 + st * 32, 16, 1024), sdesc(sk + st * 2048, 16384, 1024),
                              id3, st > 0);
+                if (!REV) {
 #pragma unroll
-                for (int st = 0; st < 4; ++st)
-                    mma_bf16(tbase + TM_D0 + bb * 64, sdesc(rr + st * 32, 16, 1024),
-                             sdesc(vv + st * 2048, 1024, 1024), id4, st > 0);
+                    for (int st = 0; st < 4; ++st)
+                        mma_bf16(tbase + TM_D0 + bb * 64, sdesc(rr + st * 32, 16, 1024),
+                                 sdesc(vv + st * 2048, 1024, 1024), id4, st > 0);
+                }
                 mma_commit(&bar[B_PMMA]);
             }
             pending = true;
             if (!mma_done()) break;
-            if (wt == 0) mbar_arrive(&bar[B_VEMPTY]);
+            if (!REV && wt == 0) mbar_arrive(&bar[B_VEMPTY]);
             if (SAVE && trow < 64) {
-                const size_t ci = ((size_t)b * H + h) * N + m;
+                const size_t ci = ((size_t)b * H + h) * N + mc;
                 float rv[64];
                 tmem_row64(tl + TM_D0 + bb * 64, rv);
                 float4 *du = reinterpret_cast<float4 *>(a.Ut + (ci * C + trow) * DV + j0);
@@ -481,6 +520,80 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         fence_proxy_async();
         wsync();
+        if (REV) {
+            // ---------------- reverse chain: S holds dS of the state leaving chunk mc ----------------
+            for (int m = 0; m < N; ++m) {
+                const int mc = N - 1 - m, bb = m & 1;
+                mbar_wait(&bar[B_READY0 + bb], (m >> 1) & 1, abort_flag);
+                mbar_wait(&bar[B_VFULL], m & 1, abort_flag);
+                if (wabort()) break;
+                {
+                    float4 *dst = reinterpret_cast<float4 *>(a.dSn + ((((size_t)b * H + h) * N + mc) * DK + trow) * DV + j0);
+#pragma unroll
+                    for (int j4 = 0; j4 < DVB / 4; ++j4)
+                        dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
+                }
+                // G = (-W)^T Kbar  and  D = A_chain^T [du ; dO]
+                if (wc == 0) {
+                    fence_after_sync();
+                    const uint32_t ac = smem_u32(sm + OFF_AC), kc = smem_u32(sm + OFF_KC + bb * 16384);
+                    const uint32_t dub = smem_u32(sm + OFF_V), dob = smem_u32(sm + OFF_U);
+                    const uint32_t idg = idesc_bf16(128, 128, 1, 1), idd = idesc_bf16(128, 64, 1, 1);
+#pragma unroll
+                    for (int st = 0; st < 4; ++st)
+                        mma_bf16(tbase + TM_G, sdesc(ac + st * 2048, 16384, 1024), sdesc(kc + st * 2048, 8192, 1024), idg,
+                                 st > 0);
+                    const int st0 = a.has_du ? 0 : 4;
+                    for (int st = st0; st < 8; ++st) {
+                        const uint32_t bsrc = st < 4 ? dub + st * 2048 : dob + (st - 4) * 2048;
+                        mma_bf16(tbase + TM_D0 + bb * 64, sdesc(ac + st * 2048, 16384, 1024), sdesc(bsrc, 1024, 1024),
+                                 idd, st > st0);
+                    }
+                    mma_commit(&bar[B_CMMA]);
+                }
+                pending = true;
+                if (!mma_done()) break;
+                if (wc == 0) mbar_arrive(&bar[B_VEMPTY]);
+                // M' = G -> bf16, K-major A operand in the A_chain region (A_chain is consumed)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float gv[64];
+                    tmem_row64(tl + TM_G + hh * 64, gv);
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_AC, (uint32_t)hh * 16384 + swz(trow, ch), gv + ch * 8);
+                }
+                fence_proxy_async();
+                fence_before_sync();
+                wsync();
+                // D += M' dS+
+                if (wc == 0) {
+                    fence_after_sync();
+                    const uint32_t ac = smem_u32(sm + OFF_AC), ss = smem_u32(sm + OFF_S);
+                    const uint32_t id = idesc_bf16(128, 64, 0, 1);
+#pragma unroll
+                    for (int st = 0; st < 8; ++st)
+                        mma_bf16(tbase + TM_D0 + bb * 64, sdesc(ac + (st >> 2) * 16384 + (st & 3) * 32, 16, 1024),
+                                 sdesc(ss + st * 2048, 1024, 1024), id, 1);
+                    mma_commit(&bar[B_CMMA]);
+                }
+                pending = true;
+                if (!mma_done()) break;
+                if (wc == 0) mbar_arrive(&bar[B_ACFREE]);
+                {
+                    float dv[64];
+                    tmem_row64(tl + TM_D0 + bb * 64, dv);
+                    const float gmc = cf[bb * 80 + 64];
+#pragma unroll
+                    for (int j = 0; j < DVB; ++j) S[j] = gmc * S[j] + dv[j];
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_S, swz(trow, ch), S + ch * 8);
+                }
+                fence_proxy_async();
+                fence_before_sync();
+                wsync();
+                if (wc == 0) mbar_arrive(&bar[B_KCFREE0 + bb]);
+            }
+        } else
         for (int m = 0; m < N; ++m) {
             const int bb = m & 1, t0 = m * C;
             const int L = min(C, T - t0);
@@ -562,7 +675,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (wc == 0) mbar_arrive(&bar[B_KCFREE0 + bb]);
         }
         if (*abort_flag == 0) {
-            if (!SAVE && a.ST) {
+            if (MODE != 1 && a.ST) {
                 float *dst = a.ST + (((size_t)b * H + h) * DK + trow) * DV + j0;
 #pragma unroll
                 for (int j = 0; j < DVB; j += 4)
@@ -581,48 +694,61 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 }  // namespace tcf2
 
-template <int VAR, int SAVE>
-static cudaError_t launch_tc2(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const tcf2::Args &a,
-                              dim3 grid, size_t smem, cudaStream_t s, Rec &rec) {
-    cudaError_t e = cudaFuncSetAttribute(tcf2::k_fwd_tc2<VAR, SAVE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <int VAR, int MODE>
+static cudaError_t launch_tc2(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                              const CUtensorMap &mx, const tcf2::Args &a, dim3 grid, size_t smem, cudaStream_t s,
+                              Rec &rec) {
+    cudaError_t e = cudaFuncSetAttribute(tcf2::k_fwd_tc2<VAR, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     rec.mark(s);
-    tcf2::k_fwd_tc2<VAR, SAVE><<<grid, tcf2::NTHREADS, smem, s>>>(mq, mk, mv, a);
-    e = cudaGetLastError();
-    rec.mark(s);
-    return e;
+    tcf2::k_fwd_tc2<VAR, MODE><<<grid, tcf2::NTHREADS, smem, s>>>(mq, mk, mv, mx, a);
+    return cudaGetLastError();
 }
 
-static cudaError_t tc2_common(const Geo &g, const Tensors &t, const SimtWs *w, cudaStream_t s, Rec &rec) {
+static cudaError_t tc2_common(const Geo &g, const Tensors &t, const SimtWs *w, int mode, cudaStream_t s, Rec &rec) {
     using namespace tcf2;
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mx;
     const uint64_t Bn = g.B, T = g.T, H = g.H;
-    const bool ok = tc::make_map_4d_bf16(&mq, t.q, DK, H, T, Bn, 64) &&
-                    tc::make_map_4d_bf16(&mk, t.k, DK, H, T, Bn, 64) &&
-                    tc::make_map_4d_bf16(&mv, t.v, g.dv, H, T, Bn, 64);
+    const void *vsrc = mode == 2 ? t.dout : t.v;
+    bool ok = tc::make_map_4d_bf16(&mq, t.q, DK, H, T, Bn, 64) && tc::make_map_4d_bf16(&mk, t.k, DK, H, T, Bn, 64) &&
+              tc::make_map_4d_bf16(&mv, vsrc, g.dv, H, T, Bn, 64);
+    if (ok && mode == 2 && t.du) ok = tc::make_map_4d_bf16(&mx, t.du, g.dv, H, T, Bn, 64);
+    else mx = mv;
     if (!ok) return cudaErrorInvalidValue;
     Args a = {};
-    a.alpha = t.alpha; a.beta = t.beta; a.S0 = t.S0; a.out = t.out; a.u = t.u; a.ST = t.S_T;
-    a.B = g.B; a.T = g.T; a.H = g.H; a.dv = g.dv; a.N = g.N;
-    if (w) {
+    a.alpha = t.alpha; a.beta = t.beta; a.B = g.B; a.T = g.T; a.H = g.H; a.dv = g.dv; a.N = g.N;
+    if (mode == 2) {
+        a.S0 = t.dS_T; a.ST = t.dS0; a.dSn = w->dSn; a.has_du = t.du != nullptr;
+    } else {
+        a.S0 = t.S0; a.out = t.out; a.u = t.u; a.ST = t.S_T;
+    }
+    if (mode == 1) {
         a.W = w->W; a.Ut = w->Ut; a.G = w->G; a.P = w->P; a.Sn = w->Sn; a.Un = w->Un;
     }
     const dim3 grid(g.dv / DVB, g.H, g.B);
     const size_t smem = SMEM_BYTES + 1024;
-    if (g.variant == VAR_GATED)
-        return w ? launch_tc2<VAR_GATED, 1>(mq, mk, mv, a, grid, smem, s, rec)
-                 : launch_tc2<VAR_GATED, 0>(mq, mk, mv, a, grid, smem, s, rec);
-    return w ? launch_tc2<VAR_DELTANET, 1>(mq, mk, mv, a, grid, smem, s, rec)
-             : launch_tc2<VAR_DELTANET, 0>(mq, mk, mv, a, grid, smem, s, rec);
+    if (g.variant == VAR_GATED) {
+        if (mode == 0) return launch_tc2<VAR_GATED, 0>(mq, mk, mv, mx, a, grid, smem, s, rec);
+        if (mode == 1) return launch_tc2<VAR_GATED, 1>(mq, mk, mv, mx, a, grid, smem, s, rec);
+        return launch_tc2<VAR_GATED, 2>(mq, mk, mv, mx, a, grid, smem, s, rec);
+    }
+    if (mode == 0) return launch_tc2<VAR_DELTANET, 0>(mq, mk, mv, mx, a, grid, smem, s, rec);
+    if (mode == 1) return launch_tc2<VAR_DELTANET, 1>(mq, mk, mv, mx, a, grid, smem, s, rec);
+    return launch_tc2<VAR_DELTANET, 2>(mq, mk, mv, mx, a, grid, smem, s, rec);
 }
 
 // Warp-specialised forward (Gated DeltaNet / DeltaNet).
-cudaError_t tc_fwd2(const Geo &g, const Tensors &t, cudaStream_t s, Rec &rec) { return tc2_common(g, t, nullptr, s, rec); }
+cudaError_t tc_fwd2(const Geo &g, const Tensors &t, cudaStream_t s, Rec &rec) { return tc2_common(g, t, nullptr, 0, s, rec); }
 
-// The same kernel in recompute mode: fills W, U~, g, P, S_n, U of the CUDA-core backward workspace.
+// The same kernel in recompute mode: fills W, U~, g, P, S_n, U of the backward workspace.
 cudaError_t tc_bwd_recompute(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec) {
-    return tc2_common(g, t, &w, s, rec);
+    return tc2_common(g, t, &w, 1, s, rec);
+}
+
+// The same kernel in reverse mode: fills dS_{n+1} of every chunk and writes dS0.
+cudaError_t tc_bwd_reverse(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec) {
+    return tc2_common(g, t, &w, 2, s, rec);
 }
 
 }  // namespace dr
