@@ -126,8 +126,7 @@ static int bwd_impl(const void *q, const void *k, const void *v, const void *alp
     if (tc_bwd_recompute_supported(g, dtype == DR_BF16)) {
         rc = launch_status(tc_bwd_recompute(g, t, w, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_bwd_reverse(g, t, w, s, rec));
-        if (rc == DR_OK) rc = launch_status(tc_bwd_state(g, t, w, s, rec));
-        if (rc == DR_OK) rc = launch_status(simt_bwd(g, t, true, w, s, rec, true, true));
+        if (rc == DR_OK) rc = launch_status(tc_bwd_chunk(g, t, w, s, rec));
     } else {
         rc = launch_status(simt_bwd(g, t, dtype == DR_BF16, w, s, rec));
     }
@@ -146,7 +145,7 @@ static int launch_plan(const Geo &g, int dtype, bool bwd, const char **names, in
     }
     if (bwd && tc_bwd_recompute_supported(g, dtype == DR_BF16)) {
         src = TC_BWD_KERNELS;
-        n = 4;
+        n = 3;
     } else {
         src = bwd ? SIMT_BWD_KERNELS : SIMT_FWD_KERNELS;
         n = bwd ? 5 : 3;

@@ -583,6 +583,7 @@ size_t simt_ws_bytes(const Geo &g, bool bwd) {
         s += al256(nc * C * DV * 4);      // dUn
         s += 3 * al256(nc * C * DK * 4);  // Qd dWm Tm
         s += al256(nc * DK * 4);          // RS
+        s += 2 * al256(nc * C * C * 4);   // Tn KK
     }
     return s;
 }
@@ -605,6 +606,8 @@ SimtWs simt_ws_carve(const Geo &g, bool bwd, void *base) {
         w.dWm = take(nc * C * DK * 4);
         w.Tm = take(nc * C * DK * 4);
         w.RS = take(nc * DK * 4);
+        w.Tn = take(nc * C * C * 4);
+        w.KK = take(nc * C * C * 4);
     }
     return w;
 }
@@ -621,7 +624,7 @@ template <typename K> static cudaError_t prep_attr(K kern, size_t smem) {
 
 const char *const SIMT_FWD_KERNELS[3] = {"k_prep", "k_scan", "k_out"};
 const char *const SIMT_BWD_KERNELS[5] = {"k_prep", "k_scan", "k_scan_bwd", "k_bwd_state", "k_bwd_intra"};
-const char *const TC_BWD_KERNELS[4] = {"k_fwd_tc2(recompute)", "k_fwd_tc2(reverse)", "k_bwd_state_tc", "k_bwd_intra"};
+const char *const TC_BWD_KERNELS[3] = {"k_fwd_tc2(recompute)", "k_fwd_tc2(reverse)", "k_bwd_chunk_tc"};
 
 template <typename TI>
 static cudaError_t forward_chain(const Geo &g, const IO<TI> &io, const SimtWs &w, const float *S0, float *ST,

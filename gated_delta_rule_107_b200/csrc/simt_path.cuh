@@ -19,6 +19,8 @@ struct SimtWs {
     float *dWm;  // [B,H,N,C,dk]  -dU S^T   (= dL/dW)
     float *Tm;   // [B,H,N,C,dk]  U dS+^T
     float *RS;   // [B,H,N,dk]    rowsum(S .* dS+)
+    float *Tn;   // [B,H,N,C,C]   T = (I+A)^-1          (tensor-core backward only)
+    float *KK;   // [B,H,N,C,C]   k k^T, no gate factor (tensor-core backward only)
 };
 
 size_t simt_ws_bytes(const Geo &g, bool bwd);
@@ -32,6 +34,6 @@ cudaError_t simt_bwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w,
 // kernel names in launch order (for the timed entry points)
 extern const char *const SIMT_FWD_KERNELS[3];
 extern const char *const SIMT_BWD_KERNELS[5];
-extern const char *const TC_BWD_KERNELS[4];
+extern const char *const TC_BWD_KERNELS[3];
 
 }  // namespace dr

@@ -81,7 +81,7 @@ struct Args {
     float *ST;
     int B, T, H, dv, N;
     // recompute mode (backward): fp32 chunk products for the CUDA-core backward kernels
-    float *W, *Ut, *G, *P, *Sn, *Un;
+    float *W, *Ut, *G, *P, *Sn, *Un, *Tn, *KK;
     // reverse mode: dL/dS of the state leaving each chunk; whether du is given
     float *dSn;
     int has_du;
@@ -331,6 +331,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                     for (int i = 0; i < 64; ++i) f[i] = __expf(gr - gc[i]);
                 }
+                if (SAVE && arow && half == 0) {
+                    float4 *dst = reinterpret_cast<float4 *>(a.KK + ((((size_t)b * H + h) * N + mc) * C + r) * C);
+#pragma unroll
+                    for (int i4 = 0; i4 < 16; ++i4)
+                        dst[i4] = make_float4(g1[4 * i4], g1[4 * i4 + 1], g1[4 * i4 + 2], g1[4 * i4 + 3]);
+                }
                 if (arow) {
                     const float br = pf[PF_BV * 64 + r];
 #pragma unroll
@@ -374,6 +380,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                         for (int e = 0; e < 8; ++e) w[e] = (ch * 8 + e <= i) ? w[e] : 0.f;
                         st_chunk(sm + OFF_TT, swz(i, ch), w);
+                        if (SAVE && half == 0) {
+                            float4 *dst = reinterpret_cast<float4 *>(
+                                a.Tn + ((((size_t)b * H + h) * N + mc) * C + i) * C + ch * 8);
+                            dst[0] = make_float4(w[0], w[1], w[2], w[3]);
+                            dst[1] = make_float4(w[4], w[5], w[6], w[7]);
+                        }
                     }
                 }
                 fence_proxy_async();
@@ -725,6 +737,7 @@ static cudaError_t tc2_common(const Geo &g, const Tensors &t, const SimtWs *w, i
     }
     if (mode == 1) {
         a.W = w->W; a.Ut = w->Ut; a.G = w->G; a.P = w->P; a.Sn = w->Sn; a.Un = w->Un;
+        a.Tn = w->Tn; a.KK = w->KK;
     }
     const dim3 grid(g.dv / DVB, g.H, g.B);
     const size_t smem = SMEM_BYTES + 1024;

@@ -14,8 +14,8 @@ cudaError_t tc_fwd2(const Geo &g, const Tensors &t, cudaStream_t s, Rec &rec);
 struct SimtWs;
 bool tc_bwd_recompute_supported(const Geo &g, bool bf16);
 cudaError_t tc_bwd_recompute(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec);
-// Per-chunk products with S and dS+ on tensor cores: dU, Qd, dWm, Tm, RS (tc_bwd.cu).
-cudaError_t tc_bwd_state(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec);
+// All intra-chunk gradients on tensor cores (tc_bwd.cu): dq, dk, dv, dbeta, d log alpha.
+cudaError_t tc_bwd_chunk(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec);
 // Reverse state chain on tensor cores: dS_{n+1} of every chunk into w.dSn, and dS0.
 cudaError_t tc_bwd_reverse(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec);
 // number of launches of tc_fwd and their names
