@@ -41,6 +41,7 @@ bool use_tc_fwd(const Geo &g, int dtype) { return tc_fwd_supported(g, dtype == D
 size_t ws_bytes(const Geo &g, int dtype, bool bwd) {
     if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
     if (!bwd && use_tc_fwd(g, dtype)) return tc_fwd_ws_bytes(g);
+    if (bwd && tc_bwd_recompute_supported(g, dtype == DR_BF16)) return tc_bwd_ws_bytes(g);
     return simt_ws_bytes(g, bwd);
 }
 
@@ -122,12 +123,13 @@ static int bwd_impl(const void *q, const void *k, const void *v, const void *alp
     t.q = q; t.k = k; t.v = v; t.alpha = alpha; t.beta = beta; t.S0 = S0;
     t.dout = dout; t.du = du; t.dS_T = dS_T;
     t.dq = dq; t.dk = dk_; t.dv = dv_; t.dalpha = dalpha; t.dbeta = dbeta; t.dS0 = dS0;
-    const SimtWs w = simt_ws_carve(g, true, workspace);
     if (tc_bwd_recompute_supported(g, dtype == DR_BF16)) {
+        const TcBwdWs w = tc_bwd_ws_carve(g, workspace);
         rc = launch_status(tc_bwd_recompute(g, t, w, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_bwd_reverse(g, t, w, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_bwd_chunk(g, t, w, s, rec));
     } else {
+        const SimtWs w = simt_ws_carve(g, true, workspace);
         rc = launch_status(simt_bwd(g, t, dtype == DR_BF16, w, s, rec));
     }
     rec.mark(s);  // end of the last launch

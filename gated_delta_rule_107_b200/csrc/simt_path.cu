@@ -583,7 +583,6 @@ size_t simt_ws_bytes(const Geo &g, bool bwd) {
         s += al256(nc * C * DV * 4);      // dUn
         s += 3 * al256(nc * C * DK * 4);  // Qd dWm Tm
         s += al256(nc * DK * 4);          // RS
-        s += 2 * al256(nc * C * C * 4);   // Tn KK
     }
     return s;
 }
@@ -606,8 +605,6 @@ SimtWs simt_ws_carve(const Geo &g, bool bwd, void *base) {
         w.dWm = take(nc * C * DK * 4);
         w.Tm = take(nc * C * DK * 4);
         w.RS = take(nc * DK * 4);
-        w.Tn = take(nc * C * C * 4);
-        w.KK = take(nc * C * C * 4);
     }
     return w;
 }
@@ -656,8 +653,7 @@ static cudaError_t fwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaSt
 }
 
 template <typename TI>
-static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec,
-                         bool recomputed, bool only_intra) {
+static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec) {
     const IO<TI> io = io_of<TI>(t);
     const size_t C = g.C, DK = g.dk, DV = g.dv;
     const dim3 gc(g.N, g.H, g.B), gs(g.dv / JB, g.H, g.B);
@@ -667,15 +663,13 @@ static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaSt
     DR_TRY(prep_attr(k_scan_bwd<TI>, sm_sb));
     DR_TRY(prep_attr(k_bwd_state<TI>, sm_st));
     DR_TRY(prep_attr(k_bwd_intra<TI>, sm_in));
-    if (!only_intra) {
-        if (!recomputed) DR_TRY(forward_chain<TI>(g, io, w, t.S0, nullptr, 0, s, rec));
-        rec.mark(s);
-        k_scan_bwd<TI><<<gs, NT, sm_sb, s>>>(g, io, w, t.dS_T, t.dS0);
-        DR_TRY(cudaGetLastError());
-        rec.mark(s);
-        k_bwd_state<TI><<<gc, NT, sm_st, s>>>(g, io, w);
-        DR_TRY(cudaGetLastError());
-    }
+    DR_TRY(forward_chain<TI>(g, io, w, t.S0, nullptr, 0, s, rec));
+    rec.mark(s);
+    k_scan_bwd<TI><<<gs, NT, sm_sb, s>>>(g, io, w, t.dS_T, t.dS0);
+    DR_TRY(cudaGetLastError());
+    rec.mark(s);
+    k_bwd_state<TI><<<gc, NT, sm_st, s>>>(g, io, w);
+    DR_TRY(cudaGetLastError());
     rec.mark(s);
     k_bwd_intra<TI><<<gc, NT, sm_in, s>>>(g, io, w);
     return cudaGetLastError();
@@ -685,10 +679,8 @@ cudaError_t simt_fwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w,
     return bf16 ? fwd_t<__nv_bfloat16>(g, t, w, s, rec) : fwd_t<float>(g, t, w, s, rec);
 }
 
-cudaError_t simt_bwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec,
-                     bool recomputed, bool only_intra) {
-    return bf16 ? bwd_t<__nv_bfloat16>(g, t, w, s, rec, recomputed, only_intra)
-                : bwd_t<float>(g, t, w, s, rec, recomputed, only_intra);
+cudaError_t simt_bwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec) {
+    return bf16 ? bwd_t<__nv_bfloat16>(g, t, w, s, rec) : bwd_t<float>(g, t, w, s, rec);
 }
 
 }  // namespace dr

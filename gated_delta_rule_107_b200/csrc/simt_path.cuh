@@ -19,18 +19,12 @@ struct SimtWs {
     float *dWm;  // [B,H,N,C,dk]  -dU S^T   (= dL/dW)
     float *Tm;   // [B,H,N,C,dk]  U dS+^T
     float *RS;   // [B,H,N,dk]    rowsum(S .* dS+)
-    float *Tn;   // [B,H,N,C,C]   T = (I+A)^-1          (tensor-core backward only)
-    float *KK;   // [B,H,N,C,C]   k k^T, no gate factor (tensor-core backward only)
 };
 
 size_t simt_ws_bytes(const Geo &g, bool bwd);
 SimtWs simt_ws_carve(const Geo &g, bool bwd, void *base);
 cudaError_t simt_fwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec);
-// recomputed = true: W, U~, G, P, S_n, U are already in the workspace (tensor-core recompute);
-// only_intra = true: dS_{n+1}, dU, Qd, dWm, Tm, RS are too (tensor-core reverse chain and
-// state products) and only the intra-chunk gradient kernel runs.
-cudaError_t simt_bwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec,
-                     bool recomputed = false, bool only_intra = false);
+cudaError_t simt_bwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec);
 // kernel names in launch order (for the timed entry points)
 extern const char *const SIMT_FWD_KERNELS[3];
 extern const char *const SIMT_BWD_KERNELS[5];

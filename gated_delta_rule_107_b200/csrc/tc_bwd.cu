@@ -22,9 +22,18 @@
 //
 // The dense products run channel-major so that M = 128 (dk or dv) fills the MMA; the two
 // token x token products (dP, dA) use M = 128 MMAs whose rows 64..127 read other (valid)
-// shared memory and are discarded.  One CTA of 128 threads per chunk; thread t owns TMEM
-// lane t.
-#include "simt_path.cuh"
+// shared memory and are discarded.  D_M + D_M^T needs no transpose: the same D_M tile is
+// read once as an MN-major and once as a K-major B operand.
+//
+// One CTA of 256 threads per chunk.  Every operand tile arrives by TMA in two groups: what
+// the first products read (S, dS+, U, dO, k, P, T, KK, du), then -- once those products
+// have consumed their inputs -- W, U~, q, k, v into the space they freed.  dq, dk and dv
+// leave through shared-memory staging tiles and TMA stores.  Warps w and w + 4 read the
+// same 32 TMEM lanes (channel rows) and split the 64 token columns; sums over channels
+// are butterfly transposes inside a warp plus four partials in shared memory.
+#include <limits.h>
+
+#include "tc_host.cuh"
 #include "tc_path.cuh"
 #include "tc_ptx.cuh"
 #include "tc_tile.cuh"
@@ -33,78 +42,93 @@ namespace dr {
 namespace tcb {
 
 using namespace dr::tc;
+using dr::tcf::ld_chunk;
 using dr::tcf::st_chunk;
-using dr::tcf::tmem_row64;
+using dr::tcf::tok_off;
 
 constexpr int C = 64, DK = 128, DV = 128;
-constexpr int NTHREADS = 128;
+constexpr int NTHREADS = 256;
 // shared memory (bytes from a 1024-aligned base); later phases reuse earlier regions
-constexpr uint32_t R_S = 0;           // 32K  S [c][j]           -> dB_k^T [c][i] (16K) | dB_v^T [j][i] (16K)
-constexpr uint32_t R_DS = 32768;      // 32K  dS+ [c][j]         -> W [i][c] (16K) | U~ [i][j] (16K)
-constexpr uint32_t R_U = 65536;       // 16K  U [r][j]           -> q [r][c]
-constexpr uint32_t R_DO = 81920;      // 16K  dO [r][j]          -> k [r][c]
-constexpr uint32_t R_KB = 98304;      // 16K  Kbar [r][c]
-constexpr uint32_t R_P = 114688;      //  8K  P [r'][r] (row-major) -> D_P [r][i]
-constexpr uint32_t R_T = 122880;      //  8K  T [r][i]           -> D_M + D_M^T [r][i]
-constexpr uint32_t R_DUT = 131072;    // 16K  dU^T [j][r]
-constexpr uint32_t R_DWT = 147456;    // 16K  dW^T [c][r]
-constexpr uint32_t R_F = 163840;      // 49K  fp32 64 x 65 scratch x 3: Pf, dPf, Zf
-constexpr uint32_t R_MISC = R_F + 50176;
+constexpr uint32_t R_S = 0;          // 32K  S [c][j]     -> dB_k^T [c][i] (16K) | dB_v^T [j][i] (16K)
+constexpr uint32_t R_DS = 32768;     // 32K  dS+ [c][j]   -> W [i][c] | U~ [i][j]  -> dk staging [r][c]
+constexpr uint32_t R_U = 65536;      // 16K  U [r][j]     -> q [r][c]
+constexpr uint32_t R_DO = 81920;     // 16K  dO [r][j]    -> k [r][c]
+constexpr uint32_t R_KB = 98304;     // 16K  Kbar [r][c]  -> v [r][j]
+constexpr uint32_t R_P = 114688;     //  8K  P [r][i]     -> D_P [r][i]
+constexpr uint32_t R_T = 122880;     //  8K  T [r][i]     -> D_M [r][i]
+constexpr uint32_t R_KK = 131072;    //  8K  KK [r][i]
+constexpr uint32_t R_DU = 139264;    // 16K  du [r][j]
+constexpr uint32_t R_DUT = 155648;   // 16K  dU^T [j][r]  -> dv staging [i][j]
+constexpr uint32_t R_DWT = 172032;   // 16K  dW^T [c][r]  -> dq staging [r][c]
+constexpr uint32_t R_MISC = 188416;  //  8K
 constexpr uint32_t SMEM_BYTES = R_MISC + 8192;
+// bytes of the two TMA load groups
+constexpr uint32_t LOAD1_BYTES = 2 * 32768 + 3 * 16384 + 3 * 8192;  // + du (16K) when given
+constexpr uint32_t LOAD2_BYTES = 5 * 16384;
 // misc (floats unless noted)
-constexpr uint32_t M_BAR = 0, M_TMEM = 64, M_ABORT = 68;
-constexpr uint32_t M_GC = 256, M_BETA = 512, M_EG = 768, M_EGC = 1024;   // [64] each
-constexpr uint32_t M_RED = 1280;     // [3 kinds][4 warps][64]: q.Qd, k.dBk, k.Tm partial sums
-constexpr uint32_t M_RDB = M_RED + 3 * 4 * 64 * 4;  // [2][4][64]: v.dBv, k.dBk (for dbeta)
-constexpr uint32_t M_RS = M_RDB + 2 * 4 * 64 * 4;   // [4]: partial sums of S .* dS+
-constexpr uint32_t M_DG = M_RS + 64;                // [64] dg
-static_assert(M_DG + 256 <= 8192, "misc overflow");
-static_assert(3 * 64 * 65 * 4 <= 50176, "fp32 scratch overflow");
+constexpr uint32_t M_BAR = 0;  // [0] MMA batches, [1] first load group, [2] second load group
+constexpr uint32_t M_TMEM = 64, M_ABORT = 68;
+constexpr uint32_t M_GC = 256, M_BETA = 512, M_EG = 768, M_EGC = 1024;  // [64] each
+constexpr uint32_t M_RED = 1280;                    // [5 kinds][4 lane quarters][64 tokens]
+constexpr uint32_t M_ROW = M_RED + 5 * 4 * 64 * 4;  // [2 column halves][64] rowsum Z, then [2][64] dbeta (A part)
+constexpr uint32_t M_RS = M_ROW + 4 * 64 * 4;       // [8 warps] partial sums of S .* dS+
+constexpr uint32_t M_DG = M_RS + 64;                // [64] dg, then [64] the k . Tm sums
+static_assert(M_DG + 512 <= 8192, "misc overflow");
+enum { RK_QQD = 0, RK_KBK, RK_KTM, RK_VBV, RK_ZC };
 // TMEM columns
 constexpr uint32_t TM_DUT = 0, TM_QD = 64, TM_TM = 128, TM_DP = 192, TM_DW = 256, TM_DBK = 320, TM_DQ = 384,
                    TM_DK = 448, TM_COLS = 512;
-// fp32 scratch (row stride 65 floats)
-constexpr int LD = 65;
 
-struct Args {
-    const void *q, *k, *v, *alpha, *beta, *dout, *du;  // bf16
-    void *dq, *dk, *dv, *dalpha, *dbeta;                // bf16
-    SimtWs w;
-    int B, T, H, N, variant;
+struct Maps {
+    CUtensorMap q, k, v, dout, du, dq, dk, dv;  // [B, T, H, 128] bf16; box 64 channels x 64 tokens
+    CUtensorMap S, dS;                          // [chunks * 128][128] bf16; box 64 x 128
+    CUtensorMap U, W, Ut;                       // [chunks * 64][128] bf16; box 64 x 64
+    CUtensorMap P, T, KK;                       // [chunks * 64][64] bf16; box 64 x 64
 };
 
-__device__ __forceinline__ void ld8f(const float *p, float *v) {
-    const float4 a = reinterpret_cast<const float4 *>(p)[0], b = reinterpret_cast<const float4 *>(p)[1];
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-
-__device__ __forceinline__ void ld8h(const void *p, float *v) {
-    const uint4 w = *reinterpret_cast<const uint4 *>(p);
-    v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
-    v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
-}
-
-__device__ __forceinline__ float bfv(const void *p, size_t i) {
-    return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
-}
+struct Args {
+    const void *beta;        // bf16 [B, T, H]
+    void *dalpha, *dbeta;    // bf16 [B, T, H]
+    const float *g;          // [chunks][64]
+    int B, T, H, N, variant, has_du;
+};
 
 __device__ __forceinline__ void st_bf(void *p, size_t i, float x) {
     reinterpret_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(x);
 }
-
-// sum over the 128 threads of per-thread values x[r] (r = 0..63), via warp shuffles and
-// red[4][64]; the result for row r is available in red[0][r] + ... + red[3][r] after a sync.
-__device__ __forceinline__ void warp_partial_rows(const float *x, float *red, int warp, int lane) {
-#pragma unroll 4
-    for (int r = 0; r < C; ++r) {
-        float v = x[r];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) red[warp * C + r] = v;
-    }
+__device__ __forceinline__ float ld_tile(const unsigned char *base, int r, int c) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(base + tok_off(r, c)));
+}
+__device__ __forceinline__ void st_tile(unsigned char *base, int r, int c, float x) {
+    *reinterpret_cast<__nv_bfloat16 *>(base + tok_off(r, c)) = __float2bfloat16_rn(x);
 }
 
-__global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(Args a) {
+// 32 fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_row32(uint32_t taddr, float *v) {
+    tmem_ld16(taddr + 0, v);
+    tmem_ld16(taddr + 16, v + 16);
+    wait_ld();
+}
+
+// v[t] (t = 0..31) held by every lane of the warp; returns sum over the 32 lanes of v[lane].
+// Butterfly transpose: at each step a lane keeps half of its live values and adds the
+// partner's copy of that half (16 + 8 + 4 + 2 + 1 shuffles).
+__device__ __forceinline__ float warp_colsum32(float *v, int lane) {
+#pragma unroll
+    for (int s = 0; s < 5; ++s) {
+        const int m = 16 >> s;
+        const bool up = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < m; ++i) {
+            const float lo = v[i], hi = v[i + m];
+            const float send = up ? lo : hi;
+            v[i] = (up ? hi : lo) + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+    }
+    return v[0];
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(const __grid_constant__ Maps mp, Args a) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -116,112 +140,97 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(Args a) {
     float *eg = reinterpret_cast<float *>(sm + R_MISC + M_EG);
     float *egc = reinterpret_cast<float *>(sm + R_MISC + M_EGC);
     float *red = reinterpret_cast<float *>(sm + R_MISC + M_RED);
-    float *rdb = reinterpret_cast<float *>(sm + R_MISC + M_RDB);
+    float *rowsum = reinterpret_cast<float *>(sm + R_MISC + M_ROW);
     float *rsp = reinterpret_cast<float *>(sm + R_MISC + M_RS);
     float *dgs = reinterpret_cast<float *>(sm + R_MISC + M_DG);
-    float *Pf = reinterpret_cast<float *>(sm + R_F);
-    float *dPf = Pf + 64 * LD;
-    float *Zf = dPf + 64 * LD;
+    float *ktm = dgs + 64;
 
     const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, hf = warp >> 2;
+    const int lr = quarter * 32 + lane;  // TMEM lane: channel row of the channel-major products
+    const int col0 = hf * 32;            // first of this thread's 32 token columns
     const int T = a.T, H = a.H, t0 = n * C, L = min(C, T - t0);
-    const size_t ci = ((size_t)b * H + h) * a.N + n;
+    const int ci = (b * H + h) * a.N + n;  // < 2^31 / 128 (checked by the launcher)
     const bool gated = a.variant == VAR_GATED;
     auto trow_g = [&](int r) -> size_t { return ((size_t)b * T + t0 + r) * H + h; };  // token row (r < L)
+    auto red_at = [&](int kind, int q, int t) -> float & { return red[(kind * 4 + q) * 64 + t]; };
 
+    // issue state of thread 0 (the only thread that issues TMA and MMA)
+    int mma_issued = 0, loads_issued = 0;
     if (tid == 0) {
-        mbar_init(bar, 1);
+        for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
+        mbar_arrive_tx(&bar[1], LOAD1_BYTES + (a.has_du ? 16384u : 0u));
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            tma_load_2d(sm + R_S + p * 16384, &mp.S, 64 * p, ci * DK, &bar[1]);
+            tma_load_2d(sm + R_DS + p * 16384, &mp.dS, 64 * p, ci * DK, &bar[1]);
+            tma_load_2d(sm + R_U + p * 8192, &mp.U, 64 * p, ci * C, &bar[1]);
+            tma_load_4d(sm + R_DO + p * 8192, &mp.dout, 64 * p, h, t0, b, &bar[1]);
+            tma_load_4d(sm + R_KB + p * 8192, &mp.k, 64 * p, h, t0, b, &bar[1]);
+            if (a.has_du) tma_load_4d(sm + R_DU + p * 8192, &mp.du, 64 * p, h, t0, b, &bar[1]);
+        }
+        tma_load_2d(sm + R_P, &mp.P, 0, ci * C, &bar[1]);
+        tma_load_2d(sm + R_T, &mp.T, 0, ci * C, &bar[1]);
+        tma_load_2d(sm + R_KK, &mp.KK, 0, ci * C, &bar[1]);
+        loads_issued = 1;
     }
     if (warp == 0) tmem_alloc(tmem_slot, TM_COLS);
-
-    // ---------------- phase 0: factors and bf16 operand tiles ----------------
-    const float *Gg = a.w.G + ci * C * DK;
     if (tid < C) {
-        const int r = tid;
-        const float x = Gg[(size_t)r * DK];
-        gc[r] = x;
-        betas[r] = (r < L) ? bfv(a.beta, trow_g(r)) : 0.f;
-        eg[r] = __expf(x);
-        egc[r] = __expf(Gg[(size_t)(C - 1) * DK] - x);
+        const float x = a.g[(size_t)ci * C + tid];
+        gc[tid] = x;
+        betas[tid] = (tid < L) ? tcf::bf(a.beta, trow_g(tid)) : 0.f;
+        eg[tid] = __expf(x);
+        egc[tid] = __expf(a.g[(size_t)ci * C + C - 1] - x);
     }
-    if (tid < 4) rsp[tid] = 0.f;
-    __syncthreads();
-    const float *Sg = a.w.Sn + ci * DK * DV, *dSg = a.w.dSn + ci * DK * DV;
-    float rs_part = 0.f;
-    for (int x = tid; x < DK * 16; x += NTHREADS) {  // S, dS+ : 128 rows x 16 chunks of 8
-        const int r = x >> 4, c16 = x & 15, p = c16 >> 3, ch = c16 & 7;
-        float v[8], w[8];
-        ld8f(Sg + (size_t)r * DV + c16 * 8, v);
-        ld8f(dSg + (size_t)r * DV + c16 * 8, w);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) rs_part += v[e] * w[e];
-        st_chunk(sm + R_S, (uint32_t)p * 16384 + swz(r, ch), v);
-        st_chunk(sm + R_DS, (uint32_t)p * 16384 + swz(r, ch), w);
-    }
-    const float *Ug = a.w.Un + ci * C * DV;
-    for (int x = tid; x < C * 16; x += NTHREADS) {  // U, dO, Kbar : 64 rows x 16 chunks
-        const int r = x >> 4, c16 = x & 15, p = c16 >> 3, ch = c16 & 7;
-        const uint32_t o = (uint32_t)p * 8192 + swz(r, ch);
-        float v[8];
-        ld8f(Ug + (size_t)r * DV + c16 * 8, v);
-        st_chunk(sm + R_U, o, v);
-        if (r < L) ld8h(reinterpret_cast<const __nv_bfloat16 *>(a.dout) + trow_g(r) * DV + c16 * 8, v);
-        else
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = 0.f;
-        st_chunk(sm + R_DO, o, v);
-        if (r < L) {
-            ld8h(reinterpret_cast<const __nv_bfloat16 *>(a.k) + trow_g(r) * DK + c16 * 8, v);
-            const float f = egc[r];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] *= f;
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = 0.f;
-        }
-        st_chunk(sm + R_KB, o, v);
-    }
-    const float *Pg = a.w.P + ci * C * C, *Tg = a.w.Tn + ci * C * C;
-    for (int x = tid; x < C * 8; x += NTHREADS) {  // P, T : 64 rows x 8 chunks
-        const int r = x >> 3, ch = x & 7;
-        float v[8];
-        ld8f(Pg + (size_t)r * C + ch * 8, v);
-        st_chunk(sm + R_P, swz(r, ch), v);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) Pf[r * LD + ch * 8 + e] = v[e];
-        ld8f(Tg + (size_t)r * C + ch * 8, v);
-        st_chunk(sm + R_T, swz(r, ch), v);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) rs_part += __shfl_xor_sync(0xffffffffu, rs_part, o);
-    if (lane == 0) rsp[warp] = rs_part;
-    fence_proxy_async();
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tbase = *tmem_slot;
-    const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);
-    uint32_t phase = 0;
-    bool ok = true;
-    auto mma_round = [&]() {
-        mma_commit(bar);
-        return;
-    };
+    const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16) + (uint32_t)col0;
+    uint32_t ph = 0;
+    auto consensus = [&](bool ok) -> bool { return !named_sync_any(1, NTHREADS, !ok || *abort_flag != 0); };
     auto wait_mma = [&]() -> bool {
-        mbar_wait(bar, phase & 1, abort_flag);
-        phase++;
+        const bool ok = mbar_wait(&bar[0], ph & 1, abort_flag);
+        ph++;
         fence_after_sync();
-        return !named_sync_any(1, NTHREADS, *abort_flag != 0);
+        return consensus(ok);
     };
     const uint32_t sS = smem_u32(sm + R_S), sD = smem_u32(sm + R_DS), sU = smem_u32(sm + R_U);
     const uint32_t sO = smem_u32(sm + R_DO), sK = smem_u32(sm + R_KB), sP = smem_u32(sm + R_P);
     const uint32_t sT = smem_u32(sm + R_T), sUT = smem_u32(sm + R_DUT), sWT = smem_u32(sm + R_DWT);
 
+    // ---------------- phase 0: Kbar = e^{g_C - g} k in place; sum of S .* dS+ ----------------
+    bool ok = mbar_wait(&bar[1], 0, abort_flag);
+    if (ok) {
+        for (int x = tid; x < 1024; x += NTHREADS) {  // 2 panels x 64 rows x 8 chunks of 16 B
+            float v[8];
+            ld_chunk(sm + R_KB, (uint32_t)x * 16, v);
+            const float f = egc[(x >> 3) & 63];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] *= f;
+            st_chunk(sm + R_KB, (uint32_t)x * 16, v);
+        }
+        float rs = 0.f;
+        for (int x = tid; x < 2048; x += NTHREADS) {  // S and dS+ share one layout
+            float v[8], w[8];
+            ld_chunk(sm + R_S, (uint32_t)x * 16, v);
+            ld_chunk(sm + R_DS, (uint32_t)x * 16, w);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) rs += v[e] * w[e];
+        }
+        rs = warp_sum(rs);
+        if (lane == 0) rsp[warp] = rs;
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    ok = consensus(ok);
+
     // ---------------- batch 1: dU^T, Qd^T, Tm^T, dP ----------------
-    if (tid == 0) {
+    if (ok && tid == 0) {
+        fence_after_sync();
         const uint32_t id_mm = idesc_bf16(128, 64, 1, 1), id_mk = idesc_bf16(128, 64, 1, 0);
         const uint32_t id_kk = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
@@ -239,28 +248,38 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(Args a) {
             mma_bf16(tbase + TM_TM, sdesc(sD + ka, 16, 1024), sdesc(sU + kb, 16, 1024), id_kk, st > 0);  // dS+ U^T
             mma_bf16(tbase + TM_DP, sdesc(sO + kb, 16, 1024), sdesc(sU + kb, 16, 1024), id_kk, st > 0);  // dO U^T
         }
-        mma_round();
+        mma_commit(&bar[0]);
+        mma_issued++;
     }
-    ok = wait_mma();
-    // ---------------- epilogue 1: dU (-> dU^T tile), dP rows ----------------
-    if (ok) {
-        float v[64];
-        tmem_row64(tl + TM_DUT, v);
-        const int j = tid;
-        if (a.du)
-            for (int r = 0; r < L; ++r) v[r] += bfv(a.du, trow_g(r) * DV + j);
+    if (ok) ok = wait_mma();
+    // second load group into the regions batch 1 has finished reading
+    if (ok && tid == 0) {
+        mbar_arrive_tx(&bar[2], LOAD2_BYTES);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_DUT, swz(j, ch), v + ch * 8);
-        if (tid < C) {
-            const int r = tid;
-            tmem_row64(tl + TM_DP, v);
-#pragma unroll
-            for (int i = 0; i < 64; ++i) dPf[r * LD + i] = (i <= r) ? v[i] : 0.f;
+        for (int p = 0; p < 2; ++p) {
+            tma_load_2d(sm + R_DS + p * 8192, &mp.W, 64 * p, ci * C, &bar[2]);
+            tma_load_2d(sm + R_DS + 16384 + p * 8192, &mp.Ut, 64 * p, ci * C, &bar[2]);
+            tma_load_4d(sm + R_U + p * 8192, &mp.q, 64 * p, h, t0, b, &bar[2]);
+            tma_load_4d(sm + R_DO + p * 8192, &mp.k, 64 * p, h, t0, b, &bar[2]);
+            tma_load_4d(sm + R_KB + p * 8192, &mp.v, 64 * p, h, t0, b, &bar[2]);
         }
+        loads_issued = 2;
+    }
+    // ---------------- epilogue 1: dU (+ du) -> dU^T tile ----------------
+    if (ok) {
+        float v[32];
+        tmem_row32(tl + TM_DUT, v);
+        const int j = lr;
+        if (a.has_du) {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) v[t] += ld_tile(sm + R_DU, col0 + t, j);
+        }
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + R_DUT, swz(j, hf * 4 + c4), v + c4 * 8);
     }
     fence_proxy_async();
     fence_before_sync();
-    ok = ok && !named_sync_any(1, NTHREADS, *abort_flag != 0);
+    ok = consensus(ok);
     // ---------------- batch 2: dW^T = -S dU^T ----------------
     if (ok && tid == 0) {
         fence_after_sync();
@@ -269,18 +288,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(Args a) {
         for (int st = 0; st < 8; ++st)
             mma_bf16(tbase + TM_DW, sdesc(sS + (st >> 2) * 16384 + (st & 3) * 32, 16, 1024),
                      sdesc(sUT + st * 2048, 1024, 1024), id, st > 0);
-        mma_round();
+        mma_commit(&bar[0]);
+        mma_issued++;
     }
     if (ok) ok = wait_mma();
     if (ok) {
-        float v[64];
-        tmem_row64(tl + TM_DW, v);
+        float v[32];
+        tmem_row32(tl + TM_DW, v);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_DWT, swz(tid, ch), v + ch * 8);
+        for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + R_DWT, swz(lr, hf * 4 + c4), v + c4 * 8);
     }
     fence_proxy_async();
     fence_before_sync();
-    ok = ok && !named_sync_any(1, NTHREADS, *abort_flag != 0);
+    ok = consensus(ok);
     // ---------------- batch 3: dB_k^T = dW^T T, dB_v^T = dU^T T ----------------
     if (ok && tid == 0) {
         fence_after_sync();
@@ -290,50 +310,42 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(Args a) {
             mma_bf16(tbase + TM_DBK, sdesc(sWT + st * 32, 16, 1024), sdesc(sT + st * 2048, 1024, 1024), id, st > 0);
             mma_bf16(tbase + TM_DUT, sdesc(sUT + st * 32, 16, 1024), sdesc(sT + st * 2048, 1024, 1024), id, st > 0);
         }
-        mma_round();
+        mma_commit(&bar[0]);
+        mma_issued++;
     }
     if (ok) ok = wait_mma();
-    // ---------------- epilogue 3: tiles dB_k^T, dB_v^T; dv; dbeta / dg partial sums ----------------
+    if (ok) ok = mbar_wait(&bar[2], 0, abort_flag);  // k, v (and W, U~, q) have landed
+    // ---------------- epilogue 3: dB_k^T, dB_v^T tiles; dv; dbeta / dg partial sums ----------------
     if (ok) {
-        float x[64], y[64];
-        const int c = tid;  // key channel for dB_k^T, value channel for dB_v^T
-        tmem_row64(tl + TM_DBK, x);
+        float x[32], y[32];
+        const int c = lr;  // key channel for dB_k^T, value channel for dB_v^T
+        tmem_row32(tl + TM_DBK, x);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_S, swz(c, ch), x + ch * 8);
+        for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + R_S, swz(c, hf * 4 + c4), x + c4 * 8);
         // e^{g_i} k_ic dB_k^T[c][i]  (-> dbeta, and beta_i times it -> dg)
-        for (int i = 0; i < C; ++i) y[i] = (i < L) ? eg[i] * bfv(a.k, trow_g(i) * DK + c) * x[i] : 0.f;
-        warp_partial_rows(y, rdb + 4 * C, warp, lane);
-        tmem_row64(tl + TM_DUT, x);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_S + 16384, swz(c, ch), x + ch * 8);
-        for (int i = 0; i < C; ++i) {
-            float vv = 0.f;
-            if (i < L) {
-                vv = bfv(a.v, trow_g(i) * DV + c);
-                st_bf(a.dv, trow_g(i) * DV + c, betas[i] * x[i]);
-            }
-            y[i] = vv * x[i];
+        for (int t = 0; t < 32; ++t) y[t] = eg[col0 + t] * ld_tile(sm + R_DO, col0 + t, c) * x[t];
+        red_at(RK_KBK, quarter, col0 + lane) = warp_colsum32(y, lane);
+        tmem_row32(tl + TM_DUT, x);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + R_S + 16384, swz(c, hf * 4 + c4), x + c4 * 8);
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            const int i = col0 + t;
+            y[t] = ld_tile(sm + R_KB, i, c) * x[t];
+            st_tile(sm + R_DUT, i, c, betas[i] * x[t]);  // dv [i][j]
         }
-        warp_partial_rows(y, rdb, warp, lane);
-    }
-    // W, U~ -> tiles (dS+ no longer needed)
-    {
-        const float *Wg = a.w.W + ci * C * DK, *Utg = a.w.Ut + ci * C * DV;
-        for (int x = tid; x < C * 16; x += NTHREADS) {
-            const int r = x >> 4, c16 = x & 15, p = c16 >> 3, ch = c16 & 7;
-            float v[8];
-            ld8f(Wg + (size_t)r * DK + c16 * 8, v);
-            st_chunk(sm + R_DS, (uint32_t)p * 8192 + swz(r, ch), v);
-            ld8f(Utg + (size_t)r * DV + c16 * 8, v);
-            st_chunk(sm + R_DS + 16384, (uint32_t)p * 8192 + swz(r, ch), v);
-        }
+        red_at(RK_VBV, quarter, col0 + lane) = warp_colsum32(y, lane);
     }
     fence_proxy_async();
     fence_before_sync();
-    ok = ok && !named_sync_any(1, NTHREADS, *abort_flag != 0);
-    // ---------------- batch 4: dA' = dB_k W^T + dB_v U~^T  (rows 0..63 valid) ----------------
+    ok = consensus(ok);
+    // ---------------- dv out; batch 4: dA' = dB_k W^T + dB_v U~^T  (rows 0..63 valid) ----------------
     if (ok && tid == 0) {
         fence_after_sync();
+        tma_store_4d(&mp.dv, sm + R_DUT, 0, h, t0, b);
+        tma_store_4d(&mp.dv, sm + R_DUT + 8192, 64, h, t0, b);
+        bulk_commit();
         const uint32_t id = idesc_bf16(128, 64, 1, 0);
         const uint32_t sBk = sS, sBv = sS + 16384, sW = sD, sUt = sD + 16384;
 #pragma unroll
@@ -342,71 +354,50 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(Args a) {
             const uint32_t bb = (st < 8 ? sW : sUt) + ((st & 7) >> 2) * 8192 + (st & 3) * 32;
             mma_bf16(tbase + TM_DW, sdesc(aa, 16384, 1024), sdesc(bb, 16, 1024), id, st > 0);
         }
-        mma_round();
+        mma_commit(&bar[0]);
+        mma_issued++;
     }
     if (ok) ok = wait_mma();
-    // ---------------- epilogue 4: D_P, D_M, Z, dbeta (A part) ----------------
-    float dbA = 0.f;
-    if (ok && tid < C) {
-        const int r = tid;
-        float v[64];
-        tmem_row64(tl + TM_DW, v);
-        const float *KKg = a.w.KK + ci * C * C + (size_t)r * C;
-        const float br = betas[r], grr = gc[r];
-        float rowz = 0.f;
-        float dp[64];
+    // ---------------- epilogue 4 (rows r < 64): D_P, D_M, Z, dbeta (A part) ----------------
+    if (ok && quarter < 2) {
+        const int r = lr;
+        float da[32], dp[32], pv[32], kk[32];
+        tmem_row32(tl + TM_DW, da);
+        tmem_row32(tl + TM_DP, dp);
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            const float e = gated ? __expf(grr - gc[i]) : 1.f;
-            const float da = (i < r) ? -v[i] : 0.f;
-            const float kk = KKg[i];
-            dbA += da * kk * e;
-            const float dpi = dPf[r * LD + i];
-            const float z = dpi * Pf[r * LD + i] + da * br * kk * e;
+        for (int c4 = 0; c4 < 4; ++c4) {
+            ld_chunk(sm + R_P, swz(r, hf * 4 + c4), pv + c4 * 8);
+            ld_chunk(sm + R_KK, swz(r, hf * 4 + c4), kk + c4 * 8);
+        }
+        const float br = betas[r], gr = gc[r];
+        float rowz = 0.f, dbA = 0.f;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            const int i = col0 + t;
+            const float e = (i <= r) ? (gated ? __expf(gr - gc[i]) : 1.f) : 0.f;
+            const float d = (i < r) ? -da[t] : 0.f;
+            const float p = (i <= r) ? dp[t] : 0.f;
+            const float dak = d * kk[t] * e;
+            dbA += dak;
+            const float z = p * pv[t] + br * dak;
             rowz += z;
-            Zf[r * LD + i] = z;
-            dp[i] = dpi * e;                 // D_P row r
-            v[i] = br * da * e;              // D_M row r
+            dp[t] = p * e;        // D_P
+            da[t] = br * d * e;   // D_M
+            pv[t] = z;
         }
-        dgs[r] = rowz;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_P, swz(r, ch), dp + ch * 8);
-#pragma unroll
-        for (int i = 0; i < 64; ++i) dPf[r * LD + i] = v[i];  // D_M (dP no longer needed)
-    }
-    __syncthreads();
-    if (ok && tid < C) {
-        const int r = tid;
-        float sym[64], colz = 0.f;
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            sym[i] = dPf[r * LD + i] + dPf[i * LD + r];
-            colz += Zf[i * LD + r];
+        for (int c4 = 0; c4 < 4; ++c4) {
+            st_chunk(sm + R_P, swz(r, hf * 4 + c4), dp + c4 * 8);
+            st_chunk(sm + R_T, swz(r, hf * 4 + c4), da + c4 * 8);
         }
-        dgs[r] -= colz;
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_T, swz(r, ch), sym + ch * 8);
-    }
-    // q, k -> tiles (U, dO no longer needed)
-    for (int x = tid; x < C * 16; x += NTHREADS) {
-        const int r = x >> 4, c16 = x & 15, p = c16 >> 3, ch = c16 & 7;
-        const uint32_t o = (uint32_t)p * 8192 + swz(r, ch);
-        float v[8];
-        if (r < L) ld8h(reinterpret_cast<const __nv_bfloat16 *>(a.q) + trow_g(r) * DK + c16 * 8, v);
-        else
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = 0.f;
-        st_chunk(sm + R_U, o, v);
-        if (r < L) ld8h(reinterpret_cast<const __nv_bfloat16 *>(a.k) + trow_g(r) * DK + c16 * 8, v);
-        else
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = 0.f;
-        st_chunk(sm + R_DO, o, v);
+        rowsum[hf * 64 + r] = rowz;
+        rowsum[128 + hf * 64 + r] = dbA;
+        red_at(RK_ZC, quarter, col0 + lane) = warp_colsum32(pv, lane);
     }
     fence_proxy_async();
     fence_before_sync();
-    ok = ok && !named_sync_any(1, NTHREADS, *abort_flag != 0);
-    // ---------------- batch 5: dq^T += k^T D_P^T;  dk^T = q^T D_P + k^T (D_M + D_M^T) ----------------
+    ok = consensus(ok);
+    // ---------------- batch 5: dq^T = k^T D_P^T;  dk^T = q^T D_P + k^T D_M + k^T D_M^T ----------------
     if (ok && tid == 0) {
         fence_after_sync();
         const uint32_t sQ = sU, sKr = sO, sDP = sP, sDM = sT;
@@ -418,72 +409,97 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(Args a) {
                      st > 0);
         }
 #pragma unroll
-        for (int st = 0; st < 4; ++st)
+        for (int st = 0; st < 4; ++st) {
             mma_bf16(tbase + TM_DK, sdesc(sKr + st * 2048, 8192, 1024), sdesc(sDM + st * 2048, 1024, 1024), id_k, 1);
-        mma_round();
+            mma_bf16(tbase + TM_DK, sdesc(sKr + st * 2048, 8192, 1024), sdesc(sDM + st * 32, 16, 1024), id_q, 1);
+        }
+        mma_commit(&bar[0]);
+        mma_issued++;
     }
     if (ok) ok = wait_mma();
-    // ---------------- epilogue 5: dq, dk; dg channel sums ----------------
+    // ---------------- epilogue 5: dq, dk staging; dg channel sums ----------------
     if (ok) {
-        const int c = tid;
-        float acc[64], w[64], x[64];
+        const int c = lr;
+        float w[32], acc[32], y[32];
         // dq = e^g (dO S^T) + D_P k ; dg += e^g q . (dO S^T)
-        tmem_row64(tl + TM_QD, w);
-        tmem_row64(tl + TM_DQ, acc);
-        for (int r = 0; r < C; ++r) {
-            float qv = 0.f;
-            if (r < L) {
-                qv = bfv(a.q, trow_g(r) * DK + c);
-                st_bf(a.dq, trow_g(r) * DK + c, eg[r] * w[r] + acc[r]);
-            }
-            x[r] = eg[r] * qv * w[r];
-        }
-        warp_partial_rows(x, red, warp, lane);
-        // dk = D_P^T q + (D_M + D_M^T) k + beta e^g dB_k + e^{gC-g} U dS+^T ; dg terms
-        tmem_row64(tl + TM_DK, acc);
-        tmem_row64(tl + TM_DBK, w);
-        float y[64];
-        tmem_row64(tl + TM_TM, y);
-        float tsum = 0.f;
-        for (int r = 0; r < C; ++r) {
-            float kv = 0.f;
-            if (r < L) {
-                kv = bfv(a.k, trow_g(r) * DK + c);
-                st_bf(a.dk, trow_g(r) * DK + c, acc[r] + betas[r] * eg[r] * w[r] + egc[r] * y[r]);
-            }
-            x[r] = egc[r] * kv * y[r];
-            tsum += x[r];
-        }
-        warp_partial_rows(x, red + 2 * 4 * C, warp, lane);
+        tmem_row32(tl + TM_QD, w);
+        tmem_row32(tl + TM_DQ, acc);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) tsum += __shfl_xor_sync(0xffffffffu, tsum, o);
-        // the chunk-end term sum_r e^{g_C - g_r} k_r . (U dS+^T)_r belongs to dg_C (last row)
-        if (lane == 0) atomicAdd(&dgs[C - 1], tsum);
+        for (int t = 0; t < 32; ++t) {
+            const int r = col0 + t;
+            st_tile(sm + R_DWT, r, c, eg[r] * w[t] + acc[t]);
+            y[t] = eg[r] * ld_tile(sm + R_U, r, c) * w[t];
+        }
+        red_at(RK_QQD, quarter, col0 + lane) = warp_colsum32(y, lane);
+        // dk = D_P^T q + (D_M + D_M^T) k + beta e^g dB_k + e^{gC-g} U dS+^T ; dg terms
+        float tm[32];
+        tmem_row32(tl + TM_DK, acc);
+        tmem_row32(tl + TM_DBK, w);
+        tmem_row32(tl + TM_TM, tm);
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            const int r = col0 + t;
+            st_tile(sm + R_DS, r, c, acc[t] + betas[r] * eg[r] * w[t] + egc[r] * tm[t]);
+            y[t] = egc[r] * ld_tile(sm + R_DO, r, c) * tm[t];
+        }
+        red_at(RK_KTM, quarter, col0 + lane) = warp_colsum32(y, lane);
     }
-    __syncthreads();
+    fence_proxy_async();
+    fence_before_sync();
+    ok = consensus(ok);
+    if (ok && tid == 0) {
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            tma_store_4d(&mp.dq, sm + R_DWT + p * 8192, 64 * p, h, t0, b);
+            tma_store_4d(&mp.dk, sm + R_DS + p * 8192, 64 * p, h, t0, b);
+        }
+        bulk_commit();
+    }
     // ---------------- dbeta, dg, d log alpha ----------------
     if (ok && tid < C) {
         const int r = tid;
         float sq = 0.f, sbk = 0.f, skt = 0.f, sv = 0.f;
 #pragma unroll
-        for (int w4 = 0; w4 < 4; ++w4) {
-            sq += red[w4 * C + r];
-            skt += red[2 * 4 * C + w4 * C + r];
-            sv += rdb[w4 * C + r];
-            sbk += rdb[4 * C + w4 * C + r];
+        for (int q = 0; q < 4; ++q) {
+            sq += red_at(RK_QQD, q, r);
+            sbk += red_at(RK_KBK, q, r);
+            skt += red_at(RK_KTM, q, r);
+            sv += red_at(RK_VBV, q, r);
         }
+        const float zc = red_at(RK_ZC, 0, r) + red_at(RK_ZC, 1, r);
+        const float rowz = rowsum[r] + rowsum[64 + r], dbA = rowsum[128 + r] + rowsum[192 + r];
         if (r < L) st_bf(a.dbeta, trow_g(r), dbA + sbk + sv);
-        dgs[r] += sq + betas[r] * sbk - skt;
+        dgs[r] = rowz - zc + sq + betas[r] * sbk - skt;
+        ktm[r] = skt;
     }
     __syncthreads();
-    if (ok && gated && tid == 0) {
+    if (ok && gated && warp == 0) {
+        float a0 = dgs[2 * lane], a1 = dgs[2 * lane + 1];
+        const float tsum = warp_sum(ktm[2 * lane] + ktm[2 * lane + 1]);
         float rs = 0.f;
 #pragma unroll
-        for (int w4 = 0; w4 < 4; ++w4) rs += rsp[w4];
-        float run = __expf(gc[C - 1]) * rs;  // the chunk-end decay e^{g_C} of the incoming state
-        for (int r = C - 1; r >= 0; --r) {
-            run += dgs[r];
-            if (r < L) st_bf(a.dalpha, trow_g(r), run);
+        for (int w8 = 0; w8 < 8; ++w8) rs += rsp[w8];
+        // the chunk-end terms belong to dg_C (last row): the k . Tm sums and the decay
+        // e^{g_C} of the incoming state
+        if (lane == 31) a1 += tsum + __expf(gc[C - 1]) * rs;
+        const float tot = a0 + a1;
+        float incl = tot;  // inclusive suffix sum over lanes
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_down_sync(0xffffffffu, incl, o);
+            if (lane + o < 32) incl += y;
+        }
+        const float excl = incl - tot;
+        if (2 * lane < L) st_bf(a.dalpha, trow_g(2 * lane), tot + excl);
+        if (2 * lane + 1 < L) st_bf(a.dalpha, trow_g(2 * lane + 1), a1 + excl);
+    }
+    if (tid == 0) {
+        bulk_wait_all();
+        if (*abort_flag) {  // let whatever was issued finish before the CTA leaves
+            volatile int dummy = 0;
+            if (mma_issued > 0) mbar_wait(&bar[0], (mma_issued - 1) & 1, &dummy, 100000000ull);
+            if (loads_issued >= 1) mbar_wait(&bar[1], 0, &dummy, 100000000ull);
+            if (loads_issued >= 2) mbar_wait(&bar[2], 0, &dummy, 100000000ull);
         }
     }
     fence_before_sync();
@@ -494,18 +510,62 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(Args a) {
 
 }  // namespace tcb
 
-cudaError_t tc_bwd_chunk(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec) {
+bool tc_bwd_recompute_supported(const Geo &g, bool bf16) {
+    return tc_fwd_supported(g, bf16) && g.variant != VAR_KDA && g.dv == 128 &&
+           (size_t)g.B * g.H * g.N * 128 <= (size_t)INT_MAX;
+}
+
+static size_t ws_al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t tc_bwd_ws_bytes(const Geo &g) {
+    const size_t nc = (size_t)g.B * g.H * g.N, C = g.C, DK = g.dk, DV = g.dv;
+    return 2 * ws_al256(nc * DK * DV * 2) + ws_al256(nc * C * DV * 2) * 2 + ws_al256(nc * C * DK * 2) +
+           3 * ws_al256(nc * C * C * 2) + ws_al256(nc * C * 4);
+}
+
+TcBwdWs tc_bwd_ws_carve(const Geo &g, void *base) {
+    const size_t nc = (size_t)g.B * g.H * g.N, C = g.C, DK = g.dk, DV = g.dv;
+    char *p = (char *)base;
+    auto take = [&](size_t bytes) { char *r = p; p += ws_al256(bytes); return r; };
+    TcBwdWs w;
+    w.Sn = (__nv_bfloat16 *)take(nc * DK * DV * 2);
+    w.dSn = (__nv_bfloat16 *)take(nc * DK * DV * 2);
+    w.Un = (__nv_bfloat16 *)take(nc * C * DV * 2);
+    w.W = (__nv_bfloat16 *)take(nc * C * DK * 2);
+    w.Ut = (__nv_bfloat16 *)take(nc * C * DV * 2);
+    w.P = (__nv_bfloat16 *)take(nc * C * C * 2);
+    w.Tn = (__nv_bfloat16 *)take(nc * C * C * 2);
+    w.KK = (__nv_bfloat16 *)take(nc * C * C * 2);
+    w.g = (float *)take(nc * C * 4);
+    return w;
+}
+
+cudaError_t tc_bwd_chunk(const Geo &g, const Tensors &t, const TcBwdWs &w, cudaStream_t s, Rec &rec) {
     using namespace tcb;
+    Maps mp;
+    const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;
+    bool ok = tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) && tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64) &&
+              tc::make_map_4d_bf16(&mp.v, t.v, DV, H, T, Bn, 64) &&
+              tc::make_map_4d_bf16(&mp.dout, t.dout, DV, H, T, Bn, 64) &&
+              tc::make_map_4d_bf16(&mp.dq, t.dq, DK, H, T, Bn, 64) &&
+              tc::make_map_4d_bf16(&mp.dk, t.dk, DK, H, T, Bn, 64) &&
+              tc::make_map_4d_bf16(&mp.dv, t.dv, DV, H, T, Bn, 64) &&
+              tc::make_map_2d_bf16(&mp.S, w.Sn, DV, NC * DK, 128) &&
+              tc::make_map_2d_bf16(&mp.dS, w.dSn, DV, NC * DK, 128) &&
+              tc::make_map_2d_bf16(&mp.U, w.Un, DV, NC * C, 64) && tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) &&
+              tc::make_map_2d_bf16(&mp.Ut, w.Ut, DV, NC * C, 64) && tc::make_map_2d_bf16(&mp.P, w.P, C, NC * C, 64) &&
+              tc::make_map_2d_bf16(&mp.T, w.Tn, C, NC * C, 64) && tc::make_map_2d_bf16(&mp.KK, w.KK, C, NC * C, 64);
+    if (ok && t.du) ok = tc::make_map_4d_bf16(&mp.du, t.du, DV, H, T, Bn, 64);
+    else mp.du = mp.dout;
+    if (!ok) return cudaErrorInvalidValue;
     Args a;
-    a.q = t.q; a.k = t.k; a.v = t.v; a.alpha = t.alpha; a.beta = t.beta; a.dout = t.dout; a.du = t.du;
-    a.dq = t.dq; a.dk = t.dk; a.dv = t.dv; a.dalpha = t.dalpha; a.dbeta = t.dbeta;
-    a.w = w;
-    a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N; a.variant = g.variant;
+    a.beta = t.beta; a.dalpha = t.dalpha; a.dbeta = t.dbeta; a.g = w.g;
+    a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N; a.variant = g.variant; a.has_du = t.du != nullptr;
     const size_t smem = SMEM_BYTES + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_bwd_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     rec.mark(s);
-    k_bwd_chunk_tc<<<dim3(g.N, g.H, g.B), NTHREADS, smem, s>>>(a);
+    k_bwd_chunk_tc<<<dim3(g.N, g.H, g.B), NTHREADS, smem, s>>>(mp, a);
     return cudaGetLastError();
 }
 

@@ -604,10 +604,6 @@ bool tc_fwd_supported(const Geo &g, bool bf16) {
 
 size_t tc_fwd_ws_bytes(const Geo &) { return 0; }
 
-bool tc_bwd_recompute_supported(const Geo &g, bool bf16) {
-    return tc_fwd_supported(g, bf16) && g.variant != VAR_KDA && g.dv == 128;
-}
-
 int tc_fwd_launches(const Geo &g, const char **names, int max_names) {
     if (names && max_names > 0) names[0] = (g.variant == VAR_KDA) ? "k_fwd_tc" : "k_fwd_tc2";
     return 1;

@@ -80,13 +80,25 @@ struct Args {
     void *out, *u;
     float *ST;
     int B, T, H, dv, N;
-    // recompute mode (backward): fp32 chunk products for the CUDA-core backward kernels
-    float *W, *Ut, *G, *P, *Sn, *Un, *Tn, *KK;
+    // recompute mode (backward): the chunk products of the tensor-core backward workspace
+    __nv_bfloat16 *W, *Ut, *P, *Sn, *Un, *Tn, *KK;
+    float *G;
     // reverse mode: dL/dS of the state leaving each chunk; whether du is given
-    float *dSn;
+    __nv_bfloat16 *dSn;
     int has_du;
 };
 
+// 8 values as bf16 at element offset elem_off (a multiple of 8) of a bf16 array
+__device__ __forceinline__ void st8_global(void *base, size_t elem_off, const float *v) {
+    uint4 w;
+    w.x = pack_bf16(v[0], v[1]);
+    w.y = pack_bf16(v[2], v[3]);
+    w.z = pack_bf16(v[4], v[5]);
+    w.w = pack_bf16(v[6], v[7]);
+    *reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(base) + elem_off) = w;
+}
+
+// 64 values as bf16 at element offset elem_off (a multiple of 8) of a bf16 array
 __device__ __forceinline__ void st_row_global(void *base, size_t elem_off, const float *v) {
     uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(base) + elem_off);
 #pragma unroll
@@ -101,9 +113,9 @@ __device__ __forceinline__ void st_row_global(void *base, size_t elem_off, const
 }
 
 // MODE 0: forward (o, u, S_T).
-// MODE 1: recompute for the backward -- no o / u / S_T; instead the chunk products W, U~,
-//         g, P, the entering state S_n and the write values U are stored in the fp32
-//         chunk-major layout the backward kernels read.
+// MODE 1: recompute for the backward -- no o / u / S_T; instead g, k k^T, P, T, W, U~,
+//         the entering state S_n and the write values U are stored (bf16 rows, fp32 g)
+//         in the chunk-major layout of TcBwdWs.
 // MODE 2: the backward's reverse state chain.  Chunks are visited last to first; the
 //         preparation is the same (A_chain = [-W ; Q~ - P W]) minus P4, the chain's copy
 //         of k is scaled to Kbar = e^{g_C - g} k, and the chain warpgroup evaluates
@@ -217,14 +229,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     bigflag[s] = dev > 80.f;
                 }
                 if (SAVE && half == 0) {
-                    float *Gc = a.G + ((((size_t)b * H + h) * N + mc) * C) * DK;
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const float4 x4 = make_float4(xs[hh], xs[hh], xs[hh], xs[hh]);
-                        float4 *dst = reinterpret_cast<float4 *>(Gc + (size_t)(lane + 32 * hh) * DK);
-#pragma unroll
-                        for (int c4 = 0; c4 < DK / 4; ++c4) dst[c4] = x4;
-                    }
+                    float *Gc = a.G + (((size_t)b * H + h) * N + mc) * C;
+                    Gc[lane] = xs[0];
+                    Gc[lane + 32] = xs[1];
                 }
             }
             __syncwarp();
@@ -331,12 +338,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                     for (int i = 0; i < 64; ++i) f[i] = __expf(gr - gc[i]);
                 }
-                if (SAVE && arow && half == 0) {
-                    float4 *dst = reinterpret_cast<float4 *>(a.KK + ((((size_t)b * H + h) * N + mc) * C + r) * C);
-#pragma unroll
-                    for (int i4 = 0; i4 < 16; ++i4)
-                        dst[i4] = make_float4(g1[4 * i4], g1[4 * i4 + 1], g1[4 * i4 + 2], g1[4 * i4 + 3]);
-                }
+                if (SAVE && arow && half == 0)
+                    st_row_global(a.KK, ((((size_t)b * H + h) * N + mc) * C + r) * C, g1);
                 if (arow) {
                     const float br = pf[PF_BV * 64 + r];
 #pragma unroll
@@ -360,12 +363,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     for (int i = 0; i < 64; ++i) g1[i] = (i <= r) ? g1[i] * f[i] : 0.f;
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_IP, swz(trow, ch), g1 + ch * 8);
-                    if (SAVE && half == 0) {
-                        float4 *dst = reinterpret_cast<float4 *>(a.P + ((((size_t)b * H + h) * N + mc) * C + r) * C);
-#pragma unroll
-                        for (int i4 = 0; i4 < 16; ++i4)
-                            dst[i4] = make_float4(g1[4 * i4], g1[4 * i4 + 1], g1[4 * i4 + 2], g1[4 * i4 + 3]);
-                    }
+                    if (SAVE && half == 0) st_row_global(a.P, ((((size_t)b * H + h) * N + mc) * C + r) * C, g1);
                 }
                 fence_before_sync();
                 wsync();
@@ -380,12 +378,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                         for (int e = 0; e < 8; ++e) w[e] = (ch * 8 + e <= i) ? w[e] : 0.f;
                         st_chunk(sm + OFF_TT, swz(i, ch), w);
-                        if (SAVE && half == 0) {
-                            float4 *dst = reinterpret_cast<float4 *>(
-                                a.Tn + ((((size_t)b * H + h) * N + mc) * C + i) * C + ch * 8);
-                            dst[0] = make_float4(w[0], w[1], w[2], w[3]);
-                            dst[1] = make_float4(w[4], w[5], w[6], w[7]);
-                        }
+                        if (SAVE && half == 0)
+                            st8_global(a.Tn, ((((size_t)b * H + h) * N + mc) * C + i) * C + ch * 8, w);
                     }
                 }
                 fence_proxy_async();
@@ -452,17 +446,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const size_t ci = ((size_t)b * H + h) * N + mc;
                 float rv[64];
                 tmem_row64(tl + TM_D0 + bb * 64, rv);
-                float4 *du = reinterpret_cast<float4 *>(a.Ut + (ci * C + trow) * DV + j0);
-#pragma unroll
-                for (int i4 = 0; i4 < 16; ++i4) du[i4] = make_float4(rv[4 * i4], rv[4 * i4 + 1], rv[4 * i4 + 2], rv[4 * i4 + 3]);
+                st_row_global(a.Ut, (ci * C + trow) * DV + j0, rv);
                 if (half == 0) {
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         tmem_row64(tl + TM_X + hh * 64, rv);
-                        float4 *dw = reinterpret_cast<float4 *>(a.W + (ci * C + trow) * DK + hh * 64);
-#pragma unroll
-                        for (int i4 = 0; i4 < 16; ++i4)
-                            dw[i4] = make_float4(rv[4 * i4], rv[4 * i4 + 1], rv[4 * i4 + 2], rv[4 * i4 + 3]);
+                        st_row_global(a.W, (ci * C + trow) * DK + hh * 64, rv);
                     }
                 }
             }
@@ -539,12 +528,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 mbar_wait(&bar[B_READY0 + bb], (m >> 1) & 1, abort_flag);
                 mbar_wait(&bar[B_VFULL], m & 1, abort_flag);
                 if (wabort()) break;
-                {
-                    float4 *dst = reinterpret_cast<float4 *>(a.dSn + ((((size_t)b * H + h) * N + mc) * DK + trow) * DV + j0);
-#pragma unroll
-                    for (int j4 = 0; j4 < DVB / 4; ++j4)
-                        dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
-                }
+                st_row_global(a.dSn, ((((size_t)b * H + h) * N + mc) * DK + trow) * DV + j0, S);
                 // G = (-W)^T Kbar  and  D = A_chain^T [du ; dO]
                 if (wc == 0) {
                     fence_after_sync();
@@ -611,11 +595,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int L = min(C, T - t0);
             mbar_wait(&bar[B_READY0 + bb], (m >> 1) & 1, abort_flag);
             if (wabort()) break;
-            if (SAVE) {
-                float4 *dst = reinterpret_cast<float4 *>(a.Sn + ((((size_t)b * H + h) * N + m) * DK + trow) * DV + j0);
-#pragma unroll
-                for (int j4 = 0; j4 < DVB / 4; ++j4) dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
-            }
+            if (SAVE) st_row_global(a.Sn, ((((size_t)b * H + h) * N + m) * DK + trow) * DV + j0, S);
             // ---------------- C1: D += A_chain . S ----------------
             if (wc == 0) {
                 fence_after_sync();
@@ -636,12 +616,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tmem_row64(tl + TM_D0 + bb * 64, dv);
                 if (trow < 64) {
                     const int r = trow;
-                    if (SAVE) {
-                        float4 *dst = reinterpret_cast<float4 *>(a.Un + ((((size_t)b * H + h) * N + m) * C + r) * DV + j0);
-#pragma unroll
-                        for (int j4 = 0; j4 < 16; ++j4)
-                            dst[j4] = make_float4(dv[4 * j4], dv[4 * j4 + 1], dv[4 * j4 + 2], dv[4 * j4 + 3]);
-                    } else if (a.u && r < L) {
+                    if (SAVE) st_row_global(a.Un, ((((size_t)b * H + h) * N + m) * C + r) * DV + j0, dv);
+                    else if (a.u && r < L) {
                         st_row_global(a.u, (((size_t)b * T + t0 + r) * H + h) * DV + j0, dv);
                     }
                     const float f = cf[bb * 80 + r];
@@ -718,7 +694,7 @@ static cudaError_t launch_tc2(const CUtensorMap &mq, const CUtensorMap &mk, cons
     return cudaGetLastError();
 }
 
-static cudaError_t tc2_common(const Geo &g, const Tensors &t, const SimtWs *w, int mode, cudaStream_t s, Rec &rec) {
+static cudaError_t tc2_common(const Geo &g, const Tensors &t, const TcBwdWs *w, int mode, cudaStream_t s, Rec &rec) {
     using namespace tcf2;
     CUtensorMap mq, mk, mv, mx;
     const uint64_t Bn = g.B, T = g.T, H = g.H;
@@ -736,7 +712,7 @@ static cudaError_t tc2_common(const Geo &g, const Tensors &t, const SimtWs *w, i
         a.S0 = t.S0; a.out = t.out; a.u = t.u; a.ST = t.S_T;
     }
     if (mode == 1) {
-        a.W = w->W; a.Ut = w->Ut; a.G = w->G; a.P = w->P; a.Sn = w->Sn; a.Un = w->Un;
+        a.W = w->W; a.Ut = w->Ut; a.G = w->g; a.P = w->P; a.Sn = w->Sn; a.Un = w->Un;
         a.Tn = w->Tn; a.KK = w->KK;
     }
     const dim3 grid(g.dv / DVB, g.H, g.B);
@@ -754,13 +730,13 @@ static cudaError_t tc2_common(const Geo &g, const Tensors &t, const SimtWs *w, i
 // Warp-specialised forward (Gated DeltaNet / DeltaNet).
 cudaError_t tc_fwd2(const Geo &g, const Tensors &t, cudaStream_t s, Rec &rec) { return tc2_common(g, t, nullptr, 0, s, rec); }
 
-// The same kernel in recompute mode: fills W, U~, g, P, S_n, U of the backward workspace.
-cudaError_t tc_bwd_recompute(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec) {
+// The same kernel in recompute mode: fills g, KK, P, T, W, U~, S_n, U of the backward workspace.
+cudaError_t tc_bwd_recompute(const Geo &g, const Tensors &t, const TcBwdWs &w, cudaStream_t s, Rec &rec) {
     return tc2_common(g, t, &w, 1, s, rec);
 }
 
 // The same kernel in reverse mode: fills dS_{n+1} of every chunk and writes dS0.
-cudaError_t tc_bwd_reverse(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec) {
+cudaError_t tc_bwd_reverse(const Geo &g, const Tensors &t, const TcBwdWs &w, cudaStream_t s, Rec &rec) {
     return tc2_common(g, t, &w, 2, s, rec);
 }
 

@@ -45,5 +45,20 @@ inline bool make_map_4d_bf16(CUtensorMap *map, const void *base, uint64_t D0, ui
     return r == CUDA_SUCCESS;
 }
 
+// Tensor map over a row-major bf16 matrix [D1][D0] (D0 innermost, a multiple of 8),
+// with a box of 64 x box_rows elements and 128-byte swizzle.
+inline bool make_map_2d_bf16(CUtensorMap *map, const void *base, uint64_t D0, uint64_t D1, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {D0, D1};
+    const cuuint64_t strides[1] = {D0 * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace tc
 }  // namespace dr
