@@ -40,8 +40,8 @@ bool use_tc_fwd(const Geo &g, int dtype) { return tc_fwd_supported(g, dtype == D
 
 size_t ws_bytes(const Geo &g, int dtype, bool bwd) {
     if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
-    if (!bwd && use_tc_fwd(g, dtype)) return tc_fwd_ws_bytes(g);
-    if (bwd && tc_bwd_recompute_supported(g, dtype == DR_BF16)) return tc_bwd_ws_bytes(g);
+    if (tc_split_supported(g, dtype == DR_BF16)) return tc_ws_bytes(g, bwd);
+    if (!bwd && use_tc_fwd(g, dtype)) return 0;
     return simt_ws_bytes(g, bwd);
 }
 
@@ -123,10 +123,11 @@ static int bwd_impl(const void *q, const void *k, const void *v, const void *alp
     t.q = q; t.k = k; t.v = v; t.alpha = alpha; t.beta = beta; t.S0 = S0;
     t.dout = dout; t.du = du; t.dS_T = dS_T;
     t.dq = dq; t.dk = dk_; t.dv = dv_; t.dalpha = dalpha; t.dbeta = dbeta; t.dS0 = dS0;
-    if (tc_bwd_recompute_supported(g, dtype == DR_BF16)) {
-        const TcBwdWs w = tc_bwd_ws_carve(g, workspace);
-        rc = launch_status(tc_bwd_recompute(g, t, w, s, rec));
-        if (rc == DR_OK) rc = launch_status(tc_bwd_reverse(g, t, w, s, rec));
+    if (tc_split_supported(g, dtype == DR_BF16)) {
+        const TcWs w = tc_ws_carve(g, true, workspace);
+        rc = launch_status(tc_chunk_prep(g, t, w, true, s, rec));
+        if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, true, s, rec));
+        if (rc == DR_OK) rc = launch_status(tc_chain_rev(g, t, w, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_bwd_chunk(g, t, w, s, rec));
     } else {
         const SimtWs w = simt_ws_carve(g, true, workspace);
@@ -145,9 +146,9 @@ static int launch_plan(const Geo &g, int dtype, bool bwd, const char **names, in
         n = tc_fwd_launches(g, names, max_names);
         return n;
     }
-    if (bwd && tc_bwd_recompute_supported(g, dtype == DR_BF16)) {
+    if (bwd && tc_split_supported(g, dtype == DR_BF16)) {
         src = TC_BWD_KERNELS;
-        n = 3;
+        n = 4;
     } else {
         src = bwd ? SIMT_BWD_KERNELS : SIMT_FWD_KERNELS;
         n = bwd ? 5 : 3;

@@ -2,7 +2,8 @@
 // word and all kernels live in one module, so no relocatable device code is needed).
 #include "simt_path.cu"
 #include "tc_fwd.cu"
-#include "tc_fwd2.cu"
+#include "tc_prep.cu"
+#include "tc_chain.cu"
 #include "tc_bwd.cu"
 #include "api.cu"
 #include "noalloc.cu"

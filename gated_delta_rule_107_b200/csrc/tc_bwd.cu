@@ -31,8 +31,6 @@
 // leave through shared-memory staging tiles and TMA stores.  Warps w and w + 4 read the
 // same 32 TMEM lanes (channel rows) and split the 64 token columns; sums over channels
 // are butterfly transposes inside a warp plus four partials in shared memory.
-#include <limits.h>
-
 #include "tc_host.cuh"
 #include "tc_path.cuh"
 #include "tc_ptx.cuh"
@@ -314,7 +312,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(const __grid_const
         mma_issued++;
     }
     if (ok) ok = wait_mma();
-    if (ok) ok = mbar_wait(&bar[2], 0, abort_flag);  // k, v (and W, U~, q) have landed
+    if (ok) ok = consensus(mbar_wait(&bar[2], 0, abort_flag));  // k, v (and W, U~, q) have landed
     // ---------------- epilogue 3: dB_k^T, dB_v^T tiles; dv; dbeta / dg partial sums ----------------
     if (ok) {
         float x[32], y[32];
@@ -510,37 +508,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(const __grid_const
 
 }  // namespace tcb
 
-bool tc_bwd_recompute_supported(const Geo &g, bool bf16) {
-    return tc_fwd_supported(g, bf16) && g.variant != VAR_KDA && g.dv == 128 &&
-           (size_t)g.B * g.H * g.N * 128 <= (size_t)INT_MAX;
-}
-
-static size_t ws_al256(size_t x) { return (x + 255) & ~(size_t)255; }
-
-size_t tc_bwd_ws_bytes(const Geo &g) {
-    const size_t nc = (size_t)g.B * g.H * g.N, C = g.C, DK = g.dk, DV = g.dv;
-    return 2 * ws_al256(nc * DK * DV * 2) + ws_al256(nc * C * DV * 2) * 2 + ws_al256(nc * C * DK * 2) +
-           3 * ws_al256(nc * C * C * 2) + ws_al256(nc * C * 4);
-}
-
-TcBwdWs tc_bwd_ws_carve(const Geo &g, void *base) {
-    const size_t nc = (size_t)g.B * g.H * g.N, C = g.C, DK = g.dk, DV = g.dv;
-    char *p = (char *)base;
-    auto take = [&](size_t bytes) { char *r = p; p += ws_al256(bytes); return r; };
-    TcBwdWs w;
-    w.Sn = (__nv_bfloat16 *)take(nc * DK * DV * 2);
-    w.dSn = (__nv_bfloat16 *)take(nc * DK * DV * 2);
-    w.Un = (__nv_bfloat16 *)take(nc * C * DV * 2);
-    w.W = (__nv_bfloat16 *)take(nc * C * DK * 2);
-    w.Ut = (__nv_bfloat16 *)take(nc * C * DV * 2);
-    w.P = (__nv_bfloat16 *)take(nc * C * C * 2);
-    w.Tn = (__nv_bfloat16 *)take(nc * C * C * 2);
-    w.KK = (__nv_bfloat16 *)take(nc * C * C * 2);
-    w.g = (float *)take(nc * C * 4);
-    return w;
-}
-
-cudaError_t tc_bwd_chunk(const Geo &g, const Tensors &t, const TcBwdWs &w, cudaStream_t s, Rec &rec) {
+cudaError_t tc_bwd_chunk(const Geo &g, const Tensors &t, const TcWs &w, cudaStream_t s, Rec &rec) {
     using namespace tcb;
     Maps mp;
     const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;

@@ -1,0 +1,586 @@
+// tc_chain.cu -- the serial state chains of the chunked gated delta rule on tcgen05
+// (Gated DeltaNet and DeltaNet; bf16 I/O, dk = dv = 128, C = 64).
+//
+// Chunked form of "线性注意力架构演进与Kimi Delta Attention创新实践" (sections 2.1, 6.1,
+// 6.2, 7.1), given the per-chunk products of tc_prep.cu (W, U~, P, g, and for the backward
+// du + P^T dO).  One CTA per (b, h, 64 value channels) walks the chunks in order; the state
+// block (128 key rows x 64 value columns) stays in fp32 registers, one row per thread, with a
+// bf16 copy in shared memory as the MMA operand.
+//
+// Forward chain, chunk n, S = S_n:
+//   D  = [W ; q] S                  rows 0-63: W S, rows 64-127: q S
+//   U  = U~ - W S                   the write values (the forward's u)
+//   O' = P U                        (M = 128 MMA; rows 0-63 discarded)
+//   o  = diag(e^g) q S + O'
+//   S_{n+1} = e^{g_C} S + k^T (e^{g_C - g} U)
+// Reverse chain, chunk n from last to first, dS+ = dL/dS_{n+1}:
+//   dU = (du + P^T dO) + diag(e^{g_C - g}) k dS+
+//   dL/dS_n = e^{g_C} dS+ + q^T diag(e^g) dO - W^T dU
+//
+// Warp 0 is a TMA producer that keeps two chunks of operands in flight; warps 1-4 run the
+// chain (thread = TMEM lane = state row).  Every wait is bounded (~1 s) and aborts are
+// agreed on per warpgroup.
+#include <limits.h>
+
+#include "tc_host.cuh"
+#include "tc_path.cuh"
+#include "tc_ptx.cuh"
+#include "tc_tile.cuh"
+
+namespace dr {
+namespace tch {
+
+using namespace dr::tc;
+using dr::tcf::ld_chunk;
+using dr::tcf::st_chunk;
+using dr::tcf::st_row_global;
+using dr::tcf::tmem_row64;
+
+constexpr int C = 64, DK = 128, DV = 128, DVB = 64;
+constexpr int NTHREADS = 160;
+// shared memory (bytes from a 1024-aligned base): two stages of 64K, then the chain's tiles
+constexpr uint32_t STAGE = 65536;
+// forward stage: [W_p0 | q_p0 | W_p1 | q_p1], [U~ (this CTA's 64 columns) | P], [k_p0 | k_p1]
+constexpr uint32_t FS_WQ = 0, FS_UP = 32768, FS_K = 49152;
+// reverse stage: k, q, W (2 panels each), dO and du + P^T dO (this CTA's 64 columns)
+constexpr uint32_t RS_K = 0, RS_Q = 16384, RS_W = 32768, RS_DO = 49152, RS_DU = 57344;
+constexpr uint32_t OFF_S = 2 * STAGE;         // 16K  bf16 state [c][j]
+constexpr uint32_t OFF_U = OFF_S + 16384;     //  8K  U [r][j]        (reverse: dU [r][j])
+constexpr uint32_t OFF_UD = OFF_U + 8192;     //  8K  e^{g_C - g} U [r][j]
+constexpr uint32_t OFF_MISC = OFF_UD + 8192;  //  4K
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 4096;
+// misc
+constexpr uint32_t M_BAR = 0;  // FULL0, FULL1, EMPTY0, EMPTY1, MMA
+constexpr uint32_t M_TMEM = 64, M_ABORT = 68;
+constexpr uint32_t M_CF = 256;  // per stage: [0..63] e^{g_C - g}, [64..127] e^g, [128] e^{g_C}
+enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_MMA, B_NUM };
+static_assert(M_CF + 2 * 132 * 4 <= 4096, "misc overflow");
+
+struct FMaps {
+    CUtensorMap q, k;   // [B, T, H, 128] bf16; box 64 x 64 tokens
+    CUtensorMap W, Ut;  // [chunks * 64][128] bf16; box 64 x 64
+    CUtensorMap P;      // [chunks * 64][64] bf16; box 64 x 64
+};
+struct RMaps {
+    CUtensorMap q, k, dout;  // [B, T, H, 128] bf16
+    CUtensorMap W, dUp;      // [chunks * 64][128] bf16
+};
+struct Args {
+    const float *g;           // [chunks][64]
+    const float *S0;          // forward: S0; reverse: dS_T (fp32 [B, H, 128, 128], may be null)
+    float *ST;                // forward: S_T; reverse: dS0 (may be null)
+    void *out, *u;            // forward outputs (bf16 [B, T, H, 128])
+    __nv_bfloat16 *Sn, *Un;   // recompute outputs
+    __nv_bfloat16 *dSn;       // reverse output
+    int B, T, H, N;
+};
+
+// Producer side: the gate factors of chunk ci into cf (e^{g_C - g}, e^g, e^{g_C}).
+__device__ __forceinline__ void chunk_factors(const float *g, size_t ci, float *cf, int lane) {
+    const float *gg = g + ci * C;
+    const float gC = gg[C - 1];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        const int r = lane + 32 * hh;
+        const float x = gg[r];
+        cf[r] = __expf(gC - x);
+        cf[64 + r] = __expf(x);
+    }
+    if (lane == 0) cf[128] = __expf(gC);
+}
+
+// ====================================== forward chain ======================================
+template <int BWD>
+__global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant__ FMaps mp, Args a) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_MISC + M_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + M_TMEM);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + M_ABORT);
+    float *cf_all = reinterpret_cast<float *>(sm + OFF_MISC + M_CF);
+
+    const int half = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int j0 = half * DVB;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = a.T, H = a.H, N = a.N;
+    const size_t ci0 = ((size_t)b * H + h) * N;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < B_NUM; ++i) mbar_init(&bar[i], (i == B_FULL0 || i == B_FULL1) ? 2 : 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, 512);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *tmem_slot;
+
+    if (warp == 0) {
+        // ================================ producer ================================
+        int issued[2] = {0, 0};
+        for (int m = 0; m < N; ++m) {
+            const int s = m & 1, t0 = m * C;
+            const int ci = (int)(ci0 + m);
+            if (m >= 2 && !mbar_wait(&bar[B_EMPTY0 + s], ((m >> 1) - 1) & 1, abort_flag)) break;
+            unsigned char *st = sm + s * STAGE;
+            if (lane == 0) {
+                mbar_arrive_tx(&bar[B_FULL0 + s], BWD ? 40960u : 65536u);
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    tma_load_2d(st + FS_WQ + p * 16384, &mp.W, 64 * p, ci * C, &bar[B_FULL0 + s]);
+                    if (!BWD) tma_load_4d(st + FS_WQ + p * 16384 + 8192, &mp.q, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
+                    tma_load_4d(st + FS_K + p * 8192, &mp.k, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
+                }
+                tma_load_2d(st + FS_UP, &mp.Ut, j0, ci * C, &bar[B_FULL0 + s]);
+                if (!BWD) tma_load_2d(st + FS_UP + 8192, &mp.P, 0, ci * C, &bar[B_FULL0 + s]);
+            }
+            chunk_factors(a.g, (size_t)ci, cf_all + s * 132, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[B_FULL0 + s]);
+            issued[s]++;
+        }
+        if (*abort_flag) {
+            volatile int dummy = 0;
+            for (int s = 0; s < 2; ++s)
+                if (issued[s] > 0) mbar_wait(&bar[B_FULL0 + s], (issued[s] - 1) & 1, &dummy, 100000000ull);
+        }
+    } else {
+        // ================================ chain ================================
+        const int wc = threadIdx.x - 32;
+        const int q4 = warp & 3, trow = q4 * 32 + lane;
+        const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
+        constexpr uint32_t TM_D = 0, TM_E = 256;  // D / O' double-buffered at 0 and 128
+        uint32_t ph = 0;
+        bool pending = false;
+        auto wabort = [&](bool ok) -> bool { return named_sync_any(2, 128, !ok || *abort_flag != 0); };
+        auto mma_done = [&]() -> bool {
+            const bool ok = mbar_wait(&bar[B_MMA], ph & 1, abort_flag);
+            ph++;
+            fence_after_sync();
+            const bool go = !wabort(ok);
+            if (go) pending = false;
+            return go;
+        };
+        const uint32_t sS = smem_u32(sm + OFF_S), sU = smem_u32(sm + OFF_U), sUD = smem_u32(sm + OFF_UD);
+        float S[DVB];
+        {
+            const float *s0 = a.S0 ? a.S0 + (((size_t)b * H + h) * DK + trow) * DV + j0 : nullptr;
+#pragma unroll
+            for (int j = 0; j < DVB; ++j) S[j] = s0 ? s0[j] : 0.f;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_S, swz(trow, ch), S + ch * 8);
+        }
+        fence_proxy_async();
+        named_sync(2, 128);
+        // o of the previous chunk is finished by lanes 64-127 while the next chunk starts
+        int prev_L = 0, prev_t0 = 0;
+        float prev_eg = 0.f;
+        uint32_t prev_buf = 0;
+        auto o_epilogue = [&]() {
+            if (BWD || trow < 64 || prev_L == 0) return;
+            const int r = trow - 64;
+            // the TMEM loads are warp-wide (.sync.aligned): every lane loads, only rows < L store
+            float d[64], p[64];
+            tmem_row64(tl + TM_D + prev_buf, d);
+            tmem_row64(tl + TM_D + prev_buf + 64, p);
+            if (r < prev_L && a.out) {
+#pragma unroll
+                for (int j = 0; j < 64; ++j) d[j] = prev_eg * d[j] + p[j];
+                st_row_global(a.out, (((size_t)b * T + prev_t0 + r) * H + h) * DV + j0, d);
+            }
+        };
+        for (int m = 0; m < N; ++m) {
+            const int s = m & 1, t0 = m * C, L = min(C, T - t0);
+            const uint32_t buf = (uint32_t)(m & 1) * 128;
+            const size_t ci = ci0 + m;
+            unsigned char *st = sm + s * STAGE;
+            const bool got = mbar_wait(&bar[B_FULL0 + s], (m >> 1) & 1, abort_flag);
+            if (wabort(got)) break;
+            // this chunk's factors, read before the stage is released
+            const float *cf = cf_all + s * 132;
+            const float egC = cf[128];
+            const float rowf = cf[trow];  // lanes 0-63: e^{gC - g_r}; lanes 64-127: e^{g_r}, r = trow - 64
+            if (BWD) st_row_global(a.Sn, (ci * DK + trow) * DV + j0, S);
+            // ---------------- D = [W ; q] S ----------------
+            if (wc == 0) {
+                fence_after_sync();
+                const uint32_t id = idesc_bf16(128, 64, 0, 1);
+                const uint32_t swq = smem_u32(st + FS_WQ);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16(tbase + TM_D + buf, sdesc(swq + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
+                             sdesc(sS + k * 2048, 1024, 1024), id, k > 0);
+                mma_commit(&bar[B_MMA]);
+            }
+            pending = true;
+            o_epilogue();  // previous chunk, lanes 64-127
+            if (!mma_done()) break;
+            // ---------------- U = U~ - W S;  u;  U and e^{gC - g} U tiles ----------------
+            if (trow < 64) {
+                const int r = trow;
+                float v[64];
+                tmem_row64(tl + TM_D + buf, v);
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    float ut[8];
+                    ld_chunk(st + FS_UP, swz(r, ch), ut);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[ch * 8 + e] = ut[e] - v[ch * 8 + e];
+                }
+                if (BWD) {
+                    st_row_global(a.Un, (ci * C + r) * DV + j0, v);
+                } else {
+                    if (a.u && r < L) st_row_global(a.u, (((size_t)b * T + t0 + r) * H + h) * DV + j0, v);
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_U, swz(r, ch), v + ch * 8);
+                }
+#pragma unroll
+                for (int j = 0; j < 64; ++j) v[j] *= rowf;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_UD, swz(r, ch), v + ch * 8);
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            if (wabort(true)) break;
+            // ---------------- E = k^T (e^{gC-g} U);  O' = [* ; P] U ----------------
+            if (wc == 0) {
+                fence_after_sync();
+                const uint32_t sk = smem_u32(st + FS_K), sup = smem_u32(st + FS_UP);
+                const uint32_t ide = idesc_bf16(128, 64, 1, 1), ido = idesc_bf16(128, 64, 0, 1);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16(tbase + TM_E, sdesc(sk + k * 2048, 8192, 1024), sdesc(sUD + k * 2048, 1024, 1024), ide,
+                             k > 0);
+                if (!BWD) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        mma_bf16(tbase + TM_D + buf + 64, sdesc(sup + k * 32, 16, 1024), sdesc(sU + k * 2048, 1024, 1024),
+                                 ido, k > 0);
+                }
+                mma_commit(&bar[B_MMA]);
+            }
+            pending = true;
+            if (!mma_done()) break;
+            if (wc == 0) mbar_arrive(&bar[B_EMPTY0 + s]);
+            // ---------------- S <- e^{gC} S + E ----------------
+            {
+                float ev[64];
+                tmem_row64(tl + TM_E, ev);
+#pragma unroll
+                for (int j = 0; j < DVB; ++j) S[j] = egC * S[j] + ev[j];
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_S, swz(trow, ch), S + ch * 8);
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            if (wabort(true)) break;
+            prev_L = L; prev_t0 = t0; prev_eg = rowf; prev_buf = buf;
+        }
+        if (*abort_flag == 0) {
+            o_epilogue();  // last chunk
+            if (!BWD && a.ST) {
+                float *dst = a.ST + (((size_t)b * H + h) * DK + trow) * DV + j0;
+#pragma unroll
+                for (int j = 0; j < DVB; j += 4)
+                    *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+            }
+        } else if (pending) {
+            volatile int dummy = 0;
+            mbar_wait(&bar[B_MMA], ph & 1, &dummy, 100000000ull);
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == 0) tmem_dealloc(tbase, 512);
+}
+
+// ====================================== reverse chain ======================================
+__global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant__ RMaps mp, Args a) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_MISC + M_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + M_TMEM);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + M_ABORT);
+    float *cf_all = reinterpret_cast<float *>(sm + OFF_MISC + M_CF);
+
+    const int half = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int j0 = half * DVB;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int H = a.H, N = a.N;
+    const size_t ci0 = ((size_t)b * H + h) * N;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < B_NUM; ++i) mbar_init(&bar[i], (i == B_FULL0 || i == B_FULL1) ? 2 : 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, 128);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *tmem_slot;
+
+    if (warp == 0) {
+        // ================================ producer ================================
+        int issued[2] = {0, 0};
+        for (int m = 0; m < N; ++m) {
+            const int mc = N - 1 - m, s = m & 1, t0 = mc * C;
+            const int ci = (int)(ci0 + mc);
+            if (m >= 2 && !mbar_wait(&bar[B_EMPTY0 + s], ((m >> 1) - 1) & 1, abort_flag)) break;
+            unsigned char *st = sm + s * STAGE;
+            if (lane == 0) {
+                mbar_arrive_tx(&bar[B_FULL0 + s], 65536u);
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    tma_load_4d(st + RS_K + p * 8192, &mp.k, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
+                    tma_load_4d(st + RS_Q + p * 8192, &mp.q, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
+                    tma_load_2d(st + RS_W + p * 8192, &mp.W, 64 * p, ci * C, &bar[B_FULL0 + s]);
+                }
+                tma_load_4d(st + RS_DO, &mp.dout, j0, h, t0, b, &bar[B_FULL0 + s]);
+                tma_load_2d(st + RS_DU, &mp.dUp, j0, ci * C, &bar[B_FULL0 + s]);
+            }
+            chunk_factors(a.g, (size_t)ci, cf_all + s * 132, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[B_FULL0 + s]);
+            issued[s]++;
+        }
+        if (*abort_flag) {
+            volatile int dummy = 0;
+            for (int s = 0; s < 2; ++s)
+                if (issued[s] > 0) mbar_wait(&bar[B_FULL0 + s], (issued[s] - 1) & 1, &dummy, 100000000ull);
+        }
+    } else {
+        // ================================ chain ================================
+        const int wc = threadIdx.x - 32;
+        const int q4 = warp & 3, trow = q4 * 32 + lane;
+        const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
+        constexpr uint32_t TM_A = 0, TM_B = 64;
+        uint32_t ph = 0;
+        bool pending = false;
+        auto wabort = [&](bool ok) -> bool { return named_sync_any(2, 128, !ok || *abort_flag != 0); };
+        auto mma_done = [&]() -> bool {
+            const bool ok = mbar_wait(&bar[B_MMA], ph & 1, abort_flag);
+            ph++;
+            fence_after_sync();
+            const bool go = !wabort(ok);
+            if (go) pending = false;
+            return go;
+        };
+        const uint32_t sS = smem_u32(sm + OFF_S), sU = smem_u32(sm + OFF_U);
+        float S[DVB];  // dL/dS of the state leaving the current chunk
+        {
+            const float *s0 = a.S0 ? a.S0 + (((size_t)b * H + h) * DK + trow) * DV + j0 : nullptr;
+#pragma unroll
+            for (int j = 0; j < DVB; ++j) S[j] = s0 ? s0[j] : 0.f;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_S, swz(trow, ch), S + ch * 8);
+        }
+        fence_proxy_async();
+        named_sync(2, 128);
+        for (int m = 0; m < N; ++m) {
+            const int mc = N - 1 - m, s = m & 1;
+            const size_t ci = ci0 + mc;
+            unsigned char *st = sm + s * STAGE;
+            const bool got = mbar_wait(&bar[B_FULL0 + s], (m >> 1) & 1, abort_flag);
+            if (wabort(got)) break;
+            const float *cf = cf_all + s * 132;
+            const float egC = cf[128];
+            st_row_global(a.dSn, (ci * DK + trow) * DV + j0, S);
+            // ---------------- D_a = k dS+  (M = 128: rows 64..127 discarded) ----------------
+            if (wc == 0) {
+                fence_after_sync();
+                const uint32_t id = idesc_bf16(128, 64, 0, 1);
+                const uint32_t sk = smem_u32(st + RS_K);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16(tbase + TM_A, sdesc(sk + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024),
+                             sdesc(sS + k * 2048, 1024, 1024), id, k > 0);
+                mma_commit(&bar[B_MMA]);
+            }
+            pending = true;
+            // dO rows scaled by e^{g_r} (for q^T diag(e^g) dO) while the MMA runs
+            for (int x = wc; x < 512; x += 128) {
+                float v[8];
+                ld_chunk(st + RS_DO, (uint32_t)x * 16, v);
+                const float f = cf[64 + (x >> 3)];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] *= f;
+                st_chunk(st + RS_DO, (uint32_t)x * 16, v);
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            if (wabort(true)) break;
+            // ---------------- D_b = q^T diag(e^g) dO  (first half of dL/dS_n) ----------------
+            if (wc == 0) {
+                fence_after_sync();
+                const uint32_t id = idesc_bf16(128, 64, 1, 1);
+                const uint32_t sq = smem_u32(st + RS_Q), sdo = smem_u32(st + RS_DO);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16(tbase + TM_B, sdesc(sq + k * 2048, 8192, 1024), sdesc(sdo + k * 2048, 1024, 1024), id,
+                             k > 0);
+            }
+            if (!mma_done()) break;
+            // ---------------- dU = (du + P^T dO) + diag(e^{gC - g}) D_a ----------------
+            if (trow < 64) {
+                const int r = trow;
+                const float f = cf[r];
+                float v[64];
+                tmem_row64(tl + TM_A, v);
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    float d[8];
+                    ld_chunk(st + RS_DU, swz(r, ch), d);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[ch * 8 + e] = d[e] + f * v[ch * 8 + e];
+                }
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_U, swz(r, ch), v + ch * 8);
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            if (wabort(true)) break;
+            // ---------------- D_b -= W^T dU ----------------
+            if (wc == 0) {
+                fence_after_sync();
+                const uint32_t id = idesc_bf16(128, 64, 1, 1, 1);
+                const uint32_t sw = smem_u32(st + RS_W);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16(tbase + TM_B, sdesc(sw + k * 2048, 8192, 1024), sdesc(sU + k * 2048, 1024, 1024), id, 1);
+                mma_commit(&bar[B_MMA]);
+            }
+            pending = true;
+            if (!mma_done()) break;
+            if (wc == 0) mbar_arrive(&bar[B_EMPTY0 + s]);
+            // ---------------- dS_n = e^{gC} dS+ + D_b ----------------
+            {
+                float dv[64];
+                tmem_row64(tl + TM_B, dv);
+#pragma unroll
+                for (int j = 0; j < DVB; ++j) S[j] = egC * S[j] + dv[j];
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_S, swz(trow, ch), S + ch * 8);
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            if (wabort(true)) break;
+        }
+        if (*abort_flag == 0) {
+            if (a.ST) {
+                float *dst = a.ST + (((size_t)b * H + h) * DK + trow) * DV + j0;
+#pragma unroll
+                for (int j = 0; j < DVB; j += 4)
+                    *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+            }
+        } else if (pending) {
+            volatile int dummy = 0;
+            mbar_wait(&bar[B_MMA], ph & 1, &dummy, 100000000ull);
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == 0) tmem_dealloc(tbase, 128);
+}
+
+}  // namespace tch
+
+bool tc_split_supported(const Geo &g, bool bf16) {
+    return bf16 && g.C == 64 && g.dk == 128 && g.dv == 128 && g.variant != VAR_KDA &&
+           (size_t)g.B * g.H * g.N * 128 <= (size_t)INT_MAX;
+}
+
+static size_t ws_al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Carves the split-path workspace from base; returns the bytes it spans.
+static size_t ws_carve(const Geo &g, bool bwd, char *base, TcWs *w) {
+    const size_t nc = (size_t)g.B * g.H * g.N, C = g.C, DK = g.dk, DV = g.dv;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { char *r = base ? base + off : nullptr; off += ws_al256(bytes); return r; };
+    *w = TcWs{};
+    w->g = (float *)take(nc * C * 4);
+    w->W = (__nv_bfloat16 *)take(nc * C * DK * 2);
+    w->Ut = (__nv_bfloat16 *)take(nc * C * DV * 2);
+    w->P = (__nv_bfloat16 *)take(nc * C * C * 2);
+    if (bwd) {
+        w->Tn = (__nv_bfloat16 *)take(nc * C * C * 2);
+        w->KK = (__nv_bfloat16 *)take(nc * C * C * 2);
+        w->dUp = (__nv_bfloat16 *)take(nc * C * DV * 2);
+        w->Sn = (__nv_bfloat16 *)take(nc * DK * DV * 2);
+        w->dSn = (__nv_bfloat16 *)take(nc * DK * DV * 2);
+        w->Un = (__nv_bfloat16 *)take(nc * C * DV * 2);
+    }
+    return off;
+}
+
+size_t tc_ws_bytes(const Geo &g, bool bwd) {
+    TcWs w;
+    return ws_carve(g, bwd, nullptr, &w);
+}
+
+TcWs tc_ws_carve(const Geo &g, bool bwd, void *base) {
+    TcWs w;
+    ws_carve(g, bwd, (char *)base, &w);
+    return w;
+}
+
+cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, bool bwd, cudaStream_t s, Rec &rec) {
+    using namespace tch;
+    FMaps mp;
+    const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;
+    const bool ok = tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) &&
+                    tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64) &&
+                    tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.Ut, w.Ut, DV, NC * C, 64) &&
+                    tc::make_map_2d_bf16(&mp.P, w.P, C, NC * C, 64);
+    if (!ok) return cudaErrorInvalidValue;
+    Args a = {};
+    a.g = w.g; a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
+    a.S0 = t.S0;
+    if (bwd) {
+        a.Sn = w.Sn; a.Un = w.Un;
+    } else {
+        a.out = t.out; a.u = t.u; a.ST = t.S_T;
+    }
+    const size_t smem = SMEM_BYTES + 1024;
+    const dim3 grid(DV / DVB, g.H, g.B);
+    cudaError_t e;
+    if (bwd) {
+        e = cudaFuncSetAttribute(k_chain_fwd<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        rec.mark(s);
+        k_chain_fwd<1><<<grid, NTHREADS, smem, s>>>(mp, a);
+    } else {
+        e = cudaFuncSetAttribute(k_chain_fwd<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        rec.mark(s);
+        k_chain_fwd<0><<<grid, NTHREADS, smem, s>>>(mp, a);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t tc_chain_rev(const Geo &g, const Tensors &t, const TcWs &w, cudaStream_t s, Rec &rec) {
+    using namespace tch;
+    RMaps mp;
+    const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;
+    const bool ok = tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) &&
+                    tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64) &&
+                    tc::make_map_4d_bf16(&mp.dout, t.dout, DV, H, T, Bn, 64) &&
+                    tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.dUp, w.dUp, DV, NC * C, 64);
+    if (!ok) return cudaErrorInvalidValue;
+    Args a = {};
+    a.g = w.g; a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
+    a.S0 = t.dS_T; a.ST = t.dS0; a.dSn = w.dSn;
+    const size_t smem = SMEM_BYTES + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_chain_rev, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    rec.mark(s);
+    k_chain_rev<<<dim3(DV / DVB, g.H, g.B), NTHREADS, smem, s>>>(mp, a);
+    return cudaGetLastError();
+}
+
+}  // namespace dr

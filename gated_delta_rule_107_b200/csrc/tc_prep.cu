@@ -1,0 +1,378 @@
+// tc_prep.cu -- the per-chunk products of the chunked gated delta rule, one CTA per chunk
+// (Gated DeltaNet and DeltaNet; bf16 I/O, dk = dv = 128, C = 64).
+//
+// Chunked form of "线性注意力架构演进与Kimi Delta Attention创新实践" (sections 2.1, 6.1,
+// 6.2, 7.1).  With g the in-chunk cumulative log gate:
+//
+//   P1   [k ; q] . k^T                        -> k.k^T (rows 0-63), q.k^T (rows 64-127)
+//        A = beta_r e^{g_r - g_i} k_r.k_i (i < r),   P = e^{g_r - g_i} q_r.k_i (i <= r)
+//   T  = (I + A)^-1                            (the UT transform; tc_inverse.cuh)
+//   W  = T diag(beta e^g) k,   U~ = T diag(beta) v
+//   backward only:  dU' = du + P^T dO, and T, k k^T kept for the gradient kernel.
+//
+// Every chunk is independent, so the grid covers all chunks of all heads at once (two
+// CTAs per SM); the serial state chains (tc_chain.cu) then only carry the state.  The
+// products leave as bf16 tiles through TMA stores (W, U~, P, dU') or row stores (T, k k^T),
+// and g as fp32.  The products with 64 rows use M = 128 MMAs whose rows 64..127 read
+// other (valid) shared memory and are discarded.
+#include "tc_host.cuh"
+#include "tc_inverse.cuh"
+#include "tc_path.cuh"
+#include "tc_ptx.cuh"
+#include "tc_tile.cuh"
+
+namespace dr {
+namespace tcp {
+
+using namespace dr::tc;
+using dr::tcf::ld_chunk;
+using dr::tcf::st_chunk;
+using dr::tcf::st8_global;
+using dr::tcf::st_row_global;
+using dr::tcf::tmem_row64;
+
+constexpr int C = 64, DK = 128, DV = 128;
+constexpr int NTHREADS = 128;
+// shared memory (bytes from a 1024-aligned base)
+constexpr uint32_t OFF_KQ = 0;         // 32K [k_p0 | q_p0 | k_p1 | q_p1]; after P1: q_p0 -> T diag(beta),
+                                       //     q_p1 -> inverse scratch, then T diag(beta e^g)
+constexpr uint32_t OFF_V = 32768;      // 16K v [i][j]
+constexpr uint32_t OFF_F = 49152;      // 32K fp32 A | T (inverse), then staging W [r][c] | U~ [r][j]
+constexpr uint32_t OFF_P = 81920;      //  8K P [r][i]
+constexpr uint32_t OFF_DO = 90112;     // 16K dO [r][j] -> staging dU' [r][j]   (backward)
+__host__ __device__ constexpr uint32_t misc_off(int bwd) { return bwd ? 106496u : 90112u; }
+__host__ __device__ constexpr uint32_t smem_bytes(int bwd) { return misc_off(bwd) + 2048; }
+// misc
+constexpr uint32_t M_BAR = 0;          // [0] loads, [1] MMA
+constexpr uint32_t M_TMEM = 64, M_ABORT = 68, M_BIG = 72;
+constexpr uint32_t M_PF = 256;         // gate factors [6][64]
+enum { PF_GC = 0, PF_ROWP, PF_COLA, PF_BV, PF_BK, PF_NUM };
+static_assert(M_PF + PF_NUM * 256 <= 2048, "misc overflow");
+// TMEM columns
+constexpr uint32_t TM_G1 = 0, TM_XW = 0, TM_XU = 128, TM_DU = 128, TM_COLS = 256;
+
+struct Maps {
+    CUtensorMap q, k, v, dout;  // [B, T, H, 128] bf16; box 64 channels x 64 tokens
+    CUtensorMap W, Ut, dUp;     // [chunks * 64][128] bf16; box 64 x 64 (stores)
+    CUtensorMap P;              // [chunks * 64][64] bf16; box 64 x 64 (store)
+};
+
+struct Args {
+    const void *alpha, *beta, *du;  // bf16 [B, T, H] / [B, T, H, 128]
+    float *g;                       // [chunks][64]
+    __nv_bfloat16 *KK, *Tn;         // [chunks][64][64] (backward)
+    int B, T, H, N;
+};
+
+template <int VAR, int BWD>
+__global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constant__ Maps mp, Args a) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    unsigned char *misc = sm + misc_off(BWD);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(misc + M_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + M_TMEM);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + M_ABORT);
+    volatile int *bigflag = reinterpret_cast<volatile int *>(misc + M_BIG);
+    float *pf = reinterpret_cast<float *>(misc + M_PF);
+
+    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int T = a.T, H = a.H, t0 = n * C, L = min(C, T - t0);
+    const int ci = (b * H + h) * a.N + n;  // < 2^31 / 128 (checked by the launcher)
+    const int trow = tid;                  // TMEM lane of this thread
+
+    int mma_issued = 0;
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        mbar_arrive_tx(&bar[0], 49152u + (BWD ? 16384u : 0u));
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            tma_load_4d(sm + OFF_KQ + p * 16384, &mp.k, 64 * p, h, t0, b, &bar[0]);
+            tma_load_4d(sm + OFF_KQ + p * 16384 + 8192, &mp.q, 64 * p, h, t0, b, &bar[0]);
+            tma_load_4d(sm + OFF_V + p * 8192, &mp.v, 64 * p, h, t0, b, &bar[0]);
+            if (BWD) tma_load_4d(sm + OFF_DO + p * 8192, &mp.dout, 64 * p, h, t0, b, &bar[0]);
+        }
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, TM_COLS);
+    if (warp == 1) {
+        // in-chunk cumulative log gate (lane owns rows lane and lane + 32) and the factors
+        float lg[2], bt[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int r = lane + 32 * hh;
+            const size_t row = ((size_t)b * T + t0 + r) * H + h;
+            lg[hh] = 0.f;
+            bt[hh] = 0.f;
+            if (r < L) {
+                if (VAR == VAR_GATED) lg[hh] = tcf::bf(a.alpha, row);
+                bt[hh] = tcf::bf(a.beta, row);
+            }
+        }
+        float x0 = lg[0], x1 = lg[1];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y0 = __shfl_up_sync(0xffffffffu, x0, o);
+            const float y1 = __shfl_up_sync(0xffffffffu, x1, o);
+            if (lane >= o) { x0 += y0; x1 += y1; }
+        }
+        x1 += __shfl_sync(0xffffffffu, x0, 31);
+        const float gm = __shfl_sync(0xffffffffu, x0, 31);  // midpoint of the chunk
+        float dev = fmaxf(fabsf(x0 - gm), fabsf(x1 - gm));
+        dev = fmaxf(dev, __shfl_xor_sync(0xffffffffu, dev, 16));
+        dev = fmaxf(dev, __shfl_xor_sync(0xffffffffu, dev, 8));
+        dev = fmaxf(dev, __shfl_xor_sync(0xffffffffu, dev, 4));
+        dev = fmaxf(dev, __shfl_xor_sync(0xffffffffu, dev, 2));
+        dev = fmaxf(dev, __shfl_xor_sync(0xffffffffu, dev, 1));
+        const float xs[2] = {x0, x1};
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int r = lane + 32 * hh;
+            const float x = xs[hh];
+            pf[PF_GC * 64 + r] = x;
+            pf[PF_ROWP * 64 + r] = __expf(x - gm);
+            pf[PF_COLA * 64 + r] = __expf(gm - x);
+            pf[PF_BV * 64 + r] = bt[hh];
+            pf[PF_BK * 64 + r] = bt[hh] * __expf(x);
+            a.g[(size_t)ci * C + r] = x;
+        }
+        if (lane == 0) *bigflag = dev > 80.f;
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);
+    auto sync = [&]() { named_sync(1, NTHREADS); };
+    auto consensus = [&](bool ok) -> bool { return !named_sync_any(1, NTHREADS, !ok || *abort_flag != 0); };
+    uint32_t ph = 0;
+    auto wait_mma = [&]() -> bool {
+        const bool ok = mbar_wait(&bar[1], ph & 1, abort_flag);
+        ph++;
+        fence_after_sync();
+        return ok;
+    };
+    float *Asc = reinterpret_cast<float *>(sm + OFF_F);
+    float *Tf = Asc + 4096;
+    float *ysc = reinterpret_cast<float *>(sm + OFF_KQ + 24576);  // q_p1, free after P1
+    const uint32_t skq = smem_u32(sm + OFF_KQ), sv = smem_u32(sm + OFF_V), sp = smem_u32(sm + OFF_P);
+    const uint32_t sdo = smem_u32(sm + OFF_DO);
+
+    bool ok = consensus(mbar_wait(&bar[0], 0, abort_flag));
+    // ---------------- P1: [k ; q] . k^T ----------------
+    if (ok && tid == 0) {
+        const uint32_t id = idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+        for (int st = 0; st < 8; ++st) {
+            const uint32_t ad = skq + (st >> 2) * 16384 + (st & 3) * 32;
+            mma_bf16(tbase + TM_G1, sdesc(ad, 16, 1024), sdesc(ad, 16, 1024), id, st > 0);
+        }
+        mma_commit(&bar[1]);
+        mma_issued++;
+    }
+    if (ok) ok = consensus(wait_mma());
+    // ---------------- A (fp32, for the inverse), P (bf16 tile), k k^T ----------------
+    if (ok) {
+        float g1[64];
+        tmem_row64(tl + TM_G1, g1);
+        const bool big = *bigflag != 0;
+        const float *gc = pf + PF_GC * 64, *cola = pf + PF_COLA * 64;
+        const bool arow = trow < 64;
+        const int r = arow ? trow : trow - 64;
+        // gate factor of each (r, i): e^{g_r - g_i}, split at the midpoint unless the range is large
+        float f[64];
+        if (VAR == VAR_DELTANET) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) f[i] = 1.f;
+        } else if (!big) {
+            const float rf = pf[PF_ROWP * 64 + r];
+#pragma unroll
+            for (int i4 = 0; i4 < 16; ++i4) {
+                const float4 c = reinterpret_cast<const float4 *>(cola)[i4];
+                f[4 * i4] = c.x * rf; f[4 * i4 + 1] = c.y * rf; f[4 * i4 + 2] = c.z * rf; f[4 * i4 + 3] = c.w * rf;
+            }
+        } else {
+            const float gr = gc[r];
+#pragma unroll
+            for (int i = 0; i < 64; ++i) f[i] = (i <= r) ? __expf(gr - gc[i]) : 0.f;
+        }
+        if (arow) {
+            if (BWD) st_row_global(a.KK, ((size_t)ci * C + r) * C, g1);
+            const float br = pf[PF_BV * 64 + r];
+#pragma unroll
+            for (int i4 = 0; i4 < 16; ++i4) {
+                float4 v;
+                v.x = (4 * i4 + 0 < r) ? g1[4 * i4 + 0] * f[4 * i4 + 0] * br : 0.f;
+                v.y = (4 * i4 + 1 < r) ? g1[4 * i4 + 1] * f[4 * i4 + 1] * br : 0.f;
+                v.z = (4 * i4 + 2 < r) ? g1[4 * i4 + 2] * f[4 * i4 + 2] * br : 0.f;
+                v.w = (4 * i4 + 3 < r) ? g1[4 * i4 + 3] * f[4 * i4 + 3] * br : 0.f;
+                *reinterpret_cast<float4 *>(&Asc[sw64(r, 4 * i4)]) = v;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) g1[i] = (i <= r) ? g1[i] * f[i] : 0.f;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_P, swz(r, ch), g1 + ch * 8);
+        }
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    ok = consensus(ok);
+    if (ok && tid == 0) {
+        fence_after_sync();
+        tma_store_2d(&mp.P, sm + OFF_P, 0, ci * C);
+        bulk_commit();
+        if (BWD) {  // dU' = P^T dO  (M = 128: rows 64..127 read dO and are discarded)
+            const uint32_t id = idesc_bf16(128, 128, 1, 1);
+#pragma unroll
+            for (int st = 0; st < 4; ++st)
+                mma_bf16(tbase + TM_DU, sdesc(sp + st * 2048, 8192, 1024), sdesc(sdo + st * 2048, 8192, 1024), id,
+                         st > 0);
+            mma_commit(&bar[1]);
+            mma_issued++;
+        }
+    }
+    // ---------------- T = (I + A)^-1 ----------------
+    if (ok) unit_lower_inverse64(Asc, Tf, ysc, tid, sync);
+    if (BWD && ok) {
+        ok = consensus(wait_mma());
+        // dU' = du + P^T dO -> staging tile in place of dO (rows 0..63 of the accumulator)
+        if (ok && trow < 64) {
+            const int r = trow;
+            const bool live = a.du != nullptr && r < L;
+            const __nv_bfloat16 *dur =
+                reinterpret_cast<const __nv_bfloat16 *>(a.du) + (((size_t)b * T + t0 + r) * H + h) * DV;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float v[64];
+                tmem_row64(tl + TM_DU + hh * 64, v);
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    if (live) {
+                        float d[8];
+                        const uint4 w = *reinterpret_cast<const uint4 *>(dur + hh * 64 + ch * 8);
+                        d[0] = bf16_lo(w.x); d[1] = bf16_hi(w.x); d[2] = bf16_lo(w.y); d[3] = bf16_hi(w.y);
+                        d[4] = bf16_lo(w.z); d[5] = bf16_hi(w.z); d[6] = bf16_lo(w.w); d[7] = bf16_hi(w.w);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v[ch * 8 + e] += d[e];
+                    }
+                    st_chunk(sm + OFF_DO, (uint32_t)hh * 8192 + swz(r, ch), v + ch * 8);
+                }
+            }
+        }
+    }
+    // ---------------- T diag(beta), T diag(beta e^g) tiles; T itself (backward) ----------------
+    if (ok) {
+        const int i = tid & 63;
+        const float *fac = pf + (tid < 64 ? PF_BV : PF_BK) * 64;
+        unsigned char *dst = sm + OFF_KQ + (tid < 64 ? 8192 : 24576);
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+            const float4 lo = *reinterpret_cast<const float4 *>(&Tf[sw64(i, ch * 8)]);
+            const float4 hi = *reinterpret_cast<const float4 *>(&Tf[sw64(i, ch * 8 + 4)]);
+            float w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w[e] = (ch * 8 + e <= i) ? w[e] : 0.f;
+            if (BWD && tid < 64) st8_global(a.Tn, ((size_t)ci * C + i) * C + ch * 8, w);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w[e] *= fac[ch * 8 + e];
+            st_chunk(dst, swz(i, ch), w);
+        }
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    ok = consensus(ok);
+    // ---------------- W = [T diag(beta e^g) ; *] k,  U~ = [T diag(beta) ; *] v ----------------
+    if (ok && tid == 0) {
+        fence_after_sync();
+        if (BWD) {
+            tma_store_2d(&mp.dUp, sm + OFF_DO, 0, ci * C);
+            tma_store_2d(&mp.dUp, sm + OFF_DO + 8192, 64, ci * C);
+            bulk_commit();
+        }
+        const uint32_t id = idesc_bf16(128, 128, 0, 1);
+#pragma unroll
+        for (int st = 0; st < 4; ++st) {
+            mma_bf16(tbase + TM_XW, sdesc(skq + 24576 + st * 32, 16, 1024), sdesc(skq + st * 2048, 16384, 1024), id,
+                     st > 0);
+            mma_bf16(tbase + TM_XU, sdesc(skq + 8192 + st * 32, 16, 1024), sdesc(sv + st * 2048, 8192, 1024), id,
+                     st > 0);
+        }
+        mma_commit(&bar[1]);
+        mma_issued++;
+    }
+    if (ok) ok = consensus(wait_mma());
+    if (ok && trow < 64) {
+        const int r = trow;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {  // W panels 0, 1, then U~ panels 0, 1
+            float v[64];
+            tmem_row64(tl + (x < 2 ? TM_XW : TM_XU) + (x & 1) * 64, v);
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_F, (uint32_t)x * 8192 + swz(r, ch), v + ch * 8);
+        }
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    ok = consensus(ok);
+    if (tid == 0) {
+        if (ok) {
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                tma_store_2d(&mp.W, sm + OFF_F + p * 8192, 64 * p, ci * C);
+                tma_store_2d(&mp.Ut, sm + OFF_F + 16384 + p * 8192, 64 * p, ci * C);
+            }
+            bulk_commit();
+        }
+        bulk_wait_all();
+        if (*abort_flag) {  // let whatever was issued finish before the CTA leaves
+            volatile int dummy = 0;
+            mbar_wait(&bar[0], 0, &dummy, 100000000ull);
+            if (mma_issued > 0) mbar_wait(&bar[1], (mma_issued - 1) & 1, &dummy, 100000000ull);
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == 0) tmem_dealloc(tbase, TM_COLS);
+}
+
+template <int VAR, int BWD>
+static cudaError_t launch_prep(const Maps &mp, const Args &a, dim3 grid, cudaStream_t s, Rec &rec) {
+    const size_t smem = smem_bytes(BWD) + 1024;
+    cudaError_t e =
+        cudaFuncSetAttribute(k_chunk_prep<VAR, BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    rec.mark(s);
+    k_chunk_prep<VAR, BWD><<<grid, NTHREADS, smem, s>>>(mp, a);
+    return cudaGetLastError();
+}
+
+}  // namespace tcp
+
+cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool bwd, cudaStream_t s, Rec &rec) {
+    using namespace tcp;
+    Maps mp;
+    const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;
+    bool ok = tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) && tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64) &&
+              tc::make_map_4d_bf16(&mp.v, t.v, DV, H, T, Bn, 64) && tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) &&
+              tc::make_map_2d_bf16(&mp.Ut, w.Ut, DV, NC * C, 64) && tc::make_map_2d_bf16(&mp.P, w.P, C, NC * C, 64);
+    if (ok && bwd)
+        ok = tc::make_map_4d_bf16(&mp.dout, t.dout, DV, H, T, Bn, 64) &&
+             tc::make_map_2d_bf16(&mp.dUp, w.dUp, DV, NC * C, 64);
+    else
+        mp.dout = mp.v, mp.dUp = mp.W;
+    if (!ok) return cudaErrorInvalidValue;
+    Args a;
+    a.alpha = t.alpha; a.beta = t.beta; a.du = bwd ? t.du : nullptr; a.g = w.g; a.KK = w.KK; a.Tn = w.Tn;
+    a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
+    const dim3 grid(g.N, g.H, g.B);
+    if (g.variant == VAR_GATED)
+        return bwd ? launch_prep<VAR_GATED, 1>(mp, a, grid, s, rec) : launch_prep<VAR_GATED, 0>(mp, a, grid, s, rec);
+    return bwd ? launch_prep<VAR_DELTANET, 1>(mp, a, grid, s, rec) : launch_prep<VAR_DELTANET, 0>(mp, a, grid, s, rec);
+}
+
+}  // namespace dr

@@ -31,6 +31,22 @@ __device__ __forceinline__ void ld_chunk(const unsigned char *base, uint32_t off
     v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
 }
 
+// 8 values as bf16 at element offset elem_off (a multiple of 8) of a bf16 array in global memory
+__device__ __forceinline__ void st8_global(void *base, size_t elem_off, const float *v) {
+    uint4 w;
+    w.x = pack_bf16(v[0], v[1]);
+    w.y = pack_bf16(v[2], v[3]);
+    w.z = pack_bf16(v[4], v[5]);
+    w.w = pack_bf16(v[6], v[7]);
+    *reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(base) + elem_off) = w;
+}
+
+// 64 values as bf16 at element offset elem_off (a multiple of 8) of a bf16 array in global memory
+__device__ __forceinline__ void st_row_global(void *base, size_t elem_off, const float *v) {
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) st8_global(base, elem_off + ch * 8, v + ch * 8);
+}
+
 // 64 fp32 columns of this thread's TMEM lane
 __device__ __forceinline__ void tmem_row64(uint32_t taddr, float *v) {
     tmem_ld16(taddr + 0, v);
