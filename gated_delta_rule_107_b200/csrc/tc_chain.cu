@@ -3,7 +3,7 @@
 //
 // Chunked form of "线性注意力架构演进与Kimi Delta Attention创新实践" (sections 2.1, 6.1,
 // 6.2, 7.1), given the per-chunk products of tc_prep.cu (W, U~, P, g, and for the backward
-// du + P^T dO).  One CTA per (b, h, 64 value channels) walks the chunks in order; the state
+// P^T dO).  One CTA per (b, h, 64 value channels) walks the chunks in order; the state
 // block (128 key rows x 64 value columns) stays in fp32 registers, one row per thread, with a
 // bf16 copy in shared memory as the MMA operand.
 //
@@ -14,8 +14,9 @@
 //   o  = diag(e^g) q S + O'
 //   S_{n+1} = e^{g_C} S + k^T (e^{g_C - g} U)
 // Reverse chain, chunk n from last to first, dS+ = dL/dS_{n+1}:
-//   dU = (du + P^T dO) + diag(e^{g_C - g}) k dS+
+//   dU = du + P^T dO + diag(e^{g_C - g}) k dS+         (stored: the gradient kernel reads it)
 //   dL/dS_n = e^{g_C} dS+ + q^T diag(e^g) dO - W^T dU
+//   and the row sums U_r . (diag(e^{g_C - g}) k dS+)_r of its 64 columns (a term of d log alpha)
 //
 // Warp 0 is a TMA producer that keeps two chunks of operands in flight; warps 1-4 run the
 // chain (thread = TMEM lane = state row).  Every wait is bounded (~1 s) and aborts are
@@ -38,12 +39,13 @@ using dr::tcf::tmem_row64;
 
 constexpr int C = 64, DK = 128, DV = 128, DVB = 64;
 constexpr int NTHREADS = 160;
-// shared memory (bytes from a 1024-aligned base): two stages of 64K, then the chain's tiles
-constexpr uint32_t STAGE = 65536;
+// shared memory (bytes from a 1024-aligned base): two stages of 80K, then the chain's tiles
+constexpr uint32_t STAGE = 81920;
 // forward stage: [W_p0 | q_p0 | W_p1 | q_p1], [U~ (this CTA's 64 columns) | P], [k_p0 | k_p1]
 constexpr uint32_t FS_WQ = 0, FS_UP = 32768, FS_K = 49152;
-// reverse stage: k, q, W (2 panels each), dO and du + P^T dO (this CTA's 64 columns)
-constexpr uint32_t RS_K = 0, RS_Q = 16384, RS_W = 32768, RS_DO = 49152, RS_DU = 57344;
+// reverse stage: k, q, W (2 panels each); dO, P^T dO, du, U (this CTA's 64 columns)
+constexpr uint32_t RS_K = 0, RS_Q = 16384, RS_W = 32768, RS_DO = 49152, RS_DU = 57344, RS_DX = 65536,
+                   RS_UN = 73728;
 constexpr uint32_t OFF_S = 2 * STAGE;         // 16K  bf16 state [c][j]
 constexpr uint32_t OFF_U = OFF_S + 16384;     //  8K  U [r][j]        (reverse: dU [r][j])
 constexpr uint32_t OFF_UD = OFF_U + 8192;     //  8K  e^{g_C - g} U [r][j]
@@ -62,22 +64,24 @@ struct FMaps {
     CUtensorMap P;      // [chunks * 64][64] bf16; box 64 x 64
 };
 struct RMaps {
-    CUtensorMap q, k, dout;  // [B, T, H, 128] bf16
-    CUtensorMap W, dUp;      // [chunks * 64][128] bf16
+    CUtensorMap q, k, dout, du;  // [B, T, H, 128] bf16
+    CUtensorMap W, dUp, Un;      // [chunks * 64][128] bf16 (loads)
+    CUtensorMap dUn;             // [chunks * 64][128] bf16 (store)
 };
 struct Args {
-    const float *g;           // [chunks][64]
+    const float *gb;          // [chunks][2][64]: g, beta
     const float *S0;          // forward: S0; reverse: dS_T (fp32 [B, H, 128, 128], may be null)
     float *ST;                // forward: S_T; reverse: dS0 (may be null)
     void *out, *u;            // forward outputs (bf16 [B, T, H, 128])
     __nv_bfloat16 *Sn, *Un;   // recompute outputs
-    __nv_bfloat16 *dSn;       // reverse output
-    int B, T, H, N;
+    __nv_bfloat16 *dSn;       // reverse outputs
+    float *skt;
+    int B, T, H, N, has_du;
 };
 
 // Producer side: the gate factors of chunk ci into cf (e^{g_C - g}, e^g, e^{g_C}).
-__device__ __forceinline__ void chunk_factors(const float *g, size_t ci, float *cf, int lane) {
-    const float *gg = g + ci * C;
+__device__ __forceinline__ void chunk_factors(const float *gb, size_t ci, float *cf, int lane) {
+    const float *gg = gb + ci * 2 * C;
     const float gC = gg[C - 1];
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -136,7 +140,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
                 tma_load_2d(st + FS_UP, &mp.Ut, j0, ci * C, &bar[B_FULL0 + s]);
                 if (!BWD) tma_load_2d(st + FS_UP + 8192, &mp.P, 0, ci * C, &bar[B_FULL0 + s]);
             }
-            chunk_factors(a.g, (size_t)ci, cf_all + s * 132, lane);
+            chunk_factors(a.gb, (size_t)ci, cf_all + s * 132, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[B_FULL0 + s]);
             issued[s]++;
@@ -202,7 +206,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             const float *cf = cf_all + s * 132;
             const float egC = cf[128];
             const float rowf = cf[trow];  // lanes 0-63: e^{gC - g_r}; lanes 64-127: e^{g_r}, r = trow - 64
-            if (BWD) st_row_global(a.Sn, (ci * DK + trow) * DV + j0, S);
             // ---------------- D = [W ; q] S ----------------
             if (wc == 0) {
                 fence_after_sync();
@@ -215,6 +218,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
                 mma_commit(&bar[B_MMA]);
             }
             pending = true;
+            if (BWD) st_row_global(a.Sn, (ci * DK + trow) * DV + j0, S);  // state entering chunk m
             o_epilogue();  // previous chunk, lanes 64-127
             if (!mma_done()) break;
             // ---------------- U = U~ - W S;  u;  U and e^{gC - g} U tiles ----------------
@@ -333,7 +337,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
             if (m >= 2 && !mbar_wait(&bar[B_EMPTY0 + s], ((m >> 1) - 1) & 1, abort_flag)) break;
             unsigned char *st = sm + s * STAGE;
             if (lane == 0) {
-                mbar_arrive_tx(&bar[B_FULL0 + s], 65536u);
+                mbar_arrive_tx(&bar[B_FULL0 + s], 73728u + (a.has_du ? 8192u : 0u));
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
                     tma_load_4d(st + RS_K + p * 8192, &mp.k, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
@@ -342,8 +346,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
                 }
                 tma_load_4d(st + RS_DO, &mp.dout, j0, h, t0, b, &bar[B_FULL0 + s]);
                 tma_load_2d(st + RS_DU, &mp.dUp, j0, ci * C, &bar[B_FULL0 + s]);
+                if (a.has_du) tma_load_4d(st + RS_DX, &mp.du, j0, h, t0, b, &bar[B_FULL0 + s]);
+                tma_load_2d(st + RS_UN, &mp.Un, j0, ci * C, &bar[B_FULL0 + s]);
             }
-            chunk_factors(a.g, (size_t)ci, cf_all + s * 132, lane);
+            chunk_factors(a.gb, (size_t)ci, cf_all + s * 132, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[B_FULL0 + s]);
             issued[s]++;
@@ -389,7 +395,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
             if (wabort(got)) break;
             const float *cf = cf_all + s * 132;
             const float egC = cf[128];
-            st_row_global(a.dSn, (ci * DK + trow) * DV + j0, S);
             // ---------------- D_a = k dS+  (M = 128: rows 64..127 discarded) ----------------
             if (wc == 0) {
                 fence_after_sync();
@@ -402,6 +407,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
                 mma_commit(&bar[B_MMA]);
             }
             pending = true;
+            st_row_global(a.dSn, (ci * DK + trow) * DV + j0, S);
+            // the dU tile of the previous chunk has been read by its TMA store
+            if (wc == 0) bulk_wait_read_all();
             // dO rows scaled by e^{g_r} (for q^T diag(e^g) dO) while the MMA runs
             for (int x = wc; x < 512; x += 128) {
                 float v[8];
@@ -425,26 +433,43 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
                              k > 0);
             }
             if (!mma_done()) break;
-            // ---------------- dU = (du + P^T dO) + diag(e^{gC - g}) D_a ----------------
+            // ---------------- dU = du + P^T dO + diag(e^{gC - g}) D_a;  U_r . (Kbar dS+)_r ----------------
             if (trow < 64) {
                 const int r = trow;
                 const float f = cf[r];
-                float v[64];
-                tmem_row64(tl + TM_A, v);
+                float rs = 0.f;
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    float d[8];
-                    ld_chunk(st + RS_DU, swz(r, ch), d);
+                for (int hh = 0; hh < 2; ++hh) {  // 32 columns at a time
+                    float v[32];
+                    tmem_ld16(tl + TM_A + hh * 32, v);
+                    tmem_ld16(tl + TM_A + hh * 32 + 16, v + 16);
+                    wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) v[ch * 8 + e] = d[e] + f * v[ch * 8 + e];
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const int ch = hh * 4 + c4;
+                        float d[8], x[8], un[8];
+                        ld_chunk(st + RS_DU, swz(r, ch), d);
+                        ld_chunk(st + RS_UN, swz(r, ch), un);
+                        if (a.has_du) {
+                            ld_chunk(st + RS_DX, swz(r, ch), x);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) d[e] += x[e];
+                        }
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float kd = f * v[c4 * 8 + e];
+                            rs += un[e] * kd;
+                            d[e] += kd;
+                        }
+                        st_chunk(sm + OFF_U, swz(r, ch), d);
+                    }
                 }
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_U, swz(r, ch), v + ch * 8);
+                a.skt[ci * 2 * C + half * C + r] = rs;
             }
             fence_proxy_async();
             fence_before_sync();
             if (wabort(true)) break;
-            // ---------------- D_b -= W^T dU ----------------
+            // ---------------- D_b -= W^T dU;  dU out ----------------
             if (wc == 0) {
                 fence_after_sync();
                 const uint32_t id = idesc_bf16(128, 64, 1, 1, 1);
@@ -453,6 +478,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
                 for (int k = 0; k < 4; ++k)
                     mma_bf16(tbase + TM_B, sdesc(sw + k * 2048, 8192, 1024), sdesc(sU + k * 2048, 1024, 1024), id, 1);
                 mma_commit(&bar[B_MMA]);
+                tma_store_2d(&mp.dUn, sm + OFF_U, j0, (int)ci * C);
+                bulk_commit();
             }
             pending = true;
             if (!mma_done()) break;
@@ -470,6 +497,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
             fence_before_sync();
             if (wabort(true)) break;
         }
+        if (wc == 0) bulk_wait_all();
         if (*abort_flag == 0) {
             if (a.ST) {
                 float *dst = a.ST + (((size_t)b * H + h) * DK + trow) * DV + j0;
@@ -503,7 +531,7 @@ static size_t ws_carve(const Geo &g, bool bwd, char *base, TcWs *w) {
     size_t off = 0;
     auto take = [&](size_t bytes) { char *r = base ? base + off : nullptr; off += ws_al256(bytes); return r; };
     *w = TcWs{};
-    w->g = (float *)take(nc * C * 4);
+    w->gb = (float *)take(nc * 2 * C * 4);
     w->W = (__nv_bfloat16 *)take(nc * C * DK * 2);
     w->Ut = (__nv_bfloat16 *)take(nc * C * DV * 2);
     w->P = (__nv_bfloat16 *)take(nc * C * C * 2);
@@ -514,6 +542,8 @@ static size_t ws_carve(const Geo &g, bool bwd, char *base, TcWs *w) {
         w->Sn = (__nv_bfloat16 *)take(nc * DK * DV * 2);
         w->dSn = (__nv_bfloat16 *)take(nc * DK * DV * 2);
         w->Un = (__nv_bfloat16 *)take(nc * C * DV * 2);
+        w->dUn = (__nv_bfloat16 *)take(nc * C * DV * 2);
+        w->skt = (float *)take(nc * 2 * C * 4);
     }
     return off;
 }
@@ -539,7 +569,7 @@ cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, bool bwd
                     tc::make_map_2d_bf16(&mp.P, w.P, C, NC * C, 64);
     if (!ok) return cudaErrorInvalidValue;
     Args a = {};
-    a.g = w.g; a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
+    a.gb = w.gb; a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
     a.S0 = t.S0;
     if (bwd) {
         a.Sn = w.Sn; a.Un = w.Un;
@@ -570,11 +600,13 @@ cudaError_t tc_chain_rev(const Geo &g, const Tensors &t, const TcWs &w, cudaStre
     const bool ok = tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) &&
                     tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64) &&
                     tc::make_map_4d_bf16(&mp.dout, t.dout, DV, H, T, Bn, 64) &&
-                    tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.dUp, w.dUp, DV, NC * C, 64);
+                    tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.dUp, w.dUp, DV, NC * C, 64) &&
+                    tc::make_map_2d_bf16(&mp.Un, w.Un, DV, NC * C, 64) && tc::make_map_2d_bf16(&mp.dUn, w.dUn, DV, NC * C, 64) &&
+                    (t.du ? tc::make_map_4d_bf16(&mp.du, t.du, DV, H, T, Bn, 64) : (mp.du = mp.dout, true));
     if (!ok) return cudaErrorInvalidValue;
     Args a = {};
-    a.g = w.g; a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
-    a.S0 = t.dS_T; a.ST = t.dS0; a.dSn = w.dSn;
+    a.gb = w.gb; a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
+    a.S0 = t.dS_T; a.ST = t.dS0; a.dSn = w.dSn; a.skt = w.skt; a.has_du = t.du != nullptr;
     const size_t smem = SMEM_BYTES + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_chain_rev, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -19,30 +19,33 @@ int tc_fwd_launches(const Geo &g, const char **names, int max_names);
 bool tc_split_supported(const Geo &g, bool bf16);
 
 // Workspace of the split path, chunk-major (ci = (b H + h) N + n), every matrix row-major:
-// bf16 tiles that later kernels load with TMA, plus the fp32 gate.  The forward uses
-// g, W, Ut and P; the backward all of it.
+// bf16 tiles that later kernels load with TMA, plus fp32 per-token factors.  The forward
+// uses gb, W, Ut and P; the backward all of it.
 struct TcWs {
-    float *g;            // [ci][C]       in-chunk cumulative log gate
+    float *gb;           // [ci][2][C]    in-chunk cumulative log gate g, then beta
     __nv_bfloat16 *W;    // [ci][C][dk]   W  = T diag(beta e^g) k
     __nv_bfloat16 *Ut;   // [ci][C][dv]   U~ = T diag(beta) v
     __nv_bfloat16 *P;    // [ci][C][C]    P  = tril(e^{g_r - g_i} q_r . k_i)
     // backward only
     __nv_bfloat16 *Tn;   // [ci][C][C]    T  = (I + A)^-1
     __nv_bfloat16 *KK;   // [ci][C][C]    k k^T (no gate factor)
-    __nv_bfloat16 *dUp;  // [ci][C][dv]   du + P^T dO
+    __nv_bfloat16 *dUp;  // [ci][C][dv]   P^T dO
     __nv_bfloat16 *Sn;   // [ci][dk][dv]  state entering chunk n
     __nv_bfloat16 *dSn;  // [ci][dk][dv]  dL/dS of the state leaving chunk n
     __nv_bfloat16 *Un;   // [ci][C][dv]   write values U = U~ - W S_n
+    __nv_bfloat16 *dUn;  // [ci][C][dv]   dL/dU = du + P^T dO + Kbar dS_{n+1}
+    float *skt;          // [ci][2][C]    per 64-column half of dv: U_r . (Kbar dS_{n+1})_r
 };
 size_t tc_ws_bytes(const Geo &g, bool bwd);
 TcWs tc_ws_carve(const Geo &g, bool bwd, void *base);
 
-// Per-chunk products (tc_prep.cu): g, W, U~, P; with bwd also T, k k^T and du + P^T dO.
+// Per-chunk products (tc_prep.cu): g and beta, W, U~, P; with bwd also T, k k^T and P^T dO.
 cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool bwd, cudaStream_t s, Rec &rec);
 // Forward state chain (tc_chain.cu).  bwd = false: o, u, S_T; bwd = true (recompute for the
 // backward): S_n and U of every chunk into the workspace.
 cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, bool bwd, cudaStream_t s, Rec &rec);
-// Reverse state chain (tc_chain.cu): dS_{n+1} of every chunk into w.dSn, and dS0.
+// Reverse state chain (tc_chain.cu): dS_{n+1} and dL/dU of every chunk (w.dSn, w.dUn), the
+// row sums w.skt, and dS0.
 cudaError_t tc_chain_rev(const Geo &g, const Tensors &t, const TcWs &w, cudaStream_t s, Rec &rec);
 // All intra-chunk gradients (tc_bwd.cu): dq, dk, dv, dbeta, d log alpha.
 cudaError_t tc_bwd_chunk(const Geo &g, const Tensors &t, const TcWs &w, cudaStream_t s, Rec &rec);

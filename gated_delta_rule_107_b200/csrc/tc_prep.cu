@@ -8,12 +8,12 @@
 //        A = beta_r e^{g_r - g_i} k_r.k_i (i < r),   P = e^{g_r - g_i} q_r.k_i (i <= r)
 //   T  = (I + A)^-1                            (the UT transform; tc_inverse.cuh)
 //   W  = T diag(beta e^g) k,   U~ = T diag(beta) v
-//   backward only:  dU' = du + P^T dO, and T, k k^T kept for the gradient kernel.
+//   backward only:  dU' = P^T dO, and T, k k^T kept for the gradient kernel.
 //
 // Every chunk is independent, so the grid covers all chunks of all heads at once (two
 // CTAs per SM); the serial state chains (tc_chain.cu) then only carry the state.  The
 // products leave as bf16 tiles through TMA stores (W, U~, P, dU') or row stores (T, k k^T),
-// and g as fp32.  The products with 64 rows use M = 128 MMAs whose rows 64..127 read
+// and g, beta as fp32.  The products with 64 rows use M = 128 MMAs whose rows 64..127 read
 // other (valid) shared memory and are discarded.
 #include "tc_host.cuh"
 #include "tc_inverse.cuh"
@@ -58,8 +58,8 @@ struct Maps {
 };
 
 struct Args {
-    const void *alpha, *beta, *du;  // bf16 [B, T, H] / [B, T, H, 128]
-    float *g;                       // [chunks][64]
+    const void *alpha, *beta;       // bf16 [B, T, H]
+    float *gb;                      // [chunks][2][64]: g, beta
     __nv_bfloat16 *KK, *Tn;         // [chunks][64][64] (backward)
     int B, T, H, N;
 };
@@ -137,7 +137,8 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
             pf[PF_COLA * 64 + r] = __expf(gm - x);
             pf[PF_BV * 64 + r] = bt[hh];
             pf[PF_BK * 64 + r] = bt[hh] * __expf(x);
-            a.g[(size_t)ci * C + r] = x;
+            a.gb[(size_t)ci * 2 * C + r] = x;
+            a.gb[(size_t)ci * 2 * C + C + r] = bt[hh];
         }
         if (lane == 0) *bigflag = dev > 80.f;
     }
@@ -239,28 +240,15 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
     if (ok) unit_lower_inverse64(Asc, Tf, ysc, tid, sync);
     if (BWD && ok) {
         ok = consensus(wait_mma());
-        // dU' = du + P^T dO -> staging tile in place of dO (rows 0..63 of the accumulator)
+        // dU' = P^T dO -> staging tile in place of dO (rows 0..63 of the accumulator)
         if (ok && trow < 64) {
             const int r = trow;
-            const bool live = a.du != nullptr && r < L;
-            const __nv_bfloat16 *dur =
-                reinterpret_cast<const __nv_bfloat16 *>(a.du) + (((size_t)b * T + t0 + r) * H + h) * DV;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 float v[64];
                 tmem_row64(tl + TM_DU + hh * 64, v);
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    if (live) {
-                        float d[8];
-                        const uint4 w = *reinterpret_cast<const uint4 *>(dur + hh * 64 + ch * 8);
-                        d[0] = bf16_lo(w.x); d[1] = bf16_hi(w.x); d[2] = bf16_lo(w.y); d[3] = bf16_hi(w.y);
-                        d[4] = bf16_lo(w.z); d[5] = bf16_hi(w.z); d[6] = bf16_lo(w.w); d[7] = bf16_hi(w.w);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) v[ch * 8 + e] += d[e];
-                    }
-                    st_chunk(sm + OFF_DO, (uint32_t)hh * 8192 + swz(r, ch), v + ch * 8);
-                }
+                for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_DO, (uint32_t)hh * 8192 + swz(r, ch), v + ch * 8);
             }
         }
     }
@@ -367,7 +355,7 @@ cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool bw
         mp.dout = mp.v, mp.dUp = mp.W;
     if (!ok) return cudaErrorInvalidValue;
     Args a;
-    a.alpha = t.alpha; a.beta = t.beta; a.du = bwd ? t.du : nullptr; a.g = w.g; a.KK = w.KK; a.Tn = w.Tn;
+    a.alpha = t.alpha; a.beta = t.beta; a.gb = w.gb; a.KK = w.KK; a.Tn = w.Tn;
     a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
     const dim3 grid(g.N, g.H, g.B);
     if (g.variant == VAR_GATED)
