@@ -27,6 +27,12 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+
 // Problem geometry shared by all kernels.  N = number of chunks = ceil(T / C).
 struct Geo {
     int B, T, H, dk, dv, C, N, variant;

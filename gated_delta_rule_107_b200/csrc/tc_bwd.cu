@@ -26,9 +26,11 @@
 // needs no transpose: one D_M tile is read as a K-major and as an MN-major A operand.
 //
 // One CTA of 256 threads per chunk.  Operands arrive by TMA in three groups (what the first
-// products read; the rest; W and U~ into the space S leaves); dq, dk, dv leave through
-// staging tiles and TMA stores.  Warps w and w + 4 read the same TMEM lanes and split the
-// columns.
+// products read; the rest; W and U~ into the space dO and dU leave); dq, dk, dv leave
+// through staging tiles and TMA stores.  Warps w and w + 4 read the same TMEM lanes and split
+// the columns; the warps of lanes 64-127 form dW and the sum of S .* dS+.  As in the
+// per-chunk kernel, e^{g_r - g_i} is split at the chunk midpoint g_m unless the chunk's
+// cumulative log gate strays more than 80 from it.
 #include "tc_host.cuh"
 #include "tc_path.cuh"
 #include "tc_ptx.cuh"
@@ -45,8 +47,8 @@ using dr::tcf::tmem_row64;
 constexpr int C = 64, DK = 128, DV = 128;
 constexpr int NTHREADS = 256;
 // shared memory (bytes from a 1024-aligned base); later phases reuse earlier regions
-constexpr uint32_t R_DOU = 0;         // 32K  [dO_p0 | dU_p0 | dO_p1 | dU_p1], [r][j]
-constexpr uint32_t R_S = 32768;       // 32K  S [c][j]  -> W [i][c] | U~ [i][j]  -> staging dq | dk [r][c]
+constexpr uint32_t R_DOU = 0;         // 32K  [dO_p0 | dU_p0 | dO_p1 | dU_p1], [r][j]  -> W [i][c] | U~ [i][j]
+constexpr uint32_t R_S = 32768;       // 32K  S [c][j]  -> staging dq | dk [r][c]
 constexpr uint32_t R_DS = 65536;      // 32K  dS+ [c][j]
 constexpr uint32_t R_U = 98304;       // 16K  U [r][j]  -> Ubar
 constexpr uint32_t R_T = 114688;      //  8K  T [r][i]  -> D_M [r][i]
@@ -61,7 +63,7 @@ constexpr uint32_t R_MISC = 221184;   //  8K
 constexpr uint32_t SMEM_BYTES = R_MISC + 8192;
 constexpr uint32_t LOAD1_BYTES = 4 * 16384 + 16384 + 512;             // dO, dU, S, U, g|beta
 constexpr uint32_t LOAD2_BYTES = 32768 + 3 * 8192 + 3 * 16384 + 512;  // dS+, T, P, KK, q, k, v, row sums
-constexpr uint32_t LOAD3_BYTES = 32768;                               // W, U~
+constexpr uint32_t LOAD3_BYTES = 32768;                               // W, U~ (after batch 3)
 // misc (floats unless noted)
 constexpr uint32_t M_BAR = 0;  // [0] MMA, [1..3] load groups
 constexpr uint32_t M_TMEM = 64, M_ABORT = 68;
@@ -72,7 +74,9 @@ constexpr uint32_t M_PART = 1792;  // [kinds][2 column halves][64] per-row parti
 constexpr uint32_t M_ZC = M_PART + 6 * 2 * 64 * 4;  // [2 lane quarters][64] column sums of Z
 constexpr uint32_t M_RS = M_ZC + 512;               // [8] partial sums of S .* dS+
 constexpr uint32_t M_DG = M_RS + 64;                // [64] dg, then [64] row sums
-static_assert(M_DG + 512 <= 8192, "misc overflow");
+constexpr uint32_t M_ROWF = M_DG + 512, M_COLF = M_ROWF + 256;  // [64] e^{g_r - g_m}, e^{g_m - g_i}
+constexpr uint32_t M_BIG = M_COLF + 256;            // int: the chunk's gate range needs exact exponentials
+static_assert(M_BIG + 16 <= 8192, "misc overflow");
 enum { PS_SQ = 0, PS_SBK, PS_SV, PS_ROWZ, PS_DBA, PS_NUM };
 // TMEM columns
 constexpr uint32_t TM_QW = 0;     // 128: rows 0-63 dO S^T, rows 64-127 dU S^T
@@ -143,6 +147,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(const __grid_const
     float *rsp = reinterpret_cast<float *>(misc + M_RS);
     float *dgs = reinterpret_cast<float *>(misc + M_DG);
     float *ktm = dgs + 64;
+    float *rowf = reinterpret_cast<float *>(misc + M_ROWF);
+    float *colf = reinterpret_cast<float *>(misc + M_COLF);
+    volatile int *bigflag = reinterpret_cast<volatile int *>(misc + M_BIG);
 
     const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -217,39 +224,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(const __grid_const
         mma_commit(&bar[0]);
         mma_issued++;
     }
-    // gate factors; the sum of S .* dS+ (S is overwritten by the third load group)
+    // gate factors
     if (ok && tid < C) {
-        const float x = gsm[tid];
+        const float x = gsm[tid], gm = gsm[31];
         eg[tid] = __expf(x);
         egc[tid] = __expf(gsm[C - 1] - x);
+        rowf[tid] = __expf(x - gm);
+        colf[tid] = __expf(gm - x);
+        const float dev = warp_max(fabsf(x - gm));
+        if (lane == 0 && warp == 0) *bigflag = 0;
+        named_sync(3, 64);
+        if (lane == 0 && dev > 80.f) *bigflag = 1;
     }
-    bool got2 = false;  // second load group seen by this thread
-    if (ok && !rowt) {
-        got2 = mbar_wait(&bar[2], 0, abort_flag);
-        float rs = 0.f;
-        if (got2) {
-            for (int x = (warp & 3) * 32 + lane - 64 + (hf * 64); x < 2048; x += 128) {  // S, dS+: one layout
-                float v[8], w[8];
-                ld_chunk(sm + R_S, (uint32_t)x * 16, v);
-                ld_chunk(sm + R_DS, (uint32_t)x * 16, w);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) rs += v[e] * w[e];
-            }
-        }
-        rs = warp_sum(rs);
-        if (lane == 0) rsp[warp] = rs;
-    }
-    if (ok) ok = wait_mma(rowt || got2);
-    // third load group into the space S leaves
-    if (ok && tid == 0) {
-        mbar_arrive_tx(&bar[3], LOAD3_BYTES);
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            tma_load_2d(sm + R_S + p * 8192, &mp.W, 64 * p, ci * C, &bar[3]);
-            tma_load_2d(sm + R_S + 16384 + p * 8192, &mp.Ut, 64 * p, ci * C, &bar[3]);
-        }
-        loads_issued = 3;
-    }
+    if (ok) ok = wait_mma(true);
     // ---------------- epilogue 1: dW = -(dU S^T) -> tile;  Ubar = diag(e^{gC - g}) U ----------------
     if (ok) {
         if (!rowt) {
@@ -274,8 +261,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(const __grid_const
     }
     fence_proxy_async();
     fence_before_sync();
-    if (ok && rowt) ok = mbar_wait(&bar[2], 0, abort_flag);  // T (the other threads waited above)
-    ok = consensus(ok);
+    ok = consensus(ok && mbar_wait(&bar[2], 0, abort_flag));  // T, k, v, ...
     // ---------------- batch 3: dB_k = T^T dW, dB_v = T^T dU ----------------
     if (ok && tid == 0) {
         fence_after_sync();
@@ -290,6 +276,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(const __grid_const
         mma_issued++;
     }
     if (ok) ok = wait_mma(true);
+    // third load group into the space dO and dU leave
+    if (ok && tid == 0) {
+        mbar_arrive_tx(&bar[3], LOAD3_BYTES);
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            tma_load_2d(sm + R_DOU + p * 8192, &mp.W, 64 * p, ci * C, &bar[3]);
+            tma_load_2d(sm + R_DOU + 16384 + p * 8192, &mp.Ut, 64 * p, ci * C, &bar[3]);
+        }
+        loads_issued = 3;
+    }
+    // the sum of S .* dS+ (lanes 64-127, idle in this epilogue)
+    if (ok && !rowt) {
+        float rs = 0.f;
+        for (int x = (q4 - 2) * 32 + lane + hf * 64; x < 2048; x += 128) {  // S, dS+: one layout
+            float v[8], w[8];
+            ld_chunk(sm + R_S, (uint32_t)x * 16, v);
+            ld_chunk(sm + R_DS, (uint32_t)x * 16, w);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) rs += v[e] * w[e];
+        }
+        rs = warp_sum(rs);
+        if (lane == 0) rsp[warp] = rs;
+    }
     // ---------------- epilogue 3: dB_k, dB_v tiles; dv; dbeta sums ----------------
     if (ok && rowt) {
         float x[64];
@@ -335,7 +344,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(const __grid_const
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
             const uint32_t ka = ((k & 7) >> 2) * 8192 + (k & 3) * 32;
-            const uint32_t aa = (k < 8 ? sDW : sBV) + ka, bb = sS + (k < 8 ? 0 : 16384) + ka;
+            const uint32_t aa = (k < 8 ? sDW : sBV) + ka, bb = sDOU + (k < 8 ? 0 : 16384) + ka;
             mma_bf16(tbase + TM_DA, sdesc(aa, 16, 1024), sdesc(bb, 16, 1024), id, k > 0);
         }
         mma_commit(&bar[0]);
@@ -353,11 +362,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(const __grid_const
             ld_chunk(sm + R_KK, swz(r, hf * 4 + c4), kk + c4 * 8);
         }
         const float br = gsm[C + r], gr = gsm[r];
+        // gate factor e^{g_r - g_i}: 1 without gates, else split at the midpoint unless the range is large
+        float ef[32];
+        if (!gated) {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) ef[t] = 1.f;
+        } else if (*bigflag == 0) {
+            const float rf = rowf[r];
+#pragma unroll
+            for (int t = 0; t < 32; ++t) ef[t] = rf * colf[hf * 32 + t];
+        } else {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) ef[t] = __expf(gr - gsm[hf * 32 + t]);
+        }
         float rowz = 0.f, dbA = 0.f;
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
             const int i = hf * 32 + t;
-            const float e = (i <= r) ? (gated ? __expf(gr - gsm[i]) : 1.f) : 0.f;
+            const float e = (i <= r) ? ef[t] : 0.f;
             const float d = (i < r) ? -da[t] : 0.f;
             const float p = (i <= r) ? dp[t] : 0.f;
             const float dak = d * kk[t] * e;

@@ -34,7 +34,6 @@ namespace tch {
 using namespace dr::tc;
 using dr::tcf::ld_chunk;
 using dr::tcf::st_chunk;
-using dr::tcf::st_row_global;
 using dr::tcf::tmem_row64;
 
 constexpr int C = 64, DK = 128, DV = 128, DVB = 64;
@@ -49,7 +48,8 @@ constexpr uint32_t RS_K = 0, RS_Q = 16384, RS_W = 32768, RS_DO = 49152, RS_DU = 
 constexpr uint32_t OFF_S = 2 * STAGE;         // 16K  bf16 state [c][j]
 constexpr uint32_t OFF_U = OFF_S + 16384;     //  8K  U [r][j]        (reverse: dU [r][j])
 constexpr uint32_t OFF_UD = OFF_U + 8192;     //  8K  e^{g_C - g} U [r][j]
-constexpr uint32_t OFF_MISC = OFF_UD + 8192;  //  4K
+constexpr uint32_t OFF_O = OFF_UD + 8192;     //  8K  o [r][j] (staging of the TMA store)
+constexpr uint32_t OFF_MISC = OFF_O + 8192;   //  4K
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 4096;
 // misc
 constexpr uint32_t M_BAR = 0;  // FULL0, FULL1, EMPTY0, EMPTY1, MMA
@@ -59,23 +59,24 @@ enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_MMA, B_NUM };
 static_assert(M_CF + 2 * 132 * 4 <= 4096, "misc overflow");
 
 struct FMaps {
-    CUtensorMap q, k;   // [B, T, H, 128] bf16; box 64 x 64 tokens
-    CUtensorMap W, Ut;  // [chunks * 64][128] bf16; box 64 x 64
-    CUtensorMap P;      // [chunks * 64][64] bf16; box 64 x 64
+    CUtensorMap q, k;       // [B, T, H, 128] bf16; box 64 x 64 tokens
+    CUtensorMap W, Ut;      // [chunks * 64][128] bf16; box 64 x 64
+    CUtensorMap P;          // [chunks * 64][64] bf16; box 64 x 64
+    CUtensorMap out, u;     // forward outputs [B, T, H, 128] (stores)
+    CUtensorMap Sn, Un;     // recompute outputs: [chunks * 128][128] box 64 x 128, [chunks * 64][128] (stores)
 };
 struct RMaps {
     CUtensorMap q, k, dout, du;  // [B, T, H, 128] bf16
     CUtensorMap W, dUp, Un;      // [chunks * 64][128] bf16 (loads)
     CUtensorMap dUn;             // [chunks * 64][128] bf16 (store)
+    CUtensorMap dSn;             // [chunks * 128][128] bf16, box 64 x 128 (store)
 };
 struct Args {
     const float *gb;          // [chunks][2][64]: g, beta
     const float *S0;          // forward: S0; reverse: dS_T (fp32 [B, H, 128, 128], may be null)
     float *ST;                // forward: S_T; reverse: dS0 (may be null)
-    void *out, *u;            // forward outputs (bf16 [B, T, H, 128])
-    __nv_bfloat16 *Sn, *Un;   // recompute outputs
-    __nv_bfloat16 *dSn;       // reverse outputs
-    float *skt;
+    int has_out, has_u;       // forward outputs requested
+    float *skt;               // reverse output
     int B, T, H, N, has_du;
 };
 
@@ -182,17 +183,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
         int prev_L = 0, prev_t0 = 0;
         float prev_eg = 0.f;
         uint32_t prev_buf = 0;
+        // lanes 64-127 stage o in OFF_O; lane 64 issues its TMA store (rows past T are clipped)
         auto o_epilogue = [&]() {
-            if (BWD || trow < 64 || prev_L == 0) return;
+            if (BWD || trow < 64 || prev_L == 0 || !a.has_out) return;
             const int r = trow - 64;
-            // the TMEM loads are warp-wide (.sync.aligned): every lane loads, only rows < L store
             float d[64], p[64];
             tmem_row64(tl + TM_D + prev_buf, d);
             tmem_row64(tl + TM_D + prev_buf + 64, p);
-            if (r < prev_L && a.out) {
 #pragma unroll
-                for (int j = 0; j < 64; ++j) d[j] = prev_eg * d[j] + p[j];
-                st_row_global(a.out, (((size_t)b * T + prev_t0 + r) * H + h) * DV + j0, d);
+            for (int j = 0; j < 64; ++j) d[j] = prev_eg * d[j] + p[j];
+            if (trow == 64) bulk_wait_read_all();  // the previous o store has read OFF_O
+            named_sync(3, 64);
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_O, swz(r, ch), d + ch * 8);
+            fence_proxy_async();
+            named_sync(3, 64);
+            if (trow == 64) {
+                tma_store_4d(&mp.out, sm + OFF_O, j0, h, prev_t0, b);
+                bulk_commit();
             }
         };
         for (int m = 0; m < N; ++m) {
@@ -209,6 +217,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             // ---------------- D = [W ; q] S ----------------
             if (wc == 0) {
                 fence_after_sync();
+                bulk_wait_read_all();  // the previous chunk's U store has read OFF_U
                 const uint32_t id = idesc_bf16(128, 64, 0, 1);
                 const uint32_t swq = smem_u32(st + FS_WQ);
 #pragma unroll
@@ -216,9 +225,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
                     mma_bf16(tbase + TM_D + buf, sdesc(swq + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
                              sdesc(sS + k * 2048, 1024, 1024), id, k > 0);
                 mma_commit(&bar[B_MMA]);
+                if (BWD) {  // the state entering chunk m, straight from its bf16 operand tile
+                    tma_store_2d(&mp.Sn, sm + OFF_S, j0, (int)ci * DK);
+                    bulk_commit();
+                }
             }
             pending = true;
-            if (BWD) st_row_global(a.Sn, (ci * DK + trow) * DV + j0, S);  // state entering chunk m
             o_epilogue();  // previous chunk, lanes 64-127
             if (!mma_done()) break;
             // ---------------- U = U~ - W S;  u;  U and e^{gC - g} U tiles ----------------
@@ -233,13 +245,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
 #pragma unroll
                     for (int e = 0; e < 8; ++e) v[ch * 8 + e] = ut[e] - v[ch * 8 + e];
                 }
-                if (BWD) {
-                    st_row_global(a.Un, (ci * C + r) * DV + j0, v);
-                } else {
-                    if (a.u && r < L) st_row_global(a.u, (((size_t)b * T + t0 + r) * H + h) * DV + j0, v);
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_U, swz(r, ch), v + ch * 8);
-                }
+                for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_U, swz(r, ch), v + ch * 8);
 #pragma unroll
                 for (int j = 0; j < 64; ++j) v[j] *= rowf;
 #pragma unroll
@@ -248,9 +255,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             fence_proxy_async();
             fence_before_sync();
             if (wabort(true)) break;
-            // ---------------- E = k^T (e^{gC-g} U);  O' = [* ; P] U ----------------
+            // ---------------- E = k^T (e^{gC-g} U);  O' = [* ; P] U;  U out ----------------
             if (wc == 0) {
                 fence_after_sync();
+                if (BWD) {
+                    tma_store_2d(&mp.Un, sm + OFF_U, j0, (int)ci * C);
+                    bulk_commit();
+                } else if (a.has_u) {
+                    tma_store_4d(&mp.u, sm + OFF_U, j0, h, t0, b);
+                    bulk_commit();
+                }
                 const uint32_t sk = smem_u32(st + FS_K), sup = smem_u32(st + FS_UP);
                 const uint32_t ide = idesc_bf16(128, 64, 1, 1), ido = idesc_bf16(128, 64, 0, 1);
 #pragma unroll
@@ -266,6 +280,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
                 mma_commit(&bar[B_MMA]);
             }
             pending = true;
+            if (BWD && wc == 0) bulk_wait_read_1();  // the S_m store has read OFF_S
             if (!mma_done()) break;
             if (wc == 0) mbar_arrive(&bar[B_EMPTY0 + s]);
             // ---------------- S <- e^{gC} S + E ----------------
@@ -282,8 +297,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             if (wabort(true)) break;
             prev_L = L; prev_t0 = t0; prev_eg = rowf; prev_buf = buf;
         }
+        if (*abort_flag == 0) o_epilogue();  // last chunk
+        if (wc == 0 || trow == 64) bulk_wait_all();
         if (*abort_flag == 0) {
-            o_epilogue();  // last chunk
             if (!BWD && a.ST) {
                 float *dst = a.ST + (((size_t)b * H + h) * DK + trow) * DV + j0;
 #pragma unroll
@@ -398,6 +414,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
             // ---------------- D_a = k dS+  (M = 128: rows 64..127 discarded) ----------------
             if (wc == 0) {
                 fence_after_sync();
+                bulk_wait_read_all();  // the previous chunk's dU store has read OFF_U
                 const uint32_t id = idesc_bf16(128, 64, 0, 1);
                 const uint32_t sk = smem_u32(st + RS_K);
 #pragma unroll
@@ -405,11 +422,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
                     mma_bf16(tbase + TM_A, sdesc(sk + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024),
                              sdesc(sS + k * 2048, 1024, 1024), id, k > 0);
                 mma_commit(&bar[B_MMA]);
+                tma_store_2d(&mp.dSn, sm + OFF_S, j0, (int)ci * DK);  // dS_{n+1} from its operand tile
+                bulk_commit();
             }
             pending = true;
-            st_row_global(a.dSn, (ci * DK + trow) * DV + j0, S);
-            // the dU tile of the previous chunk has been read by its TMA store
-            if (wc == 0) bulk_wait_read_all();
             // dO rows scaled by e^{g_r} (for q^T diag(e^g) dO) while the MMA runs
             for (int x = wc; x < 512; x += 128) {
                 float v[8];
@@ -482,6 +498,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
                 bulk_commit();
             }
             pending = true;
+            if (wc == 0) bulk_wait_read_1();  // the dS_{n+1} store has read OFF_S
             if (!mma_done()) break;
             if (wc == 0) mbar_arrive(&bar[B_EMPTY0 + s]);
             // ---------------- dS_n = e^{gC} dS+ + D_b ----------------
@@ -563,18 +580,20 @@ cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, bool bwd
     using namespace tch;
     FMaps mp;
     const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;
-    const bool ok = tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) &&
-                    tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64) &&
-                    tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.Ut, w.Ut, DV, NC * C, 64) &&
-                    tc::make_map_2d_bf16(&mp.P, w.P, C, NC * C, 64);
+    bool ok = tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) && tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64) &&
+              tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.Ut, w.Ut, DV, NC * C, 64) &&
+              tc::make_map_2d_bf16(&mp.P, w.P, C, NC * C, 64);
+    mp.out = mp.u = mp.Sn = mp.Un = mp.q;  // unused ones keep a valid map
+    if (ok && bwd)
+        ok = tc::make_map_2d_bf16(&mp.Sn, w.Sn, DV, NC * DK, 128) && tc::make_map_2d_bf16(&mp.Un, w.Un, DV, NC * C, 64);
+    if (ok && !bwd && t.out) ok = tc::make_map_4d_bf16(&mp.out, t.out, DV, H, T, Bn, 64);
+    if (ok && !bwd && t.u) ok = tc::make_map_4d_bf16(&mp.u, t.u, DV, H, T, Bn, 64);
     if (!ok) return cudaErrorInvalidValue;
     Args a = {};
     a.gb = w.gb; a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
     a.S0 = t.S0;
-    if (bwd) {
-        a.Sn = w.Sn; a.Un = w.Un;
-    } else {
-        a.out = t.out; a.u = t.u; a.ST = t.S_T;
+    if (!bwd) {
+        a.has_out = t.out != nullptr; a.has_u = t.u != nullptr; a.ST = t.S_T;
     }
     const size_t smem = SMEM_BYTES + 1024;
     const dim3 grid(DV / DVB, g.H, g.B);
@@ -602,11 +621,12 @@ cudaError_t tc_chain_rev(const Geo &g, const Tensors &t, const TcWs &w, cudaStre
                     tc::make_map_4d_bf16(&mp.dout, t.dout, DV, H, T, Bn, 64) &&
                     tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.dUp, w.dUp, DV, NC * C, 64) &&
                     tc::make_map_2d_bf16(&mp.Un, w.Un, DV, NC * C, 64) && tc::make_map_2d_bf16(&mp.dUn, w.dUn, DV, NC * C, 64) &&
+                    tc::make_map_2d_bf16(&mp.dSn, w.dSn, DV, NC * DK, 128) &&
                     (t.du ? tc::make_map_4d_bf16(&mp.du, t.du, DV, H, T, Bn, 64) : (mp.du = mp.dout, true));
     if (!ok) return cudaErrorInvalidValue;
     Args a = {};
     a.gb = w.gb; a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
-    a.S0 = t.dS_T; a.ST = t.dS0; a.dSn = w.dSn; a.skt = w.skt; a.has_du = t.du != nullptr;
+    a.S0 = t.dS_T; a.ST = t.dS0; a.skt = w.skt; a.has_du = t.du != nullptr;
     const size_t smem = SMEM_BYTES + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_chain_rev, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
