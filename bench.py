@@ -197,16 +197,21 @@ def run_ours(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    w = WORKLOADS[WORKLOAD_ID]
+    w = WORKLOADS[args.workload]
     B, T, H, dk, dv, C, var = (args.batch or w.B), w.T, w.H, w.dk, w.dv, 64, w.variant
+    vname = {0: "deltanet", 1: "gdn", 2: "kda"}[var]
     dt = binding.DR_BF16
-    x = make_inputs(var, w.dtype, B, T, H, dk, dv, seed=w.seed + 1000 * rank, grads=True, du=True, device=dev)
+    x = make_inputs(var, w.dtype, B, T, H, dk, dv, seed=w.seed + 1000 * rank, s0_std=w.s0_std, grads=True, du=True,
+                    device=dev)
+    s0 = x["S0"] if w.s0_std else None
     elem = 2
 
-    fwd_names = binding.launches(B, T, H, dk, dv, var, C, dt, 0)
-    bwd_names = binding.launches(B, T, H, dk, dv, var, C, dt, 1)
-    ws_bytes = max(binding.workspace_size(B, T, H, dk, dv, var, C, dt, 0),
-                   binding.workspace_size(B, T, H, dk, dv, var, C, dt, 1))
+    # The timed step is the training pair: the forward keeps what the backward would
+    # recompute (delta_rule_fwd_save), the backward starts from it (delta_rule_bwd_saved).
+    # The plain forward + recomputing backward is timed afterwards and reported beside it.
+    sv_bytes = binding.saved_size(B, T, H, dk, dv, var, C, dt)
+    saved = torch.empty(max(sv_bytes, 1), dtype=torch.uint8, device=dev)
+    ws_bytes = max(binding.workspace_size(B, T, H, dk, dv, var, C, dt, kind) for kind in range(4))
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     o = torch.empty_like(x["v"])
     u = torch.empty_like(x["v"])
@@ -219,27 +224,43 @@ def run_ours(args):
     sp = stream.cuda_stream
     p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
 
-    fev = [torch.cuda.Event(enable_timing=True) for _ in range(len(fwd_names) + 1)]
-    bev = [torch.cuda.Event(enable_timing=True) for _ in range(len(bwd_names) + 1)]
-    for e in fev + bev:  # torch creates the CUDA event handle on first record
-        e.record(stream)
-    torch.cuda.synchronize()
-    farr, barr = binding.event_array(fev), binding.event_array(bev)
-
-    def step(timed: bool):
-        fa = (p(x["q"]), p(x["k"]), p(x["v"]), p(x["loga"]), p(x["beta"]), None, p(o), p(u), p(S_T),
-              B, T, H, dk, dv, var, C, dt, p(ws), ws_bytes, sp)
-        ba = (p(x["q"]), p(x["k"]), p(x["v"]), p(x["loga"]), p(x["beta"]), None, p(x["dO"]), p(x["du"]),
+    def make_step(saved_pair: bool):
+        fk, bk = (2, 3) if saved_pair else (0, 1)
+        fnames = binding.launches(B, T, H, dk, dv, var, C, dt, fk)
+        bnames = binding.launches(B, T, H, dk, dv, var, C, dt, bk)
+        fe = [torch.cuda.Event(enable_timing=True) for _ in range(len(fnames) + 1)]
+        be = [torch.cuda.Event(enable_timing=True) for _ in range(len(bnames) + 1)]
+        for e in fe + be:  # torch creates the CUDA event handle on first record
+            e.record(stream)
+        torch.cuda.synchronize()
+        fa_ev, ba_ev = binding.event_array(fe), binding.event_array(be)
+        fa = (p(x["q"]), p(x["k"]), p(x["v"]), p(x["loga"]), p(x["beta"]), p(s0), p(o), p(u), p(S_T),
+              B, T, H, dk, dv, var, C, dt)
+        ba = (p(x["q"]), p(x["k"]), p(x["v"]), p(x["loga"]), p(x["beta"]), p(s0), p(x["dO"]), p(x["du"]),
               p(x["dS_T"]), p(grads["dq"]), p(grads["dk"]), p(grads["dv"]), p(grads["dalpha"]), p(grads["dbeta"]),
-              p(grads["dS0"]), B, T, H, dk, dv, var, C, dt, p(ws), ws_bytes, sp)
-        if timed:
-            rc1 = binding.fwd_timed_raw(*fa, farr, len(fev))
-            rc2 = binding.bwd_timed_raw(*ba, barr, len(bev))
-        else:
-            rc1 = binding.fwd_raw(*fa)
-            rc2 = binding.bwd_raw(*ba)
-        if rc1 or rc2:
-            raise RuntimeError(f"delta_rule call failed: {binding.strerror(rc1 or rc2)}")
+              p(grads["dS0"]), B, T, H, dk, dv, var, C, dt)
+        sv = (p(saved), sv_bytes)
+        wsa = (p(ws), ws_bytes, sp)
+
+        def step(timed: bool):
+            if saved_pair and timed:
+                rc1 = binding.fwd_save_timed_raw(*fa, *sv, *wsa, fa_ev, len(fe))
+                rc2 = binding.bwd_saved_timed_raw(*ba, *sv, *wsa, ba_ev, len(be))
+            elif saved_pair:
+                rc1 = binding.fwd_save_raw(*fa, *sv, *wsa)
+                rc2 = binding.bwd_saved_raw(*ba, *sv, *wsa)
+            elif timed:
+                rc1 = binding.fwd_timed_raw(*fa, *wsa, fa_ev, len(fe))
+                rc2 = binding.bwd_timed_raw(*ba, *wsa, ba_ev, len(be))
+            else:
+                rc1 = binding.fwd_raw(*fa, *wsa)
+                rc2 = binding.bwd_raw(*ba, *wsa)
+            if rc1 or rc2:
+                raise RuntimeError(f"delta_rule call failed: {binding.strerror(rc1 or rc2)}")
+
+        return step, fnames, bnames, fe, be
+
+    step, fwd_names, bwd_names, fev, bev = make_step(True)
 
     for _ in range(max(args.warmup, 3)):
         step(False)
@@ -276,7 +297,7 @@ def run_ours(args):
             kern.setdefault(n, []).append(t)
         fwd_ms.append(fev[0].elapsed_time(fev[-1]))
         bwd_ms.append(bev[0].elapsed_time(bev[-1]))
-        step_ms.append(fev[0].elapsed_time(bev[-1]))
+        step_ms.append(fev[0].elapsed_time(fev[-1]) + bev[0].elapsed_time(bev[-1]))
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -292,6 +313,29 @@ def run_ours(args):
     tokens = B * T * world
     value = tokens / (ms / 1e3)
 
+    # ---- the plain forward + recomputing backward, same protocol (reported beside) ----
+    rstep, rf_names, rb_names, rfev, rbev = make_step(False)
+    for _ in range(max(args.warmup, 3)):
+        rstep(False)
+    torch.cuda.synchronize()
+    r_step_ms, r_kern = [], {}
+    for _ in range(args.steps):
+        flush.fill_(1)
+        rstep(True)
+        torch.cuda.synchronize()
+        for n, i in zip(rf_names, range(len(rf_names))):
+            r_kern.setdefault(n, []).append(rfev[i].elapsed_time(rfev[i + 1]))
+        for n, i in zip(rb_names, range(len(rb_names))):
+            r_kern.setdefault("bwd:" + n, []).append(rbev[i].elapsed_time(rbev[i + 1]))
+        r_step_ms.append(rfev[0].elapsed_time(rfev[-1]) + rbev[0].elapsed_time(rbev[-1]))
+    if binding.sync_status() != binding.DR_OK:
+        raise RuntimeError("device error word set during the recompute leg")
+    r_ms = statistics.mean(r_step_ms)
+    if world > 1:
+        t = torch.tensor([r_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        r_ms = float(t.item())
+
     # ---- end to end through the public API with host buffers ----
     host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in x.items()}
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
@@ -304,11 +348,13 @@ def run_ours(args):
         for k_, v_ in host.items():
             if v_ is not None:
                 dev_in[k_].copy_(v_, non_blocking=True)
-        binding.delta_rule_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["loga"], dev_in["beta"], None,
-                               variant=var, chunk=C, workspace=ws, out=o, u=u, S_T=S_T)
-        binding.delta_rule_bwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["loga"], dev_in["beta"], None,
-                               dev_in["dO"], dev_in["du"], dev_in["dS_T"], variant=var, chunk=C, workspace=ws,
-                               grads=grads)
+        s0_in = dev_in["S0"] if s0 is not None else None
+        _, _, _, sv = binding.delta_rule_fwd_save(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["loga"],
+                                                  dev_in["beta"], s0_in, variant=var, chunk=C, saved=saved,
+                                                  workspace=ws, out=o, u=u, S_T=S_T)
+        binding.delta_rule_bwd_saved(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["loga"], dev_in["beta"], s0_in,
+                                     dev_in["dO"], dev_in["du"], dev_in["dS_T"], saved=sv, variant=var, chunk=C,
+                                     workspace=ws, grads=grads)
         for src, dst in zip(outs, host_out):
             dst.copy_(src, non_blocking=True)
 
@@ -333,7 +379,7 @@ def run_ours(args):
             e2e_ms = float(t.item())
 
     peaks = load_peaks()
-    cnt = alg_counts(B, T, H, dk, dv, C, var, elem)
+    cnt = alg_counts(B, T, H, dk, dv, C, var, elem, s0=s0 is not None)
     kern_ms = {n: statistics.mean(v) for n, v in kern.items() if v}
     total = sum(kern_ms.values())
     dominant = max(kern_ms, key=kern_ms.get)
@@ -373,7 +419,7 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": (w.name if B == w.B else w.name.replace(f"_B{w.B}_", f"_B{B}_")) + " fwd+bwd", "B": B, "T": T, "H": H, "dk": dk, "dv": dv, "chunk": C,
-                   "variant": "gdn", "io": "bf16, fp32 state", "l2": "flushed between steps (256 MiB write)",
+                   "variant": vname, "io": "bf16, fp32 state", "l2": "flushed between steps (256 MiB write)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "kernel": r_label,
@@ -387,6 +433,12 @@ def run_ours(args):
                           "frac": step_time_roof * 1e3 / ms, "fwd_ms": f_ms, "bwd_ms": b_ms},
         "kernels": {n: {"ms": round(t, 4), "share": round(t / total, 4)} for n, t in kern_ms.items()},
         "dominant_kernel": dominant,
+        "step": "delta_rule_fwd_save + delta_rule_bwd_saved (the forward keeps the chunk products and states the "
+                "backward reads; every value is computed inside the timed step)",
+        "recompute": {"step": "delta_rule_fwd + delta_rule_bwd (the backward recomputes the forward)",
+                      "ms_per_step": r_ms, "value": tokens / (r_ms / 1e3),
+                      "kernels": {n: round(statistics.mean(v), 4) for n, v in r_kern.items()}},
+        "saved_bytes": sv_bytes,
         "gpu_launches": args.steps * (len(fwd_names) + len(bwd_names)),
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -413,6 +465,8 @@ def main():
     ap.add_argument("--batch", type=int, default=0,
                     help="run the workload at this batch size instead (smaller cases for ncu captures)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--workload", type=int, default=WORKLOAD_ID, choices=(2, 3, 4, 5),
+                    help="workload id (default: the headline GDN B=8 T=4096 H=8 d=128; 3-5 are the other bf16 ones)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

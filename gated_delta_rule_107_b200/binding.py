@@ -5,12 +5,18 @@ CUDA kernels.  PyTorch supplies device memory and the current stream.  There is
 no fallback: if the shared library is missing or a call fails, an exception is
 raised.
 
-Low level: ``workspace_size``, ``fwd_raw``, ``bwd_raw``, ``strerror``,
-``sync_status`` mirror the C entry points one to one (integer pointers).
+Low level: ``workspace_size``, ``saved_size``, ``fwd_raw``, ``bwd_raw``,
+``fwd_save_raw``, ``bwd_saved_raw``, ``strerror``, ``sync_status`` mirror the C
+entry points one to one (integer pointers).
 High level: ``delta_rule_fwd`` / ``delta_rule_bwd`` take torch CUDA tensors,
 allocate outputs and the workspace with torch, and call the C ABI on the
-current stream.  ``delta_rule_fwd_host`` is the same call for host tensors
-(copies in, computes, copies out).
+current stream; ``delta_rule_fwd_save`` / ``delta_rule_bwd_saved`` are the
+training pair (the forward keeps what the backward would recompute in a saved
+buffer).  ``delta_rule_fwd_host`` is the forward for host tensors (copies in,
+computes, copies out).
+
+The ``for_bwd`` argument of ``workspace_size`` and ``launches`` names the call:
+0 forward, 1 backward, 2 saving forward, 3 backward from saved activations.
 """
 from __future__ import annotations
 
@@ -27,7 +33,9 @@ DTYPES = {torch.float32: DR_F32, torch.bfloat16: DR_BF16}
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdeltarule.so")
 EXPORTS = ("delta_rule_workspace_size", "delta_rule_fwd", "delta_rule_bwd", "delta_rule_strerror",
-           "delta_rule_sync_status", "delta_rule_launches", "delta_rule_fwd_timed", "delta_rule_bwd_timed", "delta_rule_fwd_noalloc")
+           "delta_rule_sync_status", "delta_rule_launches", "delta_rule_fwd_timed", "delta_rule_bwd_timed",
+           "delta_rule_fwd_noalloc", "delta_rule_saved_size", "delta_rule_fwd_save", "delta_rule_bwd_saved",
+           "delta_rule_fwd_save_timed", "delta_rule_bwd_saved_timed")
 
 _lib = None
 
@@ -67,6 +75,16 @@ def load(path: str | None = None):
     lib.delta_rule_bwd_timed.restype = i
     lib.delta_rule_fwd_noalloc.argtypes = [vp] * 9 + [i] * 8 + [vp]
     lib.delta_rule_fwd_noalloc.restype = i
+    lib.delta_rule_saved_size.argtypes = [i] * 8
+    lib.delta_rule_saved_size.restype = sz
+    lib.delta_rule_fwd_save.argtypes = [vp] * 9 + [i] * 8 + [vp, sz, vp, sz, vp]
+    lib.delta_rule_fwd_save.restype = i
+    lib.delta_rule_bwd_saved.argtypes = [vp] * 15 + [i] * 8 + [vp, sz, vp, sz, vp]
+    lib.delta_rule_bwd_saved.restype = i
+    lib.delta_rule_fwd_save_timed.argtypes = [vp] * 9 + [i] * 8 + [vp, sz, vp, sz, vp, ctypes.POINTER(vp), i]
+    lib.delta_rule_fwd_save_timed.restype = i
+    lib.delta_rule_bwd_saved_timed.argtypes = [vp] * 15 + [i] * 8 + [vp, sz, vp, sz, vp, ctypes.POINTER(vp), i]
+    lib.delta_rule_bwd_saved_timed.restype = i
     if path is None:
         _lib = lib
     return lib
@@ -77,16 +95,24 @@ def strerror(code: int) -> str:
 
 
 def workspace_size(B, T, H, dk, dv, variant, chunk, dtype, for_bwd) -> int:
-    n = load().delta_rule_workspace_size(B, T, H, dk, dv, variant, chunk, dtype, int(bool(for_bwd)))
+    n = load().delta_rule_workspace_size(B, T, H, dk, dv, variant, chunk, dtype, int(for_bwd))
     if n == ctypes.c_size_t(-1).value:
         raise DeltaRuleError(DR_ERR_ARG, "delta_rule_workspace_size")
+    return n
+
+
+def saved_size(B, T, H, dk, dv, variant, chunk, dtype) -> int:
+    """Bytes of the saved-activation buffer (0: this configuration has no saved form)."""
+    n = load().delta_rule_saved_size(B, T, H, dk, dv, variant, chunk, dtype)
+    if n == ctypes.c_size_t(-1).value:
+        raise DeltaRuleError(DR_ERR_ARG, "delta_rule_saved_size")
     return n
 
 
 def launches(B, T, H, dk, dv, variant, chunk, dtype, for_bwd) -> list[str]:
     """Names of the kernels one call launches, in launch order."""
     names = (ctypes.c_char_p * 16)()
-    n = load().delta_rule_launches(B, T, H, dk, dv, variant, chunk, dtype, int(bool(for_bwd)), names, 16)
+    n = load().delta_rule_launches(B, T, H, dk, dv, variant, chunk, dtype, int(for_bwd), names, 16)
     if n < 0:
         raise DeltaRuleError(n, "delta_rule_launches")
     return [names[i].decode() for i in range(n)]
@@ -119,6 +145,22 @@ def fwd_timed_raw(*args) -> int:
 
 def bwd_timed_raw(*args) -> int:
     return load().delta_rule_bwd_timed(*args)
+
+
+def fwd_save_raw(*args) -> int:
+    return load().delta_rule_fwd_save(*args)
+
+
+def bwd_saved_raw(*args) -> int:
+    return load().delta_rule_bwd_saved(*args)
+
+
+def fwd_save_timed_raw(*args) -> int:
+    return load().delta_rule_fwd_save_timed(*args)
+
+
+def bwd_saved_timed_raw(*args) -> int:
+    return load().delta_rule_bwd_saved_timed(*args)
 
 
 def sync_status(stream=None) -> int:
@@ -200,6 +242,68 @@ def delta_rule_bwd(q, k, v, alpha, beta, S0, dout, du=None, dS_T=None, variant="
                  _p(g["dq"]), _p(g["dk"]), _p(g["dv"]), _p(g["dalpha"]), _p(g["dbeta"]), _p(g["dS0"]),
                  B, T, H, dk, dv, var, chunk, dt, _p(workspace), need, stream)
     _check(rc, "delta_rule_bwd")
+    return g
+
+
+def delta_rule_fwd_save(q, k, v, alpha, beta, S0=None, variant="gdn", chunk=64, want_u=True, want_state=True,
+                        saved: torch.Tensor | None = None, workspace: torch.Tensor | None = None, out=None, u=None,
+                        S_T=None):
+    """The forward of a training step: returns (o, u or None, S_T or None, saved).
+
+    ``saved`` (a uint8 CUDA tensor, allocated here when not given or too small) holds what
+    ``delta_rule_bwd_saved`` needs instead of recomputing the forward; it is None for
+    configurations without a saved form (then this is ``delta_rule_fwd``).
+    """
+    var = _variant(variant)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = DTYPES[q.dtype]
+    dev = q.device
+    out = torch.empty((B, T, H, dv), dtype=q.dtype, device=dev) if out is None else out
+    if want_u and u is None:
+        u = torch.empty((B, T, H, dv), dtype=q.dtype, device=dev)
+    if want_state and S_T is None:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    sneed = saved_size(B, T, H, dk, dv, var, chunk, dt)
+    if saved is None or saved.numel() < sneed:
+        saved = _workspace(sneed, dev)
+    need = workspace_size(B, T, H, dk, dv, var, chunk, dt, 2)
+    if workspace is None or workspace.numel() < need:
+        workspace = _workspace(need, dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = fwd_save_raw(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(out), _p(u), _p(S_T),
+                      B, T, H, dk, dv, var, chunk, dt, _p(saved), sneed, _p(workspace), need, stream)
+    _check(rc, "delta_rule_fwd_save")
+    return out, u, S_T, saved
+
+
+def delta_rule_bwd_saved(q, k, v, alpha, beta, S0, dout, du=None, dS_T=None, saved=None, variant="gdn", chunk=64,
+                         want_dS0=True, workspace: torch.Tensor | None = None, grads: dict | None = None):
+    """The backward of a training step from ``saved`` (from ``delta_rule_fwd_save`` on the same inputs).
+
+    Returns the same dict as ``delta_rule_bwd``.
+    """
+    var = _variant(variant)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = DTYPES[q.dtype]
+    dev = q.device
+    g = dict(grads or {})
+    g.setdefault("dq", torch.empty_like(q))
+    g.setdefault("dk", torch.empty_like(k))
+    g.setdefault("dv", torch.empty_like(v))
+    g.setdefault("dalpha", torch.empty_like(alpha) if (var != DR_DELTANET and alpha is not None) else None)
+    g.setdefault("dbeta", torch.empty_like(beta))
+    g.setdefault("dS0", torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if want_dS0 else None)
+    sneed = saved_size(B, T, H, dk, dv, var, chunk, dt)
+    need = workspace_size(B, T, H, dk, dv, var, chunk, dt, 3)
+    if workspace is None or workspace.numel() < need:
+        workspace = _workspace(need, dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = bwd_saved_raw(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(dout), _p(du), _p(dS_T),
+                       _p(g["dq"]), _p(g["dk"]), _p(g["dv"]), _p(g["dalpha"]), _p(g["dbeta"]), _p(g["dS0"]),
+                       B, T, H, dk, dv, var, chunk, dt, _p(saved), sneed, _p(workspace), need, stream)
+    _check(rc, "delta_rule_bwd_saved")
     return g
 
 

@@ -38,11 +38,38 @@ int check_shape(int B, int T, int H, int dk, int dv, int variant, int chunk, int
 // Which kernels serve a call: the tensor-core forward for bf16, d = 128, C = 64.
 bool use_tc_fwd(const Geo &g, int dtype) { return tc_fwd_supported(g, dtype == DR_BF16); }
 
-size_t ws_bytes(const Geo &g, int dtype, bool bwd) {
+// Call kinds: which entry point a size / plan question is about.
+enum { K_FWD = 0, K_BWD = 1, K_FWD_SAVE = 2, K_BWD_SAVED = 3 };
+bool is_bwd(int kind) { return kind == K_BWD || kind == K_BWD_SAVED; }
+
+bool use_split(const Geo &g, int dtype) { return tc_split_supported(g, dtype == DR_BF16); }
+
+size_t ws_bytes(const Geo &g, int dtype, int kind) {
     if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
-    if (tc_split_supported(g, dtype == DR_BF16)) return tc_ws_bytes(g, bwd);
-    if (!bwd && use_tc_fwd(g, dtype)) return 0;
-    return simt_ws_bytes(g, bwd);
+    if (use_split(g, dtype)) {
+        switch (kind) {
+            case K_FWD: return tc_ws_bytes(g, WS_FWD);
+            case K_BWD: return tc_ws_bytes(g, WS_FWD | WS_KEEP | WS_REV);
+            case K_FWD_SAVE: return 0;  // everything it keeps lives in the saved buffer
+            default: return tc_ws_bytes(g, WS_REV);
+        }
+    }
+    if (!is_bwd(kind) && use_tc_fwd(g, dtype)) return 0;
+    return simt_ws_bytes(g, is_bwd(kind));
+}
+
+// Bytes of the saved-activation buffer (0: no saved form for this configuration).
+size_t saved_bytes(const Geo &g, int dtype) {
+    if (g.T == 0 || g.B == 0 || g.H == 0 || !use_split(g, dtype)) return 0;
+    return tc_ws_bytes(g, WS_FWD | WS_KEEP);
+}
+
+// Checks a caller buffer of `given` bytes against `need` (256-byte aligned when needed).
+int check_buffer(const void *p, size_t given, size_t need) {
+    if (need == 0) return DR_OK;
+    if (!p || given < need) return DR_ERR_WORKSPACE;
+    if (((uintptr_t)p & 255u) != 0) return DR_ERR_ALIGN;
+    return DR_OK;
 }
 
 int launch_status(cudaError_t e) { return e == cudaSuccess ? DR_OK : DR_ERR_CUDA; }
@@ -62,12 +89,21 @@ extern "C" size_t delta_rule_workspace_size(int B, int T, int H, int dk, int dv,
                                             int for_bwd) {
     Geo g;
     if (check_shape(B, T, H, dk, dv, variant, chunk, dtype, &g) != DR_OK) return (size_t)-1;
-    return ws_bytes(g, dtype, for_bwd != 0);
+    if (for_bwd < 0 || for_bwd > 3) return (size_t)-1;
+    return ws_bytes(g, dtype, for_bwd);
 }
 
+extern "C" size_t delta_rule_saved_size(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype) {
+    Geo g;
+    if (check_shape(B, T, H, dk, dv, variant, chunk, dtype, &g) != DR_OK) return (size_t)-1;
+    return saved_bytes(g, dtype);
+}
+
+// save: the saving forward (kind K_FWD_SAVE) with its buffer `saved`
 static int fwd_impl(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
                     const float *S0, void *out, void *u, float *S_T, int B, int T, int H, int dk, int dv, int variant,
-                    int chunk, int dtype, void *workspace, size_t ws_bytes_given, void *stream, Rec &rec) {
+                    int chunk, int dtype, bool save, void *saved, size_t saved_given, void *workspace,
+                    size_t ws_bytes_given, void *stream, Rec &rec) {
     Geo g;
     int rc = check_shape(B, T, H, dk, dv, variant, chunk, dtype, &g);
     if (rc != DR_OK) return rc;
@@ -81,14 +117,19 @@ static int fwd_impl(const void *q, const void *k, const void *v, const void *alp
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return DR_ERR_ALIGN;
     if (!aligned_elem(beta, dtype) || (variant == DR_GATED && !aligned_elem(alpha, dtype))) return DR_ERR_ALIGN;
-    const size_t need = ws_bytes(g, dtype, false);
-    if (need > 0) {
-        if (!workspace || ws_bytes_given < need) return DR_ERR_WORKSPACE;
-        if (((uintptr_t)workspace & 255u) != 0) return DR_ERR_ALIGN;
-    }
+    const int kind = save ? K_FWD_SAVE : K_FWD;
+    rc = check_buffer(workspace, ws_bytes_given, ws_bytes(g, dtype, kind));
+    if (rc == DR_OK && save) rc = check_buffer(saved, saved_given, saved_bytes(g, dtype));
+    if (rc != DR_OK) return rc;
     Tensors t = {};
     t.q = q; t.k = k; t.v = v; t.alpha = alpha; t.beta = beta; t.S0 = S0; t.out = out; t.u = u; t.S_T = S_T;
-    if (use_tc_fwd(g, dtype)) {
+    if (use_split(g, dtype)) {
+        TcWs w = {};
+        if (save) tc_ws_carve(g, WS_FWD | WS_KEEP, saved, &w);
+        else tc_ws_carve(g, WS_FWD, workspace, &w);
+        rc = launch_status(tc_chunk_prep(g, t, w, save, s, rec));
+        if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, save ? 2 : 0, s, rec));
+    } else if (use_tc_fwd(g, dtype)) {
         rc = launch_status(tc_fwd(g, t, workspace, s, rec));
     } else {
         const SimtWs w = simt_ws_carve(g, false, workspace);
@@ -98,10 +139,12 @@ static int fwd_impl(const void *q, const void *k, const void *v, const void *alp
     return rc;
 }
 
+// from_saved: the backward from saved activations (kind K_BWD_SAVED) with its buffer `saved`
 static int bwd_impl(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
                     const float *S0, const void *dout, const void *du, const float *dS_T, void *dq, void *dk_,
                     void *dv_, void *dalpha, void *dbeta, float *dS0, int B, int T, int H, int dk, int dv, int variant,
-                    int chunk, int dtype, void *workspace, size_t ws_bytes_given, void *stream, Rec &rec) {
+                    int chunk, int dtype, bool from_saved, const void *saved, size_t saved_given, void *workspace,
+                    size_t ws_bytes_given, void *stream, Rec &rec) {
     Geo g;
     int rc = check_shape(B, T, H, dk, dv, variant, chunk, dtype, &g);
     if (rc != DR_OK) return rc;
@@ -116,17 +159,24 @@ static int bwd_impl(const void *q, const void *k, const void *v, const void *alp
         if (p && !aligned16(p)) return DR_ERR_ALIGN;
     if (!aligned_elem(beta, dtype) || !aligned_elem(dbeta, dtype)) return DR_ERR_ALIGN;
     if (variant == DR_GATED && (!aligned_elem(alpha, dtype) || !aligned_elem(dalpha, dtype))) return DR_ERR_ALIGN;
-    const size_t need = ws_bytes(g, dtype, true);
-    if (!workspace || ws_bytes_given < need) return DR_ERR_WORKSPACE;
-    if (((uintptr_t)workspace & 255u) != 0) return DR_ERR_ALIGN;
+    const int kind = from_saved ? K_BWD_SAVED : K_BWD;
+    rc = check_buffer(workspace, ws_bytes_given, ws_bytes(g, dtype, kind));
+    if (rc == DR_OK && from_saved) rc = check_buffer(saved, saved_given, saved_bytes(g, dtype));
+    if (rc != DR_OK) return rc;
     Tensors t = {};
     t.q = q; t.k = k; t.v = v; t.alpha = alpha; t.beta = beta; t.S0 = S0;
     t.dout = dout; t.du = du; t.dS_T = dS_T;
     t.dq = dq; t.dk = dk_; t.dv = dv_; t.dalpha = dalpha; t.dbeta = dbeta; t.dS0 = dS0;
-    if (tc_split_supported(g, dtype == DR_BF16)) {
-        const TcWs w = tc_ws_carve(g, true, workspace);
-        rc = launch_status(tc_chunk_prep(g, t, w, true, s, rec));
-        if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, true, s, rec));
+    if (use_split(g, dtype)) {
+        TcWs w = {};
+        if (from_saved) {
+            tc_ws_carve(g, WS_FWD | WS_KEEP, const_cast<void *>(saved), &w);
+            tc_ws_carve(g, WS_REV, workspace, &w);
+        } else {
+            tc_ws_carve(g, WS_FWD | WS_KEEP | WS_REV, workspace, &w);
+            rc = launch_status(tc_chunk_prep(g, t, w, true, s, rec));
+            if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, 1, s, rec));
+        }
         if (rc == DR_OK) rc = launch_status(tc_chain_rev(g, t, w, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_bwd_chunk(g, t, w, s, rec));
     } else {
@@ -138,28 +188,35 @@ static int bwd_impl(const void *q, const void *k, const void *v, const void *alp
 }
 
 // Number of kernel launches of one call and their names (launch order).
-static int launch_plan(const Geo &g, int dtype, bool bwd, const char **names, int max_names) {
+static int launch_plan(const Geo &g, int dtype, int kind, const char **names, int max_names) {
+    static const char *const SPLIT_FWD[2] = {"k_chunk_prep", "k_chain_fwd"};
+    static const char *const SPLIT_FWD_SAVE[2] = {"k_chunk_prep(keep)", "k_chain_fwd(keep)"};
+    static const char *const SPLIT_BWD[4] = {"k_chunk_prep(keep)", "k_chain_fwd(recompute)", "k_chain_rev",
+                                             "k_bwd_chunk_tc"};
+    static const char *const SPLIT_BWD_SAVED[2] = {"k_chain_rev", "k_bwd_chunk_tc"};
     int n = 0;
     const char *const *src = nullptr;
     if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
-    if (!bwd && use_tc_fwd(g, dtype)) {
-        n = tc_fwd_launches(g, names, max_names);
-        return n;
-    }
-    if (bwd && tc_split_supported(g, dtype == DR_BF16)) {
-        src = TC_BWD_KERNELS;
-        n = 4;
+    if (use_split(g, dtype)) {
+        switch (kind) {
+            case K_FWD: src = SPLIT_FWD; n = 2; break;
+            case K_FWD_SAVE: src = SPLIT_FWD_SAVE; n = 2; break;
+            case K_BWD: src = SPLIT_BWD; n = 4; break;
+            default: src = SPLIT_BWD_SAVED; n = 2; break;
+        }
+    } else if (!is_bwd(kind) && use_tc_fwd(g, dtype)) {
+        return tc_fwd_launches(g, names, max_names);
     } else {
-        src = bwd ? SIMT_BWD_KERNELS : SIMT_FWD_KERNELS;
-        n = bwd ? 5 : 3;
+        src = is_bwd(kind) ? SIMT_BWD_KERNELS : SIMT_FWD_KERNELS;
+        n = is_bwd(kind) ? 5 : 3;
     }
     for (int i = 0; names && i < n && i < max_names; ++i) names[i] = src[i];
     return n;
 }
 
-static int make_rec(const Geo &g, int dtype, bool bwd, void *const *events, int n_events, Rec *rec) {
+static int make_rec(const Geo &g, int dtype, int kind, void *const *events, int n_events, Rec *rec) {
     if (n_events == 0 || events == nullptr) return DR_OK;
-    const int n = launch_plan(g, dtype, bwd, nullptr, 0);
+    const int n = launch_plan(g, dtype, kind, nullptr, 0);
     if (n_events < n + 1) return DR_ERR_ARG;
     rec->ev = (cudaEvent_t *)events;
     rec->n = n + 1;
@@ -171,23 +228,49 @@ extern "C" int delta_rule_fwd(const void *q, const void *k, const void *v, const
                               int variant, int chunk, int dtype, void *workspace, size_t ws_bytes_given,
                               void *stream) {
     Rec rec;
-    return fwd_impl(q, k, v, alpha, beta, S0, out, u, S_T, B, T, H, dk, dv, variant, chunk, dtype, workspace,
-                    ws_bytes_given, stream, rec);
+    return fwd_impl(q, k, v, alpha, beta, S0, out, u, S_T, B, T, H, dk, dv, variant, chunk, dtype, false, nullptr, 0,
+                    workspace, ws_bytes_given, stream, rec);
+}
+
+extern "C" int delta_rule_fwd_save(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                                   const float *S0, void *out, void *u, float *S_T, int B, int T, int H, int dk,
+                                   int dv, int variant, int chunk, int dtype, void *saved, size_t saved_given,
+                                   void *workspace, size_t ws_bytes_given, void *stream) {
+    Rec rec;
+    return fwd_impl(q, k, v, alpha, beta, S0, out, u, S_T, B, T, H, dk, dv, variant, chunk, dtype, true, saved,
+                    saved_given, workspace, ws_bytes_given, stream, rec);
+}
+
+static int fwd_timed(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                     const float *S0, void *out, void *u, float *S_T, int B, int T, int H, int dk, int dv, int variant,
+                     int chunk, int dtype, bool save, void *saved, size_t saved_given, void *workspace,
+                     size_t ws_bytes_given, void *stream, void *const *events, int n_events) {
+    Geo g;
+    int rc = check_shape(B, T, H, dk, dv, variant, chunk, dtype, &g);
+    if (rc != DR_OK) return rc;
+    Rec rec;
+    rc = make_rec(g, dtype, save ? K_FWD_SAVE : K_FWD, events, n_events, &rec);
+    if (rc != DR_OK) return rc;
+    rc = fwd_impl(q, k, v, alpha, beta, S0, out, u, S_T, B, T, H, dk, dv, variant, chunk, dtype, save, saved,
+                  saved_given, workspace, ws_bytes_given, stream, rec);
+    return (rc == DR_OK && rec.bad) ? DR_ERR_ARG : rc;
 }
 
 extern "C" int delta_rule_fwd_timed(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
                                     const float *S0, void *out, void *u, float *S_T, int B, int T, int H, int dk,
                                     int dv, int variant, int chunk, int dtype, void *workspace, size_t ws_bytes_given,
                                     void *stream, void *const *events, int n_events) {
-    Geo g;
-    int rc = check_shape(B, T, H, dk, dv, variant, chunk, dtype, &g);
-    if (rc != DR_OK) return rc;
-    Rec rec;
-    rc = make_rec(g, dtype, false, events, n_events, &rec);
-    if (rc != DR_OK) return rc;
-    rc = fwd_impl(q, k, v, alpha, beta, S0, out, u, S_T, B, T, H, dk, dv, variant, chunk, dtype, workspace,
-                  ws_bytes_given, stream, rec);
-    return (rc == DR_OK && rec.bad) ? DR_ERR_ARG : rc;
+    return fwd_timed(q, k, v, alpha, beta, S0, out, u, S_T, B, T, H, dk, dv, variant, chunk, dtype, false, nullptr, 0,
+                     workspace, ws_bytes_given, stream, events, n_events);
+}
+
+extern "C" int delta_rule_fwd_save_timed(const void *q, const void *k, const void *v, const void *alpha,
+                                         const void *beta, const float *S0, void *out, void *u, float *S_T, int B,
+                                         int T, int H, int dk, int dv, int variant, int chunk, int dtype, void *saved,
+                                         size_t saved_given, void *workspace, size_t ws_bytes_given, void *stream,
+                                         void *const *events, int n_events) {
+    return fwd_timed(q, k, v, alpha, beta, S0, out, u, S_T, B, T, H, dk, dv, variant, chunk, dtype, true, saved,
+                     saved_given, workspace, ws_bytes_given, stream, events, n_events);
 }
 
 extern "C" int delta_rule_bwd(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
@@ -197,7 +280,33 @@ extern "C" int delta_rule_bwd(const void *q, const void *k, const void *v, const
                               void *stream) {
     Rec rec;
     return bwd_impl(q, k, v, alpha, beta, S0, dout, du, dS_T, dq, dk_, dv_, dalpha, dbeta, dS0, B, T, H, dk, dv,
-                    variant, chunk, dtype, workspace, ws_bytes_given, stream, rec);
+                    variant, chunk, dtype, false, nullptr, 0, workspace, ws_bytes_given, stream, rec);
+}
+
+extern "C" int delta_rule_bwd_saved(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                                    const float *S0, const void *dout, const void *du, const float *dS_T, void *dq,
+                                    void *dk_, void *dv_, void *dalpha, void *dbeta, float *dS0, int B, int T, int H,
+                                    int dk, int dv, int variant, int chunk, int dtype, const void *saved,
+                                    size_t saved_given, void *workspace, size_t ws_bytes_given, void *stream) {
+    Rec rec;
+    return bwd_impl(q, k, v, alpha, beta, S0, dout, du, dS_T, dq, dk_, dv_, dalpha, dbeta, dS0, B, T, H, dk, dv,
+                    variant, chunk, dtype, true, saved, saved_given, workspace, ws_bytes_given, stream, rec);
+}
+
+static int bwd_timed(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                     const float *S0, const void *dout, const void *du, const float *dS_T, void *dq, void *dk_,
+                     void *dv_, void *dalpha, void *dbeta, float *dS0, int B, int T, int H, int dk, int dv,
+                     int variant, int chunk, int dtype, bool from_saved, const void *saved, size_t saved_given,
+                     void *workspace, size_t ws_bytes_given, void *stream, void *const *events, int n_events) {
+    Geo g;
+    int rc = check_shape(B, T, H, dk, dv, variant, chunk, dtype, &g);
+    if (rc != DR_OK) return rc;
+    Rec rec;
+    rc = make_rec(g, dtype, from_saved ? K_BWD_SAVED : K_BWD, events, n_events, &rec);
+    if (rc != DR_OK) return rc;
+    rc = bwd_impl(q, k, v, alpha, beta, S0, dout, du, dS_T, dq, dk_, dv_, dalpha, dbeta, dS0, B, T, H, dk, dv,
+                  variant, chunk, dtype, from_saved, saved, saved_given, workspace, ws_bytes_given, stream, rec);
+    return (rc == DR_OK && rec.bad) ? DR_ERR_ARG : rc;
 }
 
 extern "C" int delta_rule_bwd_timed(const void *q, const void *k, const void *v, const void *alpha,
@@ -206,15 +315,20 @@ extern "C" int delta_rule_bwd_timed(const void *q, const void *k, const void *v,
                                     float *dS0, int B, int T, int H, int dk, int dv, int variant, int chunk,
                                     int dtype, void *workspace, size_t ws_bytes_given, void *stream,
                                     void *const *events, int n_events) {
-    Geo g;
-    int rc = check_shape(B, T, H, dk, dv, variant, chunk, dtype, &g);
-    if (rc != DR_OK) return rc;
-    Rec rec;
-    rc = make_rec(g, dtype, true, events, n_events, &rec);
-    if (rc != DR_OK) return rc;
-    rc = bwd_impl(q, k, v, alpha, beta, S0, dout, du, dS_T, dq, dk_, dv_, dalpha, dbeta, dS0, B, T, H, dk, dv,
-                  variant, chunk, dtype, workspace, ws_bytes_given, stream, rec);
-    return (rc == DR_OK && rec.bad) ? DR_ERR_ARG : rc;
+    return bwd_timed(q, k, v, alpha, beta, S0, dout, du, dS_T, dq, dk_, dv_, dalpha, dbeta, dS0, B, T, H, dk, dv,
+                     variant, chunk, dtype, false, nullptr, 0, workspace, ws_bytes_given, stream, events, n_events);
+}
+
+extern "C" int delta_rule_bwd_saved_timed(const void *q, const void *k, const void *v, const void *alpha,
+                                          const void *beta, const float *S0, const void *dout, const void *du,
+                                          const float *dS_T, void *dq, void *dk_, void *dv_, void *dalpha,
+                                          void *dbeta, float *dS0, int B, int T, int H, int dk, int dv, int variant,
+                                          int chunk, int dtype, const void *saved, size_t saved_given,
+                                          void *workspace, size_t ws_bytes_given, void *stream, void *const *events,
+                                          int n_events) {
+    return bwd_timed(q, k, v, alpha, beta, S0, dout, du, dS_T, dq, dk_, dv_, dalpha, dbeta, dS0, B, T, H, dk, dv,
+                     variant, chunk, dtype, true, saved, saved_given, workspace, ws_bytes_given, stream, events,
+                     n_events);
 }
 
 extern "C" int delta_rule_launches(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype,
@@ -222,7 +336,8 @@ extern "C" int delta_rule_launches(int B, int T, int H, int dk, int dv, int vari
     Geo g;
     const int rc = check_shape(B, T, H, dk, dv, variant, chunk, dtype, &g);
     if (rc != DR_OK) return rc;
-    return launch_plan(g, dtype, for_bwd != 0, names, max_names);
+    if (for_bwd < 0 || for_bwd > 3) return DR_ERR_ARG;
+    return launch_plan(g, dtype, for_bwd, names, max_names);
 }
 
 extern "C" const char *delta_rule_strerror(int code) {

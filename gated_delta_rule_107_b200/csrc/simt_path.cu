@@ -621,8 +621,6 @@ template <typename K> static cudaError_t prep_attr(K kern, size_t smem) {
 
 const char *const SIMT_FWD_KERNELS[3] = {"k_prep", "k_scan", "k_out"};
 const char *const SIMT_BWD_KERNELS[5] = {"k_prep", "k_scan", "k_scan_bwd", "k_bwd_state", "k_bwd_intra"};
-const char *const TC_BWD_KERNELS[4] = {"k_chunk_prep(bwd)", "k_chain_fwd(recompute)", "k_chain_rev",
-                                       "k_bwd_chunk_tc"};
 
 template <typename TI>
 static cudaError_t forward_chain(const Geo &g, const IO<TI> &io, const SimtWs &w, const float *S0, float *ST,

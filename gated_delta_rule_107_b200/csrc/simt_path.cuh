@@ -28,6 +28,5 @@ cudaError_t simt_bwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w,
 // kernel names in launch order (for the timed entry points)
 extern const char *const SIMT_FWD_KERNELS[3];
 extern const char *const SIMT_BWD_KERNELS[5];
-extern const char *const TC_BWD_KERNELS[4];
 
 }  // namespace dr

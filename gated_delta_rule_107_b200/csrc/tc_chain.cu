@@ -2,8 +2,7 @@
 // (Gated DeltaNet and DeltaNet; bf16 I/O, dk = dv = 128, C = 64).
 //
 // Chunked form of "线性注意力架构演进与Kimi Delta Attention创新实践" (sections 2.1, 6.1,
-// 6.2, 7.1), given the per-chunk products of tc_prep.cu (W, U~, P, g, and for the backward
-// P^T dO).  One CTA per (b, h, 64 value channels) walks the chunks in order; the state
+// 6.2, 7.1), given the per-chunk products of tc_prep.cu (W, U~, P, g).  One CTA per (b, h, 64 value channels) walks the chunks in order; the state
 // block (128 key rows x 64 value columns) stays in fp32 registers, one row per thread, with a
 // bf16 copy in shared memory as the MMA operand.
 //
@@ -18,9 +17,9 @@
 //   dL/dS_n = e^{g_C} dS+ + q^T diag(e^g) dO - W^T dU
 //   and the row sums U_r . (diag(e^{g_C - g}) k dS+)_r of its 64 columns (a term of d log alpha)
 //
-// Warp 0 is a TMA producer that keeps two chunks of operands in flight; warps 1-4 run the
-// chain (thread = TMEM lane = state row).  Every wait is bounded (~1 s) and aborts are
-// agreed on per warpgroup.
+// Warp 0 is a TMA producer that keeps two chunks of operands in flight; warps 1-8 run the
+// chain (a TMEM lane = a state row; two warps per lane quarter split the value columns).
+// Every wait is bounded (~1 s) and aborts are agreed on by the chain warps.
 #include <limits.h>
 
 #include "tc_host.cuh"
@@ -37,13 +36,13 @@ using dr::tcf::st_chunk;
 using dr::tcf::tmem_row64;
 
 constexpr int C = 64, DK = 128, DV = 128, DVB = 64;
-constexpr int NTHREADS = 160;
+constexpr int NTHREADS = 288;  // warp 0 producer, warps 1-8 chain
 // shared memory (bytes from a 1024-aligned base): two stages of 80K, then the chain's tiles
 constexpr uint32_t STAGE = 81920;
 // forward stage: [W_p0 | q_p0 | W_p1 | q_p1], [U~ (this CTA's 64 columns) | P], [k_p0 | k_p1]
 constexpr uint32_t FS_WQ = 0, FS_UP = 32768, FS_K = 49152;
-// reverse stage: k, q, W (2 panels each); dO, P^T dO, du, U (this CTA's 64 columns)
-constexpr uint32_t RS_K = 0, RS_Q = 16384, RS_W = 32768, RS_DO = 49152, RS_DU = 57344, RS_DX = 65536,
+// reverse stage: k, q, W (2 panels each); dO (this CTA's 64 columns); P; du, U (this CTA's 64 columns)
+constexpr uint32_t RS_K = 0, RS_Q = 16384, RS_W = 32768, RS_DO = 49152, RS_P = 57344, RS_DX = 65536,
                    RS_UN = 73728;
 constexpr uint32_t OFF_S = 2 * STAGE;         // 16K  bf16 state [c][j]
 constexpr uint32_t OFF_U = OFF_S + 16384;     //  8K  U [r][j]        (reverse: dU [r][j])
@@ -55,8 +54,9 @@ constexpr uint32_t SMEM_BYTES = OFF_MISC + 4096;
 constexpr uint32_t M_BAR = 0;  // FULL0, FULL1, EMPTY0, EMPTY1, MMA
 constexpr uint32_t M_TMEM = 64, M_ABORT = 68;
 constexpr uint32_t M_CF = 256;  // per stage: [0..63] e^{g_C - g}, [64..127] e^g, [128] e^{g_C}
+constexpr uint32_t M_SKP = M_CF + 2 * 132 * 4;  // reverse: [2 column halves][64] row-sum partials
 enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_MMA, B_NUM };
-static_assert(M_CF + 2 * 132 * 4 <= 4096, "misc overflow");
+static_assert(M_SKP + 512 <= 4096, "misc overflow");
 
 struct FMaps {
     CUtensorMap q, k;       // [B, T, H, 128] bf16; box 64 x 64 tokens
@@ -67,7 +67,8 @@ struct FMaps {
 };
 struct RMaps {
     CUtensorMap q, k, dout, du;  // [B, T, H, 128] bf16
-    CUtensorMap W, dUp, Un;      // [chunks * 64][128] bf16 (loads)
+    CUtensorMap W, Un;           // [chunks * 64][128] bf16 (loads)
+    CUtensorMap P;               // [chunks * 64][64] bf16 (load)
     CUtensorMap dUn;             // [chunks * 64][128] bf16 (store)
     CUtensorMap dSn;             // [chunks * 128][128] bf16, box 64 x 128 (store)
 };
@@ -94,9 +95,28 @@ __device__ __forceinline__ void chunk_factors(const float *gb, size_t ci, float 
     if (lane == 0) cf[128] = __expf(gC);
 }
 
+// Chain thread layout: warps 1-8, two per TMEM lane quarter (warp & 3); the first four take
+// value columns 0-31 of this CTA's 64, the other four columns 32-63.
+struct ChainLane {
+    int wc, q4, hf, trow, cb;
+    __device__ ChainLane(int warp, int lane)
+        : wc((warp - 1) * 32 + lane), q4(warp & 3), hf((warp - 1) >> 2), trow((warp & 3) * 32 + lane),
+          cb(((warp - 1) >> 2) * 32) {}
+};
+
+// 32 fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_row32(uint32_t taddr, float *v) {
+    tmem_ld16(taddr, v);
+    tmem_ld16(taddr + 16, v + 16);
+    wait_ld();
+}
+
 // ====================================== forward chain ======================================
-template <int BWD>
+// MODE 0: forward (o, u, S_T); 1: recompute for the backward (S_n, U of every chunk);
+// 2: forward that also keeps S_n and U for the backward.
+template <int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant__ FMaps mp, Args a) {
+    constexpr bool OUT = MODE != 1, KEEP = MODE != 0;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -131,15 +151,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             if (m >= 2 && !mbar_wait(&bar[B_EMPTY0 + s], ((m >> 1) - 1) & 1, abort_flag)) break;
             unsigned char *st = sm + s * STAGE;
             if (lane == 0) {
-                mbar_arrive_tx(&bar[B_FULL0 + s], BWD ? 40960u : 65536u);
+                mbar_arrive_tx(&bar[B_FULL0 + s], OUT ? 65536u : 40960u);
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
                     tma_load_2d(st + FS_WQ + p * 16384, &mp.W, 64 * p, ci * C, &bar[B_FULL0 + s]);
-                    if (!BWD) tma_load_4d(st + FS_WQ + p * 16384 + 8192, &mp.q, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
+                    if (OUT) tma_load_4d(st + FS_WQ + p * 16384 + 8192, &mp.q, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
                     tma_load_4d(st + FS_K + p * 8192, &mp.k, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
                 }
                 tma_load_2d(st + FS_UP, &mp.Ut, j0, ci * C, &bar[B_FULL0 + s]);
-                if (!BWD) tma_load_2d(st + FS_UP + 8192, &mp.P, 0, ci * C, &bar[B_FULL0 + s]);
+                if (OUT) tma_load_2d(st + FS_UP + 8192, &mp.P, 0, ci * C, &bar[B_FULL0 + s]);
             }
             chunk_factors(a.gb, (size_t)ci, cf_all + s * 132, lane);
             __syncwarp();
@@ -153,13 +173,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
         }
     } else {
         // ================================ chain ================================
-        const int wc = threadIdx.x - 32;
-        const int q4 = warp & 3, trow = q4 * 32 + lane;
-        const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
+        const ChainLane cl(warp, lane);
+        const int wc = cl.wc, trow = cl.trow, hf = cl.hf, cb = cl.cb;
+        const uint32_t tl = tbase + ((uint32_t)(cl.q4 * 32) << 16) + (uint32_t)cb;
         constexpr uint32_t TM_D = 0, TM_E = 256;  // D / O' double-buffered at 0 and 128
+        const bool ostore = trow == 64 && hf == 0;  // issues the o stores
         uint32_t ph = 0;
         bool pending = false;
-        auto wabort = [&](bool ok) -> bool { return named_sync_any(2, 128, !ok || *abort_flag != 0); };
+        auto wabort = [&](bool ok) -> bool { return named_sync_any(2, 256, !ok || *abort_flag != 0); };
         auto mma_done = [&]() -> bool {
             const bool ok = mbar_wait(&bar[B_MMA], ph & 1, abort_flag);
             ph++;
@@ -169,36 +190,36 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             return go;
         };
         const uint32_t sS = smem_u32(sm + OFF_S), sU = smem_u32(sm + OFF_U), sUD = smem_u32(sm + OFF_UD);
-        float S[DVB];
+        float S[32];  // state row trow, value columns j0 + cb ... + 31
         {
-            const float *s0 = a.S0 ? a.S0 + (((size_t)b * H + h) * DK + trow) * DV + j0 : nullptr;
+            const float *s0 = a.S0 ? a.S0 + (((size_t)b * H + h) * DK + trow) * DV + j0 + cb : nullptr;
 #pragma unroll
-            for (int j = 0; j < DVB; ++j) S[j] = s0 ? s0[j] : 0.f;
+            for (int j = 0; j < 32; ++j) S[j] = s0 ? s0[j] : 0.f;
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_S, swz(trow, ch), S + ch * 8);
+            for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + OFF_S, swz(trow, hf * 4 + c4), S + c4 * 8);
         }
         fence_proxy_async();
-        named_sync(2, 128);
-        // o of the previous chunk is finished by lanes 64-127 while the next chunk starts
+        named_sync(2, 256);
+        // o of the previous chunk is finished by lanes 64-127 while the next chunk starts: they
+        // stage it in OFF_O and one of them issues its TMA store (rows past T are clipped)
         int prev_L = 0, prev_t0 = 0;
         float prev_eg = 0.f;
         uint32_t prev_buf = 0;
-        // lanes 64-127 stage o in OFF_O; lane 64 issues its TMA store (rows past T are clipped)
         auto o_epilogue = [&]() {
-            if (BWD || trow < 64 || prev_L == 0 || !a.has_out) return;
+            if (!OUT || trow < 64 || prev_L == 0 || !a.has_out) return;
             const int r = trow - 64;
-            float d[64], p[64];
-            tmem_row64(tl + TM_D + prev_buf, d);
-            tmem_row64(tl + TM_D + prev_buf + 64, p);
+            float d[32], p[32];
+            tmem_row32(tl + TM_D + prev_buf, d);
+            tmem_row32(tl + TM_D + prev_buf + 64, p);
 #pragma unroll
-            for (int j = 0; j < 64; ++j) d[j] = prev_eg * d[j] + p[j];
-            if (trow == 64) bulk_wait_read_all();  // the previous o store has read OFF_O
-            named_sync(3, 64);
+            for (int j = 0; j < 32; ++j) d[j] = prev_eg * d[j] + p[j];
+            if (ostore) bulk_wait_read_all();  // the previous o store has read OFF_O
+            named_sync(3, 128);
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_O, swz(r, ch), d + ch * 8);
+            for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + OFF_O, swz(r, hf * 4 + c4), d + c4 * 8);
             fence_proxy_async();
-            named_sync(3, 64);
-            if (trow == 64) {
+            named_sync(3, 128);
+            if (ostore) {
                 tma_store_4d(&mp.out, sm + OFF_O, j0, h, prev_t0, b);
                 bulk_commit();
             }
@@ -225,7 +246,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
                     mma_bf16(tbase + TM_D + buf, sdesc(swq + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
                              sdesc(sS + k * 2048, 1024, 1024), id, k > 0);
                 mma_commit(&bar[B_MMA]);
-                if (BWD) {  // the state entering chunk m, straight from its bf16 operand tile
+                if (KEEP) {  // the state entering chunk m, straight from its bf16 operand tile
                     tma_store_2d(&mp.Sn, sm + OFF_S, j0, (int)ci * DK);
                     bulk_commit();
                 }
@@ -233,24 +254,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             pending = true;
             o_epilogue();  // previous chunk, lanes 64-127
             if (!mma_done()) break;
-            // ---------------- U = U~ - W S;  u;  U and e^{gC - g} U tiles ----------------
+            // ---------------- U = U~ - W S;  U and e^{gC - g} U tiles ----------------
             if (trow < 64) {
                 const int r = trow;
-                float v[64];
-                tmem_row64(tl + TM_D + buf, v);
+                float v[32];
+                tmem_row32(tl + TM_D + buf, v);
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const uint32_t o = swz(r, hf * 4 + c4);
                     float ut[8];
-                    ld_chunk(st + FS_UP, swz(r, ch), ut);
+                    ld_chunk(st + FS_UP, o, ut);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) v[ch * 8 + e] = ut[e] - v[ch * 8 + e];
+                    for (int e = 0; e < 8; ++e) ut[e] -= v[c4 * 8 + e];
+                    st_chunk(sm + OFF_U, o, ut);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ut[e] *= rowf;
+                    st_chunk(sm + OFF_UD, o, ut);
                 }
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_U, swz(r, ch), v + ch * 8);
-#pragma unroll
-                for (int j = 0; j < 64; ++j) v[j] *= rowf;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_UD, swz(r, ch), v + ch * 8);
             }
             fence_proxy_async();
             fence_before_sync();
@@ -258,20 +278,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             // ---------------- E = k^T (e^{gC-g} U);  O' = [* ; P] U;  U out ----------------
             if (wc == 0) {
                 fence_after_sync();
-                if (BWD) {
-                    tma_store_2d(&mp.Un, sm + OFF_U, j0, (int)ci * C);
-                    bulk_commit();
-                } else if (a.has_u) {
-                    tma_store_4d(&mp.u, sm + OFF_U, j0, h, t0, b);
-                    bulk_commit();
-                }
+                if (KEEP) tma_store_2d(&mp.Un, sm + OFF_U, j0, (int)ci * C);
+                if (OUT && a.has_u) tma_store_4d(&mp.u, sm + OFF_U, j0, h, t0, b);
+                if (KEEP || (OUT && a.has_u)) bulk_commit();
                 const uint32_t sk = smem_u32(st + FS_K), sup = smem_u32(st + FS_UP);
                 const uint32_t ide = idesc_bf16(128, 64, 1, 1), ido = idesc_bf16(128, 64, 0, 1);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     mma_bf16(tbase + TM_E, sdesc(sk + k * 2048, 8192, 1024), sdesc(sUD + k * 2048, 1024, 1024), ide,
                              k > 0);
-                if (!BWD) {
+                if (OUT) {
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
                         mma_bf16(tbase + TM_D + buf + 64, sdesc(sup + k * 32, 16, 1024), sdesc(sU + k * 2048, 1024, 1024),
@@ -280,17 +296,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
                 mma_commit(&bar[B_MMA]);
             }
             pending = true;
-            if (BWD && wc == 0) bulk_wait_read_1();  // the S_m store has read OFF_S
+            if (KEEP && wc == 0) bulk_wait_read_1();  // the S_m store has read OFF_S
             if (!mma_done()) break;
             if (wc == 0) mbar_arrive(&bar[B_EMPTY0 + s]);
             // ---------------- S <- e^{gC} S + E ----------------
             {
-                float ev[64];
-                tmem_row64(tl + TM_E, ev);
+                float ev[32];
+                tmem_row32(tl + TM_E, ev);
 #pragma unroll
-                for (int j = 0; j < DVB; ++j) S[j] = egC * S[j] + ev[j];
+                for (int j = 0; j < 32; ++j) S[j] = egC * S[j] + ev[j];
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_S, swz(trow, ch), S + ch * 8);
+                for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + OFF_S, swz(trow, hf * 4 + c4), S + c4 * 8);
             }
             fence_proxy_async();
             fence_before_sync();
@@ -298,12 +314,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             prev_L = L; prev_t0 = t0; prev_eg = rowf; prev_buf = buf;
         }
         if (*abort_flag == 0) o_epilogue();  // last chunk
-        if (wc == 0 || trow == 64) bulk_wait_all();
+        if (wc == 0 || ostore) bulk_wait_all();
         if (*abort_flag == 0) {
-            if (!BWD && a.ST) {
-                float *dst = a.ST + (((size_t)b * H + h) * DK + trow) * DV + j0;
+            if (OUT && a.ST) {
+                float *dst = a.ST + (((size_t)b * H + h) * DK + trow) * DV + j0 + cb;
 #pragma unroll
-                for (int j = 0; j < DVB; j += 4)
+                for (int j = 0; j < 32; j += 4)
                     *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
             }
         } else if (pending) {
@@ -326,6 +342,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + M_TMEM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + M_ABORT);
     float *cf_all = reinterpret_cast<float *>(sm + OFF_MISC + M_CF);
+    float *skp = reinterpret_cast<float *>(sm + OFF_MISC + M_SKP);
 
     const int half = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int j0 = half * DVB;
@@ -338,7 +355,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0) tmem_alloc(tmem_slot, 128);
+    if (warp == 0) tmem_alloc(tmem_slot, 256);
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
@@ -361,7 +378,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
                     tma_load_2d(st + RS_W + p * 8192, &mp.W, 64 * p, ci * C, &bar[B_FULL0 + s]);
                 }
                 tma_load_4d(st + RS_DO, &mp.dout, j0, h, t0, b, &bar[B_FULL0 + s]);
-                tma_load_2d(st + RS_DU, &mp.dUp, j0, ci * C, &bar[B_FULL0 + s]);
+                tma_load_2d(st + RS_P, &mp.P, 0, ci * C, &bar[B_FULL0 + s]);
                 if (a.has_du) tma_load_4d(st + RS_DX, &mp.du, j0, h, t0, b, &bar[B_FULL0 + s]);
                 tma_load_2d(st + RS_UN, &mp.Un, j0, ci * C, &bar[B_FULL0 + s]);
             }
@@ -377,13 +394,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
         }
     } else {
         // ================================ chain ================================
-        const int wc = threadIdx.x - 32;
-        const int q4 = warp & 3, trow = q4 * 32 + lane;
-        const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
-        constexpr uint32_t TM_A = 0, TM_B = 64;
+        const ChainLane cl(warp, lane);
+        const int wc = cl.wc, trow = cl.trow, hf = cl.hf, cb = cl.cb;
+        const uint32_t tl = tbase + ((uint32_t)(cl.q4 * 32) << 16) + (uint32_t)cb;
+        constexpr uint32_t TM_A = 0, TM_B = 64, TM_P = 128;
         uint32_t ph = 0;
         bool pending = false;
-        auto wabort = [&](bool ok) -> bool { return named_sync_any(2, 128, !ok || *abort_flag != 0); };
+        auto wabort = [&](bool ok) -> bool { return named_sync_any(2, 256, !ok || *abort_flag != 0); };
         auto mma_done = [&]() -> bool {
             const bool ok = mbar_wait(&bar[B_MMA], ph & 1, abort_flag);
             ph++;
@@ -393,16 +410,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
             return go;
         };
         const uint32_t sS = smem_u32(sm + OFF_S), sU = smem_u32(sm + OFF_U);
-        float S[DVB];  // dL/dS of the state leaving the current chunk
+        float S[32];  // dL/dS of the state leaving the current chunk: row trow, columns j0 + cb ...
         {
-            const float *s0 = a.S0 ? a.S0 + (((size_t)b * H + h) * DK + trow) * DV + j0 : nullptr;
+            const float *s0 = a.S0 ? a.S0 + (((size_t)b * H + h) * DK + trow) * DV + j0 + cb : nullptr;
 #pragma unroll
-            for (int j = 0; j < DVB; ++j) S[j] = s0 ? s0[j] : 0.f;
+            for (int j = 0; j < 32; ++j) S[j] = s0 ? s0[j] : 0.f;
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_S, swz(trow, ch), S + ch * 8);
+            for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + OFF_S, swz(trow, hf * 4 + c4), S + c4 * 8);
         }
         fence_proxy_async();
-        named_sync(2, 128);
+        named_sync(2, 256);
         for (int m = 0; m < N; ++m) {
             const int mc = N - 1 - m, s = m & 1;
             const size_t ci = ci0 + mc;
@@ -411,80 +428,81 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
             if (wabort(got)) break;
             const float *cf = cf_all + s * 132;
             const float egC = cf[128];
-            // ---------------- D_a = k dS+  (M = 128: rows 64..127 discarded) ----------------
+            // ------- D_a = k dS+, D_p = P^T dO  (M = 128: rows 64..127 discarded) -------
             if (wc == 0) {
                 fence_after_sync();
                 bulk_wait_read_all();  // the previous chunk's dU store has read OFF_U
-                const uint32_t id = idesc_bf16(128, 64, 0, 1);
-                const uint32_t sk = smem_u32(st + RS_K);
+                const uint32_t id = idesc_bf16(128, 64, 0, 1), idp = idesc_bf16(128, 64, 1, 1);
+                const uint32_t sk = smem_u32(st + RS_K), sp = smem_u32(st + RS_P), sdo = smem_u32(st + RS_DO);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
                     mma_bf16(tbase + TM_A, sdesc(sk + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024),
                              sdesc(sS + k * 2048, 1024, 1024), id, k > 0);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16(tbase + TM_P, sdesc(sp + k * 2048, 8192, 1024), sdesc(sdo + k * 2048, 1024, 1024), idp,
+                             k > 0);
                 mma_commit(&bar[B_MMA]);
                 tma_store_2d(&mp.dSn, sm + OFF_S, j0, (int)ci * DK);  // dS_{n+1} from its operand tile
                 bulk_commit();
             }
             pending = true;
-            // dO rows scaled by e^{g_r} (for q^T diag(e^g) dO) while the MMA runs
-            for (int x = wc; x < 512; x += 128) {
+            // q rows scaled by e^{g_r} (for q^T diag(e^g) dO) while the MMAs run
+            for (int x = wc; x < 1024; x += 256) {  // 2 panels x 64 rows x 8 chunks of 16 B
                 float v[8];
-                ld_chunk(st + RS_DO, (uint32_t)x * 16, v);
-                const float f = cf[64 + (x >> 3)];
+                ld_chunk(st + RS_Q, (uint32_t)x * 16, v);
+                const float f = cf[64 + ((x >> 3) & 63)];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) v[e] *= f;
-                st_chunk(st + RS_DO, (uint32_t)x * 16, v);
+                st_chunk(st + RS_Q, (uint32_t)x * 16, v);
             }
             fence_proxy_async();
             fence_before_sync();
             if (wabort(true)) break;
-            // ---------------- D_b = q^T diag(e^g) dO  (first half of dL/dS_n) ----------------
+            // ---------------- D_b = (diag(e^g) q)^T dO  (first half of dL/dS_n) ----------------
             if (wc == 0) {
                 fence_after_sync();
-                const uint32_t id = idesc_bf16(128, 64, 1, 1);
+                const uint32_t idb = idesc_bf16(128, 64, 1, 1);
                 const uint32_t sq = smem_u32(st + RS_Q), sdo = smem_u32(st + RS_DO);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_bf16(tbase + TM_B, sdesc(sq + k * 2048, 8192, 1024), sdesc(sdo + k * 2048, 1024, 1024), id,
+                    mma_bf16(tbase + TM_B, sdesc(sq + k * 2048, 8192, 1024), sdesc(sdo + k * 2048, 1024, 1024), idb,
                              k > 0);
             }
             if (!mma_done()) break;
-            // ---------------- dU = du + P^T dO + diag(e^{gC - g}) D_a;  U_r . (Kbar dS+)_r ----------------
+        // ---------------- dU = du + P^T dO + diag(e^{gC - g}) D_a;  U_r . (Kbar dS+)_r ----------------
             if (trow < 64) {
                 const int r = trow;
                 const float f = cf[r];
-                float rs = 0.f;
+                float v[32], pd[32], rs = 0.f;
+                tmem_row32(tl + TM_A, v);
+                tmem_row32(tl + TM_P, pd);
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {  // 32 columns at a time
-                    float v[32];
-                    tmem_ld16(tl + TM_A + hh * 32, v);
-                    tmem_ld16(tl + TM_A + hh * 32 + 16, v + 16);
-                    wait_ld();
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const uint32_t o = swz(r, hf * 4 + c4);
+                    float d[8], x[8], un[8];
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        const int ch = hh * 4 + c4;
-                        float d[8], x[8], un[8];
-                        ld_chunk(st + RS_DU, swz(r, ch), d);
-                        ld_chunk(st + RS_UN, swz(r, ch), un);
-                        if (a.has_du) {
-                            ld_chunk(st + RS_DX, swz(r, ch), x);
+                    for (int e = 0; e < 8; ++e) d[e] = pd[c4 * 8 + e];
+                    ld_chunk(st + RS_UN, o, un);
+                    if (a.has_du) {
+                        ld_chunk(st + RS_DX, o, x);
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) d[e] += x[e];
-                        }
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float kd = f * v[c4 * 8 + e];
-                            rs += un[e] * kd;
-                            d[e] += kd;
-                        }
-                        st_chunk(sm + OFF_U, swz(r, ch), d);
+                        for (int e = 0; e < 8; ++e) d[e] += x[e];
                     }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float kd = f * v[c4 * 8 + e];
+                        rs += un[e] * kd;
+                        d[e] += kd;
+                    }
+                    st_chunk(sm + OFF_U, o, d);
                 }
-                a.skt[ci * 2 * C + half * C + r] = rs;
+                skp[hf * 64 + r] = rs;
             }
             fence_proxy_async();
             fence_before_sync();
             if (wabort(true)) break;
+            if (trow < 64 && hf == 0) a.skt[ci * 2 * C + half * C + trow] = skp[trow] + skp[64 + trow];
             // ---------------- D_b -= W^T dU;  dU out ----------------
             if (wc == 0) {
                 fence_after_sync();
@@ -496,19 +514,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
                 mma_commit(&bar[B_MMA]);
                 tma_store_2d(&mp.dUn, sm + OFF_U, j0, (int)ci * C);
                 bulk_commit();
+                bulk_wait_read_1();  // the dS_{n+1} store has read OFF_S
             }
             pending = true;
-            if (wc == 0) bulk_wait_read_1();  // the dS_{n+1} store has read OFF_S
             if (!mma_done()) break;
             if (wc == 0) mbar_arrive(&bar[B_EMPTY0 + s]);
             // ---------------- dS_n = e^{gC} dS+ + D_b ----------------
             {
-                float dv[64];
-                tmem_row64(tl + TM_B, dv);
+                float dv[32];
+                tmem_row32(tl + TM_B, dv);
 #pragma unroll
-                for (int j = 0; j < DVB; ++j) S[j] = egC * S[j] + dv[j];
+                for (int j = 0; j < 32; ++j) S[j] = egC * S[j] + dv[j];
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_S, swz(trow, ch), S + ch * 8);
+                for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + OFF_S, swz(trow, hf * 4 + c4), S + c4 * 8);
             }
             fence_proxy_async();
             fence_before_sync();
@@ -517,9 +535,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
         if (wc == 0) bulk_wait_all();
         if (*abort_flag == 0) {
             if (a.ST) {
-                float *dst = a.ST + (((size_t)b * H + h) * DK + trow) * DV + j0;
+                float *dst = a.ST + (((size_t)b * H + h) * DK + trow) * DV + j0 + cb;
 #pragma unroll
-                for (int j = 0; j < DVB; j += 4)
+                for (int j = 0; j < 32; j += 4)
                     *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
             }
         } else if (pending) {
@@ -530,7 +548,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
-    if (warp == 0) tmem_dealloc(tbase, 128);
+    if (warp == 0) tmem_dealloc(tbase, 256);
 }
 
 }  // namespace tch
@@ -542,72 +560,81 @@ bool tc_split_supported(const Geo &g, bool bf16) {
 
 static size_t ws_al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Carves the split-path workspace from base; returns the bytes it spans.
-static size_t ws_carve(const Geo &g, bool bwd, char *base, TcWs *w) {
+// Carves the given parts of the split-path workspace from base (or only counts, when base
+// is null); returns the bytes they span.
+static size_t ws_carve(const Geo &g, int parts, char *base, TcWs *w) {
     const size_t nc = (size_t)g.B * g.H * g.N, C = g.C, DK = g.dk, DV = g.dv;
     size_t off = 0;
     auto take = [&](size_t bytes) { char *r = base ? base + off : nullptr; off += ws_al256(bytes); return r; };
-    *w = TcWs{};
-    w->gb = (float *)take(nc * 2 * C * 4);
-    w->W = (__nv_bfloat16 *)take(nc * C * DK * 2);
-    w->Ut = (__nv_bfloat16 *)take(nc * C * DV * 2);
-    w->P = (__nv_bfloat16 *)take(nc * C * C * 2);
-    if (bwd) {
+    if (parts & WS_FWD) {
+        w->gb = (float *)take(nc * 2 * C * 4);
+        w->W = (__nv_bfloat16 *)take(nc * C * DK * 2);
+        w->Ut = (__nv_bfloat16 *)take(nc * C * DV * 2);
+        w->P = (__nv_bfloat16 *)take(nc * C * C * 2);
+    }
+    if (parts & WS_KEEP) {
         w->Tn = (__nv_bfloat16 *)take(nc * C * C * 2);
         w->KK = (__nv_bfloat16 *)take(nc * C * C * 2);
-        w->dUp = (__nv_bfloat16 *)take(nc * C * DV * 2);
         w->Sn = (__nv_bfloat16 *)take(nc * DK * DV * 2);
-        w->dSn = (__nv_bfloat16 *)take(nc * DK * DV * 2);
         w->Un = (__nv_bfloat16 *)take(nc * C * DV * 2);
+    }
+    if (parts & WS_REV) {
+        w->dSn = (__nv_bfloat16 *)take(nc * DK * DV * 2);
         w->dUn = (__nv_bfloat16 *)take(nc * C * DV * 2);
         w->skt = (float *)take(nc * 2 * C * 4);
     }
     return off;
 }
 
-size_t tc_ws_bytes(const Geo &g, bool bwd) {
-    TcWs w;
-    return ws_carve(g, bwd, nullptr, &w);
+size_t tc_ws_bytes(const Geo &g, int parts) {
+    TcWs w = {};
+    return ws_carve(g, parts, nullptr, &w);
 }
 
-TcWs tc_ws_carve(const Geo &g, bool bwd, void *base) {
-    TcWs w;
-    ws_carve(g, bwd, (char *)base, &w);
-    return w;
-}
+void tc_ws_carve(const Geo &g, int parts, void *base, TcWs *w) { ws_carve(g, parts, (char *)base, w); }
 
-cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, bool bwd, cudaStream_t s, Rec &rec) {
+cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, int mode, cudaStream_t s, Rec &rec) {
     using namespace tch;
     FMaps mp;
     const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;
+    const bool out = mode != 1, keep = mode != 0;
     bool ok = tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) && tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64) &&
               tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.Ut, w.Ut, DV, NC * C, 64) &&
               tc::make_map_2d_bf16(&mp.P, w.P, C, NC * C, 64);
     mp.out = mp.u = mp.Sn = mp.Un = mp.q;  // unused ones keep a valid map
-    if (ok && bwd)
+    if (ok && keep)
         ok = tc::make_map_2d_bf16(&mp.Sn, w.Sn, DV, NC * DK, 128) && tc::make_map_2d_bf16(&mp.Un, w.Un, DV, NC * C, 64);
-    if (ok && !bwd && t.out) ok = tc::make_map_4d_bf16(&mp.out, t.out, DV, H, T, Bn, 64);
-    if (ok && !bwd && t.u) ok = tc::make_map_4d_bf16(&mp.u, t.u, DV, H, T, Bn, 64);
+    if (ok && out && t.out) ok = tc::make_map_4d_bf16(&mp.out, t.out, DV, H, T, Bn, 64);
+    if (ok && out && t.u) ok = tc::make_map_4d_bf16(&mp.u, t.u, DV, H, T, Bn, 64);
     if (!ok) return cudaErrorInvalidValue;
     Args a = {};
     a.gb = w.gb; a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
     a.S0 = t.S0;
-    if (!bwd) {
+    if (out) {
         a.has_out = t.out != nullptr; a.has_u = t.u != nullptr; a.ST = t.S_T;
     }
     const size_t smem = SMEM_BYTES + 1024;
     const dim3 grid(DV / DVB, g.H, g.B);
     cudaError_t e;
-    if (bwd) {
-        e = cudaFuncSetAttribute(k_chain_fwd<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        rec.mark(s);
-        k_chain_fwd<1><<<grid, NTHREADS, smem, s>>>(mp, a);
-    } else {
-        e = cudaFuncSetAttribute(k_chain_fwd<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        rec.mark(s);
-        k_chain_fwd<0><<<grid, NTHREADS, smem, s>>>(mp, a);
+    switch (mode) {
+        case 0:
+            e = cudaFuncSetAttribute(k_chain_fwd<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            rec.mark(s);
+            k_chain_fwd<0><<<grid, NTHREADS, smem, s>>>(mp, a);
+            break;
+        case 1:
+            e = cudaFuncSetAttribute(k_chain_fwd<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            rec.mark(s);
+            k_chain_fwd<1><<<grid, NTHREADS, smem, s>>>(mp, a);
+            break;
+        default:
+            e = cudaFuncSetAttribute(k_chain_fwd<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            rec.mark(s);
+            k_chain_fwd<2><<<grid, NTHREADS, smem, s>>>(mp, a);
+            break;
     }
     return cudaGetLastError();
 }
@@ -619,7 +646,7 @@ cudaError_t tc_chain_rev(const Geo &g, const Tensors &t, const TcWs &w, cudaStre
     const bool ok = tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) &&
                     tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64) &&
                     tc::make_map_4d_bf16(&mp.dout, t.dout, DV, H, T, Bn, 64) &&
-                    tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.dUp, w.dUp, DV, NC * C, 64) &&
+                    tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.P, w.P, C, NC * C, 64) &&
                     tc::make_map_2d_bf16(&mp.Un, w.Un, DV, NC * C, 64) && tc::make_map_2d_bf16(&mp.dUn, w.dUn, DV, NC * C, 64) &&
                     tc::make_map_2d_bf16(&mp.dSn, w.dSn, DV, NC * DK, 128) &&
                     (t.du ? tc::make_map_4d_bf16(&mp.du, t.du, DV, H, T, Bn, 64) : (mp.du = mp.dout, true));

@@ -603,22 +603,14 @@ bool tc_fwd_supported(const Geo &g, bool bf16) {
 }
 
 int tc_fwd_launches(const Geo &g, const char **names, int max_names) {
-    if (tc_split_supported(g, true)) {
-        if (names && max_names > 0) names[0] = "k_chunk_prep";
-        if (names && max_names > 1) names[1] = "k_chain_fwd";
-        return 2;
-    }
+    (void)g;
     if (names && max_names > 0) names[0] = "k_fwd_tc";
     return 1;
 }
 
 cudaError_t tc_fwd(const Geo &g, const Tensors &t, void *workspace, cudaStream_t s, Rec &rec) {
     using namespace tcf;
-    if (tc_split_supported(g, true)) {
-        const TcWs w = tc_ws_carve(g, false, workspace);
-        cudaError_t e = tc_chunk_prep(g, t, w, false, s, rec);
-        return e == cudaSuccess ? tc_chain_fwd(g, t, w, false, s, rec) : e;
-    }
+
     CUtensorMap mq, mk, mv, mg;
     const uint64_t Bn = g.B, T = g.T, H = g.H;
     bool ok = tc::make_map_4d_bf16(&mq, t.q, DK, H, T, Bn, 64) && tc::make_map_4d_bf16(&mk, t.k, DK, H, T, Bn, 64) &&

@@ -2,14 +2,15 @@
 //
 // Gated DeltaNet and DeltaNet at dv = 128 run the split path: a per-chunk kernel over all
 // chunks at once (tc_prep.cu), the serial state chains (tc_chain.cu) and, for the
-// backward, the per-chunk gradient kernel (tc_bwd.cu).  KDA and dv = 64 run the
-// single-kernel forward of tc_fwd.cu.
+// backward, the per-chunk gradient kernel (tc_bwd.cu); api.cu sequences them.  KDA and
+// dv = 64 run the single-kernel forward of tc_fwd.cu.
 #pragma once
 #include "dr_common.cuh"
 
 namespace dr {
 
 bool tc_fwd_supported(const Geo &g, bool bf16);
+// the single-kernel forward (KDA, and Gated DeltaNet / DeltaNet at dv = 64); no workspace
 cudaError_t tc_fwd(const Geo &g, const Tensors &t, void *workspace, cudaStream_t s, Rec &rec);
 // number of launches of tc_fwd and their names
 int tc_fwd_launches(const Geo &g, const char **names, int max_names);
@@ -19,31 +20,37 @@ int tc_fwd_launches(const Geo &g, const char **names, int max_names);
 bool tc_split_supported(const Geo &g, bool bf16);
 
 // Workspace of the split path, chunk-major (ci = (b H + h) N + n), every matrix row-major:
-// bf16 tiles that later kernels load with TMA, plus fp32 per-token factors.  The forward
-// uses gb, W, Ut and P; the backward all of it.
+// bf16 tiles that later kernels load with TMA, plus fp32 per-token factors.  Three parts:
+//   WS_FWD   the forward's chunk products (gb, W, Ut, P);
+//   WS_KEEP  what the backward needs from the forward besides them (Tn, KK, Sn, Un);
+//   WS_REV   what the reverse chain hands the gradient kernel (dSn, dUn, skt).
+// The forward's workspace is WS_FWD; the recomputing backward's all three; the saved
+// activations of delta_rule_fwd_save are WS_FWD | WS_KEEP, and the backward from them needs
+// WS_REV as workspace.
 struct TcWs {
     float *gb;           // [ci][2][C]    in-chunk cumulative log gate g, then beta
     __nv_bfloat16 *W;    // [ci][C][dk]   W  = T diag(beta e^g) k
     __nv_bfloat16 *Ut;   // [ci][C][dv]   U~ = T diag(beta) v
     __nv_bfloat16 *P;    // [ci][C][C]    P  = tril(e^{g_r - g_i} q_r . k_i)
-    // backward only
     __nv_bfloat16 *Tn;   // [ci][C][C]    T  = (I + A)^-1
     __nv_bfloat16 *KK;   // [ci][C][C]    k k^T (no gate factor)
-    __nv_bfloat16 *dUp;  // [ci][C][dv]   P^T dO
     __nv_bfloat16 *Sn;   // [ci][dk][dv]  state entering chunk n
-    __nv_bfloat16 *dSn;  // [ci][dk][dv]  dL/dS of the state leaving chunk n
     __nv_bfloat16 *Un;   // [ci][C][dv]   write values U = U~ - W S_n
+    __nv_bfloat16 *dSn;  // [ci][dk][dv]  dL/dS of the state leaving chunk n
     __nv_bfloat16 *dUn;  // [ci][C][dv]   dL/dU = du + P^T dO + Kbar dS_{n+1}
     float *skt;          // [ci][2][C]    per 64-column half of dv: U_r . (Kbar dS_{n+1})_r
 };
-size_t tc_ws_bytes(const Geo &g, bool bwd);
-TcWs tc_ws_carve(const Geo &g, bool bwd, void *base);
+enum { WS_FWD = 1, WS_KEEP = 2, WS_REV = 4 };
+// Bytes of the given parts, laid out one after another in the order FWD, KEEP, REV.
+size_t tc_ws_bytes(const Geo &g, int parts);
+// Sets the pointers of the given parts, carved from base in that order; leaves the others.
+void tc_ws_carve(const Geo &g, int parts, void *base, TcWs *w);
 
-// Per-chunk products (tc_prep.cu): g and beta, W, U~, P; with bwd also T, k k^T and P^T dO.
-cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool bwd, cudaStream_t s, Rec &rec);
-// Forward state chain (tc_chain.cu).  bwd = false: o, u, S_T; bwd = true (recompute for the
-// backward): S_n and U of every chunk into the workspace.
-cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, bool bwd, cudaStream_t s, Rec &rec);
+// Per-chunk products (tc_prep.cu): g and beta, W, U~, P; with keep also T and k k^T.
+cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool keep, cudaStream_t s, Rec &rec);
+// Forward state chain (tc_chain.cu).  mode 0: o, u, S_T; mode 1 (recompute for the
+// backward): S_n and U of every chunk; mode 2: both.
+cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, int mode, cudaStream_t s, Rec &rec);
 // Reverse state chain (tc_chain.cu): dS_{n+1} and dL/dU of every chunk (w.dSn, w.dUn), the
 // row sums w.skt, and dS0.
 cudaError_t tc_chain_rev(const Geo &g, const Tensors &t, const TcWs &w, cudaStream_t s, Rec &rec);

@@ -8,12 +8,12 @@
 //        A = beta_r e^{g_r - g_i} k_r.k_i (i < r),   P = e^{g_r - g_i} q_r.k_i (i <= r)
 //   T  = (I + A)^-1                            (the UT transform; tc_inverse.cuh)
 //   W  = T diag(beta e^g) k,   U~ = T diag(beta) v
-//   backward only:  dU' = P^T dO, and T, k k^T kept for the gradient kernel.
+//   backward (and a forward that saves for it): T and k k^T kept for the gradient kernel.
 //
 // Every chunk is independent, so the grid covers all chunks of all heads at once (two
 // CTAs per SM); the serial state chains (tc_chain.cu) then only carry the state.  The
-// products leave as bf16 tiles through TMA stores (W, U~, P, dU') or row stores (T, k k^T),
-// and g, beta as fp32.  The products with 64 rows use M = 128 MMAs whose rows 64..127 read
+// products leave as bf16 tiles through TMA stores (W, U~, P) or row stores (T, k k^T), and
+// g, beta as fp32.  The products with 64 rows use M = 128 MMAs whose rows 64..127 read
 // other (valid) shared memory and are discarded.
 #include "tc_host.cuh"
 #include "tc_inverse.cuh"
@@ -39,9 +39,8 @@ constexpr uint32_t OFF_KQ = 0;         // 32K [k_p0 | q_p0 | k_p1 | q_p1]; after
 constexpr uint32_t OFF_V = 32768;      // 16K v [i][j]
 constexpr uint32_t OFF_F = 49152;      // 32K fp32 A | T (inverse), then staging W [r][c] | U~ [r][j]
 constexpr uint32_t OFF_P = 81920;      //  8K P [r][i]
-constexpr uint32_t OFF_DO = 90112;     // 16K dO [r][j] -> staging dU' [r][j]   (backward)
-__host__ __device__ constexpr uint32_t misc_off(int bwd) { return bwd ? 106496u : 90112u; }
-__host__ __device__ constexpr uint32_t smem_bytes(int bwd) { return misc_off(bwd) + 2048; }
+constexpr uint32_t OFF_MISC = 90112;   //  2K
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 2048;
 // misc
 constexpr uint32_t M_BAR = 0;          // [0] loads, [1] MMA
 constexpr uint32_t M_TMEM = 64, M_ABORT = 68, M_BIG = 72;
@@ -49,27 +48,28 @@ constexpr uint32_t M_PF = 256;         // gate factors [6][64]
 enum { PF_GC = 0, PF_ROWP, PF_COLA, PF_BV, PF_BK, PF_NUM };
 static_assert(M_PF + PF_NUM * 256 <= 2048, "misc overflow");
 // TMEM columns
-constexpr uint32_t TM_G1 = 0, TM_XW = 0, TM_XU = 128, TM_DU = 128, TM_COLS = 256;
+constexpr uint32_t TM_G1 = 0, TM_XW = 0, TM_XU = 128, TM_COLS = 256;
 
 struct Maps {
-    CUtensorMap q, k, v, dout;  // [B, T, H, 128] bf16; box 64 channels x 64 tokens
-    CUtensorMap W, Ut, dUp;     // [chunks * 64][128] bf16; box 64 x 64 (stores)
-    CUtensorMap P;              // [chunks * 64][64] bf16; box 64 x 64 (store)
+    CUtensorMap q, k, v;  // [B, T, H, 128] bf16; box 64 channels x 64 tokens
+    CUtensorMap W, Ut;    // [chunks * 64][128] bf16; box 64 x 64 (stores)
+    CUtensorMap P;        // [chunks * 64][64] bf16; box 64 x 64 (store)
 };
 
 struct Args {
     const void *alpha, *beta;       // bf16 [B, T, H]
     float *gb;                      // [chunks][2][64]: g, beta
-    __nv_bfloat16 *KK, *Tn;         // [chunks][64][64] (backward)
+    __nv_bfloat16 *KK, *Tn;         // [chunks][64][64] (kept when KEEP)
     int B, T, H, N;
 };
 
-template <int VAR, int BWD>
+// KEEP: also store T and k k^T (for the backward)
+template <int VAR, int KEEP>
 __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constant__ Maps mp, Args a) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    unsigned char *misc = sm + misc_off(BWD);
+    unsigned char *misc = sm + OFF_MISC;
     uint64_t *bar = reinterpret_cast<uint64_t *>(misc + M_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + M_TMEM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + M_ABORT);
@@ -88,13 +88,12 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
         mbar_init(&bar[1], 1);
         *abort_flag = 0;
         fence_mbar_init();
-        mbar_arrive_tx(&bar[0], 49152u + (BWD ? 16384u : 0u));
+        mbar_arrive_tx(&bar[0], 49152u);
 #pragma unroll
         for (int p = 0; p < 2; ++p) {
             tma_load_4d(sm + OFF_KQ + p * 16384, &mp.k, 64 * p, h, t0, b, &bar[0]);
             tma_load_4d(sm + OFF_KQ + p * 16384 + 8192, &mp.q, 64 * p, h, t0, b, &bar[0]);
             tma_load_4d(sm + OFF_V + p * 8192, &mp.v, 64 * p, h, t0, b, &bar[0]);
-            if (BWD) tma_load_4d(sm + OFF_DO + p * 8192, &mp.dout, 64 * p, h, t0, b, &bar[0]);
         }
     }
     if (warp == 0) tmem_alloc(tmem_slot, TM_COLS);
@@ -159,8 +158,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
     float *Asc = reinterpret_cast<float *>(sm + OFF_F);
     float *Tf = Asc + 4096;
     float *ysc = reinterpret_cast<float *>(sm + OFF_KQ + 24576);  // q_p1, free after P1
-    const uint32_t skq = smem_u32(sm + OFF_KQ), sv = smem_u32(sm + OFF_V), sp = smem_u32(sm + OFF_P);
-    const uint32_t sdo = smem_u32(sm + OFF_DO);
+    const uint32_t skq = smem_u32(sm + OFF_KQ), sv = smem_u32(sm + OFF_V);
 
     bool ok = consensus(mbar_wait(&bar[0], 0, abort_flag));
     // ---------------- P1: [k ; q] . k^T ----------------
@@ -201,7 +199,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
             for (int i = 0; i < 64; ++i) f[i] = (i <= r) ? __expf(gr - gc[i]) : 0.f;
         }
         if (arow) {
-            if (BWD) st_row_global(a.KK, ((size_t)ci * C + r) * C, g1);
+            if (KEEP) st_row_global(a.KK, ((size_t)ci * C + r) * C, g1);
             const float br = pf[PF_BV * 64 + r];
 #pragma unroll
             for (int i4 = 0; i4 < 16; ++i4) {
@@ -226,33 +224,10 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
         fence_after_sync();
         tma_store_2d(&mp.P, sm + OFF_P, 0, ci * C);
         bulk_commit();
-        if (BWD) {  // dU' = P^T dO  (M = 128: rows 64..127 read dO and are discarded)
-            const uint32_t id = idesc_bf16(128, 128, 1, 1);
-#pragma unroll
-            for (int st = 0; st < 4; ++st)
-                mma_bf16(tbase + TM_DU, sdesc(sp + st * 2048, 8192, 1024), sdesc(sdo + st * 2048, 8192, 1024), id,
-                         st > 0);
-            mma_commit(&bar[1]);
-            mma_issued++;
-        }
     }
     // ---------------- T = (I + A)^-1 ----------------
     if (ok) unit_lower_inverse64(Asc, Tf, ysc, tid, sync);
-    if (BWD && ok) {
-        ok = consensus(wait_mma());
-        // dU' = P^T dO -> staging tile in place of dO (rows 0..63 of the accumulator)
-        if (ok && trow < 64) {
-            const int r = trow;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float v[64];
-                tmem_row64(tl + TM_DU + hh * 64, v);
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_DO, (uint32_t)hh * 8192 + swz(r, ch), v + ch * 8);
-            }
-        }
-    }
-    // ---------------- T diag(beta), T diag(beta e^g) tiles; T itself (backward) ----------------
+    // ---------------- T diag(beta), T diag(beta e^g) tiles; T itself (KEEP) ----------------
     if (ok) {
         const int i = tid & 63;
         const float *fac = pf + (tid < 64 ? PF_BV : PF_BK) * 64;
@@ -264,7 +239,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
             float w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
             for (int e = 0; e < 8; ++e) w[e] = (ch * 8 + e <= i) ? w[e] : 0.f;
-            if (BWD && tid < 64) st8_global(a.Tn, ((size_t)ci * C + i) * C + ch * 8, w);
+            if (KEEP && tid < 64) st8_global(a.Tn, ((size_t)ci * C + i) * C + ch * 8, w);
 #pragma unroll
             for (int e = 0; e < 8; ++e) w[e] *= fac[ch * 8 + e];
             st_chunk(dst, swz(i, ch), w);
@@ -276,11 +251,6 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
     // ---------------- W = [T diag(beta e^g) ; *] k,  U~ = [T diag(beta) ; *] v ----------------
     if (ok && tid == 0) {
         fence_after_sync();
-        if (BWD) {
-            tma_store_2d(&mp.dUp, sm + OFF_DO, 0, ci * C);
-            tma_store_2d(&mp.dUp, sm + OFF_DO + 8192, 64, ci * C);
-            bulk_commit();
-        }
         const uint32_t id = idesc_bf16(128, 128, 0, 1);
 #pragma unroll
         for (int st = 0; st < 4; ++st) {
@@ -328,39 +298,34 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
     if (warp == 0) tmem_dealloc(tbase, TM_COLS);
 }
 
-template <int VAR, int BWD>
+template <int VAR, int KEEP>
 static cudaError_t launch_prep(const Maps &mp, const Args &a, dim3 grid, cudaStream_t s, Rec &rec) {
-    const size_t smem = smem_bytes(BWD) + 1024;
+    const size_t smem = SMEM_BYTES + 1024;
     cudaError_t e =
-        cudaFuncSetAttribute(k_chunk_prep<VAR, BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(k_chunk_prep<VAR, KEEP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     rec.mark(s);
-    k_chunk_prep<VAR, BWD><<<grid, NTHREADS, smem, s>>>(mp, a);
+    k_chunk_prep<VAR, KEEP><<<grid, NTHREADS, smem, s>>>(mp, a);
     return cudaGetLastError();
 }
 
 }  // namespace tcp
 
-cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool bwd, cudaStream_t s, Rec &rec) {
+cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool keep, cudaStream_t s, Rec &rec) {
     using namespace tcp;
     Maps mp;
     const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;
     bool ok = tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) && tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64) &&
               tc::make_map_4d_bf16(&mp.v, t.v, DV, H, T, Bn, 64) && tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) &&
               tc::make_map_2d_bf16(&mp.Ut, w.Ut, DV, NC * C, 64) && tc::make_map_2d_bf16(&mp.P, w.P, C, NC * C, 64);
-    if (ok && bwd)
-        ok = tc::make_map_4d_bf16(&mp.dout, t.dout, DV, H, T, Bn, 64) &&
-             tc::make_map_2d_bf16(&mp.dUp, w.dUp, DV, NC * C, 64);
-    else
-        mp.dout = mp.v, mp.dUp = mp.W;
     if (!ok) return cudaErrorInvalidValue;
     Args a;
     a.alpha = t.alpha; a.beta = t.beta; a.gb = w.gb; a.KK = w.KK; a.Tn = w.Tn;
     a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
     const dim3 grid(g.N, g.H, g.B);
     if (g.variant == VAR_GATED)
-        return bwd ? launch_prep<VAR_GATED, 1>(mp, a, grid, s, rec) : launch_prep<VAR_GATED, 0>(mp, a, grid, s, rec);
-    return bwd ? launch_prep<VAR_DELTANET, 1>(mp, a, grid, s, rec) : launch_prep<VAR_DELTANET, 0>(mp, a, grid, s, rec);
+        return keep ? launch_prep<VAR_GATED, 1>(mp, a, grid, s, rec) : launch_prep<VAR_GATED, 0>(mp, a, grid, s, rec);
+    return keep ? launch_prep<VAR_DELTANET, 1>(mp, a, grid, s, rec) : launch_prep<VAR_DELTANET, 0>(mp, a, grid, s, rec);
 }
 
 }  // namespace dr

@@ -87,8 +87,9 @@ enum {
 };
 
 /*
- * Bytes of workspace that delta_rule_fwd (for_bwd = 0) or delta_rule_bwd
- * (for_bwd = 1) needs for these arguments.  Returns 0 when no workspace is
+ * Bytes of workspace that delta_rule_fwd (for_bwd = 0), delta_rule_bwd
+ * (for_bwd = 1), delta_rule_fwd_save (for_bwd = 2) or delta_rule_bwd_saved
+ * (for_bwd = 3) needs for these arguments.  Returns 0 when no workspace is
  * needed, and (size_t)-1 when the arguments are invalid.
  */
 size_t delta_rule_workspace_size(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype,
@@ -119,16 +120,53 @@ int delta_rule_bwd(const void *q, const void *k, const void *v, const void *alph
                    void *workspace, size_t ws_bytes, void *stream);
 
 /*
- * Measurement hooks.  delta_rule_launches() returns how many kernels one
- * delta_rule_fwd (for_bwd = 0) or delta_rule_bwd (for_bwd = 1) call with these
- * arguments launches, and stores a static name for launch i in names[i] for
- * i < max_names (names may be NULL); it returns a negative DR_ERR_* code for
- * invalid arguments.  The *_timed variants do exactly what delta_rule_fwd /
- * delta_rule_bwd do and in addition record the caller's cudaEvent_t events[i] (created handles) on
- * `stream` immediately before launch i and events[n] after the last launch
- * (n = delta_rule_launches(...)), so that each kernel's device time is the
- * elapsed time between consecutive events.  n_events must be 0 (record nothing)
- * or at least n + 1, else DR_ERR_ARG.
+ * Saved activations: a forward / backward pair for training.
+ *
+ * delta_rule_fwd_save computes exactly what delta_rule_fwd computes and, in
+ * addition, keeps in the caller's buffer `saved` what the backward would
+ * otherwise recompute: the per-chunk products of the chunked form (the
+ * in-chunk cumulative log gate and beta, W, U~, P, T = (I + A)^-1, k k^T) and
+ * the state entering every chunk with its write values, bf16 except the gate.
+ * delta_rule_bwd_saved computes exactly what delta_rule_bwd computes for the
+ * same forward arguments, reading `saved` instead of recomputing the forward.
+ * `saved` must come from delta_rule_fwd_save on the same inputs and arguments
+ * and must not change in between; the backward only reads it.
+ *   delta_rule_saved_size  bytes of `saved` for these arguments (the buffer is
+ *              device memory, 256-byte aligned).  It is 0 for configurations
+ *              without a saved form: the saved form exists for Gated DeltaNet
+ *              and DeltaNet with bf16 I/O, dk = dv = 128 and chunk 64.  For the
+ *              others delta_rule_fwd_save behaves as delta_rule_fwd and
+ *              delta_rule_bwd_saved as delta_rule_bwd, and `saved` may be NULL.
+ *              Returns (size_t)-1 for invalid arguments.
+ *   Workspace  delta_rule_workspace_size(..., for_bwd = 2) for the saving
+ *              forward and (..., for_bwd = 3) for the backward from `saved`.
+ *   Errors     DR_ERR_WORKSPACE when `saved` is needed and missing or smaller
+ *              than delta_rule_saved_size; DR_ERR_ALIGN when it is not 256-byte
+ *              aligned; otherwise as delta_rule_fwd / delta_rule_bwd.
+ */
+size_t delta_rule_saved_size(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype);
+int delta_rule_fwd_save(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                        const float *S0, void *out, void *u, float *S_T, int B, int T, int H, int dk, int dv,
+                        int variant, int chunk, int dtype, void *saved, size_t saved_bytes, void *workspace,
+                        size_t ws_bytes, void *stream);
+int delta_rule_bwd_saved(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                         const float *S0, const void *dout, const void *du, const float *dS_T, void *dq, void *dk_,
+                         void *dv_, void *dalpha, void *dbeta, float *dS0, int B, int T, int H, int dk, int dv,
+                         int variant, int chunk, int dtype, const void *saved, size_t saved_bytes, void *workspace,
+                         size_t ws_bytes, void *stream);
+
+/*
+ * Measurement hooks.  delta_rule_launches() returns how many kernels one call
+ * with these arguments launches -- delta_rule_fwd (for_bwd = 0), delta_rule_bwd
+ * (1), delta_rule_fwd_save (2), delta_rule_bwd_saved (3) -- and stores a static
+ * name for launch i in names[i] for i < max_names (names may be NULL); it
+ * returns a negative DR_ERR_* code for invalid arguments.  The *_timed variants
+ * do exactly what their plain entry points do and in addition record the
+ * caller's cudaEvent_t events[i] (created handles) on `stream` immediately
+ * before launch i and events[n] after the last launch (n = the launch count),
+ * so that each kernel's device time is the elapsed time between consecutive
+ * events.  n_events must be 0 (record nothing) or at least n + 1, else
+ * DR_ERR_ARG.
  */
 int delta_rule_launches(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype, int for_bwd,
                         const char **names, int max_names);
@@ -141,6 +179,16 @@ int delta_rule_bwd_timed(const void *q, const void *k, const void *v, const void
                          void *dv_, void *dalpha, void *dbeta, float *dS0, int B, int T, int H, int dk, int dv,
                          int variant, int chunk, int dtype, void *workspace, size_t ws_bytes, void *stream,
                          void *const *events, int n_events);
+int delta_rule_fwd_save_timed(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                              const float *S0, void *out, void *u, float *S_T, int B, int T, int H, int dk, int dv,
+                              int variant, int chunk, int dtype, void *saved, size_t saved_bytes, void *workspace,
+                              size_t ws_bytes, void *stream, void *const *events, int n_events);
+int delta_rule_bwd_saved_timed(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                               const float *S0, const void *dout, const void *du, const float *dS_T, void *dq,
+                               void *dk_, void *dv_, void *dalpha, void *dbeta, float *dS0, int B, int T, int H,
+                               int dk, int dv, int variant, int chunk, int dtype, const void *saved,
+                               size_t saved_bytes, void *workspace, size_t ws_bytes, void *stream,
+                               void *const *events, int n_events);
 
 /*
  * Forward without any device allocation (no counterpart in the method; it is a

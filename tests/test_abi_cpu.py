@@ -58,4 +58,16 @@ def test_no_compute_validation_paths(lib):
     args = [None] * 15 + [1, 10, 1, 128, 96, 1, 64, 1, None, 0, None]
     assert binding.bwd_raw(*args) == binding.DR_ERR_UNSUPPORTED
     assert binding.strerror(binding.DR_ERR_TIMEOUT) == "device wait timed out"
+    # the saved-activation pair: sizes of the saved buffer and of each call's workspace
+    sv = binding.saved_size(8, 4096, 8, 128, 128, 1, 64, 1)
+    assert sv > 0 and sv % 256 == 0
+    assert binding.workspace_size(8, 4096, 8, 128, 128, 1, 64, 1, 2) == 0
+    assert 0 < binding.workspace_size(8, 4096, 8, 128, 128, 1, 64, 1, 3) < binding.workspace_size(
+        8, 4096, 8, 128, 128, 1, 64, 1, 1)
+    assert binding.saved_size(4, 16384, 8, 128, 128, 2, 64, 1) == 0   # KDA: no saved form
+    assert binding.saved_size(1, 256, 2, 64, 64, 0, 64, 0) == 0       # fp32 I/O: no saved form
+    assert lib.delta_rule_workspace_size(1, 10, 1, 128, 128, 1, 64, 1, 4) == ctypes.c_size_t(-1).value
+    assert lib.delta_rule_saved_size(1, 10, 1, 96, 128, 1, 64, 1) == ctypes.c_size_t(-1).value
+    args = [None] * 9 + [1, 10, 1, 128, 128, 7, 64, 1, None, 0, None, 0, None]
+    assert binding.fwd_save_raw(*args) == binding.DR_ERR_ARG
     assert binding.strerror(12345) == "unknown error code"

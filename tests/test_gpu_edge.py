@@ -144,11 +144,13 @@ def test_split_sequence_tensor_core_path():
 
 
 def test_bf16_d128_uses_the_tensor_core_kernel():
-    split_fwd = ["k_chunk_prep", "k_chain_fwd"]
-    split_bwd = ["k_chunk_prep(bwd)", "k_chain_fwd(recompute)", "k_chain_rev", "k_bwd_chunk_tc"]
+    split = {0: ["k_chunk_prep", "k_chain_fwd"],
+             1: ["k_chunk_prep(keep)", "k_chain_fwd(recompute)", "k_chain_rev", "k_bwd_chunk_tc"],
+             2: ["k_chunk_prep(keep)", "k_chain_fwd(keep)"],
+             3: ["k_chain_rev", "k_bwd_chunk_tc"]}
     for variant in (0, 1):
-        assert binding.launches(8, 4096, 8, 128, 128, variant, 64, 1, 0) == split_fwd
-        assert binding.launches(8, 4096, 8, 128, 128, variant, 64, 1, 1) == split_bwd
+        for kind, names in split.items():
+            assert binding.launches(8, 4096, 8, 128, 128, variant, 64, 1, kind) == names
     assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 0) == ["k_fwd_tc"]
     assert binding.launches(2, 512, 4, 128, 64, 1, 64, 1, 0) == ["k_fwd_tc"]
     assert binding.launches(1, 256, 2, 64, 64, 0, 64, 0, 0) == ["k_prep", "k_scan", "k_out"]
