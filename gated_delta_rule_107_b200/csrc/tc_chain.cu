@@ -447,30 +447,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
                 bulk_commit();
             }
             pending = true;
-            // q rows scaled by e^{g_r} (for q^T diag(e^g) dO) while the MMAs run
-            for (int x = wc; x < 1024; x += 256) {  // 2 panels x 64 rows x 8 chunks of 16 B
-                float v[8];
-                ld_chunk(st + RS_Q, (uint32_t)x * 16, v);
-                const float f = cf[64 + ((x >> 3) & 63)];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] *= f;
-                st_chunk(st + RS_Q, (uint32_t)x * 16, v);
-            }
-            fence_proxy_async();
-            fence_before_sync();
-            if (wabort(true)) break;
-            // ---------------- D_b = (diag(e^g) q)^T dO  (first half of dL/dS_n) ----------------
-            if (wc == 0) {
-                fence_after_sync();
-                const uint32_t idb = idesc_bf16(128, 64, 1, 1);
-                const uint32_t sq = smem_u32(st + RS_Q), sdo = smem_u32(st + RS_DO);
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_bf16(tbase + TM_B, sdesc(sq + k * 2048, 8192, 1024), sdesc(sdo + k * 2048, 1024, 1024), idb,
-                             k > 0);
-            }
             if (!mma_done()) break;
-        // ---------------- dU = du + P^T dO + diag(e^{gC - g}) D_a;  U_r . (Kbar dS+)_r ----------------
+            // ---------------- dU = du + P^T dO + diag(e^{gC - g}) D_a;  U_r . (Kbar dS+)_r ----------------
             if (trow < 64) {
                 const int r = trow;
                 const float f = cf[r];
@@ -498,16 +476,30 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
                     st_chunk(sm + OFF_U, o, d);
                 }
                 skp[hf * 64 + r] = rs;
+            } else {
+                // lanes 64-127: q rows scaled by e^{g_r} (for q^T diag(e^g) dO)
+                for (int x = (cl.q4 - 2) * 32 + lane + hf * 64; x < 1024; x += 128) {  // 128 threads
+                    float v[8];
+                    ld_chunk(st + RS_Q, (uint32_t)x * 16, v);
+                    const float f = cf[64 + ((x >> 3) & 63)];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[e] *= f;
+                    st_chunk(st + RS_Q, (uint32_t)x * 16, v);
+                }
             }
             fence_proxy_async();
             fence_before_sync();
             if (wabort(true)) break;
             if (trow < 64 && hf == 0) a.skt[ci * 2 * C + half * C + trow] = skp[trow] + skp[64 + trow];
-            // ---------------- D_b -= W^T dU;  dU out ----------------
+            // ---------------- D_b = (diag(e^g) q)^T dO - W^T dU;  dU out ----------------
             if (wc == 0) {
                 fence_after_sync();
-                const uint32_t id = idesc_bf16(128, 64, 1, 1, 1);
-                const uint32_t sw = smem_u32(st + RS_W);
+                const uint32_t idb = idesc_bf16(128, 64, 1, 1), id = idesc_bf16(128, 64, 1, 1, 1);
+                const uint32_t sq = smem_u32(st + RS_Q), sdo = smem_u32(st + RS_DO), sw = smem_u32(st + RS_W);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16(tbase + TM_B, sdesc(sq + k * 2048, 8192, 1024), sdesc(sdo + k * 2048, 1024, 1024), idb,
+                             k > 0);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     mma_bf16(tbase + TM_B, sdesc(sw + k * 2048, 8192, 1024), sdesc(sU + k * 2048, 1024, 1024), id, 1);
