@@ -75,16 +75,28 @@ __device__ __forceinline__ void st16(float *Z, int zr, int zc, float (*z)[4], fl
 template <typename Sync>
 __device__ __forceinline__ void unit_lower_inverse64(const float *A, float *T, float *Ysc, int wt, Sync sync) {
     const int warp = wt >> 5, lane = wt & 31;
-    // diagonal blocks: lane j (< 16) of warp R owns column j of T_RR
+    // diagonal blocks: lane j (< 16) of warp R owns column j of T_RR; the strictly lower part
+    // of L_RR is read into registers first (float4 groups stay whole under sw64)
     if (lane < 16) {
         const int R = warp, j = lane, o = 16 * R;
+        float a[16][16];
+#pragma unroll
+        for (int r = 1; r < 16; ++r) {
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                if (4 * c4 < r) {
+                    const float4 v = *reinterpret_cast<const float4 *>(&A[sw64(o + r, o + 4 * c4)]);
+                    a[r][4 * c4] = v.x; a[r][4 * c4 + 1] = v.y; a[r][4 * c4 + 2] = v.z; a[r][4 * c4 + 3] = v.w;
+                }
+            }
+        }
         float t[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) t[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
 #pragma unroll
-            for (int r = i + 1; r < 16; ++r) t[r] -= A[sw64(o + r, o + i)] * t[i];
+            for (int r = i + 1; r < 16; ++r) t[r] -= a[r][i] * t[i];
         }
 #pragma unroll
         for (int r = 0; r < 16; ++r) T[sw64(o + r, o + j)] = t[r];

@@ -12,8 +12,8 @@
 //
 // Every chunk is independent, so the grid covers all chunks of all heads at once (two
 // CTAs per SM); the serial state chains (tc_chain.cu) then only carry the state.  The
-// products leave as bf16 tiles through TMA stores (W, U~, P) or row stores (T, k k^T), and
-// g, beta as fp32.  The products with 64 rows use M = 128 MMAs whose rows 64..127 read
+// products leave as bf16 tiles through TMA stores (W, U~, P, and T, k k^T from tiles freed by
+// then), and g, beta as fp32.  The products with 64 rows use M = 128 MMAs whose rows 64..127 read
 // other (valid) shared memory and are discarded.
 #include "tc_host.cuh"
 #include "tc_inverse.cuh"
@@ -27,15 +27,13 @@ namespace tcp {
 using namespace dr::tc;
 using dr::tcf::ld_chunk;
 using dr::tcf::st_chunk;
-using dr::tcf::st8_global;
-using dr::tcf::st_row_global;
 using dr::tcf::tmem_row64;
 
 constexpr int C = 64, DK = 128, DV = 128;
 constexpr int NTHREADS = 128;
 // shared memory (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_KQ = 0;         // 32K [k_p0 | q_p0 | k_p1 | q_p1]; after P1: q_p0 -> T diag(beta),
-                                       //     q_p1 -> inverse scratch, then T diag(beta e^g)
+constexpr uint32_t OFF_KQ = 0;         // 32K [k_p0 | q_p0 | k_p1 | q_p1]; after P1: q_p0 -> k k^T (KEEP),
+                                       //     then T diag(beta); q_p1 -> inverse scratch, then T diag(beta e^g)
 constexpr uint32_t OFF_V = 32768;      // 16K v [i][j]
 constexpr uint32_t OFF_F = 49152;      // 32K fp32 A | T (inverse), then staging W [r][c] | U~ [r][j]
 constexpr uint32_t OFF_P = 81920;      //  8K P [r][i]
@@ -54,12 +52,12 @@ struct Maps {
     CUtensorMap q, k, v;  // [B, T, H, 128] bf16; box 64 channels x 64 tokens
     CUtensorMap W, Ut;    // [chunks * 64][128] bf16; box 64 x 64 (stores)
     CUtensorMap P;        // [chunks * 64][64] bf16; box 64 x 64 (store)
+    CUtensorMap KK, Tn;   // [chunks * 64][64] bf16; box 64 x 64 (stores, when KEEP)
 };
 
 struct Args {
     const void *alpha, *beta;       // bf16 [B, T, H]
     float *gb;                      // [chunks][2][64]: g, beta
-    __nv_bfloat16 *KK, *Tn;         // [chunks][64][64] (kept when KEEP)
     int B, T, H, N;
 };
 
@@ -157,7 +155,6 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
     };
     float *Asc = reinterpret_cast<float *>(sm + OFF_F);
     float *Tf = Asc + 4096;
-    float *ysc = reinterpret_cast<float *>(sm + OFF_KQ + 24576);  // q_p1, free after P1
     const uint32_t skq = smem_u32(sm + OFF_KQ), sv = smem_u32(sm + OFF_V);
 
     bool ok = consensus(mbar_wait(&bar[0], 0, abort_flag));
@@ -199,7 +196,11 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
             for (int i = 0; i < 64; ++i) f[i] = (i <= r) ? __expf(gr - gc[i]) : 0.f;
         }
         if (arow) {
-            if (KEEP) st_row_global(a.KK, ((size_t)ci * C + r) * C, g1);
+            // k k^T row (KEEP) into the q_p0 tile, free since P1 completed
+            if (KEEP) {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_KQ + 8192, swz(r, ch), g1 + ch * 8);
+            }
             const float br = pf[PF_BV * 64 + r];
 #pragma unroll
             for (int i4 = 0; i4 < 16; ++i4) {
@@ -223,11 +224,17 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
     if (ok && tid == 0) {
         fence_after_sync();
         tma_store_2d(&mp.P, sm + OFF_P, 0, ci * C);
+        if (KEEP) tma_store_2d(&mp.KK, sm + OFF_KQ + 8192, 0, ci * C);
         bulk_commit();
     }
     // ---------------- T = (I + A)^-1 ----------------
+    float *ysc = reinterpret_cast<float *>(sm + OFF_KQ + 24576);  // q_p1, free after P1
     if (ok) unit_lower_inverse64(Asc, Tf, ysc, tid, sync);
     // ---------------- T diag(beta), T diag(beta e^g) tiles; T itself (KEEP) ----------------
+    if (KEEP) {  // the P and k k^T stores have read the tiles that T and T diag(beta) take over
+        if (tid == 0) bulk_wait_read_all();
+        sync();
+    }
     if (ok) {
         const int i = tid & 63;
         const float *fac = pf + (tid < 64 ? PF_BV : PF_BK) * 64;
@@ -239,7 +246,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
             float w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
             for (int e = 0; e < 8; ++e) w[e] = (ch * 8 + e <= i) ? w[e] : 0.f;
-            if (KEEP && tid < 64) st8_global(a.Tn, ((size_t)ci * C + i) * C + ch * 8, w);
+            if (KEEP && tid < 64) st_chunk(sm + OFF_P, swz(i, ch), w);
 #pragma unroll
             for (int e = 0; e < 8; ++e) w[e] *= fac[ch * 8 + e];
             st_chunk(dst, swz(i, ch), w);
@@ -251,6 +258,10 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
     // ---------------- W = [T diag(beta e^g) ; *] k,  U~ = [T diag(beta) ; *] v ----------------
     if (ok && tid == 0) {
         fence_after_sync();
+        if (KEEP) {
+            tma_store_2d(&mp.Tn, sm + OFF_P, 0, ci * C);
+            bulk_commit();
+        }
         const uint32_t id = idesc_bf16(128, 128, 0, 1);
 #pragma unroll
         for (int st = 0; st < 4; ++st) {
@@ -318,9 +329,11 @@ cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool ke
     bool ok = tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) && tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64) &&
               tc::make_map_4d_bf16(&mp.v, t.v, DV, H, T, Bn, 64) && tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) &&
               tc::make_map_2d_bf16(&mp.Ut, w.Ut, DV, NC * C, 64) && tc::make_map_2d_bf16(&mp.P, w.P, C, NC * C, 64);
+    if (ok && keep)
+        ok = tc::make_map_2d_bf16(&mp.KK, w.KK, C, NC * C, 64) && tc::make_map_2d_bf16(&mp.Tn, w.Tn, C, NC * C, 64);
     if (!ok) return cudaErrorInvalidValue;
     Args a;
-    a.alpha = t.alpha; a.beta = t.beta; a.gb = w.gb; a.KK = w.KK; a.Tn = w.Tn;
+    a.alpha = t.alpha; a.beta = t.beta; a.gb = w.gb;
     a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
     const dim3 grid(g.N, g.H, g.B);
     if (g.variant == VAR_GATED)
