@@ -35,6 +35,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "delta-rule fwd+bwd tokens/s at B=8,T=4096,H=8,d=128 bf16; % of roofline"
 WORKLOAD_ID = 2
+DECODE_B = 64  # sequences in the decoding-step measurement
 FLUSH_BYTES = 256 << 20
 
 
@@ -336,6 +337,32 @@ def run_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         r_ms = float(t.item())
 
+    # ---- one decoding step (delta_rule_decode), reported beside: DECODE_B sequences, one
+    # token each, the fp32 state updated in place; L2 flushed before every call ----
+    dx = make_inputs(var, "bf16", DECODE_B, 1, H, dk, dv, seed=w.seed + 7, s0_std=0.05, device=dev)
+    dS = dx["S0"]
+    dev_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for _ in range(3):
+        binding.delta_rule_decode(dx["q"], dx["k"], dx["v"], dx["loga"], dx["beta"], dS, variant=var, inplace=True)
+    dec_ms = []
+    for _ in range(args.steps):
+        flush.fill_(1)
+        dev_ev[0].record()
+        binding.delta_rule_decode(dx["q"], dx["k"], dx["v"], dx["loga"], dx["beta"], dS, variant=var, inplace=True)
+        dev_ev[1].record()
+        torch.cuda.synchronize()
+        dec_ms.append(dev_ev[0].elapsed_time(dev_ev[1]))
+    if binding.sync_status() != binding.DR_OK:
+        raise RuntimeError("device error word set during the decode leg")
+    d_ms = statistics.mean(dec_ms)
+    g_w = {binding.DR_DELTANET: 0, binding.DR_GATED: 1, binding.DR_KDA: dk}[var]
+    d_bytes = DECODE_B * H * (2 * 4 * dk * dv + elem * (2 * dk + 3 * dv + g_w + 1))
+    decode = {"workload": f"{vname} decode bf16 B{DECODE_B} T1 H{H} d{dk}, fp32 state updated in place",
+              "ms_per_step": d_ms, "tokens_per_s": DECODE_B / (d_ms / 1e3), "alg_bytes": d_bytes,
+              "roofline": {"bound": "hbm", "achieved": d_bytes / (d_ms / 1e3) / 1e9, "unit": "GB/s",
+                           "frac": d_bytes / (d_ms / 1e3) / 1e9 / load_peaks()["hbm_gbs"]},
+              "kernel": "k_decode"}
+
     # ---- end to end through the public API with host buffers ----
     host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in x.items()}
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
@@ -439,6 +466,7 @@ def run_ours(args):
                       "ms_per_step": r_ms, "value": tokens / (r_ms / 1e3),
                       "kernels": {n: round(statistics.mean(v), 4) for n, v in r_kern.items()}},
         "saved_bytes": sv_bytes,
+        "decode": decode,
         "gpu_launches": args.steps * (len(fwd_names) + len(bwd_names)),
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

@@ -12,8 +12,9 @@ High level: ``delta_rule_fwd`` / ``delta_rule_bwd`` take torch CUDA tensors,
 allocate outputs and the workspace with torch, and call the C ABI on the
 current stream; ``delta_rule_fwd_save`` / ``delta_rule_bwd_saved`` are the
 training pair (the forward keeps what the backward would recompute in a saved
-buffer).  ``delta_rule_fwd_host`` is the forward for host tensors (copies in,
-computes, copies out).
+buffer); ``delta_rule_decode`` is the recurrent form for the few tokens of a
+decoding step (state in, state out, optionally in place).  ``delta_rule_fwd_host``
+is the forward for host tensors (copies in, computes, copies out).
 
 The ``for_bwd`` argument of ``workspace_size`` and ``launches`` names the call:
 0 forward, 1 backward, 2 saving forward, 3 backward from saved activations.
@@ -35,7 +36,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdeltarul
 EXPORTS = ("delta_rule_workspace_size", "delta_rule_fwd", "delta_rule_bwd", "delta_rule_strerror",
            "delta_rule_sync_status", "delta_rule_launches", "delta_rule_fwd_timed", "delta_rule_bwd_timed",
            "delta_rule_fwd_noalloc", "delta_rule_saved_size", "delta_rule_fwd_save", "delta_rule_bwd_saved",
-           "delta_rule_fwd_save_timed", "delta_rule_bwd_saved_timed")
+           "delta_rule_fwd_save_timed", "delta_rule_bwd_saved_timed", "delta_rule_decode")
 
 _lib = None
 
@@ -81,6 +82,8 @@ def load(path: str | None = None):
     lib.delta_rule_fwd_save.restype = i
     lib.delta_rule_bwd_saved.argtypes = [vp] * 15 + [i] * 8 + [vp, sz, vp, sz, vp]
     lib.delta_rule_bwd_saved.restype = i
+    lib.delta_rule_decode.argtypes = [vp] * 9 + [i] * 7 + [vp]
+    lib.delta_rule_decode.restype = i
     lib.delta_rule_fwd_save_timed.argtypes = [vp] * 9 + [i] * 8 + [vp, sz, vp, sz, vp, ctypes.POINTER(vp), i]
     lib.delta_rule_fwd_save_timed.restype = i
     lib.delta_rule_bwd_saved_timed.argtypes = [vp] * 15 + [i] * 8 + [vp, sz, vp, sz, vp, ctypes.POINTER(vp), i]
@@ -217,6 +220,37 @@ def delta_rule_fwd(q, k, v, alpha, beta, S0=None, variant="gdn", chunk=64, want_
                  B, T, H, dk, dv, var, chunk, dt, _p(workspace), need, stream)
     _check(rc, "delta_rule_fwd")
     return out, u, S_T
+
+
+def decode_raw(*args) -> int:
+    return load().delta_rule_decode(*args)
+
+
+def delta_rule_decode(q, k, v, alpha, beta, S=None, variant="gdn", want_u=True, inplace=False, out=None, u=None,
+                      S_out=None):
+    """Recurrent step(s) for decoding on CUDA tensors.  Returns (o, u or None, S_out).
+
+    Shapes as delta_rule_fwd; S: fp32 [B,H,dk,dv] or None (zero state).  With inplace=True the
+    state is updated in S itself (S_out is S)."""
+    var = _variant(variant)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = DTYPES[q.dtype]
+    dev = q.device
+    out = torch.empty((B, T, H, dv), dtype=q.dtype, device=dev) if out is None else out
+    if want_u and u is None:
+        u = torch.empty((B, T, H, dv), dtype=q.dtype, device=dev)
+    if inplace:
+        if S is None:
+            raise ValueError("inplace decoding needs a state tensor")
+        S_out = S
+    elif S_out is None:
+        S_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = decode_raw(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S), _p(S_out), _p(out), _p(u),
+                    B, T, H, dk, dv, var, dt, stream)
+    _check(rc, "delta_rule_decode")
+    return out, u, S_out
 
 
 def delta_rule_bwd(q, k, v, alpha, beta, S0, dout, du=None, dS_T=None, variant="gdn", chunk=64,

@@ -2,10 +2,11 @@
 //
 // Argument validation, workspace planning and dispatch.  No compute happens on
 // the host: every step of the path runs in the kernels of simt_path.cu and
-// tc_fwd.cu.  Validation failures return before anything is enqueued.
+// the tensor-core files and decode.cu.  Validation failures return before anything is enqueued.
 #include <limits.h>
 
 #include "../../include/delta_rule.h"
+#include "decode.cuh"
 #include "dr_common.cuh"
 #include "simt_path.cuh"
 #include "tc_path.cuh"
@@ -338,6 +339,28 @@ extern "C" int delta_rule_launches(int B, int T, int H, int dk, int dv, int vari
     if (rc != DR_OK) return rc;
     if (for_bwd < 0 || for_bwd > 3) return DR_ERR_ARG;
     return launch_plan(g, dtype, for_bwd, names, max_names);
+}
+
+extern "C" int delta_rule_decode(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                                 const float *S_in, float *S_out, void *out, void *u, int B, int T, int H, int dk,
+                                 int dv, int variant, int dtype, void *stream) {
+    Geo g;
+    int rc = check_shape(B, T, H, dk, dv, variant, 64, dtype, &g);
+    if (rc != DR_OK) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    const bool empty = (size_t)B * H == 0;
+    if (empty) return DR_OK;
+    if (T == 0) return S_out == S_in ? DR_OK : copy_state(S_out, S_in, g, s);
+    if (!q || !k || !v || !beta || !out) return DR_ERR_ARG;
+    if (variant != DR_DELTANET && !alpha) return DR_ERR_ARG;
+    const void *ptrs[] = {q, k, v, variant == DR_KDA ? alpha : nullptr, S_in, S_out, out, u};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return DR_ERR_ALIGN;
+    if (!aligned_elem(beta, dtype) || (variant == DR_GATED && !aligned_elem(alpha, dtype))) return DR_ERR_ALIGN;
+    Tensors t = {};
+    t.q = q; t.k = k; t.v = v; t.alpha = alpha; t.beta = beta; t.S0 = S_in; t.out = out; t.u = u; t.S_T = S_out;
+    Rec rec;
+    return launch_status(decode_fwd(g, t, dtype == DR_BF16, s, rec));
 }
 
 extern "C" const char *delta_rule_strerror(int code) {

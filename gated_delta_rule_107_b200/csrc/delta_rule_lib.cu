@@ -5,5 +5,6 @@
 #include "tc_prep.cu"
 #include "tc_chain.cu"
 #include "tc_bwd.cu"
+#include "decode.cu"
 #include "api.cu"
 #include "noalloc.cu"

@@ -216,6 +216,21 @@ int delta_rule_fwd_noalloc(const void *q, const void *k, const void *v, const vo
                            const float *S0, void *out, void *u, float *S_T, int B, int T, int H, int dk, int dv,
                            int variant, int chunk, int dtype, void *stream);
 
+/*
+ * Recurrent form for decoding.  Steps the recurrence above token by token from
+ * the state S_in (NULL = zero) through the T tokens given and writes out and u
+ * exactly as delta_rule_fwd does (u may be NULL), and the state after the last
+ * token to S_out (NULL = not written).  S_out may be the same buffer as S_in
+ * (the state is updated in place); partial overlap is not allowed.  It is meant
+ * for the few tokens of a decoding step: each (b, h) keeps its state in
+ * registers and reads and writes it once, with no chunking, workspace or saved
+ * form.  For T == 0 it copies S_in (or zeros) to S_out.  Arguments, layouts,
+ * alignment and errors follow the conventions above (no chunk argument).
+ */
+int delta_rule_decode(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
+                      const float *S_in, float *S_out, void *out, void *u, int B, int T, int H, int dk, int dv,
+                      int variant, int dtype, void *stream);
+
 /* Static text for a DR_* code ("ok", "invalid argument", ...). */
 const char *delta_rule_strerror(int code);
 
