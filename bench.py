@@ -363,6 +363,44 @@ def run_ours(args):
                            "frac": d_bytes / (d_ms / 1e3) / 1e9 / load_peaks()["hbm_gbs"]},
               "kernel": "k_decode"}
 
+    # ---- the single-pass operations around the core at this shape, reported beside ----
+    def ev_time(fn, reps=5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fn()
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.mean(ts)
+
+    gw_ = 0 if var == binding.DR_DELTANET else (dk if var == binding.DR_KDA else 1)
+    rows = B * T * H
+    raw_a = None if var == binding.DR_DELTANET else torch.randn_like(x["loga"].float()).to(x["q"].dtype) - 3.0
+    pre_out = binding.delta_rule_preop(x["q"], x["k"], x["beta"], raw_a, variant=var)
+    pre_ms = ev_time(lambda: binding.delta_rule_preop(x["q"], x["k"], x["beta"], raw_a, variant=var))
+    pre_b_ms = ev_time(lambda: binding.delta_rule_preop_bwd(x["q"], x["k"], x["beta"], raw_a, pre_out[0], pre_out[1],
+                                                            pre_out[2], pre_out[3], variant=var))
+    post_w = torch.ones(dv, device=dev)
+    post_ms = ev_time(lambda: binding.delta_rule_postop(o, u, post_w))
+    post_b_ms = ev_time(lambda: binding.delta_rule_postop_bwd(o, u, post_w, x["dO"]))
+    if binding.sync_status() != binding.DR_OK:
+        raise RuntimeError("device error word set during the pre/post leg")
+    pre_unit = rows * elem * (2 * dk + 1 + gw_)  # q, k, beta, gate of every row once
+    post_bytes = rows * elem * 3 * dv
+    hbm = load_peaks()["hbm_gbs"]
+
+    def gbs(nbytes, t_ms):
+        return {"ms": t_ms, "alg_bytes": nbytes, "achieved_gbs": nbytes / (t_ms / 1e3) / 1e9,
+                "frac": nbytes / (t_ms / 1e3) / 1e9 / hbm}
+
+    prepost = {"shape": f"B{B} T{T} H{H} d{dk} bf16", "preop": gbs(2 * pre_unit, pre_ms),
+               "preop_bwd": gbs(3 * pre_unit, pre_b_ms), "postop": gbs(post_bytes, post_ms),
+               "postop_bwd": gbs(rows * elem * 5 * dv, post_b_ms)}
+
     # ---- end to end through the public API with host buffers ----
     host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in x.items()}
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
@@ -467,6 +505,7 @@ def run_ours(args):
                       "kernels": {n: round(statistics.mean(v), 4) for n, v in r_kern.items()}},
         "saved_bytes": sv_bytes,
         "decode": decode,
+        "prepost": prepost,
         "gpu_launches": args.steps * (len(fwd_names) + len(bwd_names)),
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

@@ -13,7 +13,10 @@ allocate outputs and the workspace with torch, and call the C ABI on the
 current stream; ``delta_rule_fwd_save`` / ``delta_rule_bwd_saved`` are the
 training pair (the forward keeps what the backward would recompute in a saved
 buffer); ``delta_rule_decode`` is the recurrent form for the few tokens of a
-decoding step (state in, state out, optionally in place).  ``delta_rule_fwd_host``
+decoding step (state in, state out, optionally in place); ``delta_rule_preop`` /
+``delta_rule_postop`` and their ``_bwd`` are the single-pass operations just
+before and after the core (L2-normalised q, k, logistic gates; sigmoid-gated
+RMSNorm of the output).  ``delta_rule_fwd_host``
 is the forward for host tensors (copies in, computes, copies out).
 
 The ``for_bwd`` argument of ``workspace_size`` and ``launches`` names the call:
@@ -36,7 +39,9 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdeltarul
 EXPORTS = ("delta_rule_workspace_size", "delta_rule_fwd", "delta_rule_bwd", "delta_rule_strerror",
            "delta_rule_sync_status", "delta_rule_launches", "delta_rule_fwd_timed", "delta_rule_bwd_timed",
            "delta_rule_fwd_noalloc", "delta_rule_saved_size", "delta_rule_fwd_save", "delta_rule_bwd_saved",
-           "delta_rule_fwd_save_timed", "delta_rule_bwd_saved_timed", "delta_rule_decode")
+           "delta_rule_fwd_save_timed", "delta_rule_bwd_saved_timed", "delta_rule_decode",
+           "delta_rule_preop", "delta_rule_preop_bwd", "delta_rule_postop_workspace_size", "delta_rule_postop",
+           "delta_rule_postop_bwd")
 
 _lib = None
 
@@ -82,6 +87,16 @@ def load(path: str | None = None):
     lib.delta_rule_fwd_save.restype = i
     lib.delta_rule_bwd_saved.argtypes = [vp] * 15 + [i] * 8 + [vp, sz, vp, sz, vp]
     lib.delta_rule_bwd_saved.restype = i
+    lib.delta_rule_preop.argtypes = [vp] * 8 + [i] * 6 + [vp]
+    lib.delta_rule_preop.restype = i
+    lib.delta_rule_preop_bwd.argtypes = [vp] * 12 + [i] * 6 + [vp]
+    lib.delta_rule_preop_bwd.restype = i
+    lib.delta_rule_postop_workspace_size.argtypes = [i]
+    lib.delta_rule_postop_workspace_size.restype = sz
+    lib.delta_rule_postop.argtypes = [vp] * 4 + [i] * 5 + [vp]
+    lib.delta_rule_postop.restype = i
+    lib.delta_rule_postop_bwd.argtypes = [vp] * 7 + [i] * 5 + [vp, sz, vp]
+    lib.delta_rule_postop_bwd.restype = i
     lib.delta_rule_decode.argtypes = [vp] * 9 + [i] * 7 + [vp]
     lib.delta_rule_decode.restype = i
     lib.delta_rule_fwd_save_timed.argtypes = [vp] * 9 + [i] * 8 + [vp, sz, vp, sz, vp, ctypes.POINTER(vp), i]
@@ -251,6 +266,70 @@ def delta_rule_decode(q, k, v, alpha, beta, S=None, variant="gdn", want_u=True, 
                     B, T, H, dk, dv, var, dt, stream)
     _check(rc, "delta_rule_decode")
     return out, u, S_out
+
+
+def preop_raw(*args) -> int:
+    return load().delta_rule_preop(*args)
+
+
+def preop_bwd_raw(*args) -> int:
+    return load().delta_rule_preop_bwd(*args)
+
+
+def postop_raw(*args) -> int:
+    return load().delta_rule_postop(*args)
+
+
+def postop_bwd_raw(*args) -> int:
+    return load().delta_rule_postop_bwd(*args)
+
+
+def delta_rule_preop(q_raw, k_raw, beta_raw, gate_raw=None, variant="gdn"):
+    """The core's inputs from raw projections: (q, k, beta, loga); loga is None for deltanet."""
+    var = _variant(variant)
+    B, T, H, dk = q_raw.shape
+    q, k, beta = torch.empty_like(q_raw), torch.empty_like(k_raw), torch.empty_like(beta_raw)
+    loga = torch.empty_like(gate_raw) if (var != DR_DELTANET and gate_raw is not None) else None
+    rc = preop_raw(_p(q_raw), _p(k_raw), _p(beta_raw), _p(gate_raw), _p(q), _p(k), _p(beta), _p(loga), B, T, H, dk,
+                   var, DTYPES[q_raw.dtype], torch.cuda.current_stream(q_raw.device).cuda_stream)
+    _check(rc, "delta_rule_preop")
+    return q, k, beta, loga
+
+
+def delta_rule_preop_bwd(q_raw, k_raw, beta_raw, gate_raw, dq, dk, dbeta, dloga=None, variant="gdn"):
+    """Gradients with respect to (q_raw, k_raw, beta_raw, gate_raw); the last is None for deltanet."""
+    var = _variant(variant)
+    B, T, H, dk_ = q_raw.shape
+    gq, gk, gb = torch.empty_like(q_raw), torch.empty_like(k_raw), torch.empty_like(beta_raw)
+    ga = torch.empty_like(gate_raw) if (var != DR_DELTANET and gate_raw is not None) else None
+    rc = preop_bwd_raw(_p(q_raw), _p(k_raw), _p(beta_raw), _p(gate_raw), _p(dq), _p(dk), _p(dbeta), _p(dloga),
+                       _p(gq), _p(gk), _p(gb), _p(ga), B, T, H, dk_, var, DTYPES[q_raw.dtype],
+                       torch.cuda.current_stream(q_raw.device).cuda_stream)
+    _check(rc, "delta_rule_preop_bwd")
+    return gq, gk, gb, ga
+
+
+def delta_rule_postop(o, gate, weight=None):
+    """y = rmsnorm(o) * weight * sigmoid(gate) per (token, head) row."""
+    B, T, H, dv = o.shape
+    y = torch.empty_like(o)
+    rc = postop_raw(_p(o), _p(gate), _p(weight), _p(y), B, T, H, dv, DTYPES[o.dtype],
+                    torch.cuda.current_stream(o.device).cuda_stream)
+    _check(rc, "delta_rule_postop")
+    return y
+
+
+def delta_rule_postop_bwd(o, gate, weight, dy, want_dweight=True):
+    """Returns (do, dgate, dweight or None)."""
+    B, T, H, dv = o.shape
+    go, gg = torch.empty_like(o), torch.empty_like(gate)
+    gw = torch.empty(dv, dtype=torch.float32, device=o.device) if want_dweight else None
+    need = load().delta_rule_postop_workspace_size(dv)
+    ws = _workspace(need, o.device)
+    rc = postop_bwd_raw(_p(o), _p(gate), _p(weight), _p(dy), _p(go), _p(gg), _p(gw), B, T, H, dv, DTYPES[o.dtype],
+                        _p(ws), need, torch.cuda.current_stream(o.device).cuda_stream)
+    _check(rc, "delta_rule_postop_bwd")
+    return go, gg, gw
 
 
 def delta_rule_bwd(q, k, v, alpha, beta, S0, dout, du=None, dS_T=None, variant="gdn", chunk=64,

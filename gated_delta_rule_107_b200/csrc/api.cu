@@ -7,6 +7,7 @@
 
 #include "../../include/delta_rule.h"
 #include "decode.cuh"
+#include "prepost.cuh"
 #include "dr_common.cuh"
 #include "simt_path.cuh"
 #include "tc_path.cuh"
@@ -361,6 +362,99 @@ extern "C" int delta_rule_decode(const void *q, const void *k, const void *v, co
     t.q = q; t.k = k; t.v = v; t.alpha = alpha; t.beta = beta; t.S0 = S_in; t.out = out; t.u = u; t.S_T = S_out;
     Rec rec;
     return launch_status(decode_fwd(g, t, dtype == DR_BF16, s, rec));
+}
+
+// Shape check shared by the pre/post entry points: rows of d channels.
+static int check_rows(int B, int T, int H, int d, int dtype, size_t *rows) {
+    if (B < 0 || T < 0 || H < 0 || d <= 0) return DR_ERR_ARG;
+    if (dtype != DR_F32 && dtype != DR_BF16) return DR_ERR_ARG;
+    if (d != 64 && d != 128) return DR_ERR_UNSUPPORTED;
+    if ((double)B * T * H * d > 9.0e18 / 16) return DR_ERR_ARG;
+    *rows = (size_t)B * T * H;
+    return DR_OK;
+}
+
+static int preop_impl(const void *q_raw, const void *k_raw, const void *beta_raw, const void *gate_raw,
+                      const void *dq, const void *dk_, const void *dbeta, const void *dloga, void *q, void *k,
+                      void *beta, void *loga, int B, int T, int H, int dk, int variant, int dtype, void *stream,
+                      bool bwd) {
+    size_t rows = 0;
+    int rc = check_rows(B, T, H, dk, dtype, &rows);
+    if (rc != DR_OK) return rc;
+    if (variant < DR_DELTANET || variant > DR_KDA) return DR_ERR_ARG;
+    if (rows == 0) return DR_OK;
+    const bool gated = variant != DR_DELTANET;
+    if (!q_raw || !k_raw || !beta_raw || !q || !k || !beta) return DR_ERR_ARG;
+    if (gated && (!gate_raw || !loga)) return DR_ERR_ARG;
+    if (bwd && (!dq || !dk_ || !dbeta || (gated && !dloga))) return DR_ERR_ARG;
+    const bool kda = variant == DR_KDA;
+    const void *vec[] = {q_raw, k_raw, q, k, dq, dk_, kda ? gate_raw : nullptr, kda ? loga : nullptr,
+                         kda ? dloga : nullptr};
+    for (const void *p : vec)
+        if (p && !aligned16(p)) return DR_ERR_ALIGN;
+    const void *sca[] = {beta_raw, beta, dbeta, variant == DR_GATED ? gate_raw : nullptr,
+                         variant == DR_GATED ? loga : nullptr, variant == DR_GATED ? dloga : nullptr};
+    for (const void *p : sca)
+        if (p && !aligned_elem(p, dtype)) return DR_ERR_ALIGN;
+    PrePost pp = {};
+    pp.q = q_raw; pp.k = k_raw; pp.b = beta_raw; pp.a = gated ? gate_raw : nullptr;
+    pp.dq = dq; pp.dk = dk_; pp.db = dbeta; pp.da = gated ? dloga : nullptr;
+    pp.qo = q; pp.ko = k; pp.bo = beta; pp.ao = gated ? loga : nullptr;
+    pp.rows = rows; pp.d = dk; pp.variant = variant;
+    return launch_status(preop_run(pp, dtype == DR_BF16, bwd, (cudaStream_t)stream));
+}
+
+extern "C" int delta_rule_preop(const void *q_raw, const void *k_raw, const void *beta_raw, const void *gate_raw,
+                                void *q, void *k, void *beta, void *loga, int B, int T, int H, int dk, int variant,
+                                int dtype, void *stream) {
+    return preop_impl(q_raw, k_raw, beta_raw, gate_raw, nullptr, nullptr, nullptr, nullptr, q, k, beta, loga, B, T,
+                      H, dk, variant, dtype, stream, false);
+}
+
+extern "C" int delta_rule_preop_bwd(const void *q_raw, const void *k_raw, const void *beta_raw,
+                                    const void *gate_raw, const void *dq, const void *dk_, const void *dbeta,
+                                    const void *dloga, void *dq_raw, void *dk_raw, void *dbeta_raw, void *dgate_raw,
+                                    int B, int T, int H, int dk, int variant, int dtype, void *stream) {
+    return preop_impl(q_raw, k_raw, beta_raw, gate_raw, dq, dk_, dbeta, dloga, dq_raw, dk_raw, dbeta_raw, dgate_raw,
+                      B, T, H, dk, variant, dtype, stream, true);
+}
+
+extern "C" size_t delta_rule_postop_workspace_size(int dv) {
+    if (dv != 64 && dv != 128) return (size_t)-1;
+    return postop_ws_bytes(dv);
+}
+
+extern "C" int delta_rule_postop(const void *o, const void *gate, const float *weight, void *y, int B, int T, int H,
+                                 int dv, int dtype, void *stream) {
+    size_t rows = 0;
+    int rc = check_rows(B, T, H, dv, dtype, &rows);
+    if (rc != DR_OK) return rc;
+    if (rows == 0) return DR_OK;
+    if (!o || !gate || !y) return DR_ERR_ARG;
+    const void *vec[] = {o, gate, weight, y};
+    for (const void *p : vec)
+        if (p && !aligned16(p)) return DR_ERR_ALIGN;
+    PrePost pp = {};
+    pp.q = o; pp.k = gate; pp.w = weight; pp.qo = y; pp.rows = rows; pp.d = dv;
+    return launch_status(postop_run(pp, dtype == DR_BF16, false, (cudaStream_t)stream));
+}
+
+extern "C" int delta_rule_postop_bwd(const void *o, const void *gate, const float *weight, const void *dy, void *do_,
+                                     void *dgate, float *dweight, int B, int T, int H, int dv, int dtype,
+                                     void *workspace, size_t ws_bytes_given, void *stream) {
+    size_t rows = 0;
+    int rc = check_rows(B, T, H, dv, dtype, &rows);
+    if (rc != DR_OK) return rc;
+    if (!o || !gate || !dy || !do_ || !dgate) return DR_ERR_ARG;
+    const void *vec[] = {o, gate, weight, dy, do_, dgate, dweight};
+    for (const void *p : vec)
+        if (p && !aligned16(p)) return DR_ERR_ALIGN;
+    rc = check_buffer(workspace, ws_bytes_given, postop_ws_bytes(dv));
+    if (rc != DR_OK) return rc;
+    PrePost pp = {};
+    pp.q = o; pp.k = gate; pp.w = weight; pp.dq = dy; pp.qo = do_; pp.ko = dgate; pp.dw = dweight;
+    pp.part = (float *)workspace; pp.rows = rows; pp.d = dv;
+    return launch_status(postop_run(pp, dtype == DR_BF16, true, (cudaStream_t)stream));
 }
 
 extern "C" const char *delta_rule_strerror(int code) {

@@ -8,10 +8,12 @@
 //   o_t = S^T q_t = S'^T q_t + u_t (k_t . q_t)
 // so both column reductions of a step (S'^T k and S'^T q) come from the one decayed state.
 //
-// One CTA per (b, h, 32 value columns); 128 threads.  Lane l of warp w owns value column
-// 8 w + (l & 7) and the key rows (l >> 3) * dk / 4 ... + dk / 4 - 1 of it, so a column's
-// sums close with two shuffles and neighbouring lanes touch neighbouring columns.  The
-// tokens' q, k (and the KDA gate) are staged in shared memory 16 at a time.
+// One CTA per (b, h, 32 value columns); 128 threads.  Thread t owns the 4 value columns
+// 4 (t % 8) ... + 3 of the CTA's 32 and the key rows (t / 8) dk / 16 ... + dk / 16 - 1, so
+// the state moves as 16-byte rows; a column's sums close with two shuffles inside the warp
+// and one exchange through shared memory across the four warps (double-buffered by token,
+// so one barrier per token).  The tokens' q, k (and the KDA gate) are staged in shared
+// memory 16 at a time.
 #include "decode.cuh"
 
 namespace dr {
@@ -25,18 +27,24 @@ __global__ void __launch_bounds__(128) k_decode(const E *__restrict__ q, const E
                                                 const E *__restrict__ v, const E *__restrict__ alpha,
                                                 const E *__restrict__ beta, const float *S_in, float *S_out,
                                                 E *__restrict__ out, E *__restrict__ u, int T, int H, int dv) {
-    constexpr int RPT = DK / 4;  // key rows per thread
+    constexpr int RPT = DK / 16;  // key rows per thread
     __shared__ float sq[TT][DK], sk[TT][DK], sa[VAR == VAR_KDA ? TT : 1][DK];
     __shared__ float sv[TT][NCOL], sg[TT], sb[TT];
+    __shared__ float red[2][4][8][9];  // per token parity, warp, column group: S'^T k (4), S'^T q (4), k . q
     const int b = blockIdx.z, h = blockIdx.y, j0 = blockIdx.x * NCOL;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int jl = warp * 8 + (lane & 7), j = j0 + jl, r0 = (lane >> 3) * RPT;
+    const int rg = tid >> 3, cg = tid & 7, r0 = rg * RPT, jc = j0 + 4 * cg;
     const size_t head = ((size_t)b * H + h) * DK * dv;
 
-    float s[RPT];
+    float s[RPT][4];
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) s[i] = S_in ? S_in[head + (size_t)(r0 + i) * dv + j] : 0.f;
+    for (int i = 0; i < RPT; ++i) {
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (S_in) x = *reinterpret_cast<const float4 *>(S_in + head + (size_t)(r0 + i) * dv + jc);
+        s[i][0] = x.x; s[i][1] = x.y; s[i][2] = x.z; s[i][3] = x.w;
+    }
 
+    int par = 0;
     for (int t0 = 0; t0 < T; t0 += TT) {
         const int nt = min(TT, T - t0);
         __syncthreads();  // the previous round's tokens are no longer read
@@ -57,38 +65,78 @@ __global__ void __launch_bounds__(128) k_decode(const E *__restrict__ q, const E
             sg[tid] = VAR == VAR_GATED ? __expf(to_f(alpha[row])) : 1.f;
         }
         __syncthreads();
-        for (int tt = 0; tt < nt; ++tt) {
-            // S' = Diag(alpha) S, and this thread's parts of S'^T k, S'^T q and k . q
-            float pk = 0.f, pq = 0.f, kq = 0.f;
+        for (int tt = 0; tt < nt; ++tt, par ^= 1) {
+            // S' = Diag(alpha) S, and this thread's parts of S'^T k, S'^T q (4 columns) and k . q
+            float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f}, kq = 0.f;
 #pragma unroll
             for (int i = 0; i < RPT; ++i) {
                 const int c = r0 + i;
-                if (VAR == VAR_GATED) s[i] *= sg[tt];
-                if (VAR == VAR_KDA) s[i] *= sa[tt][c];
-                pk += s[i] * sk[tt][c];
-                pq += s[i] * sq[tt][c];
-                kq += sk[tt][c] * sq[tt][c];
+                const float kc = sk[tt][c], qc = sq[tt][c];
+                const float f = VAR == VAR_GATED ? sg[tt] : (VAR == VAR_KDA ? sa[tt][c] : 1.f);
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    if (VAR != VAR_DELTANET) s[i][jj] *= f;
+                    pk[jj] += s[i][jj] * kc;
+                    pq[jj] += s[i][jj] * qc;
+                }
+                kq += kc * qc;
             }
+            // sum over the four row groups of this warp (lanes 8 and 16 apart), then over warps
 #pragma unroll
             for (int o = 8; o < 32; o <<= 1) {
-                pk += __shfl_xor_sync(0xffffffffu, pk, o);
-                pq += __shfl_xor_sync(0xffffffffu, pq, o);
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    pk[jj] += __shfl_xor_sync(0xffffffffu, pk[jj], o);
+                    pq[jj] += __shfl_xor_sync(0xffffffffu, pq[jj], o);
+                }
                 kq += __shfl_xor_sync(0xffffffffu, kq, o);
             }
-            const float uj = sb[tt] * (sv[tt][jl] - pk);
-            const float oj = pq + uj * kq;
-#pragma unroll
-            for (int i = 0; i < RPT; ++i) s[i] += sk[tt][r0 + i] * uj;
             if (lane < 8) {
-                const size_t o_at = (((size_t)b * T + t0 + tt) * H + h) * dv + j;
-                out[o_at] = from_f<E>(oj);
-                if (u) u[o_at] = from_f<E>(uj);
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    red[par][warp][cg][jj] = pk[jj];
+                    red[par][warp][cg][4 + jj] = pq[jj];
+                }
+                red[par][warp][cg][8] = kq;
+            }
+            __syncthreads();
+            float tk[4] = {0.f, 0.f, 0.f, 0.f}, tq[4] = {0.f, 0.f, 0.f, 0.f}, tkq = 0.f;
+#pragma unroll
+            for (int wp = 0; wp < 4; ++wp) {
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    tk[jj] += red[par][wp][cg][jj];
+                    tq[jj] += red[par][wp][cg][4 + jj];
+                }
+                tkq += red[par][wp][cg][8];
+            }
+            float uj[4], oj[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                uj[jj] = sb[tt] * (sv[tt][4 * cg + jj] - tk[jj]);
+                oj[jj] = tq[jj] + uj[jj] * tkq;
+            }
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) {
+                const float kc = sk[tt][r0 + i];
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) s[i][jj] += kc * uj[jj];
+            }
+            if (rg == 0) {
+                const size_t o_at = (((size_t)b * T + t0 + tt) * H + h) * dv + jc;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    out[o_at + jj] = from_f<E>(oj[jj]);
+                    if (u) u[o_at + jj] = from_f<E>(uj[jj]);
+                }
             }
         }
     }
     if (S_out) {
 #pragma unroll
-        for (int i = 0; i < RPT; ++i) S_out[head + (size_t)(r0 + i) * dv + j] = s[i];
+        for (int i = 0; i < RPT; ++i)
+            *reinterpret_cast<float4 *>(S_out + head + (size_t)(r0 + i) * dv + jc) =
+                make_float4(s[i][0], s[i][1], s[i][2], s[i][3]);
     }
 }
 

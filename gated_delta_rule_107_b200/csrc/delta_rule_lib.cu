@@ -6,5 +6,6 @@
 #include "tc_chain.cu"
 #include "tc_bwd.cu"
 #include "decode.cu"
+#include "prepost.cu"
 #include "api.cu"
 #include "noalloc.cu"

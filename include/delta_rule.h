@@ -231,6 +231,48 @@ int delta_rule_decode(const void *q, const void *k, const void *v, const void *a
                       const float *S_in, float *S_out, void *out, void *u, int B, int T, int H, int dk, int dv,
                       int variant, int dtype, void *stream);
 
+/*
+ * Pre- and post-operations around the core, one pass over memory each
+ * (Kimi Delta Attention page: section 7.1 -- q, k L2-normalised after their
+ * projections, a logistic forget gate biased to start near sigmoid(-3), decay
+ * in log space; section 4.1 -- a sigmoid output gate on RMSNorm of the core's
+ * output).  eps = 1e-6.  Rows are the B*T*H (token, head) pairs, token-major as
+ * above; d = dk (pre) or dv (post) in {64, 128}; dtype as above for every
+ * per-token tensor; the weight w and its gradient are fp32 [dv].
+ *
+ * delta_rule_preop: from the raw projections q_raw, k_raw [B,T,H,dk], the raw
+ * write-strength logits beta_raw [B,T,H] and the raw forget logits gate_raw
+ * ([B,T,H] Gated DeltaNet, [B,T,H,dk] KDA, unused and may be NULL for
+ * DeltaNet), writes the core's inputs:
+ *     q = q_raw / sqrt(|q_raw|^2 + eps),  k likewise        (per row)
+ *     beta = sigmoid(beta_raw),  loga = -softplus(gate_raw)  (= log alpha)
+ * delta_rule_preop_bwd: the gradients of <dq, q> + <dk_, k> + <dbeta, beta> +
+ * <dloga, loga> with respect to q_raw, k_raw, beta_raw, gate_raw.
+ *
+ * delta_rule_postop: y = o / sqrt(mean(o^2) + eps) * w * sigmoid(gate) per row
+ * of dv channels, for the core's output o, caller-computed gate logits gate
+ * [B,T,H,dv] and the per-channel weight w (NULL = all ones).
+ * delta_rule_postop_bwd: for dy [B,T,H,dv], the gradients do, dgate (required)
+ * and dweight = the sum over all rows (NULL = not written).  It needs a
+ * workspace of delta_rule_postop_workspace_size(dv) bytes (256-byte aligned);
+ * dweight is summed in a fixed order, so results are deterministic.
+ *
+ * Outputs must not alias inputs.  Errors as for the other entry points.
+ */
+int delta_rule_preop(const void *q_raw, const void *k_raw, const void *beta_raw, const void *gate_raw, void *q,
+                     void *k, void *beta, void *loga, int B, int T, int H, int dk, int variant, int dtype,
+                     void *stream);
+int delta_rule_preop_bwd(const void *q_raw, const void *k_raw, const void *beta_raw, const void *gate_raw,
+                         const void *dq, const void *dk_, const void *dbeta, const void *dloga, void *dq_raw,
+                         void *dk_raw, void *dbeta_raw, void *dgate_raw, int B, int T, int H, int dk, int variant,
+                         int dtype, void *stream);
+size_t delta_rule_postop_workspace_size(int dv);
+int delta_rule_postop(const void *o, const void *gate, const float *weight, void *y, int B, int T, int H, int dv,
+                      int dtype, void *stream);
+int delta_rule_postop_bwd(const void *o, const void *gate, const float *weight, const void *dy, void *do_,
+                          void *dgate, float *dweight, int B, int T, int H, int dv, int dtype, void *workspace,
+                          size_t ws_bytes, void *stream);
+
 /* Static text for a DR_* code ("ok", "invalid argument", ...). */
 const char *delta_rule_strerror(int code);
 
