@@ -45,6 +45,10 @@ enum { K_FWD = 0, K_BWD = 1, K_FWD_SAVE = 2, K_BWD_SAVED = 3 };
 bool is_bwd(int kind) { return kind == K_BWD || kind == K_BWD_SAVED; }
 
 bool use_split(const Geo &g, int dtype) { return tc_split_supported(g, dtype == DR_BF16); }
+// KDA's forward on the split path (its backward stays on the CUDA-core kernels)
+bool use_split_kda(const Geo &g, int dtype, int kind) {
+    return !is_bwd(kind) && tc_split_kda_supported(g, dtype == DR_BF16);
+}
 
 size_t ws_bytes(const Geo &g, int dtype, int kind) {
     if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
@@ -56,6 +60,7 @@ size_t ws_bytes(const Geo &g, int dtype, int kind) {
             default: return tc_ws_bytes(g, WS_REV);
         }
     }
+    if (use_split_kda(g, dtype, kind)) return tc_ws_bytes(g, WS_FWD | WS_KDA);
     if (!is_bwd(kind) && use_tc_fwd(g, dtype)) return 0;
     return simt_ws_bytes(g, is_bwd(kind));
 }
@@ -131,6 +136,12 @@ static int fwd_impl(const void *q, const void *k, const void *v, const void *alp
         else tc_ws_carve(g, WS_FWD, workspace, &w);
         rc = launch_status(tc_chunk_prep(g, t, w, save, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, save ? 2 : 0, s, rec));
+    } else if (use_split_kda(g, dtype, kind)) {
+        TcWs w = {};
+        tc_ws_carve(g, WS_FWD | WS_KDA, workspace, &w);
+        rc = launch_status(tc_kda_gates(g, t, w, s, rec));
+        if (rc == DR_OK) rc = launch_status(tc_chunk_prep(g, t, w, false, s, rec));
+        if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, 0, s, rec));
     } else if (use_tc_fwd(g, dtype)) {
         rc = launch_status(tc_fwd(g, t, workspace, s, rec));
     } else {
@@ -196,6 +207,7 @@ static int launch_plan(const Geo &g, int dtype, int kind, const char **names, in
     static const char *const SPLIT_BWD[4] = {"k_chunk_prep(keep)", "k_chain_fwd(recompute)", "k_chain_rev",
                                              "k_bwd_chunk_tc"};
     static const char *const SPLIT_BWD_SAVED[2] = {"k_chain_rev", "k_bwd_chunk_tc"};
+    static const char *const SPLIT_KDA_FWD[3] = {"k_kda_gates", "k_chunk_prep", "k_chain_fwd"};
     int n = 0;
     const char *const *src = nullptr;
     if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
@@ -206,6 +218,9 @@ static int launch_plan(const Geo &g, int dtype, int kind, const char **names, in
             case K_BWD: src = SPLIT_BWD; n = 4; break;
             default: src = SPLIT_BWD_SAVED; n = 2; break;
         }
+    } else if (use_split_kda(g, dtype, kind)) {
+        src = SPLIT_KDA_FWD;
+        n = 3;
     } else if (!is_bwd(kind) && use_tc_fwd(g, dtype)) {
         return tc_fwd_launches(g, names, max_names);
     } else {

@@ -59,7 +59,8 @@ enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_MMA, B_NUM };
 static_assert(M_SKP + 512 <= 4096, "misc overflow");
 
 struct FMaps {
-    CUtensorMap q, k;       // [B, T, H, 128] bf16; box 64 x 64 tokens
+    CUtensorMap q, k;       // [B, T, H, 128] bf16; box 64 x 64 tokens (KDA: the workspace's
+                            // q e^g and k e^{g_C - g}, [chunks * 64][128], box 64 x 64)
     CUtensorMap W, Ut;      // [chunks * 64][128] bf16; box 64 x 64
     CUtensorMap P;          // [chunks * 64][64] bf16; box 64 x 64
     CUtensorMap out, u;     // forward outputs [B, T, H, 128] (stores)
@@ -79,7 +80,14 @@ struct Args {
     int has_out, has_u;       // forward outputs requested
     float *skt;               // reverse output
     int B, T, H, N, has_du;
+    const float *egc;         // KDA forward: [chunks][128] e^{g_C} per key channel
 };
+
+// Producer side, KDA: the per-channel decay e^{g_C} of chunk ci into cf[0..127].
+__device__ __forceinline__ void chunk_factors_kda(const float *egc, size_t ci, float *cf, int lane) {
+#pragma unroll
+    for (int c = lane; c < 128; c += 32) cf[c] = egc[ci * 128 + c];
+}
 
 // Producer side: the gate factors of chunk ci into cf (e^{g_C - g}, e^g, e^{g_C}).
 __device__ __forceinline__ void chunk_factors(const float *gb, size_t ci, float *cf, int lane) {
@@ -114,7 +122,9 @@ __device__ __forceinline__ void tmem_row32(uint32_t taddr, float *v) {
 // ====================================== forward chain ======================================
 // MODE 0: forward (o, u, S_T); 1: recompute for the backward (S_n, U of every chunk);
 // 2: forward that also keeps S_n and U for the backward.
-template <int MODE>
+// KDA (MODE 0): q and k arrive gate-scaled (q e^g, k e^{g_C - g}), so the row factors are 1,
+// and the state decays by row: S <- Diag(e^{g_C}) S + (k e^{g_C - g})^T U.
+template <int MODE, int KDA>
 __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant__ FMaps mp, Args a) {
     constexpr bool OUT = MODE != 1, KEEP = MODE != 0;
     extern __shared__ unsigned char smem_raw[];
@@ -155,13 +165,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
                     tma_load_2d(st + FS_WQ + p * 16384, &mp.W, 64 * p, ci * C, &bar[B_FULL0 + s]);
-                    if (OUT) tma_load_4d(st + FS_WQ + p * 16384 + 8192, &mp.q, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
-                    tma_load_4d(st + FS_K + p * 8192, &mp.k, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
+                    if (KDA) {
+                        tma_load_2d(st + FS_WQ + p * 16384 + 8192, &mp.q, 64 * p, ci * C, &bar[B_FULL0 + s]);
+                        tma_load_2d(st + FS_K + p * 8192, &mp.k, 64 * p, ci * C, &bar[B_FULL0 + s]);
+                    } else {
+                        if (OUT) tma_load_4d(st + FS_WQ + p * 16384 + 8192, &mp.q, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
+                        tma_load_4d(st + FS_K + p * 8192, &mp.k, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
+                    }
                 }
                 tma_load_2d(st + FS_UP, &mp.Ut, j0, ci * C, &bar[B_FULL0 + s]);
                 if (OUT) tma_load_2d(st + FS_UP + 8192, &mp.P, 0, ci * C, &bar[B_FULL0 + s]);
             }
-            chunk_factors(a.gb, (size_t)ci, cf_all + s * 132, lane);
+            if (KDA) chunk_factors_kda(a.egc, (size_t)ci, cf_all + s * 132, lane);
+            else chunk_factors(a.gb, (size_t)ci, cf_all + s * 132, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[B_FULL0 + s]);
             issued[s]++;
@@ -233,8 +249,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             if (wabort(got)) break;
             // this chunk's factors, read before the stage is released
             const float *cf = cf_all + s * 132;
-            const float egC = cf[128];
-            const float rowf = cf[trow];  // lanes 0-63: e^{gC - g_r}; lanes 64-127: e^{g_r}, r = trow - 64
+            // KDA: this thread's state row decays by e^{g_C} of its key channel; no row factors
+            const float egC = KDA ? cf[trow] : cf[128];
+            const float rowf = KDA ? 1.f : cf[trow];  // lanes 0-63: e^{gC - g_r}; lanes 64-127: e^{g_r}, r = trow - 64
             // ---------------- D = [W ; q] S ----------------
             if (wc == 0) {
                 fence_after_sync();
@@ -550,6 +567,11 @@ bool tc_split_supported(const Geo &g, bool bf16) {
            (size_t)g.B * g.H * g.N * 128 <= (size_t)INT_MAX;
 }
 
+bool tc_split_kda_supported(const Geo &g, bool bf16) {
+    return bf16 && g.C == 64 && g.dk == 128 && g.dv == 128 && g.variant == VAR_KDA &&
+           (size_t)g.B * g.H * g.N * 128 <= (size_t)INT_MAX;
+}
+
 static size_t ws_al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Carves the given parts of the split-path workspace from base (or only counts, when base
@@ -575,6 +597,11 @@ static size_t ws_carve(const Geo &g, int parts, char *base, TcWs *w) {
         w->dUn = (__nv_bfloat16 *)take(nc * C * DV * 2);
         w->skt = (float *)take(nc * 2 * C * 4);
     }
+    if (parts & WS_KDA) {
+        __nv_bfloat16 **tiles[] = {&w->Kt1, &w->Qt1, &w->Kh, &w->Kt, &w->Qt, &w->Kb};
+        for (__nv_bfloat16 **t : tiles) *t = (__nv_bfloat16 *)take(nc * C * DK * 2);
+        w->egc = (float *)take(nc * DK * 4);
+    }
     return off;
 }
 
@@ -589,8 +616,11 @@ cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, int mode
     using namespace tch;
     FMaps mp;
     const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;
-    const bool out = mode != 1, keep = mode != 0;
-    bool ok = tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) && tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64) &&
+    const bool out = mode != 1, keep = mode != 0, kda = g.variant == VAR_KDA;
+    if (kda && mode != 0) return cudaErrorInvalidValue;
+    bool ok = (kda ? tc::make_map_2d_bf16(&mp.q, w.Qt, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.k, w.Kb, DK, NC * C, 64)
+                   : tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) &&
+                         tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64)) &&
               tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.Ut, w.Ut, DV, NC * C, 64) &&
               tc::make_map_2d_bf16(&mp.P, w.P, C, NC * C, 64);
     mp.out = mp.u = mp.Sn = mp.Un = mp.q;  // unused ones keep a valid map
@@ -601,33 +631,25 @@ cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, int mode
     if (!ok) return cudaErrorInvalidValue;
     Args a = {};
     a.gb = w.gb; a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
-    a.S0 = t.S0;
+    a.S0 = t.S0; a.egc = w.egc;
     if (out) {
         a.has_out = t.out != nullptr; a.has_u = t.u != nullptr; a.ST = t.S_T;
     }
     const size_t smem = SMEM_BYTES + 1024;
     const dim3 grid(DV / DVB, g.H, g.B);
     cudaError_t e;
-    switch (mode) {
-        case 0:
-            e = cudaFuncSetAttribute(k_chain_fwd<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-            rec.mark(s);
-            k_chain_fwd<0><<<grid, NTHREADS, smem, s>>>(mp, a);
-            break;
-        case 1:
-            e = cudaFuncSetAttribute(k_chain_fwd<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-            rec.mark(s);
-            k_chain_fwd<1><<<grid, NTHREADS, smem, s>>>(mp, a);
-            break;
-        default:
-            e = cudaFuncSetAttribute(k_chain_fwd<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-            rec.mark(s);
-            k_chain_fwd<2><<<grid, NTHREADS, smem, s>>>(mp, a);
-            break;
-    }
+    auto go = [&](auto kern) -> cudaError_t {
+        cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e2 != cudaSuccess) return e2;
+        rec.mark(s);
+        kern<<<grid, NTHREADS, smem, s>>>(mp, a);
+        return cudaSuccess;
+    };
+    if (kda) e = go(k_chain_fwd<0, 1>);
+    else if (mode == 0) e = go(k_chain_fwd<0, 0>);
+    else if (mode == 1) e = go(k_chain_fwd<1, 0>);
+    else e = go(k_chain_fwd<2, 0>);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

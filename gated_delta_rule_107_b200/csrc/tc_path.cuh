@@ -18,6 +18,8 @@ int tc_fwd_launches(const Geo &g, const char **names, int max_names);
 // Split path: Gated DeltaNet / DeltaNet, bf16, dk = dv = 128, C = 64, and chunk row
 // indices that fit the 32-bit coordinates of a TMA load.
 bool tc_split_supported(const Geo &g, bool bf16);
+// The same shapes for KDA: the split forward (the backward stays on the CUDA-core path).
+bool tc_split_kda_supported(const Geo &g, bool bf16);
 
 // Workspace of the split path, chunk-major (ci = (b H + h) N + n), every matrix row-major:
 // bf16 tiles that later kernels load with TMA, plus fp32 per-token factors.  Three parts:
@@ -39,17 +41,29 @@ struct TcWs {
     __nv_bfloat16 *dSn;  // [ci][dk][dv]  dL/dS of the state leaving chunk n
     __nv_bfloat16 *dUn;  // [ci][C][dv]   dL/dU = du + P^T dO + Kbar dS_{n+1}
     float *skt;          // [ci][2][C]    per 64-column half of dv: U_r . (Kbar dS_{n+1})_r
+    // KDA forward (channel-wise gates, g = in-chunk cumulative log gate per key channel,
+    // g_m its value at the chunk's middle token, exponents clamped to [-80, 80]):
+    __nv_bfloat16 *Kt1;  // [ci][C][dk]   k e^{g - g_m}      (rows of P1's A)
+    __nv_bfloat16 *Qt1;  // [ci][C][dk]   q e^{g - g_m}      (rows of P1's A)
+    __nv_bfloat16 *Kh;   // [ci][C][dk]   k e^{g_m - g}      (P1's B)
+    __nv_bfloat16 *Kt;   // [ci][C][dk]   k e^{g}            (W = T diag(beta) Kt)
+    __nv_bfloat16 *Qt;   // [ci][C][dk]   q e^{g}            (o = Qt S + P U)
+    __nv_bfloat16 *Kb;   // [ci][C][dk]   k e^{g_C - g}      (S+ = Diag(e^{g_C}) S + Kb^T U)
+    float *egc;          // [ci][dk]      e^{g_C}
 };
-enum { WS_FWD = 1, WS_KEEP = 2, WS_REV = 4 };
+enum { WS_FWD = 1, WS_KEEP = 2, WS_REV = 4, WS_KDA = 8 };
 // Bytes of the given parts, laid out one after another in the order FWD, KEEP, REV.
 size_t tc_ws_bytes(const Geo &g, int parts);
 // Sets the pointers of the given parts, carved from base in that order; leaves the others.
 void tc_ws_carve(const Geo &g, int parts, void *base, TcWs *w);
 
+// KDA's gate-scaled operands of every chunk (tc_prep.cu): w.Kt1 ... w.Kb, w.egc.
+cudaError_t tc_kda_gates(const Geo &g, const Tensors &t, const TcWs &w, cudaStream_t s, Rec &rec);
 // Per-chunk products (tc_prep.cu): g and beta, W, U~, P; with keep also T and k k^T.
+// For KDA (no keep) from the operands of tc_kda_gates.
 cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool keep, cudaStream_t s, Rec &rec);
 // Forward state chain (tc_chain.cu).  mode 0: o, u, S_T; mode 1 (recompute for the
-// backward): S_n and U of every chunk; mode 2: both.
+// backward): S_n and U of every chunk; mode 2: both.  KDA: mode 0 only.
 cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, int mode, cudaStream_t s, Rec &rec);
 // Reverse state chain (tc_chain.cu): dS_{n+1} and dL/dU of every chunk (w.dSn, w.dUn), the
 // row sums w.skt, and dS0.

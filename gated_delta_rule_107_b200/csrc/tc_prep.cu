@@ -1,5 +1,5 @@
 // tc_prep.cu -- the per-chunk products of the chunked gated delta rule, one CTA per chunk
-// (Gated DeltaNet and DeltaNet; bf16 I/O, dk = dv = 128, C = 64).
+// (Gated DeltaNet, DeltaNet and KDA; bf16 I/O, dk = dv = 128, C = 64).
 //
 // Chunked form of "线性注意力架构演进与Kimi Delta Attention创新实践" (sections 2.1, 6.1,
 // 6.2, 7.1).  With g the in-chunk cumulative log gate:
@@ -9,6 +9,11 @@
 //   T  = (I + A)^-1                            (the UT transform; tc_inverse.cuh)
 //   W  = T diag(beta e^g) k,   U~ = T diag(beta) v
 //   backward (and a forward that saves for it): T and k k^T kept for the gradient kernel.
+// KDA's gates are per key channel, so they cannot leave the dot products as scalars: a
+// first kernel (k_kda_gates) writes the gate-scaled operands, and the same products become
+//   P1 = [k e^{g-g_m} ; q e^{g-g_m}] . (k e^{g_m-g})^T,   W = T diag(beta) (k e^g)
+// with g per channel and g_m its value at the chunk's middle token (the midpoint split
+// keeps every factor within e^{+-80}: exponents are clamped there).
 //
 // Every chunk is independent, so the grid covers all chunks of all heads at once (two
 // CTAs per SM); the serial state chains (tc_chain.cu) then only carry the state.  The
@@ -38,7 +43,8 @@ constexpr uint32_t OFF_V = 32768;      // 16K v [i][j]
 constexpr uint32_t OFF_F = 49152;      // 32K fp32 A | T (inverse), then staging W [r][c] | U~ [r][j]
 constexpr uint32_t OFF_P = 81920;      //  8K P [r][i]
 constexpr uint32_t OFF_MISC = 90112;   //  2K
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 2048;
+constexpr uint32_t OFF_X = 92160;      // 16K KDA: k e^{g_m - g} (P1's B), then k e^g (W's B)
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 2048, SMEM_KDA = OFF_X + 16384;
 // misc
 constexpr uint32_t M_BAR = 0;          // [0] loads, [1] MMA
 constexpr uint32_t M_TMEM = 64, M_ABORT = 68, M_BIG = 72;
@@ -53,6 +59,7 @@ struct Maps {
     CUtensorMap W, Ut;    // [chunks * 64][128] bf16; box 64 x 64 (stores)
     CUtensorMap P;        // [chunks * 64][64] bf16; box 64 x 64 (store)
     CUtensorMap KK, Tn;   // [chunks * 64][64] bf16; box 64 x 64 (stores, when KEEP)
+    CUtensorMap Kt1, Qt1, Kh, Kt;  // KDA: [chunks * 64][128] bf16 gate-scaled operands; box 64 x 64
 };
 
 struct Args {
@@ -80,17 +87,24 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
     const int ci = (b * H + h) * a.N + n;  // < 2^31 / 128 (checked by the launcher)
     const int trow = tid;                  // TMEM lane of this thread
 
-    int mma_issued = 0;
+    int mma_issued = 0, kt_issued = 0;
     if (tid == 0) {
         mbar_init(&bar[0], 1);
         mbar_init(&bar[1], 1);
+        mbar_init(&bar[2], 1);
         *abort_flag = 0;
         fence_mbar_init();
-        mbar_arrive_tx(&bar[0], 49152u);
+        mbar_arrive_tx(&bar[0], VAR == VAR_KDA ? 65536u : 49152u);
 #pragma unroll
         for (int p = 0; p < 2; ++p) {
-            tma_load_4d(sm + OFF_KQ + p * 16384, &mp.k, 64 * p, h, t0, b, &bar[0]);
-            tma_load_4d(sm + OFF_KQ + p * 16384 + 8192, &mp.q, 64 * p, h, t0, b, &bar[0]);
+            if (VAR == VAR_KDA) {  // the gate-scaled operands of tc_kda_gates
+                tma_load_2d(sm + OFF_KQ + p * 16384, &mp.Kt1, 64 * p, ci * C, &bar[0]);
+                tma_load_2d(sm + OFF_KQ + p * 16384 + 8192, &mp.Qt1, 64 * p, ci * C, &bar[0]);
+                tma_load_2d(sm + OFF_X + p * 8192, &mp.Kh, 64 * p, ci * C, &bar[0]);
+            } else {
+                tma_load_4d(sm + OFF_KQ + p * 16384, &mp.k, 64 * p, h, t0, b, &bar[0]);
+                tma_load_4d(sm + OFF_KQ + p * 16384 + 8192, &mp.q, 64 * p, h, t0, b, &bar[0]);
+            }
             tma_load_4d(sm + OFF_V + p * 8192, &mp.v, 64 * p, h, t0, b, &bar[0]);
         }
     }
@@ -161,15 +175,23 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
     // ---------------- P1: [k ; q] . k^T ----------------
     if (ok && tid == 0) {
         const uint32_t id = idesc_bf16(128, 64, 0, 0);
+        const uint32_t sx = smem_u32(sm + OFF_X);
 #pragma unroll
         for (int st = 0; st < 8; ++st) {
             const uint32_t ad = skq + (st >> 2) * 16384 + (st & 3) * 32;
-            mma_bf16(tbase + TM_G1, sdesc(ad, 16, 1024), sdesc(ad, 16, 1024), id, st > 0);
+            const uint32_t bd = VAR == VAR_KDA ? sx + (st >> 2) * 8192 + (st & 3) * 32 : ad;
+            mma_bf16(tbase + TM_G1, sdesc(ad, 16, 1024), sdesc(bd, 16, 1024), id, st > 0);
         }
         mma_commit(&bar[1]);
         mma_issued++;
     }
     if (ok) ok = consensus(wait_mma());
+    if (VAR == VAR_KDA && ok && tid == 0) {  // k e^g, the B of W's product, over the finished B of P1
+        mbar_arrive_tx(&bar[2], 16384u);
+#pragma unroll
+        for (int p = 0; p < 2; ++p) tma_load_2d(sm + OFF_X + p * 8192, &mp.Kt, 64 * p, ci * C, &bar[2]);
+        kt_issued = 1;
+    }
     // ---------------- A (fp32, for the inverse), P (bf16 tile), k k^T ----------------
     if (ok) {
         float g1[64];
@@ -180,7 +202,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
         const int r = arow ? trow : trow - 64;
         // gate factor of each (r, i): e^{g_r - g_i}, split at the midpoint unless the range is large
         float f[64];
-        if (VAR == VAR_DELTANET) {
+        if (VAR != VAR_GATED) {  // DeltaNet; KDA carries its gates in the operands
 #pragma unroll
             for (int i = 0; i < 64; ++i) f[i] = 1.f;
         } else if (!big) {
@@ -256,6 +278,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
     fence_before_sync();
     ok = consensus(ok);
     // ---------------- W = [T diag(beta e^g) ; *] k,  U~ = [T diag(beta) ; *] v ----------------
+    if (VAR == VAR_KDA && ok) ok = consensus(mbar_wait(&bar[2], 0, abort_flag));
     if (ok && tid == 0) {
         fence_after_sync();
         if (KEEP) {
@@ -263,10 +286,10 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
             bulk_commit();
         }
         const uint32_t id = idesc_bf16(128, 128, 0, 1);
+        const uint64_t dkb = VAR == VAR_KDA ? sdesc(smem_u32(sm + OFF_X), 8192, 1024) : sdesc(skq, 16384, 1024);
 #pragma unroll
         for (int st = 0; st < 4; ++st) {
-            mma_bf16(tbase + TM_XW, sdesc(skq + 24576 + st * 32, 16, 1024), sdesc(skq + st * 2048, 16384, 1024), id,
-                     st > 0);
+            mma_bf16(tbase + TM_XW, sdesc(skq + 24576 + st * 32, 16, 1024), sdesc_at(dkb, st * 2048), id, st > 0);
             mma_bf16(tbase + TM_XU, sdesc(skq + 8192 + st * 32, 16, 1024), sdesc(sv + st * 2048, 8192, 1024), id,
                      st > 0);
         }
@@ -300,6 +323,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
         if (*abort_flag) {  // let whatever was issued finish before the CTA leaves
             volatile int dummy = 0;
             mbar_wait(&bar[0], 0, &dummy, 100000000ull);
+            if (kt_issued) mbar_wait(&bar[2], 0, &dummy, 100000000ull);
             if (mma_issued > 0) mbar_wait(&bar[1], (mma_issued - 1) & 1, &dummy, 100000000ull);
         }
     }
@@ -309,9 +333,111 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
     if (warp == 0) tmem_dealloc(tbase, TM_COLS);
 }
 
+// ---------------------------------------------------------------- KDA gate operands
+// One CTA of 128 threads per chunk.  Thread (tg, cg) = (tid / 16, tid % 16) owns key channels
+// 8 cg ... 8 cg + 7 of tokens 8 tg ... 8 tg + 7, so every access moves 16 bytes.  The
+// in-chunk cumulative log gate g of each channel is a prefix sum over the chunk's tokens
+// (tokens past T add nothing): inside the thread's 8 tokens, then across the 8 token groups
+// through shared memory.  Then every gate-scaled operand the split path needs is written
+// row-major per chunk.  Exponents are clamped to [-80, 80] so that every factor is a finite
+// bf16.
+struct KdaArgs {
+    const __nv_bfloat16 *q, *k, *alpha;
+    __nv_bfloat16 *Kt1, *Qt1, *Kh, *Kt, *Qt, *Kb;
+    float *egc;
+    int T, H, N;
+};
+
+__device__ __forceinline__ float clamped_exp(float x) { return __expf(fminf(fmaxf(x, -80.f), 80.f)); }
+
+__device__ __forceinline__ void ld8_bf16(const __nv_bfloat16 *p, float *v) {
+    const uint4 x = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+__device__ __forceinline__ void st8_bf16(__nv_bfloat16 *p, const float *v) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = pack_bf16(v[2 * i], v[2 * i + 1]);
+    *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
+    __shared__ float tot[8][DK];
+    __shared__ float gmid[DK], gend[DK];
+    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int tg = threadIdx.x >> 4, cg = threadIdx.x & 15, c0 = 8 * cg;
+    const int t0 = n * C, L = min(C, a.T - t0);
+    const size_t ci = ((size_t)b * a.H + h) * a.N + n;
+    auto at = [&](int r) { return (((size_t)b * a.T + t0 + r) * a.H + h) * DK + c0; };
+    float g[8][8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (8 * tg + r < L) ld8_bf16(a.alpha + at(8 * tg + r), x);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) g[r][j] = (r ? g[r - 1][j] : 0.f) + x[j];
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) tot[tg][c0 + j] = g[7][j];
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float off = 0.f;
+        for (int t2 = 0; t2 < tg; ++t2) off += tot[t2][c0 + j];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) g[r][j] += off;
+        if (tg == C / 16 - 1) gmid[c0 + j] = g[7][j];  // token C/2 - 1, the middle
+        if (tg == 7) gend[c0 + j] = g[7][j];           // token C - 1, the last
+    }
+    __syncthreads();
+    float gm[8], gC[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        gm[j] = gmid[c0 + j];
+        gC[j] = gend[c0 + j];
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int tr = 8 * tg + r;
+        float kr[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, qr[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (tr < L) {
+            ld8_bf16(a.k + at(tr), kr);
+            ld8_bf16(a.q + at(tr), qr);
+        }
+        float o1[8], o2[8], o3[8], o4[8], o5[8], o6[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float em = clamped_exp(g[r][j] - gm[j]), ei = clamped_exp(gm[j] - g[r][j]);
+            const float eg = clamped_exp(g[r][j]), ec = clamped_exp(gC[j] - g[r][j]);
+            o1[j] = kr[j] * em; o2[j] = qr[j] * em; o3[j] = kr[j] * ei;
+            o4[j] = kr[j] * eg; o5[j] = qr[j] * eg; o6[j] = kr[j] * ec;
+        }
+        const size_t o = (ci * C + tr) * DK + c0;
+        st8_bf16(a.Kt1 + o, o1);
+        st8_bf16(a.Qt1 + o, o2);
+        st8_bf16(a.Kh + o, o3);
+        st8_bf16(a.Kt + o, o4);
+        st8_bf16(a.Qt + o, o5);
+        st8_bf16(a.Kb + o, o6);
+    }
+    if (tg == 0) {
+        float e[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) e[j] = clamped_exp(gC[j]);
+        *reinterpret_cast<float4 *>(a.egc + ci * DK + c0) = make_float4(e[0], e[1], e[2], e[3]);
+        *reinterpret_cast<float4 *>(a.egc + ci * DK + c0 + 4) = make_float4(e[4], e[5], e[6], e[7]);
+    }
+}
+
 template <int VAR, int KEEP>
 static cudaError_t launch_prep(const Maps &mp, const Args &a, dim3 grid, cudaStream_t s, Rec &rec) {
-    const size_t smem = SMEM_BYTES + 1024;
+    const size_t smem = (VAR == VAR_KDA ? SMEM_KDA : SMEM_BYTES) + 1024;
     cudaError_t e =
         cudaFuncSetAttribute(k_chunk_prep<VAR, KEEP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -322,6 +448,17 @@ static cudaError_t launch_prep(const Maps &mp, const Args &a, dim3 grid, cudaStr
 
 }  // namespace tcp
 
+cudaError_t tc_kda_gates(const Geo &g, const Tensors &t, const TcWs &w, cudaStream_t s, Rec &rec) {
+    using namespace tcp;
+    KdaArgs a;
+    a.q = (const __nv_bfloat16 *)t.q; a.k = (const __nv_bfloat16 *)t.k; a.alpha = (const __nv_bfloat16 *)t.alpha;
+    a.Kt1 = w.Kt1; a.Qt1 = w.Qt1; a.Kh = w.Kh; a.Kt = w.Kt; a.Qt = w.Qt; a.Kb = w.Kb; a.egc = w.egc;
+    a.T = g.T; a.H = g.H; a.N = g.N;
+    rec.mark(s);
+    k_kda_gates<<<dim3(g.N, g.H, g.B), DK, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
 cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool keep, cudaStream_t s, Rec &rec) {
     using namespace tcp;
     Maps mp;
@@ -331,11 +468,15 @@ cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool ke
               tc::make_map_2d_bf16(&mp.Ut, w.Ut, DV, NC * C, 64) && tc::make_map_2d_bf16(&mp.P, w.P, C, NC * C, 64);
     if (ok && keep)
         ok = tc::make_map_2d_bf16(&mp.KK, w.KK, C, NC * C, 64) && tc::make_map_2d_bf16(&mp.Tn, w.Tn, C, NC * C, 64);
+    if (ok && g.variant == VAR_KDA)
+        ok = tc::make_map_2d_bf16(&mp.Kt1, w.Kt1, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.Qt1, w.Qt1, DK, NC * C, 64) &&
+             tc::make_map_2d_bf16(&mp.Kh, w.Kh, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.Kt, w.Kt, DK, NC * C, 64);
     if (!ok) return cudaErrorInvalidValue;
     Args a;
     a.alpha = t.alpha; a.beta = t.beta; a.gb = w.gb;
     a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
     const dim3 grid(g.N, g.H, g.B);
+    if (g.variant == VAR_KDA) return launch_prep<VAR_KDA, 0>(mp, a, grid, s, rec);  // no saved form
     if (g.variant == VAR_GATED)
         return keep ? launch_prep<VAR_GATED, 1>(mp, a, grid, s, rec) : launch_prep<VAR_GATED, 0>(mp, a, grid, s, rec);
     return keep ? launch_prep<VAR_DELTANET, 1>(mp, a, grid, s, rec) : launch_prep<VAR_DELTANET, 0>(mp, a, grid, s, rec);

@@ -151,7 +151,10 @@ def test_bf16_d128_uses_the_tensor_core_kernel():
     for variant in (0, 1):
         for kind, names in split.items():
             assert binding.launches(8, 4096, 8, 128, 128, variant, 64, 1, kind) == names
-    assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 0) == ["k_fwd_tc"]
+    kda_split = ["k_kda_gates", "k_chunk_prep", "k_chain_fwd"]
+    assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 0) == kda_split
+    assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 2) == kda_split  # no saved form: the plain forward
+    assert binding.launches(2, 512, 4, 128, 64, 2, 64, 1, 0) == ["k_fwd_tc"]
     assert binding.launches(2, 512, 4, 128, 64, 1, 64, 1, 0) == ["k_fwd_tc"]
     assert binding.launches(1, 256, 2, 64, 64, 0, 64, 0, 0) == ["k_prep", "k_scan", "k_out"]
 
