@@ -157,6 +157,30 @@ def cpu_oracle_sample(w, steps=1, seed=0):
             "sample_seconds": t}, times, np
 
 
+# ---------------------------------------------------------------------------------------------
+# Replicas (N > 1, one rank per GPU): every rank solves its own independent (b, h) problems --
+# the path has no exchange step -- and the job's time is the slowest rank's.
+def replica_seed(seed: int, rank: int) -> int:
+    """Seed of a rank's replica: each rank draws its own inputs."""
+    return seed + 1000 * rank
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """The largest value of x over the ranks of the default process group (x itself alone)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: int, world: int, ms_max: float) -> float:
+    """Units per second of the whole job: every rank's units over the slowest rank's time."""
+    return units_per_rank * world / (ms_max / 1e3)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -202,7 +226,7 @@ def run_ours(args):
     B, T, H, dk, dv, C, var = (args.batch or w.B), w.T, w.H, w.dk, w.dv, 64, w.variant
     vname = {0: "deltanet", 1: "gdn", 2: "kda"}[var]
     dt = binding.DR_BF16
-    x = make_inputs(var, w.dtype, B, T, H, dk, dv, seed=w.seed + 1000 * rank, s0_std=w.s0_std, grads=True, du=True,
+    x = make_inputs(var, w.dtype, B, T, H, dk, dv, seed=replica_seed(w.seed, rank), s0_std=w.s0_std, grads=True, du=True,
                     device=dev)
     s0 = x["S0"] if w.s0_std else None
     elem = 2
@@ -306,13 +330,9 @@ def run_ours(args):
     if binding.sync_status() != binding.DR_OK:
         raise RuntimeError("device error word set during the timed region")
 
-    ms = statistics.mean(step_ms)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(statistics.mean(step_ms), dev)
     tokens = B * T * world
-    value = tokens / (ms / 1e3)
+    value = weak_scaling_value(B * T, world, ms)
 
     # ---- the plain forward + recomputing backward, same protocol (reported beside) ----
     rstep, rf_names, rb_names, rfev, rbev = make_step(False)
@@ -331,11 +351,7 @@ def run_ours(args):
     if binding.sync_status() != binding.DR_OK:
         raise RuntimeError("device error word set during the recompute leg")
     # the step is the sum of its kernels' device times (consecutive events of each call)
-    r_ms = sum(statistics.mean(v) for v in r_kern.values())
-    if world > 1:
-        t = torch.tensor([r_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        r_ms = float(t.item())
+    r_ms = max_over_ranks(sum(statistics.mean(v) for v in r_kern.values()), dev)
 
     # ---- one decoding step (delta_rule_decode), reported beside: DECODE_B sequences, one
     # token each, the fp32 state updated in place; L2 flushed before every call ----
@@ -437,11 +453,7 @@ def run_ours(args):
             e2e_step()
         e1.record()
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / e2e_steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
 
     peaks = load_peaks()
     cnt = alg_counts(B, T, H, dk, dv, C, var, elem, s0=s0 is not None)
