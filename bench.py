@@ -473,7 +473,7 @@ def run_ours(args):
     rk_ms = kern_ms[rk] if rk else b_ms
     achieved = r_bytes / (rk_ms / 1e3) / 1e9
     r_label = rk.split(":", 1)[1] if rk else "backward call (" + "+".join(bwd_names) + ")"
-    # the forward call (the benchmark spec's T = 4096 target) against its own algorithmic bytes
+    # the forward call at T = 4096 against its own algorithmic bytes
     f_bytes = cnt["fwd_bytes"]
     f_achieved = f_bytes / (f_ms / 1e3) / 1e9
     fwd_label = fwd_names[0] if len(fwd_names) == 1 else "forward call (" + "+".join(fwd_names) + ")"

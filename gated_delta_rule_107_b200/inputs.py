@@ -49,7 +49,7 @@ class Workload:
     seed: int = 0
 
 
-# The five workloads of the build (sizes and distributions as stated for each).
+# The five benchmark workloads (sizes and distributions as stated for each).
 WORKLOADS = {
     1: Workload("deltanet_fwd_f32_B1_T256_H2_d64", DELTANET, "f32", 1, 256, 2, 64, 64, seed=1001),
     2: Workload("gdn_bf16_B8_T4096_H8_d128", GATED, "bf16", 8, 4096, 8, 128, 128, seed=1002),

@@ -18,7 +18,7 @@ RMSNorm of the attention output), per (token, head) row of dv channels:
     n = o / sqrt(mean(o^2) + eps),   y = n * w * sigmoid(g)
 with a per-channel weight w and the gate logits g given by the caller.
 
-eps = 1e-6 in both (the pages give none).  The backward functions return the gradients of
+eps = 1e-6 in both (the method's description gives no value).  The backward functions return the gradients of
 L = sum(dy * y) (post) or of L = <dq_hat, q_hat> + <dk_hat, k_hat> + <dbeta, beta> +
 <dloga, log alpha> (pre) with respect to every input.
 """

@@ -35,7 +35,7 @@ def test_logistic_gate_symmetries():
     assert np.all(out_p["loga"] < 0) and np.all((out_p["beta"] > 0) & (out_p["beta"] < 1))
     z = pp.preop_fwd(np.ones((1, 4)), np.ones((1, 4)), np.zeros(1), np.zeros(1))
     assert z["beta"][0] == 0.5 and abs(z["loga"][0] + np.log(2.0)) < 1e-15
-    # a forget logit of -3 keeps about 95 % of the state per token (the -3 bias of the pages)
+    # a forget logit of -3 keeps about 95 % of the state per token (the -3 forget-gate bias of the Kimi Delta Attention page, section 7.1)
     assert abs(np.exp(pp.preop_fwd(np.ones((1, 4)), np.ones((1, 4)), np.zeros(1), np.array([-3.0]))["loga"][0])
                - 1 / (1 + np.exp(-3.0))) < 1e-15
     # extreme logits stay finite
