@@ -41,7 +41,7 @@ EXPORTS = ("delta_rule_workspace_size", "delta_rule_fwd", "delta_rule_bwd", "del
            "delta_rule_fwd_noalloc", "delta_rule_saved_size", "delta_rule_fwd_save", "delta_rule_bwd_saved",
            "delta_rule_fwd_save_timed", "delta_rule_bwd_saved_timed", "delta_rule_decode",
            "delta_rule_preop", "delta_rule_preop_bwd", "delta_rule_postop_workspace_size", "delta_rule_postop",
-           "delta_rule_postop_bwd")
+           "delta_rule_postop_bwd", "delta_rule_selftest_timeout")
 
 _lib = None
 
@@ -97,6 +97,8 @@ def load(path: str | None = None):
     lib.delta_rule_postop.restype = i
     lib.delta_rule_postop_bwd.argtypes = [vp] * 7 + [i] * 5 + [vp, sz, vp]
     lib.delta_rule_postop_bwd.restype = i
+    lib.delta_rule_selftest_timeout.argtypes = [ctypes.c_uint, vp]
+    lib.delta_rule_selftest_timeout.restype = i
     lib.delta_rule_decode.argtypes = [vp] * 9 + [i] * 7 + [vp]
     lib.delta_rule_decode.restype = i
     lib.delta_rule_fwd_save_timed.argtypes = [vp] * 9 + [i] * 8 + [vp, sz, vp, sz, vp, ctypes.POINTER(vp), i]
@@ -235,6 +237,11 @@ def delta_rule_fwd(q, k, v, alpha, beta, S0=None, variant="gdn", chunk=64, want_
                  B, T, H, dk, dv, var, chunk, dt, _p(workspace), need, stream)
     _check(rc, "delta_rule_fwd")
     return out, u, S_T
+
+
+def selftest_timeout(limit_us: int, stream=None) -> int:
+    """Runs the bounded-wait self-test (see include/delta_rule.h); returns the launch status."""
+    return load().delta_rule_selftest_timeout(int(limit_us), stream)
 
 
 def decode_raw(*args) -> int:

@@ -11,6 +11,7 @@
 #include "dr_common.cuh"
 #include "simt_path.cuh"
 #include "tc_path.cuh"
+#include "tc_ptx.cuh"
 
 using namespace dr;
 
@@ -470,6 +471,26 @@ extern "C" int delta_rule_postop_bwd(const void *o, const void *gate, const floa
     pp.q = o; pp.k = gate; pp.w = weight; pp.dq = dy; pp.qo = do_; pp.ko = dgate; pp.dw = dweight;
     pp.part = (float *)workspace; pp.rows = rows; pp.d = dv;
     return launch_status(postop_run(pp, dtype == DR_BF16, true, (cudaStream_t)stream));
+}
+
+// Self-test of the bounded waits: one thread waits for an mbarrier phase that nothing
+// completes; the wait gives up after limit_ns, raises the device error word and returns.
+__global__ void k_selftest_wait(unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bar, 1);
+        abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) tc::mbar_wait(&bar, 0, &abort_flag, limit_ns);
+}
+
+extern "C" int delta_rule_selftest_timeout(unsigned limit_us, void *stream) {
+    if (limit_us == 0 || limit_us > 1000000u) return DR_ERR_ARG;
+    k_selftest_wait<<<1, 32, 0, (cudaStream_t)stream>>>(1000ull * limit_us);
+    return launch_status(cudaGetLastError());
 }
 
 extern "C" const char *delta_rule_strerror(int code) {

@@ -273,6 +273,16 @@ int delta_rule_postop_bwd(const void *o, const void *gate, const float *weight, 
                           void *dgate, float *dweight, int B, int T, int H, int dv, int dtype, void *workspace,
                           size_t ws_bytes, void *stream);
 
+/*
+ * Self-test of failure detection.  Launches one kernel on `stream` whose bounded
+ * wait (the same wait every pipelined kernel uses) waits for a barrier phase that
+ * nothing completes; after limit_us microseconds (1 .. 1,000,000) it gives up,
+ * raises the device error word and returns, so that the next
+ * delta_rule_sync_status() reports DR_ERR_TIMEOUT and the context stays usable.
+ * Returns DR_ERR_ARG for a limit out of range.
+ */
+int delta_rule_selftest_timeout(unsigned limit_us, void *stream);
+
 /* Static text for a DR_* code ("ok", "invalid argument", ...). */
 const char *delta_rule_strerror(int code);
 

@@ -165,3 +165,18 @@ def test_host_buffer_entry_point():
     o, u, S = binding.delta_rule_fwd_host(h["q"], h["k"], h["v"], h["loga"], h["beta"], None, variant="gdn")
     r = gpu_fwd(x, "gdn")
     assert torch.equal(o, r["o"].cpu()) and torch.equal(u, r["u"].cpu()) and torch.equal(S, r["S_T"].cpu())
+
+
+def test_bounded_wait_runs_out_reports_and_leaves_the_context_usable():
+    """A wait that nothing completes gives up after its limit and raises the error word;
+    the next call still works."""
+    import time
+    stream = torch.cuda.current_stream().cuda_stream
+    assert binding.selftest_timeout(0, stream) == binding.DR_ERR_ARG
+    t0 = time.perf_counter()
+    assert binding.selftest_timeout(20000, stream) == binding.DR_OK  # 20 ms
+    assert binding.sync_status(stream) == binding.DR_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 5.0
+    assert binding.sync_status(stream) == binding.DR_OK  # read and cleared
+    x = gen("gdn", "bf16", 1, 70, 2, 128, 128, seed=21)
+    compare_fwd(gpu_fwd(x, "gdn"), oracle_fwd(x, "gdn"), "bf16", what="after a timed-out wait")
