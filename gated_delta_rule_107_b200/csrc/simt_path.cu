@@ -651,8 +651,9 @@ static cudaError_t fwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaSt
     return cudaGetLastError();
 }
 
+// recompute: run the forward chain first (false: the forward's W, U~, G, P, S_n, U are in w)
 template <typename TI>
-static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaStream_t s, Rec &rec) {
+static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, bool recompute, cudaStream_t s, Rec &rec) {
     const IO<TI> io = io_of<TI>(t);
     const size_t C = g.C, DK = g.dk, DV = g.dv;
     const dim3 gc(g.N, g.H, g.B), gs(g.dv / JB, g.H, g.B);
@@ -662,7 +663,7 @@ static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaSt
     DR_TRY(prep_attr(k_scan_bwd<TI>, sm_sb));
     DR_TRY(prep_attr(k_bwd_state<TI>, sm_st));
     DR_TRY(prep_attr(k_bwd_intra<TI>, sm_in));
-    DR_TRY(forward_chain<TI>(g, io, w, t.S0, nullptr, 0, s, rec));
+    if (recompute) DR_TRY(forward_chain<TI>(g, io, w, t.S0, nullptr, 0, s, rec));
     rec.mark(s);
     k_scan_bwd<TI><<<gs, NT, sm_sb, s>>>(g, io, w, t.dS_T, t.dS0);
     DR_TRY(cudaGetLastError());
@@ -679,7 +680,11 @@ cudaError_t simt_fwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w,
 }
 
 cudaError_t simt_bwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec) {
-    return bf16 ? bwd_t<__nv_bfloat16>(g, t, w, s, rec) : bwd_t<float>(g, t, w, s, rec);
+    return bf16 ? bwd_t<__nv_bfloat16>(g, t, w, true, s, rec) : bwd_t<float>(g, t, w, true, s, rec);
+}
+
+cudaError_t simt_bwd_from_fwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec) {
+    return bf16 ? bwd_t<__nv_bfloat16>(g, t, w, false, s, rec) : bwd_t<float>(g, t, w, false, s, rec);
 }
 
 }  // namespace dr

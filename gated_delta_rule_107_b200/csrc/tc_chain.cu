@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
                 for (int p = 0; p < 2; ++p) {
                     tma_load_2d(st + FS_WQ + p * 16384, &mp.W, 64 * p, ci * C, &bar[B_FULL0 + s]);
                     if (KDA) {
-                        tma_load_2d(st + FS_WQ + p * 16384 + 8192, &mp.q, 64 * p, ci * C, &bar[B_FULL0 + s]);
+                        if (OUT) tma_load_2d(st + FS_WQ + p * 16384 + 8192, &mp.q, 64 * p, ci * C, &bar[B_FULL0 + s]);
                         tma_load_2d(st + FS_K + p * 8192, &mp.k, 64 * p, ci * C, &bar[B_FULL0 + s]);
                     } else {
                         if (OUT) tma_load_4d(st + FS_WQ + p * 16384 + 8192, &mp.q, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
@@ -617,7 +617,7 @@ cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, int mode
     FMaps mp;
     const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;
     const bool out = mode != 1, keep = mode != 0, kda = g.variant == VAR_KDA;
-    if (kda && mode != 0) return cudaErrorInvalidValue;
+    if (kda && mode == 2) return cudaErrorInvalidValue;  // no saved form for KDA
     bool ok = (kda ? tc::make_map_2d_bf16(&mp.q, w.Qt, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.k, w.Kb, DK, NC * C, 64)
                    : tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) &&
                          tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64)) &&
@@ -645,7 +645,7 @@ cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, int mode
         kern<<<grid, NTHREADS, smem, s>>>(mp, a);
         return cudaSuccess;
     };
-    if (kda) e = go(k_chain_fwd<0, 1>);
+    if (kda) e = mode == 0 ? go(k_chain_fwd<0, 1>) : go(k_chain_fwd<1, 1>);
     else if (mode == 0) e = go(k_chain_fwd<0, 0>);
     else if (mode == 1) e = go(k_chain_fwd<1, 0>);
     else e = go(k_chain_fwd<2, 0>);

@@ -57,13 +57,18 @@ size_t tc_ws_bytes(const Geo &g, int parts);
 // Sets the pointers of the given parts, carved from base in that order; leaves the others.
 void tc_ws_carve(const Geo &g, int parts, void *base, TcWs *w);
 
-// KDA's gate-scaled operands of every chunk (tc_prep.cu): w.Kt1 ... w.Kb, w.egc.
-cudaError_t tc_kda_gates(const Geo &g, const Tensors &t, const TcWs &w, cudaStream_t s, Rec &rec);
+// KDA's gate-scaled operands of every chunk (tc_prep.cu): w.Kt1 ... w.Kb, w.egc; with G
+// (fp32 [chunks][64][dk], may be null) also the in-chunk cumulative log gate itself.
+cudaError_t tc_kda_gates(const Geo &g, const Tensors &t, const TcWs &w, float *G, cudaStream_t s, Rec &rec);
+// fp32 copies of the forward's chunk products and states (W, U~, P, S_n, U) for the CUDA-core
+// backward kernels (tc_prep.cu).
+cudaError_t tc_to_simt(const Geo &g, const TcWs &w, float *W, float *Ut, float *P, float *Sn, float *Un, cudaStream_t s,
+                       Rec &rec);
 // Per-chunk products (tc_prep.cu): g and beta, W, U~, P; with keep also T and k k^T.
 // For KDA (no keep) from the operands of tc_kda_gates.
 cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool keep, cudaStream_t s, Rec &rec);
 // Forward state chain (tc_chain.cu).  mode 0: o, u, S_T; mode 1 (recompute for the
-// backward): S_n and U of every chunk; mode 2: both.  KDA: mode 0 only.
+// backward): S_n and U of every chunk; mode 2: both.
 cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, int mode, cudaStream_t s, Rec &rec);
 // Reverse state chain (tc_chain.cu): dS_{n+1} and dL/dU of every chunk (w.dSn, w.dUn), the
 // row sums w.skt, and dS0.

@@ -345,6 +345,7 @@ struct KdaArgs {
     const __nv_bfloat16 *q, *k, *alpha;
     __nv_bfloat16 *Kt1, *Qt1, *Kh, *Kt, *Qt, *Kb;
     float *egc;
+    float *G;  // optional: g itself, fp32 [chunks][64][128]
     int T, H, N;
 };
 
@@ -396,6 +397,14 @@ __global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
         if (tg == 7) gend[c0 + j] = g[7][j];           // token C - 1, the last
     }
     __syncthreads();
+    if (a.G) {
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            float *dst = a.G + (ci * C + 8 * tg + r) * DK + c0;
+            *reinterpret_cast<float4 *>(dst) = make_float4(g[r][0], g[r][1], g[r][2], g[r][3]);
+            *reinterpret_cast<float4 *>(dst + 4) = make_float4(g[r][4], g[r][5], g[r][6], g[r][7]);
+        }
+    }
     float gm[8], gC[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -448,14 +457,59 @@ static cudaError_t launch_prep(const Maps &mp, const Args &a, dim3 grid, cudaStr
 
 }  // namespace tcp
 
-cudaError_t tc_kda_gates(const Geo &g, const Tensors &t, const TcWs &w, cudaStream_t s, Rec &rec) {
+cudaError_t tc_kda_gates(const Geo &g, const Tensors &t, const TcWs &w, float *G, cudaStream_t s, Rec &rec) {
     using namespace tcp;
     KdaArgs a;
     a.q = (const __nv_bfloat16 *)t.q; a.k = (const __nv_bfloat16 *)t.k; a.alpha = (const __nv_bfloat16 *)t.alpha;
-    a.Kt1 = w.Kt1; a.Qt1 = w.Qt1; a.Kh = w.Kh; a.Kt = w.Kt; a.Qt = w.Qt; a.Kb = w.Kb; a.egc = w.egc;
+    a.Kt1 = w.Kt1; a.Qt1 = w.Qt1; a.Kh = w.Kh; a.Kt = w.Kt; a.Qt = w.Qt; a.Kb = w.Kb; a.egc = w.egc; a.G = G;
     a.T = g.T; a.H = g.H; a.N = g.N;
     rec.mark(s);
     k_kda_gates<<<dim3(g.N, g.H, g.B), DK, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+namespace tcp {
+// bf16 -> fp32 copies of up to five arrays (8 elements a thread, grid-stride)
+struct Widen {
+    const __nv_bfloat16 *src[5];
+    float *dst[5];
+    size_t n8[5];  // elements / 8
+};
+__global__ void __launch_bounds__(256) k_widen(Widen a) {
+    for (int i = 0; i < 5; ++i) {
+        if (!a.src[i]) continue;
+        for (size_t x = (size_t)blockIdx.x * 256 + threadIdx.x; x < a.n8[i]; x += (size_t)gridDim.x * 256) {
+            const uint4 v = reinterpret_cast<const uint4 *>(a.src[i])[x];
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            float f[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                f[2 * j] = __uint_as_float(w4[j] << 16);
+                f[2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
+            }
+            float4 *d = reinterpret_cast<float4 *>(a.dst[i] + 8 * x);
+            d[0] = make_float4(f[0], f[1], f[2], f[3]);
+            d[1] = make_float4(f[4], f[5], f[6], f[7]);
+        }
+    }
+}
+}  // namespace tcp
+
+cudaError_t tc_to_simt(const Geo &g, const TcWs &w, float *W, float *Ut, float *P, float *Sn, float *Un, cudaStream_t s,
+                       Rec &rec) {
+    using namespace tcp;
+    const size_t nc = (size_t)g.B * g.H * g.N;
+    Widen a = {};
+    const __nv_bfloat16 *src[5] = {w.W, w.Ut, w.P, w.Sn, w.Un};
+    float *dst[5] = {W, Ut, P, Sn, Un};
+    const size_t n[5] = {nc * C * DK, nc * C * DV, nc * C * C, nc * DK * DV, nc * C * DV};
+    for (int i = 0; i < 5; ++i) {
+        a.src[i] = src[i];
+        a.dst[i] = dst[i];
+        a.n8[i] = n[i] / 8;
+    }
+    rec.mark(s);
+    k_widen<<<148 * 8, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 
