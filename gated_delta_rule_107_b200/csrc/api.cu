@@ -50,8 +50,8 @@ bool use_split(const Geo &g, int dtype) { return tc_split_supported(g, dtype == 
 bool use_split_kda(const Geo &g, int dtype, int kind) {
     return !is_bwd(kind) && tc_split_kda_supported(g, dtype == DR_BF16);
 }
-// KDA's backward: the forward's products and states from the tensor-core kernels (widened
-// to fp32), then the CUDA-core reverse chain and gradient kernels
+// KDA's backward: the forward's products and states and the reverse chain from the
+// tensor-core kernels (widened to fp32), then the CUDA-core intra-chunk gradient kernels
 bool use_kda_hybrid_bwd(const Geo &g, int dtype, int kind) {
     return is_bwd(kind) && tc_split_kda_supported(g, dtype == DR_BF16);
 }
@@ -68,7 +68,8 @@ size_t ws_bytes(const Geo &g, int dtype, int kind) {
         }
     }
     if (use_split_kda(g, dtype, kind)) return tc_ws_bytes(g, WS_FWD | WS_KDA);
-    if (use_kda_hybrid_bwd(g, dtype, kind)) return ws_al(simt_ws_bytes(g, true)) + tc_ws_bytes(g, WS_FWD | WS_KEEP | WS_KDA);
+    if (use_kda_hybrid_bwd(g, dtype, kind))
+        return ws_al(simt_ws_bytes(g, true)) + tc_ws_bytes(g, WS_FWD | WS_KEEP | WS_REV | WS_KDA);
     if (!is_bwd(kind) && use_tc_fwd(g, dtype)) return 0;
     return simt_ws_bytes(g, is_bwd(kind));
 }
@@ -203,12 +204,14 @@ static int bwd_impl(const void *q, const void *k, const void *v, const void *alp
     } else if (use_kda_hybrid_bwd(g, dtype, kind)) {
         const SimtWs sw = simt_ws_carve(g, true, workspace);
         TcWs w = {};
-        tc_ws_carve(g, WS_FWD | WS_KEEP | WS_KDA, (char *)workspace + ws_al(simt_ws_bytes(g, true)), &w);
+        tc_ws_carve(g, WS_FWD | WS_KEEP | WS_REV | WS_KDA, (char *)workspace + ws_al(simt_ws_bytes(g, true)), &w);
         rc = launch_status(tc_kda_gates(g, t, w, sw.G, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_chunk_prep(g, t, w, false, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, 1, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_to_simt(g, w, sw.W, sw.Ut, sw.P, sw.Sn, sw.Un, s, rec));
-        if (rc == DR_OK) rc = launch_status(simt_bwd_from_fwd(g, t, dtype == DR_BF16, sw, s, rec));
+        if (rc == DR_OK) rc = launch_status(tc_chain_rev(g, t, w, s, rec));
+        if (rc == DR_OK) rc = launch_status(tc_rev_to_simt(g, w, sw.dSn, sw.dUn, s, rec));
+        if (rc == DR_OK) rc = launch_status(simt_bwd_grads(g, t, dtype == DR_BF16, sw, s, rec));
     } else {
         const SimtWs w = simt_ws_carve(g, true, workspace);
         rc = launch_status(simt_bwd(g, t, dtype == DR_BF16, w, s, rec));
@@ -225,8 +228,8 @@ static int launch_plan(const Geo &g, int dtype, int kind, const char **names, in
                                              "k_bwd_chunk_tc"};
     static const char *const SPLIT_BWD_SAVED[2] = {"k_chain_rev", "k_bwd_chunk_tc"};
     static const char *const SPLIT_KDA_FWD[3] = {"k_kda_gates", "k_chunk_prep", "k_chain_fwd"};
-    static const char *const KDA_BWD[7] = {"k_kda_gates", "k_chunk_prep", "k_chain_fwd(recompute)", "k_widen",
-                                           "k_scan_bwd", "k_bwd_state", "k_bwd_intra"};
+    static const char *const KDA_BWD[8] = {"k_kda_gates", "k_chunk_prep", "k_chain_fwd(recompute)", "k_widen",
+                                           "k_chain_rev", "k_widen", "k_bwd_state", "k_bwd_intra"};
     int n = 0;
     const char *const *src = nullptr;
     if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
@@ -242,7 +245,7 @@ static int launch_plan(const Geo &g, int dtype, int kind, const char **names, in
         n = 3;
     } else if (use_kda_hybrid_bwd(g, dtype, kind)) {
         src = KDA_BWD;
-        n = 7;
+        n = 8;
     } else if (!is_bwd(kind) && use_tc_fwd(g, dtype)) {
         return tc_fwd_launches(g, names, max_names);
     } else {

@@ -651,9 +651,10 @@ static cudaError_t fwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaSt
     return cudaGetLastError();
 }
 
-// recompute: run the forward chain first (false: the forward's W, U~, G, P, S_n, U are in w)
+// from = 0: everything; 1: the forward's W, U~, G, P, S_n, U are in w already; 2: so are the
+// reverse chain's dS_{n+1} and dU (and dS0 is written)
 template <typename TI>
-static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, bool recompute, cudaStream_t s, Rec &rec) {
+static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, int from, cudaStream_t s, Rec &rec) {
     const IO<TI> io = io_of<TI>(t);
     const size_t C = g.C, DK = g.dk, DV = g.dv;
     const dim3 gc(g.N, g.H, g.B), gs(g.dv / JB, g.H, g.B);
@@ -663,10 +664,12 @@ static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, bool r
     DR_TRY(prep_attr(k_scan_bwd<TI>, sm_sb));
     DR_TRY(prep_attr(k_bwd_state<TI>, sm_st));
     DR_TRY(prep_attr(k_bwd_intra<TI>, sm_in));
-    if (recompute) DR_TRY(forward_chain<TI>(g, io, w, t.S0, nullptr, 0, s, rec));
-    rec.mark(s);
-    k_scan_bwd<TI><<<gs, NT, sm_sb, s>>>(g, io, w, t.dS_T, t.dS0);
-    DR_TRY(cudaGetLastError());
+    if (from == 0) DR_TRY(forward_chain<TI>(g, io, w, t.S0, nullptr, 0, s, rec));
+    if (from < 2) {
+        rec.mark(s);
+        k_scan_bwd<TI><<<gs, NT, sm_sb, s>>>(g, io, w, t.dS_T, t.dS0);
+        DR_TRY(cudaGetLastError());
+    }
     rec.mark(s);
     k_bwd_state<TI><<<gc, NT, sm_st, s>>>(g, io, w);
     DR_TRY(cudaGetLastError());
@@ -680,11 +683,11 @@ cudaError_t simt_fwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w,
 }
 
 cudaError_t simt_bwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec) {
-    return bf16 ? bwd_t<__nv_bfloat16>(g, t, w, true, s, rec) : bwd_t<float>(g, t, w, true, s, rec);
+    return bf16 ? bwd_t<__nv_bfloat16>(g, t, w, 0, s, rec) : bwd_t<float>(g, t, w, 0, s, rec);
 }
 
-cudaError_t simt_bwd_from_fwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec) {
-    return bf16 ? bwd_t<__nv_bfloat16>(g, t, w, false, s, rec) : bwd_t<float>(g, t, w, false, s, rec);
+cudaError_t simt_bwd_grads(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec) {
+    return bf16 ? bwd_t<__nv_bfloat16>(g, t, w, 2, s, rec) : bwd_t<float>(g, t, w, 2, s, rec);
 }
 
 }  // namespace dr

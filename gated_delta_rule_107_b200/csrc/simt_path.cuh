@@ -25,9 +25,9 @@ size_t simt_ws_bytes(const Geo &g, bool bwd);
 SimtWs simt_ws_carve(const Geo &g, bool bwd, void *base);
 cudaError_t simt_fwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec);
 cudaError_t simt_bwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec);
-// The backward's last three kernels, for a w whose G, W, Ut, P, Sn, Un already hold the
-// forward's values (from the tensor-core forward kernels).
-cudaError_t simt_bwd_from_fwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec);
+// The backward's last two kernels (k_bwd_state, k_bwd_intra), for a w whose G, W, Ut, P, Sn,
+// Un hold the forward's values and dSn, dUn the reverse chain's (from tensor-core kernels).
+cudaError_t simt_bwd_grads(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec);
 // kernel names in launch order (for the timed entry points)
 extern const char *const SIMT_FWD_KERNELS[3];
 extern const char *const SIMT_BWD_KERNELS[5];

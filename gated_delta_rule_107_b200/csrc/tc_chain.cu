@@ -351,6 +351,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
 }
 
 // ====================================== reverse chain ======================================
+// KDA: q and k arrive gate-scaled (q e^g, k e^{g_C - g}, as in the forward), so the row
+// factors are 1 and dS decays by row.
+template <int KDA>
 __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant__ RMaps mp, Args a) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm =
@@ -390,8 +393,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
                 mbar_arrive_tx(&bar[B_FULL0 + s], 73728u + (a.has_du ? 8192u : 0u));
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
-                    tma_load_4d(st + RS_K + p * 8192, &mp.k, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
-                    tma_load_4d(st + RS_Q + p * 8192, &mp.q, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
+                    if (KDA) {
+                        tma_load_2d(st + RS_K + p * 8192, &mp.k, 64 * p, ci * C, &bar[B_FULL0 + s]);
+                        tma_load_2d(st + RS_Q + p * 8192, &mp.q, 64 * p, ci * C, &bar[B_FULL0 + s]);
+                    } else {
+                        tma_load_4d(st + RS_K + p * 8192, &mp.k, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
+                        tma_load_4d(st + RS_Q + p * 8192, &mp.q, 64 * p, h, t0, b, &bar[B_FULL0 + s]);
+                    }
                     tma_load_2d(st + RS_W + p * 8192, &mp.W, 64 * p, ci * C, &bar[B_FULL0 + s]);
                 }
                 tma_load_4d(st + RS_DO, &mp.dout, j0, h, t0, b, &bar[B_FULL0 + s]);
@@ -399,7 +407,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
                 if (a.has_du) tma_load_4d(st + RS_DX, &mp.du, j0, h, t0, b, &bar[B_FULL0 + s]);
                 tma_load_2d(st + RS_UN, &mp.Un, j0, ci * C, &bar[B_FULL0 + s]);
             }
-            chunk_factors(a.gb, (size_t)ci, cf_all + s * 132, lane);
+            if (KDA) chunk_factors_kda(a.egc, (size_t)ci, cf_all + s * 132, lane);
+            else chunk_factors(a.gb, (size_t)ci, cf_all + s * 132, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[B_FULL0 + s]);
             issued[s]++;
@@ -444,7 +453,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
             const bool got = mbar_wait(&bar[B_FULL0 + s], (m >> 1) & 1, abort_flag);
             if (wabort(got)) break;
             const float *cf = cf_all + s * 132;
-            const float egC = cf[128];
+            const float egC = KDA ? cf[trow] : cf[128];  // KDA: this thread's state row decays by its channel
             // ------- D_a = k dS+, D_p = P^T dO  (M = 128: rows 64..127 discarded) -------
             if (wc == 0) {
                 fence_after_sync();
@@ -468,7 +477,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
             // ---------------- dU = du + P^T dO + diag(e^{gC - g}) D_a;  U_r . (Kbar dS+)_r ----------------
             if (trow < 64) {
                 const int r = trow;
-                const float f = cf[r];
+                const float f = KDA ? 1.f : cf[r];
                 float v[32], pd[32], rs = 0.f;
                 tmem_row32(tl + TM_A, v);
                 tmem_row32(tl + TM_P, pd);
@@ -493,7 +502,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
                     st_chunk(sm + OFF_U, o, d);
                 }
                 skp[hf * 64 + r] = rs;
-            } else {
+            } else if (!KDA) {
                 // lanes 64-127: q rows scaled by e^{g_r} (for q^T diag(e^g) dO)
                 for (int x = (cl.q4 - 2) * 32 + lane + hf * 64; x < 1024; x += 128) {  // 128 threads
                     float v[8];
@@ -657,8 +666,10 @@ cudaError_t tc_chain_rev(const Geo &g, const Tensors &t, const TcWs &w, cudaStre
     using namespace tch;
     RMaps mp;
     const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;
-    const bool ok = tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) &&
-                    tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64) &&
+    const bool kda = g.variant == VAR_KDA;
+    const bool ok = (kda ? tc::make_map_2d_bf16(&mp.q, w.Qt, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.k, w.Kb, DK, NC * C, 64)
+                         : tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) &&
+                               tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64)) &&
                     tc::make_map_4d_bf16(&mp.dout, t.dout, DV, H, T, Bn, 64) &&
                     tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.P, w.P, C, NC * C, 64) &&
                     tc::make_map_2d_bf16(&mp.Un, w.Un, DV, NC * C, 64) && tc::make_map_2d_bf16(&mp.dUn, w.dUn, DV, NC * C, 64) &&
@@ -667,13 +678,16 @@ cudaError_t tc_chain_rev(const Geo &g, const Tensors &t, const TcWs &w, cudaStre
     if (!ok) return cudaErrorInvalidValue;
     Args a = {};
     a.gb = w.gb; a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
-    a.S0 = t.dS_T; a.ST = t.dS0; a.skt = w.skt; a.has_du = t.du != nullptr;
+    a.S0 = t.dS_T; a.ST = t.dS0; a.skt = w.skt; a.has_du = t.du != nullptr; a.egc = w.egc;
     const size_t smem = SMEM_BYTES + 1024;
-    cudaError_t e = cudaFuncSetAttribute(k_chain_rev, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    rec.mark(s);
-    k_chain_rev<<<dim3(DV / DVB, g.H, g.B), NTHREADS, smem, s>>>(mp, a);
-    return cudaGetLastError();
+    auto go = [&](auto kern) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        rec.mark(s);
+        kern<<<dim3(DV / DVB, g.H, g.B), NTHREADS, smem, s>>>(mp, a);
+        return cudaGetLastError();
+    };
+    return kda ? go(k_chain_rev<1>) : go(k_chain_rev<0>);
 }
 
 }  // namespace dr

@@ -64,6 +64,8 @@ cudaError_t tc_kda_gates(const Geo &g, const Tensors &t, const TcWs &w, float *G
 // backward kernels (tc_prep.cu).
 cudaError_t tc_to_simt(const Geo &g, const TcWs &w, float *W, float *Ut, float *P, float *Sn, float *Un, cudaStream_t s,
                        Rec &rec);
+// fp32 copies of the reverse chain's dS_{n+1} and dL/dU (tc_prep.cu).
+cudaError_t tc_rev_to_simt(const Geo &g, const TcWs &w, float *dSn, float *dUn, cudaStream_t s, Rec &rec);
 // Per-chunk products (tc_prep.cu): g and beta, W, U~, P; with keep also T and k k^T.
 // For KDA (no keep) from the operands of tc_kda_gates.
 cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool keep, cudaStream_t s, Rec &rec);
@@ -71,7 +73,7 @@ cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool ke
 // backward): S_n and U of every chunk; mode 2: both.
 cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, int mode, cudaStream_t s, Rec &rec);
 // Reverse state chain (tc_chain.cu): dS_{n+1} and dL/dU of every chunk (w.dSn, w.dUn), the
-// row sums w.skt, and dS0.
+// row sums w.skt, and dS0.  KDA reads the forward's gate-scaled q and k from w.
 cudaError_t tc_chain_rev(const Geo &g, const Tensors &t, const TcWs &w, cudaStream_t s, Rec &rec);
 // All intra-chunk gradients (tc_bwd.cu): dq, dk, dv, dbeta, d log alpha.
 cudaError_t tc_bwd_chunk(const Geo &g, const Tensors &t, const TcWs &w, cudaStream_t s, Rec &rec);

@@ -513,6 +513,17 @@ cudaError_t tc_to_simt(const Geo &g, const TcWs &w, float *W, float *Ut, float *
     return cudaGetLastError();
 }
 
+cudaError_t tc_rev_to_simt(const Geo &g, const TcWs &w, float *dSn, float *dUn, cudaStream_t s, Rec &rec) {
+    using namespace tcp;
+    const size_t nc = (size_t)g.B * g.H * g.N;
+    Widen a = {};
+    a.src[0] = w.dSn; a.dst[0] = dSn; a.n8[0] = nc * DK * DV / 8;
+    a.src[1] = w.dUn; a.dst[1] = dUn; a.n8[1] = nc * C * DV / 8;
+    rec.mark(s);
+    k_widen<<<148 * 8, 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
 cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool keep, cudaStream_t s, Rec &rec) {
     using namespace tcp;
     Maps mp;
