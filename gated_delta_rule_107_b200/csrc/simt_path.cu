@@ -431,8 +431,11 @@ __global__ void __launch_bounds__(NT) k_bwd_intra(Geo g, IO<TI> io, SimtWs w) {
         }
     }
     __syncthreads();
-    // dA, dM = beta dA, dbeta (A part), dP
-    {
+    // dA = -strict_tril([dB_k | dB_v] [W | U~]^T), dM = diag(beta) dA, dbeta (A part), and
+    // dP = tril(dO U^T).  At C = 64: two 64 x 64 products, tiled through shared memory (the
+    // dM | dP region, written only at the end) in steps of K; thread t owns rows 4 (t / 16) ..
+    // + 3 and columns 4 (t % 16) .. + 3 of both results.  Smaller chunks: one warp per row.
+    if (C != 64) {
         const float *Wg = w.W + ci * C * DK, *Ug = w.Ut + ci * C * DV, *Un = w.Un + ci * C * DV;
         for (int r = warp; r < C; r += NT / 32) {
             float db = 0.f;
@@ -455,6 +458,77 @@ __global__ void __launch_bounds__(NT) k_bwd_intra(Geo g, IO<TI> io, SimtWs w) {
                 }
             }
             if (lane == 0) dbs[r] += db;
+        }
+    } else {
+        static_assert(NT == 256, "4 x 4 blocks of a 64 x 64 result");
+        const float *Wg = w.W + ci * C * DK, *Ug = w.Ut + ci * C * DV, *Un = w.Un + ci * C * DV;
+        float *stg = dM;  // 2 C C floats of staging
+        const int r0 = 4 * (tid >> 4), i0 = 4 * (tid & 15);
+        float da[4][4] = {}, dp[4][4] = {};
+        // [dB_k | dB_v] (Y, already in shared memory) times [W | U~]^T, K = dk + dv in steps of 64
+        constexpr int LD = 65;  // padded row stride of a staged 64 x 64 tile
+        for (int k0 = 0; k0 < DY; k0 += 64) {
+            __syncthreads();
+            const float *src = k0 < DK ? Wg + k0 : Ug + (k0 - DK);
+            const int ld = k0 < DK ? DK : DV;
+            for (int x = tid; x < 64 * 64; x += NT) stg[(x >> 6) * LD + (x & 63)] = src[(x >> 6) * ld + (x & 63)];
+            __syncthreads();
+#pragma unroll 4
+            for (int kk = 0; kk < 64; ++kk) {
+                float av[4], bv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    av[u] = Y[(r0 + u) * DY + k0 + kk];
+                    bv[u] = stg[(i0 + u) * LD + kk];
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int v2 = 0; v2 < 4; ++v2) da[u][v2] += av[u] * bv[v2];
+            }
+        }
+        // dO U^T, K = dv in steps of 32 (dO rows past T and a missing dO are zero)
+        constexpr int LD2 = 33;
+        for (int k0 = 0; k0 < DV && io.dout; k0 += 32) {
+            __syncthreads();
+            float *so = stg, *su = stg + 64 * LD2;
+            for (int x = tid; x < 64 * 32; x += NT) {
+                const int r = x >> 5, j = x & 31;
+                so[r * LD2 + j] = r < L ? to_f(io.dout[g.row(b, t0 + r, h) * DV + k0 + j]) : 0.f;
+                su[r * LD2 + j] = Un[r * DV + k0 + j];
+            }
+            __syncthreads();
+#pragma unroll 4
+            for (int kk = 0; kk < 32; ++kk) {
+                float av[4], bv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    av[u] = so[(r0 + u) * LD2 + kk];
+                    bv[u] = su[(i0 + u) * LD2 + kk];
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int v2 = 0; v2 < 4; ++v2) dp[u][v2] += av[u] * bv[v2];
+            }
+        }
+        __syncthreads();  // the staging region becomes dM | dP
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int r = r0 + u;
+            float db = 0.f;
+#pragma unroll
+            for (int v2 = 0; v2 < 4; ++v2) {
+                const int i = i0 + v2;
+                const float a2 = i < r ? -da[u][v2] : 0.f;
+                db += a2 * M[r * C + i];
+                dM[r * C + i] = bs[r] * a2;
+                dP[r * C + i] = i <= r ? dp[u][v2] : 0.f;
+            }
+            // the 16 threads of row block r0 / 4 are lanes 0-15 or 16-31 of one warp
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) db += __shfl_xor_sync(0xffffffffu, db, o);
+            if ((tid & 15) == 0) dbs[r] += db;
         }
     }
     __syncthreads();
