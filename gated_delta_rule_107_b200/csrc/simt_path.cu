@@ -16,7 +16,10 @@
 //   S+    = Diag(e^{g_C}) S + (K .* e^{g_C - g})^T U
 //
 // Every exponent above is of a non-positive number when log alpha <= 0, so no
-// intermediate can overflow (no e^{-g} factorisation is used on this path).
+// intermediate can overflow.  The one split exponential is in the backward at C = 64:
+// e^{g_r - g_i} = e^{g_r - m} e^{m - g_i} around a midpoint m of the chunk's gates, used
+// only where every channel's gates span at most 120 nats in that chunk (each factor within
+// e^{+-60}); other chunks take the direct form.
 //
 // Kernels (one CTA of 256 threads each):
 //   k_prep        grid (N, H, B)     g, A, P, then W and U~ by forward substitution
@@ -311,9 +314,10 @@ __global__ void __launch_bounds__(NT) k_scan_bwd(Geo g, IO<TI> io, SimtWs w, con
 // ---------------------------------------------------------------------------------------------
 // k_bwd_state: the chunk's products with S_n and dS_{n+1}:
 //   Qd = dO S^T,  dWm = -dU S^T,  Tm = U dS+^T  ([C][dk] each),  RS = rowsum(S .* dS+)  ([dk])
+// The direct form, for chunk lengths below 64: one output per thread and step.
 // smem: Qd, dWm, Tm [C][dk]; Sb, dSb [dk][JB+1]; dOb, dUb, Ub [C][JB]; rs [dk]
 template <typename TI>
-__global__ void __launch_bounds__(NT) k_bwd_state(Geo g, IO<TI> io, SimtWs w) {
+__device__ __forceinline__ void state_direct(const Geo &g, const IO<TI> &io, const SimtWs &w) {
     const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int C = g.C, DK = g.dk, DV = g.dv;
     const int t0 = n * C, L = min(C, g.T - t0);
@@ -367,6 +371,132 @@ __global__ void __launch_bounds__(NT) k_bwd_state(Geo g, IO<TI> io, SimtWs w) {
     for (int c = tid; c < DK; c += NT) w.RS[ci * DK + c] = rs[c];
 }
 
+// cp.async (4-byte) copies, global to shared, in commit groups
+__device__ __forceinline__ void cp_async4(float *dst, const float *src) {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
+
+// At C = 64: thread t keeps a 4 x (dk / 16) block of all three products in registers (rows
+// 4 (t / 16) .. + 3, columns t % 16 + 16 v), and dv passes through shared memory JB columns at a
+// time, double-buffered: the next block's fp32 operands are copied asynchronously (and its dO
+// rows loaded into registers) while the current block is multiplied.
+// smem, two stages of: Sb, dSb [dk][JB+1]; dOb, dUb, Ub [64][JB+1]
+template <typename TI, int DK>
+__device__ __forceinline__ void state_tiled(const Geo &g, const IO<TI> &io, const SimtWs &w) {
+    constexpr int C = 64, CW = DK / 16, LD = JB + 1, STG = (2 * DK + 3 * C) * LD, PO = C * JB / NT;
+    static_assert(NT == 256, "16 x 16 thread blocks");
+    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int DV = g.dv, t0 = n * C, L = min(C, g.T - t0), R = DV / JB;
+    extern __shared__ float sm[];
+    const int tid = threadIdx.x;
+    const size_t ci = g.chunk(b, h, n);
+    const int r0 = 4 * (tid >> 4), cb = tid & 15;
+    auto issue = [&](int it, float *st) {
+        const int jb = it * JB;
+        float *Sb = st, *dSb = Sb + DK * LD, *dUb = dSb + DK * LD + C * LD, *Ub = dUb + C * LD;
+        for (int x = tid; x < DK * JB; x += NT) {
+            const int c = x / JB, j = x % JB;
+            const size_t src = ci * DK * DV + (size_t)c * DV + jb + j;
+            cp_async4(Sb + c * LD + j, w.Sn + src);
+            cp_async4(dSb + c * LD + j, w.dSn + src);
+        }
+        for (int x = tid; x < C * JB; x += NT) {
+            const int r = x / JB, j = x % JB;
+            const size_t src = (ci * C + r) * DV + jb + j;
+            cp_async4(dUb + r * LD + j, w.dUn + src);
+            cp_async4(Ub + r * LD + j, w.Un + src);
+        }
+    };
+    float od[PO];
+    auto fetch_do = [&](int it) {
+#pragma unroll
+        for (int e = 0; e < PO; ++e) {
+            const int x = tid + e * NT, r = x / JB, j = x % JB;
+            od[e] = io.dout ? to_f(io.dout[g.row(b, t0 + min(r, L - 1), h) * DV + it * JB + j]) : 0.f;
+        }
+    };
+    auto store_do = [&](float *st) {
+        float *dOb = st + 2 * DK * LD;
+#pragma unroll
+        for (int e = 0; e < PO; ++e) {
+            const int x = tid + e * NT, r = x / JB, j = x % JB;
+            dOb[r * LD + j] = r < L ? od[e] : 0.f;
+        }
+    };
+    float qd[4][CW], dw[4][CW], tm[4][CW];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < CW; ++v) qd[u][v] = dw[u][v] = tm[u][v] = 0.f;
+    float rs = 0.f;
+    issue(0, sm);
+    cp_async_commit();
+    fetch_do(0);
+    store_do(sm);
+    for (int it = 0; it < R; ++it) {
+        float *cur = sm + (it & 1) * STG, *oth = sm + ((it + 1) & 1) * STG;
+        if (it + 1 < R) {
+            issue(it + 1, oth);
+            fetch_do(it + 1);
+        }
+        cp_async_commit();
+        cp_async_wait1();  // all groups but the newest: block it has landed
+        __syncthreads();
+        const float *Sb = cur, *dSb = Sb + DK * LD, *dOb = dSb + DK * LD, *dUb = dOb + C * LD, *Ub = dUb + C * LD;
+#pragma unroll 2
+        for (int j = 0; j < JB; ++j) {
+            float ao[4], ad[4], au[4], bS[CW], bD[CW];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                ao[u] = dOb[(r0 + u) * LD + j];
+                ad[u] = dUb[(r0 + u) * LD + j];
+                au[u] = Ub[(r0 + u) * LD + j];
+            }
+#pragma unroll
+            for (int v = 0; v < CW; ++v) {
+                bS[v] = Sb[(cb + 16 * v) * LD + j];
+                bD[v] = dSb[(cb + 16 * v) * LD + j];
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < CW; ++v) {
+                    qd[u][v] += ao[u] * bS[v];
+                    dw[u][v] += ad[u] * bS[v];
+                    tm[u][v] += au[u] * bD[v];
+                }
+        }
+        if (tid < DK)
+            for (int j = 0; j < JB; ++j) rs += Sb[tid * LD + j] * dSb[tid * LD + j];
+        if (it + 1 < R) store_do(oth);
+        __syncthreads();  // the current stage is refilled next
+    }
+    const size_t base = ci * C * DK;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < CW; ++v) {
+            const size_t x = base + (size_t)(r0 + u) * DK + cb + 16 * v;
+            w.Qd[x] = qd[u][v];
+            w.dWm[x] = -dw[u][v];
+            w.Tm[x] = tm[u][v];
+        }
+    if (tid < DK) w.RS[ci * DK + tid] = rs;
+}
+
+template <typename TI>
+__global__ void __launch_bounds__(NT) k_bwd_state(Geo g, IO<TI> io, SimtWs w) {
+    if (g.C == 64) {
+        if (g.dk == 128) state_tiled<TI, 128>(g, io, w);
+        else state_tiled<TI, 64>(g, io, w);
+    } else {
+        state_direct<TI>(g, io, w);
+    }
+}
+
 // ---------------------------------------------------------------------------------------------
 // k_bwd_intra: all remaining gradients of one chunk.
 //   [dB_k | dB_v] = (I+A)^-T [dW | dU]                         (back substitution)
@@ -374,9 +504,12 @@ __global__ void __launch_bounds__(NT) k_bwd_state(Geo g, IO<TI> io, SimtWs w) {
 //   dP_ri = dO_r . U_i  (i<=r)
 //   then the gradients through e^{g} q, e^{g} k, k e^{-g} pairs, k e^{g_C - g}, e^{g_C},
 //   beta, and the reverse in-chunk cumsum of dg into d log alpha.
+// This direct form takes one exponential per (row, pair, channel) and serves every chunk length;
+// at C = 64 it runs only for KDA chunks whose gates span more than the factorised form below
+// accepts.
 // smem: ks, qs, gs [C][dk]; Y [C][dk+dv]; M, dM, dP [C][C]; bs, dbs, red [C]
 template <typename TI>
-__global__ void __launch_bounds__(NT) k_bwd_intra(Geo g, IO<TI> io, SimtWs w) {
+__device__ __forceinline__ void intra_direct(const Geo &g, const IO<TI> &io, const SimtWs &w) {
     const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int C = g.C, DK = g.dk, DV = g.dv, DY = g.dk + g.dv;
     const int t0 = n * C, L = min(C, g.T - t0);
@@ -640,6 +773,446 @@ __global__ void __launch_bounds__(NT) k_bwd_intra(Geo g, IO<TI> io, SimtWs w) {
 }
 
 // ---------------------------------------------------------------------------------------------
+// The same gradients at C = 64, with every per-(row, channel) sum written as a matrix product.
+// KDA's pair factor is split at a per-channel midpoint m_c of the chunk's gates,
+//   e^{g_rc - g_ic} = e^{g_rc - m_c} e^{m_c - g_ic},
+// so that with Kp = k e^{g - m}, Km = k e^{m - g}, Qp = q e^{g - m}:
+//   M  = strict_tril(Kp Km^T)
+//   X  = e^{g - m} .* (dP Km),   Yv = e^{g - m} .* (dM Km)
+//   Z  = e^{m - g} .* (dM^T Kp + dP^T Qp)
+// It serves a chunk only when every channel's gates there span at most RANGE_MAX, so that every
+// factor lies within e^{+-RANGE_MAX/2} and each product equals the direct sum up to rounding.
+// The scalar gates fold their pair factor into M, dM and dP instead (Kp = Km = k, Qp = q).  The
+// back substitution through (I+A)^T runs right-looking with one column of [dW | dU] in registers.
+// smem: Kp, Km, Qp [64][dk]; Y [64][dk+dv]; M, dM, dP [64][LDC]; bs, dbs, red, grow [64]; gm [dk]
+static constexpr int LDC = 68;             // padded row stride of the 64 x 64 matrices
+static constexpr float RANGE_MAX = 120.f;  // widest in-chunk gate span of a channel (nats)
+
+__host__ __device__ constexpr int tiled_gm_offset(int dk, int dv) {
+    return 3 * 64 * dk + 64 * (dk + dv) + 3 * 64 * LDC + 4 * 64;
+}
+__device__ __forceinline__ float clamp_half_range(float x) {
+    return fminf(fmaxf(x, -0.5f * RANGE_MAX), 0.5f * RANGE_MAX);
+}
+
+// acc[u][v] += sum_{k < K1 + K2} A[(r0 + u) lda + k] B(k)[i0 + v]: one thread's 4 x 4 block of a
+// 64 x 64 product whose K columns come from B1 (ld1, K1 columns) and then B2 (ld2, K2 columns).
+// B passes through stg (64 x 65 floats) 64 columns at a time, the next block held in registers
+// while the current one is multiplied.  K1 and K2 are multiples of 64.  Opens with a barrier;
+// the caller synchronises before stg is written again.
+__device__ __forceinline__ void nt64(const float *A, int lda, const float *B1, int ld1, int K1, const float *B2,
+                                     int ld2, int K2, float *stg, int r0, int i0, float (&acc)[4][4]) {
+    constexpr int LD = 65, PER = 64 * 64 / NT;
+    const int K = K1 + K2;
+    float nxt[PER];
+    auto fetch = [&](int k0) {
+        const float *B = k0 < K1 ? B1 + k0 : B2 + (k0 - K1);
+        const int ldb = k0 < K1 ? ld1 : ld2;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const int x = threadIdx.x + e * NT;
+            nxt[e] = B[(size_t)(x >> 6) * ldb + (x & 63)];
+        }
+    };
+    fetch(0);
+    for (int k0 = 0; k0 < K; k0 += 64) {
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const int x = threadIdx.x + e * NT;
+            stg[(x >> 6) * LD + (x & 63)] = nxt[e];
+        }
+        __syncthreads();
+        if (k0 + 64 < K) fetch(k0 + 64);
+#pragma unroll 4
+        for (int kk = 0; kk < 64; ++kk) {
+            float av[4], bv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                av[u] = A[(r0 + u) * lda + k0 + kk];
+                bv[u] = stg[(i0 + u) * LD + kk];
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < 4; ++v) acc[u][v] += av[u] * bv[v];
+        }
+    }
+}
+
+template <int N> __device__ __forceinline__ void ld4s(float (&d)[N], const float *p) {
+#pragma unroll
+    for (int v = 0; v < N; v += 4) {
+        const float4 t = *reinterpret_cast<const float4 *>(p + v);
+        d[v] = t.x; d[v + 1] = t.y; d[v + 2] = t.z; d[v + 3] = t.w;
+    }
+}
+
+template <typename TI, int DK, int DV>
+__device__ __forceinline__ void intra_tiled(const Geo &g, const IO<TI> &io, const SimtWs &w) {
+    constexpr int C = 64, DY = DK + DV, CW = DK / 16;
+    static_assert(NT == 256, "16 x 16 thread blocks over the 64 x 64 products");
+    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int t0 = n * C, L = min(C, g.T - t0);
+    extern __shared__ float sm[];
+    float *Kp = sm, *Km = Kp + C * DK, *Qp = Km + C * DK, *Y = Qp + C * DK;
+    float *M = Y + C * DY, *dM = M + C * LDC, *dP = dM + C * LDC;
+    float *bs = dP + C * LDC, *dbs = bs + C, *red = dbs + C, *grow = red + C, *gm = grow + C;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool kda = g.variant == VAR_KDA, gated = g.variant == VAR_GATED;
+    const size_t ci = g.chunk(b, h, n);
+    const float *Gg = w.G + ci * C * DK;
+
+    // loads in batches of 8 per thread, all issued before any is used
+#pragma unroll
+    for (int e0 = 0; e0 < C * DK / NT; e0 += 8) {
+        float kv[8], qv[8], gv[8], dw[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int x = tid + (e0 + e) * NT, r = x / DK, c = x % DK;
+            const size_t row = g.row(b, t0 + min(r, L - 1), h);
+            kv[e] = to_f(io.k[row * DK + c]);
+            qv[e] = to_f(io.q[row * DK + c]);
+            gv[e] = Gg[x];
+            dw[e] = w.dWm[ci * C * DK + x];
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int x = tid + (e0 + e) * NT, r = x / DK, c = x % DK;
+            const float k1 = r < L ? kv[e] : 0.f, q1 = r < L ? qv[e] : 0.f;
+            float ep = 1.f, em = 1.f;
+            if (kda) {
+                const float a = clamp_half_range(gv[e] - gm[c]);
+                ep = __expf(a);
+                em = __expf(-a);
+            }
+            Kp[x] = k1 * ep; Km[x] = k1 * em; Qp[x] = q1 * ep;
+            Y[r * DY + c] = dw[e];
+        }
+    }
+#pragma unroll
+    for (int e0 = 0; e0 < C * DV / NT; e0 += 8) {
+        float du[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) du[e] = w.dUn[ci * C * DV + tid + (e0 + e) * NT];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int x = tid + (e0 + e) * NT;
+            Y[(x / DV) * DY + DK + (x % DV)] = du[e];
+        }
+    }
+    for (int r = tid; r < C; r += NT) {
+        bs[r] = r < L ? to_f(io.beta[g.row(b, t0 + r, h)]) : 0.f;
+        dbs[r] = 0.f;
+        grow[r] = Gg[r * DK];
+    }
+    // 4 x 4 blocks of the 64 x 64 products: rows r0.., columns i0..
+    const int r0 = 4 * (tid >> 4), i0 = 4 * (tid & 15);
+    {
+        float acc[4][4] = {};
+        nt64(Kp, DK, Km, DK, DK, nullptr, 0, 0, dM, r0, i0, acc);  // its first barrier publishes the loads above
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int r = r0 + u, i = i0 + v;
+                float m = 0.f;
+                if (i < r) m = gated ? acc[u][v] * __expf(grow[r] - grow[i]) : acc[u][v];
+                M[r * LDC + i] = m;
+            }
+    }
+    __syncthreads();
+    // [dB_k | dB_v]_i = Y_i - sum_{r > i} beta_r M_ri [dB]_r: once row r is final it updates every
+    // row above it, so the 63 steps each carry up to 63 independent updates
+    if (tid < DY) {
+        float y[C];
+#pragma unroll
+        for (int r = 0; r < C; ++r) y[r] = Y[r * DY + tid];
+#pragma unroll
+        for (int r = C - 1; r >= 1; --r) {
+            const float t = bs[r] * y[r];
+#pragma unroll
+            for (int i = 0; i < r; i += 4) {
+                const float4 m4 = *reinterpret_cast<const float4 *>(M + r * LDC + i);
+                y[i] -= m4.x * t;
+                if (i + 1 < r) y[i + 1] -= m4.y * t;
+                if (i + 2 < r) y[i + 2] -= m4.z * t;
+                if (i + 3 < r) y[i + 3] -= m4.w * t;
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < C; ++r) Y[r * DY + tid] = y[r];
+    }
+    // dA = -strict_tril([dB_k | dB_v] [W | U~]^T), dM = diag(beta) dA, the A part of dbeta, and
+    // dP = tril(dO U^T)
+    {
+        const float *Wg = w.W + ci * C * DK, *Ug = w.Ut + ci * C * DV, *Un = w.Un + ci * C * DV;
+        float da[4][4] = {}, dp[4][4] = {};
+        nt64(Y, DY, Wg, DK, DK, Ug, DV, DV, dM, r0, i0, da);
+        constexpr int LD2 = 33, PER2 = 64 * 32 / NT;
+        float *so = dM, *su = dM + 64 * LD2;
+        float no[PER2], nu[PER2];
+        auto fetch2 = [&](int k0) {
+#pragma unroll
+            for (int e = 0; e < PER2; ++e) {
+                const int x = tid + e * NT, r = x >> 5, j = x & 31;
+                no[e] = to_f(io.dout[g.row(b, t0 + min(r, L - 1), h) * DV + k0 + j]);
+                nu[e] = Un[r * DV + k0 + j];
+            }
+        };
+        if (io.dout) fetch2(0);
+        for (int k0 = 0; k0 < DV && io.dout; k0 += 32) {
+            __syncthreads();
+#pragma unroll
+            for (int e = 0; e < PER2; ++e) {
+                const int x = tid + e * NT, r = x >> 5, j = x & 31;
+                so[r * LD2 + j] = r < L ? no[e] : 0.f;
+                su[r * LD2 + j] = nu[e];
+            }
+            __syncthreads();
+            if (k0 + 32 < DV) fetch2(k0 + 32);
+#pragma unroll 4
+            for (int kk = 0; kk < 32; ++kk) {
+                float av[4], bv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    av[u] = so[(r0 + u) * LD2 + kk];
+                    bv[u] = su[(i0 + u) * LD2 + kk];
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) dp[u][v] += av[u] * bv[v];
+            }
+        }
+        __syncthreads();  // the staging region becomes dM | dP
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int r = r0 + u;
+            float db = 0.f;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int i = i0 + v;
+                const float a2 = i < r ? -da[u][v] : 0.f;
+                db += a2 * M[r * LDC + i];
+                const float e = (gated && i <= r) ? __expf(grow[r] - grow[i]) : 1.f;
+                dM[r * LDC + i] = bs[r] * a2 * e;
+                dP[r * LDC + i] = i <= r ? dp[u][v] * e : 0.f;
+            }
+            // the 16 threads of one row block are lanes 0-15 or 16-31 of a warp
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) db += __shfl_xor_sync(0xffffffffu, db, o);
+            if ((tid & 15) == 0) dbs[r] += db;
+        }
+    }
+    __syncthreads();
+    // dv and the v part of dbeta, one warp per row
+#pragma unroll
+    for (int r = warp; r < C; r += NT / 32) {
+        float dbv = 0.f;
+        if (r < L) {
+            const size_t row = g.row(b, t0 + r, h);
+            float vv[DV / 32];
+#pragma unroll
+            for (int e = 0; e < DV / 32; ++e) vv[e] = to_f(io.v[row * DV + lane + 32 * e]);
+#pragma unroll
+            for (int e = 0; e < DV / 32; ++e) {
+                const float dBv = Y[r * DY + DK + lane + 32 * e];
+                dbv += dBv * vv[e];
+                io.dv[row * DV + lane + 32 * e] = from_f<TI>(bs[r] * dBv);
+            }
+        }
+        dbv = warp_sum(dbv);
+        if (lane == 0) dbs[r] += dbv;
+    }
+    // [64][dk] products: warp w owns the 8 rows of group rg (the two halves of the warp 4 each) and
+    // all dk columns, CW per lane.  dP and dM are lower triangular, so the first products stop at
+    // the group's last row and the transposed ones start at its first; warps w and w + 4 share a
+    // scheduler and get groups rg and 7 - rg, the same number of steps between them.
+    const int rg = warp < 4 ? warp : 11 - warp;
+    const int rb = 2 * rg + (lane >> 4), q0 = 4 * rb, c0 = CW * (lane & 15);
+    float *part = M;  // [16][dk] row-block sums of k e^{g_C - g} Tm (M is not read again)
+    const float *Qd = w.Qd + ci * C * DK, *Tm = w.Tm + ci * C * DK;
+    {
+        float X[4][CW], V[4][CW];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < CW; ++v) X[u][v] = V[u][v] = 0.f;
+        const int iend = 8 * rg + 8;
+        for (int i = 0; i < iend; ++i) {
+            float ap[4], am[4], bk[CW];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                ap[u] = dP[(q0 + u) * LDC + i];
+                am[u] = dM[(q0 + u) * LDC + i];
+            }
+            ld4s(bk, Km + i * DK + c0);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < CW; ++v) {
+                    X[u][v] += ap[u] * bk[v];
+                    V[u][v] += am[u] * bk[v];
+                }
+        }
+        __syncthreads();  // Km and M are overwritten below
+        float dgc[CW], gl[CW];
+        ld4s(gl, Gg + (C - 1) * DK + c0);
+#pragma unroll
+        for (int v = 0; v < CW; ++v) dgc[v] = 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int r = q0 + u;
+            const bool live = r < L;
+            const size_t row = g.row(b, t0 + min(r, L - 1), h);
+            float gr[CW], qdv[CW], tmv[CW], kr[CW], qr[CW];
+            ld4s(gr, Gg + r * DK + c0);
+            ld4s(qdv, Qd + r * DK + c0);
+            ld4s(tmv, Tm + r * DK + c0);
+#pragma unroll
+            for (int v = 0; v < CW; ++v) {
+                kr[v] = to_f(io.k[row * DK + c0 + v]);
+                qr[v] = to_f(io.q[row * DK + c0 + v]);
+            }
+            float dbk = 0.f;
+#pragma unroll
+            for (int v = 0; v < CW; ++v) {
+                const int c = c0 + v;
+                const float grc = gr[v], gam = __expf(grc), eb = __expf(gl[v] - grc);
+                const float kv = live ? kr[v] : 0.f, qv = live ? qr[v] : 0.f;
+                const float f = kda ? __expf(clamp_half_range(grc - gm[c])) : 1.f;
+                const float xs = X[u][v] * f, ys = V[u][v] * f;
+                const float dBk = Y[r * DY + c], et = eb * tmv[v];
+                const float dq = gam * qdv[v] + xs, sb = bs[r] * gam * dBk;
+                Km[r * DK + c] = ys + sb + et;                  // dk but for its Z term
+                Y[r * DY + c] = qv * dq + kv * (ys + sb - et);  // dg but for its -k Z term
+                dbk += kv * gam * dBk;
+                dgc[v] += kv * et;
+                if (live) io.dq[row * DK + c] = from_f<TI>(dq);
+            }
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) dbk += __shfl_xor_sync(0xffffffffu, dbk, o);
+            if ((lane & 15) == 0) dbs[r] += dbk;
+        }
+#pragma unroll
+        for (int v = 0; v < CW; ++v) part[rb * DK + c0 + v] = dgc[v];
+    }
+    {
+        float Z[4][CW];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < CW; ++v) Z[u][v] = 0.f;
+        for (int r2 = 8 * rg; r2 < C; ++r2) {
+            float am[4], ap[4], bk[CW], bq[CW];
+            ld4s(am, dM + r2 * LDC + q0);
+            ld4s(ap, dP + r2 * LDC + q0);
+            ld4s(bk, Kp + r2 * DK + c0);
+            ld4s(bq, Qp + r2 * DK + c0);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < CW; ++v) Z[u][v] += am[u] * bk[v] + ap[u] * bq[v];
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int r = q0 + u;
+            const bool live = r < L;
+            const size_t row = g.row(b, t0 + min(r, L - 1), h);
+            float gr[CW], kr[CW];
+            ld4s(gr, Gg + r * DK + c0);
+#pragma unroll
+            for (int v = 0; v < CW; ++v) kr[v] = to_f(io.k[row * DK + c0 + v]);
+#pragma unroll
+            for (int v = 0; v < CW; ++v) {
+                const int c = c0 + v;
+                const float f = kda ? __expf(clamp_half_range(gm[c] - gr[v])) : 1.f;
+                const float z = Z[u][v] * f;
+                const float kv = live ? kr[v] : 0.f;
+                if (live) io.dk[row * DK + c] = from_f<TI>(Km[r * DK + c] + z);
+                Y[r * DY + c] -= kv * z;
+            }
+        }
+    }
+    __syncthreads();
+    if (g.variant == VAR_DELTANET) {
+        for (int r = tid; r < L; r += NT) io.dbeta[g.row(b, t0 + r, h)] = from_f<TI>(dbs[r]);
+        return;
+    }
+    // dg_C: the K-bar . Tm sums and gamma_C rowsum(S .* dS+), added to the last row
+    for (int c = tid; c < DK; c += NT) {
+        float acc = __expf(Gg[(C - 1) * DK + c]) * w.RS[ci * DK + c];
+#pragma unroll
+        for (int p = 0; p < 16; ++p) acc += part[p * DK + c];
+        Y[(C - 1) * DY + c] += acc;
+    }
+    __syncthreads();
+    if (kda) {
+        for (int c = tid; c < DK; c += NT) {
+            float run = 0.f;
+            for (int r = C - 1; r >= 0; --r) {
+                run += Y[r * DY + c];
+                if (r < L) io.dalpha[g.row(b, t0 + r, h) * DK + c] = from_f<TI>(run);
+            }
+        }
+    } else {
+        for (int r = warp; r < C; r += NT / 32) {
+            float s = 0.f;
+            for (int c = lane; c < DK; c += 32) s += Y[r * DY + c];
+            s = warp_sum(s);
+            if (lane == 0) red[r] = s;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            float run = 0.f;
+            for (int r = C - 1; r >= 0; --r) {
+                run += red[r];
+                if (r < L) io.dalpha[g.row(b, t0 + r, h)] = from_f<TI>(run);
+            }
+        }
+    }
+    for (int r = tid; r < L; r += NT) io.dbeta[g.row(b, t0 + r, h)] = from_f<TI>(dbs[r]);
+}
+
+// One chunk per CTA.  At C = 64 a KDA chunk first finds each channel's midpoint and span; the
+// factorised form takes every chunk it accepts, the direct form the rest.
+template <typename TI>
+__global__ void __launch_bounds__(NT) k_bwd_intra(Geo g, IO<TI> io, SimtWs w) {
+    if (g.C == 64) {
+        int wide = 0;
+        if (g.variant == VAR_KDA) {
+            extern __shared__ float sm[];
+            float *gm = sm + tiled_gm_offset(g.dk, g.dv);
+            const int n = blockIdx.x, L = min(64, g.T - n * 64);
+            const float *Gg = w.G + g.chunk(blockIdx.z, blockIdx.y, n) * 64 * g.dk;
+            for (int c = threadIdx.x; c < g.dk; c += NT) {
+                float hi = Gg[c], lo = Gg[c];
+#pragma unroll 16
+                for (int r = 1; r < L; ++r) {
+                    const float v = Gg[r * g.dk + c];
+                    hi = fmaxf(hi, v);
+                    lo = fminf(lo, v);
+                }
+                gm[c] = 0.5f * (hi + lo);
+                if (!(hi - lo <= RANGE_MAX)) wide = 1;
+            }
+        }
+        if (!__syncthreads_or(wide)) {
+            if (g.dk == 128) {
+                if (g.dv == 128) intra_tiled<TI, 128, 128>(g, io, w);
+                else intra_tiled<TI, 128, 64>(g, io, w);
+            } else {
+                if (g.dv == 128) intra_tiled<TI, 64, 128>(g, io, w);
+                else intra_tiled<TI, 64, 64>(g, io, w);
+            }
+            return;
+        }
+    }
+    intra_direct<TI>(g, io, w);
+}
+
+// ---------------------------------------------------------------------------------------------
 // host side
 static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -733,8 +1306,11 @@ static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, int fr
     const size_t C = g.C, DK = g.dk, DV = g.dv;
     const dim3 gc(g.N, g.H, g.B), gs(g.dv / JB, g.H, g.B);
     const size_t sm_sb = 4 * (DK * JB + 3 * C * DK + C * C + 2 * C * JB + DK);
-    const size_t sm_st = 4 * (3 * C * DK + 2 * DK * (JB + 1) + 3 * C * JB + DK);
-    const size_t sm_in = 4 * (3 * C * DK + C * (DK + DV) + 3 * C * C + 3 * C);
+    const size_t sm_st = C == 64 ? 2 * 4 * (2 * DK + 3 * C) * (JB + 1)
+                                 : 4 * (3 * C * DK + 2 * DK * (JB + 1) + 3 * C * JB + DK);
+    size_t sm_in = 4 * (3 * C * DK + C * (DK + DV) + 3 * C * C + 3 * C);
+    const size_t sm_tiled = 4 * ((size_t)tiled_gm_offset((int)DK, (int)DV) + DK);
+    if (C == 64 && sm_tiled > sm_in) sm_in = sm_tiled;
     DR_TRY(prep_attr(k_scan_bwd<TI>, sm_sb));
     DR_TRY(prep_attr(k_bwd_state<TI>, sm_st));
     DR_TRY(prep_attr(k_bwd_intra<TI>, sm_in));

@@ -99,3 +99,12 @@ def test_backward_workloads_full_size_sampled_heads(wid, heads):
     for key, t in g.items():
         if t is not None:
             assert torch.isfinite(t).all(), f"{w.name} {key} not finite"
+
+
+def test_kda_bwd_fast_decay_channels_take_the_direct_form():
+    """Channels whose gates fall by 3 nats a token span 192 nats over a 64-token chunk, past what the
+    midpoint-split intra-chunk gradient accepts; such chunks take the direct form, while the ragged
+    last chunk (2 tokens) takes the split form, in one call (fp32, tight bar)."""
+    x = gen("kda", "f32", 1, 130, 2, 128, 128, seed=41, s0_std=0.1, grads=True)
+    x["loga"][..., :8] = -3.0
+    compare_bwd(gpu_bwd(x, "kda"), oracle_bwd(x, "kda"), "f32", "kda", what="kda fast-decay channels")
