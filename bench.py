@@ -403,6 +403,9 @@ def run_ours(args):
     post_w = torch.ones(dv, device=dev)
     post_ms = ev_time(lambda: binding.delta_rule_postop(o, u, post_w))
     post_b_ms = ev_time(lambda: binding.delta_rule_postop_bwd(o, u, post_w, x["dO"]))
+    conv_w = 0.5 * torch.randn(H * dk, 4, device=dev)
+    conv_ms = ev_time(lambda: binding.delta_rule_shortconv(x["q"], conv_w))
+    conv_b_ms = ev_time(lambda: binding.delta_rule_shortconv_bwd(x["q"], conv_w, x["q"]))
     if binding.sync_status() != binding.DR_OK:
         raise RuntimeError("device error word set during the pre/post leg")
     pre_unit = rows * elem * (2 * dk + 1 + gw_)  # q, k, beta, gate of every row once
@@ -415,7 +418,9 @@ def run_ours(args):
 
     prepost = {"shape": f"B{B} T{T} H{H} d{dk} bf16", "preop": gbs(2 * pre_unit, pre_ms),
                "preop_bwd": gbs(3 * pre_unit, pre_b_ms), "postop": gbs(post_bytes, post_ms),
-               "postop_bwd": gbs(rows * elem * 5 * dv, post_b_ms)}
+               "postop_bwd": gbs(rows * elem * 5 * dv, post_b_ms),
+               # one [B, T, H*dk] stream: x read, y written (backward: x, dy read, dx written)
+               "shortconv": gbs(2 * rows * elem * dk, conv_ms), "shortconv_bwd": gbs(3 * rows * elem * dk, conv_b_ms)}
 
     # ---- end to end through the public API with host buffers ----
     host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in x.items()}

@@ -25,6 +25,7 @@ The ``for_bwd`` argument of ``workspace_size`` and ``launches`` names the call:
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 
 import torch
@@ -41,7 +42,8 @@ EXPORTS = ("delta_rule_workspace_size", "delta_rule_fwd", "delta_rule_bwd", "del
            "delta_rule_fwd_noalloc", "delta_rule_saved_size", "delta_rule_fwd_save", "delta_rule_bwd_saved",
            "delta_rule_fwd_save_timed", "delta_rule_bwd_saved_timed", "delta_rule_decode",
            "delta_rule_preop", "delta_rule_preop_bwd", "delta_rule_postop_workspace_size", "delta_rule_postop",
-           "delta_rule_postop_bwd", "delta_rule_selftest_timeout")
+           "delta_rule_postop_bwd", "delta_rule_selftest_timeout", "delta_rule_shortconv_workspace_size",
+           "delta_rule_shortconv", "delta_rule_shortconv_bwd")
 
 _lib = None
 
@@ -97,6 +99,12 @@ def load(path: str | None = None):
     lib.delta_rule_postop.restype = i
     lib.delta_rule_postop_bwd.argtypes = [vp] * 7 + [i] * 5 + [vp, sz, vp]
     lib.delta_rule_postop_bwd.restype = i
+    lib.delta_rule_shortconv_workspace_size.argtypes = [i] * 3
+    lib.delta_rule_shortconv_workspace_size.restype = sz
+    lib.delta_rule_shortconv.argtypes = [vp] * 5 + [i] * 4 + [vp]
+    lib.delta_rule_shortconv.restype = i
+    lib.delta_rule_shortconv_bwd.argtypes = [vp] * 7 + [i] * 4 + [vp, sz, vp]
+    lib.delta_rule_shortconv_bwd.restype = i
     lib.delta_rule_selftest_timeout.argtypes = [ctypes.c_uint, vp]
     lib.delta_rule_selftest_timeout.restype = i
     lib.delta_rule_decode.argtypes = [vp] * 9 + [i] * 7 + [vp]
@@ -337,6 +345,45 @@ def delta_rule_postop_bwd(o, gate, weight, dy, want_dweight=True):
                         _p(ws), need, torch.cuda.current_stream(o.device).cuda_stream)
     _check(rc, "delta_rule_postop_bwd")
     return go, gg, gw
+
+
+def shortconv_raw(*args) -> int:
+    return load().delta_rule_shortconv(*args)
+
+
+def shortconv_bwd_raw(*args) -> int:
+    return load().delta_rule_shortconv_bwd(*args)
+
+
+def _stream_shape(x):
+    """(B, T, D) of a [B, T, D] or [B, T, H, d] stream."""
+    return x.shape[0], x.shape[1], math.prod(x.shape[2:])
+
+
+def delta_rule_shortconv(x, weight, x_prev=None, want_cache=False):
+    """Kernel-4 depthwise causal convolution along the tokens of x ([B, T, D] or [B, T, H, d]), taps
+    weight [D, 4] fp32.  Returns y, or (y, cache) with cache [B, 3, D] when want_cache."""
+    B, T, D = _stream_shape(x)
+    y = torch.empty_like(x)
+    cache = torch.empty((B, 3, D), dtype=x.dtype, device=x.device) if want_cache else None
+    rc = shortconv_raw(_p(x), _p(weight), _p(x_prev), _p(y), _p(cache), B, T, D, DTYPES[x.dtype],
+                       torch.cuda.current_stream(x.device).cuda_stream)
+    _check(rc, "delta_rule_shortconv")
+    return (y, cache) if want_cache else y
+
+
+def delta_rule_shortconv_bwd(x, weight, dy, x_prev=None, want_dweight=True, want_dprev=False):
+    """Returns (dx, dweight or None, dx_prev or None)."""
+    B, T, D = _stream_shape(x)
+    dx = torch.empty_like(x)
+    dw = torch.empty((D, 4), dtype=torch.float32, device=x.device) if want_dweight else None
+    dprev = torch.empty((B, 3, D), dtype=x.dtype, device=x.device) if want_dprev else None
+    need = load().delta_rule_shortconv_workspace_size(B, T, D) if want_dweight else 0
+    ws = _workspace(need, x.device) if need else None
+    rc = shortconv_bwd_raw(_p(x), _p(weight), _p(x_prev), _p(dy), _p(dx), _p(dw), _p(dprev), B, T, D,
+                           DTYPES[x.dtype], _p(ws), need, torch.cuda.current_stream(x.device).cuda_stream)
+    _check(rc, "delta_rule_shortconv_bwd")
+    return dx, dw, dprev
 
 
 def delta_rule_bwd(q, k, v, alpha, beta, S0, dout, du=None, dS_T=None, variant="gdn", chunk=64,

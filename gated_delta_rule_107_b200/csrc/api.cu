@@ -8,6 +8,7 @@
 #include "../../include/delta_rule.h"
 #include "decode.cuh"
 #include "prepost.cuh"
+#include "shortconv.cuh"
 #include "dr_common.cuh"
 #include "simt_path.cuh"
 #include "tc_path.cuh"
@@ -495,6 +496,61 @@ extern "C" int delta_rule_postop_bwd(const void *o, const void *gate, const floa
     pp.q = o; pp.k = gate; pp.w = weight; pp.dq = dy; pp.qo = do_; pp.ko = dgate; pp.dw = dweight;
     pp.part = (float *)workspace; pp.rows = rows; pp.d = dv;
     return launch_status(postop_run(pp, dtype == DR_BF16, true, (cudaStream_t)stream));
+}
+
+// Shape check of the short convolution: B sequences of T tokens with D channels.
+static int check_conv(int B, int T, int D, int dtype) {
+    if (B < 0 || T < 0 || D <= 0) return DR_ERR_ARG;
+    if (dtype != DR_F32 && dtype != DR_BF16) return DR_ERR_ARG;
+    if (D % 8 != 0) return DR_ERR_UNSUPPORTED;
+    if ((double)B * ((double)T + 3) * D > 9.0e18 / 16) return DR_ERR_ARG;
+    const bool bf16 = dtype == DR_BF16;
+    if (shortconv_ctas(B, T, D, bf16, false) > INT_MAX || shortconv_ctas(B, T, D, bf16, true) > INT_MAX)
+        return DR_ERR_UNSUPPORTED;
+    return DR_OK;
+}
+
+extern "C" size_t delta_rule_shortconv_workspace_size(int B, int T, int D) {
+    if (B < 0 || T < 0 || D <= 0 || D % 8 != 0) return (size_t)-1;
+    return shortconv_ws_bytes(B, T, D);
+}
+
+extern "C" int delta_rule_shortconv(const void *x, const float *w, const void *x_prev, void *y, void *cache_out,
+                                    int B, int T, int D, int dtype, void *stream) {
+    int rc = check_conv(B, T, D, dtype);
+    if (rc != DR_OK) return rc;
+    if (B == 0) return DR_OK;
+    if (!w || (T > 0 && (!x || !y))) return DR_ERR_ARG;
+    const void *vec[] = {x, x_prev, y, cache_out};
+    for (const void *p : vec)
+        if (p && !aligned16(p)) return DR_ERR_ALIGN;
+    if (!aligned_elem(w, DR_F32)) return DR_ERR_ALIGN;
+    if (T == 0 && !cache_out) return DR_OK;
+    ShortConv sc = {};
+    sc.x = x; sc.w = w; sc.cin = x_prev; sc.y = y; sc.cout = cache_out; sc.B = B; sc.T = T; sc.D = D;
+    return launch_status(shortconv_run(sc, dtype == DR_BF16, false, (cudaStream_t)stream));
+}
+
+extern "C" int delta_rule_shortconv_bwd(const void *x, const float *w, const void *x_prev, const void *dy,
+                                        void *dx, float *dw, void *dx_prev, int B, int T, int D, int dtype,
+                                        void *workspace, size_t ws_bytes_given, void *stream) {
+    int rc = check_conv(B, T, D, dtype);
+    if (rc != DR_OK) return rc;
+    if (B == 0) return DR_OK;
+    if (!w || (T > 0 && (!x || !dy || !dx))) return DR_ERR_ARG;
+    const void *vec[] = {x, x_prev, dy, dx, dx_prev};
+    for (const void *p : vec)
+        if (p && !aligned16(p)) return DR_ERR_ALIGN;
+    if (!aligned_elem(w, DR_F32) || (dw && !aligned_elem(dw, DR_F32))) return DR_ERR_ALIGN;
+    if (dw) {
+        rc = check_buffer(workspace, ws_bytes_given, shortconv_ws_bytes(B, T, D));
+        if (rc != DR_OK) return rc;
+    }
+    if (T == 0 && !dw && !dx_prev) return DR_OK;
+    ShortConv sc = {};
+    sc.x = x; sc.w = w; sc.cin = x_prev; sc.dy = dy; sc.dx = dx; sc.dw = dw; sc.dcin = dx_prev;
+    sc.part = (float *)workspace; sc.B = B; sc.T = T; sc.D = D;
+    return launch_status(shortconv_run(sc, dtype == DR_BF16, true, (cudaStream_t)stream));
 }
 
 // Self-test of the bounded waits: one thread waits for an mbarrier phase that nothing

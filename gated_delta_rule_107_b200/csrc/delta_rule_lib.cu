@@ -7,5 +7,6 @@
 #include "tc_bwd.cu"
 #include "decode.cu"
 #include "prepost.cu"
+#include "shortconv.cu"
 #include "api.cu"
 #include "noalloc.cu"

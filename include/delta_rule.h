@@ -274,6 +274,35 @@ int delta_rule_postop_bwd(const void *o, const void *gate, const float *weight, 
                           size_t ws_bytes, void *stream);
 
 /*
+ * Short convolution (Kimi Delta Attention page, section 4.2: a depthwise
+ * convolution of kernel size 4 on the q/k/v path).  Each of the D channels of a
+ * token-major stream x [B,T,D] (for q, k or v: D = H*d, the [B,T,H,d] layout
+ * above) is filtered causally with its own four taps w [D][4] (fp32, tap 3 on
+ * the current token), across each sequence b separately:
+ *     y[b,t,c] = sum_{j=0..3} w[c][j] * x[b, t-3+j, c]
+ * where x at t < 0 is read from the three-token cache x_prev [B,3,D] (row 3+t;
+ * NULL = zeros).  No bias and no activation.  cache_out [B,3,D] (NULL = not
+ * written) receives the last three tokens of [x_prev ; x], which a later call on
+ * the continuation of the stream takes as its x_prev; it must not alias x_prev.
+ * D must be a multiple of 8 (else DR_ERR_UNSUPPORTED); x, x_prev, y, cache_out,
+ * dy, dx, dx_prev 16-byte aligned; T = 0 writes only cache_out.
+ *
+ * delta_rule_shortconv_bwd: for dy [B,T,D], dx [B,T,D] (required when T > 0),
+ * dw [D][4] = sum over b, t of dy[b,t,c] * x[b,t-3+j,c] (NULL = not written) and
+ * dx_prev [B,3,D], the gradient of the cache tokens (NULL = not written).  dw
+ * needs a workspace of delta_rule_shortconv_workspace_size(B, T, D) bytes
+ * (256-byte aligned) and is summed in a fixed order (deterministic).  The
+ * cache_out of the forward is a copy of input tokens; gradients reaching it are
+ * the caller's to add to dx.
+ */
+size_t delta_rule_shortconv_workspace_size(int B, int T, int D);
+int delta_rule_shortconv(const void *x, const float *w, const void *x_prev, void *y, void *cache_out, int B, int T,
+                         int D, int dtype, void *stream);
+int delta_rule_shortconv_bwd(const void *x, const float *w, const void *x_prev, const void *dy, void *dx, float *dw,
+                             void *dx_prev, int B, int T, int D, int dtype, void *workspace, size_t ws_bytes,
+                             void *stream);
+
+/*
  * Self-test of failure detection.  Launches one kernel on `stream` whose bounded
  * wait (the same wait every pipelined kernel uses) waits for a barrier phase that
  * nothing completes; after limit_us microseconds (1 .. 1,000,000) it gives up,
