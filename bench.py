@@ -403,6 +403,13 @@ def run_ours(args):
     post_w = torch.ones(dv, device=dev)
     post_ms = ev_time(lambda: binding.delta_rule_postop(o, u, post_w))
     post_b_ms = ev_time(lambda: binding.delta_rule_postop_bwd(o, u, post_w, x["dO"]))
+    # cross-layer routing of this step's write values into a hidden stream of H*dv channels
+    n_hid = H * dv
+    clvr_W = (0.05 * torch.randn(H * dv, n_hid, device=dev)).to(u.dtype)
+    clvr_h = torch.randn(B, T, n_hid, device=dev).to(u.dtype)
+    clvr_ws = torch.empty(binding.load().delta_rule_clvr_workspace_size(), dtype=torch.uint8, device=dev)
+    clvr_ms = ev_time(lambda: binding.delta_rule_clvr(u, clvr_W, clvr_h, workspace=clvr_ws))
+    clvr_b_ms = ev_time(lambda: binding.delta_rule_clvr_bwd(u, clvr_W, clvr_h, workspace=clvr_ws))
     conv_w = 0.5 * torch.randn(H * dk, 4, device=dev)
     conv_ms = ev_time(lambda: binding.delta_rule_shortconv(x["q"], conv_w))
     conv_b_ms = ev_time(lambda: binding.delta_rule_shortconv_bwd(x["q"], conv_w, x["q"]))
@@ -421,6 +428,14 @@ def run_ours(args):
                "postop_bwd": gbs(rows * elem * 5 * dv, post_b_ms),
                # one [B, T, H*dk] stream: x read, y written (backward: x, dy read, dx written)
                "shortconv": gbs(2 * rows * elem * dk, conv_ms), "shortconv_bwd": gbs(3 * rows * elem * dk, conv_b_ms)}
+
+    clvr_flops = 2.0 * B * T * (H * dv) * n_hid
+    bf16_peak = load_peaks().get("bf16_tflops")
+    clvr = {"shape": f"M{B * T} K{H * dv} N{n_hid} bf16 (cuBLASLt)", "fwd_ms": clvr_ms, "bwd_ms": clvr_b_ms,
+            "fwd_tflops": clvr_flops / (clvr_ms / 1e3) / 1e12, "bwd_tflops": 2 * clvr_flops / (clvr_b_ms / 1e3) / 1e12}
+    if bf16_peak:
+        clvr["fwd_frac"] = clvr["fwd_tflops"] / bf16_peak
+        clvr["bwd_frac"] = clvr["bwd_tflops"] / bf16_peak
 
     # ---- end to end through the public API with host buffers ----
     host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in x.items()}
@@ -523,6 +538,7 @@ def run_ours(args):
         "saved_bytes": sv_bytes,
         "decode": decode,
         "prepost": prepost,
+        "clvr": clvr,
         "gpu_launches": args.steps * (len(fwd_names) + len(bwd_names)),
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

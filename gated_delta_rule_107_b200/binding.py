@@ -43,7 +43,8 @@ EXPORTS = ("delta_rule_workspace_size", "delta_rule_fwd", "delta_rule_bwd", "del
            "delta_rule_fwd_save_timed", "delta_rule_bwd_saved_timed", "delta_rule_decode",
            "delta_rule_preop", "delta_rule_preop_bwd", "delta_rule_postop_workspace_size", "delta_rule_postop",
            "delta_rule_postop_bwd", "delta_rule_selftest_timeout", "delta_rule_shortconv_workspace_size",
-           "delta_rule_shortconv", "delta_rule_shortconv_bwd")
+           "delta_rule_shortconv", "delta_rule_shortconv_bwd", "delta_rule_clvr_workspace_size", "delta_rule_clvr",
+           "delta_rule_clvr_bwd")
 
 _lib = None
 
@@ -105,6 +106,12 @@ def load(path: str | None = None):
     lib.delta_rule_shortconv.restype = i
     lib.delta_rule_shortconv_bwd.argtypes = [vp] * 7 + [i] * 4 + [vp, sz, vp]
     lib.delta_rule_shortconv_bwd.restype = i
+    lib.delta_rule_clvr_workspace_size.argtypes = []
+    lib.delta_rule_clvr_workspace_size.restype = sz
+    lib.delta_rule_clvr.argtypes = [vp] * 4 + [i] * 4 + [vp, sz, vp]
+    lib.delta_rule_clvr.restype = i
+    lib.delta_rule_clvr_bwd.argtypes = [vp] * 5 + [i] * 4 + [vp, sz, vp]
+    lib.delta_rule_clvr_bwd.restype = i
     lib.delta_rule_selftest_timeout.argtypes = [ctypes.c_uint, vp]
     lib.delta_rule_selftest_timeout.restype = i
     lib.delta_rule_decode.argtypes = [vp] * 9 + [i] * 7 + [vp]
@@ -384,6 +391,43 @@ def delta_rule_shortconv_bwd(x, weight, dy, x_prev=None, want_dweight=True, want
                            DTYPES[x.dtype], _p(ws), need, torch.cuda.current_stream(x.device).cuda_stream)
     _check(rc, "delta_rule_shortconv_bwd")
     return dx, dw, dprev
+
+
+def clvr_raw(*args) -> int:
+    return load().delta_rule_clvr(*args)
+
+
+def clvr_bwd_raw(*args) -> int:
+    return load().delta_rule_clvr_bwd(*args)
+
+
+def delta_rule_clvr(u, W, h=None, out=None, workspace=None):
+    """h + u W for write values u ([B, T, H, dv] or [M, K]) and W [K, N]; returns [..., N] shaped like h
+    (or [M, N]).  out may be h itself (in-place residual add)."""
+    K, N = W.shape
+    M = u.numel() // K
+    if out is None:
+        out = torch.empty((M, N) if h is None else h.shape, dtype=u.dtype, device=u.device)
+    need = load().delta_rule_clvr_workspace_size()
+    ws = workspace if workspace is not None else _workspace(need, u.device)
+    rc = clvr_raw(_p(u), _p(W), _p(h), _p(out), M, K, N, DTYPES[u.dtype], _p(ws), need,
+                  torch.cuda.current_stream(u.device).cuda_stream)
+    _check(rc, "delta_rule_clvr")
+    return out
+
+
+def delta_rule_clvr_bwd(u, W, dh_out, want_du=True, want_dW=True, workspace=None):
+    """Returns (du shaped like u or None, dW [K, N] fp32 or None)."""
+    K, N = W.shape
+    M = u.numel() // K
+    du = torch.empty_like(u) if want_du else None
+    dW = torch.empty((K, N), dtype=torch.float32, device=u.device) if want_dW else None
+    need = load().delta_rule_clvr_workspace_size()
+    ws = workspace if workspace is not None else _workspace(need, u.device)
+    rc = clvr_bwd_raw(_p(u), _p(W), _p(dh_out), _p(du), _p(dW), M, K, N, DTYPES[u.dtype], _p(ws), need,
+                      torch.cuda.current_stream(u.device).cuda_stream)
+    _check(rc, "delta_rule_clvr_bwd")
+    return du, dW
 
 
 def delta_rule_bwd(q, k, v, alpha, beta, S0, dout, du=None, dS_T=None, variant="gdn", chunk=64,

@@ -16,6 +16,7 @@ NVCC_FLAGS = [
     "-Xcompiler", "-fPIC", "-shared",
     "--expt-relaxed-constexpr",
     "-Xptxas", "-warn-spills",
+    "-lcublasLt", "-Xlinker", "-rpath=/usr/local/cuda/lib64",
 ]
 
 

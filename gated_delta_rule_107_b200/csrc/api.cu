@@ -9,6 +9,7 @@
 #include "decode.cuh"
 #include "prepost.cuh"
 #include "shortconv.cuh"
+#include "clvr.cuh"
 #include "dr_common.cuh"
 #include "simt_path.cuh"
 #include "tc_path.cuh"
@@ -551,6 +552,46 @@ extern "C" int delta_rule_shortconv_bwd(const void *x, const float *w, const voi
     sc.x = x; sc.w = w; sc.cin = x_prev; sc.dy = dy; sc.dx = dx; sc.dw = dw; sc.dcin = dx_prev;
     sc.part = (float *)workspace; sc.B = B; sc.T = T; sc.D = D;
     return launch_status(shortconv_run(sc, dtype == DR_BF16, true, (cudaStream_t)stream));
+}
+
+// Shape check of the routing products: M tokens, K = H dv write-value channels, N hidden channels.
+static int check_clvr(int M, int K, int N, int dtype) {
+    if (M < 0 || K <= 0 || N <= 0) return DR_ERR_ARG;
+    if (dtype != DR_F32 && dtype != DR_BF16) return DR_ERR_ARG;
+    if (K % 8 != 0 || N % 8 != 0) return DR_ERR_UNSUPPORTED;
+    return DR_OK;
+}
+
+extern "C" size_t delta_rule_clvr_workspace_size(void) { return clvr_ws_bytes(); }
+
+extern "C" int delta_rule_clvr(const void *u, const void *W, const void *h, void *h_out, int M, int K, int N,
+                               int dtype, void *workspace, size_t ws_bytes_given, void *stream) {
+    int rc = check_clvr(M, K, N, dtype);
+    if (rc != DR_OK || M == 0) return rc;
+    if (!u || !W || !h_out) return DR_ERR_ARG;
+    const void *vec[] = {u, W, h, h_out};
+    for (const void *p : vec)
+        if (p && !aligned16(p)) return DR_ERR_ALIGN;
+    rc = check_buffer(workspace, ws_bytes_given, clvr_ws_bytes());
+    if (rc != DR_OK) return rc;
+    return clvr_fwd_run(u, W, h, h_out, M, K, N, dtype == DR_BF16, workspace, ws_bytes_given, (cudaStream_t)stream);
+}
+
+extern "C" int delta_rule_clvr_bwd(const void *u, const void *W, const void *dh_out, void *du, float *dW, int M,
+                                   int K, int N, int dtype, void *workspace, size_t ws_bytes_given, void *stream) {
+    int rc = check_clvr(M, K, N, dtype);
+    if (rc != DR_OK) return rc;
+    if (!u || !W || !dh_out) return M == 0 ? DR_OK : DR_ERR_ARG;
+    const void *vec[] = {u, W, dh_out, du, dW};
+    for (const void *p : vec)
+        if (p && !aligned16(p)) return DR_ERR_ALIGN;
+    if (M == 0) {  // no tokens: dW is an empty sum
+        return dW ? launch_status(cudaMemsetAsync(dW, 0, (size_t)K * N * sizeof(float), (cudaStream_t)stream)) : DR_OK;
+    }
+    rc = check_buffer(workspace, ws_bytes_given, clvr_ws_bytes());
+    if (rc != DR_OK) return rc;
+    return clvr_bwd_run(u, W, dh_out, du, dW, M, K, N, dtype == DR_BF16, workspace, ws_bytes_given,
+                        (cudaStream_t)stream);
 }
 
 // Self-test of the bounded waits: one thread waits for an mbarrier phase that nothing

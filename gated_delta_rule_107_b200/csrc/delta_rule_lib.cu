@@ -8,5 +8,6 @@
 #include "decode.cu"
 #include "prepost.cu"
 #include "shortconv.cu"
+#include "clvr.cu"
 #include "api.cu"
 #include "noalloc.cu"

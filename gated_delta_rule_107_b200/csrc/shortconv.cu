@@ -19,7 +19,7 @@ namespace scv {
 
 constexpr int K = 4;      // taps
 constexpr int NT = 256;   // threads per CTA
-constexpr int TBF = 16;   // tokens per thread, forward
+constexpr int TBF = 32;   // tokens per thread, forward
 constexpr int TBB = 64;   // tokens per thread, backward (one dw partial per block)
 
 inline int blocks_of(int T, int tb) { return T <= 0 ? 1 : (T + tb - 1) / tb; }

@@ -303,6 +303,27 @@ int delta_rule_shortconv_bwd(const void *x, const float *w, const void *x_prev, 
                              void *stream);
 
 /*
+ * Cross-layer value routing (ETH news page on the architecture study, section 七;
+ * the explainer's CLVR section): a layer's write values u (the u output of the
+ * forward, [B,T,H,dv] read as an M x K matrix, M = B*T, K = H*dv) enter a higher
+ * layer's hidden stream h [M,N] through a projection W [K,N] that starts at zero:
+ *     h_out = h + u W          (h NULL: h_out = u W; h_out may alias h)
+ * delta_rule_clvr_bwd: for dh_out [M,N], du = dh_out W^T [M,K] (NULL = not
+ * written) and dW = u^T dh_out [K,N], fp32 (NULL = not written); the gradient of
+ * h is dh_out itself.  u, W, h, h_out, dh_out and du have the I/O dtype.  These
+ * are plain dense products and run as cuBLASLt GEMMs (bf16 operands with fp32
+ * accumulation, or fp32 throughout for fp32 I/O) with a caller workspace of
+ * delta_rule_clvr_workspace_size() bytes (256-byte aligned).  The first call
+ * creates the process's one cuBLASLt handle.  K and N must be multiples of 8;
+ * every pointer 16-byte aligned.
+ */
+size_t delta_rule_clvr_workspace_size(void);
+int delta_rule_clvr(const void *u, const void *W, const void *h, void *h_out, int M, int K, int N, int dtype,
+                    void *workspace, size_t ws_bytes, void *stream);
+int delta_rule_clvr_bwd(const void *u, const void *W, const void *dh_out, void *du, float *dW, int M, int K, int N,
+                        int dtype, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Self-test of failure detection.  Launches one kernel on `stream` whose bounded
  * wait (the same wait every pipelined kernel uses) waits for a barrier phase that
  * nothing completes; after limit_us microseconds (1 .. 1,000,000) it gives up,

@@ -25,7 +25,7 @@ def _inputs(dtype, B, T, D, seed, prev=True):
 
 
 def _check(got, ref, tol, what):
-    err = rel_err(np64(got), ref)
+    err = rel_err(got if isinstance(got, np.ndarray) else np64(got), ref)
     assert err <= tol, f"{what}: {err} (tol {tol})"
 
 
