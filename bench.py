@@ -505,7 +505,8 @@ def run_ours(args):
             with open(tfile) as f:
                 tr = json.load(f)
             ent = tr.get(r_label)
-            if ent and ent.get("source_digest") == source_digest():
+            # counters stay valid while the files that define the kernel are unchanged
+            if ent and ent.get("source_digest") == source_digest(ent.get("source_files")):
                 traffic = ent["bytes_per_launch"] * (B / ent.get("batch", B))
         except Exception:
             traffic = None

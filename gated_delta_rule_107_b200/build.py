@@ -25,15 +25,24 @@ def sources() -> list[str]:
                   + glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
-def source_digest() -> str:
-    """sha256 over the library sources (identifies the kernels a profile was taken on)."""
+def source_digest(files: list[str] | None = None) -> str:
+    """sha256 over library sources (identifies the code a profile was taken on): every source,
+    or only the named files of csrc/ (those that define one kernel and its launch)."""
     import hashlib
     h = hashlib.sha256()
-    for p in sources():
+    paths = sources() if files is None else [os.path.join(CSRC, f) for f in sorted(files)]
+    for p in paths:
         h.update(os.path.basename(p).encode())
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+# the files that define each profiled kernel and its launch
+KERNEL_FILES = {
+    "k_bwd_chunk_tc": ["tc_bwd.cu", "tc_ptx.cuh", "tc_tile.cuh", "tc_inverse.cuh", "tc_host.cuh", "tc_path.cuh",
+                       "dr_common.cuh"],
+}
 
 
 def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
