@@ -210,10 +210,12 @@ static int bwd_impl(const void *q, const void *k, const void *v, const void *alp
         rc = launch_status(tc_kda_gates(g, t, w, sw.G, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_chunk_prep(g, t, w, false, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, 1, s, rec));
-        if (rc == DR_OK) rc = launch_status(tc_to_simt(g, w, sw.W, sw.Ut, sw.P, sw.Sn, sw.Un, s, rec));
+        // the CUDA-core gradient kernel reads W, U~, U, dU widened to fp32 and the state products
+        if (rc == DR_OK) rc = launch_status(tc_to_simt(g, w, sw.W, sw.Ut, nullptr, nullptr, sw.Un, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_chain_rev(g, t, w, s, rec));
-        if (rc == DR_OK) rc = launch_status(tc_rev_to_simt(g, w, sw.dSn, sw.dUn, s, rec));
-        if (rc == DR_OK) rc = launch_status(simt_bwd_grads(g, t, dtype == DR_BF16, sw, s, rec));
+        if (rc == DR_OK) rc = launch_status(tc_rev_to_simt(g, w, nullptr, sw.dUn, s, rec));
+        if (rc == DR_OK) rc = launch_status(tc_state_to_simt(g, t, w, sw.Qd, sw.dWm, sw.Tm, sw.RS, s, rec));
+        if (rc == DR_OK) rc = launch_status(simt_bwd_intra(g, t, dtype == DR_BF16, sw, s, rec));
     } else {
         const SimtWs w = simt_ws_carve(g, true, workspace);
         rc = launch_status(simt_bwd(g, t, dtype == DR_BF16, w, s, rec));
@@ -231,7 +233,7 @@ static int launch_plan(const Geo &g, int dtype, int kind, const char **names, in
     static const char *const SPLIT_BWD_SAVED[2] = {"k_chain_rev", "k_bwd_chunk_tc"};
     static const char *const SPLIT_KDA_FWD[3] = {"k_kda_gates", "k_chunk_prep", "k_chain_fwd"};
     static const char *const KDA_BWD[8] = {"k_kda_gates", "k_chunk_prep", "k_chain_fwd(recompute)", "k_widen",
-                                           "k_chain_rev", "k_widen", "k_bwd_state", "k_bwd_intra"};
+                                           "k_chain_rev", "k_widen", "k_state_tc", "k_bwd_intra"};
     int n = 0;
     const char *const *src = nullptr;
     if (g.T == 0 || g.B == 0 || g.H == 0) return 0;

@@ -5,6 +5,7 @@
 #include "tc_prep.cu"
 #include "tc_chain.cu"
 #include "tc_bwd.cu"
+#include "tc_state.cu"
 #include "decode.cu"
 #include "prepost.cu"
 #include "shortconv.cu"

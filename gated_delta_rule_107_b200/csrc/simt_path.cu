@@ -1299,7 +1299,8 @@ static cudaError_t fwd_t(const Geo &g, const Tensors &t, const SimtWs &w, cudaSt
 }
 
 // from = 0: everything; 1: the forward's W, U~, G, P, S_n, U are in w already; 2: so are the
-// reverse chain's dS_{n+1} and dU (and dS0 is written)
+// reverse chain's dS_{n+1} and dU (and dS0 is written); 3: so are the state products Qd, dWm,
+// Tm, RS (only k_bwd_intra runs)
 template <typename TI>
 static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, int from, cudaStream_t s, Rec &rec) {
     const IO<TI> io = io_of<TI>(t);
@@ -1320,9 +1321,11 @@ static cudaError_t bwd_t(const Geo &g, const Tensors &t, const SimtWs &w, int fr
         k_scan_bwd<TI><<<gs, NT, sm_sb, s>>>(g, io, w, t.dS_T, t.dS0);
         DR_TRY(cudaGetLastError());
     }
-    rec.mark(s);
-    k_bwd_state<TI><<<gc, NT, sm_st, s>>>(g, io, w);
-    DR_TRY(cudaGetLastError());
+    if (from < 3) {
+        rec.mark(s);
+        k_bwd_state<TI><<<gc, NT, sm_st, s>>>(g, io, w);
+        DR_TRY(cudaGetLastError());
+    }
     rec.mark(s);
     k_bwd_intra<TI><<<gc, NT, sm_in, s>>>(g, io, w);
     return cudaGetLastError();
@@ -1338,6 +1341,10 @@ cudaError_t simt_bwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w,
 
 cudaError_t simt_bwd_grads(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec) {
     return bf16 ? bwd_t<__nv_bfloat16>(g, t, w, 2, s, rec) : bwd_t<float>(g, t, w, 2, s, rec);
+}
+
+cudaError_t simt_bwd_intra(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec) {
+    return bf16 ? bwd_t<__nv_bfloat16>(g, t, w, 3, s, rec) : bwd_t<float>(g, t, w, 3, s, rec);
 }
 
 }  // namespace dr

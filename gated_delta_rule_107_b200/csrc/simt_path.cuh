@@ -28,6 +28,9 @@ cudaError_t simt_bwd(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w,
 // The backward's last two kernels (k_bwd_state, k_bwd_intra), for a w whose G, W, Ut, P, Sn,
 // Un hold the forward's values and dSn, dUn the reverse chain's (from tensor-core kernels).
 cudaError_t simt_bwd_grads(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec);
+// The intra-chunk gradient kernel alone: w holds, besides what simt_bwd_grads reads, the
+// state products Qd, dWm, Tm, RS.
+cudaError_t simt_bwd_intra(const Geo &g, const Tensors &t, bool bf16, const SimtWs &w, cudaStream_t s, Rec &rec);
 // kernel names in launch order (for the timed entry points)
 extern const char *const SIMT_FWD_KERNELS[3];
 extern const char *const SIMT_BWD_KERNELS[5];

@@ -66,6 +66,11 @@ cudaError_t tc_to_simt(const Geo &g, const TcWs &w, float *W, float *Ut, float *
                        Rec &rec);
 // fp32 copies of the reverse chain's dS_{n+1} and dL/dU (tc_prep.cu).
 cudaError_t tc_rev_to_simt(const Geo &g, const TcWs &w, float *dSn, float *dUn, cudaStream_t s, Rec &rec);
+// The KDA backward's products with the chunk states on tcgen05, from the bf16 workspace tiles
+// (S_n, dS_{n+1}, U, dU) and dO: Qd = dO S^T, dWm = -dU S^T, Tm = U dS+^T, RS = rowsum(S .* dS+),
+// written to the CUDA-core workspace ([ci][C][dk] fp32 each; RS [ci][dk]).
+cudaError_t tc_state_to_simt(const Geo &g, const Tensors &t, const TcWs &w, float *Qd, float *dWm, float *Tm,
+                             float *RS, cudaStream_t s, Rec &rec);
 // Per-chunk products (tc_prep.cu): g and beta, W, U~, P; with keep also T and k k^T.
 // For KDA (no keep) from the operands of tc_kda_gates.
 cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool keep, cudaStream_t s, Rec &rec);

@@ -503,8 +503,8 @@ cudaError_t tc_to_simt(const Geo &g, const TcWs &w, float *W, float *Ut, float *
     const __nv_bfloat16 *src[5] = {w.W, w.Ut, w.P, w.Sn, w.Un};
     float *dst[5] = {W, Ut, P, Sn, Un};
     const size_t n[5] = {nc * C * DK, nc * C * DV, nc * C * C, nc * DK * DV, nc * C * DV};
-    for (int i = 0; i < 5; ++i) {
-        a.src[i] = src[i];
+    for (int i = 0; i < 5; ++i) {  // an absent destination is not widened
+        a.src[i] = dst[i] ? src[i] : nullptr;
         a.dst[i] = dst[i];
         a.n8[i] = n[i] / 8;
     }
@@ -517,8 +517,8 @@ cudaError_t tc_rev_to_simt(const Geo &g, const TcWs &w, float *dSn, float *dUn, 
     using namespace tcp;
     const size_t nc = (size_t)g.B * g.H * g.N;
     Widen a = {};
-    a.src[0] = w.dSn; a.dst[0] = dSn; a.n8[0] = nc * DK * DV / 8;
-    a.src[1] = w.dUn; a.dst[1] = dUn; a.n8[1] = nc * C * DV / 8;
+    a.src[0] = dSn ? w.dSn : nullptr; a.dst[0] = dSn; a.n8[0] = nc * DK * DV / 8;
+    a.src[1] = dUn ? w.dUn : nullptr; a.dst[1] = dUn; a.n8[1] = nc * C * DV / 8;
     rec.mark(s);
     k_widen<<<148 * 8, 256, 0, s>>>(a);
     return cudaGetLastError();

@@ -155,7 +155,7 @@ def test_bf16_d128_uses_the_tensor_core_kernel():
     assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 0) == kda_split
     assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 2) == kda_split  # no saved form: the plain forward
     kda_bwd = ["k_kda_gates", "k_chunk_prep", "k_chain_fwd(recompute)", "k_widen", "k_chain_rev", "k_widen",
-               "k_bwd_state", "k_bwd_intra"]
+               "k_state_tc", "k_bwd_intra"]
     assert binding.launches(8, 4096, 16, 128, 128, 2, 64, 1, 1) == kda_bwd
     assert binding.launches(8, 4096, 16, 128, 128, 2, 64, 1, 3) == kda_bwd
     assert binding.launches(2, 512, 4, 128, 64, 2, 64, 1, 0) == ["k_fwd_tc"]
