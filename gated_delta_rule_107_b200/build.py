@@ -40,8 +40,7 @@ def source_digest(files: list[str] | None = None) -> str:
 
 # the files that define each profiled kernel and its launch
 KERNEL_FILES = {
-    "k_bwd_chunk_tc": ["tc_bwd.cu", "tc_ptx.cuh", "tc_tile.cuh", "tc_inverse.cuh", "tc_host.cuh", "tc_path.cuh",
-                       "dr_common.cuh"],
+    "k_bwd_chunk_tc": ["tc_bwd.cu", "tc_ptx.cuh", "tc_tile.cuh", "tc_inverse.cuh", "tc_host.cuh", "dr_common.cuh"],
 }
 
 
