@@ -100,3 +100,41 @@ def test_postop_backward_matches_finite_differences():
     assert np.allclose(got["do"], _fd(lambda x: loss(x, g, w), o), atol=1e-7)
     assert np.allclose(got["dg"], _fd(lambda x: loss(o, x, w), g), atol=1e-7)
     assert np.allclose(got["dw"], _fd(lambda x: loss(o, g, x), w), atol=1e-7)
+
+
+# ---- planted mistakes in copies of the oracle's source must each fail a pin above ----
+import types  # noqa: E402
+
+PINS = [test_l2norm_gives_unit_rows_and_is_scale_invariant, test_zero_row_stays_finite, test_logistic_gate_symmetries,
+        test_rmsnorm_output_has_the_weights_rms, lambda: test_preop_backward_matches_finite_differences(True),
+        lambda: test_preop_backward_matches_finite_differences(False),
+        test_postop_backward_matches_finite_differences]
+
+MUTANTS = [
+    ("l2norm_sum_not_root", "return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + EPS)",
+     "return x / (np.sum(x * x, axis=-1, keepdims=True) + EPS)"),
+    ("l2norm_bwd_projection_dropped", "return (dy - y * np.sum(y * dy, axis=-1, keepdims=True)) / r", "return dy / r"),
+    ("beta_grad_without_derivative", '"db": _f64(dbeta) * beta * (1.0 - beta)', '"db": _f64(dbeta) * beta'),
+    ("gate_grad_sign", 'out["da"] = -_f64(dloga) * _sigmoid(_f64(a))', 'out["da"] = _f64(dloga) * _sigmoid(_f64(a))'),
+    ("softplus_sign", '"loga": None if a is None else -_softplus(a)}', '"loga": None if a is None else _softplus(a)}'),
+    ("rms_sum_not_mean", "n = o / np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + EPS)",
+     "n = o / np.sqrt(np.sum(o * o, axis=-1, keepdims=True) + EPS)"),
+    ("postop_dw_without_n", "dw = np.sum((dz * n).reshape(-1, d), axis=0)", "dw = np.sum(dz.reshape(-1, d), axis=0)"),
+    ("postop_do_projection_dropped", "do = r * (dn - n * np.mean(dn * n, axis=-1, keepdims=True))", "do = r * dn"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(name, old, new, monkeypatch):
+    src = open(pp.__file__).read()
+    assert src.count(old) == 1, f"mutation site for {name}"
+    mod = types.ModuleType(f"prepost_{name}")
+    exec(compile(src.replace(old, new), f"<{name}>", "exec"), mod.__dict__)
+    monkeypatch.setitem(globals(), "pp", mod)  # the pins above read the module through this name
+    caught = 0
+    for pin in PINS:
+        try:
+            pin()
+        except AssertionError:
+            caught += 1
+    assert caught > 0, f"no pin catches {name}"
