@@ -71,3 +71,38 @@ def test_no_compute_validation_paths(lib):
     args = [None] * 9 + [1, 10, 1, 128, 128, 7, 64, 1, None, 0, None, 0, None]
     assert binding.fwd_save_raw(*args) == binding.DR_ERR_ARG
     assert binding.strerror(12345) == "unknown error code"
+
+
+def test_operations_around_the_core_validate_before_any_launch(lib):
+    """The short convolution, the routing products, decoding and the pre/post operations reject bad
+    shapes, enums and pointers with their codes, and size their workspaces, without a GPU."""
+    from gated_delta_rule_107_b200 import binding
+    bad = ctypes.c_size_t(-1).value
+    # short convolution: D a multiple of 8; workspace = one fp32 [D][4] partial per (sequence, 64 tokens)
+    assert lib.delta_rule_shortconv_workspace_size(8, 4096, 1024) == 8 * 64 * 1024 * 4 * 4
+    assert lib.delta_rule_shortconv_workspace_size(2, 0, 64) == 2 * 1 * 64 * 4 * 4
+    assert lib.delta_rule_shortconv_workspace_size(1, 10, 60) == bad
+    assert binding.shortconv_raw(None, None, None, None, None, 1, 10, 60, binding.DR_BF16, None) == \
+        binding.DR_ERR_UNSUPPORTED
+    assert binding.shortconv_raw(None, None, None, None, None, 1, 10, 64, 3, None) == binding.DR_ERR_ARG
+    assert binding.shortconv_raw(None, None, None, None, None, -1, 10, 64, binding.DR_BF16, None) == binding.DR_ERR_ARG
+    assert binding.shortconv_raw(None, None, None, None, None, 0, 10, 64, binding.DR_BF16, None) == binding.DR_OK
+    assert binding.shortconv_raw(None, None, None, None, None, 1, 10, 64, binding.DR_BF16, None) == binding.DR_ERR_ARG
+    assert binding.shortconv_bwd_raw(None, None, None, None, None, None, None, 1, 10, 64, binding.DR_BF16, None, 0,
+                                     None) == binding.DR_ERR_ARG
+    # routing: K, N multiples of 8, a caller workspace, M = 0 a no-op
+    assert lib.delta_rule_clvr_workspace_size() >= 1 << 20
+    assert binding.clvr_raw(None, None, None, None, 4, 60, 64, binding.DR_BF16, None, 0, None) == \
+        binding.DR_ERR_UNSUPPORTED
+    assert binding.clvr_raw(None, None, None, None, 4, 64, 64, 7, None, 0, None) == binding.DR_ERR_ARG
+    assert binding.clvr_raw(None, None, None, None, 0, 64, 64, binding.DR_BF16, None, 0, None) == binding.DR_OK
+    assert binding.clvr_raw(None, None, None, None, 4, 64, 64, binding.DR_BF16, None, 0, None) == binding.DR_ERR_ARG
+    assert binding.clvr_bwd_raw(None, None, None, None, None, 4, 64, 64, binding.DR_BF16, None, 0, None) == \
+        binding.DR_ERR_ARG
+    # decoding and the pre/post operations
+    assert binding.decode_raw(*([None] * 9), 1, 2, 1, 96, 128, binding.DR_GATED, binding.DR_BF16, None) == \
+        binding.DR_ERR_UNSUPPORTED
+    assert binding.preop_raw(*([None] * 8), 1, 4, 1, 96, binding.DR_GATED, binding.DR_BF16, None) == \
+        binding.DR_ERR_UNSUPPORTED
+    assert binding.postop_raw(None, None, None, None, 1, 4, 1, 128, 5, None) == binding.DR_ERR_ARG
+    assert lib.delta_rule_postop_workspace_size(96) == bad
