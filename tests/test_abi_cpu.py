@@ -106,3 +106,28 @@ def test_operations_around_the_core_validate_before_any_launch(lib):
         binding.DR_ERR_UNSUPPORTED
     assert binding.postop_raw(None, None, None, None, 1, 4, 1, 128, 5, None) == binding.DR_ERR_ARG
     assert lib.delta_rule_postop_workspace_size(96) == bad
+
+
+def test_launch_plans(lib):
+    """Which kernels each call launches (host logic, no GPU): the tensor-core paths for bf16 at
+    d = 128, the KDA hybrid backward, the fused dv = 64 kernel and the CUDA-core path."""
+    from gated_delta_rule_107_b200 import binding
+    split = {0: ["k_chunk_prep", "k_chain_fwd"],
+             1: ["k_chunk_prep(keep)", "k_chain_fwd(recompute)", "k_chain_rev", "k_bwd_chunk_tc"],
+             2: ["k_chunk_prep(keep)", "k_chain_fwd(keep)"],
+             3: ["k_chain_rev", "k_bwd_chunk_tc"]}
+    for variant in (0, 1):
+        for kind, names in split.items():
+            assert binding.launches(8, 4096, 8, 128, 128, variant, 64, 1, kind) == names
+    kda_split = ["k_kda_gates", "k_chunk_prep", "k_chain_fwd"]
+    assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 0) == kda_split
+    assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 2) == kda_split  # no saved form: the plain forward
+    kda_bwd = ["k_kda_gates", "k_chunk_prep", "k_chain_fwd(recompute)", "k_widen", "k_chain_rev", "k_widen",
+               "k_state_tc", "k_bwd_intra"]
+    assert binding.launches(8, 4096, 16, 128, 128, 2, 64, 1, 1) == kda_bwd
+    assert binding.launches(8, 4096, 16, 128, 128, 2, 64, 1, 3) == kda_bwd
+    assert binding.launches(2, 512, 4, 128, 64, 2, 64, 1, 0) == ["k_fwd_tc"]
+    assert binding.launches(2, 512, 4, 128, 64, 1, 64, 1, 0) == ["k_fwd_tc"]
+    assert binding.launches(1, 256, 2, 64, 64, 0, 64, 0, 0) == ["k_prep", "k_scan", "k_out"]
+    assert binding.launches(1, 256, 2, 64, 64, 0, 64, 0, 1) == ["k_prep", "k_scan", "k_scan_bwd", "k_bwd_state",
+                                                             "k_bwd_intra"]

@@ -143,26 +143,6 @@ def test_split_sequence_tensor_core_path():
     assert rel_err(np64(rb["S_T"]), ref["S_T"]) < 2e-2
 
 
-def test_bf16_d128_uses_the_tensor_core_kernel():
-    split = {0: ["k_chunk_prep", "k_chain_fwd"],
-             1: ["k_chunk_prep(keep)", "k_chain_fwd(recompute)", "k_chain_rev", "k_bwd_chunk_tc"],
-             2: ["k_chunk_prep(keep)", "k_chain_fwd(keep)"],
-             3: ["k_chain_rev", "k_bwd_chunk_tc"]}
-    for variant in (0, 1):
-        for kind, names in split.items():
-            assert binding.launches(8, 4096, 8, 128, 128, variant, 64, 1, kind) == names
-    kda_split = ["k_kda_gates", "k_chunk_prep", "k_chain_fwd"]
-    assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 0) == kda_split
-    assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 2) == kda_split  # no saved form: the plain forward
-    kda_bwd = ["k_kda_gates", "k_chunk_prep", "k_chain_fwd(recompute)", "k_widen", "k_chain_rev", "k_widen",
-               "k_state_tc", "k_bwd_intra"]
-    assert binding.launches(8, 4096, 16, 128, 128, 2, 64, 1, 1) == kda_bwd
-    assert binding.launches(8, 4096, 16, 128, 128, 2, 64, 1, 3) == kda_bwd
-    assert binding.launches(2, 512, 4, 128, 64, 2, 64, 1, 0) == ["k_fwd_tc"]
-    assert binding.launches(2, 512, 4, 128, 64, 1, 64, 1, 0) == ["k_fwd_tc"]
-    assert binding.launches(1, 256, 2, 64, 64, 0, 64, 0, 0) == ["k_prep", "k_scan", "k_out"]
-
-
 def test_host_buffer_entry_point():
     x = gen("gdn", "bf16", 1, 100, 2, 128, 128, seed=6)
     h = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in x.items()}
