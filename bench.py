@@ -51,7 +51,19 @@ def alg_counts(B, T, H, dk, dv, C, variant, elem, s0=False, du=True):
     bwd_bytes = th * elem * bwd_in_out + heads * 4 * dk * dv * (2 + int(s0))
     return {"fwd_flops": fwd_flops, "fwd_bytes": fwd_bytes, "bwd_flops": 2 * fwd_flops, "bwd_bytes": bwd_bytes,
             # the per-token-head backward inputs and outputs, without the per-head states
-            "bwd_io_bytes": th * elem * bwd_in_out}
+            "bwd_io_bytes": th * elem * bwd_in_out,
+            # what the intra-chunk gradient kernel itself reads and writes: the same without du,
+            # which the reverse chain consumes (it hands the kernel dL/dU instead)
+            "bwd_grad_kernel_bytes": th * elem * (bwd_in_out - (dv if du else 0))}
+
+
+def workload_config(w, B, world):
+    """The config object of the JSON line; both arms print the same one."""
+    name = w.name if B == w.B else w.name.replace(f"_B{w.B}_", f"_B{B}_")
+    return {"workload": name + " fwd+bwd", "B": B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv, "chunk": 64,
+            "variant": {0: "deltanet", 1: "gdn", 2: "kda"}[w.variant], "io": "bf16, fp32 state",
+            "l2": "flushed between steps (256 MiB write)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
 def load_peaks():
@@ -152,7 +164,7 @@ def cpu_oracle_sample(w, steps=1, seed=0):
     full_time = t * (w.B * w.H) / units
     value = w.B * w.T / full_time
     sample = (f"fp64 oracle fwd+bwd on {units} (b,h) sequences of T={w.T} (of {w.B * w.H}); "
-              f"{t:.2f} s per sample, extrapolated by the (b,h) count")
+              f"{t:.2f} s per sample; the rate is extrapolated to the workload by the (b,h) count")
     return {"value": value, "unit": "tokens/s", "cores": units, "kind": "oracle", "sample": sample,
             "sample_seconds": t}, times, np
 
@@ -189,13 +201,15 @@ def run_reference(args):
     w = WORKLOADS[WORKLOAD_ID]
     cpu_oracle_sample(w, steps=max(args.warmup, 0) or 1)  # warm-up
     base, times, _ = cpu_oracle_sample(w, steps=args.steps)
-    ms = statistics.mean(times) * (w.B * w.H) / base["cores"] * 1e3
+    ms_sample = statistics.mean(times) * 1e3  # one step as run: the bounded sample
     line = {
         "impl": "reference", "metric": METRIC, "value": base["value"], "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_sample, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name + " fwd+bwd", "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
-                   "chunk": 64, "variant": "gdn", "parallelism": "oracle threads over (b,h)"},
+        "config": workload_config(w, w.B, 1),
+        "step": f"the fp64 oracle (fwd + bwd) on {base['cores']} of the workload's {w.B * w.H} (b,h) sequences, "
+                "full length, one thread each",
+        "ms_per_step_whole_workload_extrapolated": ms_sample * (w.B * w.H) / base["cores"],
         "cpu_baseline": base,
         "e2e": {"value": base["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -518,14 +532,15 @@ def run_ours(args):
     dominant = max(kern_ms, key=kern_ms.get)
     f_ms = statistics.mean(fwd_ms)
     b_ms = statistics.mean(bwd_ms)
-    # Roofline of the gradient kernel (the largest share of the step): it reads every backward
-    # input (q, k, v, beta, the gate, dO, du) and writes every backward output (dq, dk, dv,
-    # dbeta, d log alpha), so its algorithmic bytes per launch are the per-token-head backward
-    # count times B*T*H; the states dS_T / dS0 belong to the reverse chain.
+    # Roofline of the gradient kernel (the largest share of the step): it reads the backward
+    # inputs q, k, v, beta, the gate and dO and writes every backward output (dq, dk, dv, dbeta,
+    # d log alpha), so its algorithmic bytes per launch are those per-token-head counts times
+    # B*T*H; du goes to the reverse chain (which hands the kernel dL/dU), and so do the states
+    # dS_T / dS0.
     rk = "bwd:k_bwd_chunk_tc"
     if rk not in kern_ms:  # another path (e.g. KDA): the whole backward call
         rk = None
-    r_bytes = cnt["bwd_io_bytes"] if rk else cnt["bwd_bytes"]
+    r_bytes = cnt["bwd_grad_kernel_bytes"] if rk else cnt["bwd_bytes"]
     rk_ms = kern_ms[rk] if rk else b_ms
     achieved = r_bytes / (rk_ms / 1e3) / 1e9
     r_label = rk.split(":", 1)[1] if rk else "backward call (" + "+".join(bwd_names) + ")"
@@ -552,9 +567,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": (w.name if B == w.B else w.name.replace(f"_B{w.B}_", f"_B{B}_")) + " fwd+bwd", "B": B, "T": T, "H": H, "dk": dk, "dv": dv, "chunk": C,
-                   "variant": vname, "io": "bf16, fp32 state", "l2": "flushed between steps (256 MiB write)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": workload_config(w, B, world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "kernel": r_label,
                      "alg_bytes_per_launch": r_bytes, "ms_per_launch": rk_ms,

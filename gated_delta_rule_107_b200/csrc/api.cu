@@ -59,27 +59,36 @@ bool use_kda_hybrid_bwd(const Geo &g, int dtype, int kind) {
 }
 size_t ws_al(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Parts of the split-path workspace (tc_path.cuh) that each call kind uses
+constexpr int GDN_SAVED = WS_FWD | WS_KEEP | WS_STATE;
+constexpr int KDA_FWD = WS_FWD | WS_KDA | WS_KDAC;
+constexpr int KDA_SAVED = WS_FWD | WS_STATE | WS_KDAC | WS_KDAG;
+
 size_t ws_bytes(const Geo &g, int dtype, int kind) {
     if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
     if (use_split(g, dtype)) {
         switch (kind) {
             case K_FWD: return tc_ws_bytes(g, WS_FWD);
-            case K_BWD: return tc_ws_bytes(g, WS_FWD | WS_KEEP | WS_REV);
+            case K_BWD: return tc_ws_bytes(g, GDN_SAVED | WS_REV);
             case K_FWD_SAVE: return 0;  // everything it keeps lives in the saved buffer
             default: return tc_ws_bytes(g, WS_REV);
         }
     }
-    if (use_split_kda(g, dtype, kind)) return tc_ws_bytes(g, WS_FWD | WS_KDA);
+    if (use_split_kda(g, dtype, kind))  // the saving forward keeps all but its forward-only tiles
+        return tc_ws_bytes(g, kind == K_FWD_SAVE ? WS_KDA : KDA_FWD);
     if (use_kda_hybrid_bwd(g, dtype, kind))
-        return ws_al(simt_ws_bytes(g, true)) + tc_ws_bytes(g, WS_FWD | WS_KEEP | WS_REV | WS_KDA);
+        return ws_al(simt_ws_bytes(g, true)) +
+               tc_ws_bytes(g, kind == K_BWD_SAVED ? WS_REV : WS_FWD | WS_STATE | WS_REV | WS_KDA | WS_KDAC);
     if (!is_bwd(kind) && use_tc_fwd(g, dtype)) return 0;
     return simt_ws_bytes(g, is_bwd(kind));
 }
 
 // Bytes of the saved-activation buffer (0: no saved form for this configuration).
 size_t saved_bytes(const Geo &g, int dtype) {
-    if (g.T == 0 || g.B == 0 || g.H == 0 || !use_split(g, dtype)) return 0;
-    return tc_ws_bytes(g, WS_FWD | WS_KEEP);
+    if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
+    if (use_split(g, dtype)) return tc_ws_bytes(g, GDN_SAVED);
+    if (tc_split_kda_supported(g, dtype == DR_BF16)) return tc_ws_bytes(g, KDA_SAVED);
+    return 0;
 }
 
 // Checks a caller buffer of `given` bytes against `need` (256-byte aligned when needed).
@@ -143,16 +152,21 @@ static int fwd_impl(const void *q, const void *k, const void *v, const void *alp
     t.q = q; t.k = k; t.v = v; t.alpha = alpha; t.beta = beta; t.S0 = S0; t.out = out; t.u = u; t.S_T = S_T;
     if (use_split(g, dtype)) {
         TcWs w = {};
-        if (save) tc_ws_carve(g, WS_FWD | WS_KEEP, saved, &w);
+        if (save) tc_ws_carve(g, GDN_SAVED, saved, &w);
         else tc_ws_carve(g, WS_FWD, workspace, &w);
         rc = launch_status(tc_chunk_prep(g, t, w, save, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, save ? 2 : 0, s, rec));
     } else if (use_split_kda(g, dtype, kind)) {
         TcWs w = {};
-        tc_ws_carve(g, WS_FWD | WS_KDA, workspace, &w);
-        rc = launch_status(tc_kda_gates(g, t, w, nullptr, s, rec));
+        if (save) {  // the chain operands, states and G go to the saved buffer
+            tc_ws_carve(g, KDA_SAVED, saved, &w);
+            tc_ws_carve(g, WS_KDA, workspace, &w);
+        } else {
+            tc_ws_carve(g, KDA_FWD, workspace, &w);
+        }
+        rc = launch_status(tc_kda_gates(g, t, w, save ? w.G : nullptr, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_chunk_prep(g, t, w, false, s, rec));
-        if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, 0, s, rec));
+        if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, save ? 2 : 0, s, rec));
     } else if (use_tc_fwd(g, dtype)) {
         rc = launch_status(tc_fwd(g, t, workspace, s, rec));
     } else {
@@ -194,22 +208,29 @@ static int bwd_impl(const void *q, const void *k, const void *v, const void *alp
     if (use_split(g, dtype)) {
         TcWs w = {};
         if (from_saved) {
-            tc_ws_carve(g, WS_FWD | WS_KEEP, const_cast<void *>(saved), &w);
+            tc_ws_carve(g, GDN_SAVED, const_cast<void *>(saved), &w);
             tc_ws_carve(g, WS_REV, workspace, &w);
         } else {
-            tc_ws_carve(g, WS_FWD | WS_KEEP | WS_REV, workspace, &w);
+            tc_ws_carve(g, GDN_SAVED | WS_REV, workspace, &w);
             rc = launch_status(tc_chunk_prep(g, t, w, true, s, rec));
             if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, 1, s, rec));
         }
         if (rc == DR_OK) rc = launch_status(tc_chain_rev(g, t, w, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_bwd_chunk(g, t, w, s, rec));
     } else if (use_kda_hybrid_bwd(g, dtype, kind)) {
-        const SimtWs sw = simt_ws_carve(g, true, workspace);
+        SimtWs sw = simt_ws_carve(g, true, workspace);
+        char *tcbase = (char *)workspace + ws_al(simt_ws_bytes(g, true));
         TcWs w = {};
-        tc_ws_carve(g, WS_FWD | WS_KEEP | WS_REV | WS_KDA, (char *)workspace + ws_al(simt_ws_bytes(g, true)), &w);
-        rc = launch_status(tc_kda_gates(g, t, w, sw.G, s, rec));
-        if (rc == DR_OK) rc = launch_status(tc_chunk_prep(g, t, w, false, s, rec));
-        if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, 1, s, rec));
+        if (from_saved) {  // the saving forward's chain operands, states and G
+            tc_ws_carve(g, KDA_SAVED, const_cast<void *>(saved), &w);
+            tc_ws_carve(g, WS_REV, tcbase, &w);
+            sw.G = w.G;
+        } else {
+            tc_ws_carve(g, WS_FWD | WS_STATE | WS_REV | WS_KDA | WS_KDAC, tcbase, &w);
+            rc = launch_status(tc_kda_gates(g, t, w, sw.G, s, rec));
+            if (rc == DR_OK) rc = launch_status(tc_chunk_prep(g, t, w, false, s, rec));
+            if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, 1, s, rec));
+        }
         // the CUDA-core gradient kernel reads W, U~, U, dU widened to fp32 and the state products
         if (rc == DR_OK) rc = launch_status(tc_to_simt(g, w, sw.W, sw.Ut, nullptr, nullptr, sw.Un, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_chain_rev(g, t, w, s, rec));
@@ -231,9 +252,10 @@ static int launch_plan(const Geo &g, int dtype, int kind, const char **names, in
     static const char *const SPLIT_BWD[4] = {"k_chunk_prep(keep)", "k_chain_fwd(recompute)", "k_chain_rev",
                                              "k_bwd_chunk_tc"};
     static const char *const SPLIT_BWD_SAVED[2] = {"k_chain_rev", "k_bwd_chunk_tc"};
-    static const char *const SPLIT_KDA_FWD[3] = {"k_kda_gates", "k_chunk_prep", "k_chain_fwd"};
-    static const char *const KDA_BWD[8] = {"k_kda_gates", "k_chunk_prep", "k_chain_fwd(recompute)", "k_widen",
-                                           "k_chain_rev", "k_widen", "k_state_tc", "k_bwd_intra"};
+    static const char *const SPLIT_KDA_FWD[4] = {"k_kda_gates", "k_kda_diag", "k_chunk_prep", "k_chain_fwd"};
+    static const char *const KDA_BWD[9] = {"k_kda_gates", "k_kda_diag", "k_chunk_prep", "k_chain_fwd(recompute)",
+                                           "k_widen", "k_chain_rev", "k_widen", "k_state_tc", "k_bwd_intra"};
+    static const char *const KDA_FWD_SAVE[4] = {"k_kda_gates", "k_kda_diag", "k_chunk_prep", "k_chain_fwd(keep)"};
     int n = 0;
     const char *const *src = nullptr;
     if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
@@ -245,11 +267,11 @@ static int launch_plan(const Geo &g, int dtype, int kind, const char **names, in
             default: src = SPLIT_BWD_SAVED; n = 2; break;
         }
     } else if (use_split_kda(g, dtype, kind)) {
-        src = SPLIT_KDA_FWD;
-        n = 3;
+        src = kind == K_FWD_SAVE ? KDA_FWD_SAVE : SPLIT_KDA_FWD;
+        n = 4;
     } else if (use_kda_hybrid_bwd(g, dtype, kind)) {
-        src = KDA_BWD;
-        n = 8;
+        src = kind == K_BWD_SAVED ? KDA_BWD + 4 : KDA_BWD;  // from saved: no recompute
+        n = kind == K_BWD_SAVED ? 5 : 9;
     } else if (!is_bwd(kind) && use_tc_fwd(g, dtype)) {
         return tc_fwd_launches(g, names, max_names);
     } else {

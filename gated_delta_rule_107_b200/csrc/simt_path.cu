@@ -798,8 +798,9 @@ __device__ __forceinline__ float clamp_half_range(float x) {
 // acc[u][v] += sum_{k < K1 + K2} A[(r0 + u) lda + k] B(k)[i0 + v]: one thread's 4 x 4 block of a
 // 64 x 64 product whose K columns come from B1 (ld1, K1 columns) and then B2 (ld2, K2 columns).
 // B passes through stg (64 x 65 floats) 64 columns at a time, the next block held in registers
-// while the current one is multiplied.  K1 and K2 are multiples of 64.  Opens with a barrier;
-// the caller synchronises before stg is written again.
+// while the current one is multiplied.  K1 and K2 are multiples of 64.  The first block of B is
+// read before the first barrier: a B in shared memory must be complete when nt64 is called.
+// The caller synchronises before stg is written again.
 __device__ __forceinline__ void nt64(const float *A, int lda, const float *B1, int ld1, int K1, const float *B2,
                                      int ld2, int K2, float *stg, int r0, int i0, float (&acc)[4][4]) {
     constexpr int LD = 65, PER = 64 * 64 / NT;
@@ -910,7 +911,10 @@ __device__ __forceinline__ void intra_tiled(const Geo &g, const IO<TI> &io, cons
     const int r0 = 4 * (tid >> 4), i0 = 4 * (tid & 15);
     {
         float acc[4][4] = {};
-        nt64(Kp, DK, Km, DK, DK, nullptr, 0, 0, dM, r0, i0, acc);  // its first barrier publishes the loads above
+        // nt64 reads its first block of B (here Km, written above by other threads) before its
+        // first barrier, so the loads are published here
+        __syncthreads();
+        nt64(Kp, DK, Km, DK, DK, nullptr, 0, 0, dM, r0, i0, acc);
 #pragma unroll
         for (int u = 0; u < 4; ++u)
 #pragma unroll

@@ -578,7 +578,7 @@ bool tc_split_supported(const Geo &g, bool bf16) {
 
 bool tc_split_kda_supported(const Geo &g, bool bf16) {
     return bf16 && g.C == 64 && g.dk == 128 && g.dv == 128 && g.variant == VAR_KDA &&
-           (size_t)g.B * g.H * g.N * 128 <= (size_t)INT_MAX;
+           (size_t)g.B * g.H * g.N * KDA_KH_ROWS <= (size_t)INT_MAX;
 }
 
 static size_t ws_al256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -598,6 +598,8 @@ static size_t ws_carve(const Geo &g, int parts, char *base, TcWs *w) {
     if (parts & WS_KEEP) {
         w->Tn = (__nv_bfloat16 *)take(nc * C * C * 2);
         w->KK = (__nv_bfloat16 *)take(nc * C * C * 2);
+    }
+    if (parts & WS_STATE) {
         w->Sn = (__nv_bfloat16 *)take(nc * DK * DV * 2);
         w->Un = (__nv_bfloat16 *)take(nc * C * DV * 2);
     }
@@ -607,10 +609,18 @@ static size_t ws_carve(const Geo &g, int parts, char *base, TcWs *w) {
         w->skt = (float *)take(nc * 2 * C * 4);
     }
     if (parts & WS_KDA) {
-        __nv_bfloat16 **tiles[] = {&w->Kt1, &w->Qt1, &w->Kh, &w->Kt, &w->Qt, &w->Kb};
+        __nv_bfloat16 **tiles[] = {&w->Kt1, &w->Qt1, &w->Kt};
         for (__nv_bfloat16 **t : tiles) *t = (__nv_bfloat16 *)take(nc * C * DK * 2);
+        w->Kh = (__nv_bfloat16 *)take(nc * KDA_KH_ROWS * DK * 2);
+        w->kwide = (int *)take(nc * 4);
+        w->Dx = (float *)take(nc * 2 * C * 16 * 4);
+    }
+    if (parts & WS_KDAC) {
+        w->Qt = (__nv_bfloat16 *)take(nc * C * DK * 2);
+        w->Kb = (__nv_bfloat16 *)take(nc * C * DK * 2);
         w->egc = (float *)take(nc * DK * 4);
     }
+    if (parts & WS_KDAG) w->G = (float *)take(nc * C * DK * 4);
     return off;
 }
 
@@ -626,7 +636,6 @@ cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, int mode
     FMaps mp;
     const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;
     const bool out = mode != 1, keep = mode != 0, kda = g.variant == VAR_KDA;
-    if (kda && mode == 2) return cudaErrorInvalidValue;  // no saved form for KDA
     bool ok = (kda ? tc::make_map_2d_bf16(&mp.q, w.Qt, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.k, w.Kb, DK, NC * C, 64)
                    : tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) &&
                          tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64)) &&
@@ -654,7 +663,7 @@ cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, int mode
         kern<<<grid, NTHREADS, smem, s>>>(mp, a);
         return cudaSuccess;
     };
-    if (kda) e = mode == 0 ? go(k_chain_fwd<0, 1>) : go(k_chain_fwd<1, 1>);
+    if (kda) e = mode == 0 ? go(k_chain_fwd<0, 1>) : mode == 1 ? go(k_chain_fwd<1, 1>) : go(k_chain_fwd<2, 1>);
     else if (mode == 0) e = go(k_chain_fwd<0, 0>);
     else if (mode == 1) e = go(k_chain_fwd<1, 0>);
     else e = go(k_chain_fwd<2, 0>);

@@ -9,8 +9,8 @@
 // obtained by stacking two 64-row operands:
 //
 //   P1   [beta k ; q] . k^T          -> A (rows 0-63), P (rows 64-127)
-//        (Gated / DeltaNet: the gate factor e^{g_r - g_i} <= 1 is applied
-//         exactly in the epilogue; KDA: the operands carry e^{+-(g - g_mid)})
+//        (the scalar gate factor e^{g_r - g_i} <= 1 is applied exactly in the
+//         epilogue)
 //   T  = (I + A)^-1                    blocked forward substitution (CUDA cores)
 //   IPT  R = [I ; P] . T  = [T ; P T]
 //   P3   X = R . (beta e^{g} k)       -> [W ; P W]
@@ -21,8 +21,11 @@
 //   C3   E = Kbar^T . U                (Kbar = k e^{g_C - g})
 //        S <- Diag(e^{g_C}) S + E      (fp32, registers)
 //
-// Warp roles: warp 0 = producer (TMA loads of q, k, v and, for KDA, the gate
-// tile; plain loads of the scalar gate and beta); warps 1-4 = one warpgroup
+// Serves Gated DeltaNet and DeltaNet (KDA's channel-wise gates take the split
+// path at dv = 128 and the CUDA-core path otherwise).
+//
+// Warp roles: warp 0 = producer (TMA loads of q, k, v; plain loads of the
+// scalar gate and beta); warps 1-4 = one warpgroup
 // that does all epilogues / CUDA-core work and issues the MMAs from one elected
 // thread.  Every wait is bounded (about 1 s); on expiry the kernel raises the
 // device error word and leaves through the common teardown (TMEM freed).
@@ -55,7 +58,6 @@ constexpr uint32_t OFF_U = OFF_AC + 32768;     //  8K  U (64 token rows, 1 panel
 constexpr uint32_t OFF_S = OFF_U + 8192;       // 16K  bf16 S (128 rows, 1 panel)
 constexpr uint32_t OFF_MISC = OFF_S + 16384;   //  4K  barriers and small vectors
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 4096;
-constexpr uint32_t KDA_G = SLOT;               // KDA uses one input slot; its gate tile sits in the second
 
 // misc sub-offsets
 constexpr uint32_t M_BAR = 0;      // 8 mbarriers
@@ -65,8 +67,7 @@ constexpr uint32_t M_GB = 128;     // [2 slots][2][64] floats: raw log gate, bet
 constexpr uint32_t M_GC = M_GB + 1024;    // [64] cumulative g (Gated)
 constexpr uint32_t M_FAC = M_GC + 256;    // [4][64] row factors: beta, beta e^g, e^{gC-g}, e^g
 constexpr uint32_t M_GAM = M_FAC + 1024;  // [128] e^{g_C} per channel
-constexpr uint32_t M_EGM = M_GAM + 512;   // [128] e^{g_mid} per channel (KDA)
-static_assert(M_EGM + 512 <= 4096, "misc overflow");
+static_assert(M_GAM + 512 <= 4096, "misc overflow");
 
 // TMEM columns
 constexpr uint32_t TM_G1 = 0;    // 64: P1 output, then R
@@ -79,7 +80,7 @@ constexpr uint32_t TM_COLS = 512;
 enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_VFULL, B_VEMPTY, B_MMA, B_NUM };
 
 struct Args {
-    const void *alpha;   // raw log gate (Gated: [B,T,H]); KDA uses the tensor map
+    const void *alpha;   // raw log gate (Gated: [B,T,H])
     const void *beta;    // [B,T,H]
     const float *S0;     // [B,H,dk,dv] or null
     void *out, *u;       // [B,T,H,dv]
@@ -90,10 +91,11 @@ struct Args {
 template <int VAR>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_fwd_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g, Args a) {
+             const __grid_constant__ CUtensorMap tm_v, Args a) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    constexpr int NSLOT = (VAR == VAR_KDA) ? 1 : 2;
+    static_assert(VAR != VAR_KDA, "channel-wise gates take the split or the CUDA-core path");
+    constexpr int NSLOT = 2;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_MISC + M_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + M_TMEM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + M_ABORT);
@@ -101,7 +103,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     float *gc = reinterpret_cast<float *>(sm + OFF_MISC + M_GC);
     float *fac = reinterpret_cast<float *>(sm + OFF_MISC + M_FAC);    // [4][64]
     float *gam = reinterpret_cast<float *>(sm + OFF_MISC + M_GAM);
-    float *egm = reinterpret_cast<float *>(sm + OFF_MISC + M_EGM);
 
     const int half = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int j0 = half * DVB;
@@ -131,7 +132,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
-            if (VAR == VAR_KDA) prefetch_tmap(&tm_g);
         }
         int issued[2] = {0, 0}, v_issued = 0;
         for (int m = 0; m < N; ++m) {
@@ -141,16 +141,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!ok) break;
             unsigned char *slot = sm + s * SLOT;
             if (lane == 0) {
-                const uint32_t bytes = (VAR == VAR_KDA) ? 3 * 16384 : 2 * 16384;
+                const uint32_t bytes = 2 * 16384;
                 mbar_arrive_tx(&bar[B_FULL0 + s], bytes);
                 tma_load_4d(slot + IN_Q, &tm_q, 0, h, t0, b, &bar[B_FULL0 + s]);
                 tma_load_4d(slot + IN_Q + 8192, &tm_q, 64, h, t0, b, &bar[B_FULL0 + s]);
                 tma_load_4d(slot + IN_K, &tm_k, 0, h, t0, b, &bar[B_FULL0 + s]);
                 tma_load_4d(slot + IN_K + 8192, &tm_k, 64, h, t0, b, &bar[B_FULL0 + s]);
-                if (VAR == VAR_KDA) {
-                    tma_load_4d(sm + KDA_G, &tm_g, 0, h, t0, b, &bar[B_FULL0 + s]);
-                    tma_load_4d(sm + KDA_G + 8192, &tm_g, 64, h, t0, b, &bar[B_FULL0 + s]);
-                }
             }
             float *gbs = gb + s * 128;
             for (int r = lane; r < C; r += 32) {
@@ -226,85 +222,49 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (wg_abort()) break;
             const float *lg = gb + s * 128, *bt = gb + s * 128 + 64;
             // ------------------------------ M1: gates and operand tiles ------------------------------
-            if (VAR != VAR_KDA) {
-                if (wt < 32) {
-                    // inclusive scan of the 64 log gates (two per lane)
-                    float x0 = lg[lane], x1 = lg[lane + 32];
+            if (wt < 32) {
+                // inclusive scan of the 64 log gates (two per lane)
+                float x0 = lg[lane], x1 = lg[lane + 32];
 #pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const float y0 = __shfl_up_sync(0xffffffffu, x0, o);
-                        const float y1 = __shfl_up_sync(0xffffffffu, x1, o);
-                        if (lane >= o) { x0 += y0; x1 += y1; }
-                    }
-                    x1 += __shfl_sync(0xffffffffu, x0, 31);
-                    const float gC = __shfl_sync(0xffffffffu, x1, 31);
-                    gc[lane] = x0;
-                    gc[lane + 32] = x1;
-                    fac[0 * 64 + lane] = bt[lane];
-                    fac[0 * 64 + lane + 32] = bt[lane + 32];
-                    fac[1 * 64 + lane] = bt[lane] * __expf(x0);
-                    fac[1 * 64 + lane + 32] = bt[lane + 32] * __expf(x1);
-                    fac[2 * 64 + lane] = __expf(gC - x0);
-                    fac[2 * 64 + lane + 32] = __expf(gC - x1);
-                    fac[3 * 64 + lane] = __expf(x0);
-                    fac[3 * 64 + lane + 32] = __expf(x1);
-                    const float eg = __expf(gC);
-                    for (int c = lane; c < DK; c += 32) gam[c] = eg;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y0 = __shfl_up_sync(0xffffffffu, x0, o);
+                    const float y1 = __shfl_up_sync(0xffffffffu, x1, o);
+                    if (lane >= o) { x0 += y0; x1 += y1; }
                 }
-                wg_sync();
-                // q, k -> [beta k ; q], beta e^g k, Kbar ; 64 rows x 16 chunks
-                for (int x = wt; x < C * 16; x += 128) {
-                    const int r = x >> 4, j = x & 15, p = j >> 3;
-                    const uint32_t o = (uint32_t)p * 8192 + swz(r, j & 7);
-                    float kv[8], qv[8], w[8];
-                    ld_chunk(slot + IN_K, o, kv);
-                    ld_chunk(slot + IN_Q, o, qv);
-                    const float f0 = fac[r], f1 = fac[64 + r], f2 = fac[128 + r];
+                x1 += __shfl_sync(0xffffffffu, x0, 31);
+                const float gC = __shfl_sync(0xffffffffu, x1, 31);
+                gc[lane] = x0;
+                gc[lane + 32] = x1;
+                fac[0 * 64 + lane] = bt[lane];
+                fac[0 * 64 + lane + 32] = bt[lane + 32];
+                fac[1 * 64 + lane] = bt[lane] * __expf(x0);
+                fac[1 * 64 + lane + 32] = bt[lane + 32] * __expf(x1);
+                fac[2 * 64 + lane] = __expf(gC - x0);
+                fac[2 * 64 + lane + 32] = __expf(gC - x1);
+                fac[3 * 64 + lane] = __expf(x0);
+                fac[3 * 64 + lane + 32] = __expf(x1);
+                const float eg = __expf(gC);
+                for (int c = lane; c < DK; c += 32) gam[c] = eg;
+            }
+            wg_sync();
+            // q, k -> [beta k ; q], beta e^g k, Kbar ; 64 rows x 16 chunks
+            for (int x = wt; x < C * 16; x += 128) {
+                const int r = x >> 4, j = x & 15, p = j >> 3;
+                const uint32_t o = (uint32_t)p * 8192 + swz(r, j & 7);
+                float kv[8], qv[8], w[8];
+                ld_chunk(slot + IN_K, o, kv);
+                ld_chunk(slot + IN_Q, o, qv);
+                const float f0 = fac[r], f1 = fac[64 + r], f2 = fac[128 + r];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) w[e] = f0 * kv[e];
-                    st_chunk(sm + OFF_PA, (uint32_t)p * 16384 + swz(r, j & 7), w);
-                    st_chunk(sm + OFF_PA, (uint32_t)p * 16384 + 8192 + swz(r, j & 7), qv);
+                for (int e = 0; e < 8; ++e) w[e] = f0 * kv[e];
+                st_chunk(sm + OFF_PA, (uint32_t)p * 16384 + swz(r, j & 7), w);
+                st_chunk(sm + OFF_PA, (uint32_t)p * 16384 + 8192 + swz(r, j & 7), qv);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) w[e] = f1 * kv[e];
-                    st_chunk(sm + OFF_BKT, o, w);
+                for (int e = 0; e < 8; ++e) w[e] = f1 * kv[e];
+                st_chunk(sm + OFF_BKT, o, w);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) w[e] = f2 * kv[e];
-                    st_chunk(sm + OFF_KB, o, w);
-                }
-            } else {
-                // KDA: thread wt owns channel c; two passes over the 64 tokens
-                const int c = wt;
-                const uint32_t cp = (uint32_t)(c >> 6) * 8192, cc = (uint32_t)((c & 63) >> 3), ce = (uint32_t)(c & 7) * 2;
-                const unsigned char *gt = sm + KDA_G;
-                float run = 0.f, gmid = 0.f;
-                for (int r = 0; r < C; ++r) {
-                    run += __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(gt + cp + swz(r, cc) + ce));
-                    if (r == 31) gmid = run;
-                }
-                const float gC = run;
-                gam[c] = __expf(gC);
-                egm[c] = __expf(gmid);
-                run = 0.f;
-                for (int r = 0; r < C; ++r) {
-                    const uint32_t o = cp + swz(r, cc) + ce;
-                    run += __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(gt + o));
-                    const float e1 = __expf(fminf(run - gmid, 80.f));      // e^{g - g_mid}
-                    const float e2 = __expf(fminf(gmid - run, 80.f));      // e^{g_mid - g}
-                    const float e3 = __expf(run);                          // e^{g}
-                    const float e4 = __expf(gC - run);                     // e^{g_C - g}
-                    __nv_bfloat16 *kp = reinterpret_cast<__nv_bfloat16 *>(slot + IN_K + o);
-                    const float kv = __bfloat162float(*kp);
-                    const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(slot + IN_Q + o));
-                    const float br = bt[r];
-                    const uint32_t pa = (uint32_t)(c >> 6) * 16384 + swz(r, cc) + ce;
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_PA + pa) = __float2bfloat16_rn(br * kv * e1);
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_PA + pa + 8192) = __float2bfloat16_rn(qv * e1);
-                    *kp = __float2bfloat16_rn(kv * e2);
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_BKT + o) = __float2bfloat16_rn(br * kv * e3);
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_KB + o) = __float2bfloat16_rn(kv * e4);
-                }
-                if (wt < 64) fac[wt] = bt[wt];
-                wg_sync();
+                for (int e = 0; e < 8; ++e) w[e] = f2 * kv[e];
+                st_chunk(sm + OFF_KB, o, w);
             }
             fence_proxy_async();
             wg_sync();
@@ -485,7 +445,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             ld_chunk(sm + OFF_PA, (uint32_t)half2 * 16384 + 8192 + swz(rr, ch), qv);
 #pragma unroll
                             for (int e = 0; e < 8; ++e) {
-                                const float sc = (VAR == VAR_KDA) ? egm[half2 * 64 + ch * 8 + e] : fac[192 + rr];
+                                const float sc = fac[192 + rr];
                                 xv[ch * 8 + e] = qv[e] * sc - xv[ch * 8 + e];
                             }
                         }
@@ -599,7 +559,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }  // namespace tcf
 
 bool tc_fwd_supported(const Geo &g, bool bf16) {
-    return bf16 && g.C == tcf::C && g.dk == tcf::DK && (g.dv == 64 || g.dv == 128);
+    return bf16 && g.C == tcf::C && g.dk == tcf::DK && (g.dv == 64 || g.dv == 128) && g.variant != VAR_KDA;
 }
 
 int tc_fwd_launches(const Geo &g, const char **names, int max_names) {
@@ -611,13 +571,11 @@ int tc_fwd_launches(const Geo &g, const char **names, int max_names) {
 cudaError_t tc_fwd(const Geo &g, const Tensors &t, void *workspace, cudaStream_t s, Rec &rec) {
     using namespace tcf;
 
-    CUtensorMap mq, mk, mv, mg;
+    CUtensorMap mq, mk, mv;
     const uint64_t Bn = g.B, T = g.T, H = g.H;
     bool ok = tc::make_map_4d_bf16(&mq, t.q, DK, H, T, Bn, 64) && tc::make_map_4d_bf16(&mk, t.k, DK, H, T, Bn, 64) &&
               tc::make_map_4d_bf16(&mv, t.v, g.dv, H, T, Bn, 64);
-    if (ok && g.variant == VAR_KDA) ok = tc::make_map_4d_bf16(&mg, t.alpha, DK, H, T, Bn, 64);
-    else mg = mq;
-    if (!ok) return cudaErrorInvalidValue;
+    if (!ok || g.variant == VAR_KDA) return cudaErrorInvalidValue;
     Args a;
     a.alpha = t.alpha; a.beta = t.beta; a.S0 = t.S0; a.out = t.out; a.u = t.u; a.ST = t.S_T;
     a.B = g.B; a.T = g.T; a.H = g.H; a.dv = g.dv; a.N = g.N;
@@ -629,20 +587,16 @@ cudaError_t tc_fwd(const Geo &g, const Tensors &t, void *workspace, cudaStream_t
             e = cudaFuncSetAttribute(k_fwd_tc<VAR_DELTANET>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
             rec.mark(s);
-            k_fwd_tc<VAR_DELTANET><<<grid, NTHREADS, smem, s>>>(mq, mk, mv, mg, a);
+            k_fwd_tc<VAR_DELTANET><<<grid, NTHREADS, smem, s>>>(mq, mk, mv, a);
             break;
         case VAR_GATED:
             e = cudaFuncSetAttribute(k_fwd_tc<VAR_GATED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
             rec.mark(s);
-            k_fwd_tc<VAR_GATED><<<grid, NTHREADS, smem, s>>>(mq, mk, mv, mg, a);
+            k_fwd_tc<VAR_GATED><<<grid, NTHREADS, smem, s>>>(mq, mk, mv, a);
             break;
         default:
-            e = cudaFuncSetAttribute(k_fwd_tc<VAR_KDA>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-            rec.mark(s);
-            k_fwd_tc<VAR_KDA><<<grid, NTHREADS, smem, s>>>(mq, mk, mv, mg, a);
-            break;
+            return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
 }

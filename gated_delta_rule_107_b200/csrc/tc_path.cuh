@@ -2,7 +2,8 @@
 //
 // Gated DeltaNet and DeltaNet at dv = 128 run the split path: a per-chunk kernel over all
 // chunks at once (tc_prep.cu), the serial state chains (tc_chain.cu) and, for the
-// backward, the per-chunk gradient kernel (tc_bwd.cu); api.cu sequences them.  KDA and
+// backward, the per-chunk gradient kernel (tc_bwd.cu); api.cu sequences them.  KDA at
+// dv = 128 runs the split forward after its gate kernels; Gated DeltaNet and DeltaNet at
 // dv = 64 run the single-kernel forward of tc_fwd.cu.
 #pragma once
 #include "dr_common.cuh"
@@ -10,7 +11,7 @@
 namespace dr {
 
 bool tc_fwd_supported(const Geo &g, bool bf16);
-// the single-kernel forward (KDA, and Gated DeltaNet / DeltaNet at dv = 64); no workspace
+// the single-kernel forward (Gated DeltaNet / DeltaNet, bf16, dk = 128); no workspace
 cudaError_t tc_fwd(const Geo &g, const Tensors &t, void *workspace, cudaStream_t s, Rec &rec);
 // number of launches of tc_fwd and their names
 int tc_fwd_launches(const Geo &g, const char **names, int max_names);
@@ -22,13 +23,19 @@ bool tc_split_supported(const Geo &g, bool bf16);
 bool tc_split_kda_supported(const Geo &g, bool bf16);
 
 // Workspace of the split path, chunk-major (ci = (b H + h) N + n), every matrix row-major:
-// bf16 tiles that later kernels load with TMA, plus fp32 per-token factors.  Three parts:
-//   WS_FWD   the forward's chunk products (gb, W, Ut, P);
-//   WS_KEEP  what the backward needs from the forward besides them (Tn, KK, Sn, Un);
-//   WS_REV   what the reverse chain hands the gradient kernel (dSn, dUn, skt).
-// The forward's workspace is WS_FWD; the recomputing backward's all three; the saved
-// activations of delta_rule_fwd_save are WS_FWD | WS_KEEP, and the backward from them needs
-// WS_REV as workspace.
+// bf16 tiles that later kernels load with TMA, plus fp32 per-token factors.  Parts:
+//   WS_FWD    the forward's chunk products (gb, W, Ut, P);
+//   WS_KEEP   the chunk products only the scalar-gate gradient kernel reads (Tn, KK);
+//   WS_STATE  the chunk states and write values of the forward chain (Sn, Un);
+//   WS_REV    what the reverse chain hands the gradient kernels (dSn, dUn, skt);
+//   WS_KDA    KDA's forward-only gate-scaled operands (Kt1, Qt1, Kh, Kt, kwide, Dx);
+//   WS_KDAC   KDA's operands of both chains (Qt, Kb, egc);
+//   WS_KDAG   KDA's in-chunk cumulative log gate G (fp32, read by its gradient kernel).
+// Gated DeltaNet / DeltaNet: the forward's workspace is WS_FWD; the recomputing backward's
+// FWD | KEEP | STATE | REV; the saved activations of delta_rule_fwd_save are FWD | KEEP | STATE,
+// and the backward from them needs WS_REV as workspace.  KDA: the forward's workspace is
+// FWD | KDA | KDAC; the saved activations are FWD | STATE | KDAC | KDAG (the saving forward's
+// workspace WS_KDA), and the backward from them needs WS_REV beside the CUDA-core workspace.
 struct TcWs {
     float *gb;           // [ci][2][C]    in-chunk cumulative log gate g, then beta
     __nv_bfloat16 *W;    // [ci][C][dk]   W  = T diag(beta e^g) k
@@ -41,24 +48,41 @@ struct TcWs {
     __nv_bfloat16 *dSn;  // [ci][dk][dv]  dL/dS of the state leaving chunk n
     __nv_bfloat16 *dUn;  // [ci][C][dv]   dL/dU = du + P^T dO + Kbar dS_{n+1}
     float *skt;          // [ci][2][C]    per 64-column half of dv: U_r . (Kbar dS_{n+1})_r
-    // KDA forward (channel-wise gates, g = in-chunk cumulative log gate per key channel,
-    // g_m its value at the chunk's middle token, exponents clamped to [-80, 80]):
-    __nv_bfloat16 *Kt1;  // [ci][C][dk]   k e^{g - g_m}      (rows of P1's A)
-    __nv_bfloat16 *Qt1;  // [ci][C][dk]   q e^{g - g_m}      (rows of P1's A)
-    __nv_bfloat16 *Kh;   // [ci][C][dk]   k e^{g_m - g}      (P1's B)
-    __nv_bfloat16 *Kt;   // [ci][C][dk]   k e^{g}            (W = T diag(beta) Kt)
-    __nv_bfloat16 *Qt;   // [ci][C][dk]   q e^{g}            (o = Qt S + P U)
-    __nv_bfloat16 *Kb;   // [ci][C][dk]   k e^{g_C - g}      (S+ = Diag(e^{g_C}) S + Kb^T U)
+    // KDA forward (channel-wise gates, g = in-chunk cumulative log gate per key channel).  The
+    // pair factor e^{g_r - g_i} is split at a reference token of row r's 16-token block,
+    // b(r) = 16 floor(r / 16):  e^{g_r - g_b(r)} e^{g_b(r) - g_i}.  For i before the block both
+    // factors are <= 1; inside the block the second is >= 1 (at most e^{the block's span}).
+    __nv_bfloat16 *Kt1;  // [ci][C][dk]   k e^{g - g_b}            (rows of P1's A)
+    __nv_bfloat16 *Qt1;  // [ci][C][dk]   q e^{g - g_b}            (rows of P1's A)
+    __nv_bfloat16 *Kh;   // [ci][KDA_KH_ROWS][dk]  P1's B: four sections, section R (R = 0..3)
+                         //               at row 8 R (R + 1), rows i = 0 .. 16 R + 15:
+                         //               k_i e^{g_16R - g_i} (exponent clamped at 80)
+    __nv_bfloat16 *Kt;   // [ci][C][dk]   k e^{g}                  (W = T diag(beta) Kt)
+    __nv_bfloat16 *Qt;   // [ci][C][dk]   q e^{g}                  (o = Qt S + P U)
+    __nv_bfloat16 *Kb;   // [ci][C][dk]   k e^{g_C - g}            (S+ = Diag(e^{g_C}) S + Kb^T U)
     float *egc;          // [ci][dk]      e^{g_C}
+    int *kwide;          // [ci]          1: some channel's gate falls by more than KDA_DIAG_SPAN
+                         //               inside a 16-token block (the in-block factors would
+                         //               leave the range where the split is exact)
+    float *Dx;           // [ci][2][C][16] for such chunks only: the exact in-block sums
+                         //               sum_c k_rc k_ic e^{g_rc - g_ic} ([0]) and
+                         //               sum_c q_rc k_ic e^{g_rc - g_ic} ([1]), i = b(r) + 0..15
+    float *G;            // [ci][C][dk]   KDA: g itself (fp32)
 };
-enum { WS_FWD = 1, WS_KEEP = 2, WS_REV = 4, WS_KDA = 8 };
-// Bytes of the given parts, laid out one after another in the order FWD, KEEP, REV.
+// rows of the stacked KDA column operand (16 + 32 + 48 + 64), and the widest in-block fall of
+// a channel's cumulative log gate (nats) for which the block-reference split is used as is
+constexpr int KDA_KH_ROWS = 160;
+constexpr float KDA_DIAG_SPAN = 64.f;
+enum { WS_FWD = 1, WS_KEEP = 2, WS_REV = 4, WS_KDA = 8, WS_STATE = 16, WS_KDAC = 32, WS_KDAG = 64 };
+// Bytes of the given parts, laid out one after another in the order FWD, KEEP, STATE, REV, KDA,
+// KDAC, KDAG.
 size_t tc_ws_bytes(const Geo &g, int parts);
 // Sets the pointers of the given parts, carved from base in that order; leaves the others.
 void tc_ws_carve(const Geo &g, int parts, void *base, TcWs *w);
 
-// KDA's gate-scaled operands of every chunk (tc_prep.cu): w.Kt1 ... w.Kb, w.egc; with G
-// (fp32 [chunks][64][dk], may be null) also the in-chunk cumulative log gate itself.
+// KDA's gate-scaled operands of every chunk (tc_prep.cu): w.Kt1 ... w.Kb, w.egc, w.kwide; with G
+// (fp32 [chunks][64][dk], may be null) also the in-chunk cumulative log gate itself.  Then, for
+// the chunks marked in w.kwide, the exact in-block sums w.Dx (a second kernel; the others exit).
 cudaError_t tc_kda_gates(const Geo &g, const Tensors &t, const TcWs &w, float *G, cudaStream_t s, Rec &rec);
 // fp32 copies of the forward's chunk products and states (W, U~, P, S_n, U) for the CUDA-core
 // backward kernels (tc_prep.cu).

@@ -10,10 +10,17 @@
 //   W  = T diag(beta e^g) k,   U~ = T diag(beta) v
 //   backward (and a forward that saves for it): T and k k^T kept for the gradient kernel.
 // KDA's gates are per key channel, so they cannot leave the dot products as scalars: a
-// first kernel (k_kda_gates) writes the gate-scaled operands, and the same products become
-//   P1 = [k e^{g-g_m} ; q e^{g-g_m}] . (k e^{g_m-g})^T,   W = T diag(beta) (k e^g)
-// with g per channel and g_m its value at the chunk's middle token (the midpoint split
-// keeps every factor within e^{+-80}: exponents are clamped there).
+// first kernel (k_kda_gates) writes the gate-scaled operands.  The pair factor of row r and
+// column i <= r is split at the first token b = 16 floor(r / 16) of r's 16-token block,
+// e^{g_r - g_i} = e^{g_r - g_b} e^{g_b - g_i} (log-space gates, section 7.1; second-level
+// blocking, section 2.2): the row factor is <= 1, and so is the column factor for every i
+// before the block.  Each block of rows has its own column operand, so P1 becomes one N = 160
+// product against the four column operands stacked,
+//   P1 = [k e^{g - g_b} ; q e^{g - g_b}] . [K_0 ; K_1 ; K_2 ; K_3]^T,   K_R = k_i e^{g_16R - g_i}
+// (i = 0 .. 16 R + 15), of which row r reads the section of its block; W = T diag(beta) (k e^g).
+// Inside a block the column factor is at most e^{the block's fall}; a chunk where some channel
+// falls by more than KDA_DIAG_SPAN inside a block takes its in-block entries from exact
+// per-pair sums instead (k_kda_diag).
 //
 // Every chunk is independent, so the grid covers all chunks of all heads at once (two
 // CTAs per SM); the serial state chains (tc_chain.cu) then only carry the state.  The
@@ -43,8 +50,11 @@ constexpr uint32_t OFF_V = 32768;      // 16K v [i][j]
 constexpr uint32_t OFF_F = 49152;      // 32K fp32 A | T (inverse), then staging W [r][c] | U~ [r][j]
 constexpr uint32_t OFF_P = 81920;      //  8K P [r][i]
 constexpr uint32_t OFF_MISC = 90112;   //  2K
-constexpr uint32_t OFF_X = 92160;      // 16K KDA: k e^{g_m - g} (P1's B), then k e^g (W's B)
+constexpr uint32_t OFF_X = 92160;      // 16K KDA: k e^g (W's B)
+constexpr uint32_t OFF_KH = OFF_F;     // 40K KDA: P1's stacked B (two panels of 160 rows), over F and P
+constexpr uint32_t KH_PANEL = KDA_KH_ROWS * 128;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 2048, SMEM_KDA = OFF_X + 16384;
+static_assert(OFF_P == OFF_F + 32768 && OFF_KH + 2 * KH_PANEL <= OFF_MISC, "the KDA B operand spans F and P");
 // misc
 constexpr uint32_t M_BAR = 0;          // [0] loads, [1] MMA
 constexpr uint32_t M_TMEM = 64, M_ABORT = 68, M_BIG = 72;
@@ -59,14 +69,20 @@ struct Maps {
     CUtensorMap W, Ut;    // [chunks * 64][128] bf16; box 64 x 64 (stores)
     CUtensorMap P;        // [chunks * 64][64] bf16; box 64 x 64 (store)
     CUtensorMap KK, Tn;   // [chunks * 64][64] bf16; box 64 x 64 (stores, when KEEP)
-    CUtensorMap Kt1, Qt1, Kh, Kt;  // KDA: [chunks * 64][128] bf16 gate-scaled operands; box 64 x 64
+    CUtensorMap Kt1, Qt1, Kt;  // KDA: [chunks * 64][128] bf16 gate-scaled operands; box 64 x 64
+    CUtensorMap Kh;            // KDA: [chunks * 160][128] bf16; box 64 x 160
 };
 
 struct Args {
     const void *alpha, *beta;       // bf16 [B, T, H]
     float *gb;                      // [chunks][2][64]: g, beta
+    const int *kwide;               // KDA: [chunks] in-block sums from Dx
+    const float *Dx;                // KDA: [chunks][2][64][16]
     int B, T, H, N;
 };
+
+// first column of block R's section of the KDA product (16 R (R + 1) / 2)
+__host__ __device__ constexpr uint32_t kda_sec(int R) { return (uint32_t)(8 * R * (R + 1)); }
 
 // KEEP: also store T and k k^T (for the backward)
 template <int VAR, int KEEP>
@@ -84,23 +100,23 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
     const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int T = a.T, H = a.H, t0 = n * C, L = min(C, T - t0);
-    const int ci = (b * H + h) * a.N + n;  // < 2^31 / 128 (checked by the launcher)
+    const int ci = (b * H + h) * a.N + n;  // ci * 160 < 2^31 (checked by the launcher)
     const int trow = tid;                  // TMEM lane of this thread
 
-    int mma_issued = 0, kt_issued = 0;
+    int mma_issued = 0;
     if (tid == 0) {
         mbar_init(&bar[0], 1);
         mbar_init(&bar[1], 1);
-        mbar_init(&bar[2], 1);
         *abort_flag = 0;
         fence_mbar_init();
-        mbar_arrive_tx(&bar[0], VAR == VAR_KDA ? 65536u : 49152u);
+        mbar_arrive_tx(&bar[0], VAR == VAR_KDA ? 65536u + 2 * KH_PANEL : 49152u);
 #pragma unroll
         for (int p = 0; p < 2; ++p) {
             if (VAR == VAR_KDA) {  // the gate-scaled operands of tc_kda_gates
                 tma_load_2d(sm + OFF_KQ + p * 16384, &mp.Kt1, 64 * p, ci * C, &bar[0]);
                 tma_load_2d(sm + OFF_KQ + p * 16384 + 8192, &mp.Qt1, 64 * p, ci * C, &bar[0]);
-                tma_load_2d(sm + OFF_X + p * 8192, &mp.Kh, 64 * p, ci * C, &bar[0]);
+                tma_load_2d(sm + OFF_KH + p * KH_PANEL, &mp.Kh, 64 * p, ci * KDA_KH_ROWS, &bar[0]);
+                tma_load_2d(sm + OFF_X + p * 8192, &mp.Kt, 64 * p, ci * C, &bar[0]);
             } else {
                 tma_load_4d(sm + OFF_KQ + p * 16384, &mp.k, 64 * p, h, t0, b, &bar[0]);
                 tma_load_4d(sm + OFF_KQ + p * 16384 + 8192, &mp.q, 64 * p, h, t0, b, &bar[0]);
@@ -172,30 +188,55 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
     const uint32_t skq = smem_u32(sm + OFF_KQ), sv = smem_u32(sm + OFF_V);
 
     bool ok = consensus(mbar_wait(&bar[0], 0, abort_flag));
-    // ---------------- P1: [k ; q] . k^T ----------------
+    // ---------------- P1: [k ; q] . k^T (KDA: against the four stacked sections) ----------------
     if (ok && tid == 0) {
-        const uint32_t id = idesc_bf16(128, 64, 0, 0);
-        const uint32_t sx = smem_u32(sm + OFF_X);
+        const uint32_t id = idesc_bf16(128, VAR == VAR_KDA ? KDA_KH_ROWS : 64, 0, 0);
+        const uint32_t skh = smem_u32(sm + OFF_KH);
 #pragma unroll
         for (int st = 0; st < 8; ++st) {
             const uint32_t ad = skq + (st >> 2) * 16384 + (st & 3) * 32;
-            const uint32_t bd = VAR == VAR_KDA ? sx + (st >> 2) * 8192 + (st & 3) * 32 : ad;
+            const uint32_t bd = VAR == VAR_KDA ? skh + (st >> 2) * KH_PANEL + (st & 3) * 32 : ad;
             mma_bf16(tbase + TM_G1, sdesc(ad, 16, 1024), sdesc(bd, 16, 1024), id, st > 0);
         }
         mma_commit(&bar[1]);
         mma_issued++;
     }
     if (ok) ok = consensus(wait_mma());
-    if (VAR == VAR_KDA && ok && tid == 0) {  // k e^g, the B of W's product, over the finished B of P1
-        mbar_arrive_tx(&bar[2], 16384u);
-#pragma unroll
-        for (int p = 0; p < 2; ++p) tma_load_2d(sm + OFF_X + p * 8192, &mp.Kt, 64 * p, ci * C, &bar[2]);
-        kt_issued = 1;
-    }
     // ---------------- A (fp32, for the inverse), P (bf16 tile), k k^T ----------------
     if (ok) {
         float g1[64];
-        tmem_row64(tl + TM_G1, g1);
+        if (VAR == VAR_KDA) {
+            // lanes 0-15 of this warp hold rows of block R0, lanes 16-31 of block R0 + 1; each
+            // reads columns i = 0 .. 16 R + 15 of its block's section (the rest of the row is 0)
+            const int R0 = 2 * (warp & 1);
+            const bool first = lane < 16;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float x0[16], x1[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) x0[e] = x1[e] = 0.f;
+                if (j <= R0) tmem_ld16(tl + TM_G1 + kda_sec(R0) + 16 * j, x0);  // warp-uniform conditions
+                if (j <= R0 + 1) tmem_ld16(tl + TM_G1 + kda_sec(R0 + 1) + 16 * j, x1);
+                wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) g1[16 * j + e] = first ? x0[e] : x1[e];
+            }
+            if (a.kwide[ci]) {  // exact in-block entries (row r's own block, columns b(r) .. b(r) + 15)
+                const int r = trow & 63, R = r >> 4;
+                const float *dx = a.Dx + (((size_t)ci * 2 + (trow < 64 ? 0 : 1)) * C + r) * 16;
+                float d[16];
+#pragma unroll
+                for (int e = 0; e < 16; e += 4) {
+                    const float4 t4 = *reinterpret_cast<const float4 *>(dx + e);
+                    d[e] = t4.x; d[e + 1] = t4.y; d[e + 2] = t4.z; d[e + 3] = t4.w;
+                }
+#pragma unroll
+                for (int i = 0; i < 64; ++i)
+                    if ((i >> 4) == R) g1[i] = d[i & 15];
+            }
+        } else {
+            tmem_row64(tl + TM_G1, g1);
+        }
         const bool big = *bigflag != 0;
         const float *gc = pf + PF_GC * 64, *cola = pf + PF_COLA * 64;
         const bool arow = trow < 64;
@@ -278,7 +319,6 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
     fence_before_sync();
     ok = consensus(ok);
     // ---------------- W = [T diag(beta e^g) ; *] k,  U~ = [T diag(beta) ; *] v ----------------
-    if (VAR == VAR_KDA && ok) ok = consensus(mbar_wait(&bar[2], 0, abort_flag));
     if (ok && tid == 0) {
         fence_after_sync();
         if (KEEP) {
@@ -323,7 +363,6 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
         if (*abort_flag) {  // let whatever was issued finish before the CTA leaves
             volatile int dummy = 0;
             mbar_wait(&bar[0], 0, &dummy, 100000000ull);
-            if (kt_issued) mbar_wait(&bar[2], 0, &dummy, 100000000ull);
             if (mma_issued > 0) mbar_wait(&bar[1], (mma_issued - 1) & 1, &dummy, 100000000ull);
         }
     }
@@ -335,21 +374,22 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
 
 // ---------------------------------------------------------------- KDA gate operands
 // One CTA of 128 threads per chunk.  Thread (tg, cg) = (tid / 16, tid % 16) owns key channels
-// 8 cg ... 8 cg + 7 of tokens 8 tg ... 8 tg + 7, so every access moves 16 bytes.  The
-// in-chunk cumulative log gate g of each channel is a prefix sum over the chunk's tokens
-// (tokens past T add nothing): inside the thread's 8 tokens, then across the 8 token groups
-// through shared memory.  Then every gate-scaled operand the split path needs is written
-// row-major per chunk.  Exponents are clamped to [-80, 80] so that every factor is a finite
-// bf16.
+// 8 cg ... 8 cg + 7 of tokens 8 tg ... 8 tg + 7, so every access moves 16 bytes; warp w holds
+// the 16 tokens of block w.  The in-chunk cumulative log gate g of each channel is a prefix sum
+// over the chunk's tokens (tokens past T add nothing): inside the thread's 8 tokens, then across
+// the 8 token groups through shared memory.  Then every gate-scaled operand the split path needs
+// is written row-major per chunk.  The factors e^{g_r - g_b(r)}, e^{g}, e^{g_C - g} and the column
+// factors of earlier tokens are <= 1 (log alpha <= 0); only the in-block column factors grow,
+// and their exponent is clamped at 80 (chunks where it would pass KDA_DIAG_SPAN are marked).
 struct KdaArgs {
     const __nv_bfloat16 *q, *k, *alpha;
     __nv_bfloat16 *Kt1, *Qt1, *Kh, *Kt, *Qt, *Kb;
     float *egc;
+    int *kwide;
+    float *Dx;
     float *G;  // optional: g itself, fp32 [chunks][64][128]
     int T, H, N;
 };
-
-__device__ __forceinline__ float clamped_exp(float x) { return __expf(fminf(fmaxf(x, -80.f), 80.f)); }
 
 __device__ __forceinline__ void ld8_bf16(const __nv_bfloat16 *p, float *v) {
     const uint4 x = *reinterpret_cast<const uint4 *>(p);
@@ -370,9 +410,9 @@ __device__ __forceinline__ void st8_bf16(__nv_bfloat16 *p, const float *v) {
 
 __global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
     __shared__ float tot[8][DK];
-    __shared__ float gmid[DK], gend[DK];
+    __shared__ float gblk[4][DK], gend[DK];
     const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int tg = threadIdx.x >> 4, cg = threadIdx.x & 15, c0 = 8 * cg;
+    const int tg = threadIdx.x >> 4, cg = threadIdx.x & 15, c0 = 8 * cg, R = tg >> 1;
     const int t0 = n * C, L = min(C, a.T - t0);
     const size_t ci = ((size_t)b * a.H + h) * a.N + n;
     auto at = [&](int r) { return (((size_t)b * a.T + t0 + r) * a.H + h) * DK + c0; };
@@ -393,7 +433,7 @@ __global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
         for (int t2 = 0; t2 < tg; ++t2) off += tot[t2][c0 + j];
 #pragma unroll
         for (int r = 0; r < 8; ++r) g[r][j] += off;
-        if (tg == C / 16 - 1) gmid[c0 + j] = g[7][j];  // token C/2 - 1, the middle
+        if ((tg & 1) == 0) gblk[R][c0 + j] = g[0][j];  // token 16 R, the first of block R
         if (tg == 7) gend[c0 + j] = g[7][j];           // token C - 1, the last
     }
     __syncthreads();
@@ -405,11 +445,14 @@ __global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
             *reinterpret_cast<float4 *>(dst + 4) = make_float4(g[r][4], g[r][5], g[r][6], g[r][7]);
         }
     }
-    float gm[8], gC[8];
+    float gb[8], gC[8];  // g at the first token of this thread's block, and at the chunk's last
+    bool wide = false;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        gm[j] = gmid[c0 + j];
+        gb[j] = gblk[R][c0 + j];
         gC[j] = gend[c0 + j];
+        // the fall of the gate inside block R, from its first token to its last (held by tg odd)
+        if (tg & 1) wide |= !(gb[j] - g[7][j] <= KDA_DIAG_SPAN);
     }
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
@@ -419,28 +462,91 @@ __global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
             ld8_bf16(a.k + at(tr), kr);
             ld8_bf16(a.q + at(tr), qr);
         }
-        float o1[8], o2[8], o3[8], o4[8], o5[8], o6[8];
+        float o1[8], o2[8], o4[8], o5[8], o6[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const float em = clamped_exp(g[r][j] - gm[j]), ei = clamped_exp(gm[j] - g[r][j]);
-            const float eg = clamped_exp(g[r][j]), ec = clamped_exp(gC[j] - g[r][j]);
-            o1[j] = kr[j] * em; o2[j] = qr[j] * em; o3[j] = kr[j] * ei;
+            // every exponent here is <= 0 for log alpha <= 0; the clamp only keeps other input finite
+            const float eb = __expf(fminf(g[r][j] - gb[j], 80.f));  // row factor
+            const float eg = __expf(fminf(g[r][j], 80.f)), ec = __expf(fminf(gC[j] - g[r][j], 80.f));
+            o1[j] = kr[j] * eb; o2[j] = qr[j] * eb;
             o4[j] = kr[j] * eg; o5[j] = qr[j] * eg; o6[j] = kr[j] * ec;
         }
         const size_t o = (ci * C + tr) * DK + c0;
         st8_bf16(a.Kt1 + o, o1);
         st8_bf16(a.Qt1 + o, o2);
-        st8_bf16(a.Kh + o, o3);
         st8_bf16(a.Kt + o, o4);
         st8_bf16(a.Qt + o, o5);
         st8_bf16(a.Kb + o, o6);
+        // column operand of every block R2 >= R (token tr is one of its rows 0 .. 16 R2 + 15)
+#pragma unroll
+        for (int R2 = 0; R2 < 4; ++R2) {
+            if (R2 < R) continue;
+            float oh[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) oh[j] = kr[j] * __expf(fminf(gblk[R2][c0 + j] - g[r][j], 80.f));
+            st8_bf16(a.Kh + (ci * KDA_KH_ROWS + kda_sec(R2) + tr) * DK + c0, oh);
+        }
     }
     if (tg == 0) {
         float e[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) e[j] = clamped_exp(gC[j]);
+        for (int j = 0; j < 8; ++j) e[j] = __expf(fminf(gC[j], 80.f));
         *reinterpret_cast<float4 *>(a.egc + ci * DK + c0) = make_float4(e[0], e[1], e[2], e[3]);
         *reinterpret_cast<float4 *>(a.egc + ci * DK + c0 + 4) = make_float4(e[4], e[5], e[6], e[7]);
+    }
+    wide = __syncthreads_or(wide);
+    if (threadIdx.x == 0) a.kwide[ci] = wide ? 1 : 0;
+}
+
+// The exact in-block sums of the chunks k_kda_gates marked (one CTA of 128 threads per chunk;
+// the others return at once).  Thread c forms channel c's cumulative log gate; then warp w takes
+// the pairs i <= r of block w, lane l channels l, l + 32, l + 64, l + 96, with one exponential
+// per pair and channel (every exponent <= 0):
+//   Dx[0][r][i - 16 w] = sum_c k_rc k_ic e^{g_rc - g_ic},  Dx[1][r][i - 16 w] = sum_c q_rc k_ic e^{g_rc - g_ic}
+// (0 for i > r).  smem: g, k, q [64][128] fp32.
+constexpr uint32_t DIAG_SMEM = 3 * C * DK * 4;
+
+__global__ void __launch_bounds__(128) k_kda_diag(KdaArgs a) {
+    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const size_t ci = ((size_t)b * a.H + h) * a.N + n;
+    if (!a.kwide[ci]) return;  // uniform over the CTA
+    extern __shared__ float dsm[];
+    float *gsm = dsm, *ksm = gsm + C * DK, *qsm = ksm + C * DK;
+    const int t0 = n * C, L = min(C, a.T - t0), c = threadIdx.x, warp = c >> 5, lane = c & 31;
+    float run = 0.f;
+    for (int r = 0; r < C; ++r) {
+        float kv = 0.f, qv = 0.f;
+        if (r < L) {
+            const size_t x = (((size_t)b * a.T + t0 + r) * a.H + h) * DK + c;
+            run += __bfloat162float(a.alpha[x]);
+            kv = __bfloat162float(a.k[x]);
+            qv = __bfloat162float(a.q[x]);
+        }
+        gsm[r * DK + c] = run;
+        ksm[r * DK + c] = kv;
+        qsm[r * DK + c] = qv;
+    }
+    __syncthreads();
+    const int r0 = 16 * warp;
+    for (int r = r0; r < r0 + 16; ++r) {
+        for (int i = r0; i < r0 + 16; ++i) {
+            float sk = 0.f, sq = 0.f;
+            if (i <= r) {
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const int cc = lane + 32 * m;
+                    const float e = __expf(gsm[r * DK + cc] - gsm[i * DK + cc]) * ksm[i * DK + cc];
+                    sk += ksm[r * DK + cc] * e;
+                    sq += qsm[r * DK + cc] * e;
+                }
+                sk = warp_sum(sk);
+                sq = warp_sum(sq);
+            }
+            if (lane == 0) {
+                a.Dx[((ci * 2 + 0) * C + r) * 16 + (i - r0)] = sk;
+                a.Dx[((ci * 2 + 1) * C + r) * 16 + (i - r0)] = sq;
+            }
+        }
     }
 }
 
@@ -462,9 +568,16 @@ cudaError_t tc_kda_gates(const Geo &g, const Tensors &t, const TcWs &w, float *G
     KdaArgs a;
     a.q = (const __nv_bfloat16 *)t.q; a.k = (const __nv_bfloat16 *)t.k; a.alpha = (const __nv_bfloat16 *)t.alpha;
     a.Kt1 = w.Kt1; a.Qt1 = w.Qt1; a.Kh = w.Kh; a.Kt = w.Kt; a.Qt = w.Qt; a.Kb = w.Kb; a.egc = w.egc; a.G = G;
+    a.kwide = w.kwide; a.Dx = w.Dx;
     a.T = g.T; a.H = g.H; a.N = g.N;
+    cudaError_t e = cudaFuncSetAttribute(k_kda_diag, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DIAG_SMEM);
+    if (e != cudaSuccess) return e;
     rec.mark(s);
     k_kda_gates<<<dim3(g.N, g.H, g.B), DK, 0, s>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    rec.mark(s);
+    k_kda_diag<<<dim3(g.N, g.H, g.B), DK, DIAG_SMEM, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -535,10 +648,11 @@ cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool ke
         ok = tc::make_map_2d_bf16(&mp.KK, w.KK, C, NC * C, 64) && tc::make_map_2d_bf16(&mp.Tn, w.Tn, C, NC * C, 64);
     if (ok && g.variant == VAR_KDA)
         ok = tc::make_map_2d_bf16(&mp.Kt1, w.Kt1, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.Qt1, w.Qt1, DK, NC * C, 64) &&
-             tc::make_map_2d_bf16(&mp.Kh, w.Kh, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.Kt, w.Kt, DK, NC * C, 64);
+             tc::make_map_2d_bf16(&mp.Kh, w.Kh, DK, NC * KDA_KH_ROWS, KDA_KH_ROWS) &&
+             tc::make_map_2d_bf16(&mp.Kt, w.Kt, DK, NC * C, 64);
     if (!ok) return cudaErrorInvalidValue;
     Args a;
-    a.alpha = t.alpha; a.beta = t.beta; a.gb = w.gb;
+    a.alpha = t.alpha; a.beta = t.beta; a.gb = w.gb; a.kwide = w.kwide; a.Dx = w.Dx;
     a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
     const dim3 grid(g.N, g.H, g.B);
     if (g.variant == VAR_KDA) return launch_prep<VAR_KDA, 0>(mp, a, grid, s, rec);  // no saved form

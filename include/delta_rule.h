@@ -126,15 +126,17 @@ int delta_rule_bwd(const void *q, const void *k, const void *v, const void *alph
  * addition, keeps in the caller's buffer `saved` what the backward would
  * otherwise recompute: the per-chunk products of the chunked form (the
  * in-chunk cumulative log gate and beta, W, U~, P, T = (I + A)^-1, k k^T) and
- * the state entering every chunk with its write values, bf16 except the gate.
+ * the state entering every chunk with its write values, bf16 except the gate
+ * (KDA: W, U~, P, the gate-scaled q e^g and k e^{g_C - g}, e^{g_C}, the states
+ * and write values, and the per-channel cumulative log gate in fp32).
  * delta_rule_bwd_saved computes exactly what delta_rule_bwd computes for the
  * same forward arguments, reading `saved` instead of recomputing the forward.
  * `saved` must come from delta_rule_fwd_save on the same inputs and arguments
  * and must not change in between; the backward only reads it.
  *   delta_rule_saved_size  bytes of `saved` for these arguments (the buffer is
  *              device memory, 256-byte aligned).  It is 0 for configurations
- *              without a saved form: the saved form exists for Gated DeltaNet
- *              and DeltaNet with bf16 I/O, dk = dv = 128 and chunk 64.  For the
+ *              without a saved form: the saved form exists for all three
+ *              variants with bf16 I/O, dk = dv = 128 and chunk 64.  For the
  *              others delta_rule_fwd_save behaves as delta_rule_fwd and
  *              delta_rule_bwd_saved as delta_rule_bwd, and `saved` may be NULL.
  *              Returns (size_t)-1 for invalid arguments.
@@ -195,17 +197,22 @@ int delta_rule_bwd_saved_timed(const void *q, const void *k, const void *v, cons
  * deployment convenience).  Some callers cannot call cudaMalloc at all: code
  * inside a CUDA graph being captured, allocator-less embedded runtimes, and
  * plugins that a host framework hands only their input and output buffers.
- * This entry point computes exactly what delta_rule_fwd computes (same
+ * This entry point computes the same quantities as delta_rule_fwd (same
  * arguments, minus the workspace), always on the CUDA-core forward kernels,
  * with their scratch taken from a buffer of DELTA_RULE_NOALLOC_SCRATCH_BYTES
  * that is compiled into the library; every GPU that loads the library holds it
  * until the process exits.  The caller still passes every input and output.
+ * Where delta_rule_fwd runs the same CUDA-core kernels (fp32 I/O, or dk = 64)
+ * the results are bit-identical; where it takes the tensor-core path (bf16,
+ * dk = 128) the two agree within the bf16 tolerance.
  *   - Problems whose scratch (delta_rule_workspace_size of the CUDA-core
  *     forward) exceeds the buffer return DR_ERR_WORKSPACE without launching;
  *     about 210 KB per (batch, head, chunk) at dk = dv = 128, chunk 64.
  *   - The first call on each device looks up the buffer's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept for the process: after
+ *     cudaDeviceReset on a device it is stale, so do not call this entry point
+ *     on that device again in the same process.
  *   - All calls on a device share the one buffer and it keeps the last call's
  *     contents (nothing in it needs to start at zero): calls whose kernels
  *     overlap on the GPU (different streams, or different threads without

@@ -64,8 +64,14 @@ def test_no_compute_validation_paths(lib):
     assert binding.workspace_size(8, 4096, 8, 128, 128, 1, 64, 1, 2) == 0
     assert 0 < binding.workspace_size(8, 4096, 8, 128, 128, 1, 64, 1, 3) < binding.workspace_size(
         8, 4096, 8, 128, 128, 1, 64, 1, 1)
-    assert binding.saved_size(4, 16384, 8, 128, 128, 2, 64, 1) == 0   # KDA: no saved form
+    # KDA: the saved buffer holds per chunk g|beta (512 B), W, U~, U, q e^g, k e^{g_C - g} (16 KiB
+    # each), P (8 KiB), e^{g_C} (512 B), the state entering the chunk and the fp32 gate (32 KiB each)
+    n_chunks = 8 * 16 * 64
+    assert binding.saved_size(8, 4096, 16, 128, 128, 2, 64, 1) == n_chunks * (512 + 5 * 16384 + 8192 + 512 + 2 * 32768)
+    assert 0 < binding.workspace_size(8, 4096, 16, 128, 128, 2, 64, 1, 3) < binding.workspace_size(
+        8, 4096, 16, 128, 128, 2, 64, 1, 1)
     assert binding.saved_size(1, 256, 2, 64, 64, 0, 64, 0) == 0       # fp32 I/O: no saved form
+    assert binding.saved_size(1, 256, 2, 64, 64, 2, 64, 1) == 0       # d = 64: no saved form
     assert lib.delta_rule_workspace_size(1, 10, 1, 128, 128, 1, 64, 1, 4) == ctypes.c_size_t(-1).value
     assert lib.delta_rule_saved_size(1, 10, 1, 96, 128, 1, 64, 1) == ctypes.c_size_t(-1).value
     args = [None] * 9 + [1, 10, 1, 128, 128, 7, 64, 1, None, 0, None, 0, None]
@@ -119,14 +125,15 @@ def test_launch_plans(lib):
     for variant in (0, 1):
         for kind, names in split.items():
             assert binding.launches(8, 4096, 8, 128, 128, variant, 64, 1, kind) == names
-    kda_split = ["k_kda_gates", "k_chunk_prep", "k_chain_fwd"]
+    kda_split = ["k_kda_gates", "k_kda_diag", "k_chunk_prep", "k_chain_fwd"]
     assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 0) == kda_split
-    assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 2) == kda_split  # no saved form: the plain forward
-    kda_bwd = ["k_kda_gates", "k_chunk_prep", "k_chain_fwd(recompute)", "k_widen", "k_chain_rev", "k_widen",
-               "k_state_tc", "k_bwd_intra"]
+    assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 2) == kda_split[:3] + ["k_chain_fwd(keep)"]
+    kda_bwd = ["k_kda_gates", "k_kda_diag", "k_chunk_prep", "k_chain_fwd(recompute)", "k_widen", "k_chain_rev",
+               "k_widen", "k_state_tc", "k_bwd_intra"]
     assert binding.launches(8, 4096, 16, 128, 128, 2, 64, 1, 1) == kda_bwd
-    assert binding.launches(8, 4096, 16, 128, 128, 2, 64, 1, 3) == kda_bwd
-    assert binding.launches(2, 512, 4, 128, 64, 2, 64, 1, 0) == ["k_fwd_tc"]
+    assert binding.launches(8, 4096, 16, 128, 128, 2, 64, 1, 3) == kda_bwd[4:]  # from saved: no recompute
+    # KDA at dv = 64 takes the CUDA-core forward; the fused dv = 64 kernel serves scalar gates
+    assert binding.launches(2, 512, 4, 128, 64, 2, 64, 1, 0) == ["k_prep", "k_scan", "k_out"]
     assert binding.launches(2, 512, 4, 128, 64, 1, 64, 1, 0) == ["k_fwd_tc"]
     assert binding.launches(1, 256, 2, 64, 64, 0, 64, 0, 0) == ["k_prep", "k_scan", "k_out"]
     assert binding.launches(1, 256, 2, 64, 64, 0, 64, 0, 1) == ["k_prep", "k_scan", "k_scan_bwd", "k_bwd_state",

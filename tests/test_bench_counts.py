@@ -44,3 +44,20 @@ def test_flops_and_du(bench):
     # no du: the backward reads dv fewer elements per token-head
     d = bench.alg_counts(8, 4096, 8, 128, 128, 64, 1, 2, du=False)
     assert c["bwd_bytes"] - d["bwd_bytes"] == 8 * 4096 * 8 * 2 * 128
+
+
+def test_gradient_kernel_bytes_leave_out_du(bench):
+    """The intra-chunk gradient kernel reads q, k, v, beta, the gate and dO and writes dq, dk, dv,
+    dbeta, d log alpha: (4 dk + 3 dv + 2 + 2) elements a token-head for Gated DeltaNet, 471.9 MB at
+    the headline shape; du goes to the reverse chain."""
+    c = bench.alg_counts(8, 4096, 8, 128, 128, 64, 1, 2)
+    assert c["bwd_grad_kernel_bytes"] == 8 * 4096 * 8 * 2 * (4 * 128 + 3 * 128 + 2 + 2) == 471_859_200
+    assert c["bwd_io_bytes"] - c["bwd_grad_kernel_bytes"] == 8 * 4096 * 8 * 2 * 128
+
+
+def test_both_arms_print_the_same_config(bench):
+    from gated_delta_rule_107_b200.inputs import WORKLOADS
+    w = WORKLOADS[2]
+    cfg = bench.workload_config(w, w.B, 1)
+    assert cfg["workload"].endswith("fwd+bwd") and cfg["B"] == 8 and cfg["T"] == 4096 and cfg["H"] == 8
+    assert set(cfg) == {"workload", "B", "T", "H", "dk", "dv", "chunk", "variant", "io", "l2", "parallelism"}

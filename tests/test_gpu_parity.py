@@ -108,3 +108,67 @@ def test_kda_bwd_fast_decay_channels_take_the_direct_form():
     x = gen("kda", "f32", 1, 130, 2, 128, 128, seed=41, s0_std=0.1, grads=True)
     x["loga"][..., :8] = -3.0
     compare_bwd(gpu_bwd(x, "kda"), oracle_bwd(x, "kda"), "f32", "kda", what="kda fast-decay channels")
+
+
+# ---- fast-decaying gates on the bf16 tensor-core path --------------------------------------
+# The workload distribution log alpha = -softplus(N(-3, 1)) keeps a chunk's cumulative gate
+# within a few nats; these cases make some channels (KDA) or heads (Gated DeltaNet) fall by
+# 3 nats a token (192 over a chunk), and by 12 (far past the exponent range of one factor).
+@pytest.mark.parametrize("dv", (128, 64))
+def test_kda_bf16_fast_decay_channels_forward(dv):
+    """KDA's pair factors e^{g_r - g_i} on channels falling 3 nats a token: split at each 16-token
+    block's first token, every factor stays in range (a split at the chunk midpoint does not)."""
+    x = gen("kda", "bf16", 2, 200, 3, 128, dv, seed=43, s0_std=0.1)
+    x["loga"][..., :8] = -3.0
+    compare_fwd(gpu_fwd(x, "kda"), oracle_fwd(x, "kda"), "bf16", what=f"kda bf16 dv={dv} fast-decay channels")
+
+
+def test_kda_bf16_fast_decay_channels_backward():
+    x = gen("kda", "bf16", 2, 200, 2, 128, 128, seed=44, s0_std=0.1, grads=True)
+    x["loga"][..., :8] = -3.0
+    compare_bwd(gpu_bwd(x, "kda"), oracle_bwd(x, "kda"), "bf16", "kda", what="kda bf16 fast-decay channels")
+
+
+@pytest.mark.parametrize("T", (64, 137))
+def test_kda_bf16_extreme_decay_takes_exact_in_block_sums(T):
+    """Channels falling 12 nats a token fall 180 inside one 16-token block, past what one factor
+    can carry: such chunks take their in-block entries from exact per-pair sums (k_kda_diag),
+    next to ordinary chunks and a ragged last chunk in the same call."""
+    x = gen("kda", "bf16", 2, T, 2, 128, 128, seed=45, s0_std=0.1, grads=True)
+    x["loga"][0, :, :, :4] = -12.0  # batch 0 only: batch 1 keeps ordinary chunks
+    x["loga"][..., 4:8] = -3.0
+    compare_fwd(gpu_fwd(x, "kda"), oracle_fwd(x, "kda"), "bf16", what=f"kda bf16 extreme decay T={T}")
+    compare_bwd(gpu_bwd(x, "kda"), oracle_bwd(x, "kda"), "bf16", "kda", what=f"kda bf16 extreme decay T={T}")
+
+
+@pytest.mark.parametrize("dv", (128, 64))
+def test_gdn_bf16_fast_decay_heads(dv):
+    """A head whose gate falls 3 nats a token strays more than 80 nats from the chunk midpoint, so
+    its chunks take the exact per-pair exponentials of the tensor-core kernels, forward and
+    backward; the other heads keep the midpoint split."""
+    x = gen("gdn", "bf16", 2, 200, 3, 128, dv, seed=46, s0_std=0.1, grads=True)
+    x["loga"][:, :, 0] = -3.0
+    compare_fwd(gpu_fwd(x, "gdn"), oracle_fwd(x, "gdn"), "bf16", what=f"gdn bf16 dv={dv} fast-decay head")
+    compare_bwd(gpu_bwd(x, "gdn"), oracle_bwd(x, "gdn"), "bf16", "gdn", what=f"gdn bf16 dv={dv} fast-decay head")
+
+
+# ---- run-to-run determinism ----------------------------------------------------------------
+def _bitwise_equal(a, b, what):
+    for key in a:
+        if a[key] is None:
+            continue
+        assert torch.equal(a[key], b[key]), f"{what}: {key} differs between two identical calls"
+
+
+def test_kda_backward_is_deterministic_at_workload5_size():
+    """Two identical KDA backward calls at the training workload's size (B8 T4096 H16) return the
+    same bits: the library has no atomics in its arithmetic, so any difference is a race."""
+    w, x = _workload(5)
+    _bitwise_equal(gpu_bwd(x, w.variant), gpu_bwd(x, w.variant), w.name)
+
+
+@pytest.mark.parametrize("variant", VARS)
+def test_cuda_core_backward_is_deterministic(variant):
+    """The CUDA-core path (fp32 I/O) at C = 64, where every chunk takes the tiled gradient kernel."""
+    x = gen(variant, "f32", 4, 1024, 8, 128, 128, seed=47, s0_std=0.1, grads=True)
+    _bitwise_equal(gpu_bwd(x, variant), gpu_bwd(x, variant), f"{variant} f32")

@@ -40,7 +40,7 @@ def test_saved_pair_equals_recompute_and_oracle(variant, T, du, s0):
 
 
 def test_configurations_without_a_saved_form_run_the_plain_calls():
-    # KDA and fp32 I/O have no saved form: saved_size is 0 and the pair equals fwd / bwd
+    # d = 64 and fp32 I/O have no saved form: saved_size is 0 and the pair equals fwd / bwd
     for variant, dtype, code in (("kda", "bf16", binding.DR_BF16), ("gdn", "f32", binding.DR_F32)):
         x = gen(variant, dtype, 1, 100, 2, 64, 64, seed=41, grads=True)
         assert binding.saved_size(1, 100, 2, 64, 64, binding.VARIANTS[variant], 64, code) == 0
@@ -96,6 +96,36 @@ def test_saved_pair_headline_shape_equals_recompute():
     x = gen("gdn", "bf16", 8, 4096, 8, 128, 128, seed=1002, grads=True, du=True)
     fwd_ref, bwd_ref = gpu_fwd(x, "gdn"), gpu_bwd(x, "gdn")
     fwd, g, _ = _save_pair(x, "gdn")
+    for key in ("o", "u", "S_T"):
+        assert torch.equal(fwd[key], fwd_ref[key]), key
+    for key, t in g.items():
+        if t is not None:
+            assert torch.equal(t, bwd_ref[key]), key
+
+
+@pytest.mark.parametrize("T,du,s0", ((64, True, 0.0), (130, False, 0.1), (257, True, 0.1)))
+def test_kda_saved_pair_equals_recompute_and_oracle(T, du, s0):
+    x = gen("kda", "bf16", 2, T, 3, 128, 128, seed=61 + T, s0_std=s0, grads=True, du=du)
+    fwd_ref, bwd_ref = gpu_fwd(x, "kda"), gpu_bwd(x, "kda")
+    fwd, g, saved = _save_pair(x, "kda")
+    assert saved is not None and saved.numel() == binding.saved_size(2, T, 3, 128, 128, binding.DR_KDA, 64,
+                                                                       binding.DR_BF16)
+    for key in ("o", "u", "S_T"):
+        assert torch.equal(fwd[key], fwd_ref[key]), key
+    for key, t in g.items():
+        if t is not None:
+            assert torch.equal(t, bwd_ref[key]), key
+    compare_bwd(g, oracle_bwd(x, "kda"), "bf16", "kda", what=f"saved kda T={T}")
+
+
+def test_kda_saved_pair_training_shape_equals_recompute():
+    """KDA at the training workload's size (B8 T4096 H16 d128, with du): the training pair
+    bit-equals the plain forward and the recomputing backward."""
+    from gated_delta_rule_107_b200.inputs import WORKLOADS
+    w = WORKLOADS[5]
+    x = gen("kda", "bf16", w.B, w.T, w.H, w.dk, w.dv, seed=w.seed, s0_std=w.s0_std, grads=True, du=w.du)
+    fwd_ref, bwd_ref = gpu_fwd(x, "kda"), gpu_bwd(x, "kda")
+    fwd, g, _ = _save_pair(x, "kda")
     for key in ("o", "u", "S_T"):
         assert torch.equal(fwd[key], fwd_ref[key]), key
     for key, t in g.items():
