@@ -443,9 +443,33 @@ def run_ours(args):
                # one [B, T, H*dk] stream: x read, y written (backward: x, dy read, dx written)
                "shortconv": gbs(2 * rows * elem * dk, conv_ms), "shortconv_bwd": gbs(3 * rows * elem * dk, conv_b_ms)}
 
+    # the fused forward (pre-operation, forward and post-operation in the core's own kernels)
+    # against the three separate calls, on the same raw inputs (Gated DeltaNet / DeltaNet only)
+    fused = None
+    if var != binding.DR_KDA:
+        go_ = torch.randn_like(x["v"].float()).to(x["v"].dtype)
+        w_ = torch.ones(dv, device=dev)
+        fws = torch.empty(binding.fused_workspace_size(B, T, H, dk, dv, var, C, binding.DR_BF16), dtype=torch.uint8,
+                          device=dev)
+        fused_ms = ev_time(lambda: binding.delta_rule_fwd_fused(x["q"], x["k"], x["v"], raw_a, x["beta"], go_, w_,
+                                                                 variant=var, workspace=fws))
+
+        def three():
+            q_, k_, b_, a_ = binding.delta_rule_preop(x["q"], x["k"], x["beta"], raw_a, variant=var)
+            o_, _, _ = binding.delta_rule_fwd(q_, k_, x["v"], a_, b_, None, variant=var)
+            binding.delta_rule_postop(o_, go_, w_)
+
+        three_ms = ev_time(three)
+        if binding.sync_status() != binding.DR_OK:
+            raise RuntimeError("device error word set during the fused leg")
+        f_alg = rows * elem * (2 * dk + 2 * dv + gw_ + 1 + 2 * dv)  # raw q, k, v, gate, beta, out gate in; y, u out
+        fused = {"shape": f"B{B} T{T} H{H} d{dk} bf16", "fused_ms": fused_ms, "separate_ms": three_ms,
+                 "saved_ms": three_ms - fused_ms, "kernels": ["k_chunk_prep(raw)", "k_chain_fwd(fused, 2-CTA clusters)"],
+                 "alg_bytes": f_alg, "fused_frac": f_alg / (fused_ms / 1e3) / 1e9 / hbm}
+
     clvr_flops = 2.0 * B * T * (H * dv) * n_hid
     bf16_peak = load_peaks().get("bf16_tflops")
-    clvr = {"shape": f"M{B * T} K{H * dv} N{n_hid} bf16 (cuBLASLt)", "fwd_ms": clvr_ms, "bwd_ms": clvr_b_ms,
+    clvr = {"shape": f"M{B * T} K{H * dv} N{n_hid} bf16 (k_gemm_tc)", "fwd_ms": clvr_ms, "bwd_ms": clvr_b_ms,
             "fwd_tflops": clvr_flops / (clvr_ms / 1e3) / 1e12, "bwd_tflops": 2 * clvr_flops / (clvr_b_ms / 1e3) / 1e12}
     if bf16_peak:
         clvr["fwd_frac"] = clvr["fwd_tflops"] / bf16_peak
@@ -588,6 +612,7 @@ def run_ours(args):
         "saved_bytes": sv_bytes,
         "decode": decode,
         "prepost": prepost,
+        "fused": fused,
         "clvr": clvr,
         "gpu_launches": args.steps * (len(fwd_names) + len(bwd_names)),
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,

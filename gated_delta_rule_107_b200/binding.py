@@ -44,7 +44,7 @@ EXPORTS = ("delta_rule_workspace_size", "delta_rule_fwd", "delta_rule_bwd", "del
            "delta_rule_preop", "delta_rule_preop_bwd", "delta_rule_postop_workspace_size", "delta_rule_postop",
            "delta_rule_postop_bwd", "delta_rule_selftest_timeout", "delta_rule_shortconv_workspace_size",
            "delta_rule_shortconv", "delta_rule_shortconv_bwd", "delta_rule_clvr_workspace_size", "delta_rule_clvr",
-           "delta_rule_clvr_bwd")
+           "delta_rule_clvr_bwd", "delta_rule_fwd_fused_workspace_size", "delta_rule_fwd_fused")
 
 _lib = None
 
@@ -120,6 +120,10 @@ def load(path: str | None = None):
     lib.delta_rule_fwd_save_timed.restype = i
     lib.delta_rule_bwd_saved_timed.argtypes = [vp] * 15 + [i] * 8 + [vp, sz, vp, sz, vp, ctypes.POINTER(vp), i]
     lib.delta_rule_bwd_saved_timed.restype = i
+    lib.delta_rule_fwd_fused_workspace_size.argtypes = [i] * 8
+    lib.delta_rule_fwd_fused_workspace_size.restype = sz
+    lib.delta_rule_fwd_fused.argtypes = [vp] * 12 + [i] * 8 + [vp, sz, vp]
+    lib.delta_rule_fwd_fused.restype = i
     if path is None:
         _lib = lib
     return lib
@@ -516,6 +520,40 @@ def delta_rule_bwd_saved(q, k, v, alpha, beta, S0, dout, du=None, dS_T=None, sav
                        B, T, H, dk, dv, var, chunk, dt, _p(saved), sneed, _p(workspace), need, stream)
     _check(rc, "delta_rule_bwd_saved")
     return g
+
+
+def fwd_fused_raw(*args) -> int:
+    return load().delta_rule_fwd_fused(*args)
+
+
+def fused_workspace_size(B, T, H, dk, dv, variant, chunk, dtype) -> int:
+    n = load().delta_rule_fwd_fused_workspace_size(B, T, H, dk, dv, variant, chunk, dtype)
+    if n == ctypes.c_size_t(-1).value:
+        raise DeltaRuleError(DR_ERR_UNSUPPORTED, "delta_rule_fwd_fused_workspace_size")
+    return n
+
+
+def delta_rule_fwd_fused(q_raw, k_raw, v, gate_raw, beta_raw, gate_out, w_norm, S0=None, variant="gdn", chunk=64,
+                         want_o=False, want_u=True, want_state=True, workspace: torch.Tensor | None = None):
+    """Pre-operation, forward and post-operation in the core's kernels: returns (y, o or None, u or None,
+    S_T or None) for raw q, k projections and raw gate / beta logits (Gated DeltaNet, DeltaNet)."""
+    var = _variant(variant)
+    B, T, H, dk = q_raw.shape
+    dv = v.shape[-1]
+    dt = DTYPES[q_raw.dtype]
+    dev = q_raw.device
+    y = torch.empty((B, T, H, dv), dtype=q_raw.dtype, device=dev)
+    o = torch.empty_like(y) if want_o else None
+    u = torch.empty_like(y) if want_u else None
+    S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if want_state else None
+    need = fused_workspace_size(B, T, H, dk, dv, var, chunk, dt)
+    if workspace is None or workspace.numel() < need:
+        workspace = _workspace(need, dev)
+    rc = fwd_fused_raw(_p(q_raw), _p(k_raw), _p(v), _p(gate_raw), _p(beta_raw), _p(S0), _p(gate_out), _p(w_norm),
+                       _p(y), _p(o), _p(u), _p(S_T), B, T, H, dk, dv, var, chunk, dt, _p(workspace), need,
+                       torch.cuda.current_stream(dev).cuda_stream)
+    _check(rc, "delta_rule_fwd_fused")
+    return y, o, u, S_T
 
 
 def delta_rule_fwd_host(q, k, v, alpha, beta, S0=None, variant="gdn", chunk=64, device="cuda"):

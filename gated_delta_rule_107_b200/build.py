@@ -16,7 +16,7 @@ NVCC_FLAGS = [
     "-Xcompiler", "-fPIC", "-shared",
     "--expt-relaxed-constexpr",
     "-Xptxas", "-warn-spills",
-    "-lcublasLt", "-Xlinker", "-rpath=/usr/local/cuda/lib64",
+    "-Xlinker", "-z,defs",  # an undefined symbol fails the build, not the first load
 ]
 
 

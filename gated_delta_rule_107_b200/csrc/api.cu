@@ -62,7 +62,8 @@ size_t ws_al(size_t x) { return (x + 255) & ~(size_t)255; }
 // Parts of the split-path workspace (tc_path.cuh) that each call kind uses
 constexpr int GDN_SAVED = WS_FWD | WS_KEEP | WS_STATE;
 constexpr int KDA_FWD = WS_FWD | WS_KDA | WS_KDAC;
-constexpr int KDA_SAVED = WS_FWD | WS_STATE | WS_KDAC | WS_KDAG;
+constexpr int KDA_SAVED = WS_FWD | WS_KEEP | WS_STATE | WS_KDAC | WS_KDAG;
+constexpr int KDA_BWD = WS_FWD | WS_KEEP | WS_STATE | WS_REV | WS_KDA | WS_KDAC;
 
 size_t ws_bytes(const Geo &g, int dtype, int kind) {
     if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
@@ -78,7 +79,7 @@ size_t ws_bytes(const Geo &g, int dtype, int kind) {
         return tc_ws_bytes(g, kind == K_FWD_SAVE ? WS_KDA : KDA_FWD);
     if (use_kda_hybrid_bwd(g, dtype, kind))
         return ws_al(simt_ws_bytes(g, true)) +
-               tc_ws_bytes(g, kind == K_BWD_SAVED ? WS_REV : WS_FWD | WS_STATE | WS_REV | WS_KDA | WS_KDAC);
+               tc_ws_bytes(g, kind == K_BWD_SAVED ? WS_REV : KDA_BWD);
     if (!is_bwd(kind) && use_tc_fwd(g, dtype)) return 0;
     return simt_ws_bytes(g, is_bwd(kind));
 }
@@ -165,7 +166,7 @@ static int fwd_impl(const void *q, const void *k, const void *v, const void *alp
             tc_ws_carve(g, KDA_FWD, workspace, &w);
         }
         rc = launch_status(tc_kda_gates(g, t, w, save ? w.G : nullptr, s, rec));
-        if (rc == DR_OK) rc = launch_status(tc_chunk_prep(g, t, w, false, s, rec));
+        if (rc == DR_OK) rc = launch_status(tc_chunk_prep(g, t, w, save, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, save ? 2 : 0, s, rec));
     } else if (use_tc_fwd(g, dtype)) {
         rc = launch_status(tc_fwd(g, t, workspace, s, rec));
@@ -226,22 +227,73 @@ static int bwd_impl(const void *q, const void *k, const void *v, const void *alp
             tc_ws_carve(g, WS_REV, tcbase, &w);
             sw.G = w.G;
         } else {
-            tc_ws_carve(g, WS_FWD | WS_STATE | WS_REV | WS_KDA | WS_KDAC, tcbase, &w);
+            tc_ws_carve(g, KDA_BWD, tcbase, &w);
             rc = launch_status(tc_kda_gates(g, t, w, sw.G, s, rec));
-            if (rc == DR_OK) rc = launch_status(tc_chunk_prep(g, t, w, false, s, rec));
+            if (rc == DR_OK) rc = launch_status(tc_chunk_prep(g, t, w, true, s, rec));
             if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, 1, s, rec));
         }
-        // the CUDA-core gradient kernel reads W, U~, U, dU widened to fp32 and the state products
-        if (rc == DR_OK) rc = launch_status(tc_to_simt(g, w, sw.W, sw.Ut, nullptr, nullptr, sw.Un, s, rec));
         if (rc == DR_OK) rc = launch_status(tc_chain_rev(g, t, w, s, rec));
-        if (rc == DR_OK) rc = launch_status(tc_rev_to_simt(g, w, nullptr, sw.dUn, s, rec));
-        if (rc == DR_OK) rc = launch_status(tc_state_to_simt(g, t, w, sw.Qd, sw.dWm, sw.Tm, sw.RS, s, rec));
+        // the intra-chunk gradients on tcgen05 for every chunk whose gates stay within the block
+        // split's range; the others (w.kwide) on the CUDA-core kernel, which reads W, U~, U, dU
+        // widened to fp32 and the state products (these kernels pass over the other chunks)
+        if (rc == DR_OK) rc = launch_status(tc_bwd_kda(g, t, w, s, rec));
+        sw.only = w.kwide;
+        if (rc == DR_OK) rc = launch_status(tc_to_simt(g, w, sw.W, sw.Ut, nullptr, nullptr, sw.Un, s, rec, w.kwide));
+        if (rc == DR_OK) rc = launch_status(tc_rev_to_simt(g, w, nullptr, sw.dUn, s, rec, w.kwide));
+        if (rc == DR_OK)
+            rc = launch_status(tc_state_to_simt(g, t, w, sw.Qd, sw.dWm, sw.Tm, sw.RS, s, rec, w.kwide));
         if (rc == DR_OK) rc = launch_status(simt_bwd_intra(g, t, dtype == DR_BF16, sw, s, rec));
     } else {
         const SimtWs w = simt_ws_carve(g, true, workspace);
         rc = launch_status(simt_bwd(g, t, dtype == DR_BF16, w, s, rec));
     }
     rec.mark(s);  // end of the last launch
+    return rc;
+}
+
+// The fused forward: pre-operation, core forward and post-operation in the split path's two
+// kernels (Gated DeltaNet / DeltaNet, bf16, dk = dv = 128, chunk 64).
+static int fused_shape(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype, Geo *g) {
+    const int rc = check_shape(B, T, H, dk, dv, variant, chunk, dtype, g);
+    if (rc != DR_OK) return rc;
+    return use_split(*g, dtype) ? DR_OK : DR_ERR_UNSUPPORTED;
+}
+
+extern "C" size_t delta_rule_fwd_fused_workspace_size(int B, int T, int H, int dk, int dv, int variant, int chunk,
+                                                      int dtype) {
+    Geo g;
+    if (fused_shape(B, T, H, dk, dv, variant, chunk, dtype, &g) != DR_OK) return (size_t)-1;
+    if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
+    return tc_ws_bytes(g, WS_FWD | WS_RN);
+}
+
+extern "C" int delta_rule_fwd_fused(const void *q_raw, const void *k_raw, const void *v, const void *gate_raw,
+                                    const void *beta_raw, const float *S0, const void *gate_out, const float *w_norm,
+                                    void *y, void *o, void *u, float *S_T, int B, int T, int H, int dk, int dv,
+                                    int variant, int chunk, int dtype, void *workspace, size_t ws_bytes_given,
+                                    void *stream) {
+    Geo g;
+    int rc = fused_shape(B, T, H, dk, dv, variant, chunk, dtype, &g);
+    if (rc != DR_OK) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    const bool empty = (size_t)B * H == 0;
+    if (T == 0 || empty) return empty ? DR_OK : copy_state(S_T, S0, g, s);
+    if (!q_raw || !k_raw || !v || !beta_raw || !gate_out || !w_norm || !y) return DR_ERR_ARG;
+    if (variant != DR_DELTANET && !gate_raw) return DR_ERR_ARG;
+    const void *ptrs[] = {q_raw, k_raw, v, S0, gate_out, w_norm, y, o, u, S_T};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return DR_ERR_ALIGN;
+    if (!aligned_elem(beta_raw, dtype) || (variant == DR_GATED && !aligned_elem(gate_raw, dtype))) return DR_ERR_ALIGN;
+    rc = check_buffer(workspace, ws_bytes_given, tc_ws_bytes(g, WS_FWD | WS_RN));
+    if (rc != DR_OK) return rc;
+    Tensors t = {};
+    t.q = q_raw; t.k = k_raw; t.v = v; t.alpha = gate_raw; t.beta = beta_raw; t.S0 = S0;
+    t.out = o; t.u = u; t.S_T = S_T; t.gate_o = gate_out; t.w_norm = w_norm; t.y = y;
+    TcWs w = {};
+    tc_ws_carve(g, WS_FWD | WS_RN, workspace, &w);
+    Rec rec;
+    rc = launch_status(tc_chunk_prep(g, t, w, false, s, rec, true));
+    if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, 3, s, rec));
     return rc;
 }
 
@@ -253,9 +305,10 @@ static int launch_plan(const Geo &g, int dtype, int kind, const char **names, in
                                              "k_bwd_chunk_tc"};
     static const char *const SPLIT_BWD_SAVED[2] = {"k_chain_rev", "k_bwd_chunk_tc"};
     static const char *const SPLIT_KDA_FWD[4] = {"k_kda_gates", "k_kda_diag", "k_chunk_prep", "k_chain_fwd"};
-    static const char *const KDA_BWD[9] = {"k_kda_gates", "k_kda_diag", "k_chunk_prep", "k_chain_fwd(recompute)",
-                                           "k_widen", "k_chain_rev", "k_widen", "k_state_tc", "k_bwd_intra"};
-    static const char *const KDA_FWD_SAVE[4] = {"k_kda_gates", "k_kda_diag", "k_chunk_prep", "k_chain_fwd(keep)"};
+    static const char *const KDA_BWD_NAMES[10] = {"k_kda_gates", "k_kda_diag", "k_chunk_prep(keep)",
+                                                  "k_chain_fwd(recompute)", "k_chain_rev", "k_bwd_kda_tc", "k_widen",
+                                                  "k_widen", "k_state_tc", "k_bwd_intra"};
+    static const char *const KDA_FWD_SAVE[4] = {"k_kda_gates", "k_kda_diag", "k_chunk_prep(keep)", "k_chain_fwd(keep)"};
     int n = 0;
     const char *const *src = nullptr;
     if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
@@ -270,8 +323,8 @@ static int launch_plan(const Geo &g, int dtype, int kind, const char **names, in
         src = kind == K_FWD_SAVE ? KDA_FWD_SAVE : SPLIT_KDA_FWD;
         n = 4;
     } else if (use_kda_hybrid_bwd(g, dtype, kind)) {
-        src = kind == K_BWD_SAVED ? KDA_BWD + 4 : KDA_BWD;  // from saved: no recompute
-        n = kind == K_BWD_SAVED ? 5 : 9;
+        src = kind == K_BWD_SAVED ? KDA_BWD_NAMES + 4 : KDA_BWD_NAMES;  // from saved: no recompute
+        n = kind == K_BWD_SAVED ? 6 : 10;
     } else if (!is_bwd(kind) && use_tc_fwd(g, dtype)) {
         return tc_fwd_launches(g, names, max_names);
     } else {

@@ -5,125 +5,355 @@
 // residual stream all layers share, through a projection W that starts at zero.  With U the write
 // values as [B*T, H*dv] (the core's u output, unchanged), W [H*dv, D] and h [B*T, D]:
 //     h_out = h + U W,      dU = dH W^T,      dW = U^T dH,      dh = dH.
-// These are plain dense products, so they run as cuBLASLt GEMMs: bf16 operands on the tensor
-// cores with fp32 accumulation (fp32 operands and arithmetic for fp32 I/O), the residual add as
-// the GEMM's beta = 1 term, so that h_out is written in the same pass.  The routing step and
-// its weight are the model's; the library only needs U, which the core writes anyway.
-#include <cublasLt.h>
-
-#include <mutex>
-
+//
+// bf16: one persistent tcgen05 GEMM kernel serves all three products.  A CTA per SM walks
+// 128 x 256 output tiles; warp 0 feeds a three-stage ring of 64-wide K slices by TMA, warp 1
+// issues the MMAs (M = 128, N = 256, fp32 accumulators in TMEM, two accumulators so that a
+// tile's epilogue overlaps the next tile's products), warps 2-5 drain the accumulator.  Either
+// operand may be stored K-major or MN-major (U^T and W^T are read in place, no transposes):
+//   h_out = h + U W     A = U K-major,    B = W MN-major,   residual tile h added in the epilogue
+//   dU    = dH W^T      A = dH K-major,   B = W K-major
+//   dW    = U^T dH      A = U MN-major,   B = dH MN-major,  fp32 out; the long reduction over the
+//                       tokens is split into slices whose fp32 partials a second kernel adds in a
+//                       fixed order (deterministic)
+// The bf16 results leave through TMA stores of the output tile, rows and columns past the matrix
+// clipped; loads past it read zeros.  fp32 I/O runs a register-blocked CUDA-core GEMM in fp32.
 #include "../../include/delta_rule.h"
 #include "clvr.cuh"
+#include "tc_host.cuh"
+#include "tc_ptx.cuh"
+#include "tc_tile.cuh"
 
 namespace dr {
 namespace clv {
 
-constexpr size_t WS = (size_t)32 << 20;  // cuBLASLt workspace, provided by the caller
+using namespace dr::tc;
+using dr::tcf::ld_chunk;
+using dr::tcf::st_chunk;
 
-// One cuBLASLt handle per process, created on first use (the library's only host-side state).
-cublasLtHandle_t handle(bool *ok) {
-    static cublasLtHandle_t h = nullptr;
-    static cublasStatus_t st = CUBLAS_STATUS_SUCCESS;
-    static std::once_flag once;
-    std::call_once(once, [] { st = cublasLtCreate(&h); });
-    *ok = st == CUBLAS_STATUS_SUCCESS;
-    return h;
-}
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 3;
+constexpr uint32_t A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2;  // 16 KB, 32 KB per stage
+constexpr uint32_t OFF_A = 0, OFF_B = STAGES * A_BYTES, OFF_C = OFF_B + STAGES * B_BYTES;
+constexpr uint32_t C_BYTES = BM * BN * 2;  // bf16 output tile: 4 panels [128 rows][64 columns]
+constexpr uint32_t OFF_MISC = OFF_C + C_BYTES;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 256;
+enum { B_FULL = 0, B_EMPTY = STAGES, B_ACCF = 2 * STAGES, B_ACCE = B_ACCF + 2, B_CF = B_ACCE + 2, B_NUM };
+constexpr uint32_t M_TMEM = 8 * B_NUM, M_ABORT = M_TMEM + 4;
+static_assert(M_ABORT + 4 <= 256, "misc overflow");
+constexpr int NTHREADS = 192;  // warp 0 TMA, warp 1 MMA and TMEM owner, warps 2-5 epilogue
+constexpr uint32_t TM_COLS = 512;  // two 256-column accumulators
+constexpr int MAX_SPLIT = 8;
+constexpr size_t WS = (size_t)32 << 20;  // split-reduction partials of dW (fp32)
 
-// Row-major D [m][n] = op(A) op(B) + beta C, op(A) [m][k] being A [m][k] or, with ta, the
-// transpose of A [k][m]; op(B) [k][n] being B [k][n] or, with tb, the transpose of B [n][k].
-// cuBLASLt works column-major, so it forms D^T = op(B)^T op(A)^T from the same buffers.  The
-// descriptors and the chosen algorithm of each distinct problem are kept for the process (a
-// short list under a mutex), so that a repeated call costs one cublasLtMatmul.
-struct Plan {
-    int m, n, k, ta, tb, ab, cd;
-    size_t wsb;
-    cublasLtMatmulDesc_t op;
-    cublasLtMatrixLayout_t La, Lb, Lc;
-    cublasLtMatmulAlgo_t algo;
+struct Maps {
+    CUtensorMap a, b;  // operands (box per layout below)
+    CUtensorMap c, d;  // bf16 residual and output [M][N], box 64 columns x 128 rows
 };
-constexpr int MAX_PLANS = 64;
 
-cublasStatus_t make_plan(cublasLtHandle_t lt, Plan &p) {
-    const cublasOperation_t o1 = p.tb ? CUBLAS_OP_T : CUBLAS_OP_N, o2 = p.ta ? CUBLAS_OP_T : CUBLAS_OP_N;
-    const cudaDataType_t ab = (cudaDataType_t)p.ab, cd = (cudaDataType_t)p.cd;
-    const int m = p.m, n = p.n, k = p.k;
-    cublasLtMatmulPreference_t pref = nullptr;
-    cublasStatus_t st = cublasLtMatmulDescCreate(&p.op, CUBLAS_COMPUTE_32F, CUDA_R_32F);
-    if (st == CUBLAS_STATUS_SUCCESS) st = cublasLtMatmulDescSetAttribute(p.op, CUBLASLT_MATMUL_DESC_TRANSA, &o1, sizeof(o1));
-    if (st == CUBLAS_STATUS_SUCCESS) st = cublasLtMatmulDescSetAttribute(p.op, CUBLASLT_MATMUL_DESC_TRANSB, &o2, sizeof(o2));
-    // first operand, B: column-major n x k (ld n), or k x n (ld k) read transposed
-    if (st == CUBLAS_STATUS_SUCCESS) st = cublasLtMatrixLayoutCreate(&p.La, ab, p.tb ? k : n, p.tb ? n : k, p.tb ? k : n);
-    // second operand, A: column-major k x m (ld k), or m x k (ld m) read transposed
-    if (st == CUBLAS_STATUS_SUCCESS) st = cublasLtMatrixLayoutCreate(&p.Lb, ab, p.ta ? m : k, p.ta ? k : m, p.ta ? m : k);
-    if (st == CUBLAS_STATUS_SUCCESS) st = cublasLtMatrixLayoutCreate(&p.Lc, cd, n, m, n);
-    if (st == CUBLAS_STATUS_SUCCESS) st = cublasLtMatmulPreferenceCreate(&pref);
-    if (st == CUBLAS_STATUS_SUCCESS)
-        st = cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &p.wsb, sizeof(p.wsb));
-    cublasLtMatmulHeuristicResult_t res = {};
-    int found = 0;
-    if (st == CUBLAS_STATUS_SUCCESS)
-        st = cublasLtMatmulAlgoGetHeuristic(lt, p.op, p.La, p.Lb, p.Lc, p.Lc, pref, 1, &res, &found);
-    if (st == CUBLAS_STATUS_SUCCESS && found == 0) st = CUBLAS_STATUS_NOT_SUPPORTED;
-    if (st == CUBLAS_STATUS_SUCCESS) p.algo = res.algo;
-    if (pref) cublasLtMatmulPreferenceDestroy(pref);
-    return st;
+struct Args {
+    int M, N, K;      // D [M][N] = op(A) [M][K] op(B) [K][N]
+    int a_mn, b_mn;   // 1: the operand is stored MN-major (its K index is the row)
+    int has_c;        // add the residual tile of map c
+    float *d32;       // fp32 output (slice s at d32 + s * slice_elems) instead of the bf16 map d
+    size_t slice_elems;
+    int nsplit, kslice;  // slice s reduces k in [s kslice, min(K, (s + 1) kslice)), kslice % 64 == 0
+};
+
+// Loads of one K slice of one operand tile into shared memory (the layouts the MMA reads):
+//   K-major, R rows: one box of 64 (K) x R rows -> [R rows][128 B], 128-byte swizzle
+//   MN-major, R columns: R / 64 boxes of 64 (MN) x 64 (K rows) -> panel p = [64 K rows][128 B]
+__device__ __forceinline__ void load_operand(unsigned char *dst, const CUtensorMap *map, bool mn, int rows, int r0,
+                                             int k0, uint64_t *bar) {
+    if (!mn) {
+        tma_load_2d(dst, map, k0, r0, bar);
+    } else {
+        for (int p = 0; p < rows / 64; ++p) tma_load_2d(dst + p * 8192, map, r0 + 64 * p, k0, bar);
+    }
 }
 
-void free_plan(Plan &p) {
-    if (p.Lc) cublasLtMatrixLayoutDestroy(p.Lc);
-    if (p.Lb) cublasLtMatrixLayoutDestroy(p.Lb);
-    if (p.La) cublasLtMatrixLayoutDestroy(p.La);
-    if (p.op) cublasLtMatmulDescDestroy(p.op);
+// Shared-memory descriptor of K step kk (16 elements) of an operand tile laid out as above
+__device__ __forceinline__ uint64_t operand_desc(uint32_t base, bool mn, int kk) {
+    return mn ? sdesc(base + kk * 2048, 8192, 1024) : sdesc(base + kk * 32, 16, 1024);
 }
 
-cublasStatus_t gemm(cublasLtHandle_t lt, const void *A, bool ta, const void *B, bool tb, const void *C, void *D,
-                    int m, int n, int k, cudaDataType_t ab, cudaDataType_t cd, float beta, void *ws, size_t wsb,
-                    cudaStream_t s) {
-    static std::mutex mu;
-    static Plan plans[MAX_PLANS];
-    static int nplans = 0;
-    Plan key = {m, n, k, (int)ta, (int)tb, (int)ab, (int)cd, wsb, nullptr, nullptr, nullptr, nullptr, {}};
-    const Plan *use = nullptr;
-    Plan local = key;
-    {
-        std::lock_guard<std::mutex> g(mu);
-        for (int i = 0; i < nplans && !use; ++i) {
-            const Plan &q = plans[i];
-            if (q.m == m && q.n == n && q.k == k && q.ta == key.ta && q.tb == key.tb && q.ab == key.ab &&
-                q.cd == key.cd && q.wsb == wsb)
-                use = &q;
-        }
-        if (!use && nplans < MAX_PLANS) {
-            Plan &q = plans[nplans];
-            q = key;
-            const cublasStatus_t st = make_plan(lt, q);
-            if (st != CUBLAS_STATUS_SUCCESS) {
-                free_plan(q);
-                return st;
+__global__ void __launch_bounds__(NTHREADS, 1) k_gemm_tc(const __grid_constant__ Maps mp, Args a) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_MISC);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + M_TMEM);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + M_ABORT);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int mt = (a.M + BM - 1) / BM, nt = (a.N + BN - 1) / BN;
+    const int tiles = mt * nt * a.nsplit;
+    const int kblocks_full = (a.kslice + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < B_NUM; ++i) mbar_init(&bar[i], (i >= B_ACCE && i < B_CF) ? 4 : 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, TM_COLS);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *tmem_slot;
+
+    // tile t -> split slice, row block, column block (consecutive tiles share the A rows)
+    auto tile_of = [&](int t, int &s, int &mb, int &nb) {
+        s = t % a.nsplit;
+        const int r = t / a.nsplit;
+        nb = r % nt;
+        mb = r / nt;
+    };
+    auto kblocks_of = [&](int s) {
+        const int k0 = s * a.kslice, k1 = min(a.K, k0 + a.kslice);
+        return k1 > k0 ? min(kblocks_full, (k1 - k0 + BK - 1) / BK) : 0;
+    };
+
+    if (warp == 0) {
+        // ================================ TMA producer ================================
+        int slot = 0, use = 0, issued[STAGES] = {0, 0, 0};
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+            int s, mb, nb;
+            tile_of(t, s, mb, nb);
+            const int nk = kblocks_of(s);
+            for (int kb = 0; kb < nk; ++kb) {
+                if (use > 0 && !mbar_wait(&bar[B_EMPTY + slot], (use - 1) & 1, abort_flag)) goto producer_done;
+                if (lane == 0) {
+                    const int k0 = s * a.kslice + kb * BK;
+                    mbar_arrive_tx(&bar[B_FULL + slot], A_BYTES + B_BYTES);
+                    load_operand(sm + OFF_A + slot * A_BYTES, &mp.a, a.a_mn, BM, mb * BM, k0, &bar[B_FULL + slot]);
+                    load_operand(sm + OFF_B + slot * B_BYTES, &mp.b, a.b_mn, BN, nb * BN, k0, &bar[B_FULL + slot]);
+                }
+                __syncwarp();
+                issued[slot]++;
+                if (++slot == STAGES) { slot = 0; ++use; }
             }
-            use = &plans[nplans++];
         }
-    }
-    if (!use) {  // the list is full: a plan for this call only
-        const cublasStatus_t st = make_plan(lt, local);
-        if (st != CUBLAS_STATUS_SUCCESS) {
-            free_plan(local);
-            return st;
+    producer_done:
+        if (*abort_flag && lane == 0) {  // let the issued copies land before the CTA retires
+            volatile int dummy = 0;
+            for (int i = 0; i < STAGES; ++i)
+                if (issued[i] > 0) mbar_wait(&bar[B_FULL + i], (issued[i] - 1) & 1, &dummy, 100000000ull);
         }
+    } else if (warp == 1) {
+        // ================================ MMA issuer ================================
+        const uint32_t id = idesc_bf16(BM, BN, a.a_mn, a.b_mn);
+        int slot = 0, use = 0, it = 0, committed[2] = {0, 0};
+        bool ok = true;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++it) {
+            int s, mb, nb;
+            tile_of(t, s, mb, nb);
+            const int nk = kblocks_of(s), acc = it & 1;
+            // the epilogue of the tile two back has drained this accumulator
+            if (it >= 2 && !(ok = mbar_wait(&bar[B_ACCE + acc], ((it >> 1) - 1) & 1, abort_flag))) break;
+            fence_after_sync();
+            for (int kb = 0; kb < nk; ++kb) {
+                if (!(ok = mbar_wait(&bar[B_FULL + slot], use & 1, abort_flag))) break;
+                fence_after_sync();
+                if (lane == 0) {
+                    const uint32_t sa = smem_u32(sm + OFF_A + slot * A_BYTES), sb = smem_u32(sm + OFF_B + slot * B_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_bf16(tbase + acc * BN, operand_desc(sa, a.a_mn, kk), operand_desc(sb, a.b_mn, kk), id,
+                                 kb > 0 || kk > 0);
+                    mma_commit(&bar[B_EMPTY + slot]);  // frees the stage once these MMAs have read it
+                }
+                __syncwarp();
+                if (++slot == STAGES) { slot = 0; ++use; }
+            }
+            if (!ok) break;
+            if (lane == 0) mma_commit(&bar[B_ACCF + acc]);  // nk == 0: completes at once (zero tile)
+            __syncwarp();
+            committed[acc]++;
+        }
+        if (*abort_flag && lane == 0) {  // let issued MMAs finish before TMEM is released
+            volatile int dummy = 0;
+            for (int i = 0; i < 2; ++i)
+                if (committed[i] > 0) mbar_wait(&bar[B_ACCF + i], (committed[i] - 1) & 1, &dummy, 100000000ull);
+        }
+    } else {
+        // ================================ epilogue ================================
+        const int q4 = warp & 3, r = q4 * 32 + lane;  // TMEM lane = output row of the tile
+        const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
+        const bool leader = warp == 2 && lane == 0;   // issues the residual loads and the stores
+        int it = 0, cloads = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+            int s, mb, nb;
+            tile_of(t, s, mb, nb);
+            const int acc = it & 1;
+            const bool zero = kblocks_of(s) == 0;
+            if (a.d32 == nullptr) {
+                // the output tile is free once the previous tile's store has read it; then the residual
+                if (leader) {
+                    bulk_wait_read_all();
+                    if (a.has_c) {
+                        mbar_arrive_tx(&bar[B_CF], C_BYTES);
+                        for (int p = 0; p < 4; ++p)
+                            tma_load_2d(sm + OFF_C + p * 16384, &mp.c, nb * BN + 64 * p, mb * BM, &bar[B_CF]);
+                    }
+                }
+                named_sync(1, 128);
+            }
+            bool ok = mbar_wait(&bar[B_ACCF + acc], (it >> 1) & 1, abort_flag);
+            if (ok && a.has_c && a.d32 == nullptr) ok = mbar_wait(&bar[B_CF], cloads & 1, abort_flag);
+            if (a.has_c && a.d32 == nullptr) cloads++;
+            fence_after_sync();
+            if (named_sync_any(1, 128, !ok || *abort_flag != 0)) break;
+            const int grow = mb * BM + r;
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                float v[32];
+                tmem_ld16(tl + acc * BN + c0, v);
+                tmem_ld16(tl + acc * BN + c0 + 16, v + 16);
+                wait_ld();
+                if (zero) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = 0.f;
+                }
+                if (a.d32) {
+                    const int gc = nb * BN + c0;
+                    if (grow < a.M) {
+                        float *dst = a.d32 + (size_t)s * a.slice_elems + (size_t)grow * a.N + gc;
+                        if (gc + 32 <= a.N) {
+#pragma unroll
+                            for (int j = 0; j < 32; j += 4)
+                                *reinterpret_cast<float4 *>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                        } else {
+                            for (int j = 0; j < 32 && gc + j < a.N; ++j) dst[j] = v[j];
+                        }
+                    }
+                } else {
+                    const int p = c0 >> 6;
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        const uint32_t o = (uint32_t)p * 16384 + swz(r, ((c0 & 63) >> 3) + ch);
+                        if (a.has_c) {
+                            float h8[8];
+                            ld_chunk(sm + OFF_C, o, h8);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) v[ch * 8 + e] += h8[e];
+                        }
+                        st_chunk(sm + OFF_C, o, v + ch * 8);
+                    }
+                }
+            }
+            // this accumulator is drained (each epilogue warp arrives once)
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[B_ACCE + acc]);
+            if (a.d32 == nullptr) {
+                fence_proxy_async();
+                named_sync(1, 128);
+                if (leader) {
+                    for (int p = 0; p < 4; ++p) tma_store_2d(&mp.d, sm + OFF_C + p * 16384, nb * BN + 64 * p, mb * BM);
+                    bulk_commit();
+                }
+            }
+        }
+        if (leader) bulk_wait_all();
     }
-    const Plan &p = use ? *use : local;
-    const float alpha = 1.f;
-    const cublasStatus_t st =
-        cublasLtMatmul(lt, p.op, &alpha, B, p.La, A, p.Lb, &beta, C ? C : D, p.Lc, D, p.Lc, &p.algo, ws, wsb, s);
-    if (!use) free_plan(local);
-    return st;
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == 1) tmem_dealloc(tbase, TM_COLS);
 }
 
-int status(cublasStatus_t st) {
-    if (st == CUBLAS_STATUS_SUCCESS) return DR_OK;
-    return st == CUBLAS_STATUS_NOT_SUPPORTED ? DR_ERR_UNSUPPORTED : DR_ERR_CUDA;
+// dW = the sum of the split partials, in slice order
+__global__ void __launch_bounds__(256) k_sum_slices(const float *part, float *out, size_t n, int nsplit) {
+    for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < n / 4; i += (size_t)gridDim.x * 256) {
+        float4 acc = reinterpret_cast<const float4 *>(part)[i];
+        for (int s = 1; s < nsplit; ++s) {
+            const float4 x = reinterpret_cast<const float4 *>(part + (size_t)s * n)[i];
+            acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+        }
+        reinterpret_cast<float4 *>(out)[i] = acc;
+    }
+}
+
+// ---------------------------------------------------------------- fp32 I/O (CUDA cores)
+// D [M][N] = op(A) op(B) (+ C): 64 x 64 tiles, 256 threads, 4 x 4 outputs per thread, K in
+// steps of 16 through shared memory.  a_t: A stored [K][M]; b_t: B stored [N][K].
+__global__ void __launch_bounds__(256) k_gemm_f32(const float *A, const float *B, const float *Cres, float *D, int M,
+                                                  int N, int K, int a_t, int b_t) {
+    __shared__ float As[16][64 + 4], Bs[16][64 + 4];
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+    float acc[4][4] = {};
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        for (int x = threadIdx.x; x < 16 * 64; x += 256) {
+            const int kk = x >> 6, i = x & 63;  // As[kk][i] = op(A)[m0 + i][k0 + kk]
+            const int m = m0 + i, k = k0 + kk;
+            As[kk][i] = (m < M && k < K) ? (a_t ? A[(size_t)k * M + m] : A[(size_t)m * K + k]) : 0.f;
+            const int n = n0 + i;  // Bs[kk][i] = op(B)[k0 + kk][n0 + i]
+            Bs[kk][i] = (n < N && k < K) ? (b_t ? B[(size_t)n * K + k] : B[(size_t)k * N + n]) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+            float av[4], bv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                av[u] = As[kk][ty * 4 + u];
+                bv[u] = Bs[kk][tx * 4 + u];
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int w = 0; w < 4; ++w) acc[u][w] += av[u] * bv[w];
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int m = m0 + ty * 4 + u;
+        if (m >= M) continue;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const int n = n0 + tx * 4 + w;
+            if (n < N) D[(size_t)m * N + n] = acc[u][w] + (Cres ? Cres[(size_t)m * N + n] : 0.f);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- host side
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return n;
+}
+
+// One bf16 product.  A: [M][K] (a_mn = 0) or [K][M] (a_mn = 1); B: [N][K] (b_mn = 0) or [K][N]
+// (b_mn = 1); D: bf16 [M][N] (+ the residual C), or fp32 d32 with nsplit slices.
+int gemm_bf16(const void *A, int a_mn, const void *B, int b_mn, const void *C, void *D, float *d32, int M, int N,
+              int K, int nsplit, size_t slice_elems, cudaStream_t s) {
+    Maps mp;
+    bool ok = a_mn ? make_map_2d_bf16(&mp.a, A, M, K, 64) : make_map_2d_bf16(&mp.a, A, K, M, BM);
+    ok = ok && (b_mn ? make_map_2d_bf16(&mp.b, B, N, K, 64) : make_map_2d_bf16(&mp.b, B, K, N, BN));
+    mp.c = mp.d = mp.a;  // unused ones keep a valid map
+    if (ok && C) ok = make_map_2d_bf16(&mp.c, C, N, M, BM);
+    if (ok && D) ok = make_map_2d_bf16(&mp.d, D, N, M, BM);
+    if (!ok) return DR_ERR_CUDA;
+    Args a;
+    a.M = M; a.N = N; a.K = K; a.a_mn = a_mn; a.b_mn = b_mn; a.has_c = C != nullptr;
+    a.d32 = d32; a.slice_elems = slice_elems; a.nsplit = nsplit;
+    a.kslice = ((K + nsplit - 1) / nsplit + BK - 1) / BK * BK;
+    const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN) * nsplit, sms = sm_count();
+    if (sms <= 0) return DR_ERR_CUDA;
+    const size_t smem = SMEM_BYTES + 1024;
+    if (cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return DR_ERR_CUDA;
+    k_gemm_tc<<<tiles < sms ? tiles : sms, NTHREADS, smem, s>>>(mp, a);
+    return cudaGetLastError() == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+}
+
+int gemm_f32(const float *A, int a_t, const float *B, int b_t, const float *C, float *D, int M, int N, int K,
+             cudaStream_t s) {
+    const dim3 grid((N + 63) / 64, (M + 63) / 64);
+    if (grid.y > 65535) return DR_ERR_UNSUPPORTED;
+    k_gemm_f32<<<grid, 256, 0, s>>>(A, B, C, D, M, N, K, a_t, b_t);
+    return cudaGetLastError() == cudaSuccess ? DR_OK : DR_ERR_CUDA;
 }
 
 }  // namespace clv
@@ -132,25 +362,41 @@ size_t clvr_ws_bytes() { return clv::WS; }
 
 int clvr_fwd_run(const void *U, const void *W, const void *h, void *h_out, int M, int K, int N, bool bf16,
                  void *ws, size_t ws_bytes, cudaStream_t s) {
-    bool ok = false;
-    cublasLtHandle_t lt = clv::handle(&ok);
-    if (!ok) return DR_ERR_CUDA;
-    const cudaDataType_t t = bf16 ? CUDA_R_16BF : CUDA_R_32F;
-    return clv::status(clv::gemm(lt, U, false, W, false, h, h_out, M, N, K, t, t, h ? 1.f : 0.f, ws, ws_bytes, s));
+    (void)ws; (void)ws_bytes;
+    if (!bf16)
+        return clv::gemm_f32((const float *)U, 0, (const float *)W, 0, (const float *)h, (float *)h_out, M, N, K, s);
+    // A = U [M][K] (K-major), B = W [K][N] (MN-major)
+    return clv::gemm_bf16(U, 0, W, 1, h, h_out, nullptr, M, N, K, 1, 0, s);
 }
 
 int clvr_bwd_run(const void *U, const void *W, const void *dH, void *dU, float *dW, int M, int K, int N, bool bf16,
                  void *ws, size_t ws_bytes, cudaStream_t s) {
-    bool ok = false;
-    cublasLtHandle_t lt = clv::handle(&ok);
-    if (!ok) return DR_ERR_CUDA;
-    const cudaDataType_t t = bf16 ? CUDA_R_16BF : CUDA_R_32F;
-    if (dU) {  // dU [M][K] = dH [M][N] W^T, W [K][N]
-        const int rc = clv::status(clv::gemm(lt, dH, false, W, true, nullptr, dU, M, K, N, t, t, 0.f, ws, ws_bytes, s));
+    if (!bf16) {
+        int rc = DR_OK;
+        if (dU) rc = clv::gemm_f32((const float *)dH, 0, (const float *)W, 1, nullptr, (float *)dU, M, K, N, s);
+        if (rc == DR_OK && dW) rc = clv::gemm_f32((const float *)U, 1, (const float *)dH, 0, nullptr, dW, K, N, M, s);
+        return rc;
+    }
+    if (dU) {  // dU [M][K] = dH [M][N] W^T: A = dH (K-major), B = W [K][N] read as [N'=K][K'=N] (K-major)
+        const int rc = clv::gemm_bf16(dH, 0, W, 0, nullptr, dU, nullptr, M, K, N, 1, 0, s);
         if (rc != DR_OK) return rc;
     }
-    if (dW)  // dW [K][N] = U^T dH, U [M][K]
-        return clv::status(clv::gemm(lt, U, true, dH, false, nullptr, dW, K, N, M, t, CUDA_R_32F, 0.f, ws, ws_bytes, s));
+    if (dW) {  // dW [K][N] = U^T dH: A = U [M][K] (MN-major), B = dH [M][N] (MN-major); the M-long
+               // reduction in slices (enough work items for every SM) with fp32 partials
+        const size_t elems = (size_t)K * N;
+        const int tiles = ((K + clv::BM - 1) / clv::BM) * ((N + clv::BN - 1) / clv::BN), sms = clv::sm_count();
+        int nsplit = sms > 0 ? (sms + tiles - 1) / tiles : 1;
+        nsplit = nsplit < clv::MAX_SPLIT ? nsplit : clv::MAX_SPLIT;
+        const int kb = (M + clv::BK - 1) / clv::BK;
+        nsplit = nsplit < kb ? nsplit : (kb > 0 ? kb : 1);
+        while (nsplit > 1 && (size_t)nsplit * elems * sizeof(float) > ws_bytes) --nsplit;
+        if (nsplit == 1) return clv::gemm_bf16(U, 1, dH, 1, nullptr, nullptr, dW, K, N, M, 1, elems, s);
+        float *part = (float *)ws;
+        int rc = clv::gemm_bf16(U, 1, dH, 1, nullptr, nullptr, part, K, N, M, nsplit, elems, s);
+        if (rc != DR_OK) return rc;
+        clv::k_sum_slices<<<148 * 4, 256, 0, s>>>(part, dW, elems, nsplit);
+        return cudaGetLastError() == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+    }
     return DR_OK;
 }
 

@@ -56,6 +56,11 @@ struct Tensors {
     const float *dS_T;
     void *dq, *dk, *dv, *dalpha, *dbeta;
     float *dS0;
+    // the fused forward (delta_rule_fwd_fused): q, k, alpha, beta hold the raw projections and
+    // logits; the post-operation's gate logits and weight, and its output y
+    const void *gate_o;
+    const float *w_norm;
+    void *y;
 };
 
 // Optional launch timing: records ev[i] on the stream just before kernel launch i

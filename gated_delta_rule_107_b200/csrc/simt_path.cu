@@ -1183,6 +1183,7 @@ __device__ __forceinline__ void intra_tiled(const Geo &g, const IO<TI> &io, cons
 // factorised form takes every chunk it accepts, the direct form the rest.
 template <typename TI>
 __global__ void __launch_bounds__(NT) k_bwd_intra(Geo g, IO<TI> io, SimtWs w) {
+    if (w.only && !w.only[g.chunk(blockIdx.z, blockIdx.y, blockIdx.x)]) return;  // uniform over the CTA
     if (g.C == 64) {
         int wide = 0;
         if (g.variant == VAR_KDA) {

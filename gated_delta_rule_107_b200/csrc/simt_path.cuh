@@ -19,6 +19,7 @@ struct SimtWs {
     float *dWm;  // [B,H,N,C,dk]  -dU S^T   (= dL/dW)
     float *Tm;   // [B,H,N,C,dk]  U dS+^T
     float *RS;   // [B,H,N,dk]    rowsum(S .* dS+)
+    const int *only;  // optional [B,H,N]: the intra-chunk gradient kernel serves the flagged chunks alone
 };
 
 size_t simt_ws_bytes(const Geo &g, bool bwd);

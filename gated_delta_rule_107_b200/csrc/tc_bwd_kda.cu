@@ -1,0 +1,510 @@
+// tc_bwd_kda.cu -- KDA's intra-chunk gradients on tcgen05 (bf16, dk = dv = 128, C = 64).
+//
+// Backward of the chunked form of "线性注意力架构演进与Kimi Delta Attention创新实践" (sections
+// 2.1, 2.2, 6.2, 7.1) for one chunk of one (b, h), with channel-wise gates.  With g[r][c] the
+// in-chunk cumulative log gate, S = S_n, dS+ = dL/dS_{n+1}, dU = dL/dU (the reverse chain's), U,
+// W, U~, T = (I + A)^-1 and M[r][i] = sum_c k_rc k_ic e^{g_rc - g_ic} (the forward's, kept):
+//   Qd = dO S^T,  dWm = -dU S^T,  Tm = U dS+^T,  RS_c = sum_j S_cj dS+_cj
+//   dB_k = T^T dWm,  dB_v = T^T dU
+//   dA = -strict_tril(dB_k W^T + dB_v U~^T),  dM = diag(beta) dA,  dP = tril(dO U^T)
+//   X_rc  = sum_i dP_ri k_ic e^{g_rc - g_ic},   Yv_rc = sum_i dM_ri k_ic e^{g_rc - g_ic}
+//   Z_ic  = sum_r (dM_ri k_rc + dP_ri q_rc) e^{g_rc - g_ic}
+//   dq = e^g Qd + X,   dk = Yv + Z + beta e^g dB_k + e^{g_C - g} Tm,   dv = diag(beta) dB_v
+//   dg = q dq + k (Yv - Z) + beta e^g k dB_k - k e^{g_C - g} Tm;  dg_C += sum_r k e^{g_C - g} Tm + e^{g_C} RS
+//   dbeta_r = sum_i dA_ri M_ri + e^g k . dB_k + v . dB_v;   d log alpha = reverse cumsum of dg
+//
+// Every per-(token, channel) quantity is formed channel-major -- the transposed product, with the
+// key channel c as the 128-row side -- so that TMEM lane c holds channel c of every token: the
+// gate factors, the chunk-end terms and the reverse cumulative sum are then per-thread work, and
+// each warp's stores cover 32 consecutive channels.  The pair factors e^{g_rc - g_ic} are split at
+// a token of each 16-token block (as in the forward): for X and Yv at the first token b of row
+// r's block (operand sections Km_R = k_i e^{g_b - g_i}), for Z at the last token e of row i's
+// block (Kp_I = k_r e^{g_r - g_e}, Qp_I likewise); every factor outside the diagonal block is
+// <= 1, inside it at most e^{the block's fall}.  Chunks whose gate falls more than KDA_DIAG_SPAN
+// inside a block are left to the CUDA-core gradient kernel (this kernel skips them).
+//
+// One CTA of 128 threads per chunk, phases in order (each a batch of MMAs, then an epilogue):
+//   A  loads; [Qd^T | -dWm^T] = S [dO ; dU]^T, Tm^T = dS+ U^T;  RS, g (from log alpha), dWm^T tile
+//   B  loads of M, W, U~;  dB_k^T = dWm^T T,  dB_v^T = dU^T T;  their bf16 tiles
+//   C  dA' = dB [W | U~]^T and its transpose, [dO ; U][dO ; U]^T (dP and dP^T in one product);
+//      dM, dP, dM^T, dP^T tiles, the dbeta part of A;  the gate-scaled sections Km, Kp, Qp
+//   D  X^T, Yv^T, Z^T (block by block, N = 16);  the final per-channel epilogue
+// Every wait is bounded (~1 s); an expired wait raises the device error word.
+#include "tc_host.cuh"
+#include "tc_path.cuh"
+#include "tc_ptx.cuh"
+#include "tc_tile.cuh"
+
+namespace dr {
+namespace tck {
+
+using namespace dr::tc;
+using dr::tcf::ld_chunk;
+using dr::tcf::st_chunk;
+
+constexpr int C = 64, DK = 128, DV = 128;
+constexpr int NTHREADS = 128;
+// shared memory (bytes from a 1024-aligned base); regions are reused phase by phase
+//   phase A:   S [0, 32K), dS+ [32K, 64K), [dO ; dU] [64K, 96K), [dO ; U] [96K, 128K),
+//              T [128K, 136K), log alpha [136K, 152K), q [152K, 168K), k [168K, 184K)
+//   E0 writes: G (fp32) [184K, 216K), dWm^T [136K, 152K) (after log alpha is read)
+//   phase B:   M [0, 8K), W [8K, 24K), U~ [24K, 40K);  E1 writes dB_k^T [64K, 80K), dB_v^T [80K, 96K)
+//   E2 writes: dM [120K, 128K), dP [128K, 136K), dM^T [136K, 144K), dP^T [144K, 152K)
+//   build:     Km [0, 40K), Kp [40K, 80K), Qp [80K, 120K)
+constexpr uint32_t R_S = 0, R_DS = 32768, R_OU = 65536, R_OV = 98304, R_T = 131072, R_AL = 139264;
+constexpr uint32_t R_Q = 155648, R_K = 172032, R_G = 188416, R_DWM = 139264;
+constexpr uint32_t R_M = 0, R_W = 8192, R_UT = 24576, R_DBK = 65536, R_DBV = 81920;
+constexpr uint32_t R_DM = 122880, R_DP = 131072, R_DMT = 139264, R_DPT = 147456;
+constexpr uint32_t R_KM = 0, R_KP = 40960, R_QP = 81920;
+constexpr uint32_t SEC_PANEL = KDA_KH_ROWS * 128;  // 160 rows x 128 B: one 64-channel panel of a section set
+constexpr uint32_t R_MISC = R_G + 32768;           // 216K
+// misc: barriers, TMEM slot, abort flag, then per-token and per-channel vectors (floats)
+constexpr uint32_t M_BAR = 0;  // [0] phase-A loads, [1] phase-B loads, [2] MMA
+constexpr uint32_t M_TMEM = 32, M_ABORT = 36;
+constexpr uint32_t M_BETA = 64;          // [64] beta
+constexpr uint32_t M_DBA = M_BETA + 256;  // [64] the dbeta part of A
+constexpr uint32_t M_RED = M_DBA + 256;   // [2 kinds][4 warps][64] dbeta partial sums
+constexpr uint32_t SMEM_BYTES = R_MISC + M_RED + 2 * 4 * 64 * 4;
+static_assert(R_MISC + M_RED + 2048 <= 227 * 1024 - 1024, "shared memory");
+// TMEM columns (lane = key channel c, or value channel j for dB_v^T, or token row for dA', dP)
+constexpr uint32_t TM_QD = 0, TM_X = 64, TM_TM = 128, TM_DBK = 192, TM_DBV = 256, TM_YV = 320, TM_D5 = 384,
+                   TM_Z = 384, TM_COLS = 512;
+constexpr uint32_t LOADA_BYTES = 4 * 32768 + 8192 + 3 * 16384, LOADB_BYTES = 8192 + 2 * 16384;
+
+struct Maps {
+    CUtensorMap q, k, dout, alpha;  // [B, T, H, 128] bf16; box 64 channels x 64 tokens
+    CUtensorMap S, dS;              // [chunks * 128][128] bf16; box 64 x 128
+    CUtensorMap U, dU, W, Ut;       // [chunks * 64][128] bf16; box 64 x 64
+    CUtensorMap T, M;               // [chunks * 64][64] bf16; box 64 x 64
+};
+
+struct Args {
+    const __nv_bfloat16 *beta, *v;  // [B, T, H], [B, T, H, 128]
+    __nv_bfloat16 *dq, *dk, *dv, *dalpha, *dbeta;
+    const int *kwide;               // [chunks]: left to the CUDA-core kernel
+    int T, H, N;
+};
+
+// first row of Km's section R (rows i = 0 .. 16 R + 15) and of Kp's / Qp's section I (rows 16 I .. 63)
+__host__ __device__ constexpr int km_sec(int R) { return 8 * R * (R + 1); }
+__host__ __device__ constexpr int kp_sec(int I) { return 64 * I - 8 * I * (I - 1); }
+static_assert(km_sec(4) == KDA_KH_ROWS && kp_sec(4) == KDA_KH_ROWS, "160 rows per section set");
+
+// element (row, c) of a [rows][128] bf16 tile stored as two 64-column swizzled panels of `panel` bytes
+__device__ __forceinline__ uint32_t el_off(int row, int c, uint32_t panel) {
+    return (uint32_t)(c >> 6) * panel + swz(row, (c & 63) >> 3) + (c & 7) * 2;
+}
+__device__ __forceinline__ float ld_bf(const unsigned char *base, uint32_t off) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(base + off));
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constant__ Maps mp, Args a) {
+    const int ci = blockIdx.x;
+    if (a.kwide[ci]) return;  // uniform: the CUDA-core kernel takes this chunk
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    unsigned char *misc = sm + R_MISC;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(misc + M_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + M_TMEM);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + M_ABORT);
+    float *betas = reinterpret_cast<float *>(misc + M_BETA);
+    float *dba = reinterpret_cast<float *>(misc + M_DBA);
+    float *red = reinterpret_cast<float *>(misc + M_RED);
+    const float *G = reinterpret_cast<const float *>(sm + R_G);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n = ci % a.N, bh = ci / a.N, h = bh % a.H, b = bh / a.H;
+    const int T = a.T, H = a.H, t0 = n * C, L = min(C, T - t0);
+    auto trow_g = [&](int rr) -> size_t { return ((size_t)b * T + t0 + rr) * H + h; };
+
+    int armed[3] = {0, 0, 0};
+    if (tid == 0) {
+        for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        mbar_arrive_tx(&bar[0], LOADA_BYTES);
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            tma_load_2d(sm + R_S + p * 16384, &mp.S, 64 * p, ci * DK, &bar[0]);
+            tma_load_2d(sm + R_DS + p * 16384, &mp.dS, 64 * p, ci * DK, &bar[0]);
+            tma_load_4d(sm + R_OU + p * 16384, &mp.dout, 64 * p, h, t0, b, &bar[0]);
+            tma_load_2d(sm + R_OU + p * 16384 + 8192, &mp.dU, 64 * p, ci * C, &bar[0]);
+            tma_load_4d(sm + R_OV + p * 16384, &mp.dout, 64 * p, h, t0, b, &bar[0]);
+            tma_load_2d(sm + R_OV + p * 16384 + 8192, &mp.U, 64 * p, ci * C, &bar[0]);
+            tma_load_4d(sm + R_AL + p * 8192, &mp.alpha, 64 * p, h, t0, b, &bar[0]);
+            tma_load_4d(sm + R_Q + p * 8192, &mp.q, 64 * p, h, t0, b, &bar[0]);
+            tma_load_4d(sm + R_K + p * 8192, &mp.k, 64 * p, h, t0, b, &bar[0]);
+        }
+        tma_load_2d(sm + R_T, &mp.T, 0, ci * C, &bar[0]);
+        armed[0] = 1;
+    }
+    if (tid < C) betas[tid] = tid < L ? __bfloat162float(a.beta[trow_g(tid)]) : 0.f;
+    if (warp == 0) tmem_alloc(tmem_slot, TM_COLS);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);  // this warp's lane quarter
+    auto consensus = [&](bool ok) -> bool { return !named_sync_any(1, NTHREADS, !ok || *abort_flag != 0); };
+    uint32_t ph = 0;
+    auto wait_mma = [&]() -> bool {
+        const bool ok = mbar_wait(&bar[2], ph & 1, abort_flag);
+        ph++;
+        fence_after_sync();
+        return consensus(ok);
+    };
+    auto commit = [&]() {
+        mma_commit(&bar[2]);
+        armed[2]++;
+    };
+    auto u32 = [&](uint32_t off) { return smem_u32(sm + off); };
+    const int c = tid;  // this thread's key channel (TMEM lane)
+
+    bool ok = consensus(mbar_wait(&bar[0], 0, abort_flag));
+    // ======================= phase A products =======================
+    if (ok && tid == 0) {
+        const uint32_t id0 = idesc_bf16(128, 128, 0, 0), id1 = idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {  // K = dv in steps of 16
+            const uint32_t ka = (k >> 2) * 16384 + (k & 3) * 32;
+            mma_bf16(tbase + TM_QD, sdesc(u32(R_S) + ka, 16, 1024), sdesc(u32(R_OU) + ka, 16, 1024), id0, k > 0);
+            mma_bf16(tbase + TM_TM, sdesc(u32(R_DS) + ka, 16, 1024), sdesc(u32(R_OV) + 8192 + ka, 16, 1024), id1,
+                     k > 0);
+        }
+        commit();
+    }
+    // while they run: g of channel c (prefix sum over the chunk's tokens; tokens past T add 0)
+    if (ok) {
+        float run = 0.f;
+        float *Gw = reinterpret_cast<float *>(sm + R_G);
+        for (int r = 0; r < C; ++r) {
+            run += ld_bf(sm + R_AL, el_off(r, c, 8192));
+            Gw[r * DK + c] = run;
+        }
+    }
+    if (ok) ok = wait_mma();
+    float rs = 0.f;  // RS_c
+    if (ok) {
+        // RS_c from the state tiles; then -dWm^T row c (TMEM columns 64..127 of [Qd^T | dU S^T]) as
+        // the bf16 A operand of dB_k^T, over the log-alpha tile (read by every thread above)
+#pragma unroll
+        for (int p = 0; p < 2; ++p)
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                float s8[8], d8[8];
+                const uint32_t o = (uint32_t)p * 16384 + swz(c, ch);
+                ld_chunk(sm + R_S, o, s8);
+                ld_chunk(sm + R_DS, o, d8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) rs += s8[e] * d8[e];
+            }
+    }
+    ok = consensus(ok);  // the log-alpha tile and the state tiles are read
+    if (ok) {
+        float v[64];
+        tmem_ld16(tl + TM_QD + 64, v); tmem_ld16(tl + TM_QD + 80, v + 16);
+        tmem_ld16(tl + TM_QD + 96, v + 32); tmem_ld16(tl + TM_QD + 112, v + 48);
+        wait_ld();
+#pragma unroll
+        for (int j = 0; j < 64; ++j) v[j] = -v[j];  // dWm^T = -(dU S^T)^T
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_DWM, swz(c, ch), v + ch * 8);
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    ok = consensus(ok);
+    // ======================= phase B =======================
+    if (ok && tid == 0) {
+        fence_after_sync();
+        mbar_arrive_tx(&bar[1], LOADB_BYTES);
+        tma_load_2d(sm + R_M, &mp.M, 0, ci * C, &bar[1]);
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            tma_load_2d(sm + R_W + p * 8192, &mp.W, 64 * p, ci * C, &bar[1]);
+            tma_load_2d(sm + R_UT + p * 8192, &mp.Ut, 64 * p, ci * C, &bar[1]);
+        }
+        armed[1] = 1;
+        // dB_k^T = dWm^T T (A K-major [c][r]; B = T [r][i] MN-major)
+        // dB_v^T = dU^T T  (A = dU [r][j] MN-major: the two 64-column panels 16K apart in [dO ; dU])
+        const uint32_t idk = idesc_bf16(128, 64, 0, 1), idv = idesc_bf16(128, 64, 1, 1);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            mma_bf16(tbase + TM_DBK, sdesc(u32(R_DWM) + k * 32, 16, 1024), sdesc(u32(R_T) + k * 2048, 8192, 1024), idk,
+                     k > 0);
+            mma_bf16(tbase + TM_DBV, sdesc(u32(R_OU) + 8192 + k * 2048, 16384, 1024),
+                     sdesc(u32(R_T) + k * 2048, 8192, 1024), idv, k > 0);
+        }
+        commit();
+    }
+    if (ok) ok = wait_mma();
+    if (ok) {  // the bf16 tiles dB_k^T [c][i] and dB_v^T [j][i] (lane = c, or j)
+        float v[64];
+        tmem_ld16(tl + TM_DBK, v); tmem_ld16(tl + TM_DBK + 16, v + 16);
+        tmem_ld16(tl + TM_DBK + 32, v + 32); tmem_ld16(tl + TM_DBK + 48, v + 48);
+        wait_ld();
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_DBK, swz(c, ch), v + ch * 8);
+        tmem_ld16(tl + TM_DBV, v); tmem_ld16(tl + TM_DBV + 16, v + 16);
+        tmem_ld16(tl + TM_DBV + 32, v + 32); tmem_ld16(tl + TM_DBV + 48, v + 48);
+        wait_ld();
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_DBV, swz(c, ch), v + ch * 8);
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    ok = consensus(ok);
+    if (ok) ok = consensus(mbar_wait(&bar[1], 0, abort_flag));  // M, W, U~
+    // ======================= phase C products =======================
+    if (ok && tid == 0) {
+        fence_after_sync();
+        // dA'[r][i] = dB_k[r] . W[i] + dB_v[r] . U~[i]: A = dB^T tiles read MN-major (rows 64-127 of
+        // the M = 128 product are discarded), B = W, U~ K-major
+        const uint32_t ida = idesc_bf16(128, 64, 1, 0), idt = idesc_bf16(128, 64, 0, 1), id5 = idesc_bf16(128, 128, 0, 0);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const uint32_t at = (k < 8 ? u32(R_DBK) : u32(R_DBV)) + (k & 7) * 2048;
+            const uint32_t bw = (k < 8 ? u32(R_W) : u32(R_UT)) + ((k & 7) >> 2) * 8192 + (k & 3) * 32;
+            mma_bf16(tbase + TM_X, sdesc(at, 8192, 1024), sdesc(bw, 16, 1024), ida, k > 0);
+        }
+        // dA'^T[i][r]: A = W, U~ K-major, B = dB^T tiles MN-major
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const uint32_t aw = (k < 8 ? u32(R_W) : u32(R_UT)) + ((k & 7) >> 2) * 8192 + (k & 3) * 32;
+            const uint32_t bt = (k < 8 ? u32(R_DBK) : u32(R_DBV)) + (k & 7) * 2048;
+            mma_bf16(tbase + TM_YV, sdesc(aw, 16, 1024), sdesc(bt, 8192, 1024), idt, k > 0);
+        }
+        // [dO ; U] [dO ; U]^T: dP = dO U^T at lanes 0-63 / columns 64-127, dP^T at lanes 64-127 / 0-63
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const uint32_t ka = (k >> 2) * 16384 + (k & 3) * 32;
+            mma_bf16(tbase + TM_D5, sdesc(u32(R_OV) + ka, 16, 1024), sdesc(u32(R_OV) + ka, 16, 1024), id5, k > 0);
+        }
+        commit();
+    }
+    if (ok) ok = wait_mma();
+    // ---- E2: the masked tiles dM, dP [r][i] and dM^T, dP^T [i][r]; the dbeta part of A ----
+    if (ok) {
+        float x[64];
+        if (warp < 2) {
+            const int r = tid;  // token row r (and, for the transposed products, row i = tid)
+            // dA'[r][i] -> dM[r][i] = -beta_r dA' (i < r), dbeta_A
+            tmem_ld16(tl + TM_X, x); tmem_ld16(tl + TM_X + 16, x + 16);
+            tmem_ld16(tl + TM_X + 32, x + 32); tmem_ld16(tl + TM_X + 48, x + 48);
+            wait_ld();
+            float db = 0.f;
+            const float br = betas[r];
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                float m8[8], w8[8];
+                ld_chunk(sm + R_M, swz(r, ch), m8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int i = ch * 8 + e;
+                    const float d = i < r ? -x[i] : 0.f;
+                    db += d * m8[e];
+                    w8[e] = br * d;
+                }
+                st_chunk(sm + R_DM, swz(r, ch), w8);
+            }
+            dba[r] = db;
+            // dP[r][i] (i <= r)
+            tmem_ld16(tl + TM_D5 + 64, x); tmem_ld16(tl + TM_D5 + 80, x + 16);
+            tmem_ld16(tl + TM_D5 + 96, x + 32); tmem_ld16(tl + TM_D5 + 112, x + 48);
+            wait_ld();
+#pragma unroll
+            for (int i = 0; i < 64; ++i) x[i] = i <= r ? x[i] : 0.f;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_DP, swz(r, ch), x + ch * 8);
+            // dA'^T[i][r] -> dM^T[i][r] = -beta_r dA'^T (r > i)
+            const int i = tid;
+            tmem_ld16(tl + TM_YV, x); tmem_ld16(tl + TM_YV + 16, x + 16);
+            tmem_ld16(tl + TM_YV + 32, x + 32); tmem_ld16(tl + TM_YV + 48, x + 48);
+            wait_ld();
+#pragma unroll
+            for (int rr = 0; rr < 64; ++rr) x[rr] = rr > i ? -betas[rr] * x[rr] : 0.f;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_DMT, swz(i, ch), x + ch * 8);
+        } else {
+            const int i = tid - 64;  // dP^T[i][r] (r >= i)
+            tmem_ld16(tl + TM_D5, x); tmem_ld16(tl + TM_D5 + 16, x + 16);
+            tmem_ld16(tl + TM_D5 + 32, x + 32); tmem_ld16(tl + TM_D5 + 48, x + 48);
+            wait_ld();
+#pragma unroll
+            for (int rr = 0; rr < 64; ++rr) x[rr] = rr >= i ? x[rr] : 0.f;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_DPT, swz(i, ch), x + ch * 8);
+        }
+    }
+    ok = consensus(ok);  // M, W, U~ and the dB tiles are read: the sections may take their space
+    // ---- the gate-scaled sections (thread = 16-byte chunk of a row, 8 channels) ----
+    //   Km_R[i] = k_i e^{g_16R - g_i} (i <= 16 R + 15);  Kp_I[r] = k_r e^{g_r - g_{16 I + 15}},
+    //   Qp_I[r] = q_r e^{g_r - g_{16 I + 15}} (r >= 16 I); exponents clamped at 80 (they exceed 0
+    //   only inside a block, by at most KDA_DIAG_SPAN here)
+    if (ok) {
+        for (int x = tid; x < KDA_KH_ROWS * 16; x += NTHREADS) {
+            const int row = x >> 4, cc = x & 15, c0 = cc * 8;
+            const uint32_t o = (uint32_t)(cc >> 3) * SEC_PANEL + swz(row, cc & 7);
+            // Km row: section R, token i
+            int R = 0;
+            while (R < 3 && row >= km_sec(R + 1)) ++R;
+            const int ti = row - km_sec(R);
+            // Kp / Qp row: section I, token r
+            int I = 0;
+            while (I < 3 && row >= kp_sec(I + 1)) ++I;
+            const int tr = 16 * I + (row - kp_sec(I));
+            float ki[8], kr[8], qr[8], vm[8], vp[8], vq[8];
+            ld_chunk(sm + R_K, (uint32_t)(c0 >> 6) * 8192 + swz(ti, (c0 & 63) >> 3), ki);
+            ld_chunk(sm + R_K, (uint32_t)(c0 >> 6) * 8192 + swz(tr, (c0 & 63) >> 3), kr);
+            ld_chunk(sm + R_Q, (uint32_t)(c0 >> 6) * 8192 + swz(tr, (c0 & 63) >> 3), qr);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int cc2 = c0 + e;
+                vm[e] = ki[e] * __expf(fminf(G[16 * R * DK + cc2] - G[ti * DK + cc2], 80.f));
+                const float f = __expf(fminf(G[tr * DK + cc2] - G[(16 * I + 15) * DK + cc2], 80.f));
+                vp[e] = kr[e] * f;
+                vq[e] = qr[e] * f;
+            }
+            st_chunk(sm + R_KM, o, vm);
+            st_chunk(sm + R_KP, o, vp);
+            st_chunk(sm + R_QP, o, vq);
+        }
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    ok = consensus(ok);
+    // ======================= phase D products: X^T, Yv^T, Z^T (N = 16 per block) =======================
+    if (ok && tid == 0) {
+        fence_after_sync();
+        const uint32_t id = idesc_bf16(128, 16, 1, 0);
+        for (int R = 0; R < 4; ++R) {
+            for (int kk = 0; kk <= R; ++kk) {  // tokens i of the blocks up to R
+                const uint64_t am = sdesc(u32(R_KM) + (uint32_t)(km_sec(R) + 16 * kk) * 128, SEC_PANEL, 1024);
+                mma_bf16(tbase + TM_X + 16 * R, am, sdesc(u32(R_DP) + 2048 * R + kk * 32, 16, 1024), id, kk > 0);
+                mma_bf16(tbase + TM_YV + 16 * R, am, sdesc(u32(R_DM) + 2048 * R + kk * 32, 16, 1024), id, kk > 0);
+            }
+        }
+        for (int I = 0; I < 4; ++I) {
+            for (int kk = I; kk < 4; ++kk) {  // tokens r of the blocks from I on
+                const uint32_t ro = (uint32_t)(kp_sec(I) + 16 * (kk - I)) * 128;
+                mma_bf16(tbase + TM_Z + 16 * I, sdesc(u32(R_KP) + ro, SEC_PANEL, 1024),
+                         sdesc(u32(R_DMT) + 2048 * I + kk * 32, 16, 1024), id, kk > I);
+                mma_bf16(tbase + TM_Z + 16 * I, sdesc(u32(R_QP) + ro, SEC_PANEL, 1024),
+                         sdesc(u32(R_DPT) + 2048 * I + kk * 32, 16, 1024), id, 1);
+            }
+        }
+        commit();
+    }
+    if (ok) ok = wait_mma();
+    // ======================= final epilogue: thread c (and thread j = c for dv) =======================
+    if (ok) {
+        const float gL = G[(C - 1) * DK + c];
+        float dgr[64];
+        float dgc = 0.f;
+#pragma unroll
+        for (int rb = 0; rb < 4; ++rb) {
+            float qd[16], tm[16], bk[16], xx[16], yv[16], zz[16], bv[16];
+            tmem_ld16(tl + TM_QD + 16 * rb, qd);
+            tmem_ld16(tl + TM_TM + 16 * rb, tm);
+            tmem_ld16(tl + TM_DBK + 16 * rb, bk);
+            tmem_ld16(tl + TM_X + 16 * rb, xx);
+            tmem_ld16(tl + TM_YV + 16 * rb, yv);
+            tmem_ld16(tl + TM_Z + 16 * rb, zz);
+            tmem_ld16(tl + TM_DBV + 16 * rb, bv);
+            wait_ld();
+            const float gb = G[16 * rb * DK + c], ge = G[(16 * rb + 15) * DK + c];
+            float sbk[16], sbv[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int r = 16 * rb + e;
+                const float g = G[r * DK + c], br = betas[r];
+                const float qv = ld_bf(sm + R_Q, el_off(r, c, 8192)), kv = ld_bf(sm + R_K, el_off(r, c, 8192));
+                const float gam = __expf(g), eb = __expf(gL - g);
+                const float fb = __expf(g - gb), fe = __expf(fminf(ge - g, 80.f));
+                const float X = fb * xx[e], Yv = fb * yv[e], Z = fe * zz[e];
+                const float dq = gam * qd[e] + X;
+                const float t = eb * tm[e], sb = br * gam * bk[e];
+                const float dk = Yv + Z + sb + t;
+                dgr[r] = qv * dq + kv * (Yv - Z + sb - t);
+                dgc += kv * t;
+                sbk[e] = gam * kv * bk[e];
+                if (r < L) {
+                    const size_t o = trow_g(r) * DK + c;
+                    a.dq[o] = __float2bfloat16_rn(dq);
+                    a.dk[o] = __float2bfloat16_rn(dk);
+                }
+                // thread c is also value channel j = c of dB_v^T
+                float vv = 0.f;
+                if (r < L) {
+                    const size_t o = trow_g(r) * DV + c;
+                    vv = __bfloat162float(a.v[o]);
+                    a.dv[o] = __float2bfloat16_rn(br * bv[e]);
+                }
+                sbv[e] = vv * bv[e];
+            }
+            // sums over the channels (threads) per token: warps, then 4 partials
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const float s1 = warp_sum(sbk[e]), s2 = warp_sum(sbv[e]);
+                if (lane == 0) {
+                    red[(0 * 4 + warp) * 64 + 16 * rb + e] = s1;
+                    red[(1 * 4 + warp) * 64 + 16 * rb + e] = s2;
+                }
+            }
+        }
+        // d log alpha: the chunk-end terms belong to the last row, then the reverse cumulative sum
+        float run = dgc + __expf(gL) * rs;
+#pragma unroll
+        for (int r = C - 1; r >= 0; --r) {
+            run += dgr[r];
+            if (r < L) a.dalpha[trow_g(r) * DK + c] = __float2bfloat16_rn(run);
+        }
+    }
+    ok = consensus(ok);
+    if (ok && tid < L) {
+        float s = dba[tid];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) s += red[(0 * 4 + w) * 64 + tid] + red[(1 * 4 + w) * 64 + tid];
+        a.dbeta[trow_g(tid)] = __float2bfloat16_rn(s);
+    }
+    if (tid == 0 && *abort_flag) {  // let whatever was issued land before the CTA leaves
+        volatile int dummy = 0;
+        for (int i = 0; i < 2; ++i)
+            if (armed[i] > 0) mbar_wait(&bar[i], 0, &dummy, 100000000ull);
+        // every MMA batch ends with a commit: wait for the phases not waited for yet, in order
+        for (uint32_t p = ph; p < (uint32_t)armed[2]; ++p) mbar_wait(&bar[2], p & 1, &dummy, 100000000ull);
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == 0) tmem_dealloc(tbase, TM_COLS);
+}
+
+}  // namespace tck
+
+cudaError_t tc_bwd_kda(const Geo &g, const Tensors &t, const TcWs &w, cudaStream_t s, Rec &rec) {
+    using namespace tck;
+    Maps mp;
+    const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;
+    bool ok = tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) && tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64) &&
+              tc::make_map_4d_bf16(&mp.alpha, t.alpha, DK, H, T, Bn, 64) &&
+              tc::make_map_2d_bf16(&mp.S, w.Sn, DV, NC * DK, 128) && tc::make_map_2d_bf16(&mp.dS, w.dSn, DV, NC * DK, 128) &&
+              tc::make_map_2d_bf16(&mp.U, w.Un, DV, NC * C, 64) && tc::make_map_2d_bf16(&mp.dU, w.dUn, DV, NC * C, 64) &&
+              tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.Ut, w.Ut, DV, NC * C, 64) &&
+              tc::make_map_2d_bf16(&mp.T, w.Tn, C, NC * C, 64) && tc::make_map_2d_bf16(&mp.M, w.KK, C, NC * C, 64);
+    if (ok) ok = t.dout && tc::make_map_4d_bf16(&mp.dout, t.dout, DV, H, T, Bn, 64);  // the backward requires dO
+    if (!ok) return cudaErrorInvalidValue;
+    Args a;
+    a.beta = (const __nv_bfloat16 *)t.beta; a.v = (const __nv_bfloat16 *)t.v;
+    a.dq = (__nv_bfloat16 *)t.dq; a.dk = (__nv_bfloat16 *)t.dk; a.dv = (__nv_bfloat16 *)t.dv;
+    a.dalpha = (__nv_bfloat16 *)t.dalpha; a.dbeta = (__nv_bfloat16 *)t.dbeta; a.kwide = w.kwide;
+    a.T = g.T; a.H = g.H; a.N = g.N;
+    const size_t smem = SMEM_BYTES + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_bwd_kda_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    rec.mark(s);
+    k_bwd_kda_tc<<<(unsigned)NC, NTHREADS, smem, s>>>(mp, a);
+    return cudaGetLastError();
+}
+
+}  // namespace dr

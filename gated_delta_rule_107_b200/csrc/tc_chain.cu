@@ -39,8 +39,9 @@ constexpr int C = 64, DK = 128, DV = 128, DVB = 64;
 constexpr int NTHREADS = 288;  // warp 0 producer, warps 1-8 chain
 // shared memory (bytes from a 1024-aligned base): two stages of 80K, then the chain's tiles
 constexpr uint32_t STAGE = 81920;
-// forward stage: [W_p0 | q_p0 | W_p1 | q_p1], [U~ (this CTA's 64 columns) | P], [k_p0 | k_p1]
-constexpr uint32_t FS_WQ = 0, FS_UP = 32768, FS_K = 49152;
+// forward stage: [W_p0 | q_p0 | W_p1 | q_p1], [U~ (this CTA's 64 columns) | P], [k_p0 | k_p1],
+// and for the fused forward the output gate logits (this CTA's 64 columns)
+constexpr uint32_t FS_WQ = 0, FS_UP = 32768, FS_K = 49152, FS_G = 65536;
 // reverse stage: k, q, W (2 panels each); dO (this CTA's 64 columns); P; du, U (this CTA's 64 columns)
 constexpr uint32_t RS_K = 0, RS_Q = 16384, RS_W = 32768, RS_DO = 49152, RS_P = 57344, RS_DX = 65536,
                    RS_UN = 73728;
@@ -48,15 +49,22 @@ constexpr uint32_t OFF_S = 2 * STAGE;         // 16K  bf16 state [c][j]
 constexpr uint32_t OFF_U = OFF_S + 16384;     //  8K  U [r][j]        (reverse: dU [r][j])
 constexpr uint32_t OFF_UD = OFF_U + 8192;     //  8K  e^{g_C - g} U [r][j]
 constexpr uint32_t OFF_O = OFF_UD + 8192;     //  8K  o [r][j] (staging of the TMA store)
-constexpr uint32_t OFF_MISC = OFF_O + 8192;   //  4K
+constexpr uint32_t OFF_Y = OFF_O + 8192;      //  8K  fused forward: y [r][j] (staging)
+constexpr uint32_t OFF_MISC = OFF_Y + 8192;   //  4K
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 4096;
 // misc
 constexpr uint32_t M_BAR = 0;  // FULL0, FULL1, EMPTY0, EMPTY1, MMA
 constexpr uint32_t M_TMEM = 64, M_ABORT = 68;
 constexpr uint32_t M_CF = 256;  // per stage: [0..63] e^{g_C - g}, [64..127] e^g, [128] e^{g_C}
-constexpr uint32_t M_SKP = M_CF + 2 * 132 * 4;  // reverse: [2 column halves][64] row-sum partials
-enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_MMA, B_NUM };
-static_assert(M_SKP + 512 <= 4096, "misc overflow");
+constexpr uint32_t M_SKP = M_CF + 2 * 132 * 4;  // reverse: [2 column halves][64] row-sum partials;
+                                                // fused forward: the same for o's squares
+constexpr uint32_t M_XS = M_SKP + 512;          // fused forward: [2 chunk parities][64] the partner's
+                                                // row sums of squares (written by the partner CTA)
+constexpr uint32_t M_WN = M_XS + 512;           // fused forward: this CTA's 64 RMSNorm weights
+// B_XS0/1 (fused forward): the partner's row sums of a chunk parity have arrived
+enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_MMA, B_XS0, B_XS1, B_NUM };
+static_assert(B_NUM * 8 <= M_TMEM && M_WN + 256 <= 4096, "misc overflow");
+constexpr float POST_EPS = 1e-6f;  // y = o / sqrt(mean(o^2) + eps) w sigmoid(gate)
 
 struct FMaps {
     CUtensorMap q, k;       // [B, T, H, 128] bf16; box 64 x 64 tokens (KDA: the workspace's
@@ -65,6 +73,7 @@ struct FMaps {
     CUtensorMap P;          // [chunks * 64][64] bf16; box 64 x 64
     CUtensorMap out, u;     // forward outputs [B, T, H, 128] (stores)
     CUtensorMap Sn, Un;     // recompute outputs: [chunks * 128][128] box 64 x 128, [chunks * 64][128] (stores)
+    CUtensorMap gate, y;    // fused forward: output gate logits (load) and y (store), [B, T, H, 128]
 };
 struct RMaps {
     CUtensorMap q, k, dout, du;  // [B, T, H, 128] bf16
@@ -81,6 +90,8 @@ struct Args {
     float *skt;               // reverse output
     int B, T, H, N, has_du;
     const float *egc;         // KDA forward: [chunks][128] e^{g_C} per key channel
+    const float *rn;          // fused forward: [chunks][2][64] 1 / |k_r|, 1 / |q_r|
+    const float *wn;          // fused forward: RMSNorm weight [128]
 };
 
 // Producer side, KDA: the per-channel decay e^{g_C} of chunk ci into cf[0..127].
@@ -103,6 +114,23 @@ __device__ __forceinline__ void chunk_factors(const float *gb, size_t ci, float 
     if (lane == 0) cf[128] = __expf(gC);
 }
 
+// Fused forward: the same with the raw rows' norms folded in (k's rows by 1 / |k_r|, o's by 1 / |q_r|).
+__device__ __forceinline__ void chunk_factors_fused(const float *gb, const float *rn, size_t ci, float *cf,
+                                                    int lane) {
+    const float *gg = gb + ci * 2 * C, *rr = rn + ci * 2 * C;
+    const float gC = gg[C - 1];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        const int r = lane + 32 * hh;
+        const float x = gg[r];
+        cf[r] = __expf(gC - x) * rr[r];
+        cf[64 + r] = __expf(x) * rr[C + r];
+    }
+    if (lane == 0) cf[128] = __expf(gC);
+}
+
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + __expf(-x)); }
+
 // Chain thread layout: warps 1-8, two per TMEM lane quarter (warp & 3); the first four take
 // value columns 0-31 of this CTA's 64, the other four columns 32-63.
 struct ChainLane {
@@ -121,12 +149,15 @@ __device__ __forceinline__ void tmem_row32(uint32_t taddr, float *v) {
 
 // ====================================== forward chain ======================================
 // MODE 0: forward (o, u, S_T); 1: recompute for the backward (S_n, U of every chunk);
-// 2: forward that also keeps S_n and U for the backward.
+// 2: forward that also keeps S_n and U for the backward; 3: the fused forward (raw q, k through
+// the row norms; y = RMSNorm(o) w sigmoid(gate) in the output epilogue, the row sums of squares
+// exchanged with the partner CTA of the cluster; o stored only when requested).
 // KDA (MODE 0): q and k arrive gate-scaled (q e^g, k e^{g_C - g}), so the row factors are 1,
 // and the state decays by row: S <- Diag(e^{g_C}) S + (k e^{g_C - g})^T U.
 template <int MODE, int KDA>
 __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant__ FMaps mp, Args a) {
-    constexpr bool OUT = MODE != 1, KEEP = MODE != 0;
+    constexpr bool OUT = MODE != 1, KEEP = MODE == 1 || MODE == 2, FUSED = MODE == 3;
+    static_assert(!FUSED || !KDA, "the fused forward serves scalar gates");
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -142,14 +173,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
     const size_t ci0 = ((size_t)b * H + h) * N;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < B_NUM; ++i) mbar_init(&bar[i], (i == B_FULL0 || i == B_FULL1) ? 2 : 1);
+        for (int i = 0; i < B_NUM; ++i)
+            mbar_init(&bar[i], (i == B_FULL0 || i == B_FULL1) ? 2 : (i == B_XS0 || i == B_XS1) ? 64 : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
+    if (FUSED && threadIdx.x < DVB)
+        reinterpret_cast<float *>(sm + OFF_MISC + M_WN)[threadIdx.x] = a.wn[j0 + threadIdx.x];
     if (warp == 0) tmem_alloc(tmem_slot, 512);
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
+    if (FUSED) cluster_sync();  // the partner's barriers are initialised before any remote arrival
     const uint32_t tbase = *tmem_slot;
 
     if (warp == 0) {
@@ -161,7 +196,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             if (m >= 2 && !mbar_wait(&bar[B_EMPTY0 + s], ((m >> 1) - 1) & 1, abort_flag)) break;
             unsigned char *st = sm + s * STAGE;
             if (lane == 0) {
-                mbar_arrive_tx(&bar[B_FULL0 + s], OUT ? 65536u : 40960u);
+                mbar_arrive_tx(&bar[B_FULL0 + s], (OUT ? 65536u : 40960u) + (FUSED ? 8192u : 0u));
+                if (FUSED) tma_load_4d(st + FS_G, &mp.gate, j0, h, t0, b, &bar[B_FULL0 + s]);
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
                     tma_load_2d(st + FS_WQ + p * 16384, &mp.W, 64 * p, ci * C, &bar[B_FULL0 + s]);
@@ -177,6 +213,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
                 if (OUT) tma_load_2d(st + FS_UP + 8192, &mp.P, 0, ci * C, &bar[B_FULL0 + s]);
             }
             if (KDA) chunk_factors_kda(a.egc, (size_t)ci, cf_all + s * 132, lane);
+            else if (FUSED) chunk_factors_fused(a.gb, a.rn, (size_t)ci, cf_all + s * 132, lane);
             else chunk_factors(a.gb, (size_t)ci, cf_all + s * 132, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[B_FULL0 + s]);
@@ -218,25 +255,64 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
         named_sync(2, 256);
         // o of the previous chunk is finished by lanes 64-127 while the next chunk starts: they
         // stage it in OFF_O and one of them issues its TMA store (rows past T are clipped)
-        int prev_L = 0, prev_t0 = 0;
+        int prev_L = 0, prev_t0 = 0, prev_m = 0;
         float prev_eg = 0.f;
         uint32_t prev_buf = 0;
+        uint32_t gpk[16];  // fused forward, lanes 64-127: the chunk's output gate logits (bf16 pairs)
         auto o_epilogue = [&]() {
-            if (!OUT || trow < 64 || prev_L == 0 || !a.has_out) return;
+            if (!OUT || trow < 64 || prev_L == 0 || (!FUSED && !a.has_out)) return;
             const int r = trow - 64;
             float d[32], p[32];
             tmem_row32(tl + TM_D + prev_buf, d);
             tmem_row32(tl + TM_D + prev_buf + 64, p);
 #pragma unroll
             for (int j = 0; j < 32; ++j) d[j] = prev_eg * d[j] + p[j];
-            if (ostore) bulk_wait_read_all();  // the previous o store has read OFF_O
-            named_sync(3, 128);
+            float y[32];
+            if (FUSED) {
+                // y = o / sqrt(mean(o^2) + eps) w sigmoid(gate): the mean runs over all dv columns,
+                // half of them in the partner CTA; this CTA's row sums go to the partner's slot of
+                // this chunk's parity, and the partner's arrive in ours
+                float *ssp = reinterpret_cast<float *>(sm + OFF_MISC + M_SKP);
+                float *xs = reinterpret_cast<float *>(sm + OFF_MISC + M_XS);
+                const float *wn = reinterpret_cast<const float *>(sm + OFF_MISC + M_WN);
+                float ss = 0.f;
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + OFF_O, swz(r, hf * 4 + c4), d + c4 * 8);
+                for (int j = 0; j < 32; ++j) ss += d[j] * d[j];
+                ssp[hf * 64 + r] = ss;
+                named_sync(3, 128);
+                const float local = ssp[r] + ssp[64 + r];
+                const int slot = prev_m & 1;
+                if (hf == 0) {
+                    const uint32_t partner = (uint32_t)half ^ 1u;
+                    st_cluster_f32(map_to_rank(xs + slot * 64 + r, partner), local);
+                    mbar_arrive_cluster(map_to_rank(&bar[B_XS0 + slot], partner));
+                }
+                const bool gx = mbar_wait_cluster(&bar[B_XS0 + slot], (uint32_t)(prev_m >> 1) & 1, abort_flag);
+                // lanes 64-127 agree; an abort is then agreed on by the chain's next barrier
+                if (named_sync_any(3, 128, !gx || *abort_flag != 0)) return;
+                const float inv = rsqrtf((local + xs[slot * 64 + r]) * (1.f / DV) + POST_EPS);
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    const uint32_t gw = gpk[j >> 1];
+                    y[j] = d[j] * inv * wn[cb + j] * sigmoid_f(bf16_lo(gw));
+                    y[j + 1] = d[j + 1] * inv * wn[cb + j + 1] * sigmoid_f(bf16_hi(gw));
+                }
+            }
+            if (ostore) bulk_wait_read_all();  // the previous chunk's stores have read OFF_O / OFF_Y
+            named_sync(3, 128);
+            if (a.has_out) {
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + OFF_O, swz(r, hf * 4 + c4), d + c4 * 8);
+            }
+            if (FUSED) {
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + OFF_Y, swz(r, hf * 4 + c4), y + c4 * 8);
+            }
             fence_proxy_async();
             named_sync(3, 128);
             if (ostore) {
-                tma_store_4d(&mp.out, sm + OFF_O, j0, h, prev_t0, b);
+                if (a.has_out) tma_store_4d(&mp.out, sm + OFF_O, j0, h, prev_t0, b);
+                if (FUSED) tma_store_4d(&mp.y, sm + OFF_Y, j0, h, prev_t0, b);
                 bulk_commit();
             }
         };
@@ -288,6 +364,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
                     for (int e = 0; e < 8; ++e) ut[e] *= rowf;
                     st_chunk(sm + OFF_UD, o, ut);
                 }
+            } else if (FUSED) {  // lanes 64-127, idle here: this chunk's gate logits, kept for its o
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const uint4 g4 = *reinterpret_cast<const uint4 *>(st + FS_G + swz(trow - 64, hf * 4 + c4));
+                    gpk[c4 * 4] = g4.x; gpk[c4 * 4 + 1] = g4.y; gpk[c4 * 4 + 2] = g4.z; gpk[c4 * 4 + 3] = g4.w;
+                }
             }
             fence_proxy_async();
             fence_before_sync();
@@ -328,7 +410,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             fence_proxy_async();
             fence_before_sync();
             if (wabort(true)) break;
-            prev_L = L; prev_t0 = t0; prev_eg = rowf; prev_buf = buf;
+            prev_L = L; prev_t0 = t0; prev_eg = rowf; prev_buf = buf; prev_m = m;
         }
         if (*abort_flag == 0) o_epilogue();  // last chunk
         if (wc == 0 || ostore) bulk_wait_all();
@@ -347,6 +429,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
+    if (FUSED) cluster_sync();  // no CTA leaves while its partner may still reach its shared memory
     if (warp == 0) tmem_dealloc(tbase, 512);
 }
 
@@ -612,15 +695,16 @@ static size_t ws_carve(const Geo &g, int parts, char *base, TcWs *w) {
         __nv_bfloat16 **tiles[] = {&w->Kt1, &w->Qt1, &w->Kt};
         for (__nv_bfloat16 **t : tiles) *t = (__nv_bfloat16 *)take(nc * C * DK * 2);
         w->Kh = (__nv_bfloat16 *)take(nc * KDA_KH_ROWS * DK * 2);
-        w->kwide = (int *)take(nc * 4);
         w->Dx = (float *)take(nc * 2 * C * 16 * 4);
     }
     if (parts & WS_KDAC) {
         w->Qt = (__nv_bfloat16 *)take(nc * C * DK * 2);
         w->Kb = (__nv_bfloat16 *)take(nc * C * DK * 2);
         w->egc = (float *)take(nc * DK * 4);
+        w->kwide = (int *)take(nc * 4);
     }
     if (parts & WS_KDAG) w->G = (float *)take(nc * C * DK * 4);
+    if (parts & WS_RN) w->rn = (float *)take(nc * 2 * C * 4);
     return off;
 }
 
@@ -635,13 +719,16 @@ cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, int mode
     using namespace tch;
     FMaps mp;
     const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;
-    const bool out = mode != 1, keep = mode != 0, kda = g.variant == VAR_KDA;
+    const bool out = mode != 1, keep = mode == 1 || mode == 2, kda = g.variant == VAR_KDA, fused = mode == 3;
+    if (fused && (kda || !t.y || !t.gate_o || !t.w_norm || !w.rn)) return cudaErrorInvalidValue;
     bool ok = (kda ? tc::make_map_2d_bf16(&mp.q, w.Qt, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.k, w.Kb, DK, NC * C, 64)
                    : tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) &&
                          tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64)) &&
               tc::make_map_2d_bf16(&mp.W, w.W, DK, NC * C, 64) && tc::make_map_2d_bf16(&mp.Ut, w.Ut, DV, NC * C, 64) &&
               tc::make_map_2d_bf16(&mp.P, w.P, C, NC * C, 64);
-    mp.out = mp.u = mp.Sn = mp.Un = mp.q;  // unused ones keep a valid map
+    mp.out = mp.u = mp.Sn = mp.Un = mp.gate = mp.y = mp.q;  // unused ones keep a valid map
+    if (ok && fused)
+        ok = tc::make_map_4d_bf16(&mp.gate, t.gate_o, DV, H, T, Bn, 64) && tc::make_map_4d_bf16(&mp.y, t.y, DV, H, T, Bn, 64);
     if (ok && keep)
         ok = tc::make_map_2d_bf16(&mp.Sn, w.Sn, DV, NC * DK, 128) && tc::make_map_2d_bf16(&mp.Un, w.Un, DV, NC * C, 64);
     if (ok && out && t.out) ok = tc::make_map_4d_bf16(&mp.out, t.out, DV, H, T, Bn, 64);
@@ -649,7 +736,7 @@ cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, int mode
     if (!ok) return cudaErrorInvalidValue;
     Args a = {};
     a.gb = w.gb; a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
-    a.S0 = t.S0; a.egc = w.egc;
+    a.S0 = t.S0; a.egc = w.egc; a.rn = w.rn; a.wn = t.w_norm;
     if (out) {
         a.has_out = t.out != nullptr; a.has_u = t.u != nullptr; a.ST = t.S_T;
     }
@@ -660,13 +747,30 @@ cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, int mode
         cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e2 != cudaSuccess) return e2;
         rec.mark(s);
-        kern<<<grid, NTHREADS, smem, s>>>(mp, a);
-        return cudaSuccess;
+        if (!fused) {
+            kern<<<grid, NTHREADS, smem, s>>>(mp, a);
+            return cudaSuccess;
+        }
+        // the two value halves of a (b, h) form a cluster (they exchange the output's row sums)
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(NTHREADS);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, kern, mp, a);
     };
     if (kda) e = mode == 0 ? go(k_chain_fwd<0, 1>) : mode == 1 ? go(k_chain_fwd<1, 1>) : go(k_chain_fwd<2, 1>);
     else if (mode == 0) e = go(k_chain_fwd<0, 0>);
     else if (mode == 1) e = go(k_chain_fwd<1, 0>);
-    else e = go(k_chain_fwd<2, 0>);
+    else if (mode == 2) e = go(k_chain_fwd<2, 0>);
+    else e = go(k_chain_fwd<3, 0>);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -28,8 +28,8 @@ bool tc_split_kda_supported(const Geo &g, bool bf16);
 //   WS_KEEP   the chunk products only the scalar-gate gradient kernel reads (Tn, KK);
 //   WS_STATE  the chunk states and write values of the forward chain (Sn, Un);
 //   WS_REV    what the reverse chain hands the gradient kernels (dSn, dUn, skt);
-//   WS_KDA    KDA's forward-only gate-scaled operands (Kt1, Qt1, Kh, Kt, kwide, Dx);
-//   WS_KDAC   KDA's operands of both chains (Qt, Kb, egc);
+//   WS_KDA    KDA's forward-only gate-scaled operands (Kt1, Qt1, Kh, Kt, Dx);
+//   WS_KDAC   KDA's operands of both chains (Qt, Kb, egc) and the chunk flags kwide;
 //   WS_KDAG   KDA's in-chunk cumulative log gate G (fp32, read by its gradient kernel).
 // Gated DeltaNet / DeltaNet: the forward's workspace is WS_FWD; the recomputing backward's
 // FWD | KEEP | STATE | REV; the saved activations of delta_rule_fwd_save are FWD | KEEP | STATE,
@@ -68,14 +68,15 @@ struct TcWs {
                          //               sum_c k_rc k_ic e^{g_rc - g_ic} ([0]) and
                          //               sum_c q_rc k_ic e^{g_rc - g_ic} ([1]), i = b(r) + 0..15
     float *G;            // [ci][C][dk]   KDA: g itself (fp32)
+    float *rn;           // [ci][2][C]    fused forward: 1 / |k_r|, 1 / |q_r| of the raw rows
 };
 // rows of the stacked KDA column operand (16 + 32 + 48 + 64), and the widest in-block fall of
 // a channel's cumulative log gate (nats) for which the block-reference split is used as is
 constexpr int KDA_KH_ROWS = 160;
 constexpr float KDA_DIAG_SPAN = 64.f;
-enum { WS_FWD = 1, WS_KEEP = 2, WS_REV = 4, WS_KDA = 8, WS_STATE = 16, WS_KDAC = 32, WS_KDAG = 64 };
+enum { WS_FWD = 1, WS_KEEP = 2, WS_REV = 4, WS_KDA = 8, WS_STATE = 16, WS_KDAC = 32, WS_KDAG = 64, WS_RN = 128 };
 // Bytes of the given parts, laid out one after another in the order FWD, KEEP, STATE, REV, KDA,
-// KDAC, KDAG.
+// KDAC, KDAG, RN (the row norms of the fused forward).
 size_t tc_ws_bytes(const Geo &g, int parts);
 // Sets the pointers of the given parts, carved from base in that order; leaves the others.
 void tc_ws_carve(const Geo &g, int parts, void *base, TcWs *w);
@@ -85,26 +86,37 @@ void tc_ws_carve(const Geo &g, int parts, void *base, TcWs *w);
 // the chunks marked in w.kwide, the exact in-block sums w.Dx (a second kernel; the others exit).
 cudaError_t tc_kda_gates(const Geo &g, const Tensors &t, const TcWs &w, float *G, cudaStream_t s, Rec &rec);
 // fp32 copies of the forward's chunk products and states (W, U~, P, S_n, U) for the CUDA-core
-// backward kernels (tc_prep.cu).
+// backward kernels (tc_prep.cu); with only (per-chunk flags), of the flagged chunks alone.
 cudaError_t tc_to_simt(const Geo &g, const TcWs &w, float *W, float *Ut, float *P, float *Sn, float *Un, cudaStream_t s,
-                       Rec &rec);
-// fp32 copies of the reverse chain's dS_{n+1} and dL/dU (tc_prep.cu).
-cudaError_t tc_rev_to_simt(const Geo &g, const TcWs &w, float *dSn, float *dUn, cudaStream_t s, Rec &rec);
+                       Rec &rec, const int *only = nullptr);
+// fp32 copies of the reverse chain's dS_{n+1} and dL/dU (tc_prep.cu), likewise.
+cudaError_t tc_rev_to_simt(const Geo &g, const TcWs &w, float *dSn, float *dUn, cudaStream_t s, Rec &rec,
+                           const int *only = nullptr);
 // The KDA backward's products with the chunk states on tcgen05, from the bf16 workspace tiles
 // (S_n, dS_{n+1}, U, dU) and dO: Qd = dO S^T, dWm = -dU S^T, Tm = U dS+^T, RS = rowsum(S .* dS+),
 // written to the CUDA-core workspace ([ci][C][dk] fp32 each; RS [ci][dk]).
 cudaError_t tc_state_to_simt(const Geo &g, const Tensors &t, const TcWs &w, float *Qd, float *dWm, float *Tm,
-                             float *RS, cudaStream_t s, Rec &rec);
+                             float *RS, cudaStream_t s, Rec &rec, const int *only = nullptr);
 // Per-chunk products (tc_prep.cu): g and beta, W, U~, P; with keep also T and k k^T.
-// For KDA (no keep) from the operands of tc_kda_gates.
-cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool keep, cudaStream_t s, Rec &rec);
+// For KDA (no keep) from the operands of tc_kda_gates.  raw (Gated DeltaNet / DeltaNet, no
+// keep): t.q, t.k are the raw projections and t.alpha, t.beta the raw logits; the prep applies
+// the pre-operation (L2 normalisation, log alpha = -softplus, beta = sigmoid) on the fly and
+// writes the row norms to w.rn.
+cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool keep, cudaStream_t s, Rec &rec,
+                          bool raw = false);
 // Forward state chain (tc_chain.cu).  mode 0: o, u, S_T; mode 1 (recompute for the
-// backward): S_n and U of every chunk; mode 2: both.
+// backward): S_n and U of every chunk; mode 2: both; mode 3 (Gated DeltaNet / DeltaNet): the
+// fused forward of delta_rule_fwd_fused -- raw q, k with the row norms of w.rn, and the
+// post-operation y = RMSNorm(o) w * sigmoid(gate) in the output epilogue (the two CTAs of a
+// (b, h) form a cluster and exchange their halves' row sums of squares); o optional.
 cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, int mode, cudaStream_t s, Rec &rec);
 // Reverse state chain (tc_chain.cu): dS_{n+1} and dL/dU of every chunk (w.dSn, w.dUn), the
 // row sums w.skt, and dS0.  KDA reads the forward's gate-scaled q and k from w.
 cudaError_t tc_chain_rev(const Geo &g, const Tensors &t, const TcWs &w, cudaStream_t s, Rec &rec);
 // All intra-chunk gradients (tc_bwd.cu): dq, dk, dv, dbeta, d log alpha.
 cudaError_t tc_bwd_chunk(const Geo &g, const Tensors &t, const TcWs &w, cudaStream_t s, Rec &rec);
+// KDA's intra-chunk gradients on tcgen05 (tc_bwd_kda.cu) for the chunks with w.kwide == 0, from the
+// forward's W, U~, T, M (w.KK), states and write values and the reverse chain's dS_{n+1}, dU.
+cudaError_t tc_bwd_kda(const Geo &g, const Tensors &t, const TcWs &w, cudaStream_t s, Rec &rec);
 
 }  // namespace dr

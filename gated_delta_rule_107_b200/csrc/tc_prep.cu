@@ -59,7 +59,7 @@ static_assert(OFF_P == OFF_F + 32768 && OFF_KH + 2 * KH_PANEL <= OFF_MISC, "the 
 constexpr uint32_t M_BAR = 0;          // [0] loads, [1] MMA
 constexpr uint32_t M_TMEM = 64, M_ABORT = 68, M_BIG = 72;
 constexpr uint32_t M_PF = 256;         // gate factors [6][64]
-enum { PF_GC = 0, PF_ROWP, PF_COLA, PF_BV, PF_BK, PF_NUM };
+enum { PF_GC = 0, PF_ROWP, PF_COLA, PF_BV, PF_BK, PF_RNK, PF_RNQ, PF_NUM };
 static_assert(M_PF + PF_NUM * 256 <= 2048, "misc overflow");
 // TMEM columns
 constexpr uint32_t TM_G1 = 0, TM_XW = 0, TM_XU = 128, TM_COLS = 256;
@@ -74,8 +74,9 @@ struct Maps {
 };
 
 struct Args {
-    const void *alpha, *beta;       // bf16 [B, T, H]
+    const void *alpha, *beta;       // bf16 [B, T, H] (RAW: the raw forget and write-strength logits)
     float *gb;                      // [chunks][2][64]: g, beta
+    float *rn;                      // RAW: [chunks][2][64] 1 / |k_r|, 1 / |q_r|
     const int *kwide;               // KDA: [chunks] in-block sums from Dx
     const float *Dx;                // KDA: [chunks][2][64][16]
     int B, T, H, N;
@@ -84,9 +85,18 @@ struct Args {
 // first column of block R's section of the KDA product (16 R (R + 1) / 2)
 __host__ __device__ constexpr uint32_t kda_sec(int R) { return (uint32_t)(8 * R * (R + 1)); }
 
-// KEEP: also store T and k k^T (for the backward)
-template <int VAR, int KEEP>
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + __expf(-x)); }
+// softplus(x) = max(x, 0) + log(1 + e^{-|x|}), finite for every x
+__device__ __forceinline__ float softplus_f(float x) { return fmaxf(x, 0.f) + log1pf(__expf(-fabsf(x))); }
+constexpr float PRE_EPS = 1e-6f;  // q_hat = q / sqrt(|q|^2 + eps), as the standalone pre-operation
+
+// KEEP: also store T and k k^T (for the backward).  RAW: the fused pre-operation (KDA page
+// section 7.1): q, k arrive as raw projections and are normalised through per-row factors
+// (1/|k_i| joins the column factors of A and P and the row factor of W's operand), the gate
+// and beta as raw logits (log alpha = -softplus(a), beta = sigmoid(b)).
+template <int VAR, int KEEP, int RAW>
 __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constant__ Maps mp, Args a) {
+    static_assert(!RAW || (VAR != VAR_KDA && !KEEP), "the fused pre-operation serves the scalar-gate forward");
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm =
         reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -135,8 +145,8 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
             lg[hh] = 0.f;
             bt[hh] = 0.f;
             if (r < L) {
-                if (VAR == VAR_GATED) lg[hh] = tcf::bf(a.alpha, row);
-                bt[hh] = tcf::bf(a.beta, row);
+                if (VAR == VAR_GATED) lg[hh] = RAW ? -softplus_f(tcf::bf(a.alpha, row)) : tcf::bf(a.alpha, row);
+                bt[hh] = RAW ? sigmoid_f(tcf::bf(a.beta, row)) : tcf::bf(a.beta, row);
             }
         }
         float x0 = lg[0], x1 = lg[1];
@@ -201,6 +211,23 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
         mma_commit(&bar[1]);
         mma_issued++;
     }
+    if (RAW && ok) {  // while P1 runs: 1 / sqrt(|x|^2 + eps) of k row tid (tid < 64) or q row tid - 64
+        const int r = trow & 63;
+        const uint32_t base = OFF_KQ + (trow < 64 ? 0u : 8192u);
+        float ss = 0.f;
+#pragma unroll
+        for (int p = 0; p < 2; ++p)
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                float x[8];
+                ld_chunk(sm + base + p * 16384, swz(r, ch), x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
+            }
+        const float rn = rsqrtf(ss + PRE_EPS);
+        pf[(trow < 64 ? PF_RNK : PF_RNQ) * 64 + r] = rn;
+        a.rn[(size_t)ci * 2 * C + (trow < 64 ? 0 : C) + r] = rn;
+    }
     if (ok) ok = consensus(wait_mma());
     // ---------------- A (fp32, for the inverse), P (bf16 tile), k k^T ----------------
     if (ok) {
@@ -258,6 +285,12 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
 #pragma unroll
             for (int i = 0; i < 64; ++i) f[i] = (i <= r) ? __expf(gr - gc[i]) : 0.f;
         }
+        if (RAW) {  // the raw rows' norms: row factor 1/|k_r| or 1/|q_r|, column factor 1/|k_i|
+            const float rr = pf[(arow ? PF_RNK : PF_RNQ) * 64 + r];
+            const float *rk = pf + PF_RNK * 64;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) f[i] *= rr * rk[i];
+        }
         if (arow) {
             // k k^T row (KEEP) into the q_p0 tile, free since P1 completed
             if (KEEP) {
@@ -312,6 +345,10 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
             if (KEEP && tid < 64) st_chunk(sm + OFF_P, swz(i, ch), w);
 #pragma unroll
             for (int e = 0; e < 8; ++e) w[e] *= fac[ch * 8 + e];
+            if (RAW && tid >= 64) {  // W's operand k is the normalised one: 1/|k_j| per column
+#pragma unroll
+                for (int e = 0; e < 8; ++e) w[e] *= pf[PF_RNK * 64 + ch * 8 + e];
+            }
             st_chunk(dst, swz(i, ch), w);
         }
     }
@@ -550,14 +587,14 @@ __global__ void __launch_bounds__(128) k_kda_diag(KdaArgs a) {
     }
 }
 
-template <int VAR, int KEEP>
+template <int VAR, int KEEP, int RAW = 0>
 static cudaError_t launch_prep(const Maps &mp, const Args &a, dim3 grid, cudaStream_t s, Rec &rec) {
     const size_t smem = (VAR == VAR_KDA ? SMEM_KDA : SMEM_BYTES) + 1024;
     cudaError_t e =
-        cudaFuncSetAttribute(k_chunk_prep<VAR, KEEP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(k_chunk_prep<VAR, KEEP, RAW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     rec.mark(s);
-    k_chunk_prep<VAR, KEEP><<<grid, NTHREADS, smem, s>>>(mp, a);
+    k_chunk_prep<VAR, KEEP, RAW><<<grid, NTHREADS, smem, s>>>(mp, a);
     return cudaGetLastError();
 }
 
@@ -586,12 +623,15 @@ namespace tcp {
 struct Widen {
     const __nv_bfloat16 *src[5];
     float *dst[5];
-    size_t n8[5];  // elements / 8
+    size_t n8[5];     // elements / 8
+    size_t per8[5];   // elements / 8 of one chunk
+    const int *only;  // optional: widen the chunks flagged here alone
 };
 __global__ void __launch_bounds__(256) k_widen(Widen a) {
     for (int i = 0; i < 5; ++i) {
         if (!a.src[i]) continue;
         for (size_t x = (size_t)blockIdx.x * 256 + threadIdx.x; x < a.n8[i]; x += (size_t)gridDim.x * 256) {
+            if (a.only && !a.only[x / a.per8[i]]) continue;
             const uint4 v = reinterpret_cast<const uint4 *>(a.src[i])[x];
             const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
             float f[8];
@@ -609,35 +649,40 @@ __global__ void __launch_bounds__(256) k_widen(Widen a) {
 }  // namespace tcp
 
 cudaError_t tc_to_simt(const Geo &g, const TcWs &w, float *W, float *Ut, float *P, float *Sn, float *Un, cudaStream_t s,
-                       Rec &rec) {
+                       Rec &rec, const int *only) {
     using namespace tcp;
     const size_t nc = (size_t)g.B * g.H * g.N;
     Widen a = {};
     const __nv_bfloat16 *src[5] = {w.W, w.Ut, w.P, w.Sn, w.Un};
     float *dst[5] = {W, Ut, P, Sn, Un};
-    const size_t n[5] = {nc * C * DK, nc * C * DV, nc * C * C, nc * DK * DV, nc * C * DV};
+    const size_t per[5] = {(size_t)C * DK, (size_t)C * DV, (size_t)C * C, (size_t)DK * DV, (size_t)C * DV};
     for (int i = 0; i < 5; ++i) {  // an absent destination is not widened
         a.src[i] = dst[i] ? src[i] : nullptr;
         a.dst[i] = dst[i];
-        a.n8[i] = n[i] / 8;
+        a.n8[i] = nc * per[i] / 8;
+        a.per8[i] = per[i] / 8;
     }
+    a.only = only;
     rec.mark(s);
     k_widen<<<148 * 8, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 
-cudaError_t tc_rev_to_simt(const Geo &g, const TcWs &w, float *dSn, float *dUn, cudaStream_t s, Rec &rec) {
+cudaError_t tc_rev_to_simt(const Geo &g, const TcWs &w, float *dSn, float *dUn, cudaStream_t s, Rec &rec,
+                           const int *only) {
     using namespace tcp;
     const size_t nc = (size_t)g.B * g.H * g.N;
     Widen a = {};
-    a.src[0] = dSn ? w.dSn : nullptr; a.dst[0] = dSn; a.n8[0] = nc * DK * DV / 8;
-    a.src[1] = dUn ? w.dUn : nullptr; a.dst[1] = dUn; a.n8[1] = nc * C * DV / 8;
+    a.src[0] = dSn ? w.dSn : nullptr; a.dst[0] = dSn; a.n8[0] = nc * DK * DV / 8; a.per8[0] = DK * DV / 8;
+    a.src[1] = dUn ? w.dUn : nullptr; a.dst[1] = dUn; a.n8[1] = nc * C * DV / 8; a.per8[1] = C * DV / 8;
+    a.only = only;
     rec.mark(s);
     k_widen<<<148 * 8, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 
-cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool keep, cudaStream_t s, Rec &rec) {
+cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool keep, cudaStream_t s, Rec &rec,
+                          bool raw) {
     using namespace tcp;
     Maps mp;
     const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;
@@ -652,10 +697,18 @@ cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool ke
              tc::make_map_2d_bf16(&mp.Kt, w.Kt, DK, NC * C, 64);
     if (!ok) return cudaErrorInvalidValue;
     Args a;
-    a.alpha = t.alpha; a.beta = t.beta; a.gb = w.gb; a.kwide = w.kwide; a.Dx = w.Dx;
+    a.alpha = t.alpha; a.beta = t.beta; a.gb = w.gb; a.kwide = w.kwide; a.Dx = w.Dx; a.rn = w.rn;
     a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
     const dim3 grid(g.N, g.H, g.B);
-    if (g.variant == VAR_KDA) return launch_prep<VAR_KDA, 0>(mp, a, grid, s, rec);  // no saved form
+    if (g.variant == VAR_KDA) {  // KEEP: T and the gated k k^T products M (for the KDA gradient kernel)
+        if (raw) return cudaErrorInvalidValue;
+        return keep ? launch_prep<VAR_KDA, 1>(mp, a, grid, s, rec) : launch_prep<VAR_KDA, 0>(mp, a, grid, s, rec);
+    }
+    if (raw) {
+        if (keep || !w.rn) return cudaErrorInvalidValue;
+        return g.variant == VAR_GATED ? launch_prep<VAR_GATED, 0, 1>(mp, a, grid, s, rec)
+                                      : launch_prep<VAR_DELTANET, 0, 1>(mp, a, grid, s, rec);
+    }
     if (g.variant == VAR_GATED)
         return keep ? launch_prep<VAR_GATED, 1>(mp, a, grid, s, rec) : launch_prep<VAR_GATED, 0>(mp, a, grid, s, rec);
     return keep ? launch_prep<VAR_DELTANET, 1>(mp, a, grid, s, rec) : launch_prep<VAR_DELTANET, 0>(mp, a, grid, s, rec);

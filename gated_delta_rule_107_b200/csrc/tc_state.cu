@@ -43,6 +43,7 @@ struct Maps {
 
 struct Args {
     float *Qd, *dWm, *Tm, *RS;  // [ci][C][dk] x3, [ci][dk] (fp32)
+    const int *only;            // optional: the chunks flagged here alone
     int has_dout, T, H, N;
 };
 
@@ -55,6 +56,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_state_tc(const __grid_constant_
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + R_MISC + 20);
     const int tid = threadIdx.x, warp = tid >> 5;
     const int ci = blockIdx.x, n = ci % a.N, bh = ci / a.N, h = bh % a.H, b = bh / a.H, t0 = n * C;
+    if (a.only && !a.only[ci]) return;  // uniform over the CTA
     const uint32_t load_bytes = 2 * 32768 + (a.has_dout ? 16384 : 0) + 16384 + 16384;
     if (!a.has_dout)  // no output gradient: the dO rows of the stacked operand are zero
         for (int x = tid; x < 2 * 8192 / 16; x += NTHREADS)
@@ -142,7 +144,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_state_tc(const __grid_constant_
 }  // namespace tcs
 
 cudaError_t tc_state_to_simt(const Geo &g, const Tensors &t, const TcWs &w, float *Qd, float *dWm, float *Tm,
-                             float *RS, cudaStream_t s, Rec &rec) {
+                             float *RS, cudaStream_t s, Rec &rec, const int *only) {
     using namespace tcs;
     Maps mp;
     const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;
@@ -151,7 +153,7 @@ cudaError_t tc_state_to_simt(const Geo &g, const Tensors &t, const TcWs &w, floa
     if (ok && t.dout) ok = tc::make_map_4d_bf16(&mp.dout, t.dout, DV, H, T, Bn, 64);
     if (!ok) return cudaErrorInvalidValue;
     Args a;
-    a.Qd = Qd; a.dWm = dWm; a.Tm = Tm; a.RS = RS;
+    a.Qd = Qd; a.dWm = dWm; a.Tm = Tm; a.RS = RS; a.only = only;
     a.has_dout = t.dout != nullptr; a.T = g.T; a.H = g.H; a.N = g.N;
     const size_t smem = SMEM_BYTES + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_state_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -41,6 +41,13 @@ __device__ __forceinline__ void st8_global(void *base, size_t elem_off, const fl
     *reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(base) + elem_off) = w;
 }
 
+// 8 bf16 values at p (16-byte aligned) in global memory, widened
+__device__ __forceinline__ void ld8_global(const __nv_bfloat16 *p, float *v) {
+    const uint4 w = *reinterpret_cast<const uint4 *>(p);
+    v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+    v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
+}
+
 // 64 values as bf16 at element offset elem_off (a multiple of 8) of a bf16 array in global memory
 __device__ __forceinline__ void st_row_global(void *base, size_t elem_off, const float *v) {
 #pragma unroll

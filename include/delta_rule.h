@@ -224,6 +224,31 @@ int delta_rule_fwd_noalloc(const void *q, const void *k, const void *v, const vo
                            int variant, int chunk, int dtype, void *stream);
 
 /*
+ * Fused forward: the pre-operation, the forward and the post-operation below in
+ * the core's own kernels, with no pass over memory of their own (Kimi Delta
+ * Attention page: section 7.1 -- q, k L2-normalised, logistic gates in log
+ * space; section 4.1 -- sigmoid output gate on RMSNorm of the core's output).
+ * From the raw projections q_raw, k_raw [B,T,H,dk], the raw forget logits
+ * gate_raw [B,T,H] (Gated DeltaNet; unused and may be NULL for DeltaNet) and
+ * the raw write-strength logits beta_raw [B,T,H] it computes, exactly as
+ * delta_rule_preop then delta_rule_fwd then delta_rule_postop would (up to
+ * rounding order: the normalised q, k and the gates stay in fp32 on chip),
+ *     y = RMSNorm(o) * w_norm * sigmoid(gate_out)   [B,T,H,dv]
+ * and, when their pointers are not NULL, o itself (before the normalisation),
+ * u and S_T.  gate_out [B,T,H,dv] has the I/O dtype, w_norm is fp32 [dv].
+ * Served for Gated DeltaNet and DeltaNet with bf16 I/O, dk = dv = 128 and
+ * chunk 64 (DR_ERR_UNSUPPORTED otherwise; the separate calls serve every
+ * configuration).  The workspace is delta_rule_fwd_fused_workspace_size()
+ * bytes ((size_t)-1 for arguments it does not serve), 256-byte aligned.
+ * Errors, alignment and the asynchronous contract as delta_rule_fwd.
+ */
+size_t delta_rule_fwd_fused_workspace_size(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype);
+int delta_rule_fwd_fused(const void *q_raw, const void *k_raw, const void *v, const void *gate_raw,
+                         const void *beta_raw, const float *S0, const void *gate_out, const float *w_norm, void *y,
+                         void *o, void *u, float *S_T, int B, int T, int H, int dk, int dv, int variant, int chunk,
+                         int dtype, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Recurrent form for decoding.  Steps the recurrence above token by token from
  * the state S_in (NULL = zero) through the T tokens given and writes out and u
  * exactly as delta_rule_fwd does (u may be NULL), and the state after the last
@@ -317,12 +342,13 @@ int delta_rule_shortconv_bwd(const void *x, const float *w, const void *x_prev, 
  *     h_out = h + u W          (h NULL: h_out = u W; h_out may alias h)
  * delta_rule_clvr_bwd: for dh_out [M,N], du = dh_out W^T [M,K] (NULL = not
  * written) and dW = u^T dh_out [K,N], fp32 (NULL = not written); the gradient of
- * h is dh_out itself.  u, W, h, h_out, dh_out and du have the I/O dtype.  These
- * are plain dense products and run as cuBLASLt GEMMs (bf16 operands with fp32
- * accumulation, or fp32 throughout for fp32 I/O) with a caller workspace of
- * delta_rule_clvr_workspace_size() bytes (256-byte aligned).  The first call
- * creates the process's one cuBLASLt handle.  K and N must be multiples of 8;
- * every pointer 16-byte aligned.
+ * h is dh_out itself.  u, W, h, h_out, dh_out and du have the I/O dtype.  bf16
+ * runs the library's tcgen05 GEMM (bf16 operands read in place, transposed or
+ * not, fp32 accumulation in tensor memory, the residual added in the epilogue;
+ * dW's reduction over the M tokens is split into slices whose fp32 partials are
+ * added in a fixed order), fp32 I/O a CUDA-core GEMM in fp32.  The caller passes
+ * a workspace of delta_rule_clvr_workspace_size() bytes (256-byte aligned) for
+ * those partials.  K and N must be multiples of 8; every pointer 16-byte aligned.
  */
 size_t delta_rule_clvr_workspace_size(void);
 int delta_rule_clvr(const void *u, const void *W, const void *h, void *h_out, int M, int K, int N, int dtype,

@@ -65,9 +65,11 @@ def test_no_compute_validation_paths(lib):
     assert 0 < binding.workspace_size(8, 4096, 8, 128, 128, 1, 64, 1, 3) < binding.workspace_size(
         8, 4096, 8, 128, 128, 1, 64, 1, 1)
     # KDA: the saved buffer holds per chunk g|beta (512 B), W, U~, U, q e^g, k e^{g_C - g} (16 KiB
-    # each), P (8 KiB), e^{g_C} (512 B), the state entering the chunk and the fp32 gate (32 KiB each)
+    # each), P, T and the gated k k^T (8 KiB each), e^{g_C} (512 B), the chunk flag (4 B), the state
+    # entering the chunk and the fp32 gate (32 KiB each)
     n_chunks = 8 * 16 * 64
-    assert binding.saved_size(8, 4096, 16, 128, 128, 2, 64, 1) == n_chunks * (512 + 5 * 16384 + 8192 + 512 + 2 * 32768)
+    assert binding.saved_size(8, 4096, 16, 128, 128, 2, 64, 1) == n_chunks * (
+        512 + 5 * 16384 + 3 * 8192 + 512 + 4 + 2 * 32768)
     assert 0 < binding.workspace_size(8, 4096, 16, 128, 128, 2, 64, 1, 3) < binding.workspace_size(
         8, 4096, 16, 128, 128, 2, 64, 1, 1)
     assert binding.saved_size(1, 256, 2, 64, 64, 0, 64, 0) == 0       # fp32 I/O: no saved form
@@ -127,9 +129,11 @@ def test_launch_plans(lib):
             assert binding.launches(8, 4096, 8, 128, 128, variant, 64, 1, kind) == names
     kda_split = ["k_kda_gates", "k_kda_diag", "k_chunk_prep", "k_chain_fwd"]
     assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 0) == kda_split
-    assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 2) == kda_split[:3] + ["k_chain_fwd(keep)"]
-    kda_bwd = ["k_kda_gates", "k_kda_diag", "k_chunk_prep", "k_chain_fwd(recompute)", "k_widen", "k_chain_rev",
-               "k_widen", "k_state_tc", "k_bwd_intra"]
+    assert binding.launches(4, 16384, 8, 128, 128, 2, 64, 1, 2) == kda_split[:2] + ["k_chunk_prep(keep)",
+                                                                                   "k_chain_fwd(keep)"]
+    # the tensor-core intra-chunk gradient, then the CUDA-core one for chunks past the block split's range
+    kda_bwd = ["k_kda_gates", "k_kda_diag", "k_chunk_prep(keep)", "k_chain_fwd(recompute)", "k_chain_rev",
+               "k_bwd_kda_tc", "k_widen", "k_widen", "k_state_tc", "k_bwd_intra"]
     assert binding.launches(8, 4096, 16, 128, 128, 2, 64, 1, 1) == kda_bwd
     assert binding.launches(8, 4096, 16, 128, 128, 2, 64, 1, 3) == kda_bwd[4:]  # from saved: no recompute
     # KDA at dv = 64 takes the CUDA-core forward; the fused dv = 64 kernel serves scalar gates

@@ -107,3 +107,17 @@ def test_clvr_rejects_bad_arguments():
         binding.DR_OK
     torch.cuda.synchronize()
     assert torch.equal(dW, torch.zeros_like(dW))  # no tokens: an empty sum
+
+
+def test_dw_split_reduction_is_deterministic():
+    """dW's reduction over the tokens runs in slices whose partials are added in a fixed order:
+    two calls return the same bits."""
+    g = torch.Generator().manual_seed(9)
+    u = (0.3 * torch.randn(4, 1000, 4, 128, generator=g)).to(torch.bfloat16).cuda()
+    W = (0.05 * torch.randn(512, 768, generator=g)).to(torch.bfloat16).cuda()
+    dh = torch.randn(4, 1000, 768, generator=g).to(torch.bfloat16).cuda()
+    _, dW1 = binding.delta_rule_clvr_bwd(u, W, dh)
+    _, dW2 = binding.delta_rule_clvr_bwd(u, W, dh)
+    torch.cuda.synchronize()
+    assert torch.equal(dW1, dW2)
+    _check(dW1, cl.clvr_bwd(np64(u), np64(W), np64(dh))["dW"], TOL["bf16"], "dW")
