@@ -50,19 +50,20 @@ constexpr uint32_t OFF_U = OFF_S + 16384;     //  8K  U [r][j]        (reverse: 
 constexpr uint32_t OFF_UD = OFF_U + 8192;     //  8K  e^{g_C - g} U [r][j]
 constexpr uint32_t OFF_O = OFF_UD + 8192;     //  8K  o [r][j] (staging of the TMA store)
 constexpr uint32_t OFF_Y = OFF_O + 8192;      //  8K  fused forward: y [r][j] (staging)
-constexpr uint32_t OFF_MISC = OFF_Y + 8192;   //  4K
+constexpr uint32_t OFF_O1 = OFF_Y + 8192;     //  8K  fused forward: o of odd chunks (even: OFF_O)
+constexpr uint32_t OFF_MISC = OFF_O1 + 8192;  //  4K
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 4096;
 // misc
 constexpr uint32_t M_BAR = 0;  // FULL0, FULL1, EMPTY0, EMPTY1, MMA
-constexpr uint32_t M_TMEM = 64, M_ABORT = 68;
+constexpr uint32_t M_TMEM = 128, M_ABORT = 132;
 constexpr uint32_t M_CF = 256;  // per stage: [0..63] e^{g_C - g}, [64..127] e^g, [128] e^{g_C}
 constexpr uint32_t M_SKP = M_CF + 2 * 132 * 4;  // reverse: [2 column halves][64] row-sum partials;
                                                 // fused forward: the same for o's squares
-constexpr uint32_t M_XS = M_SKP + 512;          // fused forward: [2 chunk parities][64] the partner's
+constexpr uint32_t M_XS = M_SKP + 512;          // fused forward: [4 slots (chunk mod 4)][64] the partner's
                                                 // row sums of squares (written by the partner CTA)
-constexpr uint32_t M_WN = M_XS + 512;           // fused forward: this CTA's 64 RMSNorm weights
-// B_XS0/1 (fused forward): the partner's row sums of a chunk parity have arrived
-enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_MMA, B_XS0, B_XS1, B_NUM };
+constexpr uint32_t M_WN = M_XS + 1024;          // fused forward: this CTA's 64 RMSNorm weights
+// B_XS0..3 (fused forward): the partner's row sums of a chunk (mod 4) have arrived
+enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_MMA, B_XS0, B_XS1, B_XS2, B_XS3, B_NUM };
 static_assert(B_NUM * 8 <= M_TMEM && M_WN + 256 <= 4096, "misc overflow");
 constexpr float POST_EPS = 1e-6f;  // y = o / sqrt(mean(o^2) + eps) w sigmoid(gate)
 
@@ -174,7 +175,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < B_NUM; ++i)
-            mbar_init(&bar[i], (i == B_FULL0 || i == B_FULL1) ? 2 : (i == B_XS0 || i == B_XS1) ? 64 : 1);
+            mbar_init(&bar[i], (i == B_FULL0 || i == B_FULL1) ? 2 : (i >= B_XS0 && i <= B_XS3) ? 64 : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -254,11 +255,45 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
         fence_proxy_async();
         named_sync(2, 256);
         // o of the previous chunk is finished by lanes 64-127 while the next chunk starts: they
-        // stage it in OFF_O and one of them issues its TMA store (rows past T are clipped)
+        // stage it in OFF_O and one of them issues its TMA store (rows past T are clipped).
+        // Fused forward: y = o / sqrt(mean(o^2) + eps) w sigmoid(gate), the mean over all dv columns,
+        // half of them in the partner CTA.  The row sums of squares of chunk p go to the partner's
+        // slot p mod 4 while o(p) waits as bf16 in the buffer of p's parity; y(p) is finished one
+        // chunk later, when the partner's sums have long arrived, so that no chunk waits for the
+        // partner.  (The partner writes slot p mod 4 again for chunk p + 4, which it reaches only
+        // after this CTA has sent its sums of chunk p + 2, i.e. after y(p) is done here.)
         int prev_L = 0, prev_t0 = 0, prev_m = 0;
-        float prev_eg = 0.f;
+        float prev_eg = 0.f, prev_local = 0.f;
         uint32_t prev_buf = 0;
-        uint32_t gpk[16];  // fused forward, lanes 64-127: the chunk's output gate logits (bf16 pairs)
+        uint32_t gpk0[16], gpk1[16];  // fused, lanes 64-127: output gate logits of even / odd chunks
+        auto gate_of = [&](int j, int par) -> float {
+            const uint32_t gw = par ? gpk1[j >> 1] : gpk0[j >> 1];
+            return (j & 1) ? bf16_hi(gw) : bf16_lo(gw);
+        };
+        // fused: y of chunk q from its bf16 o (buffer of q's parity) into the y staging tile
+        auto y_tile = [&](int q, float inv) {
+            const int r = trow - 64;
+            const float *wn = reinterpret_cast<const float *>(sm + OFF_MISC + M_WN);
+            const unsigned char *ob = sm + ((q & 1) ? OFF_O1 : OFF_O);
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                float o8[8], y8[8];
+                ld_chunk(ob, swz(r, hf * 4 + c4), o8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int j = c4 * 8 + e;
+                    y8[e] = o8[e] * inv * wn[cb + j] * sigmoid_f((q & 1) ? gate_of(j, 1) : gate_of(j, 0));
+                }
+                st_chunk(sm + OFF_Y, swz(r, hf * 4 + c4), y8);
+            }
+        };
+        // fused: the inverse RMS of chunk q's row from this CTA's sums and the partner's
+        auto fused_inv = [&](int q, bool *ok) -> float {
+            const float *xs = reinterpret_cast<const float *>(sm + OFF_MISC + M_XS);
+            const bool gx = mbar_wait_cluster(&bar[B_XS0 + (q & 3)], (uint32_t)(q >> 2) & 1, abort_flag);
+            *ok = !named_sync_any(3, 128, !gx || *abort_flag != 0);  // lanes 64-127 agree
+            return rsqrtf((prev_local + xs[(q & 3) * 64 + trow - 64]) * (1.f / DV) + POST_EPS);
+        };
         auto o_epilogue = [&]() {
             if (!OUT || trow < 64 || prev_L == 0 || (!FUSED && !a.has_out)) return;
             const int r = trow - 64;
@@ -267,52 +302,57 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             tmem_row32(tl + TM_D + prev_buf + 64, p);
 #pragma unroll
             for (int j = 0; j < 32; ++j) d[j] = prev_eg * d[j] + p[j];
-            float y[32];
+            float inv = 0.f, local = 0.f;
             if (FUSED) {
-                // y = o / sqrt(mean(o^2) + eps) w sigmoid(gate): the mean runs over all dv columns,
-                // half of them in the partner CTA; this CTA's row sums go to the partner's slot of
-                // this chunk's parity, and the partner's arrive in ours
                 float *ssp = reinterpret_cast<float *>(sm + OFF_MISC + M_SKP);
                 float *xs = reinterpret_cast<float *>(sm + OFF_MISC + M_XS);
-                const float *wn = reinterpret_cast<const float *>(sm + OFF_MISC + M_WN);
                 float ss = 0.f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) ss += d[j] * d[j];
                 ssp[hf * 64 + r] = ss;
                 named_sync(3, 128);
-                const float local = ssp[r] + ssp[64 + r];
-                const int slot = prev_m & 1;
-                if (hf == 0) {
-                    const uint32_t partner = (uint32_t)half ^ 1u;
+                local = ssp[r] + ssp[64 + r];
+                if (hf == 0) {  // this chunk's sums to the partner
+                    const uint32_t partner = (uint32_t)half ^ 1u, slot = (uint32_t)prev_m & 3;
                     st_cluster_f32(map_to_rank(xs + slot * 64 + r, partner), local);
                     mbar_arrive_cluster(map_to_rank(&bar[B_XS0 + slot], partner));
                 }
-                const bool gx = mbar_wait_cluster(&bar[B_XS0 + slot], (uint32_t)(prev_m >> 1) & 1, abort_flag);
-                // lanes 64-127 agree; an abort is then agreed on by the chain's next barrier
-                if (named_sync_any(3, 128, !gx || *abort_flag != 0)) return;
-                const float inv = rsqrtf((local + xs[slot * 64 + r]) * (1.f / DV) + POST_EPS);
-#pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    const uint32_t gw = gpk[j >> 1];
-                    y[j] = d[j] * inv * wn[cb + j] * sigmoid_f(bf16_lo(gw));
-                    y[j + 1] = d[j + 1] * inv * wn[cb + j + 1] * sigmoid_f(bf16_hi(gw));
+                if (prev_m >= 1) {  // the previous chunk's y
+                    bool fok = true;
+                    inv = fused_inv(prev_m - 1, &fok);
+                    if (!fok) return;
                 }
             }
-            if (ostore) bulk_wait_read_all();  // the previous chunk's stores have read OFF_O / OFF_Y
+            if (ostore) bulk_wait_read_all();  // the earlier stores have read their staging tiles
             named_sync(3, 128);
-            if (a.has_out) {
+            unsigned char *ob = sm + ((FUSED && (prev_m & 1)) ? OFF_O1 : OFF_O);
+            if (FUSED || a.has_out) {
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + OFF_O, swz(r, hf * 4 + c4), d + c4 * 8);
+                for (int c4 = 0; c4 < 4; ++c4) st_chunk(ob, swz(r, hf * 4 + c4), d + c4 * 8);
             }
-            if (FUSED) {
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + OFF_Y, swz(r, hf * 4 + c4), y + c4 * 8);
-            }
+            if (FUSED && prev_m >= 1) y_tile(prev_m - 1, inv);
             fence_proxy_async();
             named_sync(3, 128);
             if (ostore) {
-                if (a.has_out) tma_store_4d(&mp.out, sm + OFF_O, j0, h, prev_t0, b);
-                if (FUSED) tma_store_4d(&mp.y, sm + OFF_Y, j0, h, prev_t0, b);
+                if (a.has_out) tma_store_4d(&mp.out, ob, j0, h, prev_t0, b);
+                if (FUSED && prev_m >= 1) tma_store_4d(&mp.y, sm + OFF_Y, j0, h, prev_t0 - C, b);
+                bulk_commit();
+            }
+            prev_local = local;
+        };
+        // fused: y of the last chunk, after the loop
+        auto y_last = [&]() {
+            if (!FUSED || trow < 64 || prev_L == 0) return;
+            bool fok = true;
+            const float inv = fused_inv(prev_m, &fok);
+            if (!fok) return;
+            if (ostore) bulk_wait_read_all();
+            named_sync(3, 128);
+            y_tile(prev_m, inv);
+            fence_proxy_async();
+            named_sync(3, 128);
+            if (ostore) {
+                tma_store_4d(&mp.y, sm + OFF_Y, j0, h, prev_t0, b);
                 bulk_commit();
             }
         };
@@ -364,11 +404,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
                     for (int e = 0; e < 8; ++e) ut[e] *= rowf;
                     st_chunk(sm + OFF_UD, o, ut);
                 }
-            } else if (FUSED) {  // lanes 64-127, idle here: this chunk's gate logits, kept for its o
+            } else if (FUSED) {  // lanes 64-127, idle here: this chunk's gate logits, kept for its y
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
                     const uint4 g4 = *reinterpret_cast<const uint4 *>(st + FS_G + swz(trow - 64, hf * 4 + c4));
-                    gpk[c4 * 4] = g4.x; gpk[c4 * 4 + 1] = g4.y; gpk[c4 * 4 + 2] = g4.z; gpk[c4 * 4 + 3] = g4.w;
+                    if (m & 1) {
+                        gpk1[c4 * 4] = g4.x; gpk1[c4 * 4 + 1] = g4.y; gpk1[c4 * 4 + 2] = g4.z; gpk1[c4 * 4 + 3] = g4.w;
+                    } else {
+                        gpk0[c4 * 4] = g4.x; gpk0[c4 * 4 + 1] = g4.y; gpk0[c4 * 4 + 2] = g4.z; gpk0[c4 * 4 + 3] = g4.w;
+                    }
                 }
             }
             fence_proxy_async();
@@ -413,6 +457,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             prev_L = L; prev_t0 = t0; prev_eg = rowf; prev_buf = buf; prev_m = m;
         }
         if (*abort_flag == 0) o_epilogue();  // last chunk
+        if (*abort_flag == 0) y_last();
         if (wc == 0 || ostore) bulk_wait_all();
         if (*abort_flag == 0) {
             if (OUT && a.ST) {
