@@ -23,12 +23,15 @@
 // <= 1, inside it at most e^{the block's fall}.  Chunks whose gate falls more than KDA_DIAG_SPAN
 // inside a block are left to the CUDA-core gradient kernel (this kernel skips them).
 //
-// One CTA of 128 threads per chunk, phases in order (each a batch of MMAs, then an epilogue):
+// One CTA of 256 threads per chunk (two threads per key channel: warps w and w + 4 share TMEM
+// lane quarter w, and split each epilogue's token columns in halves), phases in order:
 //   A  loads; [Qd^T | -dWm^T] = S [dO ; dU]^T, Tm^T = dS+ U^T;  RS, g (from log alpha), dWm^T tile
-//   B  loads of M, W, U~;  dB_k^T = dWm^T T,  dB_v^T = dU^T T;  their bf16 tiles
+//   B  loads of M, W, U~, v;  dB_k^T = dWm^T T,  dB_v^T = dU^T T;  their bf16 tiles, dv, v . dB_v
 //   C  dA' = dB [W | U~]^T and its transpose, [dO ; U][dO ; U]^T (dP and dP^T in one product);
 //      dM, dP, dM^T, dP^T tiles, the dbeta part of A;  the gate-scaled sections Km, Kp, Qp
 //   D  X^T, Yv^T, Z^T (block by block, N = 16);  the final per-channel epilogue
+// Sums over the channels of one token (dbeta's) reduce 32 tokens across a warp's 32 lanes in 31
+// shuffles (recursive halving), then over the four warps of a lane quarter through shared memory.
 // Every wait is bounded (~1 s); an expired wait raises the device error word.
 #include "tc_host.cuh"
 #include "tc_path.cuh"
@@ -43,17 +46,18 @@ using dr::tcf::ld_chunk;
 using dr::tcf::st_chunk;
 
 constexpr int C = 64, DK = 128, DV = 128;
-constexpr int NTHREADS = 128;
+constexpr int NTHREADS = 256;
 // shared memory (bytes from a 1024-aligned base); regions are reused phase by phase
 //   phase A:   S [0, 32K), dS+ [32K, 64K), [dO ; dU] [64K, 96K), [dO ; U] [96K, 128K),
 //              T [128K, 136K), log alpha [136K, 152K), q [152K, 168K), k [168K, 184K)
 //   E0 writes: G (fp32) [184K, 216K), dWm^T [136K, 152K) (after log alpha is read)
-//   phase B:   M [0, 8K), W [8K, 24K), U~ [24K, 40K);  E1 writes dB_k^T [64K, 80K), dB_v^T [80K, 96K)
+//   phase B:   M [0, 8K), W [8K, 24K), U~ [24K, 40K), v [40K, 56K) (dS+ is read by then);
+//              E1 writes dB_k^T [64K, 80K), dB_v^T [80K, 96K)
 //   E2 writes: dM [120K, 128K), dP [128K, 136K), dM^T [136K, 144K), dP^T [144K, 152K)
 //   build:     Km [0, 40K), Kp [40K, 80K), Qp [80K, 120K)
 constexpr uint32_t R_S = 0, R_DS = 32768, R_OU = 65536, R_OV = 98304, R_T = 131072, R_AL = 139264;
 constexpr uint32_t R_Q = 155648, R_K = 172032, R_G = 188416, R_DWM = 139264;
-constexpr uint32_t R_M = 0, R_W = 8192, R_UT = 24576, R_DBK = 65536, R_DBV = 81920;
+constexpr uint32_t R_M = 0, R_W = 8192, R_UT = 24576, R_V = 40960, R_DBK = 65536, R_DBV = 81920;
 constexpr uint32_t R_DM = 122880, R_DP = 131072, R_DMT = 139264, R_DPT = 147456;
 constexpr uint32_t R_KM = 0, R_KP = 40960, R_QP = 81920;
 constexpr uint32_t SEC_PANEL = KDA_KH_ROWS * 128;  // 160 rows x 128 B: one 64-channel panel of a section set
@@ -63,23 +67,25 @@ constexpr uint32_t M_BAR = 0;  // [0] phase-A loads, [1] phase-B loads, [2] MMA
 constexpr uint32_t M_TMEM = 32, M_ABORT = 36;
 constexpr uint32_t M_BETA = 64;          // [64] beta
 constexpr uint32_t M_DBA = M_BETA + 256;  // [64] the dbeta part of A
-constexpr uint32_t M_RED = M_DBA + 256;   // [2 kinds][4 warps][64] dbeta partial sums
-constexpr uint32_t SMEM_BYTES = R_MISC + M_RED + 2 * 4 * 64 * 4;
-static_assert(R_MISC + M_RED + 2048 <= 227 * 1024 - 1024, "shared memory");
+constexpr uint32_t M_RED = M_DBA + 256;   // [2 kinds][4 lane quarters][64 tokens] dbeta partial sums
+constexpr uint32_t M_XCH = M_RED + 2048;  // [2 halves][3][128]: dg_C and RS partials, the upper half's dg sum
+constexpr uint32_t SMEM_BYTES = R_MISC + M_XCH + 3 * 2 * 128 * 4;
+static_assert(SMEM_BYTES <= 227 * 1024 - 1024, "shared memory");
+static_assert(R_V + 16384 <= R_DS + 32768 && R_V >= R_UT + 16384, "v tile inside the dead dS+ tile");
 // TMEM columns (lane = key channel c, or value channel j for dB_v^T, or token row for dA', dP)
 constexpr uint32_t TM_QD = 0, TM_X = 64, TM_TM = 128, TM_DBK = 192, TM_DBV = 256, TM_YV = 320, TM_D5 = 384,
                    TM_Z = 384, TM_COLS = 512;
-constexpr uint32_t LOADA_BYTES = 4 * 32768 + 8192 + 3 * 16384, LOADB_BYTES = 8192 + 2 * 16384;
+constexpr uint32_t LOADA_BYTES = 4 * 32768 + 8192 + 3 * 16384, LOADB_BYTES = 8192 + 3 * 16384;
 
 struct Maps {
-    CUtensorMap q, k, dout, alpha;  // [B, T, H, 128] bf16; box 64 channels x 64 tokens
+    CUtensorMap q, k, v, dout, alpha;  // [B, T, H, 128] bf16; box 64 channels x 64 tokens
     CUtensorMap S, dS;              // [chunks * 128][128] bf16; box 64 x 128
     CUtensorMap U, dU, W, Ut;       // [chunks * 64][128] bf16; box 64 x 64
     CUtensorMap T, M;               // [chunks * 64][64] bf16; box 64 x 64
 };
 
 struct Args {
-    const __nv_bfloat16 *beta, *v;  // [B, T, H], [B, T, H, 128]
+    const __nv_bfloat16 *beta;  // [B, T, H]
     __nv_bfloat16 *dq, *dk, *dv, *dalpha, *dbeta;
     const int *kwide;               // [chunks]: left to the CUDA-core kernel
     int T, H, N;
@@ -97,6 +103,31 @@ __device__ __forceinline__ uint32_t el_off(int row, int c, uint32_t panel) {
 __device__ __forceinline__ float ld_bf(const unsigned char *base, uint32_t off) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(base + off));
 }
+// x[t] (t < 32) summed over the warp's lanes, by recursive halving: each step keeps half of the
+// remaining tokens and adds the partner lane's copy of them; afterwards x[0] of lane l is token l's sum
+__device__ __forceinline__ float warp_sum32(float (&x)[32], int lane) {
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) {
+        const bool up = (lane & s) != 0;
+#pragma unroll
+        for (int i = 0; i < s; ++i) {
+            const float send = up ? x[i] : x[i + s], keep = up ? x[i + s] : x[i];
+            x[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+        }
+    }
+    return x[0];
+}
+// 8 consecutive floats of a [64][128] fp32 tile (c0 a multiple of 8).  The two 16-byte halves are
+// read in an order that depends on bit 2 of c0 / 8, so that the eight threads of a quarter warp
+// reading one row at c0 = 0, 8, ..., 56 (or 64, ..., 120) hit eight different 4-bank groups.
+__device__ __forceinline__ void ld_g8(const float *G, int row, int c0, float *o) {
+    const int h = (c0 >> 5) & 1;
+    const float4 a = *reinterpret_cast<const float4 *>(G + row * 128 + c0 + 4 * h);
+    const float4 b = *reinterpret_cast<const float4 *>(G + row * 128 + c0 + 4 * (1 - h));
+    const float lo[4] = {h ? b.x : a.x, h ? b.y : a.y, h ? b.z : a.z, h ? b.w : a.w};
+    const float hi[4] = {h ? a.x : b.x, h ? a.y : b.y, h ? a.z : b.z, h ? a.w : b.w};
+    o[0] = lo[0]; o[1] = lo[1]; o[2] = lo[2]; o[3] = lo[3]; o[4] = hi[0]; o[5] = hi[1]; o[6] = hi[2]; o[7] = hi[3];
+}
 
 __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constant__ Maps mp, Args a) {
     const int ci = blockIdx.x;
@@ -111,9 +142,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
     float *betas = reinterpret_cast<float *>(misc + M_BETA);
     float *dba = reinterpret_cast<float *>(misc + M_DBA);
     float *red = reinterpret_cast<float *>(misc + M_RED);
+    float *xch = reinterpret_cast<float *>(misc + M_XCH);
     const float *G = reinterpret_cast<const float *>(sm + R_G);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q4 = warp & 3, hf = warp >> 2;  // lane quarter; half of the token columns
     const int n = ci % a.N, bh = ci / a.N, h = bh % a.H, b = bh / a.H;
     const int T = a.T, H = a.H, t0 = n * C, L = min(C, T - t0);
     auto trow_g = [&](int rr) -> size_t { return ((size_t)b * T + t0 + rr) * H + h; };
@@ -145,21 +178,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
     __syncthreads();
     fence_after_sync();
     const uint32_t tbase = *tmem_slot;
-    const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);  // this warp's lane quarter
+    const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);  // this warp's lane quarter
     auto consensus = [&](bool ok) -> bool { return !named_sync_any(1, NTHREADS, !ok || *abort_flag != 0); };
     uint32_t ph = 0;
-    auto wait_mma = [&]() -> bool {
+    auto wait_mma = [&](bool also_ok) -> bool {
         const bool ok = mbar_wait(&bar[2], ph & 1, abort_flag);
         ph++;
         fence_after_sync();
-        return consensus(ok);
+        return consensus(ok && also_ok);
     };
     auto commit = [&]() {
         mma_commit(&bar[2]);
         armed[2]++;
     };
     auto u32 = [&](uint32_t off) { return smem_u32(sm + off); };
-    const int c = tid;  // this thread's key channel (TMEM lane)
+    const int c = tid & (DK - 1);  // this thread's key channel (TMEM lane); also value channel j = c
+    const int r0 = 32 * hf;         // first token of this thread's column half
 
     bool ok = consensus(mbar_wait(&bar[0], 0, abort_flag));
     // ======================= phase A products =======================
@@ -174,42 +208,45 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
         }
         commit();
     }
-    // while they run: g of channel c (prefix sum over the chunk's tokens; tokens past T add 0)
+    // while they run: g of channel c at this half's tokens (prefix sum over the chunk; tokens past T
+    // add 0), and this half's part of RS_c (the state tiles' panel hf)
     if (ok) {
         float run = 0.f;
         float *Gw = reinterpret_cast<float *>(sm + R_G);
-        for (int r = 0; r < C; ++r) {
+        if (hf) {
+#pragma unroll 8
+            for (int r = 0; r < 32; ++r) run += ld_bf(sm + R_AL, el_off(r, c, 8192));
+        }
+#pragma unroll 8
+        for (int r = r0; r < r0 + 32; ++r) {
             run += ld_bf(sm + R_AL, el_off(r, c, 8192));
             Gw[r * DK + c] = run;
         }
+        float rs = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+            float s8[8], d8[8];
+            const uint32_t o = (uint32_t)hf * 16384 + swz(c, ch);
+            ld_chunk(sm + R_S, o, s8);
+            ld_chunk(sm + R_DS, o, d8);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) rs += s8[e] * d8[e];
+        }
+        xch[(hf * 3 + 1) * 128 + c] = rs;
     }
-    if (ok) ok = wait_mma();
-    float rs = 0.f;  // RS_c
+    ok = consensus(ok);  // the log-alpha tile is read: dWm^T may take its space
+    if (ok) ok = wait_mma(true);
     if (ok) {
-        // RS_c from the state tiles; then -dWm^T row c (TMEM columns 64..127 of [Qd^T | dU S^T]) as
-        // the bf16 A operand of dB_k^T, over the log-alpha tile (read by every thread above)
-#pragma unroll
-        for (int p = 0; p < 2; ++p)
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                float s8[8], d8[8];
-                const uint32_t o = (uint32_t)p * 16384 + swz(c, ch);
-                ld_chunk(sm + R_S, o, s8);
-                ld_chunk(sm + R_DS, o, d8);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) rs += s8[e] * d8[e];
-            }
-    }
-    ok = consensus(ok);  // the log-alpha tile and the state tiles are read
-    if (ok) {
-        float v[64];
-        tmem_ld16(tl + TM_QD + 64, v); tmem_ld16(tl + TM_QD + 80, v + 16);
-        tmem_ld16(tl + TM_QD + 96, v + 32); tmem_ld16(tl + TM_QD + 112, v + 48);
+        // -dWm^T row c (TMEM columns 64..127 of [Qd^T | dU S^T]), this half's 32 tokens, as the
+        // bf16 A operand of dB_k^T
+        float v[32];
+        tmem_ld16(tl + TM_QD + 64 + r0, v);
+        tmem_ld16(tl + TM_QD + 80 + r0, v + 16);
         wait_ld();
 #pragma unroll
-        for (int j = 0; j < 64; ++j) v[j] = -v[j];  // dWm^T = -(dU S^T)^T
+        for (int j = 0; j < 32; ++j) v[j] = -v[j];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_DWM, swz(c, ch), v + ch * 8);
+        for (int ch = 0; ch < 4; ++ch) st_chunk(sm + R_DWM, swz(c, 4 * hf + ch), v + ch * 8);
     }
     fence_proxy_async();
     fence_before_sync();
@@ -223,6 +260,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
         for (int p = 0; p < 2; ++p) {
             tma_load_2d(sm + R_W + p * 8192, &mp.W, 64 * p, ci * C, &bar[1]);
             tma_load_2d(sm + R_UT + p * 8192, &mp.Ut, 64 * p, ci * C, &bar[1]);
+            tma_load_4d(sm + R_V + p * 8192, &mp.v, 64 * p, h, t0, b, &bar[1]);
         }
         armed[1] = 1;
         // dB_k^T = dWm^T T (A K-major [c][r]; B = T [r][i] MN-major)
@@ -237,24 +275,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
         }
         commit();
     }
-    if (ok) ok = wait_mma();
-    if (ok) {  // the bf16 tiles dB_k^T [c][i] and dB_v^T [j][i] (lane = c, or j)
-        float v[64];
-        tmem_ld16(tl + TM_DBK, v); tmem_ld16(tl + TM_DBK + 16, v + 16);
-        tmem_ld16(tl + TM_DBK + 32, v + 32); tmem_ld16(tl + TM_DBK + 48, v + 48);
+    if (ok) ok = wait_mma(mbar_wait(&bar[1], 0, abort_flag));  // the products; M, W, U~, v
+    if (ok) {
+        // the bf16 tiles dB_k^T [c][i] and dB_v^T [j][i] (this half's 32 tokens), dv, and v . dB_v
+        float v[32];
+        tmem_ld16(tl + TM_DBK + r0, v);
+        tmem_ld16(tl + TM_DBK + 16 + r0, v + 16);
         wait_ld();
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_DBK, swz(c, ch), v + ch * 8);
-        tmem_ld16(tl + TM_DBV, v); tmem_ld16(tl + TM_DBV + 16, v + 16);
-        tmem_ld16(tl + TM_DBV + 32, v + 32); tmem_ld16(tl + TM_DBV + 48, v + 48);
+        for (int ch = 0; ch < 4; ++ch) st_chunk(sm + R_DBK, swz(c, 4 * hf + ch), v + ch * 8);
+        tmem_ld16(tl + TM_DBV + r0, v);
+        tmem_ld16(tl + TM_DBV + 16 + r0, v + 16);
         wait_ld();
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_DBV, swz(c, ch), v + ch * 8);
+        for (int ch = 0; ch < 4; ++ch) st_chunk(sm + R_DBV, swz(c, 4 * hf + ch), v + ch * 8);
+        float sv[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int r = r0 + e;
+            sv[e] = ld_bf(sm + R_V, el_off(r, c, 8192)) * v[e];
+            if (r < L) a.dv[trow_g(r) * DV + c] = __float2bfloat16_rn(betas[r] * v[e]);
+        }
+        red[(4 + q4) * 64 + r0 + lane] = warp_sum32(sv, lane);
     }
     fence_proxy_async();
     fence_before_sync();
     ok = consensus(ok);
-    if (ok) ok = consensus(mbar_wait(&bar[1], 0, abort_flag));  // M, W, U~
     // ======================= phase C products =======================
     if (ok && tid == 0) {
         fence_after_sync();
@@ -282,58 +328,62 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
         }
         commit();
     }
-    if (ok) ok = wait_mma();
+    if (ok) ok = wait_mma(true);
     // ---- E2: the masked tiles dM, dP [r][i] and dM^T, dP^T [i][r]; the dbeta part of A ----
+    //   lanes 0-63 (quarters 0, 1): half 0 takes dA' (-> dM, dbeta_A), half 1 takes dP, and each
+    //   half takes 32 columns of dA'^T (-> dM^T);  lanes 64-127: each half takes 32 columns of dP^T
     if (ok) {
         float x[64];
-        if (warp < 2) {
-            const int r = tid;  // token row r (and, for the transposed products, row i = tid)
-            // dA'[r][i] -> dM[r][i] = -beta_r dA' (i < r), dbeta_A
-            tmem_ld16(tl + TM_X, x); tmem_ld16(tl + TM_X + 16, x + 16);
-            tmem_ld16(tl + TM_X + 32, x + 32); tmem_ld16(tl + TM_X + 48, x + 48);
-            wait_ld();
-            float db = 0.f;
-            const float br = betas[r];
+        const int rl = (warp & 1) * 32 + lane;  // the product's row (r, or i for the transposes)
+        if (q4 < 2) {
+            if (hf == 0) {
+                const int r = rl;  // dA'[r][i] -> dM[r][i] = -beta_r dA' (i < r), dbeta_A
+                tmem_ld16(tl + TM_X, x); tmem_ld16(tl + TM_X + 16, x + 16);
+                tmem_ld16(tl + TM_X + 32, x + 32); tmem_ld16(tl + TM_X + 48, x + 48);
+                wait_ld();
+                float db = 0.f;
+                const float br = betas[r];
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                float m8[8], w8[8];
-                ld_chunk(sm + R_M, swz(r, ch), m8);
+                for (int ch = 0; ch < 8; ++ch) {
+                    float m8[8], w8[8];
+                    ld_chunk(sm + R_M, swz(r, ch), m8);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int i = ch * 8 + e;
-                    const float d = i < r ? -x[i] : 0.f;
-                    db += d * m8[e];
-                    w8[e] = br * d;
+                    for (int e = 0; e < 8; ++e) {
+                        const int i = ch * 8 + e;
+                        const float d = i < r ? -x[i] : 0.f;
+                        db += d * m8[e];
+                        w8[e] = br * d;
+                    }
+                    st_chunk(sm + R_DM, swz(r, ch), w8);
                 }
-                st_chunk(sm + R_DM, swz(r, ch), w8);
+                dba[r] = db;
+            } else {
+                const int r = rl;  // dP[r][i] (i <= r)
+                tmem_ld16(tl + TM_D5 + 64, x); tmem_ld16(tl + TM_D5 + 80, x + 16);
+                tmem_ld16(tl + TM_D5 + 96, x + 32); tmem_ld16(tl + TM_D5 + 112, x + 48);
+                wait_ld();
+#pragma unroll
+                for (int i = 0; i < 64; ++i) x[i] = i <= r ? x[i] : 0.f;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_DP, swz(r, ch), x + ch * 8);
             }
-            dba[r] = db;
-            // dP[r][i] (i <= r)
-            tmem_ld16(tl + TM_D5 + 64, x); tmem_ld16(tl + TM_D5 + 80, x + 16);
-            tmem_ld16(tl + TM_D5 + 96, x + 32); tmem_ld16(tl + TM_D5 + 112, x + 48);
+            const int i = rl;  // dA'^T[i][r] -> dM^T[i][r] = -beta_r dA'^T (r > i), r in this half
+            tmem_ld16(tl + TM_YV + r0, x);
+            tmem_ld16(tl + TM_YV + 16 + r0, x + 16);
             wait_ld();
 #pragma unroll
-            for (int i = 0; i < 64; ++i) x[i] = i <= r ? x[i] : 0.f;
+            for (int e = 0; e < 32; ++e) x[e] = r0 + e > i ? -betas[r0 + e] * x[e] : 0.f;
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_DP, swz(r, ch), x + ch * 8);
-            // dA'^T[i][r] -> dM^T[i][r] = -beta_r dA'^T (r > i)
-            const int i = tid;
-            tmem_ld16(tl + TM_YV, x); tmem_ld16(tl + TM_YV + 16, x + 16);
-            tmem_ld16(tl + TM_YV + 32, x + 32); tmem_ld16(tl + TM_YV + 48, x + 48);
-            wait_ld();
-#pragma unroll
-            for (int rr = 0; rr < 64; ++rr) x[rr] = rr > i ? -betas[rr] * x[rr] : 0.f;
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_DMT, swz(i, ch), x + ch * 8);
+            for (int ch = 0; ch < 4; ++ch) st_chunk(sm + R_DMT, swz(i, 4 * hf + ch), x + ch * 8);
         } else {
-            const int i = tid - 64;  // dP^T[i][r] (r >= i)
-            tmem_ld16(tl + TM_D5, x); tmem_ld16(tl + TM_D5 + 16, x + 16);
-            tmem_ld16(tl + TM_D5 + 32, x + 32); tmem_ld16(tl + TM_D5 + 48, x + 48);
+            const int i = rl;  // dP^T[i][r] (r >= i), r in this half
+            tmem_ld16(tl + TM_D5 + r0, x);
+            tmem_ld16(tl + TM_D5 + 16 + r0, x + 16);
             wait_ld();
 #pragma unroll
-            for (int rr = 0; rr < 64; ++rr) x[rr] = rr >= i ? x[rr] : 0.f;
+            for (int e = 0; e < 32; ++e) x[e] = r0 + e >= i ? x[e] : 0.f;
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_DPT, swz(i, ch), x + ch * 8);
+            for (int ch = 0; ch < 4; ++ch) st_chunk(sm + R_DPT, swz(i, 4 * hf + ch), x + ch * 8);
         }
     }
     ok = consensus(ok);  // M, W, U~ and the dB tiles are read: the sections may take their space
@@ -353,21 +403,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
             int I = 0;
             while (I < 3 && row >= kp_sec(I + 1)) ++I;
             const int tr = 16 * I + (row - kp_sec(I));
-            float ki[8], kr[8], qr[8], vm[8], vp[8], vq[8];
+            float ki[8], kr[8], qr[8], gb[8], gi[8], gr[8], ge[8];
             ld_chunk(sm + R_K, (uint32_t)(c0 >> 6) * 8192 + swz(ti, (c0 & 63) >> 3), ki);
             ld_chunk(sm + R_K, (uint32_t)(c0 >> 6) * 8192 + swz(tr, (c0 & 63) >> 3), kr);
             ld_chunk(sm + R_Q, (uint32_t)(c0 >> 6) * 8192 + swz(tr, (c0 & 63) >> 3), qr);
+            ld_g8(G, 16 * R, c0, gb);
+            ld_g8(G, ti, c0, gi);
+            ld_g8(G, tr, c0, gr);
+            ld_g8(G, 16 * I + 15, c0, ge);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const int cc2 = c0 + e;
-                vm[e] = ki[e] * __expf(fminf(G[16 * R * DK + cc2] - G[ti * DK + cc2], 80.f));
-                const float f = __expf(fminf(G[tr * DK + cc2] - G[(16 * I + 15) * DK + cc2], 80.f));
-                vp[e] = kr[e] * f;
-                vq[e] = qr[e] * f;
+                ki[e] *= __expf(fminf(gb[e] - gi[e], 80.f));
+                const float f = __expf(fminf(gr[e] - ge[e], 80.f));
+                kr[e] *= f;
+                qr[e] *= f;
             }
-            st_chunk(sm + R_KM, o, vm);
-            st_chunk(sm + R_KP, o, vp);
-            st_chunk(sm + R_QP, o, vq);
+            st_chunk(sm + R_KM, o, ki);
+            st_chunk(sm + R_KP, o, kr);
+            st_chunk(sm + R_QP, o, qr);
         }
     }
     fence_proxy_async();
@@ -395,28 +448,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
         }
         commit();
     }
-    if (ok) ok = wait_mma();
-    // ======================= final epilogue: thread c (and thread j = c for dv) =======================
+    if (ok) ok = wait_mma(true);
+    // ======================= final epilogue: thread (c, half): tokens r0 .. r0 + 31 =======================
+    const float gL = G[(C - 1) * DK + c];
+    float dgr[32];
     if (ok) {
-        const float gL = G[(C - 1) * DK + c];
-        float dgr[64];
-        float dgc = 0.f;
+        float dgc = 0.f, sbk[32];
 #pragma unroll
-        for (int rb = 0; rb < 4; ++rb) {
-            float qd[16], tm[16], bk[16], xx[16], yv[16], zz[16], bv[16];
+        for (int rh = 0; rh < 2; ++rh) {
+            const int rb = 2 * hf + rh;
+            float qd[16], tm[16], bk[16], xx[16], yv[16], zz[16];
             tmem_ld16(tl + TM_QD + 16 * rb, qd);
             tmem_ld16(tl + TM_TM + 16 * rb, tm);
             tmem_ld16(tl + TM_DBK + 16 * rb, bk);
             tmem_ld16(tl + TM_X + 16 * rb, xx);
             tmem_ld16(tl + TM_YV + 16 * rb, yv);
             tmem_ld16(tl + TM_Z + 16 * rb, zz);
-            tmem_ld16(tl + TM_DBV + 16 * rb, bv);
             wait_ld();
             const float gb = G[16 * rb * DK + c], ge = G[(16 * rb + 15) * DK + c];
-            float sbk[16], sbv[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-                const int r = 16 * rb + e;
+                const int r = 16 * rb + e, idx = 16 * rh + e;
                 const float g = G[r * DK + c], br = betas[r];
                 const float qv = ld_bf(sm + R_Q, el_off(r, c, 8192)), kv = ld_bf(sm + R_K, el_off(r, c, 8192));
                 const float gam = __expf(g), eb = __expf(gL - g);
@@ -425,47 +477,42 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
                 const float dq = gam * qd[e] + X;
                 const float t = eb * tm[e], sb = br * gam * bk[e];
                 const float dk = Yv + Z + sb + t;
-                dgr[r] = qv * dq + kv * (Yv - Z + sb - t);
+                dgr[idx] = qv * dq + kv * (Yv - Z + sb - t);
                 dgc += kv * t;
-                sbk[e] = gam * kv * bk[e];
+                sbk[idx] = gam * kv * bk[e];
                 if (r < L) {
                     const size_t o = trow_g(r) * DK + c;
                     a.dq[o] = __float2bfloat16_rn(dq);
                     a.dk[o] = __float2bfloat16_rn(dk);
                 }
-                // thread c is also value channel j = c of dB_v^T
-                float vv = 0.f;
-                if (r < L) {
-                    const size_t o = trow_g(r) * DV + c;
-                    vv = __bfloat162float(a.v[o]);
-                    a.dv[o] = __float2bfloat16_rn(br * bv[e]);
-                }
-                sbv[e] = vv * bv[e];
-            }
-            // sums over the channels (threads) per token: warps, then 4 partials
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const float s1 = warp_sum(sbk[e]), s2 = warp_sum(sbv[e]);
-                if (lane == 0) {
-                    red[(0 * 4 + warp) * 64 + 16 * rb + e] = s1;
-                    red[(1 * 4 + warp) * 64 + 16 * rb + e] = s2;
-                }
             }
         }
-        // d log alpha: the chunk-end terms belong to the last row, then the reverse cumulative sum
-        float run = dgc + __expf(gL) * rs;
+        red[q4 * 64 + r0 + lane] = warp_sum32(sbk, lane);
+        xch[(hf * 3 + 0) * 128 + c] = dgc;
+        if (hf) {
+            float tot = 0.f;
 #pragma unroll
-        for (int r = C - 1; r >= 0; --r) {
-            run += dgr[r];
-            if (r < L) a.dalpha[trow_g(r) * DK + c] = __float2bfloat16_rn(run);
+            for (int e = 0; e < 32; ++e) tot += dgr[e];
+            xch[(1 * 3 + 2) * 128 + c] = tot;
         }
     }
     ok = consensus(ok);
-    if (ok && tid < L) {
-        float s = dba[tid];
+    if (ok) {
+        // d log alpha: the chunk-end terms (dg_C and e^{g_C} RS) belong to the last row, then the
+        // reverse cumulative sum; the lower half starts from the upper half's total
+        float run = xch[0 * 128 + c] + xch[3 * 128 + c] + __expf(gL) * (xch[1 * 128 + c] + xch[4 * 128 + c]);
+        if (!hf) run += xch[5 * 128 + c];
 #pragma unroll
-        for (int w = 0; w < 4; ++w) s += red[(0 * 4 + w) * 64 + tid] + red[(1 * 4 + w) * 64 + tid];
-        a.dbeta[trow_g(tid)] = __float2bfloat16_rn(s);
+        for (int e = 31; e >= 0; --e) {
+            run += dgr[e];
+            if (r0 + e < L) a.dalpha[trow_g(r0 + e) * DK + c] = __float2bfloat16_rn(run);
+        }
+        if (tid < L) {
+            float s = dba[tid];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) s += red[w * 64 + tid] + red[(4 + w) * 64 + tid];
+            a.dbeta[trow_g(tid)] = __float2bfloat16_rn(s);
+        }
     }
     if (tid == 0 && *abort_flag) {  // let whatever was issued land before the CTA leaves
         volatile int dummy = 0;
@@ -487,6 +534,7 @@ cudaError_t tc_bwd_kda(const Geo &g, const Tensors &t, const TcWs &w, cudaStream
     Maps mp;
     const uint64_t Bn = g.B, T = g.T, H = g.H, NC = (uint64_t)g.B * g.H * g.N;
     bool ok = tc::make_map_4d_bf16(&mp.q, t.q, DK, H, T, Bn, 64) && tc::make_map_4d_bf16(&mp.k, t.k, DK, H, T, Bn, 64) &&
+              tc::make_map_4d_bf16(&mp.v, t.v, DV, H, T, Bn, 64) &&
               tc::make_map_4d_bf16(&mp.alpha, t.alpha, DK, H, T, Bn, 64) &&
               tc::make_map_2d_bf16(&mp.S, w.Sn, DV, NC * DK, 128) && tc::make_map_2d_bf16(&mp.dS, w.dSn, DV, NC * DK, 128) &&
               tc::make_map_2d_bf16(&mp.U, w.Un, DV, NC * C, 64) && tc::make_map_2d_bf16(&mp.dU, w.dUn, DV, NC * C, 64) &&
@@ -495,7 +543,7 @@ cudaError_t tc_bwd_kda(const Geo &g, const Tensors &t, const TcWs &w, cudaStream
     if (ok) ok = t.dout && tc::make_map_4d_bf16(&mp.dout, t.dout, DV, H, T, Bn, 64);  // the backward requires dO
     if (!ok) return cudaErrorInvalidValue;
     Args a;
-    a.beta = (const __nv_bfloat16 *)t.beta; a.v = (const __nv_bfloat16 *)t.v;
+    a.beta = (const __nv_bfloat16 *)t.beta;
     a.dq = (__nv_bfloat16 *)t.dq; a.dk = (__nv_bfloat16 *)t.dk; a.dv = (__nv_bfloat16 *)t.dv;
     a.dalpha = (__nv_bfloat16 *)t.dalpha; a.dbeta = (__nv_bfloat16 *)t.dbeta; a.kwide = w.kwide;
     a.T = g.T; a.H = g.H; a.N = g.N;

@@ -62,9 +62,12 @@ constexpr uint32_t M_SKP = M_CF + 2 * 132 * 4;  // reverse: [2 column halves][64
 constexpr uint32_t M_XS = M_SKP + 512;          // fused forward: [4 slots (chunk mod 4)][64] the partner's
                                                 // row sums of squares (written by the partner CTA)
 constexpr uint32_t M_WN = M_XS + 1024;          // fused forward: this CTA's 64 RMSNorm weights
-// B_XS0..3 (fused forward): the partner's row sums of a chunk (mod 4) have arrived
+constexpr uint32_t M_SQ1 = M_WN + 256;          // fused forward: o's row-sum partials of odd chunks
+                                                // (even chunks: M_SKP)
+// B_XS0..3 (fused forward): the partner's row sums of a chunk (mod 4) have arrived (256 bytes of
+// asynchronous remote stores, armed by this CTA)
 enum { B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_MMA, B_XS0, B_XS1, B_XS2, B_XS3, B_NUM };
-static_assert(B_NUM * 8 <= M_TMEM && M_WN + 256 <= 4096, "misc overflow");
+static_assert(B_NUM * 8 <= M_TMEM && M_SQ1 + 512 <= 4096 && M_WN % 16 == 0, "misc overflow");
 constexpr float POST_EPS = 1e-6f;  // y = o / sqrt(mean(o^2) + eps) w sigmoid(gate)
 
 struct FMaps {
@@ -95,42 +98,58 @@ struct Args {
     const float *wn;          // fused forward: RMSNorm weight [128]
 };
 
-// Producer side, KDA: the per-channel decay e^{g_C} of chunk ci into cf[0..127].
-__device__ __forceinline__ void chunk_factors_kda(const float *egc, size_t ci, float *cf, int lane) {
+// The producer's gate factors of a chunk (e^{g_C - g}, e^g, e^{g_C}; fused forward: with the raw
+// rows' norms folded in, k's rows by 1 / |k_r|, o's by 1 / |q_r|; KDA: e^{g_C} per key channel).
+// Their inputs are fetched into registers before the producer waits for a free stage, so that the
+// global loads' latency overlaps the wait.
+struct FactorIn {
+    float x[4], r[4], gc;
+};
+template <bool KDA, bool FUSED>
+__device__ __forceinline__ void factors_fetch(const Args &a, size_t ci, int lane, FactorIn &f) {
+    if (KDA) {
 #pragma unroll
-    for (int c = lane; c < 128; c += 32) cf[c] = egc[ci * 128 + c];
-}
-
-// Producer side: the gate factors of chunk ci into cf (e^{g_C - g}, e^g, e^{g_C}).
-__device__ __forceinline__ void chunk_factors(const float *gb, size_t ci, float *cf, int lane) {
-    const float *gg = gb + ci * 2 * C;
-    const float gC = gg[C - 1];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        const int r = lane + 32 * hh;
-        const float x = gg[r];
-        cf[r] = __expf(gC - x);
-        cf[64 + r] = __expf(x);
+        for (int k = 0; k < 4; ++k) f.x[k] = a.egc[ci * 128 + lane + 32 * k];
+    } else {
+        const float *gg = a.gb + ci * 2 * C;
+        f.gc = gg[C - 1];
+        f.x[0] = gg[lane];
+        f.x[1] = gg[lane + 32];
+        if (FUSED) {
+            const float *rr = a.rn + ci * 2 * C;
+            f.r[0] = rr[lane];
+            f.r[1] = rr[lane + 32];
+            f.r[2] = rr[C + lane];
+            f.r[3] = rr[C + lane + 32];
+        }
     }
-    if (lane == 0) cf[128] = __expf(gC);
 }
-
-// Fused forward: the same with the raw rows' norms folded in (k's rows by 1 / |k_r|, o's by 1 / |q_r|).
-__device__ __forceinline__ void chunk_factors_fused(const float *gb, const float *rn, size_t ci, float *cf,
-                                                    int lane) {
-    const float *gg = gb + ci * 2 * C, *rr = rn + ci * 2 * C;
-    const float gC = gg[C - 1];
+template <bool KDA, bool FUSED>
+__device__ __forceinline__ void factors_store(const FactorIn &f, float *cf, int lane) {
+    if (KDA) {
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        const int r = lane + 32 * hh;
-        const float x = gg[r];
-        cf[r] = __expf(gC - x) * rr[r];
-        cf[64 + r] = __expf(x) * rr[C + r];
+        for (int k = 0; k < 4; ++k) cf[lane + 32 * k] = f.x[k];
+    } else {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int r = lane + 32 * hh;
+            cf[r] = __expf(f.gc - f.x[hh]) * (FUSED ? f.r[hh] : 1.f);
+            cf[64 + r] = __expf(f.x[hh]) * (FUSED ? f.r[2 + hh] : 1.f);
+        }
+        if (lane == 0) cf[128] = __expf(f.gc);
     }
-    if (lane == 0) cf[128] = __expf(gC);
 }
 
-__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + __expf(-x)); }
+// sigmoid of a pair of bf16 values, as a pair of bf16: (1 + tanh(x / 2)) / 2 in packed bf16
+// arithmetic (the hardware tanh approximation; x / 2 is exact)
+__device__ __forceinline__ uint32_t sigmoid_bf16x2(uint32_t x) {
+    constexpr uint32_t HALF2 = 0x3f003f00u;  // (0.5, 0.5)
+    uint32_t hx, t, sg;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(hx) : "r"(x), "r"(HALF2));
+    asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t) : "r"(hx));
+    asm("fma.rn.bf16x2 %0, %1, %2, %2;" : "=r"(sg) : "r"(t), "r"(HALF2));
+    return sg;
+}
 
 // Chain thread layout: warps 1-8, two per TMEM lane quarter (warp & 3); the first four take
 // value columns 0-31 of this CTA's 64, the other four columns 32-63.
@@ -175,9 +194,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < B_NUM; ++i)
-            mbar_init(&bar[i], (i == B_FULL0 || i == B_FULL1) ? 2 : (i >= B_XS0 && i <= B_XS3) ? 64 : 1);
+            mbar_init(&bar[i], (i == B_FULL0 || i == B_FULL1) ? 2 : 1);
         *abort_flag = 0;
         fence_mbar_init();
+        if (FUSED)  // each exchange slot expects the partner's 64 row sums of chunks 0-3 (re-armed as consumed)
+            for (int i = 0; i < 4; ++i) mbar_arrive_tx(&bar[B_XS0 + i], 64 * 4);
     }
     if (FUSED && threadIdx.x < DVB)
         reinterpret_cast<float *>(sm + OFF_MISC + M_WN)[threadIdx.x] = a.wn[j0 + threadIdx.x];
@@ -191,9 +212,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
     if (warp == 0) {
         // ================================ producer ================================
         int issued[2] = {0, 0};
+        FactorIn fin;
         for (int m = 0; m < N; ++m) {
             const int s = m & 1, t0 = m * C;
             const int ci = (int)(ci0 + m);
+            factors_fetch<KDA != 0, FUSED>(a, (size_t)ci, lane, fin);
             if (m >= 2 && !mbar_wait(&bar[B_EMPTY0 + s], ((m >> 1) - 1) & 1, abort_flag)) break;
             unsigned char *st = sm + s * STAGE;
             if (lane == 0) {
@@ -213,9 +236,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
                 tma_load_2d(st + FS_UP, &mp.Ut, j0, ci * C, &bar[B_FULL0 + s]);
                 if (OUT) tma_load_2d(st + FS_UP + 8192, &mp.P, 0, ci * C, &bar[B_FULL0 + s]);
             }
-            if (KDA) chunk_factors_kda(a.egc, (size_t)ci, cf_all + s * 132, lane);
-            else if (FUSED) chunk_factors_fused(a.gb, a.rn, (size_t)ci, cf_all + s * 132, lane);
-            else chunk_factors(a.gb, (size_t)ci, cf_all + s * 132, lane);
+            factors_store<KDA != 0, FUSED>(fin, cf_all + s * 132, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[B_FULL0 + s]);
             issued[s]++;
@@ -257,42 +278,65 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
         // o of the previous chunk is finished by lanes 64-127 while the next chunk starts: they
         // stage it in OFF_O and one of them issues its TMA store (rows past T are clipped).
         // Fused forward: y = o / sqrt(mean(o^2) + eps) w sigmoid(gate), the mean over all dv columns,
-        // half of them in the partner CTA.  The row sums of squares of chunk p go to the partner's
-        // slot p mod 4 while o(p) waits as bf16 in the buffer of p's parity; y(p) is finished one
-        // chunk later, when the partner's sums have long arrived, so that no chunk waits for the
-        // partner.  (The partner writes slot p mod 4 again for chunk p + 4, which it reaches only
-        // after this CTA has sent its sums of chunk p + 2, i.e. after y(p) is done here.)
+        // half of them in the partner CTA.  On the critical path (while the next chunk's first
+        // product runs) only o is formed: the partial row sums of its squares and z = o sigmoid(gate) w
+        // (bf16, in the buffer of the chunk's parity; lanes 0-63 turn the gate tile into
+        // sigmoid(gate) meanwhile).  In the window where lanes 0-63 form U, lanes 64-127 keep the new chunk's
+        // sigmoid(gate), add up the two column halves' sums of the chunk before and send them to
+        // the partner's slot (chunk mod 4); while the second product runs, they finish y = z / rms
+        // of the chunk two back, in place, and store it.  (The partner writes slot p mod 4 again for
+        // chunk p + 4, which it reaches only after this CTA has sent its sums of chunk p + 3, i.e.
+        // after y(p) is done here.)
         int prev_L = 0, prev_t0 = 0, prev_m = 0;
-        float prev_eg = 0.f, prev_local = 0.f;
+        float prev_eg = 0.f, inv_y = 0.f;
         uint32_t prev_buf = 0;
-        uint32_t gpk0[16], gpk1[16];  // fused, lanes 64-127: output gate logits of even / odd chunks
-        auto gate_of = [&](int j, int par) -> float {
-            const uint32_t gw = par ? gpk1[j >> 1] : gpk0[j >> 1];
-            return (j & 1) ? bf16_hi(gw) : bf16_lo(gw);
+        uint32_t sg0[16] = {}, sg1[16] = {};  // fused, lanes 64-127: sigmoid(gate) of even / odd chunks (bf16 pairs)
+        float loc_prev = 0.f;                 // fused: this CTA's full row sum of squares of the chunk before
+        auto zbuf = [&](int par) -> unsigned char * { return sm + (par ? OFF_O1 : OFF_Y); };
+        // fused: the partial row sums of squares of chunks of parity par, [2 column halves][64]
+        auto sq_tile = [&](int par) -> float * {
+            return reinterpret_cast<float *>(sm + OFF_MISC + (par ? M_SQ1 : M_SKP));
         };
-        // fused: y of chunk q from its bf16 o (buffer of q's parity) into the y staging tile
-        auto y_tile = [&](int q, float inv) {
+        // fused: the inverse RMS of chunk q's row from this CTA's sums (loc_prev) and the partner's;
+        // a wait that gives up raises the abort flag, which the next consensus acts on.  Once its
+        // own wait is over, one thread arms the slot for chunk q + 4 (the partner sends those sums
+        // only after this CTA has sent its sums of chunk q + 3, long after every wait on chunk q here).
+        auto fused_inv = [&](int q) -> float {
+            const float *xs = reinterpret_cast<const float *>(sm + OFF_MISC + M_XS);
+            mbar_wait(&bar[B_XS0 + (q & 3)], (uint32_t)(q >> 2) & 1, abort_flag);
+            if (ostore) mbar_arrive_tx(&bar[B_XS0 + (q & 3)], 64 * 4);
+            return rsqrtf((loc_prev + xs[(q & 3) * 64 + trow - 64]) * (1.f / DV) + POST_EPS);
+        };
+        // fused: this CTA's row sums of chunk q (both column halves) into loc_prev, and to the partner
+        auto send_sums = [&](int q) {
             const int r = trow - 64;
-            const float *wn = reinterpret_cast<const float *>(sm + OFF_MISC + M_WN);
-            const unsigned char *ob = sm + ((q & 1) ? OFF_O1 : OFF_O);
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                float o8[8], y8[8];
-                ld_chunk(ob, swz(r, hf * 4 + c4), o8);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int j = c4 * 8 + e;
-                    y8[e] = o8[e] * inv * wn[cb + j] * sigmoid_f((q & 1) ? gate_of(j, 1) : gate_of(j, 0));
-                }
-                st_chunk(sm + OFF_Y, swz(r, hf * 4 + c4), y8);
+            const float *sq = sq_tile(q & 1);
+            loc_prev = sq[r] + sq[64 + r];
+            if (hf == 0) {
+                const uint32_t partner = (uint32_t)half ^ 1u, slot = (uint32_t)q & 3;
+                float *xs = reinterpret_cast<float *>(sm + OFF_MISC + M_XS);
+                st_async_f32(map_to_rank(xs + slot * 64 + r, partner), loc_prev,
+                             map_to_rank(&bar[B_XS0 + slot], partner));
             }
         };
-        // fused: the inverse RMS of chunk q's row from this CTA's sums and the partner's
-        auto fused_inv = [&](int q, bool *ok) -> float {
-            const float *xs = reinterpret_cast<const float *>(sm + OFF_MISC + M_XS);
-            const bool gx = mbar_wait_cluster(&bar[B_XS0 + (q & 3)], (uint32_t)(q >> 2) & 1, abort_flag);
-            *ok = !named_sync_any(3, 128, !gx || *abort_flag != 0);  // lanes 64-127 agree
-            return rsqrtf((prev_local + xs[(q & 3) * 64 + trow - 64]) * (1.f / DV) + POST_EPS);
+        // fused: y of chunk q = z inv, in place in its buffer, then stored (lanes 64-127 together)
+        auto y_step = [&](int q, float inv) {
+            const int r = trow - 64;
+            unsigned char *zb = zbuf(q & 1);
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                float z8[8];
+                ld_chunk(zb, swz(r, hf * 4 + c4), z8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) z8[e] *= inv;
+                st_chunk(zb, swz(r, hf * 4 + c4), z8);
+            }
+            fence_proxy_async();
+            named_sync(3, 128);
+            if (ostore) {
+                tma_store_4d(&mp.y, zb, j0, h, q * C, b);
+                bulk_commit();
+            }
         };
         auto o_epilogue = [&]() {
             if (!OUT || trow < 64 || prev_L == 0 || (!FUSED && !a.has_out)) return;
@@ -302,59 +346,52 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             tmem_row32(tl + TM_D + prev_buf + 64, p);
 #pragma unroll
             for (int j = 0; j < 32; ++j) d[j] = prev_eg * d[j] + p[j];
-            float inv = 0.f, local = 0.f;
             if (FUSED) {
-                float *ssp = reinterpret_cast<float *>(sm + OFF_MISC + M_SKP);
-                float *xs = reinterpret_cast<float *>(sm + OFF_MISC + M_XS);
                 float ss = 0.f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) ss += d[j] * d[j];
-                ssp[hf * 64 + r] = ss;
-                named_sync(3, 128);
-                local = ssp[r] + ssp[64 + r];
-                if (hf == 0) {  // this chunk's sums to the partner
-                    const uint32_t partner = (uint32_t)half ^ 1u, slot = (uint32_t)prev_m & 3;
-                    st_cluster_f32(map_to_rank(xs + slot * 64 + r, partner), local);
-                    mbar_arrive_cluster(map_to_rank(&bar[B_XS0 + slot], partner));
-                }
-                if (prev_m >= 1) {  // the previous chunk's y
-                    bool fok = true;
-                    inv = fused_inv(prev_m - 1, &fok);
-                    if (!fok) return;
-                }
+                sq_tile(prev_m & 1)[hf * 64 + r] = ss;
             }
             if (ostore) bulk_wait_read_all();  // the earlier stores have read their staging tiles
             named_sync(3, 128);
-            unsigned char *ob = sm + ((FUSED && (prev_m & 1)) ? OFF_O1 : OFF_O);
-            if (FUSED || a.has_out) {
+            if (a.has_out) {
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) st_chunk(ob, swz(r, hf * 4 + c4), d + c4 * 8);
+                for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + OFF_O, swz(r, hf * 4 + c4), d + c4 * 8);
             }
-            if (FUSED && prev_m >= 1) y_tile(prev_m - 1, inv);
+            if (FUSED) {  // z = o sigmoid(gate) w
+                unsigned char *zb = zbuf(prev_m & 1);
+                const float4 *wn4 = reinterpret_cast<const float4 *>(sm + OFF_MISC + M_WN) + cb / 4;
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const float4 w0 = wn4[c4 * 2], w1 = wn4[c4 * 2 + 1];
+                    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        const uint32_t sgw = (prev_m & 1) ? sg1[c4 * 4 + x] : sg0[c4 * 4 + x];
+                        d[c4 * 8 + 2 * x] *= bf16_lo(sgw) * wv[2 * x];
+                        d[c4 * 8 + 2 * x + 1] *= bf16_hi(sgw) * wv[2 * x + 1];
+                    }
+                    st_chunk(zb, swz(r, hf * 4 + c4), d + c4 * 8);
+                }
+            }
             fence_proxy_async();
             named_sync(3, 128);
-            if (ostore) {
-                if (a.has_out) tma_store_4d(&mp.out, ob, j0, h, prev_t0, b);
-                if (FUSED && prev_m >= 1) tma_store_4d(&mp.y, sm + OFF_Y, j0, h, prev_t0 - C, b);
+            if (ostore && a.has_out) {
+                tma_store_4d(&mp.out, sm + OFF_O, j0, h, prev_t0, b);
                 bulk_commit();
             }
-            prev_local = local;
         };
-        // fused: y of the last chunk, after the loop
+        // fused: y of the last two chunks, after the loop (lanes 64-127 only)
         auto y_last = [&]() {
-            if (!FUSED || trow < 64 || prev_L == 0) return;
-            bool fok = true;
-            const float inv = fused_inv(prev_m, &fok);
-            if (!fok) return;
-            if (ostore) bulk_wait_read_all();
-            named_sync(3, 128);
-            y_tile(prev_m, inv);
-            fence_proxy_async();
-            named_sync(3, 128);
-            if (ostore) {
-                tma_store_4d(&mp.y, sm + OFF_Y, j0, h, prev_t0, b);
-                bulk_commit();
+            if (prev_m >= 1) {
+                if (ostore) bulk_wait_read_all();  // buffers of the earlier y stores
+                named_sync(3, 128);
+                y_step(prev_m - 1, fused_inv(prev_m - 1));
             }
+            named_sync(3, 128);  // both column halves' sums of the last chunk are in place
+            send_sums(prev_m);
+            const float inv = fused_inv(prev_m);
+            y_step(prev_m, inv);
         };
         for (int m = 0; m < N; ++m) {
             const int s = m & 1, t0 = m * C, L = min(C, T - t0);
@@ -386,6 +423,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             }
             pending = true;
             o_epilogue();  // previous chunk, lanes 64-127
+            if (FUSED && trow < 64) {
+                // lanes 0-63, idle while D runs: this chunk's gate logits -> sigmoid(gate), in place
+                // (bf16; row trow, this thread's 32 columns), read by lanes 64-127 after the next barrier
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    uint4 *gp = reinterpret_cast<uint4 *>(st + FS_G + swz(trow, hf * 4 + c4));
+                    const uint4 g4 = *gp;
+                    *gp = make_uint4(sigmoid_bf16x2(g4.x), sigmoid_bf16x2(g4.y), sigmoid_bf16x2(g4.z),
+                                     sigmoid_bf16x2(g4.w));
+                }
+            }
             if (!mma_done()) break;
             // ---------------- U = U~ - W S;  U and e^{gC - g} U tiles ----------------
             if (trow < 64) {
@@ -404,16 +452,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
                     for (int e = 0; e < 8; ++e) ut[e] *= rowf;
                     st_chunk(sm + OFF_UD, o, ut);
                 }
-            } else if (FUSED) {  // lanes 64-127, idle here: this chunk's gate logits, kept for its y
+            } else if (FUSED) {
+                // lanes 64-127, idle here: this chunk's sigmoid(gate), kept for its z; the inverse
+                // RMS of the chunk two back; the previous chunk's row sums (its o epilogue just ran)
+                // to the partner
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
                     const uint4 g4 = *reinterpret_cast<const uint4 *>(st + FS_G + swz(trow - 64, hf * 4 + c4));
                     if (m & 1) {
-                        gpk1[c4 * 4] = g4.x; gpk1[c4 * 4 + 1] = g4.y; gpk1[c4 * 4 + 2] = g4.z; gpk1[c4 * 4 + 3] = g4.w;
+                        sg1[c4 * 4] = g4.x; sg1[c4 * 4 + 1] = g4.y; sg1[c4 * 4 + 2] = g4.z; sg1[c4 * 4 + 3] = g4.w;
                     } else {
-                        gpk0[c4 * 4] = g4.x; gpk0[c4 * 4 + 1] = g4.y; gpk0[c4 * 4 + 2] = g4.z; gpk0[c4 * 4 + 3] = g4.w;
+                        sg0[c4 * 4] = g4.x; sg0[c4 * 4 + 1] = g4.y; sg0[c4 * 4 + 2] = g4.z; sg0[c4 * 4 + 3] = g4.w;
                     }
                 }
+                if (m >= 2) inv_y = fused_inv(m - 2);
+                if (m >= 1) send_sums(m - 1);
             }
             fence_proxy_async();
             fence_before_sync();
@@ -440,6 +493,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             }
             pending = true;
             if (KEEP && wc == 0) bulk_wait_read_1();  // the S_m store has read OFF_S
+            if (FUSED && trow >= 64 && m >= 2) y_step(m - 2, inv_y);  // while the second product runs
             if (!mma_done()) break;
             if (wc == 0) mbar_arrive(&bar[B_EMPTY0 + s]);
             // ---------------- S <- e^{gC} S + E ----------------
@@ -456,8 +510,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             if (wabort(true)) break;
             prev_L = L; prev_t0 = t0; prev_eg = rowf; prev_buf = buf; prev_m = m;
         }
-        if (*abort_flag == 0) o_epilogue();  // last chunk
-        if (*abort_flag == 0) y_last();
+        // the last chunk (all chain threads agree first: the fused epilogue waits on the partner)
+        const bool fin = !named_sync_any(2, 256, *abort_flag != 0);
+        if (fin) o_epilogue();
+        if (FUSED && fin && trow >= 64 && prev_L > 0 && !named_sync_any(3, 128, *abort_flag != 0)) y_last();
         if (wc == 0 || ostore) bulk_wait_all();
         if (*abort_flag == 0) {
             if (OUT && a.ST) {
@@ -512,9 +568,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
     if (warp == 0) {
         // ================================ producer ================================
         int issued[2] = {0, 0};
+        FactorIn fin;
         for (int m = 0; m < N; ++m) {
             const int mc = N - 1 - m, s = m & 1, t0 = mc * C;
             const int ci = (int)(ci0 + mc);
+            factors_fetch<KDA != 0, false>(a, (size_t)ci, lane, fin);
             if (m >= 2 && !mbar_wait(&bar[B_EMPTY0 + s], ((m >> 1) - 1) & 1, abort_flag)) break;
             unsigned char *st = sm + s * STAGE;
             if (lane == 0) {
@@ -535,8 +593,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
                 if (a.has_du) tma_load_4d(st + RS_DX, &mp.du, j0, h, t0, b, &bar[B_FULL0 + s]);
                 tma_load_2d(st + RS_UN, &mp.Un, j0, ci * C, &bar[B_FULL0 + s]);
             }
-            if (KDA) chunk_factors_kda(a.egc, (size_t)ci, cf_all + s * 132, lane);
-            else chunk_factors(a.gb, (size_t)ci, cf_all + s * 132, lane);
+            factors_store<KDA != 0, false>(fin, cf_all + s * 132, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[B_FULL0 + s]);
             issued[s]++;

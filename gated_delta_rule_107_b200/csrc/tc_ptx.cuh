@@ -187,34 +187,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 
 // Bounded wait as mbar_wait, with acquire at cluster scope: for a barrier that threads of another
 // CTA of the cluster arrive on (their release.cluster arrivals publish their earlier stores).
-__device__ __forceinline__ bool mbar_try_cluster(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                                  uint64_t limit_ns = 1000000000ull) {
-    if (mbar_try_cluster(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_cluster(bar, parity)) return true;
-        if ((it & 63) == 0) {
-            if (*abort) return false;
-            if (globaltimer_ns() - t0 > limit_ns) {
-                atomicOr(&g_dev_error, DEVERR_TIMEOUT);
-                *abort = 1;
-                return false;
-            }
-        }
-    }
-}
-
 // ------------------------------------------------------------------ clusters (distributed shared memory)
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -227,12 +199,12 @@ __device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
     return r;
 }
-__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-// arrive on an mbarrier of another CTA of the cluster, releasing this thread's earlier stores
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+// asynchronous store of v into another CTA's shared memory (shared::cluster address), counted as
+// 4 bytes of transaction on that CTA's mbarrier (shared::cluster address); the sender does not wait
+__device__ __forceinline__ void st_async_f32(uint32_t addr, float v, uint32_t mbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];" ::"r"(addr), "f"(v),
+                 "r"(mbar)
+                 : "memory");
 }
 // every thread of every CTA of the cluster (warp-uniform)
 __device__ __forceinline__ void cluster_sync() {
