@@ -424,12 +424,11 @@ struct KdaArgs {
     float *egc;
     int *kwide;
     float *Dx;
-    float *G;  // optional: g itself, fp32 [chunks][64][128]
+    float *G;  // optional: g itself, fp32 [chunks][64][128] (written for the marked chunks only)
     int T, H, N;
 };
 
-__device__ __forceinline__ void ld8_bf16(const __nv_bfloat16 *p, float *v) {
-    const uint4 x = *reinterpret_cast<const uint4 *>(p);
+__device__ __forceinline__ void unpack8_bf16(const uint4 x, float *v) {
     const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -453,11 +452,21 @@ __global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
     const int t0 = n * C, L = min(C, a.T - t0);
     const size_t ci = ((size_t)b * a.H + h) * a.N + n;
     auto at = [&](int r) { return (((size_t)b * a.T + t0 + r) * a.H + h) * DK + c0; };
+    // every input row of this thread at once (24 16-byte loads in flight; rows past T read as 0)
+    uint4 ar[8], kw[8], qw[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        const bool in = 8 * tg + r < L;
+        ar[r] = in ? __ldg(reinterpret_cast<const uint4 *>(a.alpha + at(8 * tg + r))) : z;
+        kw[r] = in ? __ldg(reinterpret_cast<const uint4 *>(a.k + at(8 * tg + r))) : z;
+        qw[r] = in ? __ldg(reinterpret_cast<const uint4 *>(a.q + at(8 * tg + r))) : z;
+    }
     float g[8][8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-        float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (8 * tg + r < L) ld8_bf16(a.alpha + at(8 * tg + r), x);
+        float x[8];
+        unpack8_bf16(ar[r], x);
 #pragma unroll
         for (int j = 0; j < 8; ++j) g[r][j] = (r ? g[r - 1][j] : 0.f) + x[j];
     }
@@ -474,14 +483,6 @@ __global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
         if (tg == 7) gend[c0 + j] = g[7][j];           // token C - 1, the last
     }
     __syncthreads();
-    if (a.G) {
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            float *dst = a.G + (ci * C + 8 * tg + r) * DK + c0;
-            *reinterpret_cast<float4 *>(dst) = make_float4(g[r][0], g[r][1], g[r][2], g[r][3]);
-            *reinterpret_cast<float4 *>(dst + 4) = make_float4(g[r][4], g[r][5], g[r][6], g[r][7]);
-        }
-    }
     float gb[8], gC[8];  // g at the first token of this thread's block, and at the chunk's last
     bool wide = false;
 #pragma unroll
@@ -494,11 +495,9 @@ __global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
         const int tr = 8 * tg + r;
-        float kr[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, qr[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (tr < L) {
-            ld8_bf16(a.k + at(tr), kr);
-            ld8_bf16(a.q + at(tr), qr);
-        }
+        float kr[8], qr[8];
+        unpack8_bf16(kw[r], kr);
+        unpack8_bf16(qw[r], qr);
         float o1[8], o2[8], o4[8], o5[8], o6[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -533,6 +532,14 @@ __global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
     }
     wide = __syncthreads_or(wide);
     if (threadIdx.x == 0) a.kwide[ci] = wide ? 1 : 0;
+    if (wide && a.G) {  // g itself, for the CUDA-core gradient kernel that takes the marked chunks
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            float *dst = a.G + (ci * C + 8 * tg + r) * DK + c0;
+            *reinterpret_cast<float4 *>(dst) = make_float4(g[r][0], g[r][1], g[r][2], g[r][3]);
+            *reinterpret_cast<float4 *>(dst + 4) = make_float4(g[r][4], g[r][5], g[r][6], g[r][7]);
+        }
+    }
 }
 
 // The exact in-block sums of the chunks k_kda_gates marked (one CTA of 128 threads per chunk;
