@@ -30,8 +30,10 @@
 //   C  dA' = dB [W | U~]^T and its transpose, [dO ; U][dO ; U]^T (dP and dP^T in one product);
 //      dM, dP, dM^T, dP^T tiles, the dbeta part of A;  the gate-scaled sections Km, Kp, Qp
 //   D  X^T, Yv^T, Z^T (block by block, N = 16);  the final per-channel epilogue
-// Sums over the channels of one token (dbeta's) reduce 32 tokens across a warp's 32 lanes in 31
-// shuffles (recursive halving), then over the four warps of a lane quarter through shared memory.
+// Sums over the channels of one token (dbeta's) reduce 4 tokens at a time across a warp's 32 lanes
+// (6 shuffles), then over the four warps of a lane quarter through shared memory.  The per-token
+// loops are rolled over groups of 4 or 8 tokens (TMEM loads of 4 or 8 columns), so that every
+// phase runs from a small loop body instead of long straight-line code.
 // Every wait is bounded (~1 s); an expired wait raises the device error word.
 #include "tc_host.cuh"
 #include "tc_path.cuh"
@@ -103,19 +105,20 @@ __device__ __forceinline__ uint32_t el_off(int row, int c, uint32_t panel) {
 __device__ __forceinline__ float ld_bf(const unsigned char *base, uint32_t off) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(base + off));
 }
-// x[t] (t < 32) summed over the warp's lanes, by recursive halving: each step keeps half of the
-// remaining tokens and adds the partner lane's copy of them; afterwards x[0] of lane l is token l's sum
-__device__ __forceinline__ float warp_sum32(float (&x)[32], int lane) {
+// x[t] (t < 4) summed over the warp's lanes: two halving steps, then a plain sum over the
+// remaining lane bits; afterwards every lane l holds the sum of token l / 8
+__device__ __forceinline__ float warp_sum4(float (&x)[4], int lane) {
+    const bool u16 = (lane & 16) != 0, u8 = (lane & 8) != 0;
 #pragma unroll
-    for (int s = 16; s >= 1; s >>= 1) {
-        const bool up = (lane & s) != 0;
-#pragma unroll
-        for (int i = 0; i < s; ++i) {
-            const float send = up ? x[i] : x[i + s], keep = up ? x[i + s] : x[i];
-            x[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
-        }
+    for (int i = 0; i < 2; ++i) {
+        const float send = u16 ? x[i] : x[i + 2], keep = u16 ? x[i + 2] : x[i];
+        x[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
     }
-    return x[0];
+    float v = (u8 ? x[1] : x[0]) + __shfl_xor_sync(0xffffffffu, u8 ? x[0] : x[1], 8);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    return v;
 }
 // 8 consecutive floats of a [64][128] fp32 tile (c0 a multiple of 8).  The two 16-byte halves are
 // read in an order that depends on bit 2 of c0 / 8, so that the eight threads of a quarter warp
@@ -199,7 +202,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
     // ======================= phase A products =======================
     if (ok && tid == 0) {
         const uint32_t id0 = idesc_bf16(128, 128, 0, 0), id1 = idesc_bf16(128, 64, 0, 0);
-#pragma unroll
+#pragma unroll 1
         for (int k = 0; k < 8; ++k) {  // K = dv in steps of 16
             const uint32_t ka = (k >> 2) * 16384 + (k & 3) * 32;
             mma_bf16(tbase + TM_QD, sdesc(u32(R_S) + ka, 16, 1024), sdesc(u32(R_OU) + ka, 16, 1024), id0, k > 0);
@@ -266,7 +269,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
         // dB_k^T = dWm^T T (A K-major [c][r]; B = T [r][i] MN-major)
         // dB_v^T = dU^T T  (A = dU [r][j] MN-major: the two 64-column panels 16K apart in [dO ; dU])
         const uint32_t idk = idesc_bf16(128, 64, 0, 1), idv = idesc_bf16(128, 64, 1, 1);
-#pragma unroll
+#pragma unroll 1
         for (int k = 0; k < 4; ++k) {
             mma_bf16(tbase + TM_DBK, sdesc(u32(R_DWM) + k * 32, 16, 1024), sdesc(u32(R_T) + k * 2048, 8192, 1024), idk,
                      k > 0);
@@ -277,26 +280,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
     }
     if (ok) ok = wait_mma(mbar_wait(&bar[1], 0, abort_flag));  // the products; M, W, U~, v
     if (ok) {
-        // the bf16 tiles dB_k^T [c][i] and dB_v^T [j][i] (this half's 32 tokens), dv, and v . dB_v
-        float v[32];
-        tmem_ld16(tl + TM_DBK + r0, v);
-        tmem_ld16(tl + TM_DBK + 16 + r0, v + 16);
-        wait_ld();
+        // the bf16 tiles dB_k^T [c][i] and dB_v^T [j][i] (this half's 32 tokens), dv, and v . dB_v,
+        // eight tokens at a time
+#pragma unroll 1
+        for (int k8 = 0; k8 < 4; ++k8) {
+            const int rr = r0 + 8 * k8;
+            float bk[8], bv[8];
+            tmem_ld8(tl + TM_DBK + rr, bk);
+            tmem_ld8(tl + TM_DBV + rr, bv);
+            wait_ld();
+            st_chunk(sm + R_DBK, swz(c, rr >> 3), bk);
+            st_chunk(sm + R_DBV, swz(c, rr >> 3), bv);
+            float s0[4], s1[4];
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) st_chunk(sm + R_DBK, swz(c, 4 * hf + ch), v + ch * 8);
-        tmem_ld16(tl + TM_DBV + r0, v);
-        tmem_ld16(tl + TM_DBV + 16 + r0, v + 16);
-        wait_ld();
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) st_chunk(sm + R_DBV, swz(c, 4 * hf + ch), v + ch * 8);
-        float sv[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            const int r = r0 + e;
-            sv[e] = ld_bf(sm + R_V, el_off(r, c, 8192)) * v[e];
-            if (r < L) a.dv[trow_g(r) * DV + c] = __float2bfloat16_rn(betas[r] * v[e]);
+            for (int e = 0; e < 8; ++e) {
+                const int r = rr + e;
+                const float sv = ld_bf(sm + R_V, el_off(r, c, 8192)) * bv[e];
+                if (e < 4) s0[e] = sv;
+                else s1[e - 4] = sv;
+                if (r < L) a.dv[trow_g(r) * DV + c] = __float2bfloat16_rn(betas[r] * bv[e]);
+            }
+            const float t0s = warp_sum4(s0, lane), t1s = warp_sum4(s1, lane);
+            if ((lane & 7) == 0) {
+                red[(4 + q4) * 64 + rr + (lane >> 3)] = t0s;
+                red[(4 + q4) * 64 + rr + 4 + (lane >> 3)] = t1s;
+            }
         }
-        red[(4 + q4) * 64 + r0 + lane] = warp_sum32(sv, lane);
     }
     fence_proxy_async();
     fence_before_sync();
@@ -307,21 +316,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
         // dA'[r][i] = dB_k[r] . W[i] + dB_v[r] . U~[i]: A = dB^T tiles read MN-major (rows 64-127 of
         // the M = 128 product are discarded), B = W, U~ K-major
         const uint32_t ida = idesc_bf16(128, 64, 1, 0), idt = idesc_bf16(128, 64, 0, 1), id5 = idesc_bf16(128, 128, 0, 0);
-#pragma unroll
+#pragma unroll 1
         for (int k = 0; k < 16; ++k) {
             const uint32_t at = (k < 8 ? u32(R_DBK) : u32(R_DBV)) + (k & 7) * 2048;
             const uint32_t bw = (k < 8 ? u32(R_W) : u32(R_UT)) + ((k & 7) >> 2) * 8192 + (k & 3) * 32;
             mma_bf16(tbase + TM_X, sdesc(at, 8192, 1024), sdesc(bw, 16, 1024), ida, k > 0);
         }
         // dA'^T[i][r]: A = W, U~ K-major, B = dB^T tiles MN-major
-#pragma unroll
+#pragma unroll 1
         for (int k = 0; k < 16; ++k) {
             const uint32_t aw = (k < 8 ? u32(R_W) : u32(R_UT)) + ((k & 7) >> 2) * 8192 + (k & 3) * 32;
             const uint32_t bt = (k < 8 ? u32(R_DBK) : u32(R_DBV)) + (k & 7) * 2048;
             mma_bf16(tbase + TM_YV, sdesc(aw, 16, 1024), sdesc(bt, 8192, 1024), idt, k > 0);
         }
         // [dO ; U] [dO ; U]^T: dP = dO U^T at lanes 0-63 / columns 64-127, dP^T at lanes 64-127 / 0-63
-#pragma unroll
+#pragma unroll 1
         for (int k = 0; k < 8; ++k) {
             const uint32_t ka = (k >> 2) * 16384 + (k & 3) * 32;
             mma_bf16(tbase + TM_D5, sdesc(u32(R_OV) + ka, 16, 1024), sdesc(u32(R_OV) + ka, 16, 1024), id5, k > 0);
@@ -333,24 +342,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
     //   lanes 0-63 (quarters 0, 1): half 0 takes dA' (-> dM, dbeta_A), half 1 takes dP, and each
     //   half takes 32 columns of dA'^T (-> dM^T);  lanes 64-127: each half takes 32 columns of dP^T
     if (ok) {
-        float x[64];
         const int rl = (warp & 1) * 32 + lane;  // the product's row (r, or i for the transposes)
         if (q4 < 2) {
             if (hf == 0) {
                 const int r = rl;  // dA'[r][i] -> dM[r][i] = -beta_r dA' (i < r), dbeta_A
-                tmem_ld16(tl + TM_X, x); tmem_ld16(tl + TM_X + 16, x + 16);
-                tmem_ld16(tl + TM_X + 32, x + 32); tmem_ld16(tl + TM_X + 48, x + 48);
-                wait_ld();
                 float db = 0.f;
                 const float br = betas[r];
-#pragma unroll
+#pragma unroll 1
                 for (int ch = 0; ch < 8; ++ch) {
-                    float m8[8], w8[8];
+                    float x8[8], m8[8], w8[8];
+                    tmem_ld8(tl + TM_X + 8 * ch, x8);
+                    wait_ld();
                     ld_chunk(sm + R_M, swz(r, ch), m8);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const int i = ch * 8 + e;
-                        const float d = i < r ? -x[i] : 0.f;
+                        const float d = ch * 8 + e < r ? -x8[e] : 0.f;
                         db += d * m8[e];
                         w8[e] = br * d;
                     }
@@ -359,31 +365,39 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
                 dba[r] = db;
             } else {
                 const int r = rl;  // dP[r][i] (i <= r)
-                tmem_ld16(tl + TM_D5 + 64, x); tmem_ld16(tl + TM_D5 + 80, x + 16);
-                tmem_ld16(tl + TM_D5 + 96, x + 32); tmem_ld16(tl + TM_D5 + 112, x + 48);
-                wait_ld();
+#pragma unroll 1
+                for (int ch = 0; ch < 8; ++ch) {
+                    float x8[8];
+                    tmem_ld8(tl + TM_D5 + 64 + 8 * ch, x8);
+                    wait_ld();
 #pragma unroll
-                for (int i = 0; i < 64; ++i) x[i] = i <= r ? x[i] : 0.f;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) st_chunk(sm + R_DP, swz(r, ch), x + ch * 8);
+                    for (int e = 0; e < 8; ++e) x8[e] = ch * 8 + e <= r ? x8[e] : 0.f;
+                    st_chunk(sm + R_DP, swz(r, ch), x8);
+                }
             }
             const int i = rl;  // dA'^T[i][r] -> dM^T[i][r] = -beta_r dA'^T (r > i), r in this half
-            tmem_ld16(tl + TM_YV + r0, x);
-            tmem_ld16(tl + TM_YV + 16 + r0, x + 16);
-            wait_ld();
+#pragma unroll 1
+            for (int k8 = 0; k8 < 4; ++k8) {
+                const int rr = r0 + 8 * k8;
+                float x8[8];
+                tmem_ld8(tl + TM_YV + rr, x8);
+                wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] = r0 + e > i ? -betas[r0 + e] * x[e] : 0.f;
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) st_chunk(sm + R_DMT, swz(i, 4 * hf + ch), x + ch * 8);
+                for (int e = 0; e < 8; ++e) x8[e] = rr + e > i ? -betas[rr + e] * x8[e] : 0.f;
+                st_chunk(sm + R_DMT, swz(i, rr >> 3), x8);
+            }
         } else {
             const int i = rl;  // dP^T[i][r] (r >= i), r in this half
-            tmem_ld16(tl + TM_D5 + r0, x);
-            tmem_ld16(tl + TM_D5 + 16 + r0, x + 16);
-            wait_ld();
+#pragma unroll 1
+            for (int k8 = 0; k8 < 4; ++k8) {
+                const int rr = r0 + 8 * k8;
+                float x8[8];
+                tmem_ld8(tl + TM_D5 + rr, x8);
+                wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] = r0 + e >= i ? x[e] : 0.f;
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) st_chunk(sm + R_DPT, swz(i, 4 * hf + ch), x + ch * 8);
+                for (int e = 0; e < 8; ++e) x8[e] = rr + e >= i ? x8[e] : 0.f;
+                st_chunk(sm + R_DPT, swz(i, rr >> 3), x8);
+            }
         }
     }
     ok = consensus(ok);  // M, W, U~ and the dB tiles are read: the sections may take their space
@@ -430,14 +444,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
     if (ok && tid == 0) {
         fence_after_sync();
         const uint32_t id = idesc_bf16(128, 16, 1, 0);
+#pragma unroll 1
         for (int R = 0; R < 4; ++R) {
+#pragma unroll 1
             for (int kk = 0; kk <= R; ++kk) {  // tokens i of the blocks up to R
                 const uint64_t am = sdesc(u32(R_KM) + (uint32_t)(km_sec(R) + 16 * kk) * 128, SEC_PANEL, 1024);
                 mma_bf16(tbase + TM_X + 16 * R, am, sdesc(u32(R_DP) + 2048 * R + kk * 32, 16, 1024), id, kk > 0);
                 mma_bf16(tbase + TM_YV + 16 * R, am, sdesc(u32(R_DM) + 2048 * R + kk * 32, 16, 1024), id, kk > 0);
             }
         }
+#pragma unroll 1
         for (int I = 0; I < 4; ++I) {
+#pragma unroll 1
             for (int kk = I; kk < 4; ++kk) {  // tokens r of the blocks from I on
                 const uint32_t ro = (uint32_t)(kp_sec(I) + 16 * (kk - I)) * 128;
                 mma_bf16(tbase + TM_Z + 16 * I, sdesc(u32(R_KP) + ro, SEC_PANEL, 1024),
@@ -449,26 +467,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
         commit();
     }
     if (ok) ok = wait_mma(true);
-    // ======================= final epilogue: thread (c, half): tokens r0 .. r0 + 31 =======================
+    // ======================= final epilogue: thread (c, half): tokens r0 .. r0 + 31, four at a time
     const float gL = G[(C - 1) * DK + c];
-    float dgr[32];
+    float *DG = reinterpret_cast<float *>(sm + R_KM);  // [64][128] dg (the sections are read by now)
     if (ok) {
-        float dgc = 0.f, sbk[32];
-#pragma unroll
-        for (int rh = 0; rh < 2; ++rh) {
-            const int rb = 2 * hf + rh;
-            float qd[16], tm[16], bk[16], xx[16], yv[16], zz[16];
-            tmem_ld16(tl + TM_QD + 16 * rb, qd);
-            tmem_ld16(tl + TM_TM + 16 * rb, tm);
-            tmem_ld16(tl + TM_DBK + 16 * rb, bk);
-            tmem_ld16(tl + TM_X + 16 * rb, xx);
-            tmem_ld16(tl + TM_YV + 16 * rb, yv);
-            tmem_ld16(tl + TM_Z + 16 * rb, zz);
+        float dgc = 0.f, tot = 0.f;
+#pragma unroll 1
+        for (int g4 = 0; g4 < 8; ++g4) {
+            const int rr = r0 + 4 * g4, rb = rr >> 4;
+            float qd[4], tm[4], bk[4], xx[4], yv[4], zz[4];
+            tmem_ld4(tl + TM_QD + rr, qd);
+            tmem_ld4(tl + TM_TM + rr, tm);
+            tmem_ld4(tl + TM_DBK + rr, bk);
+            tmem_ld4(tl + TM_X + rr, xx);
+            tmem_ld4(tl + TM_YV + rr, yv);
+            tmem_ld4(tl + TM_Z + rr, zz);
             wait_ld();
             const float gb = G[16 * rb * DK + c], ge = G[(16 * rb + 15) * DK + c];
+            float sbk[4];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int r = 16 * rb + e, idx = 16 * rh + e;
+            for (int e = 0; e < 4; ++e) {
+                const int r = rr + e;
                 const float g = G[r * DK + c], br = betas[r];
                 const float qv = ld_bf(sm + R_Q, el_off(r, c, 8192)), kv = ld_bf(sm + R_K, el_off(r, c, 8192));
                 const float gam = __expf(g), eb = __expf(gL - g);
@@ -477,24 +496,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
                 const float dq = gam * qd[e] + X;
                 const float t = eb * tm[e], sb = br * gam * bk[e];
                 const float dk = Yv + Z + sb + t;
-                dgr[idx] = qv * dq + kv * (Yv - Z + sb - t);
+                const float dg = qv * dq + kv * (Yv - Z + sb - t);
+                DG[r * DK + c] = dg;
+                tot += dg;
                 dgc += kv * t;
-                sbk[idx] = gam * kv * bk[e];
+                sbk[e] = gam * kv * bk[e];
                 if (r < L) {
                     const size_t o = trow_g(r) * DK + c;
                     a.dq[o] = __float2bfloat16_rn(dq);
                     a.dk[o] = __float2bfloat16_rn(dk);
                 }
             }
+            const float s4 = warp_sum4(sbk, lane);
+            if ((lane & 7) == 0) red[q4 * 64 + rr + (lane >> 3)] = s4;
         }
-        red[q4 * 64 + r0 + lane] = warp_sum32(sbk, lane);
         xch[(hf * 3 + 0) * 128 + c] = dgc;
-        if (hf) {
-            float tot = 0.f;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) tot += dgr[e];
-            xch[(1 * 3 + 2) * 128 + c] = tot;
-        }
+        if (hf) xch[(1 * 3 + 2) * 128 + c] = tot;
     }
     ok = consensus(ok);
     if (ok) {
@@ -502,9 +519,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
         // reverse cumulative sum; the lower half starts from the upper half's total
         float run = xch[0 * 128 + c] + xch[3 * 128 + c] + __expf(gL) * (xch[1 * 128 + c] + xch[4 * 128 + c]);
         if (!hf) run += xch[5 * 128 + c];
-#pragma unroll
+#pragma unroll 4
         for (int e = 31; e >= 0; --e) {
-            run += dgr[e];
+            run += DG[(r0 + e) * DK + c];
             if (r0 + e < L) a.dalpha[trow_g(r0 + e) * DK + c] = __float2bfloat16_rn(run);
         }
         if (tid < L) {

@@ -109,6 +109,24 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *r) {
     for (int i = 0; i < 16; ++i) r[i] = __uint_as_float(v[i]);
 }
 
+// the same for 4 and 8 consecutive columns
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, float *r) {
+    uint32_t v[4];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                 : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) r[i] = __uint_as_float(v[i]);
+}
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float *r) {
+    uint32_t v[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+                 : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r[i] = __uint_as_float(v[i]);
+}
+
 // ------------------------------------------------------------------ proxies / fences
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy (MMA, TMA).
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
