@@ -519,10 +519,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
         // reverse cumulative sum; the lower half starts from the upper half's total
         float run = xch[0 * 128 + c] + xch[3 * 128 + c] + __expf(gL) * (xch[1 * 128 + c] + xch[4 * 128 + c]);
         if (!hf) run += xch[5 * 128 + c];
+        const size_t rstep = (size_t)H * DK;  // one token further in [B, T, H, 128]
+        __nv_bfloat16 *da = a.dalpha + trow_g(r0 + 31) * DK + c;
 #pragma unroll 4
-        for (int e = 31; e >= 0; --e) {
+        for (int e = 31; e >= 0; --e, da -= rstep) {
             run += DG[(r0 + e) * DK + c];
-            if (r0 + e < L) a.dalpha[trow_g(r0 + e) * DK + c] = __float2bfloat16_rn(run);
+            if (r0 + e < L) *da = __float2bfloat16_rn(run);
         }
         if (tid < L) {
             float s = dba[tid];

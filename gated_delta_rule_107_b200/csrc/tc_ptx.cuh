@@ -203,14 +203,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
-// Bounded wait as mbar_wait, with acquire at cluster scope: for a barrier that threads of another
-// CTA of the cluster arrive on (their release.cluster arrivals publish their earlier stores).
 // ------------------------------------------------------------------ clusters (distributed shared memory)
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
 // the shared::cluster address of this CTA's shared-memory object p in the CTA of the given rank
 __device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
     uint32_t r;
@@ -247,21 +240,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         "[%4];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
         : "memory");
-}
-
-// L2 prefetch of a 2-D / 4-D tiled box (no shared memory, no completion to wait for);
-// boxes outside the tensor fetch nothing.
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *map, int c0, int c1) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(c0), "r"(c1)
-                 : "memory");
-}
-__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3) {
-    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-                 : "memory");
 }
 
 // Plain (untiled) bulk copy global -> shared, completion counted on `bar`.  Both addresses

@@ -11,11 +11,6 @@ __device__ __forceinline__ float bf(const void *p, size_t i) {
     return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
 }
 
-// element (r, c) of a token-major tile of 64-row panels (panel stride 8K)
-__device__ __forceinline__ uint32_t tok_off(int r, int c) {
-    return (uint32_t)((c >> 6) * 8192) + swz(r, (c & 63) >> 3) + (c & 7) * 2;
-}
-
 __device__ __forceinline__ void st_chunk(unsigned char *base, uint32_t off, const float *v) {
     uint4 w;
     w.x = pack_bf16(v[0], v[1]);
@@ -29,29 +24,6 @@ __device__ __forceinline__ void ld_chunk(const unsigned char *base, uint32_t off
     const uint4 w = *reinterpret_cast<const uint4 *>(base + off);
     v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
     v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
-}
-
-// 8 values as bf16 at element offset elem_off (a multiple of 8) of a bf16 array in global memory
-__device__ __forceinline__ void st8_global(void *base, size_t elem_off, const float *v) {
-    uint4 w;
-    w.x = pack_bf16(v[0], v[1]);
-    w.y = pack_bf16(v[2], v[3]);
-    w.z = pack_bf16(v[4], v[5]);
-    w.w = pack_bf16(v[6], v[7]);
-    *reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(base) + elem_off) = w;
-}
-
-// 8 bf16 values at p (16-byte aligned) in global memory, widened
-__device__ __forceinline__ void ld8_global(const __nv_bfloat16 *p, float *v) {
-    const uint4 w = *reinterpret_cast<const uint4 *>(p);
-    v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
-    v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
-}
-
-// 64 values as bf16 at element offset elem_off (a multiple of 8) of a bf16 array in global memory
-__device__ __forceinline__ void st_row_global(void *base, size_t elem_off, const float *v) {
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch) st8_global(base, elem_off + ch * 8, v + ch * 8);
 }
 
 // 64 fp32 columns of this thread's TMEM lane
