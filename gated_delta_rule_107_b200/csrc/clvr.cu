@@ -37,7 +37,8 @@ constexpr uint32_t OFF_A = 0, OFF_B = STAGES * A_BYTES, OFF_C = OFF_B + STAGES *
 constexpr uint32_t C_BYTES = BM * BN * 2;  // bf16 output tile: 4 panels [128 rows][64 columns]
 constexpr uint32_t OFF_MISC = OFF_C + C_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 256;
-enum { B_FULL = 0, B_EMPTY = STAGES, B_ACCF = 2 * STAGES, B_ACCE = B_ACCF + 2, B_CF = B_ACCE + 2, B_NUM };
+// B_CF + p: panel p (64 columns) of a tile's residual has landed in the output tile
+enum { B_FULL = 0, B_EMPTY = STAGES, B_ACCF = 2 * STAGES, B_ACCE = B_ACCF + 2, B_CF = B_ACCE + 2, B_NUM = B_CF + 4 };
 constexpr uint32_t M_TMEM = 8 * B_NUM, M_ABORT = M_TMEM + 4;
 static_assert(M_ABORT + 4 <= 256, "misc overflow");
 constexpr int NTHREADS = 192;  // warp 0 TMA, warp 1 MMA and TMEM owner, warps 2-5 epilogue
@@ -69,6 +70,12 @@ __device__ __forceinline__ void load_operand(unsigned char *dst, const CUtensorM
     } else {
         for (int p = 0; p < rows / 64; ++p) tma_load_2d(dst + p * 8192, map, r0 + 64 * p, k0, bar);
     }
+}
+
+// at most N of this thread's committed bulk groups still reading shared memory (N a constant 0..7)
+template <int N>
+__device__ __forceinline__ void bulk_wait_read_n() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 
 // Shared-memory descriptor of K step kk (16 elements) of an operand tile laid out as above
@@ -175,80 +182,105 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_gemm_tc(const __grid_constant__
         }
     } else {
         // ================================ epilogue ================================
+        // The output tile is staged as four 64-column panels, each stored (one bulk group per panel)
+        // as soon as it is formed.  With a residual, the leader loads the next tile's residual panel
+        // p as soon as panel p's store has read the staging tile, so that the load is in flight
+        // while this CTA's next accumulator fills.
         const int q4 = warp & 3, r = q4 * 32 + lane;  // TMEM lane = output row of the tile
         const uint32_t tl = tbase + ((uint32_t)(q4 * 32) << 16);
         const bool leader = warp == 2 && lane == 0;   // issues the residual loads and the stores
-        int it = 0, cloads = 0;
+        const bool staged = a.d32 == nullptr, resid = staged && a.has_c;
+        auto load_resid_panel = [&](int t, int p) {
+            int s2, mb2, nb2;
+            tile_of(t, s2, mb2, nb2);
+            mbar_arrive_tx(&bar[B_CF + p], 16384);
+            tma_load_2d(sm + OFF_C + p * 16384, &mp.c, nb2 * BN + 64 * p, mb2 * BM, &bar[B_CF + p]);
+        };
+        if (resid && leader && (int)blockIdx.x < tiles)
+            for (int p = 0; p < 4; ++p) load_resid_panel(blockIdx.x, p);
+        int it = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
             int s, mb, nb;
             tile_of(t, s, mb, nb);
             const int acc = it & 1;
             const bool zero = kblocks_of(s) == 0;
-            if (a.d32 == nullptr) {
-                // the output tile is free once the previous tile's store has read it; then the residual
-                if (leader) {
-                    bulk_wait_read_all();
-                    if (a.has_c) {
-                        mbar_arrive_tx(&bar[B_CF], C_BYTES);
-                        for (int p = 0; p < 4; ++p)
-                            tma_load_2d(sm + OFF_C + p * 16384, &mp.c, nb * BN + 64 * p, mb * BM, &bar[B_CF]);
-                    }
-                }
-                named_sync(1, 128);
-            }
             bool ok = mbar_wait(&bar[B_ACCF + acc], (it >> 1) & 1, abort_flag);
-            if (ok && a.has_c && a.d32 == nullptr) ok = mbar_wait(&bar[B_CF], cloads & 1, abort_flag);
-            if (a.has_c && a.d32 == nullptr) cloads++;
             fence_after_sync();
             if (named_sync_any(1, 128, !ok || *abort_flag != 0)) break;
             const int grow = mb * BM + r;
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                float v[32];
-                tmem_ld16(tl + acc * BN + c0, v);
-                tmem_ld16(tl + acc * BN + c0 + 16, v + 16);
-                wait_ld();
-                if (zero) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = 0.f;
+            bool fail = false;
+            for (int p = 0; p < 4; ++p) {
+                if (staged) {
+                    // the staging panel holds this tile's residual, or is free: the store of the
+                    // same panel one tile back has read it (the leader waited before reloading it)
+                    bool pok = true;
+                    if (resid) pok = mbar_wait(&bar[B_CF + p], (uint32_t)it & 1, abort_flag);
+                    else if (leader) bulk_wait_read_n<3>();  // no residual: panel p's previous store is done
+                    if (named_sync_any(1, 128, !pok || *abort_flag != 0)) {
+                        fail = true;
+                        break;
+                    }
                 }
-                if (a.d32) {
-                    const int gc = nb * BN + c0;
-                    if (grow < a.M) {
-                        float *dst = a.d32 + (size_t)s * a.slice_elems + (size_t)grow * a.N + gc;
-                        if (gc + 32 <= a.N) {
+                for (int c0 = 64 * p; c0 < 64 * p + 64; c0 += 32) {
+                    float v[32];
+                    tmem_ld16(tl + acc * BN + c0, v);
+                    tmem_ld16(tl + acc * BN + c0 + 16, v + 16);
+                    wait_ld();
+                    if (zero) {
 #pragma unroll
-                            for (int j = 0; j < 32; j += 4)
-                                *reinterpret_cast<float4 *>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-                        } else {
-                            for (int j = 0; j < 32 && gc + j < a.N; ++j) dst[j] = v[j];
+                        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+                    }
+                    if (!staged) {
+                        const int gc = nb * BN + c0;
+                        if (grow < a.M) {
+                            float *dst = a.d32 + (size_t)s * a.slice_elems + (size_t)grow * a.N + gc;
+                            if (gc + 32 <= a.N) {
+#pragma unroll
+                                for (int j = 0; j < 32; j += 4)
+                                    *reinterpret_cast<float4 *>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                            } else {
+                                for (int j = 0; j < 32 && gc + j < a.N; ++j) dst[j] = v[j];
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int ch = 0; ch < 4; ++ch) {
+                            const uint32_t o = (uint32_t)p * 16384 + swz(r, ((c0 & 63) >> 3) + ch);
+                            if (resid) {
+                                float h8[8];
+                                ld_chunk(sm + OFF_C, o, h8);
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) v[ch * 8 + e] += h8[e];
+                            }
+                            st_chunk(sm + OFF_C, o, v + ch * 8);
                         }
                     }
-                } else {
-                    const int p = c0 >> 6;
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        const uint32_t o = (uint32_t)p * 16384 + swz(r, ((c0 & 63) >> 3) + ch);
-                        if (a.has_c) {
-                            float h8[8];
-                            ld_chunk(sm + OFF_C, o, h8);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) v[ch * 8 + e] += h8[e];
-                        }
-                        st_chunk(sm + OFF_C, o, v + ch * 8);
+                }
+                if (p == 3) {  // this accumulator is drained (each epilogue warp arrives once)
+                    fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bar[B_ACCE + acc]);
+                }
+                if (staged) {
+                    fence_proxy_async();
+                    named_sync(1, 128);
+                    if (leader) {
+                        tma_store_2d(&mp.d, sm + OFF_C + p * 16384, nb * BN + 64 * p, mb * BM);
+                        bulk_commit();
                     }
                 }
             }
-            // this accumulator is drained (each epilogue warp arrives once)
-            fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[B_ACCE + acc]);
-            if (a.d32 == nullptr) {
-                fence_proxy_async();
-                named_sync(1, 128);
-                if (leader) {
-                    for (int p = 0; p < 4; ++p) tma_store_2d(&mp.d, sm + OFF_C + p * 16384, nb * BN + 64 * p, mb * BM);
-                    bulk_commit();
-                }
+            if (fail) break;
+            // the next tile's residual panels, each once this tile's store of it has read the panel
+            if (resid && leader && t + (int)gridDim.x < tiles) {
+                bulk_wait_read_n<3>();
+                load_resid_panel(t + gridDim.x, 0);
+                bulk_wait_read_n<2>();
+                load_resid_panel(t + gridDim.x, 1);
+                bulk_wait_read_n<1>();
+                load_resid_panel(t + gridDim.x, 2);
+                bulk_wait_read_n<0>();
+                load_resid_panel(t + gridDim.x, 3);
             }
         }
         if (leader) bulk_wait_all();
