@@ -80,7 +80,23 @@ struct Args {
     const int *kwide;               // KDA: [chunks] in-block sums from Dx
     const float *Dx;                // KDA: [chunks][2][64][16]
     int B, T, H, N;
+    int wave;                       // CTAs resident at once (2 per SM): the L2 prefetch distance
 };
+
+// L2 prefetch of a tiled box (no shared memory, nothing to wait for; a box outside the tensor
+// fetches nothing)
+__device__ __forceinline__ void l2_prefetch_2d(const CUtensorMap *map, int c0, int c1) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void l2_prefetch_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
 
 // first column of block R's section of the KDA product (16 R (R + 1) / 2)
 __host__ __device__ constexpr uint32_t kda_sec(int R) { return (uint32_t)(8 * R * (R + 1)); }
@@ -132,6 +148,28 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
                 tma_load_4d(sm + OFF_KQ + p * 16384 + 8192, &mp.q, 64 * p, h, t0, b, &bar[0]);
             }
             tma_load_4d(sm + OFF_V + p * 8192, &mp.v, 64 * p, h, t0, b, &bar[0]);
+        }
+        // the inputs of the CTA that starts one wave later (CTAs are dispatched in launch order),
+        // into L2 while this one computes: its loads then wait on L2 rather than HBM
+        const long long lin = blockIdx.x + (long long)gridDim.x * (blockIdx.y + (long long)gridDim.y * blockIdx.z);
+        const long long nx = lin + a.wave;
+        if (a.wave > 0 && nx < (long long)gridDim.x * gridDim.y * gridDim.z) {
+            const int n2 = (int)(nx % gridDim.x), h2 = (int)((nx / gridDim.x) % gridDim.y),
+                      b2 = (int)(nx / ((long long)gridDim.x * gridDim.y));
+            const int ci2 = (b2 * H + h2) * a.N + n2;
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                if (VAR == VAR_KDA) {
+                    l2_prefetch_2d(&mp.Kt1, 64 * p, ci2 * C);
+                    l2_prefetch_2d(&mp.Qt1, 64 * p, ci2 * C);
+                    l2_prefetch_2d(&mp.Kh, 64 * p, ci2 * KDA_KH_ROWS);
+                    l2_prefetch_2d(&mp.Kt, 64 * p, ci2 * C);
+                } else {
+                    l2_prefetch_4d(&mp.k, 64 * p, h2, n2 * C, b2);
+                    l2_prefetch_4d(&mp.q, 64 * p, h2, n2 * C, b2);
+                }
+                l2_prefetch_4d(&mp.v, 64 * p, h2, n2 * C, b2);
+            }
         }
     }
     if (warp == 0) tmem_alloc(tmem_slot, TM_COLS);
@@ -706,6 +744,10 @@ cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool ke
     Args a;
     a.alpha = t.alpha; a.beta = t.beta; a.gb = w.gb; a.kwide = w.kwide; a.Dx = w.Dx; a.rn = w.rn;
     a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return cudaErrorInvalidValue;
+    a.wave = 2 * sms;
     const dim3 grid(g.N, g.H, g.B);
     if (g.variant == VAR_KDA) {  // KEEP: T and the gated k k^T products M (for the KDA gradient kernel)
         if (raw) return cudaErrorInvalidValue;
