@@ -230,9 +230,11 @@ int delta_rule_fwd_noalloc(const void *q, const void *k, const void *v, const vo
  * space; section 4.1 -- sigmoid output gate on RMSNorm of the core's output).
  * From the raw projections q_raw, k_raw [B,T,H,dk], the raw forget logits
  * gate_raw [B,T,H] (Gated DeltaNet; unused and may be NULL for DeltaNet) and
- * the raw write-strength logits beta_raw [B,T,H] it computes, exactly as
- * delta_rule_preop then delta_rule_fwd then delta_rule_postop would (up to
- * rounding order: the normalised q, k and the gates stay in fp32 on chip),
+ * the raw write-strength logits beta_raw [B,T,H] it computes what
+ * delta_rule_preop then delta_rule_fwd then delta_rule_postop compute, to
+ * within bf16 rounding (the normalised q, k and the gates stay in fp32 on chip;
+ * sigmoid(gate_out) is formed in packed bf16 arithmetic with the hardware tanh,
+ * and o enters y through a bf16 copy; y is within 1 % of the fp64 definition),
  *     y = RMSNorm(o) * w_norm * sigmoid(gate_out)   [B,T,H,dv]
  * and, when their pointers are not NULL, o itself (before the normalisation),
  * u and S_T.  gate_out [B,T,H,dv] has the I/O dtype, w_norm is fp32 [dv].
