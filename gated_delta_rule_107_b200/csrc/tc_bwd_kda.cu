@@ -27,7 +27,7 @@
 // lane quarter w, and split each epilogue's token columns in halves), phases in order:
 //   A  loads; [Qd^T | -dWm^T] = S [dO ; dU]^T, Tm^T = dS+ U^T;  RS, g (from log alpha), dWm^T tile
 //   B  loads of M, W, U~, v;  dB_k^T = dWm^T T,  dB_v^T = dU^T T;  their bf16 tiles, dv, v . dB_v
-//   C  dA' = dB [W | U~]^T and its transpose, [dO ; U][dO ; U]^T (dP and dP^T in one product);
+//   C  dA' = dB [W | U~]^T, [dO ; U][dO ; U]^T (dP and dP^T in one product);
 //      dM, dP, dM^T, dP^T tiles, the dbeta part of A;  the gate-scaled sections Km, Kp, Qp
 //   D  X^T, Yv^T, Z^T (block by block, N = 16);  the final per-channel epilogue
 // Sums over the channels of one token (dbeta's) reduce 4 tokens at a time across a warp's 32 lanes
@@ -315,19 +315,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
         fence_after_sync();
         // dA'[r][i] = dB_k[r] . W[i] + dB_v[r] . U~[i]: A = dB^T tiles read MN-major (rows 64-127 of
         // the M = 128 product are discarded), B = W, U~ K-major
-        const uint32_t ida = idesc_bf16(128, 64, 1, 0), idt = idesc_bf16(128, 64, 0, 1), id5 = idesc_bf16(128, 128, 0, 0);
+        const uint32_t ida = idesc_bf16(128, 64, 1, 0), id5 = idesc_bf16(128, 128, 0, 0);
 #pragma unroll 1
         for (int k = 0; k < 16; ++k) {
             const uint32_t at = (k < 8 ? u32(R_DBK) : u32(R_DBV)) + (k & 7) * 2048;
             const uint32_t bw = (k < 8 ? u32(R_W) : u32(R_UT)) + ((k & 7) >> 2) * 8192 + (k & 3) * 32;
             mma_bf16(tbase + TM_X, sdesc(at, 8192, 1024), sdesc(bw, 16, 1024), ida, k > 0);
-        }
-        // dA'^T[i][r]: A = W, U~ K-major, B = dB^T tiles MN-major
-#pragma unroll 1
-        for (int k = 0; k < 16; ++k) {
-            const uint32_t aw = (k < 8 ? u32(R_W) : u32(R_UT)) + ((k & 7) >> 2) * 8192 + (k & 3) * 32;
-            const uint32_t bt = (k < 8 ? u32(R_DBK) : u32(R_DBV)) + (k & 7) * 2048;
-            mma_bf16(tbase + TM_YV, sdesc(aw, 16, 1024), sdesc(bt, 8192, 1024), idt, k > 0);
         }
         // [dO ; U] [dO ; U]^T: dP = dO U^T at lanes 0-63 / columns 64-127, dP^T at lanes 64-127 / 0-63
 #pragma unroll 1
@@ -339,8 +332,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
     }
     if (ok) ok = wait_mma(true);
     // ---- E2: the masked tiles dM, dP [r][i] and dM^T, dP^T [i][r]; the dbeta part of A ----
-    //   lanes 0-63 (quarters 0, 1): half 0 takes dA' (-> dM, dbeta_A), half 1 takes dP, and each
-    //   half takes 32 columns of dA'^T (-> dM^T);  lanes 64-127: each half takes 32 columns of dP^T
+    //   lanes 0-63 (quarters 0, 1): half 0 takes dA' (-> dM and, element by element at the
+    //   transposed place, dM^T, dbeta_A), half 1 takes dP;  lanes 64-127: each half takes 32
+    //   columns of dP^T
     if (ok) {
         const int rl = (warp & 1) * 32 + lane;  // the product's row (r, or i for the transposes)
         if (q4 < 2) {
@@ -359,6 +353,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
                         const float d = ch * 8 + e < r ? -x8[e] : 0.f;
                         db += d * m8[e];
                         w8[e] = br * d;
+                        // dM^T[i][r] = dM[r][i]: the same bf16 at row i, column r
+                        *reinterpret_cast<__nv_bfloat16 *>(sm + R_DMT + swz(ch * 8 + e, r >> 3) + (r & 7) * 2) =
+                            __float2bfloat16_rn(w8[e]);
                     }
                     st_chunk(sm + R_DM, swz(r, ch), w8);
                 }
@@ -374,17 +371,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constan
                     for (int e = 0; e < 8; ++e) x8[e] = ch * 8 + e <= r ? x8[e] : 0.f;
                     st_chunk(sm + R_DP, swz(r, ch), x8);
                 }
-            }
-            const int i = rl;  // dA'^T[i][r] -> dM^T[i][r] = -beta_r dA'^T (r > i), r in this half
-#pragma unroll 1
-            for (int k8 = 0; k8 < 4; ++k8) {
-                const int rr = r0 + 8 * k8;
-                float x8[8];
-                tmem_ld8(tl + TM_YV + rr, x8);
-                wait_ld();
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x8[e] = rr + e > i ? -betas[rr + e] * x8[e] : 0.f;
-                st_chunk(sm + R_DMT, swz(i, rr >> 3), x8);
             }
         } else {
             const int i = rl;  // dP^T[i][r] (r >= i), r in this half
