@@ -482,24 +482,41 @@ __device__ __forceinline__ void st8_bf16(__nv_bfloat16 *p, const float *v) {
     *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// shared memory of k_kda_gates: g [64][128] fp32, k and q [64][128] bf16, block sums and edges
+constexpr uint32_t KG_G = 0, KG_K = 32768, KG_Q = 49152, KG_TOT = 65536, KG_BLK = KG_TOT + 8 * DK * 4,
+                   KG_END = KG_BLK + 4 * DK * 4, KG_SMEM = KG_END + DK * 4;
+
+// 16 bytes global -> shared without registers (zeros when !in)
+__device__ __forceinline__ void cp16(void *dst, const void *src, bool in) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(in ? 16 : 0)
+                 : "memory");
+}
+
 __global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
-    __shared__ float tot[8][DK];
-    __shared__ float gblk[4][DK], gend[DK];
+    extern __shared__ __align__(16) unsigned char kg_sm[];
+    float *sg = reinterpret_cast<float *>(kg_sm + KG_G);
+    __nv_bfloat16 *sk = reinterpret_cast<__nv_bfloat16 *>(kg_sm + KG_K), *sq = reinterpret_cast<__nv_bfloat16 *>(kg_sm + KG_Q);
+    float(*tot)[DK] = reinterpret_cast<float(*)[DK]>(kg_sm + KG_TOT);
+    float(*gblk)[DK] = reinterpret_cast<float(*)[DK]>(kg_sm + KG_BLK);
+    float *gend = reinterpret_cast<float *>(kg_sm + KG_END);
     const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int tg = threadIdx.x >> 4, cg = threadIdx.x & 15, c0 = 8 * cg, R = tg >> 1;
     const int t0 = n * C, L = min(C, a.T - t0);
     const size_t ci = ((size_t)b * a.H + h) * a.N + n;
     auto at = [&](int r) { return (((size_t)b * a.T + t0 + r) * a.H + h) * DK + c0; };
-    // every input row of this thread at once (24 16-byte loads in flight; rows past T read as 0)
-    uint4 ar[8], kw[8], qw[8];
+    // every input row of this thread at once: k and q straight into shared memory, log alpha into
+    // registers (24 16-byte loads in flight; rows past T read as 0)
+    uint4 ar[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        const bool in = 8 * tg + r < L;
-        ar[r] = in ? __ldg(reinterpret_cast<const uint4 *>(a.alpha + at(8 * tg + r))) : z;
-        kw[r] = in ? __ldg(reinterpret_cast<const uint4 *>(a.k + at(8 * tg + r))) : z;
-        qw[r] = in ? __ldg(reinterpret_cast<const uint4 *>(a.q + at(8 * tg + r))) : z;
+        const int tr = 8 * tg + r;
+        const bool in = tr < L;
+        const size_t src = in ? at(tr) : 0;
+        cp16(sk + tr * DK + c0, a.k + src, in);
+        cp16(sq + tr * DK + c0, a.q + src, in);
+        ar[r] = in ? __ldg(reinterpret_cast<const uint4 *>(a.alpha + src)) : make_uint4(0u, 0u, 0u, 0u);
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
     float g[8][8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
@@ -520,6 +537,14 @@ __global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
         if ((tg & 1) == 0) gblk[R][c0 + j] = g[0][j];  // token 16 R, the first of block R
         if (tg == 7) gend[c0 + j] = g[7][j];           // token C - 1, the last
     }
+    // this thread's g rows to shared memory (read back row by row below)
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        float *d = sg + (8 * tg + r) * DK + c0;
+        *reinterpret_cast<float4 *>(d) = make_float4(g[r][0], g[r][1], g[r][2], g[r][3]);
+        *reinterpret_cast<float4 *>(d + 4) = make_float4(g[r][4], g[r][5], g[r][6], g[r][7]);
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();
     float gb[8], gC[8];  // g at the first token of this thread's block, and at the chunk's last
     bool wide = false;
@@ -530,18 +555,24 @@ __global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
         // the fall of the gate inside block R, from its first token to its last (held by tg odd)
         if (tg & 1) wide |= !(gb[j] - g[7][j] <= KDA_DIAG_SPAN);
     }
-#pragma unroll
+#pragma unroll 1
     for (int r = 0; r < 8; ++r) {
         const int tr = 8 * tg + r;
-        float kr[8], qr[8];
-        unpack8_bf16(kw[r], kr);
-        unpack8_bf16(qw[r], qr);
+        float kr[8], qr[8], gr[8];
+        unpack8_bf16(*reinterpret_cast<const uint4 *>(sk + tr * DK + c0), kr);
+        unpack8_bf16(*reinterpret_cast<const uint4 *>(sq + tr * DK + c0), qr);
+        {
+            const float4 u0 = *reinterpret_cast<const float4 *>(sg + tr * DK + c0);
+            const float4 u1 = *reinterpret_cast<const float4 *>(sg + tr * DK + c0 + 4);
+            gr[0] = u0.x; gr[1] = u0.y; gr[2] = u0.z; gr[3] = u0.w;
+            gr[4] = u1.x; gr[5] = u1.y; gr[6] = u1.z; gr[7] = u1.w;
+        }
         float o1[8], o2[8], o4[8], o5[8], o6[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             // every exponent here is <= 0 for log alpha <= 0; the clamp only keeps other input finite
-            const float eb = __expf(fminf(g[r][j] - gb[j], 80.f));  // row factor
-            const float eg = __expf(fminf(g[r][j], 80.f)), ec = __expf(fminf(gC[j] - g[r][j], 80.f));
+            const float eb = __expf(fminf(gr[j] - gb[j], 80.f));  // row factor
+            const float eg = __expf(fminf(gr[j], 80.f)), ec = __expf(fminf(gC[j] - gr[j], 80.f));
             o1[j] = kr[j] * eb; o2[j] = qr[j] * eb;
             o4[j] = kr[j] * eg; o5[j] = qr[j] * eg; o6[j] = kr[j] * ec;
         }
@@ -552,12 +583,11 @@ __global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
         st8_bf16(a.Qt + o, o5);
         st8_bf16(a.Kb + o, o6);
         // column operand of every block R2 >= R (token tr is one of its rows 0 .. 16 R2 + 15)
-#pragma unroll
-        for (int R2 = 0; R2 < 4; ++R2) {
-            if (R2 < R) continue;
+#pragma unroll 1
+        for (int R2 = R; R2 < 4; ++R2) {
             float oh[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) oh[j] = kr[j] * __expf(fminf(gblk[R2][c0 + j] - g[r][j], 80.f));
+            for (int j = 0; j < 8; ++j) oh[j] = kr[j] * __expf(fminf(gblk[R2][c0 + j] - gr[j], 80.f));
             st8_bf16(a.Kh + (ci * KDA_KH_ROWS + kda_sec(R2) + tr) * DK + c0, oh);
         }
     }
@@ -571,11 +601,12 @@ __global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
     wide = __syncthreads_or(wide);
     if (threadIdx.x == 0) a.kwide[ci] = wide ? 1 : 0;
     if (wide && a.G) {  // g itself, for the CUDA-core gradient kernel that takes the marked chunks
-#pragma unroll
+#pragma unroll 1
         for (int r = 0; r < 8; ++r) {
+            const float *src = sg + (8 * tg + r) * DK + c0;
             float *dst = a.G + (ci * C + 8 * tg + r) * DK + c0;
-            *reinterpret_cast<float4 *>(dst) = make_float4(g[r][0], g[r][1], g[r][2], g[r][3]);
-            *reinterpret_cast<float4 *>(dst + 4) = make_float4(g[r][4], g[r][5], g[r][6], g[r][7]);
+            *reinterpret_cast<float4 *>(dst) = *reinterpret_cast<const float4 *>(src);
+            *reinterpret_cast<float4 *>(dst + 4) = *reinterpret_cast<const float4 *>(src + 4);
         }
     }
 }
@@ -654,8 +685,10 @@ cudaError_t tc_kda_gates(const Geo &g, const Tensors &t, const TcWs &w, float *G
     a.T = g.T; a.H = g.H; a.N = g.N;
     cudaError_t e = cudaFuncSetAttribute(k_kda_diag, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DIAG_SMEM);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k_kda_gates, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KG_SMEM);
+    if (e != cudaSuccess) return e;
     rec.mark(s);
-    k_kda_gates<<<dim3(g.N, g.H, g.B), DK, 0, s>>>(a);
+    k_kda_gates<<<dim3(g.N, g.H, g.B), DK, KG_SMEM, s>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     rec.mark(s);
