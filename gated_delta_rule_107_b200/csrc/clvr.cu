@@ -543,14 +543,21 @@ int clvr_bwd_run(const void *U, const void *W, const void *dH, void *dU, float *
         if (rc != DR_OK) return rc;
     }
     if (dW) {  // dW [K][N] = U^T dH: A = U [M][K] (MN-major), B = dH [M][N] (MN-major); the M-long
-               // reduction in slices (enough work items for every pair of SMs) with fp32 partials
+               // reduction in slices with fp32 partials: the slice count that minimises the rounds of
+               // work items over the SM pairs times the slice length (fewest slices on a tie), within
+               // the workspace
         const size_t elems = (size_t)K * N;
         const int tiles = ((K + clv::BM - 1) / clv::BM) * ((N + clv::BN - 1) / clv::BN), pairs = clv::sm_count() / 2;
-        int nsplit = pairs > 0 ? (pairs + tiles - 1) / tiles : 1;
-        nsplit = nsplit < clv::MAX_SPLIT ? nsplit : clv::MAX_SPLIT;
         const int kb = (M + clv::BK - 1) / clv::BK;
-        nsplit = nsplit < kb ? nsplit : (kb > 0 ? kb : 1);
-        while (nsplit > 1 && (size_t)nsplit * elems * sizeof(float) > ws_bytes) --nsplit;
+        int nsplit = 1;
+        if (pairs > 0) {
+            double best = 0.0;
+            for (int ns = 1; ns <= clv::MAX_SPLIT && ns <= (kb > 0 ? kb : 1); ++ns) {
+                if (ns > 1 && (size_t)ns * elems * sizeof(float) > ws_bytes) break;
+                const double cost = (double)((tiles * ns + pairs - 1) / pairs) * ((kb + ns - 1) / ns);
+                if (ns == 1 || cost < best) { best = cost; nsplit = ns; }
+            }
+        }
         if (nsplit == 1) return clv::gemm_bf16(U, 1, dH, 1, nullptr, nullptr, dW, K, N, M, 1, elems, s);
         float *part = (float *)ws;
         int rc = clv::gemm_bf16(U, 1, dH, 1, nullptr, nullptr, part, K, N, M, nsplit, elems, s);
