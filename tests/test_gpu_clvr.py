@@ -21,7 +21,10 @@ def _check(got, ref, tol, what):
 
 
 @pytest.mark.parametrize("dtype", ("f32", "bf16"))
-@pytest.mark.parametrize("shape", ((1, 5, 2, 64, 128), (2, 150, 8, 128, 1024), (3, 37, 4, 64, 40)))
+# (2, 200, 3, 128, 384): M = 400 and N = 384, so in the last row and column blocks of 256 the
+# first CTA of a pair holds 128 valid rows / columns and the second a part (rows 384-399) or none
+@pytest.mark.parametrize("shape", ((1, 5, 2, 64, 128), (2, 150, 8, 128, 1024), (3, 37, 4, 64, 40),
+                                   (2, 200, 3, 128, 384)))
 def test_forward_and_backward(dtype, shape):
     B, T, H, dv, N = shape
     g = torch.Generator().manual_seed(B * 1000 + T)
