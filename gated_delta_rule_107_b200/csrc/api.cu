@@ -5,6 +5,8 @@
 // the tensor-core files and decode.cu.  Validation failures return before anything is enqueued.
 #include <limits.h>
 
+#include <mutex>
+
 #include "../../include/delta_rule.h"
 #include "decode.cuh"
 #include "prepost.cuh"
@@ -59,6 +61,110 @@ bool use_kda_hybrid_bwd(const Geo &g, int dtype, int kind) {
 }
 size_t ws_al(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// ---- segments of the chunk range (Gated DeltaNet / DeltaNet on the split path) ----
+// The chain kernels run one CTA per (b, h, 64 value columns) and walk a sequence's chunks in
+// order.  With few (b, h) pairs they occupy few SMs, so the chunk range is cut into segments: the
+// prep of segment k + 1 runs on a second stream beside the forward chain of segment k, and the
+// gradient kernel of segment k + 1 beside the reverse chain of segment k; the fp32 states at the
+// cuts go through the workspace.  Each chain segment is enqueued before the kernel meant to run
+// beside it, so that when both can start the chain's CTAs are placed first.
+int seg_count(const Geo &g) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 1;
+    const long long chain_ctas = 2LL * g.B * g.H;  // (b, h, value half)
+    if (chain_ctas * 2 > sms || g.N < 32) return 1;
+    return 4;
+}
+size_t seg_cut_bytes(const Geo &g) {
+    const int S = seg_count(g);
+    return S > 1 ? ws_al((size_t)(S - 1) * g.B * g.H * g.dk * g.dv * sizeof(float)) : 0;
+}
+// the library's second stream on the current device (created once, non-blocking)
+cudaStream_t side_stream() {
+    static std::mutex mu;
+    static cudaStream_t st[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!st[dev] && cudaStreamCreateWithFlags(&st[dev], cudaStreamNonBlocking) != cudaSuccess) st[dev] = nullptr;
+    return st[dev];
+}
+struct SegEvents {  // events of one call, released when the call has enqueued its work
+    cudaEvent_t ev[8] = {};
+    int n = 0;
+    bool make(int k) {
+        for (n = 0; n < k; ++n)
+            if (cudaEventCreateWithFlags(&ev[n], cudaEventDisableTiming) != cudaSuccess) return false;
+        return true;
+    }
+    ~SegEvents() {
+        for (int i = 0; i < n; ++i) cudaEventDestroy(ev[i]);
+    }
+};
+int seg_bound(const Geo &g, int S, int k) { return (int)((long long)g.N * k / S); }
+
+// prep + forward chain in S segments; cuts: S - 1 fp32 states [B, H, dk, dv]
+cudaError_t fwd_segmented(const Geo &g, const Tensors &t, const TcWs &w, bool save, float *cuts, cudaStream_t s) {
+    const int S = seg_count(g);
+    const size_t stride = (size_t)g.B * g.H * g.dk * g.dv;
+    cudaStream_t ss = side_stream();
+    SegEvents se;
+    if (!ss || !se.make(S)) return cudaErrorMemoryAllocation;
+    Rec none;
+    TcWs wk = w;
+    wk.m0 = seg_bound(g, S, 0); wk.m1 = seg_bound(g, S, 1);
+    cudaError_t e = tc_chunk_prep(g, t, wk, save, s, none);
+    if (e == cudaSuccess) e = cudaEventRecord(se.ev[0], s);
+    for (int k = 0; k < S && e == cudaSuccess; ++k) {
+        Tensors tk = t;
+        tk.S0 = k == 0 ? t.S0 : cuts + (k - 1) * stride;
+        tk.S_T = k == S - 1 ? t.S_T : cuts + k * stride;
+        wk.m0 = seg_bound(g, S, k); wk.m1 = seg_bound(g, S, k + 1);
+        if (k > 0) e = cudaStreamWaitEvent(s, se.ev[k], 0);
+        if (e == cudaSuccess) e = tc_chain_fwd(g, tk, wk, save ? 2 : 0, s, none);
+        if (e == cudaSuccess && k + 1 < S) {  // the next segment's products, beside this chain
+            if (k == 0) e = cudaStreamWaitEvent(ss, se.ev[0], 0);
+            wk.m0 = seg_bound(g, S, k + 1); wk.m1 = seg_bound(g, S, k + 2);
+            if (e == cudaSuccess) e = tc_chunk_prep(g, t, wk, save, ss, none);
+            if (e == cudaSuccess) e = cudaEventRecord(se.ev[k + 1], ss);
+        }
+    }
+    return e;  // the last chain waited for the side stream's last prep
+}
+
+// reverse chain + gradient kernel in S segments, the last segment first; cuts: S - 1 fp32 dL/dS
+cudaError_t bwd_segmented(const Geo &g, const Tensors &t, const TcWs &w, float *cuts, cudaStream_t s) {
+    const int S = seg_count(g);
+    const size_t stride = (size_t)g.B * g.H * g.dk * g.dv;
+    cudaStream_t ss = side_stream();
+    SegEvents se;  // one per segment, and the side stream's end
+    if (!ss || !se.make(S + 1)) return cudaErrorMemoryAllocation;
+    Rec none;
+    TcWs wk = w;
+    cudaError_t e = cudaSuccess;
+    for (int k = S - 1; k >= 0 && e == cudaSuccess; --k) {
+        Tensors tk = t;
+        tk.dS_T = k == S - 1 ? t.dS_T : cuts + k * stride;  // dL/dS after the segment
+        tk.dS0 = k == 0 ? t.dS0 : cuts + (k - 1) * stride;   // dL/dS entering it
+        wk.m0 = seg_bound(g, S, k); wk.m1 = seg_bound(g, S, k + 1);
+        e = tc_chain_rev(g, tk, wk, s, none);
+        if (e == cudaSuccess) e = cudaEventRecord(se.ev[k], s);
+        if (e == cudaSuccess && k + 1 < S) {  // the gradients of the segment after, beside this chain
+            wk.m0 = seg_bound(g, S, k + 1); wk.m1 = seg_bound(g, S, k + 2);
+            e = cudaStreamWaitEvent(ss, se.ev[k + 1], 0);
+            if (e == cudaSuccess) e = tc_bwd_chunk(g, t, wk, ss, none);
+        }
+    }
+    if (e == cudaSuccess) {  // the first segment's gradients on the caller's stream; then join
+        wk.m0 = seg_bound(g, S, 0); wk.m1 = seg_bound(g, S, 1);
+        e = tc_bwd_chunk(g, t, wk, s, none);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(se.ev[S], ss);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, se.ev[S], 0);
+    return e;
+}
+
 // Parts of the split-path workspace (tc_path.cuh) that each call kind uses
 constexpr int GDN_SAVED = WS_FWD | WS_KEEP | WS_STATE;
 constexpr int KDA_FWD = WS_FWD | WS_KDA | WS_KDAC;
@@ -68,11 +174,14 @@ constexpr int KDA_BWD = WS_FWD | WS_KEEP | WS_STATE | WS_REV | WS_KDA | WS_KDAC;
 size_t ws_bytes(const Geo &g, int dtype, int kind) {
     if (g.T == 0 || g.B == 0 || g.H == 0) return 0;
     if (use_split(g, dtype)) {
+        // the parts below, then (only for shapes cut into segments) the states at the cuts
+        const size_t cut = seg_cut_bytes(g);
+        auto with_cut = [&](size_t x) { return cut ? ws_al(x) + cut : x; };
         switch (kind) {
-            case K_FWD: return tc_ws_bytes(g, WS_FWD);
-            case K_BWD: return tc_ws_bytes(g, GDN_SAVED | WS_REV);
-            case K_FWD_SAVE: return 0;  // everything it keeps lives in the saved buffer
-            default: return tc_ws_bytes(g, WS_REV);
+            case K_FWD: return with_cut(tc_ws_bytes(g, WS_FWD));
+            case K_BWD: return with_cut(tc_ws_bytes(g, GDN_SAVED | WS_REV));
+            case K_FWD_SAVE: return cut;  // everything it keeps lives in the saved buffer
+            default: return with_cut(tc_ws_bytes(g, WS_REV));
         }
     }
     if (use_split_kda(g, dtype, kind))  // the saving forward keeps all but its forward-only tiles
@@ -155,8 +264,13 @@ static int fwd_impl(const void *q, const void *k, const void *v, const void *alp
         TcWs w = {};
         if (save) tc_ws_carve(g, GDN_SAVED, saved, &w);
         else tc_ws_carve(g, WS_FWD, workspace, &w);
-        rc = launch_status(tc_chunk_prep(g, t, w, save, s, rec));
-        if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, save ? 2 : 0, s, rec));
+        if (seg_count(g) > 1 && rec.ev == nullptr) {  // (the timed entry points run one launch each)
+            float *cuts = (float *)((char *)workspace + (save ? 0 : ws_al(tc_ws_bytes(g, WS_FWD))));
+            rc = launch_status(fwd_segmented(g, t, w, save, cuts, s));
+        } else {
+            rc = launch_status(tc_chunk_prep(g, t, w, save, s, rec));
+            if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, save ? 2 : 0, s, rec));
+        }
     } else if (use_split_kda(g, dtype, kind)) {
         TcWs w = {};
         if (save) {  // the chain operands, states and G go to the saved buffer
@@ -216,8 +330,13 @@ static int bwd_impl(const void *q, const void *k, const void *v, const void *alp
             rc = launch_status(tc_chunk_prep(g, t, w, true, s, rec));
             if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, 1, s, rec));
         }
-        if (rc == DR_OK) rc = launch_status(tc_chain_rev(g, t, w, s, rec));
-        if (rc == DR_OK) rc = launch_status(tc_bwd_chunk(g, t, w, s, rec));
+        if (rc == DR_OK && seg_count(g) > 1 && rec.ev == nullptr) {
+            float *cuts = (float *)((char *)workspace + ws_al(tc_ws_bytes(g, from_saved ? WS_REV : (GDN_SAVED | WS_REV))));
+            rc = launch_status(bwd_segmented(g, t, w, cuts, s));
+        } else {
+            if (rc == DR_OK) rc = launch_status(tc_chain_rev(g, t, w, s, rec));
+            if (rc == DR_OK) rc = launch_status(tc_bwd_chunk(g, t, w, s, rec));
+        }
     } else if (use_kda_hybrid_bwd(g, dtype, kind)) {
         SimtWs sw = simt_ws_carve(g, true, workspace);
         char *tcbase = (char *)workspace + ws_al(simt_ws_bytes(g, true));

@@ -102,7 +102,7 @@ struct Args {
     void *dalpha, *dbeta;  // bf16 [B, T, H]
     const float *gb;       // [chunks][2][64]: g, beta
     const float *skt;      // [chunks][2][64]
-    int B, T, H, N, variant;
+    int B, T, H, N, variant;    int m0, m1;            // the chunks [m0, m1) of each sequence (m1 = 0: all)
 };
 
 __device__ __forceinline__ void st_bf(void *p, size_t i, float x) {
@@ -158,14 +158,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(const __grid_const
     const int q4 = warp & 3, hf = warp >> 2;
     const bool rowt = q4 < 2;            // owns token row r of the accumulators
     const int r = (q4 & 1) * 32 + lane;  // token row (TMEM rows 64 + r for q4 >= 2)
-    const int T = a.T, H = a.H, N = a.N, total = a.B * H * N;
+    const int T = a.T, H = a.H, N = a.N, m0 = a.m0, NS = (a.m1 > 0 ? a.m1 : N) - m0, total = a.B * H * NS;
     const bool gated = a.variant == VAR_GATED;
     auto part_at = [&](int kind, int half, int rr) -> float & { return part[(kind * 2 + half) * 64 + rr]; };
     struct Pos { int ci, n, h, b, t0; };
-    auto pos_of = [&](int ci) -> Pos {  // ci = (b H + h) N + n
+    auto pos_of = [&](int wi) -> Pos {  // work item wi: chunk n = m0 + wi % NS of sequence (b, h) = wi / NS
         Pos p;
-        p.ci = ci; p.n = ci % N;
-        const int bh = ci / N;
+        p.n = m0 + wi % NS;
+        const int bh = wi / NS;
+        p.ci = bh * N + p.n;
         p.h = bh % H; p.b = bh / H; p.t0 = p.n * C;
         return p;
     };
@@ -623,7 +624,7 @@ cudaError_t tc_bwd_chunk(const Geo &g, const Tensors &t, const TcWs &w, cudaStre
     if (!ok) return cudaErrorInvalidValue;
     Args a;
     a.dalpha = t.dalpha; a.dbeta = t.dbeta; a.gb = w.gb; a.skt = w.skt;
-    a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N; a.variant = g.variant;
+    a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N; a.variant = g.variant; a.m0 = w.m0; a.m1 = w.m1;
     const size_t smem = SMEM_BYTES + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_bwd_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -632,7 +633,7 @@ cudaError_t tc_bwd_chunk(const Geo &g, const Tensors &t, const TcWs &w, cudaStre
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    const long long total = (long long)g.B * g.H * g.N;
+    const long long total = (long long)g.B * g.H * ((w.m1 > 0 ? w.m1 : g.N) - w.m0);
     const int grid = (int)(total < sms ? total : sms);
     k_bwd_chunk_tc<<<grid, NTHREADS, smem, s>>>(mp, a);
     return cudaGetLastError();

@@ -96,6 +96,9 @@ struct Args {
     const float *egc;         // KDA forward: [chunks][128] e^{g_C} per key channel
     const float *rn;          // fused forward: [chunks][2][64] 1 / |k_r|, 1 / |q_r|
     const float *wn;          // fused forward: RMSNorm weight [128]
+    int m0, m1;               // the chunks [m0, m1) of each sequence (m1 = 0: to the end); forward: S0
+                              // the state entering chunk m0, ST the state after chunk m1 - 1; reverse:
+                              // S0 = dL/dS after chunk m1 - 1, ST = dL/dS entering chunk m0
 };
 
 // The producer's gate factors of a chunk (e^{g_C - g}, e^g, e^{g_C}; fused forward: with the raw
@@ -190,6 +193,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
     const int j0 = half * DVB;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = a.T, H = a.H, N = a.N;
+    const int m0 = a.m0, NS = (a.m1 > 0 ? a.m1 : N) - m0;  // this launch's chunks: [m0, m0 + NS)
     const size_t ci0 = ((size_t)b * H + h) * N;
 
     if (threadIdx.x == 0) {
@@ -213,11 +217,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
         // ================================ producer ================================
         int issued[2] = {0, 0};
         FactorIn fin;
-        for (int m = 0; m < N; ++m) {
-            const int s = m & 1, t0 = m * C;
+        for (int mi = 0; mi < NS; ++mi) {  // mi: this launch's chunk count so far (stages, phases)
+            const int m = m0 + mi, s = mi & 1, t0 = m * C;
             const int ci = (int)(ci0 + m);
             factors_fetch<KDA != 0, FUSED>(a, (size_t)ci, lane, fin);
-            if (m >= 2 && !mbar_wait(&bar[B_EMPTY0 + s], ((m >> 1) - 1) & 1, abort_flag)) break;
+            if (mi >= 2 && !mbar_wait(&bar[B_EMPTY0 + s], ((mi >> 1) - 1) & 1, abort_flag)) break;
             unsigned char *st = sm + s * STAGE;
             if (lane == 0) {
                 mbar_arrive_tx(&bar[B_FULL0 + s], (OUT ? 65536u : 40960u) + (FUSED ? 8192u : 0u));
@@ -393,12 +397,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             const float inv = fused_inv(prev_m);
             y_step(prev_m, inv);
         };
-        for (int m = 0; m < N; ++m) {
-            const int s = m & 1, t0 = m * C, L = min(C, T - t0);
-            const uint32_t buf = (uint32_t)(m & 1) * 128;
+        for (int mi = 0; mi < NS; ++mi) {  // stages and phases by mi; m is the chunk of the sequence
+            const int m = m0 + mi, s = mi & 1, t0 = m * C, L = min(C, T - t0);
+            const uint32_t buf = (uint32_t)(mi & 1) * 128;
             const size_t ci = ci0 + m;
             unsigned char *st = sm + s * STAGE;
-            const bool got = mbar_wait(&bar[B_FULL0 + s], (m >> 1) & 1, abort_flag);
+            const bool got = mbar_wait(&bar[B_FULL0 + s], (mi >> 1) & 1, abort_flag);
             if (wabort(got)) break;
             // this chunk's factors, read before the stage is released
             const float *cf = cf_all + s * 132;
@@ -459,14 +463,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
                     const uint4 g4 = *reinterpret_cast<const uint4 *>(st + FS_G + swz(trow - 64, hf * 4 + c4));
-                    if (m & 1) {
+                    if (mi & 1) {
                         sg1[c4 * 4] = g4.x; sg1[c4 * 4 + 1] = g4.y; sg1[c4 * 4 + 2] = g4.z; sg1[c4 * 4 + 3] = g4.w;
                     } else {
                         sg0[c4 * 4] = g4.x; sg0[c4 * 4 + 1] = g4.y; sg0[c4 * 4 + 2] = g4.z; sg0[c4 * 4 + 3] = g4.w;
                     }
                 }
-                if (m >= 2) inv_y = fused_inv(m - 2);
-                if (m >= 1) send_sums(m - 1);
+                if (mi >= 2) inv_y = fused_inv(mi - 2);  // (the fused forward runs whole sequences: mi = m)
+                if (mi >= 1) send_sums(mi - 1);
             }
             fence_proxy_async();
             fence_before_sync();
@@ -493,7 +497,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             }
             pending = true;
             if (KEEP && wc == 0) bulk_wait_read_1();  // the S_m store has read OFF_S
-            if (FUSED && trow >= 64 && m >= 2) y_step(m - 2, inv_y);  // while the second product runs
+            if (FUSED && trow >= 64 && mi >= 2) y_step(mi - 2, inv_y);  // while the second product runs
             if (!mma_done()) break;
             if (wc == 0) mbar_arrive(&bar[B_EMPTY0 + s]);
             // ---------------- S <- e^{gC} S + E ----------------
@@ -508,7 +512,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_fwd(const __grid_constant
             fence_proxy_async();
             fence_before_sync();
             if (wabort(true)) break;
-            prev_L = L; prev_t0 = t0; prev_eg = rowf; prev_buf = buf; prev_m = m;
+            prev_L = L; prev_t0 = t0; prev_eg = rowf; prev_buf = buf; prev_m = mi;
         }
         // the last chunk (all chain threads agree first: the fused epilogue waits on the partner)
         const bool fin = !named_sync_any(2, 256, *abort_flag != 0);
@@ -552,6 +556,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
     const int j0 = half * DVB;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int H = a.H, N = a.N;
+    const int M1 = a.m1 > 0 ? a.m1 : N, NS = M1 - a.m0;  // this launch's chunks [m0, M1), last first
     const size_t ci0 = ((size_t)b * H + h) * N;
 
     if (threadIdx.x == 0) {
@@ -569,8 +574,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
         // ================================ producer ================================
         int issued[2] = {0, 0};
         FactorIn fin;
-        for (int m = 0; m < N; ++m) {
-            const int mc = N - 1 - m, s = m & 1, t0 = mc * C;
+        for (int m = 0; m < NS; ++m) {
+            const int mc = M1 - 1 - m, s = m & 1, t0 = mc * C;
             const int ci = (int)(ci0 + mc);
             factors_fetch<KDA != 0, false>(a, (size_t)ci, lane, fin);
             if (m >= 2 && !mbar_wait(&bar[B_EMPTY0 + s], ((m >> 1) - 1) & 1, abort_flag)) break;
@@ -631,8 +636,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_chain_rev(const __grid_constant
         }
         fence_proxy_async();
         named_sync(2, 256);
-        for (int m = 0; m < N; ++m) {
-            const int mc = N - 1 - m, s = m & 1;
+        for (int m = 0; m < NS; ++m) {
+            const int mc = M1 - 1 - m, s = m & 1;
             const size_t ci = ci0 + mc;
             unsigned char *st = sm + s * STAGE;
             const bool got = mbar_wait(&bar[B_FULL0 + s], (m >> 1) & 1, abort_flag);
@@ -838,7 +843,7 @@ cudaError_t tc_chain_fwd(const Geo &g, const Tensors &t, const TcWs &w, int mode
     if (!ok) return cudaErrorInvalidValue;
     Args a = {};
     a.gb = w.gb; a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
-    a.S0 = t.S0; a.egc = w.egc; a.rn = w.rn; a.wn = t.w_norm;
+    a.S0 = t.S0; a.egc = w.egc; a.rn = w.rn; a.wn = t.w_norm; a.m0 = w.m0; a.m1 = w.m1;
     if (out) {
         a.has_out = t.out != nullptr; a.has_u = t.u != nullptr; a.ST = t.S_T;
     }
@@ -894,6 +899,7 @@ cudaError_t tc_chain_rev(const Geo &g, const Tensors &t, const TcWs &w, cudaStre
     Args a = {};
     a.gb = w.gb; a.B = g.B; a.T = g.T; a.H = g.H; a.N = g.N;
     a.S0 = t.dS_T; a.ST = t.dS0; a.skt = w.skt; a.has_du = t.du != nullptr; a.egc = w.egc;
+    a.m0 = w.m0; a.m1 = w.m1;
     const size_t smem = SMEM_BYTES + 1024;
     auto go = [&](auto kern) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -81,6 +81,7 @@ struct Args {
     const float *Dx;                // KDA: [chunks][2][64][16]
     int B, T, H, N;
     int wave;                       // CTAs resident at once (2 per SM): the L2 prefetch distance
+    int n0;                         // chunk of blockIdx.x = 0 (a launch may cover chunks n0 ..)
 };
 
 // L2 prefetch of a tiled box (no shared memory, nothing to wait for; a box outside the tensor
@@ -123,7 +124,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
     volatile int *bigflag = reinterpret_cast<volatile int *>(misc + M_BIG);
     float *pf = reinterpret_cast<float *>(misc + M_PF);
 
-    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int n = a.n0 + (int)blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int T = a.T, H = a.H, t0 = n * C, L = min(C, T - t0);
     const int ci = (b * H + h) * a.N + n;  // ci * 160 < 2^31 (checked by the launcher)
@@ -154,7 +155,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) k_chunk_prep(const __grid_constan
         const long long lin = blockIdx.x + (long long)gridDim.x * (blockIdx.y + (long long)gridDim.y * blockIdx.z);
         const long long nx = lin + a.wave;
         if (a.wave > 0 && nx < (long long)gridDim.x * gridDim.y * gridDim.z) {
-            const int n2 = (int)(nx % gridDim.x), h2 = (int)((nx / gridDim.x) % gridDim.y),
+            const int n2 = a.n0 + (int)(nx % gridDim.x), h2 = (int)((nx / gridDim.x) % gridDim.y),
                       b2 = (int)(nx / ((long long)gridDim.x * gridDim.y));
             const int ci2 = (b2 * H + h2) * a.N + n2;
 #pragma unroll
@@ -781,7 +782,8 @@ cudaError_t tc_chunk_prep(const Geo &g, const Tensors &t, const TcWs &w, bool ke
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return cudaErrorInvalidValue;
     a.wave = 2 * sms;
-    const dim3 grid(g.N, g.H, g.B);
+    a.n0 = w.m0;  // the chunks [m0, m1) of each sequence (m1 = 0: to the end)
+    const dim3 grid((w.m1 > 0 ? w.m1 : g.N) - w.m0, g.H, g.B);
     if (g.variant == VAR_KDA) {  // KEEP: T and the gated k k^T products M (for the KDA gradient kernel)
         if (raw) return cudaErrorInvalidValue;
         return keep ? launch_prep<VAR_KDA, 1>(mp, a, grid, s, rec) : launch_prep<VAR_KDA, 0>(mp, a, grid, s, rec);
