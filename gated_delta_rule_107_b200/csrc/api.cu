@@ -104,17 +104,24 @@ struct SegEvents {  // events of one call, released when the call has enqueued i
 };
 int seg_bound(const Geo &g, int S, int k) { return (int)((long long)g.N * k / S); }
 
-// prep + forward chain in S segments; cuts: S - 1 fp32 states [B, H, dk, dv]
-cudaError_t fwd_segmented(const Geo &g, const Tensors &t, const TcWs &w, bool save, float *cuts, cudaStream_t s) {
+// prep (KDA: gates and prep; G as for tc_kda_gates) + forward chain in S segments; cuts: S - 1
+// fp32 states [B, H, dk, dv]
+cudaError_t fwd_segmented(const Geo &g, const Tensors &t, const TcWs &w, bool save, float *cuts, float *G,
+                          cudaStream_t s) {
     const int S = seg_count(g);
     const size_t stride = (size_t)g.B * g.H * g.dk * g.dv;
     cudaStream_t ss = side_stream();
     SegEvents se;
     if (!ss || !se.make(S)) return cudaErrorMemoryAllocation;
     Rec none;
+    const bool kda = g.variant == VAR_KDA;
+    auto products = [&](const TcWs &ws, cudaStream_t st) -> cudaError_t {
+        cudaError_t e2 = kda ? tc_kda_gates(g, t, ws, G, st, none) : cudaSuccess;
+        return e2 == cudaSuccess ? tc_chunk_prep(g, t, ws, save, st, none) : e2;
+    };
     TcWs wk = w;
     wk.m0 = seg_bound(g, S, 0); wk.m1 = seg_bound(g, S, 1);
-    cudaError_t e = tc_chunk_prep(g, t, wk, save, s, none);
+    cudaError_t e = products(wk, s);
     if (e == cudaSuccess) e = cudaEventRecord(se.ev[0], s);
     for (int k = 0; k < S && e == cudaSuccess; ++k) {
         Tensors tk = t;
@@ -126,14 +133,15 @@ cudaError_t fwd_segmented(const Geo &g, const Tensors &t, const TcWs &w, bool sa
         if (e == cudaSuccess && k + 1 < S) {  // the next segment's products, beside this chain
             if (k == 0) e = cudaStreamWaitEvent(ss, se.ev[0], 0);
             wk.m0 = seg_bound(g, S, k + 1); wk.m1 = seg_bound(g, S, k + 2);
-            if (e == cudaSuccess) e = tc_chunk_prep(g, t, wk, save, ss, none);
+            if (e == cudaSuccess) e = products(wk, ss);
             if (e == cudaSuccess) e = cudaEventRecord(se.ev[k + 1], ss);
         }
     }
     return e;  // the last chain waited for the side stream's last prep
 }
 
-// reverse chain + gradient kernel in S segments, the last segment first; cuts: S - 1 fp32 dL/dS
+// reverse chain + gradient kernel (KDA: the tensor-core one) in S segments, the last segment
+// first; cuts: S - 1 fp32 dL/dS
 cudaError_t bwd_segmented(const Geo &g, const Tensors &t, const TcWs &w, float *cuts, cudaStream_t s) {
     const int S = seg_count(g);
     const size_t stride = (size_t)g.B * g.H * g.dk * g.dv;
@@ -141,6 +149,9 @@ cudaError_t bwd_segmented(const Geo &g, const Tensors &t, const TcWs &w, float *
     SegEvents se;  // one per segment, and the side stream's end
     if (!ss || !se.make(S + 1)) return cudaErrorMemoryAllocation;
     Rec none;
+    auto grads = [&](const TcWs &ws, cudaStream_t st) -> cudaError_t {
+        return g.variant == VAR_KDA ? tc_bwd_kda(g, t, ws, st, none) : tc_bwd_chunk(g, t, ws, st, none);
+    };
     TcWs wk = w;
     cudaError_t e = cudaSuccess;
     for (int k = S - 1; k >= 0 && e == cudaSuccess; --k) {
@@ -153,12 +164,12 @@ cudaError_t bwd_segmented(const Geo &g, const Tensors &t, const TcWs &w, float *
         if (e == cudaSuccess && k + 1 < S) {  // the gradients of the segment after, beside this chain
             wk.m0 = seg_bound(g, S, k + 1); wk.m1 = seg_bound(g, S, k + 2);
             e = cudaStreamWaitEvent(ss, se.ev[k + 1], 0);
-            if (e == cudaSuccess) e = tc_bwd_chunk(g, t, wk, ss, none);
+            if (e == cudaSuccess) e = grads(wk, ss);
         }
     }
     if (e == cudaSuccess) {  // the first segment's gradients on the caller's stream; then join
         wk.m0 = seg_bound(g, S, 0); wk.m1 = seg_bound(g, S, 1);
-        e = tc_bwd_chunk(g, t, wk, s, none);
+        e = grads(wk, s);
     }
     if (e == cudaSuccess) e = cudaEventRecord(se.ev[S], ss);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(s, se.ev[S], 0);
@@ -184,11 +195,15 @@ size_t ws_bytes(const Geo &g, int dtype, int kind) {
             default: return with_cut(tc_ws_bytes(g, WS_REV));
         }
     }
-    if (use_split_kda(g, dtype, kind))  // the saving forward keeps all but its forward-only tiles
-        return tc_ws_bytes(g, kind == K_FWD_SAVE ? WS_KDA : KDA_FWD);
-    if (use_kda_hybrid_bwd(g, dtype, kind))
-        return ws_al(simt_ws_bytes(g, true)) +
-               tc_ws_bytes(g, kind == K_BWD_SAVED ? WS_REV : KDA_BWD);
+    if (use_split_kda(g, dtype, kind)) {  // the saving forward keeps all but its forward-only tiles
+        const size_t x = tc_ws_bytes(g, kind == K_FWD_SAVE ? WS_KDA : KDA_FWD), cut = seg_cut_bytes(g);
+        return cut ? ws_al(x) + cut : x;  // (the states at the cuts of a segmented call after them)
+    }
+    if (use_kda_hybrid_bwd(g, dtype, kind)) {
+        const size_t x = ws_al(simt_ws_bytes(g, true)) + tc_ws_bytes(g, kind == K_BWD_SAVED ? WS_REV : KDA_BWD),
+                     cut = seg_cut_bytes(g);
+        return cut ? ws_al(x) + cut : x;
+    }
     if (!is_bwd(kind) && use_tc_fwd(g, dtype)) return 0;
     return simt_ws_bytes(g, is_bwd(kind));
 }
@@ -266,7 +281,7 @@ static int fwd_impl(const void *q, const void *k, const void *v, const void *alp
         else tc_ws_carve(g, WS_FWD, workspace, &w);
         if (seg_count(g) > 1 && rec.ev == nullptr) {  // (the timed entry points run one launch each)
             float *cuts = (float *)((char *)workspace + (save ? 0 : ws_al(tc_ws_bytes(g, WS_FWD))));
-            rc = launch_status(fwd_segmented(g, t, w, save, cuts, s));
+            rc = launch_status(fwd_segmented(g, t, w, save, cuts, nullptr, s));
         } else {
             rc = launch_status(tc_chunk_prep(g, t, w, save, s, rec));
             if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, save ? 2 : 0, s, rec));
@@ -279,9 +294,14 @@ static int fwd_impl(const void *q, const void *k, const void *v, const void *alp
         } else {
             tc_ws_carve(g, KDA_FWD, workspace, &w);
         }
-        rc = launch_status(tc_kda_gates(g, t, w, save ? w.G : nullptr, s, rec));
-        if (rc == DR_OK) rc = launch_status(tc_chunk_prep(g, t, w, save, s, rec));
-        if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, save ? 2 : 0, s, rec));
+        if (seg_count(g) > 1 && rec.ev == nullptr) {
+            float *cuts = (float *)((char *)workspace + ws_al(tc_ws_bytes(g, save ? WS_KDA : KDA_FWD)));
+            rc = launch_status(fwd_segmented(g, t, w, save, cuts, save ? w.G : nullptr, s));
+        } else {
+            rc = launch_status(tc_kda_gates(g, t, w, save ? w.G : nullptr, s, rec));
+            if (rc == DR_OK) rc = launch_status(tc_chunk_prep(g, t, w, save, s, rec));
+            if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, save ? 2 : 0, s, rec));
+        }
     } else if (use_tc_fwd(g, dtype)) {
         rc = launch_status(tc_fwd(g, t, workspace, s, rec));
     } else {
@@ -351,11 +371,17 @@ static int bwd_impl(const void *q, const void *k, const void *v, const void *alp
             if (rc == DR_OK) rc = launch_status(tc_chunk_prep(g, t, w, true, s, rec));
             if (rc == DR_OK) rc = launch_status(tc_chain_fwd(g, t, w, 1, s, rec));
         }
-        if (rc == DR_OK) rc = launch_status(tc_chain_rev(g, t, w, s, rec));
         // the intra-chunk gradients on tcgen05 for every chunk whose gates stay within the block
         // split's range; the others (w.kwide) on the CUDA-core kernel, which reads W, U~, U, dU
         // widened to fp32 and the state products (these kernels pass over the other chunks)
-        if (rc == DR_OK) rc = launch_status(tc_bwd_kda(g, t, w, s, rec));
+        if (rc == DR_OK && seg_count(g) > 1 && rec.ev == nullptr) {
+            float *cuts = (float *)((char *)workspace + ws_al(ws_al(simt_ws_bytes(g, true)) +
+                                                              tc_ws_bytes(g, from_saved ? WS_REV : KDA_BWD)));
+            rc = launch_status(bwd_segmented(g, t, w, cuts, s));
+        } else {
+            if (rc == DR_OK) rc = launch_status(tc_chain_rev(g, t, w, s, rec));
+            if (rc == DR_OK) rc = launch_status(tc_bwd_kda(g, t, w, s, rec));
+        }
         sw.only = w.kwide;
         if (rc == DR_OK) rc = launch_status(tc_to_simt(g, w, sw.W, sw.Ut, nullptr, nullptr, sw.Un, s, rec, w.kwide));
         if (rc == DR_OK) rc = launch_status(tc_rev_to_simt(g, w, nullptr, sw.dUn, s, rec, w.kwide));

@@ -91,6 +91,7 @@ struct Args {
     __nv_bfloat16 *dq, *dk, *dv, *dalpha, *dbeta;
     const int *kwide;               // [chunks]: left to the CUDA-core kernel
     int T, H, N;
+    int m0, m1;                     // the chunks [m0, m1) of each sequence (m1 = 0: all)
 };
 
 // first row of Km's section R (rows i = 0 .. 16 R + 15) and of Kp's / Qp's section I (rows 16 I .. 63)
@@ -133,7 +134,8 @@ __device__ __forceinline__ void ld_g8(const float *G, int row, int c0, float *o)
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_kda_tc(const __grid_constant__ Maps mp, Args a) {
-    const int ci = blockIdx.x;
+    const int ns = (a.m1 > 0 ? a.m1 : a.N) - a.m0;  // one CTA per chunk of the range, sequence by sequence
+    const int ci = (int)(blockIdx.x / (unsigned)ns) * a.N + a.m0 + (int)(blockIdx.x % (unsigned)ns);
     if (a.kwide[ci]) return;  // uniform: the CUDA-core kernel takes this chunk
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm =
@@ -551,12 +553,13 @@ cudaError_t tc_bwd_kda(const Geo &g, const Tensors &t, const TcWs &w, cudaStream
     a.beta = (const __nv_bfloat16 *)t.beta;
     a.dq = (__nv_bfloat16 *)t.dq; a.dk = (__nv_bfloat16 *)t.dk; a.dv = (__nv_bfloat16 *)t.dv;
     a.dalpha = (__nv_bfloat16 *)t.dalpha; a.dbeta = (__nv_bfloat16 *)t.dbeta; a.kwide = w.kwide;
-    a.T = g.T; a.H = g.H; a.N = g.N;
+    a.T = g.T; a.H = g.H; a.N = g.N; a.m0 = w.m0; a.m1 = w.m1;
     const size_t smem = SMEM_BYTES + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_bwd_kda_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     rec.mark(s);
-    k_bwd_kda_tc<<<(unsigned)NC, NTHREADS, smem, s>>>(mp, a);
+    const uint64_t nrange = (uint64_t)g.B * g.H * ((w.m1 > 0 ? w.m1 : g.N) - w.m0);
+    k_bwd_kda_tc<<<(unsigned)nrange, NTHREADS, smem, s>>>(mp, a);
     return cudaGetLastError();
 }
 

@@ -69,8 +69,8 @@ struct TcWs {
                          //               sum_c q_rc k_ic e^{g_rc - g_ic} ([1]), i = b(r) + 0..15
     float *G;            // [ci][C][dk]   KDA: g itself (fp32)
     float *rn;           // [ci][2][C]    fused forward: 1 / |k_r|, 1 / |q_r| of the raw rows
-    int m0, m1;          // GDN / DeltaNet prep, chains and gradient kernel: only the chunks
-                         // [m0, m1) of each sequence (m1 = 0: all)
+    int m0, m1;          // prep (and KDA gates), chains and the tensor-core gradient kernels: only
+                         // the chunks [m0, m1) of each sequence (m1 = 0: all)
 };
 // rows of the stacked KDA column operand (16 + 32 + 48 + 64), and the widest in-block fall of
 // a channel's cumulative log gate (nats) for which the block-reference split is used as is

@@ -465,6 +465,7 @@ struct KdaArgs {
     float *Dx;
     float *G;  // optional: g itself, fp32 [chunks][64][128] (written for the marked chunks only)
     int T, H, N;
+    int n0;    // chunk of blockIdx.x = 0 (a launch may cover chunks n0 ..)
 };
 
 __device__ __forceinline__ void unpack8_bf16(const uint4 x, float *v) {
@@ -500,7 +501,7 @@ __global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
     float(*tot)[DK] = reinterpret_cast<float(*)[DK]>(kg_sm + KG_TOT);
     float(*gblk)[DK] = reinterpret_cast<float(*)[DK]>(kg_sm + KG_BLK);
     float *gend = reinterpret_cast<float *>(kg_sm + KG_END);
-    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int n = a.n0 + (int)blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int tg = threadIdx.x >> 4, cg = threadIdx.x & 15, c0 = 8 * cg, R = tg >> 1;
     const int t0 = n * C, L = min(C, a.T - t0);
     const size_t ci = ((size_t)b * a.H + h) * a.N + n;
@@ -621,7 +622,7 @@ __global__ void __launch_bounds__(128) k_kda_gates(KdaArgs a) {
 constexpr uint32_t DIAG_SMEM = 3 * C * DK * 4;
 
 __global__ void __launch_bounds__(128) k_kda_diag(KdaArgs a) {
-    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int n = a.n0 + (int)blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const size_t ci = ((size_t)b * a.H + h) * a.N + n;
     if (!a.kwide[ci]) return;  // uniform over the CTA
     extern __shared__ float dsm[];
@@ -684,16 +685,18 @@ cudaError_t tc_kda_gates(const Geo &g, const Tensors &t, const TcWs &w, float *G
     a.Kt1 = w.Kt1; a.Qt1 = w.Qt1; a.Kh = w.Kh; a.Kt = w.Kt; a.Qt = w.Qt; a.Kb = w.Kb; a.egc = w.egc; a.G = G;
     a.kwide = w.kwide; a.Dx = w.Dx;
     a.T = g.T; a.H = g.H; a.N = g.N;
+    a.n0 = w.m0;  // the chunks [m0, m1) of each sequence (m1 = 0: to the end)
+    const unsigned ns = (unsigned)((w.m1 > 0 ? w.m1 : g.N) - w.m0);
     cudaError_t e = cudaFuncSetAttribute(k_kda_diag, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DIAG_SMEM);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(k_kda_gates, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KG_SMEM);
     if (e != cudaSuccess) return e;
     rec.mark(s);
-    k_kda_gates<<<dim3(g.N, g.H, g.B), DK, KG_SMEM, s>>>(a);
+    k_kda_gates<<<dim3(ns, g.H, g.B), DK, KG_SMEM, s>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     rec.mark(s);
-    k_kda_diag<<<dim3(g.N, g.H, g.B), DK, DIAG_SMEM, s>>>(a);
+    k_kda_diag<<<dim3(ns, g.H, g.B), DK, DIAG_SMEM, s>>>(a);
     return cudaGetLastError();
 }
 

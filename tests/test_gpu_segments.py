@@ -1,8 +1,9 @@
-"""Long sequences with few (b, h) pairs: the library cuts each sequence's chunk range into four
-segments, so that the prep of one segment runs beside the forward chain of the one before and
-the gradient kernel of one beside the reverse chain of the one before, with the states at the
-cuts kept in fp32.  The timed entry points run one launch per kernel over the whole range, so
-both must give the same results bit for bit, and those match the fp64 oracle."""
+"""Long sequences with few (b, h) pairs (Gated DeltaNet, DeltaNet, KDA on the tensor-core path):
+the library cuts each sequence's chunk range into four segments, so that the prep of one
+segment runs beside the forward chain of the one before and the gradient kernel of one beside
+the reverse chain of the one before, with the states at the cuts kept in fp32.  The timed entry
+points run one launch per kernel over the whole range, so both must give the same results bit
+for bit, and those match the fp64 oracle."""
 import pytest
 import torch
 
@@ -53,10 +54,18 @@ def _saved_pair(x, variant, timed):
     return {"o": o, "u": u, "S_T": S_T}, {k: v for k, v in g.items() if v is not None}
 
 
-# (variant, B, T, H, du, S0 std): 8 and 12 chains with 65 and 33 chunks (segments of 16-17 and 8-9)
-@pytest.mark.parametrize("variant,B,T,H,du,s0", (("gdn", 1, 4133, 4, True, 0.1), ("deltanet", 2, 2100, 3, False, 0.0)))
-def test_segments_equal_whole_range_and_oracle(variant, B, T, H, du, s0):
+# (variant, B, T, H, du, S0 std, fast): 8 or 12 chains with 65 or 33 chunks (segments of 16-17
+# or 8-9); fast: KDA channels whose gates fall by 12 nats a token in one sequence, so that
+# some chunks go to the CUDA-core gradient kernel after the segments
+@pytest.mark.parametrize("variant,B,T,H,du,s0,fast", (("gdn", 1, 4133, 4, True, 0.1, False),
+                                                      ("deltanet", 2, 2100, 3, False, 0.0, False),
+                                                      ("kda", 1, 2100, 4, True, 0.1, False),
+                                                      ("kda", 2, 2100, 2, True, 0.0, True)))
+def test_segments_equal_whole_range_and_oracle(variant, B, T, H, du, s0, fast):
     x = gen(variant, "bf16", B, T, H, 128, 128, seed=71 + T, s0_std=s0, grads=True, du=du)
+    if fast:
+        x["loga"][0, :, :, :4] = -12.0
+        x["loga"][..., 4:8] = -3.0
     f_seg, g_seg = _saved_pair(x, variant, timed=False)
     f_one, g_one = _saved_pair(x, variant, timed=True)
     for key in f_one:
