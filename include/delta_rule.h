@@ -48,16 +48,23 @@
  *              channel dimension (q, k, v, out, u, the KDA gate and all their
  *              gradients) and the fp32 states must be 16-byte aligned; beta, dbeta
  *              and the Gated-DeltaNet gate need only their element alignment.
- *              The caller owns every buffer; the library allocates nothing, keeps
- *              no pointer after returning and has no global state except the
- *              device error word below.  Inputs are never written.  Outputs must
+ *              The caller owns every buffer; the library allocates no device
+ *              memory, keeps no pointer after returning and has no global state
+ *              except the device error word below and, once a call has run in
+ *              segments (see Stream), one CUDA stream per device.  Inputs are never written.  Outputs must
  *              not alias inputs or each other.
  *   Workspace  caller-provided device scratch of at least
  *              delta_rule_workspace_size(...) bytes, 256-byte aligned; its
  *              contents on entry do not matter.  Two calls that run at the same
  *              time need distinct workspaces.
- *   Stream     `stream` is a cudaStream_t (NULL = the legacy default stream).  All
- *              work is enqueued on it; the call returns without synchronising.
+ *   Stream     `stream` is a cudaStream_t (NULL = the legacy default stream).  A
+ *              call's work follows the work enqueued on it before and precedes
+ *              the work enqueued after; the call returns without synchronising.
+ *              The tensor-core forward and backward of long sequences with few
+ *              (b, h) pairs (at most one (b, h) per 4 SMs, at least 32 chunks)
+ *              run in four segments of the chunk range: part of their kernels
+ *              on the library's own non-blocking stream, ordered against
+ *              `stream` by events, which the call joins back before returning.
  *   Errors     every entry point validates its arguments first and returns a
  *              negative DR_ERR_* code without launching anything when they are
  *              bad.  Launch failures return DR_ERR_CUDA.  Faults detected on the
@@ -163,7 +170,9 @@ int delta_rule_bwd_saved(const void *q, const void *k, const void *v, const void
  * (1), delta_rule_fwd_save (2), delta_rule_bwd_saved (3) -- and stores a static
  * name for launch i in names[i] for i < max_names (names may be NULL); it
  * returns a negative DR_ERR_* code for invalid arguments.  The *_timed variants
- * do exactly what their plain entry points do and in addition record the
+ * compute what their plain entry points compute, bit for bit, but always with
+ * one launch per kernel over the whole chunk range (never in segments; those
+ * launches are what delta_rule_launches counts), and in addition record the
  * caller's cudaEvent_t events[i] (created handles) on `stream` immediately
  * before launch i and events[n] after the last launch (n = the launch count),
  * so that each kernel's device time is the elapsed time between consecutive
