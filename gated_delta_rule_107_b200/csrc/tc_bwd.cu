@@ -162,10 +162,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_bwd_chunk_tc(const __grid_const
     const bool gated = a.variant == VAR_GATED;
     auto part_at = [&](int kind, int half, int rr) -> float & { return part[(kind * 2 + half) * 64 + rr]; };
     struct Pos { int ci, n, h, b, t0; };
-    auto pos_of = [&](int wi) -> Pos {  // work item wi: chunk n = m0 + wi % NS of sequence (b, h) = wi / NS
+    // work item wi: chunk n = m0 + wi / (B H) of sequence (b, h) = wi % (B H), chunk by chunk from the
+    // first: the reverse chain wrote the first chunks' dS and dU last, so they are read while in L2
+    const int BH = a.B * H;
+    auto pos_of = [&](int wi) -> Pos {
         Pos p;
-        p.n = m0 + wi % NS;
-        const int bh = wi / NS;
+        p.n = m0 + wi / BH;
+        const int bh = wi % BH;
         p.ci = bh * N + p.n;
         p.h = bh % H; p.b = bh / H; p.t0 = p.n * C;
         return p;
