@@ -78,6 +78,8 @@ def load(path: str | None = None):
     lib.delta_rule_sync_status.restype = i
     lib.delta_rule_launches.argtypes = [i] * 9 + [ctypes.POINTER(ctypes.c_char_p), i]
     lib.delta_rule_launches.restype = i
+    lib.delta_rule_plain_launches.argtypes = [i] * 9
+    lib.delta_rule_plain_launches.restype = i
     lib.delta_rule_fwd_timed.argtypes = [vp] * 9 + [i] * 8 + [vp, sz, vp, ctypes.POINTER(vp), i]
     lib.delta_rule_fwd_timed.restype = i
     lib.delta_rule_bwd_timed.argtypes = [vp] * 15 + [i] * 8 + [vp, sz, vp, ctypes.POINTER(vp), i]
@@ -145,6 +147,14 @@ def saved_size(B, T, H, dk, dv, variant, chunk, dtype) -> int:
     n = load().delta_rule_saved_size(B, T, H, dk, dv, variant, chunk, dtype)
     if n == ctypes.c_size_t(-1).value:
         raise DeltaRuleError(DR_ERR_ARG, "delta_rule_saved_size")
+    return n
+
+
+def plain_launches(B, T, H, dk, dv, variant, chunk, dtype, for_bwd) -> int:
+    """How many kernels the plain entry point launches (more than ``launches`` when it runs in segments)."""
+    n = load().delta_rule_plain_launches(B, T, H, dk, dv, variant, chunk, dtype, int(for_bwd))
+    if n < 0:
+        raise DeltaRuleError(n, "delta_rule_plain_launches")
     return n
 
 

@@ -606,6 +606,22 @@ extern "C" int delta_rule_launches(int B, int T, int H, int dk, int dv, int vari
     return launch_plan(g, dtype, for_bwd, names, max_names);
 }
 
+extern "C" int delta_rule_plain_launches(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype,
+                                         int for_bwd) {
+    Geo g;
+    const int rc = check_shape(B, T, H, dk, dv, variant, chunk, dtype, &g);
+    if (rc != DR_OK) return rc;
+    if (for_bwd < 0 || for_bwd > 3) return DR_ERR_ARG;
+    const int n = launch_plan(g, dtype, for_bwd, nullptr, 0);
+    if (n <= 0 || T == 0 || (size_t)B * H == 0) return n;
+    const bool split = use_split(g, dtype) || use_split_kda(g, dtype, for_bwd) || use_kda_hybrid_bwd(g, dtype, for_bwd);
+    const int S = split ? seg_count(g) : 1;
+    if (S == 1) return n;
+    // in segments: every forward kernel once per segment; the backward's reverse chain and
+    // gradient kernel once per segment, the rest once
+    return is_bwd(for_bwd) ? n - 2 + 2 * S : n * S;
+}
+
 extern "C" int delta_rule_decode(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
                                  const float *S_in, float *S_out, void *out, void *u, int B, int T, int H, int dk,
                                  int dv, int variant, int dtype, void *stream) {

@@ -181,6 +181,10 @@ int delta_rule_bwd_saved(const void *q, const void *k, const void *v, const void
  */
 int delta_rule_launches(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype, int for_bwd,
                         const char **names, int max_names);
+/* The number of kernels the plain entry point launches for these arguments (for_bwd as
+ * above): delta_rule_launches' count, or more when the call runs in segments (see
+ * Stream); a negative DR_ERR_* code for invalid arguments. */
+int delta_rule_plain_launches(int B, int T, int H, int dk, int dv, int variant, int chunk, int dtype, int for_bwd);
 int delta_rule_fwd_timed(const void *q, const void *k, const void *v, const void *alpha, const void *beta,
                          const float *S0, void *out, void *u, float *S_T, int B, int T, int H, int dk, int dv,
                          int variant, int chunk, int dtype, void *workspace, size_t ws_bytes, void *stream,

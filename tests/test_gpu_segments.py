@@ -80,3 +80,15 @@ def test_segments_equal_whole_range_and_oracle(variant, B, T, H, du, s0, fast):
         assert torch.equal(g_plain[key], g_one[key]), key
     compare_fwd(f_seg, oracle_fwd(x, variant), "bf16", what=f"segmented {variant} T={T}")
     compare_bwd(g_seg, oracle_bwd(x, variant), "bf16", variant, what=f"segmented {variant} T={T}")
+
+
+def test_plain_launch_counts():
+    # segmented: each of the forward's two kernels and the backward's two once per segment
+    args = (1, 4133, 4, 128, 128, binding.VARIANTS["gdn"], C, DT)
+    assert len(binding.launches(*args, 2)) == 2 and binding.plain_launches(*args, 2) == 8
+    assert len(binding.launches(*args, 3)) == 2 and binding.plain_launches(*args, 3) == 8
+    assert binding.plain_launches(*args, 1) == 4 - 2 + 8  # the recompute's prep and chain once
+    # the headline shape (128 chain CTAs) runs whole: the same count as the timed form
+    args = (8, 4096, 8, 128, 128, binding.VARIANTS["gdn"], C, DT)
+    for kind in range(4):
+        assert binding.plain_launches(*args, kind) == len(binding.launches(*args, kind))
